@@ -1,0 +1,455 @@
+"""Throughput of the outlier-aware W4A8 quantized linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one pass of the whole hot path -- targeted momentum update,
+per-token INT8 quantization, tcgen05 INT8 GEMM with the fused dequant and
+outlier compensation -- over every linear of the workload at every token
+count, on NL distinct copies of the packed weights (so the weights streamed
+in one step exceed the 126 MB L2 and come from HBM).  Default workload:
+LLaMA-2-7B-shaped linears (q, k, v, o 4096x4096; gate, up 4096->11008; down
+11008->4096), W4A8 per-channel, M in {1, 4, 16, 64}, 1% outlier channels
+x100, synthetic seeded data.
+
+metric / unit: effective GB/s = algorithmic bytes of the step / step time
+(weights K*N/2, scales 4N, W_O 2*n_O*N, X 2MK, Xq written and read 2MK,
+a 4M, outlier codes M*n_O, Y 2MN); TOPS (2MNK) are reported beside it.
+
+N > 1 (torchrun): data-parallel over tokens, weak scaling: every rank runs
+the same step on its own token batch with replicated weights; the outlier
+column maxima of all linears are combined with one all-reduce(MAX) per step
+so every replica keeps the same momentum state.
+
+``--impl reference`` times the CPU oracle (single thread) on a bounded
+sample of the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_linear_layers_token_b200 import synth  # noqa: E402
+
+METRIC = "W4A8/W8A8 quantized-linear effective TOPS, GB/s and % of INT8/HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def algorithmic_bytes(M, K, N, nO, fmt):
+    wbytes = K * N // 2 if fmt != synth.W8_PERCHANNEL else K * N
+    gemm = wbytes + 4 * N + (2 * (K // 128) * N if fmt == synth.W4_G128 else 0) + 2 * nO * N \
+        + M * K + 4 * M + M * nO + 2 * M * N
+    act = 2 * M * K + M * K + 4 * M + M * nO
+    return gemm, act
+
+
+def gemm_only_bytes(M, K, N, nO, fmt):
+    return algorithmic_bytes(M, K, N, nO, fmt)[0]
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload: every linear at
+    ``sample_m`` tokens (one weight copy).  Packing is offline and untimed."""
+
+    def __init__(self, wl, sample_m):
+        from oracle import oracle
+        self.o = oracle
+        self.wl = wl
+        self.m = sample_m
+        self.items = []
+        for si, (name, K, N) in enumerate(wl.shapes):
+            L = synth.layer(wl, si, M=sample_m)
+            Xb = np.ascontiguousarray(L["X"]).view(np.uint16)
+            Wb = np.ascontiguousarray(L["W"]).view(np.uint16)
+            pk = oracle.pack_layer(Wb, L["O"], wl.fmt)
+            self.items.append((Xb, Wb, pk, len(L["O"]), K, N))
+        self.bytes = sum(sum(algorithmic_bytes(sample_m, K, N, nO, wl.fmt)) for _, _, _, nO, K, N in self.items)
+        self.ops = sum(2 * sample_m * K * N for *_, K, N in self.items)
+
+    def step(self):
+        t0 = time.perf_counter()
+        for Xb, Wb, pk, nO, K, N in self.items:
+            self.o.forward(Xb, Wb, pk, np.ones(nO, np.float32), self.wl.gamma, update_momentum=True)
+        return time.perf_counter() - t0
+
+    def describe(self, seconds):
+        return (f"every linear of {self.wl.name} ({len(self.items)}) at M={self.m}, one weight copy: "
+                f"momentum update, quantization, int64 GEMM, fp64 dequant; {seconds:.1f} s of "
+                f"single-threaded CPU time; host has {os.cpu_count()} cores")
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sample = OracleSample(wl, 4)
+    for _ in range(args.warmup):
+        sample.step()
+    t = sum(sample.step() for _ in range(args.steps))
+    gbs = args.steps * sample.bytes / t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64",
+        "data": "synthetic", "tops": args.steps * sample.ops / t / 1e12,
+        "config": {"workload": wl.name, "sample": f"all {len(wl.shapes)} linears at M={sample.m}",
+                   "parallelism": "single thread"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample.describe(t / args.steps) + " (per step)"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def build_problem(wl, copies, device):
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    layers = []  # per shape: list of PackedLayer copies
+    meta = []
+    for si, (name, K, N) in enumerate(wl.shapes):
+        L = synth.layer(wl, si, M=1)
+        W = torch.from_numpy(L["W"]).to(device)
+        base = qlin.PackedLayer.pack(W, L["O"], wl.fmt)
+        del W
+        cps = [base] + [base.clone() for _ in range(copies - 1)]
+        layers.append(cps)
+        meta.append({"name": name, "K": K, "N": N, "O": L["O"]})
+    inputs = {}
+    for M in wl.ms:
+        for si, (name, K, N) in enumerate(wl.shapes):
+            L = synth.layer(wl, si, M=M, with_weights=False)
+            inputs[(M, si)] = L["X"]
+    return layers, meta, inputs
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama7b_w4_decode")
+    ap.add_argument("--copies", type=int, default=4)
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    layers, meta, inputs_np = build_problem(wl, args.copies, device)
+    ms = wl.ms
+    nshape = len(wl.shapes)
+
+    # per (M, shape, copy): device input, output, momentum state, workspace
+    slots = []
+    for M in ms:
+        for c in range(args.copies):
+            for si in range(nshape):
+                lay = layers[si][c]
+                X = torch.from_numpy(inputs_np[(M, si)]).to(device)
+                Y = torch.empty((M, meta[si]["N"]), dtype=torch.float16, device=device)
+                s = torch.ones(max(len(meta[si]["O"]), 1), dtype=torch.float32, device=device)
+                nws = qlin.qlin_forward_workspace(M, lay.w)
+                ws = qlin.empty_workspace(nws)
+                slots.append({"M": M, "si": si, "c": c, "layer": lay, "X": X, "Y": Y, "s": s, "ws": ws,
+                              "nws": nws})
+    stream = torch.cuda.Stream(device)
+
+    # DP exchange buffers (N > 1): all outlier column maxima of a step in one vector
+    offs = []
+    tot = 0
+    for sl in slots:
+        offs.append(tot)
+        tot += len(meta[sl["si"]]["O"])
+    cmax_all = torch.zeros(max(tot, 1), dtype=torch.float32, device=device)
+
+    def step_single():
+        for sl in slots:
+            qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
+                              sl["nws"], stream)
+
+    def step_dp():
+        for sl, o in zip(slots, offs):
+            nO = len(meta[sl["si"]]["O"])
+            if nO:
+                qlin.qlin_outlier_colmax(sl["X"], sl["M"], sl["layer"].w, cmax_all[o:o + nO], stream)
+        with torch.cuda.stream(stream):
+            dist.all_reduce(cmax_all, op=dist.ReduceOp.MAX)
+        for sl, o in zip(slots, offs):
+            nO = len(meta[sl["si"]]["O"])
+            lay = sl["layer"]
+            if nO:
+                qlin.qlin_momentum_update(lay.w, cmax_all[o:o + nO], sl["s"], wl.gamma, stream)
+            ws = sl["ws"]
+            # quant_act(update=0) + gemm through the split entry points
+            M, K = sl["M"], meta[sl["si"]]["K"]
+            qlin.qlin_forward(sl["X"], M, lay.w, sl["s"], wl.gamma, False, sl["Y"], ws, sl["nws"], stream)
+
+    step = step_single if world == 1 else step_dp
+
+    # warm-up (eager; sets kernel attributes and resolves the driver entry point)
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    graph = None
+    if world == 1:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+
+    def run_steps(k):
+        for _ in range(k):
+            if graph is not None:
+                with torch.cuda.stream(stream):
+                    graph.replay()
+            else:
+                step()
+
+    # ---------------------------------------------------------------- timed region
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        run_steps(args.steps)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms_step], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    clocks = clk.summary()
+
+    step_bytes = 0
+    step_ops = 0
+    gemm_bytes = 0
+    for sl in slots:
+        m = meta[sl["si"]]
+        g, a = algorithmic_bytes(sl["M"], m["K"], m["N"], len(m["O"]), wl.fmt)
+        step_bytes += g + a
+        gemm_bytes += g
+        step_ops += 2 * sl["M"] * m["K"] * m["N"]
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    # ---------------------------------------------------------------- GEMM-only timing (roofline)
+    gemm_slots = []
+    for sl in slots:
+        M, lay = sl["M"], sl["layer"]
+        K, nO = meta[sl["si"]]["K"], len(meta[sl["si"]]["O"])
+        Xq = torch.empty((M, K), dtype=torch.int8, device=device)
+        a = torch.empty(M, dtype=torch.float32, device=device)
+        XqO = torch.empty((M, max(nO, 1)), dtype=torch.int8, device=device)
+        naws = qlin.qlin_quant_act_workspace(M, lay.w)
+        aws = qlin.empty_workspace(naws)
+        qlin.qlin_quant_act(sl["X"], M, lay.w, sl["s"], wl.gamma, False, Xq, a, XqO, aws, naws, stream)
+        gemm_slots.append((sl, Xq, a, XqO))
+    torch.cuda.synchronize()
+
+    def gemm_pass():
+        # qlin_gemm = the compensation-operand kernel (when n_O > 0) + the tcgen05 GEMM kernel
+        for sl, Xq, a, XqO in gemm_slots:
+            qlin.qlin_gemm(sl["layer"].w, Xq, a, XqO, sl["s"], sl["M"], sl["Y"], None, sl["ws"], sl["nws"], stream)
+
+    gemm_pass()
+    torch.cuda.synchronize()
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        gemm_pass()
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            g2.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = max(5, args.steps)
+    e0.record(stream)
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            g2.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    gemm_ms = e0.elapsed_time(e1) / reps
+    n_gemm_launches = len(gemm_slots)
+
+    hbm, bf16, bf16_sus, peak_kind = read_peaks()
+    achieved = gemm_bytes / (gemm_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": None, "peak_source": f"hbm_gbs of {peak_kind} peaks (copy burst)",
+                "kernel": "qlin_gemm (comp operand + tcgen05 GEMM), all launches of one step",
+                "ms_per_step": gemm_ms, "launches_per_step": n_gemm_launches}
+
+    # ---------------------------------------------------------------- end to end through the API
+    e2e = None
+    if world == 1:
+        host_x = [torch.from_numpy(inputs_np[(sl["M"], sl["si"])]).pin_memory() for sl in slots]
+        host_y = [torch.empty(sl["Y"].shape, dtype=torch.float16).pin_memory() for sl in slots]
+        h2d = sum(x.numel() * 2 for x in host_x)
+        d2h = sum(y.numel() * 2 for y in host_y)
+
+        def e2e_step():
+            for sl, hx, hy in zip(slots, host_x, host_y):
+                sl["X"].copy_(hx, non_blocking=True)
+                qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
+                                  sl["nws"], stream)
+                hy.copy_(sl["Y"], non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+        torch.cuda.synchronize()
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g3, stream=stream):
+            e2e_step()
+        with torch.cuda.stream(stream):
+            g3.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                g3.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        e2e = {"value": step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "note": "pinned host X -> device, qlin_forward, device -> pinned host Y, per linear, "
+                       "replayed as one CUDA graph per step"}
+
+    # ---------------------------------------------------------------- CPU baseline (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1:
+        sample = OracleSample(wl, 16)
+        t = sample.step()
+        cpu = {"value": sample.bytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": sample.describe(t)}
+
+    launches_per_forward = {sl["si"]: (3 if len(meta[sl["si"]]["O"]) else 2) for sl in slots}
+    gpu_launches = args.steps * sum(launches_per_forward[sl["si"]] for sl in slots)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "tops": world * step_ops / (ms_step * 1e-3) / 1e12,
+            "config": {"workload": wl.name, "shapes": [[n, K, N] for n, K, N in wl.shapes], "M": ms,
+                       "weight_copies": args.copies,
+                       "weight_bytes_per_step": int(sum(layers[si][0].nbytes for si in range(nshape)) * args.copies
+                                                    * len(ms)),
+                       "l2": "inputs larger than L2 (distinct packed-weight copies rotated each step)",
+                       "outlier_frac": wl.outlier_frac, "gamma": wl.gamma, "format": "W4A8 per-channel"
+                       if wl.fmt == 0 else ("W4A8 g128" if wl.fmt == 1 else "W8A8"),
+                       "parallelism": f"dp{world}", "forwards_per_step": len(slots),
+                       "timing": "CUDA graph of one step, CUDA events on the launch stream"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"]},
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

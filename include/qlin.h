@@ -1,0 +1,220 @@
+/*
+ * qlin.h -- C ABI of the B200 (sm_100a) outlier-aware quantized linear layer
+ *
+ *     Y = Q(X) . Q(W)
+ *       = a (.) [ c' (.) (Xq . B) ]  +  a (.) [ XqO . diag(s_O - 1) . W_O ]
+ *
+ * Three stages run on the GPU:
+ *   1. per-token symmetric INT8 activation quantization on X_hat = X (/) s,
+ *      where s is the targeted momentum scale kept only on the outlier
+ *      channel set O ("Quaff: Quantized Parameter-Efficient Fine-Tuning under
+ *      Outlier Spatial Stability Hypothesis", sections 目标动量缩放 and
+ *      整体框架);
+ *   2. an INT8 tensor-core GEMM whose weight operand comes from one of three
+ *      packed formats -- INT4 per output channel unpacked to INT8 by a left
+ *      shift of 4, INT4 with g=128 group scales requantized to INT8 through
+ *      the folded group/channel ratio, or plain INT8 per channel ("QQQ:
+ *      Quality Quattuor-Bit Quantization for Large Language Models", section
+ *      W4A8 GEMM内核: per-channel GEMM, per-group GEMM, FusedDequantQuant,
+ *      FastFP16toINT8);
+ *   3. a fused INT32 -> FP16 dequant epilogue that adds the sparse outlier
+ *      compensation term X_hat[:,O] (s_O - 1) W_O (Quaff notes, section
+ *      关键设计, decoupled WAQ formula).
+ *
+ * Conventions for every entry point
+ *   - "device" pointers are CUDA device memory owned by the caller; "host"
+ *     pointers are ordinary host memory owned by the caller.  The library
+ *     never allocates, frees or retains memory and keeps no state across
+ *     calls other than a per-thread last-error string and one device error
+ *     word (see qlin_poll_device_status).
+ *   - fp16 values are IEEE binary16 bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Every call only enqueues work on `stream` and returns without
+ *     synchronizing; argument errors are detected on the host before anything
+ *     is enqueued and leave all buffers untouched.
+ *   - Matrices are row-major with dense rows (no padding) unless stated.
+ *   - Device pointers must be 16-byte aligned (QLIN_ERR_ALIGN otherwise).
+ *   - Shapes: K % 32 == 0, N % 16 == 0, 1 <= K < 131072, N >= 16; for the
+ *     g128 format K % 128 == 0; 0 <= n_outlier <= min(K, 4096).
+ *   - Workspaces: buffers whose size comes from the matching *_workspace
+ *     call.  A workspace must be zero-filled before its first use (for
+ *     example with cudaMemsetAsync); every successful call leaves it
+ *     zero-filled again in the parts that must start at zero, so it can be
+ *     reused by later calls on the same stream without clearing.  Calls that
+ *     share a workspace must not overlap on the GPU.
+ *   - No entry point is thread-hostile; concurrent calls on different
+ *     streams must use different outputs and workspaces.
+ */
+#ifndef QLIN_H_
+#define QLIN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLIN_API __attribute__((visibility("default")))
+#else
+#define QLIN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLIN_OK = 0,
+  QLIN_ERR_ARG = 1,       /* null pointer, negative size, bad O (not sorted/unique/in range), bad fmt */
+  QLIN_ERR_SHAPE = 2,     /* shape outside the supported set listed above */
+  QLIN_ERR_ALIGN = 3,     /* a device pointer is not 16-byte aligned */
+  QLIN_ERR_WORKSPACE = 4, /* workspace smaller than the *_workspace size */
+  QLIN_ERR_CUDA = 5,      /* a CUDA runtime / driver call or a launch failed */
+  QLIN_ERR_TIMEOUT = 6    /* a bounded device-side wait gave up (see qlin_poll_device_status) */
+} qlin_status;
+
+typedef enum {
+  QLIN_W4_PERCHANNEL = 0, /* INT4 codes in [-7,7], one fp32 scale per output channel */
+  QLIN_W4_G128 = 1,       /* INT4 codes in [-7,7] per group of 128 input channels, requantized to INT8 */
+  QLIN_W8_PERCHANNEL = 2  /* INT8 codes in [-127,127], one fp32 scale per output channel */
+} qlin_wfmt;
+
+/* Packed weights of one linear layer with K input and N output channels.
+ * Plain descriptor: every pointer is device memory owned by the caller, and
+ * qlin_weights_bind() can carve all of them out of one allocation.
+ *
+ *   codes        W4 formats: uint8 [N][K/2].  For the 32-bit little-endian
+ *                word of row n that covers input channels k0..k0+7, byte b
+ *                (0..3) holds q[k0+b] in its low nibble and q[k0+4+b] in its
+ *                high nibble (two's complement).  Then (word << 4) & 0xF0F0F0F0
+ *                holds the INT8 lanes 16*q[k0..k0+3] and word & 0xF0F0F0F0
+ *                the lanes 16*q[k0+4..k0+7].
+ *                W8 format: int8 [N][K] (row n = output channel n).
+ *   chan_scale   c_n, fp32 [N].  Per-channel formats: c_n = max_k|W[k][n]| / qmax
+ *                (qmax = 7 or 127).  g128: c_n = 7 * max_j g[j][n] / 127.
+ *   group_scale  g128 only: g[j][n] = fp16(max_{k in group j}|W[k][n]| / 7), fp16 [K/128][N].
+ *   fold_ratio   g128 only: r[j][n] = fp16(g[j][n] / c_n), fp16 [K/128][N].
+ *   outlier_idx  O, int32 [n_outlier], strictly increasing, in [0, K).
+ *   W_Ot         fp16 [N][n_outlier_pad]: W_Ot[n][i] = W[O_i][n]; columns
+ *                n_outlier .. n_outlier_pad-1 are zero.  The outlier rows of
+ *                W kept in full precision.
+ *   wmax_O       fp32 [n_outlier]: max_n |W[O_i][n]| (the weight side of beta).
+ */
+typedef struct {
+  int32_t K;
+  int32_t N;
+  int32_t fmt;           /* qlin_wfmt */
+  int32_t group;         /* 128 for QLIN_W4_G128, else 0 */
+  int32_t n_outlier;     /* |O| */
+  int32_t n_outlier_pad; /* n_outlier rounded up to a multiple of 8 */
+  void* codes;
+  float* chan_scale;
+  uint16_t* group_scale;
+  uint16_t* fold_ratio;
+  int32_t* outlier_idx;
+  uint16_t* W_Ot;
+  float* wmax_O;
+} qlin_weights;
+
+/* Human-readable name of a status code (static string). */
+QLIN_API const char* qlin_status_string(qlin_status status);
+
+/* Description of the last error returned on the calling host thread
+ * (static thread-local buffer, valid until the next call on that thread). */
+QLIN_API const char* qlin_last_error(void);
+
+/* Bytes needed to hold all packed buffers of a layer (each sub-buffer
+ * aligned to 256 bytes).  Host-only; enqueues nothing. */
+QLIN_API qlin_status qlin_weights_bytes(int32_t K, int32_t N, int32_t fmt, int32_t n_outlier,
+                               size_t* bytes);
+
+/* Fill `w` with the shape fields and sub-buffer pointers carved out of the
+ * device allocation [base, base + bytes).  Host-only; enqueues nothing and
+ * does not touch the memory.  base must be 256-byte aligned. */
+QLIN_API qlin_status qlin_weights_bind(qlin_weights* w, int32_t K, int32_t N, int32_t fmt,
+                              int32_t n_outlier, void* base, size_t bytes);
+
+/* Quantize and pack one layer's weights (offline step of both pages: Quaff
+ * quantizes the frozen W to W_int and keeps the outlier rows W_O in full
+ * precision; QQQ stores INT4 codes with per-channel or per-group scales and
+ * folds the group scale by the channel scale).
+ *   W       device fp16 [K][N] (row k = input channel k).
+ *   O_host  host int32 [w->n_outlier], strictly increasing, in [0, K); read
+ *           during the call only.  May be NULL when n_outlier == 0.
+ *   w       bound descriptor (qlin_weights_bind) whose buffers are written.
+ * Codes: per-channel q = clamp(rne(w * (qmax / wmax_n)), -qmax, qmax) in
+ * fp32; g128 q4 = clamp(rne(w / g), -7, 7) and the INT8 operand
+ * q8 = rne(q4 * r) with one rounding. */
+QLIN_API qlin_status qlin_pack_weights(const uint16_t* W, const int32_t* O_host, const qlin_weights* w,
+                              void* stream);
+
+/* Workspace for qlin_quant_act (holds the outlier column maxima and a
+ * completion counter).  0 when n_outlier == 0. */
+QLIN_API qlin_status qlin_quant_act_workspace(int32_t M, const qlin_weights* w, size_t* bytes);
+
+/* Stage 1: targeted momentum update and per-token INT8 quantization.
+ *   X        device fp16 [M][K] activations (token-major).
+ *   s        device fp32 [n_outlier] momentum state, read and (when
+ *            update_momentum != 0) updated in place:
+ *              beta_i = max(1, sqrt(max_m|X[m,O_i]| / wmax_O[i]))   (1 if wmax_O[i] == 0)
+ *              s_i   <- gamma * s_i + (1 - gamma) * beta_i          (fp32, this association)
+ *            then the updated s quantizes this same X.
+ *   Xq       device int8 [M][K]: clamp(rne(x_hat * (127 / amax_m)), -127, 127),
+ *            x_hat[m,k] = X[m,k] / s_i for k = O_i, else X[m,k].
+ *   a        device fp32 [M]: amax_m / 127 (0 for an all-zero token).
+ *   XqO      device int8 [M][n_outlier]: Xq[m, O_i] (may be NULL when n_outlier == 0).
+ * M may be 0 (nothing is enqueued). */
+QLIN_API qlin_status qlin_quant_act(const uint16_t* X, int32_t M, const qlin_weights* w, float* s,
+                           float gamma, int32_t update_momentum, int8_t* Xq, float* a,
+                           int8_t* XqO, void* workspace, size_t ws_bytes, void* stream);
+
+/* Data-parallel split of the momentum update, for callers that shard tokens
+ * across GPUs and must keep one s on every replica: qlin_outlier_colmax
+ * writes cmax[i] = max_m |X[m, O_i]| (device fp32 [n_outlier]) over this
+ * GPU's tokens; the caller reduces cmax with MAX across ranks; then
+ * qlin_momentum_update applies the recurrence above to s in place, and
+ * qlin_quant_act(..., update_momentum = 0, ...) quantizes. */
+QLIN_API qlin_status qlin_outlier_colmax(const uint16_t* X, int32_t M, const qlin_weights* w, float* cmax,
+                                void* stream);
+QLIN_API qlin_status qlin_momentum_update(const qlin_weights* w, const float* cmax, float* s, float gamma,
+                                 void* stream);
+
+/* Workspace for qlin_gemm at token count M. */
+QLIN_API qlin_status qlin_gemm_workspace(int32_t M, const qlin_weights* w, size_t* bytes);
+
+/* Stages 2 and 3: INT8 tensor-core GEMM with fused dequant + compensation.
+ *   Xq, a, XqO, s  as produced by qlin_quant_act (s is the state used to
+ *                  quantize; only read).
+ *   Y         device fp16 [M][N]:
+ *               Y[m][n] = fp16( a_m * ( c'_n * acc[m][n] + comp[m][n] ) )
+ *               acc[m][n]  = sum_k Xq[m][k] * B[k][n] (exact int32), B the
+ *                            INT8 operand (16*q, q8 or q);
+ *               c'_n       = c_n / 16 (W4 per-channel) or c_n;
+ *               comp[m][n] = sum_i XqO[m][i] * (s_i - 1) * W_Ot[n][i], with
+ *                            each product u = XqO*(s-1) formed in fp32 and
+ *                            carried as fp16(u) + fp16(u - fp16(u)), the sum
+ *                            accumulated in fp32 on the tensor cores.
+ *   acc_debug NULL, or device int32 [M][N] receiving acc (for parity checks).
+ * Y must not alias any input. */
+QLIN_API qlin_status qlin_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, const int8_t* XqO,
+                      const float* s, int32_t M, uint16_t* Y, int32_t* acc_debug,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace for qlin_forward at token count M (holds Xq, a, XqO and the
+ * scratch of the two stages). */
+QLIN_API qlin_status qlin_forward_workspace(int32_t M, const qlin_weights* w, size_t* bytes);
+
+/* The whole layer: qlin_quant_act followed by qlin_gemm on one stream, with
+ * the compensation operand produced directly by the quantization kernel. */
+QLIN_API qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weights* w, float* s,
+                         float gamma, int32_t update_momentum, uint16_t* Y, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream`, then reports and clears the device error word that
+ * kernels set when a bounded wait gives up: QLIN_ERR_TIMEOUT if it was set,
+ * QLIN_ERR_CUDA if the stream reported an error, else QLIN_OK. */
+QLIN_API qlin_status qlin_poll_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLIN_H_ */

@@ -1,0 +1,233 @@
+// act_quant.cuh -- stage 1: targeted momentum scaling on the outlier
+// channels and per-token symmetric INT8 quantization.
+//
+// Quaff notes, 目标动量缩放: for i in O,
+//   beta_i = max(1, sqrt(max_m |X[m,O_i]| / max_n |W[O_i,n]|)),
+//   s_i   <- gamma * s_i + (1 - gamma) * beta_i;
+// channels outside O keep s = 1, so only |O| values are ever touched.
+// The activations the integer GEMM sees are X_hat = X (/) s, quantized per
+// token with a symmetric INT8 scale a_m = max_k |x_hat[m,k]| / 127 (QQQ
+// review: symmetric activation quantization).
+//
+// Kernels:
+//   colmax_kernel   grid over row blocks; per-CTA maxima of |X[:,O]| in
+//                   shared memory, merged with one global atomicMax per
+//                   column; with `update` set, the last CTA to finish (a
+//                   completion counter, no spinning) applies the momentum
+//                   recurrence to s in place and clears its scratch.
+//   quant_kernel    one CTA per token: 128-bit loads of the row, warp-shuffle
+//                   + shared-memory row max, RNE codes, 64-bit stores; also
+//                   emits the compact outlier codes XqO and, when asked, the
+//                   fp16 compensation operand U = XqO * (s - 1) as hi + lo.
+#pragma once
+
+#include "pack.cuh"
+
+namespace qlin {
+
+constexpr int kColmaxRows = 32;   // rows per CTA of colmax_kernel
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ float block_max_256(float v, float* red /* >= 8 floats */) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kQuantThreads / 32; ++w) r = fmaxf(r, red[w]);
+  return r;
+}
+
+// Momentum recurrence in fp32, exactly this association (no contraction).
+__device__ __forceinline__ float momentum_step(float s, float gamma, float cmax, float wmax) {
+  float beta = 1.f;
+  if (wmax > 0.f) {
+    const float r = __fsqrt_rn(__fdiv_rn(cmax, wmax));
+    beta = r > 1.f ? r : 1.f;
+  }
+  return __fadd_rn(__fmul_rn(gamma, s), __fmul_rn(__fsub_rn(1.f, gamma), beta));
+}
+
+// cmax_bits: fp32 bit patterns of non-negative maxima (ordered like uints).
+// With update != 0 the scratch (cmax_bits, counter) must be zero on entry
+// and is zero again on exit.
+__global__ void colmax_kernel(const uint16_t* __restrict__ X, int M, int K, const int32_t* __restrict__ O,
+                              int nO, unsigned* __restrict__ cmax_bits, int update,
+                              const float* __restrict__ wmaxO, float* __restrict__ s, float gamma,
+                              unsigned* __restrict__ counter) {
+  extern __shared__ unsigned char colmax_smem[];
+  int* sO = reinterpret_cast<int*>(colmax_smem);
+  unsigned* scm = reinterpret_cast<unsigned*>(sO + nO);
+  __shared__ int is_last;
+  for (int i = threadIdx.x; i < nO; i += blockDim.x) {
+    sO[i] = O[i];
+    scm[i] = 0u;
+  }
+  __syncthreads();
+  const int r0 = blockIdx.x * kColmaxRows;
+  const int r1 = min(M, r0 + kColmaxRows);
+  const int total = (r1 - r0) * nO;
+  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    const int m = r0 + idx / nO;
+    const int i = idx - (idx / nO) * nO;
+    const float v = fabsf(h2f(X[static_cast<size_t>(m) * K + sO[i]]));
+    atomicMax(&scm[i], __float_as_uint(v));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nO; i += blockDim.x)
+    if (scm[i]) atomicMax(&cmax_bits[i], scm[i]);
+  if (!update) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(counter, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < nO; i += blockDim.x) {
+    const float cm = __uint_as_float(atomicExch(&cmax_bits[i], 0u));
+    s[i] = momentum_step(s[i], gamma, cm, wmaxO[i]);
+  }
+  if (threadIdx.x == 0) *counter = 0u;
+}
+
+// Apply the recurrence from externally reduced maxima (data-parallel use).
+__global__ void momentum_kernel(const float* __restrict__ cmax, const float* __restrict__ wmaxO,
+                                float* __restrict__ s, float gamma, int nO) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < nO) s[i] = momentum_step(s[i], gamma, cmax[i], wmaxO[i]);
+}
+
+__device__ __forceinline__ int lower_bound_sorted(const int* a, int n, int key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int quant_code(float xh, float inv) {
+  return rne_clamp(__fmul_rn(xh, inv), 127);
+}
+
+// Compensation operand for one (token, outlier) pair: u = q * (s - 1) in
+// fp32, carried as hi = fp16(u) and lo = fp16(u - hi) (u - hi is exact in
+// fp32), so hi + lo matches u to about 2^-22 relative.  A single fp16
+// rounding of u is not accurate enough for the 2e-3 output tolerance when
+// the outlier terms cancel.
+__device__ __forceinline__ uint2 comp_split(int q, float s) {
+  const float u = __fmul_rn(static_cast<float>(q), __fsub_rn(s, 1.f));
+  const __half hi = __float2half_rn(u);
+  const __half lo = __float2half_rn(__fsub_rn(u, __half2float(hi)));
+  return make_uint2(__half_as_ushort(hi), __half_as_ushort(lo));
+}
+
+// One CTA per token row.  VPT = 8-element vectors per thread (K <= 2048*VPT).
+template <int VPT>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ O, int nO,
+             const float* __restrict__ s, int8_t* __restrict__ Xq, float* __restrict__ a,
+             int8_t* __restrict__ XqO, uint16_t* __restrict__ U, int nOp) {
+  extern __shared__ unsigned char quant_smem[];
+  int* sO = reinterpret_cast<int*>(quant_smem);
+  float* sS = reinterpret_cast<float*>(sO + nO);
+  unsigned* mask = reinterpret_cast<unsigned*>(sS + nO);
+  __shared__ float red[kQuantThreads / 32];
+
+  const int m = blockIdx.x;
+  const int nmask = K >> 5;
+  for (int w = threadIdx.x; w < nmask; w += kQuantThreads) mask[w] = 0u;
+  for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
+    sO[i] = O[i];
+    sS[i] = s[i];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nO; i += kQuantThreads) atomicOr(&mask[sO[i] >> 5], 1u << (sO[i] & 31));
+  __syncthreads();
+
+  const uint16_t* xrow = X + static_cast<size_t>(m) * K;
+  const uint4* xv = reinterpret_cast<const uint4*>(xrow);
+  const int nvec = K >> 3;
+  uint4 v[VPT];
+  float lmax = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int vi = threadIdx.x + j * kQuantThreads;
+    if (vi < nvec) {
+      v[j] = __ldg(xv + vi);
+      const unsigned mb = (mask[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint16_t hb = static_cast<uint16_t>(w4[e >> 1] >> ((e & 1) * 16));
+        const float f = fabsf(h2f(hb));
+        if (!((mb >> e) & 1u)) lmax = f > lmax ? f : lmax;
+      }
+    }
+  }
+  for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
+    const float xh = __fdiv_rn(h2f(xrow[sO[i]]), sS[i]);
+    const float f = fabsf(xh);
+    lmax = f > lmax ? f : lmax;
+  }
+  const float amax = block_max_256(lmax, red);
+  const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+  if (threadIdx.x == 0) a[m] = __fdiv_rn(amax, 127.f);
+
+  int8_t* qrow = Xq + static_cast<size_t>(m) * K;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int vi = threadIdx.x + j * kQuantThreads;
+    if (vi < nvec) {
+      const unsigned mb = (mask[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
+      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      int q[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint16_t hb = static_cast<uint16_t>(w4[e >> 1] >> ((e & 1) * 16));
+        float xh = h2f(hb);
+        if ((mb >> e) & 1u) {
+          const int i = lower_bound_sorted(sO, nO, vi * 8 + e);
+          xh = __fdiv_rn(xh, sS[i]);
+        }
+        q[e] = quant_code(xh, inv);
+      }
+      *reinterpret_cast<uint2*>(qrow + static_cast<size_t>(vi) * 8) = pack8_bytes(q);
+    }
+  }
+  const size_t lo_off = static_cast<size_t>(gridDim.x) * nOp;  // U holds [2][M][nOp]: hi rows, then lo rows
+  for (int i = threadIdx.x; i < nOp; i += kQuantThreads) {
+    if (i < nO) {
+      const float xh = __fdiv_rn(h2f(xrow[sO[i]]), sS[i]);
+      const int q = quant_code(xh, inv);
+      XqO[static_cast<size_t>(m) * nO + i] = static_cast<int8_t>(q);
+      if (U) {
+        const uint2 hl = comp_split(q, sS[i]);
+        U[static_cast<size_t>(m) * nOp + i] = static_cast<uint16_t>(hl.x);
+        U[lo_off + static_cast<size_t>(m) * nOp + i] = static_cast<uint16_t>(hl.y);
+      }
+    } else if (U) {
+      U[static_cast<size_t>(m) * nOp + i] = 0;
+      U[lo_off + static_cast<size_t>(m) * nOp + i] = 0;
+    }
+  }
+}
+
+// Compensation operand from already quantized outlier codes (qlin_gemm path):
+// U[0][m][i] = hi, U[1][m][i] = lo of XqO[m][i] * (s_i - 1); zero in the
+// padding columns.
+__global__ void comp_operand_kernel(const int8_t* __restrict__ XqO, const float* __restrict__ s, int M,
+                                    int nO, int nOp, uint16_t* __restrict__ U) {
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t total = static_cast<size_t>(M) * nOp;
+  if (idx >= total) return;
+  const int m = static_cast<int>(idx / nOp);
+  const int i = static_cast<int>(idx - static_cast<size_t>(m) * nOp);
+  uint2 hl = make_uint2(0u, 0u);
+  if (i < nO) hl = comp_split(XqO[static_cast<size_t>(m) * nO + i], s[i]);
+  U[idx] = static_cast<uint16_t>(hl.x);
+  U[total + idx] = static_cast<uint16_t>(hl.y);
+}
+
+}  // namespace qlin

@@ -1,0 +1,498 @@
+// qlin.cu -- the C ABI declared in include/qlin.h: host-side validation,
+// TMA descriptor encoding, launch selection.  All kernels live in the
+// headers included below so the library is one translation unit (the device
+// error word needs no relocatable device code).
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "qlin.h"
+#include "act_quant.cuh"
+#include "gemm.cuh"
+#include "pack.cuh"
+
+using namespace qlin;
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+qlin_status fail(qlin_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define QLIN_CUDA_TRY(expr)                                                                    \
+  do {                                                                                         \
+    cudaError_t e_ = (expr);                                                                   \
+    if (e_ != cudaSuccess)                                                                     \
+      return fail(QLIN_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));              \
+  } while (0)
+
+#define QLIN_LAUNCH_CHECK(what)                                                                \
+  do {                                                                                         \
+    cudaError_t e_ = cudaGetLastError();                                                       \
+    if (e_ != cudaSuccess) return fail(QLIN_ERR_CUDA, "%s launch failed: %s", what,           \
+                                       cudaGetErrorString(e_));                                \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int pad8(int n) { return (n + 7) / 8 * 8; }
+
+qlin_status check_shape(int32_t K, int32_t N, int32_t fmt, int32_t nO) {
+  if (fmt != QLIN_W4_PERCHANNEL && fmt != QLIN_W4_G128 && fmt != QLIN_W8_PERCHANNEL)
+    return fail(QLIN_ERR_ARG, "unknown weight format %d", fmt);
+  if (K <= 0 || N <= 0 || nO < 0) return fail(QLIN_ERR_ARG, "negative or zero size K=%d N=%d n_outlier=%d", K, N, nO);
+  if (K % 32 != 0 || K >= 131072) return fail(QLIN_ERR_SHAPE, "K=%d must be a multiple of 32 below 131072", K);
+  if (N % 16 != 0) return fail(QLIN_ERR_SHAPE, "N=%d must be a multiple of 16", N);
+  if (fmt == QLIN_W4_G128 && K % 128 != 0) return fail(QLIN_ERR_SHAPE, "g128 needs K %% 128 == 0 (K=%d)", K);
+  if (nO > K || nO > 4096) return fail(QLIN_ERR_SHAPE, "n_outlier=%d must be <= min(K, 4096)", nO);
+  return QLIN_OK;
+}
+
+struct Layout {
+  size_t codes, chan, group, fold, oidx, wot, wmax, total;
+};
+
+Layout weights_layout(int32_t K, int32_t N, int32_t fmt, int32_t nO) {
+  Layout L{};
+  size_t off = 0;
+  const size_t codes_b = (fmt == QLIN_W8_PERCHANNEL) ? size_t(K) * N : size_t(K) * N / 2;
+  L.codes = off; off = round_up(off + codes_b, kAlign);
+  L.chan = off; off = round_up(off + size_t(N) * 4, kAlign);
+  const size_t gb = (fmt == QLIN_W4_G128) ? size_t(K / 128) * N * 2 : 0;
+  L.group = off; off = round_up(off + gb, kAlign);
+  L.fold = off; off = round_up(off + gb, kAlign);
+  L.oidx = off; off = round_up(off + size_t(nO) * 4, kAlign);
+  L.wot = off; off = round_up(off + size_t(N) * pad8(nO) * 2, kAlign);
+  L.wmax = off; off = round_up(off + size_t(nO) * 4, kAlign);
+  L.total = off;
+  return L;
+}
+
+qlin_status check_weights(const qlin_weights* w) {
+  if (!w) return fail(QLIN_ERR_ARG, "weights descriptor is NULL");
+  qlin_status st = check_shape(w->K, w->N, w->fmt, w->n_outlier);
+  if (st != QLIN_OK) return st;
+  if (w->n_outlier_pad != pad8(w->n_outlier))
+    return fail(QLIN_ERR_ARG, "n_outlier_pad=%d must be n_outlier rounded up to 8 (%d)", w->n_outlier_pad, pad8(w->n_outlier));
+  if (w->fmt == QLIN_W4_G128 && w->group != 128) return fail(QLIN_ERR_ARG, "g128 format needs group=128");
+  if (w->fmt != QLIN_W4_G128 && w->group != 0) return fail(QLIN_ERR_ARG, "per-channel formats need group=0");
+  if (!w->codes || !w->chan_scale) return fail(QLIN_ERR_ARG, "codes/chan_scale is NULL");
+  if (w->fmt == QLIN_W4_G128 && (!w->group_scale || !w->fold_ratio)) return fail(QLIN_ERR_ARG, "g128 scales are NULL");
+  if (w->n_outlier > 0 && (!w->outlier_idx || !w->W_Ot || !w->wmax_O))
+    return fail(QLIN_ERR_ARG, "outlier buffers are NULL");
+  if (!aligned16(w->codes) || !aligned16(w->chan_scale) || (w->group_scale && !aligned16(w->group_scale)) ||
+      (w->fold_ratio && !aligned16(w->fold_ratio)) || (w->W_Ot && !aligned16(w->W_Ot)) ||
+      (w->outlier_idx && !aligned16(w->outlier_idx)) || (w->wmax_O && !aligned16(w->wmax_O)))
+    return fail(QLIN_ERR_ALIGN, "a weights buffer is not 16-byte aligned");
+  return QLIN_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+qlin_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(QLIN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  return QLIN_OK;
+}
+
+// 2-D map over a row-major [outer][inner] array of `esize`-byte elements.
+qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner,
+                     uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(esize)};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return QLIN_OK;
+}
+
+// ---------------------------------------------------------------- GEMM launch
+template <int FMT, int BT>
+qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_t* U, const GemmArgs& args,
+                          cudaStream_t stream) {
+  using C = GemmCfg<FMT, BT>;
+  constexpr int NCW = (FMT == kFmtW4G128) ? 8 : 4;
+  auto kern = gemm_kernel<FMT, BT, NCW>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+
+  CUtensorMap tmW, tmX, tmR, tmWO, tmU;
+  memset(&tmR, 0, sizeof(tmR));
+  memset(&tmWO, 0, sizeof(tmWO));
+  memset(&tmU, 0, sizeof(tmU));
+  qlin_status st;
+  const int K = w->K, N = w->N, M = args.M;
+  if (FMT == kFmtW8)
+    st = make_map(&tmW, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    st = make_map(&tmW, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != QLIN_OK) return st;
+  st = make_map(&tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, BT, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLIN_OK) return st;
+  if (FMT == kFmtW4G128) {
+    st = make_map(&tmR, w->fold_ratio, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, K / 128, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != QLIN_OK) return st;
+  }
+  if (w->n_outlier > 0) {
+    const int nOp = w->n_outlier_pad;
+    st = make_map(&tmWO, w->W_Ot, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, nOp, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QLIN_OK) return st;
+    st = make_map(&tmU, U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, nOp, 2 * static_cast<uint64_t>(M), 64, BT,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QLIN_OK) return st;
+  }
+  dim3 grid((N + C::kBN - 1) / C::kBN, (M + BT - 1) / BT);
+  kern<<<grid, 64 + 32 * NCW, C::kSmemBytes, stream>>>(tmW, tmX, tmR, tmWO, tmU, args);
+  QLIN_LAUNCH_CHECK("gemm_kernel");
+  return QLIN_OK;
+}
+
+template <int FMT>
+qlin_status launch_gemm_fmt(const qlin_weights* w, const int8_t* Xq, const uint16_t* U, const GemmArgs& args,
+                            cudaStream_t stream) {
+  const int M = args.M;
+  if (M <= 16) return launch_gemm_t<FMT, 16>(w, Xq, U, args, stream);
+  if (M <= 32) return launch_gemm_t<FMT, 32>(w, Xq, U, args, stream);
+  if (M <= 64) return launch_gemm_t<FMT, 64>(w, Xq, U, args, stream);
+  if (M <= 128) return launch_gemm_t<FMT, 128>(w, Xq, U, args, stream);
+  return launch_gemm_t<FMT, 256>(w, Xq, U, args, stream);
+}
+
+qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, const uint16_t* U, int M,
+                        uint16_t* Y, int32_t* acc_debug, cudaStream_t stream) {
+  qlin_status st = get_encoder();
+  if (st != QLIN_OK) return st;
+  GemmArgs args;
+  args.cscale = w->chan_scale;
+  args.a = a;
+  args.Y = Y;
+  args.acc_debug = acc_debug;
+  args.M = M;
+  args.N = w->N;
+  args.K = w->K;
+  args.nO = w->n_outlier;
+  switch (w->fmt) {
+    case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC>(w, Xq, U, args, stream);
+    case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128>(w, Xq, U, args, stream);
+    default: return launch_gemm_fmt<kFmtW8>(w, Xq, U, args, stream);
+  }
+}
+
+// ---------------------------------------------------------------- act quant
+size_t act_ws_bytes(const qlin_weights* w) {
+  return w->n_outlier > 0 ? round_up(size_t(w->n_outlier) * 4 + 4, kAlign) : 0;
+}
+
+qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float* s, float gamma, int update,
+                         int8_t* Xq, float* a, int8_t* XqO, uint16_t* U, void* act_ws, cudaStream_t stream) {
+  const int K = w->K, nO = w->n_outlier;
+  if (M == 0) return QLIN_OK;
+  if (update && nO > 0) {
+    unsigned* cmax = static_cast<unsigned*>(act_ws);
+    unsigned* counter = cmax + nO;
+    const int grid = (M + kColmaxRows - 1) / kColmaxRows;
+    colmax_kernel<<<grid, 256, size_t(nO) * 8, stream>>>(X, M, K, w->outlier_idx, nO, cmax, 1, w->wmax_O, s, gamma,
+                                                          counter);
+    QLIN_LAUNCH_CHECK("colmax_kernel");
+  }
+  const int nvec = K / 8;
+  const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
+  const size_t smem = size_t(nO) * 8 + size_t(K / 32) * 4;
+  const int nOp = w->n_outlier_pad;
+#define QLIN_QUANT_CASE(V)                                                                                \
+  quant_kernel<V><<<M, kQuantThreads, smem, stream>>>(X, K, w->outlier_idx, nO, s, Xq, a, XqO, U, nOp); \
+  QLIN_LAUNCH_CHECK("quant_kernel");                                                                      \
+  return QLIN_OK;
+  if (vpt <= 1) { QLIN_QUANT_CASE(1) }
+  if (vpt <= 2) { QLIN_QUANT_CASE(2) }
+  if (vpt <= 4) { QLIN_QUANT_CASE(4) }
+  if (vpt <= 8) { QLIN_QUANT_CASE(8) }
+  if (vpt <= 16) { QLIN_QUANT_CASE(16) }
+  if (vpt <= 32) { QLIN_QUANT_CASE(32) }
+  if (vpt <= 64) { QLIN_QUANT_CASE(64) }
+#undef QLIN_QUANT_CASE
+  return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", K);
+}
+
+size_t gemm_ws_bytes(int M, const qlin_weights* w) {
+  return w->n_outlier > 0 ? round_up(size_t(2) * M * w->n_outlier_pad * 2, kAlign) : 0;
+}
+
+struct FwdLayout {
+  size_t act, xq, a, xqo, u, total;
+};
+
+FwdLayout forward_layout(int M, const qlin_weights* w) {
+  FwdLayout L{};
+  size_t off = 0;
+  L.act = off; off = round_up(off + act_ws_bytes(w), kAlign);
+  L.xq = off; off = round_up(off + size_t(M) * w->K, kAlign);
+  L.a = off; off = round_up(off + size_t(M) * 4, kAlign);
+  L.xqo = off; off = round_up(off + size_t(M) * w->n_outlier, kAlign);
+  L.u = off; off = round_up(off + gemm_ws_bytes(M, w), kAlign);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* qlin_status_string(qlin_status s) {
+  switch (s) {
+    case QLIN_OK: return "QLIN_OK";
+    case QLIN_ERR_ARG: return "QLIN_ERR_ARG";
+    case QLIN_ERR_SHAPE: return "QLIN_ERR_SHAPE";
+    case QLIN_ERR_ALIGN: return "QLIN_ERR_ALIGN";
+    case QLIN_ERR_WORKSPACE: return "QLIN_ERR_WORKSPACE";
+    case QLIN_ERR_CUDA: return "QLIN_ERR_CUDA";
+    case QLIN_ERR_TIMEOUT: return "QLIN_ERR_TIMEOUT";
+  }
+  return "QLIN_UNKNOWN_STATUS";
+}
+
+const char* qlin_last_error(void) { return t_last_error; }
+
+qlin_status qlin_weights_bytes(int32_t K, int32_t N, int32_t fmt, int32_t n_outlier, size_t* bytes) {
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  qlin_status st = check_shape(K, N, fmt, n_outlier);
+  if (st != QLIN_OK) return st;
+  *bytes = weights_layout(K, N, fmt, n_outlier).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_weights_bind(qlin_weights* w, int32_t K, int32_t N, int32_t fmt, int32_t n_outlier, void* base,
+                              size_t bytes) {
+  if (!w || !base) return fail(QLIN_ERR_ARG, "weights descriptor or base is NULL");
+  qlin_status st = check_shape(K, N, fmt, n_outlier);
+  if (st != QLIN_OK) return st;
+  if (reinterpret_cast<uintptr_t>(base) % kAlign) return fail(QLIN_ERR_ALIGN, "base must be 256-byte aligned");
+  Layout L = weights_layout(K, N, fmt, n_outlier);
+  if (bytes < L.total) return fail(QLIN_ERR_WORKSPACE, "buffer of %zu bytes < %zu needed", bytes, L.total);
+  char* b = static_cast<char*>(base);
+  memset(w, 0, sizeof(*w));
+  w->K = K;
+  w->N = N;
+  w->fmt = fmt;
+  w->group = fmt == QLIN_W4_G128 ? 128 : 0;
+  w->n_outlier = n_outlier;
+  w->n_outlier_pad = pad8(n_outlier);
+  w->codes = b + L.codes;
+  w->chan_scale = reinterpret_cast<float*>(b + L.chan);
+  if (fmt == QLIN_W4_G128) {
+    w->group_scale = reinterpret_cast<uint16_t*>(b + L.group);
+    w->fold_ratio = reinterpret_cast<uint16_t*>(b + L.fold);
+  }
+  if (n_outlier > 0) {
+    w->outlier_idx = reinterpret_cast<int32_t*>(b + L.oidx);
+    w->W_Ot = reinterpret_cast<uint16_t*>(b + L.wot);
+    w->wmax_O = reinterpret_cast<float*>(b + L.wmax);
+  }
+  return QLIN_OK;
+}
+
+qlin_status qlin_pack_weights(const uint16_t* W, const int32_t* O_host, const qlin_weights* w, void* stream_) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (!W) return fail(QLIN_ERR_ARG, "W is NULL");
+  if (!aligned16(W)) return fail(QLIN_ERR_ALIGN, "W is not 16-byte aligned");
+  const int K = w->K, N = w->N, nO = w->n_outlier;
+  if (nO > 0) {
+    if (!O_host) return fail(QLIN_ERR_ARG, "O_host is NULL with n_outlier=%d", nO);
+    for (int i = 0; i < nO; ++i) {
+      if (O_host[i] < 0 || O_host[i] >= K) return fail(QLIN_ERR_ARG, "O[%d]=%d outside [0, K)", i, O_host[i]);
+      if (i > 0 && O_host[i] <= O_host[i - 1]) return fail(QLIN_ERR_ARG, "O is not strictly increasing at %d", i);
+    }
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const int threads = 128;
+  const int blocks = (N + threads - 1) / threads;
+  uint8_t* codes = static_cast<uint8_t*>(w->codes);
+  switch (w->fmt) {
+    case QLIN_W4_PERCHANNEL:
+      pack_per_channel_kernel<7, true><<<blocks, threads, 0, stream>>>(W, K, N, codes, w->chan_scale);
+      break;
+    case QLIN_W8_PERCHANNEL:
+      pack_per_channel_kernel<127, false><<<blocks, threads, 0, stream>>>(W, K, N, codes, w->chan_scale);
+      break;
+    default:
+      pack_group_kernel<128><<<blocks, threads, 0, stream>>>(W, K, N, codes, w->chan_scale, w->group_scale,
+                                                             w->fold_ratio);
+  }
+  QLIN_LAUNCH_CHECK("pack kernel");
+  if (nO > 0) {
+    QLIN_CUDA_TRY(cudaMemcpyAsync(w->outlier_idx, O_host, size_t(nO) * 4, cudaMemcpyHostToDevice, stream));
+    QLIN_CUDA_TRY(cudaMemsetAsync(w->W_Ot, 0, size_t(N) * w->n_outlier_pad * 2, stream));
+    pack_outliers_kernel<<<nO, 256, 0, stream>>>(W, N, w->outlier_idx, w->n_outlier_pad, w->W_Ot, w->wmax_O);
+    QLIN_LAUNCH_CHECK("pack_outliers_kernel");
+  }
+  return QLIN_OK;
+}
+
+qlin_status qlin_quant_act_workspace(int32_t M, const qlin_weights* w, size_t* bytes) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (!bytes || M < 0) return fail(QLIN_ERR_ARG, "bad arguments");
+  *bytes = act_ws_bytes(w);
+  return QLIN_OK;
+}
+
+qlin_status qlin_quant_act(const uint16_t* X, int32_t M, const qlin_weights* w, float* s, float gamma,
+                           int32_t update_momentum, int8_t* Xq, float* a, int8_t* XqO, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  const int nO = w->n_outlier;
+  if (M > 0 && (!X || !Xq || !a)) return fail(QLIN_ERR_ARG, "X/Xq/a is NULL");
+  if (nO > 0 && M > 0 && (!s || !XqO)) return fail(QLIN_ERR_ARG, "s/XqO is NULL with n_outlier=%d", nO);
+  if (!(gamma >= 0.f && gamma <= 1.f)) return fail(QLIN_ERR_ARG, "gamma=%g outside [0, 1]", double(gamma));
+  if ((X && !aligned16(X)) || (Xq && !aligned16(Xq)) || (a && !aligned16(a)) || (s && !aligned16(s)) ||
+      (XqO && !aligned16(XqO)))
+    return fail(QLIN_ERR_ALIGN, "an activation buffer is not 16-byte aligned");
+  const size_t need = (update_momentum ? act_ws_bytes(w) : 0);
+  if (ws_bytes < need || (need && !workspace)) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, need);
+  return launch_quant(X, M, w, s, gamma, update_momentum, Xq, a, XqO, nullptr, workspace,
+                      static_cast<cudaStream_t>(stream));
+}
+
+qlin_status qlin_outlier_colmax(const uint16_t* X, int32_t M, const qlin_weights* w, float* cmax, void* stream_) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  const int nO = w->n_outlier;
+  if (nO == 0) return QLIN_OK;
+  if (!cmax || (M > 0 && !X)) return fail(QLIN_ERR_ARG, "X/cmax is NULL");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  QLIN_CUDA_TRY(cudaMemsetAsync(cmax, 0, size_t(nO) * 4, stream));
+  if (M == 0) return QLIN_OK;
+  const int grid = (M + kColmaxRows - 1) / kColmaxRows;
+  colmax_kernel<<<grid, 256, size_t(nO) * 8, stream>>>(X, M, w->K, w->outlier_idx, nO,
+                                                        reinterpret_cast<unsigned*>(cmax), 0, nullptr, nullptr,
+                                                        0.f, nullptr);
+  QLIN_LAUNCH_CHECK("colmax_kernel");
+  return QLIN_OK;
+}
+
+qlin_status qlin_momentum_update(const qlin_weights* w, const float* cmax, float* s, float gamma, void* stream) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  const int nO = w->n_outlier;
+  if (nO == 0) return QLIN_OK;
+  if (!cmax || !s) return fail(QLIN_ERR_ARG, "cmax/s is NULL");
+  if (!(gamma >= 0.f && gamma <= 1.f)) return fail(QLIN_ERR_ARG, "gamma=%g outside [0, 1]", double(gamma));
+  momentum_kernel<<<(nO + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(cmax, w->wmax_O, s, gamma, nO);
+  QLIN_LAUNCH_CHECK("momentum_kernel");
+  return QLIN_OK;
+}
+
+qlin_status qlin_gemm_workspace(int32_t M, const qlin_weights* w, size_t* bytes) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (!bytes || M < 0) return fail(QLIN_ERR_ARG, "bad arguments");
+  *bytes = gemm_ws_bytes(M, w);
+  return QLIN_OK;
+}
+
+qlin_status qlin_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, const int8_t* XqO, const float* s,
+                      int32_t M, uint16_t* Y, int32_t* acc_debug, void* workspace, size_t ws_bytes,
+                      void* stream_) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  if (M == 0) return QLIN_OK;
+  const int nO = w->n_outlier;
+  if (!Xq || !a || !Y) return fail(QLIN_ERR_ARG, "Xq/a/Y is NULL");
+  if (nO > 0 && (!XqO || !s)) return fail(QLIN_ERR_ARG, "XqO/s is NULL with n_outlier=%d", nO);
+  if (!aligned16(Xq) || !aligned16(a) || !aligned16(Y) || (acc_debug && !aligned16(acc_debug)) ||
+      (XqO && !aligned16(XqO)) || (s && !aligned16(s)))
+    return fail(QLIN_ERR_ALIGN, "a GEMM buffer is not 16-byte aligned");
+  const size_t need = gemm_ws_bytes(M, w);
+  if (ws_bytes < need || (need && !workspace)) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, need);
+  if (need && !aligned16(workspace)) return fail(QLIN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint16_t* U = nullptr;
+  if (nO > 0) {
+    U = static_cast<uint16_t*>(workspace);
+    const size_t total = size_t(M) * w->n_outlier_pad;
+    comp_operand_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(XqO, s, M, nO,
+                                                                                       w->n_outlier_pad, U);
+    QLIN_LAUNCH_CHECK("comp_operand_kernel");
+  }
+  return launch_gemm(w, Xq, a, U, M, Y, acc_debug, stream);
+}
+
+qlin_status qlin_forward_workspace(int32_t M, const qlin_weights* w, size_t* bytes) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (!bytes || M < 0) return fail(QLIN_ERR_ARG, "bad arguments");
+  *bytes = forward_layout(M, w).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weights* w, float* s, float gamma,
+                         int32_t update_momentum, uint16_t* Y, void* workspace, size_t ws_bytes, void* stream_) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  if (M == 0) return QLIN_OK;
+  const int nO = w->n_outlier;
+  if (!X || !Y) return fail(QLIN_ERR_ARG, "X/Y is NULL");
+  if (nO > 0 && !s) return fail(QLIN_ERR_ARG, "s is NULL with n_outlier=%d", nO);
+  if (!(gamma >= 0.f && gamma <= 1.f)) return fail(QLIN_ERR_ARG, "gamma=%g outside [0, 1]", double(gamma));
+  if (!aligned16(X) || !aligned16(Y) || (s && !aligned16(s)))
+    return fail(QLIN_ERR_ALIGN, "X/Y/s is not 16-byte aligned");
+  FwdLayout L = forward_layout(M, w);
+  if (ws_bytes < L.total || !workspace) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, L.total);
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
+  char* ws = static_cast<char*>(workspace);
+  int8_t* Xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* a = reinterpret_cast<float*>(ws + L.a);
+  int8_t* XqO = nO > 0 ? reinterpret_cast<int8_t*>(ws + L.xqo) : nullptr;
+  uint16_t* U = nO > 0 ? reinterpret_cast<uint16_t*>(ws + L.u) : nullptr;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  st = launch_quant(X, M, w, s, gamma, update_momentum, Xq, a, XqO, U, ws + L.act, stream);
+  if (st != QLIN_OK) return st;
+  return launch_gemm(w, Xq, a, U, M, Y, nullptr, stream);
+}
+
+qlin_status qlin_poll_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
+  int flag = 0;
+  QLIN_CUDA_TRY(cudaMemcpyFromSymbol(&flag, qlin::g_device_error, sizeof(int)));
+  if (flag) {
+    const int zero = 0;
+    QLIN_CUDA_TRY(cudaMemcpyToSymbol(qlin::g_device_error, &zero, sizeof(int)));
+    return fail(QLIN_ERR_TIMEOUT, "a device-side bounded wait gave up (code %d)", flag);
+  }
+  return QLIN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,235 @@
+"""Thin ctypes binding of ``libqlin.so`` (the C ABI in include/qlin.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA
+library.  Tensors are torch CUDA tensors (PyTorch provides device memory and
+streams); each function passes their raw pointers and the current CUDA
+stream and raises :class:`QlinError` on a non-OK status.  There is no CPU or
+PyTorch fallback: if the library is missing, importing it fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlin.so")
+
+QLIN_W4_PERCHANNEL = 0
+QLIN_W4_G128 = 1
+QLIN_W8_PERCHANNEL = 2
+
+STATUS = {0: "QLIN_OK", 1: "QLIN_ERR_ARG", 2: "QLIN_ERR_SHAPE", 3: "QLIN_ERR_ALIGN",
+          4: "QLIN_ERR_WORKSPACE", 5: "QLIN_ERR_CUDA", 6: "QLIN_ERR_TIMEOUT"}
+
+EXPORTED = [
+    "qlin_status_string", "qlin_last_error", "qlin_weights_bytes", "qlin_weights_bind",
+    "qlin_pack_weights", "qlin_quant_act_workspace", "qlin_quant_act", "qlin_outlier_colmax",
+    "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
+    "qlin_forward", "qlin_poll_device_status",
+]
+
+
+class QlinError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class qlin_weights(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int32), ("N", ctypes.c_int32), ("fmt", ctypes.c_int32),
+        ("group", ctypes.c_int32), ("n_outlier", ctypes.c_int32), ("n_outlier_pad", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("chan_scale", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
+        ("fold_ratio", ctypes.c_void_p), ("outlier_idx", ctypes.c_void_p), ("W_Ot", ctypes.c_void_p),
+        ("wmax_O", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+P = ctypes.c_void_p
+I32 = ctypes.c_int32
+SZ = ctypes.c_size_t
+F32 = ctypes.c_float
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m quantized_linear_layers_token_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.qlin_status_string.argtypes = [ctypes.c_int]
+        L.qlin_status_string.restype = ctypes.c_char_p
+        L.qlin_last_error.argtypes = []
+        L.qlin_last_error.restype = ctypes.c_char_p
+        W = ctypes.POINTER(qlin_weights)
+        sigs = {
+            "qlin_weights_bytes": [I32, I32, I32, I32, ctypes.POINTER(SZ)],
+            "qlin_weights_bind": [W, I32, I32, I32, I32, P, SZ],
+            "qlin_pack_weights": [P, P, W, P],
+            "qlin_quant_act_workspace": [I32, W, ctypes.POINTER(SZ)],
+            "qlin_quant_act": [P, I32, W, P, F32, I32, P, P, P, P, SZ, P],
+            "qlin_outlier_colmax": [P, I32, W, P, P],
+            "qlin_momentum_update": [W, P, P, F32, P],
+            "qlin_gemm_workspace": [I32, W, ctypes.POINTER(SZ)],
+            "qlin_gemm": [W, P, P, P, P, I32, P, P, P, SZ, P],
+            "qlin_forward_workspace": [I32, W, ctypes.POINTER(SZ)],
+            "qlin_forward": [P, I32, W, P, F32, I32, P, P, SZ, P],
+            "qlin_poll_device_status": [P],
+        }
+        for name, argt in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = argt
+            fn.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise QlinError(status, where, lib().qlin_last_error().decode(errors="replace"))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _size(fn, *args) -> int:
+    out = SZ(0)
+    _check(fn(*args, ctypes.byref(out)), fn.__name__)
+    return int(out.value)
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+
+def qlin_weights_bytes(K: int, N: int, fmt: int, n_outlier: int) -> int:
+    return _size(lib().qlin_weights_bytes, K, N, fmt, n_outlier)
+
+
+def qlin_weights_bind(K: int, N: int, fmt: int, n_outlier: int, base: int, nbytes: int) -> qlin_weights:
+    w = qlin_weights()
+    _check(lib().qlin_weights_bind(ctypes.byref(w), K, N, fmt, n_outlier, base, nbytes), "qlin_weights_bind")
+    return w
+
+
+def qlin_pack_weights(W: torch.Tensor, O_host: np.ndarray, w: qlin_weights, stream=None):
+    O_host = np.ascontiguousarray(O_host, dtype=np.int32)
+    optr = O_host.ctypes.data if len(O_host) else None
+    _check(lib().qlin_pack_weights(_ptr(W), optr, ctypes.byref(w), _stream(stream)), "qlin_pack_weights")
+
+
+def qlin_quant_act_workspace(M: int, w: qlin_weights) -> int:
+    return _size(lib().qlin_quant_act_workspace, M, ctypes.byref(w))
+
+
+def qlin_quant_act(X, M: int, w: qlin_weights, s, gamma: float, update_momentum: bool, Xq, a, XqO,
+                   workspace, ws_bytes: int, stream=None):
+    _check(lib().qlin_quant_act(_ptr(X), M, ctypes.byref(w), _ptr(s), float(gamma), int(bool(update_momentum)),
+                                _ptr(Xq), _ptr(a), _ptr(XqO), _ptr(workspace), ws_bytes, _stream(stream)),
+           "qlin_quant_act")
+
+
+def qlin_outlier_colmax(X, M: int, w: qlin_weights, cmax, stream=None):
+    _check(lib().qlin_outlier_colmax(_ptr(X), M, ctypes.byref(w), _ptr(cmax), _stream(stream)),
+           "qlin_outlier_colmax")
+
+
+def qlin_momentum_update(w: qlin_weights, cmax, s, gamma: float, stream=None):
+    _check(lib().qlin_momentum_update(ctypes.byref(w), _ptr(cmax), _ptr(s), float(gamma), _stream(stream)),
+           "qlin_momentum_update")
+
+
+def qlin_gemm_workspace(M: int, w: qlin_weights) -> int:
+    return _size(lib().qlin_gemm_workspace, M, ctypes.byref(w))
+
+
+def qlin_gemm(w: qlin_weights, Xq, a, XqO, s, M: int, Y, acc_debug, workspace, ws_bytes: int, stream=None):
+    _check(lib().qlin_gemm(ctypes.byref(w), _ptr(Xq), _ptr(a), _ptr(XqO), _ptr(s), M, _ptr(Y), _ptr(acc_debug),
+                           _ptr(workspace), ws_bytes, _stream(stream)), "qlin_gemm")
+
+
+def qlin_forward_workspace(M: int, w: qlin_weights) -> int:
+    return _size(lib().qlin_forward_workspace, M, ctypes.byref(w))
+
+
+def qlin_forward(X, M: int, w: qlin_weights, s, gamma: float, update_momentum: bool, Y, workspace,
+                 ws_bytes: int, stream=None):
+    _check(lib().qlin_forward(_ptr(X), M, ctypes.byref(w), _ptr(s), float(gamma), int(bool(update_momentum)),
+                              _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)), "qlin_forward")
+
+
+def qlin_poll_device_status(stream=None):
+    _check(lib().qlin_poll_device_status(_stream(stream)), "qlin_poll_device_status")
+
+
+# ---------------------------------------------------------------------------
+# small conveniences over the entry points (allocation via torch only)
+# ---------------------------------------------------------------------------
+
+def empty_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zero-filled device buffer, 256-byte aligned (torch's allocator aligns
+    to 512 bytes), usable as any workspace."""
+    return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+class PackedLayer:
+    """One layer's packed weights in a single device buffer."""
+
+    def __init__(self, K: int, N: int, fmt: int, n_outlier: int, device="cuda"):
+        self.K, self.N, self.fmt, self.n_outlier = K, N, fmt, n_outlier
+        self.nbytes = qlin_weights_bytes(K, N, fmt, n_outlier)
+        self.buffer = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+        self.w = qlin_weights_bind(K, N, fmt, n_outlier, self.buffer.data_ptr(), self.nbytes)
+
+    @classmethod
+    def pack(cls, W: torch.Tensor, O: np.ndarray, fmt: int, stream=None) -> "PackedLayer":
+        K, N = W.shape
+        layer = cls(K, N, fmt, len(O), device=W.device)
+        qlin_pack_weights(W, O, layer.w, stream)
+        return layer
+
+    def clone(self) -> "PackedLayer":
+        """A copy at a distinct device address (same packed bytes)."""
+        other = PackedLayer(self.K, self.N, self.fmt, self.n_outlier, device=self.buffer.device)
+        other.buffer.copy_(self.buffer)
+        return other
+
+    def view(self, name: str) -> torch.Tensor:
+        """Typed view of one packed sub-buffer (for parity checks)."""
+        w = self.w
+        base = self.buffer.data_ptr()
+        K, N, nO, nOp = w.K, w.N, w.n_outlier, w.n_outlier_pad
+        spec = {
+            "codes": (w.codes, torch.uint8, (N, K // 2) if self.fmt != QLIN_W8_PERCHANNEL else (N, K)),
+            "chan_scale": (w.chan_scale, torch.float32, (N,)),
+            "group_scale": (w.group_scale, torch.int16, (K // 128, N)),
+            "fold_ratio": (w.fold_ratio, torch.int16, (K // 128, N)),
+            "outlier_idx": (w.outlier_idx, torch.int32, (nO,)),
+            "W_Ot": (w.W_Ot, torch.int16, (N, nOp)),
+            "wmax_O": (w.wmax_O, torch.float32, (nO,)),
+        }[name]
+        ptr, dtype, shape = spec
+        if ptr is None:
+            raise ValueError(f"{name} is not present in this format")
+        off = ptr - base
+        nbytes = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+        return self.buffer[off:off + nbytes].view(dtype).view(*shape)

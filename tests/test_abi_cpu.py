@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point declared in include/qlin.h, and the host-only calls and
+argument validation behave as documented (errors are returned before
+anything is enqueued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def q():
+    from quantized_linear_layers_token_b200 import build, qlin
+    build.build()
+    return qlin
+
+
+def declared_entry_points():
+    with open(os.path.join(ROOT, "include", "qlin.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"QLIN_API\s+(?:const\s+char\s*\*|qlin_status)\s+(qlin_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for must in ["qlin_pack_weights", "qlin_quant_act", "qlin_gemm", "qlin_forward"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(q):
+    L = ctypes.CDLL(q.LIB_PATH)
+    for name in declared_entry_points():
+        assert hasattr(L, name), name
+    assert set(declared_entry_points()) <= set(q.EXPORTED) | {"qlin_status_string", "qlin_last_error"}
+
+
+def test_status_strings(q):
+    L = q.lib()
+    for code, name in q.STATUS.items():
+        assert L.qlin_status_string(code).decode() == name
+
+
+def test_weights_bytes_and_bind(q):
+    K, N, nO = 4096, 11008, 41
+    for fmt in (0, 1, 2):
+        n = q.qlin_weights_bytes(K, N, fmt, nO)
+        codes = K * N if fmt == 2 else K * N // 2
+        assert n >= codes + 4 * N + N * 48 * 2
+        base = 1 << 20  # host-only: the descriptor is filled, memory untouched
+        w = q.qlin_weights_bind(K, N, fmt, nO, base, n)
+        assert (w.K, w.N, w.fmt, w.n_outlier, w.n_outlier_pad) == (K, N, fmt, nO, 48)
+        assert w.group == (128 if fmt == 1 else 0)
+        ptrs = [w.codes, w.chan_scale, w.outlier_idx, w.W_Ot, w.wmax_O]
+        assert all(p % 256 == 0 and base <= p < base + n for p in ptrs)
+        assert (w.group_scale is None) == (fmt != 1)
+
+
+@pytest.mark.parametrize("K,N,fmt,nO,status", [
+    (4100, 128, 0, 0, "QLIN_ERR_SHAPE"),   # K % 32
+    (4096, 120, 0, 0, "QLIN_ERR_SHAPE"),   # N % 16
+    (4064, 128, 1, 0, "QLIN_ERR_SHAPE"),   # g128 needs K % 128
+    (512, 128, 7, 0, "QLIN_ERR_ARG"),      # unknown format
+    (512, 128, 0, -1, "QLIN_ERR_ARG"),
+    (512, 128, 0, 600, "QLIN_ERR_SHAPE"),  # more outliers than channels
+    (0, 128, 0, 0, "QLIN_ERR_ARG"),
+])
+def test_shape_validation(q, K, N, fmt, nO, status):
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_weights_bytes(K, N, fmt, nO)
+    assert q.STATUS[e.value.status] == status
+
+
+def test_pack_rejects_bad_outlier_sets(q):
+    import numpy as np
+    K, N, nO = 256, 128, 3
+    n = q.qlin_weights_bytes(K, N, 0, nO)
+    w = q.qlin_weights_bind(K, N, 0, nO, 1 << 20, n)
+    fakeW = 1 << 24
+    for O in ([5, 5, 9], [9, 5, 7], [1, 2, 256], [-1, 2, 3]):
+        with pytest.raises(q.QlinError) as e:
+            q.qlin_pack_weights(fakeW, np.array(O, np.int32), w, stream=0)
+        assert q.STATUS[e.value.status] == "QLIN_ERR_ARG"
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_pack_weights(fakeW + 8, np.array([1, 2, 3], np.int32), w, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_ALIGN"
+
+
+def test_workspace_and_alignment_errors(q):
+    K, N, nO, M = 512, 128, 5, 16
+    n = q.qlin_weights_bytes(K, N, 0, nO)
+    w = q.qlin_weights_bind(K, N, 0, nO, 1 << 20, n)
+    need = q.qlin_forward_workspace(M, w)
+    assert need >= M * K + 4 * M + M * nO
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_forward(1 << 24, M, w, 1 << 25, 0.9, True, 1 << 26, 1 << 27, need - 1, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_WORKSPACE"
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_gemm(w, (1 << 24) + 4, 1 << 25, 1 << 26, 1 << 27, M, 1 << 28, None, 1 << 29, 1 << 20, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_ALIGN"
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_quant_act(1 << 24, M, w, 1 << 25, 1.5, True, 1 << 26, 1 << 27, 1 << 28, 1 << 29, 4096, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_ARG"  # gamma outside [0, 1]
