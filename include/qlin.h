@@ -166,6 +166,29 @@ QLIN_API qlin_status qlin_quant_act(const uint16_t* X, int32_t M, const qlin_wei
                            float gamma, int32_t update_momentum, int8_t* Xq, float* a,
                            int8_t* XqO, void* workspace, size_t ws_bytes, void* stream);
 
+/* qlin_quant_act without a workspace argument, for callers that cannot
+ * allocate device memory: code running inside a host framework that owns all
+ * GPU memory and forbids cudaMalloc once it has started (a plugin of an
+ * inference server, a custom pool), or a latency-bound loop that must not
+ * allocate because cudaMalloc may synchronize the device and take unbounded
+ * time.  The pages have no counterpart to this entry point; it only changes
+ * where the momentum update's scratch lives.
+ * Same arguments and results as qlin_quant_act.  The scratch (outlier column
+ * maxima and a completion counter) is a fixed array inside the library
+ * (16.25 KiB on every GPU that loads it, held until the process exits), so:
+ *   - n_outlier must be <= 1024, else QLIN_ERR_SHAPE and nothing is enqueued;
+ *   - no memory is allocated or freed; the call clears the part of the
+ *     scratch it uses with cudaMemsetAsync on `stream` before its kernels;
+ *   - every call on a device shares that one scratch: calls whose work
+ *     overlaps on the GPU (different streams, or different host threads)
+ *     race and may produce wrong momentum updates; serialize them;
+ *   - the first call on each device looks up the scratch's device address
+ *     (cudaGetSymbolAddress with that device current) and caches it; make
+ *     that first call before any stream capture. */
+QLIN_API qlin_status qlin_quant_act_noalloc(const uint16_t* X, int32_t M, const qlin_weights* w, float* s,
+                                            float gamma, int32_t update_momentum, int8_t* Xq, float* a,
+                                            int8_t* XqO, void* stream);
+
 /* Data-parallel split of the momentum update, for callers that shard tokens
  * across GPUs and must keep one s on every replica: qlin_outlier_colmax
  * writes cmax[i] = max_m |X[m, O_i]| (device fp32 [n_outlier]) over this

@@ -261,6 +261,41 @@ FwdLayout forward_layout(int M, const qlin_weights* w) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- allocation-free quantization
+// Fixed scratch for qlin_quant_act_noalloc: the outlier column maxima and the
+// completion counter of the momentum update.  It is a file-scope device
+// array, so every GPU that loads this library holds it (16.25 KiB) until the
+// process exits, and every call on a device shares the same copy.
+#define QLIN_NOALLOC_MAX_OUTLIERS 1024
+static __device__ __align__(256) unsigned g_noalloc_scratch[QLIN_NOALLOC_MAX_OUTLIERS + 64];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device.  In host code the
+// symbol names a host-side shadow, not device memory, so the address is
+// looked up once per device (with that device current) and cached.
+qlin_status noalloc_scratch(unsigned** out) {
+  int dev = -1;
+  QLIN_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(QLIN_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(QLIN_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return QLIN_OK;
+}
+
+}  // namespace
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -380,6 +415,34 @@ qlin_status qlin_quant_act(const uint16_t* X, int32_t M, const qlin_weights* w, 
   if (ws_bytes < need || (need && !workspace)) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, need);
   return launch_quant(X, M, w, s, gamma, update_momentum, Xq, a, XqO, nullptr, workspace,
                       static_cast<cudaStream_t>(stream));
+}
+
+qlin_status qlin_quant_act_noalloc(const uint16_t* X, int32_t M, const qlin_weights* w, float* s, float gamma,
+                                   int32_t update_momentum, int8_t* Xq, float* a, int8_t* XqO, void* stream_) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  const int nO = w->n_outlier;
+  if (nO > QLIN_NOALLOC_MAX_OUTLIERS)
+    return fail(QLIN_ERR_SHAPE, "n_outlier=%d exceeds the %d outlier channels the fixed scratch of "
+                "qlin_quant_act_noalloc holds; use qlin_quant_act with a workspace", nO, QLIN_NOALLOC_MAX_OUTLIERS);
+  if (M > 0 && (!X || !Xq || !a)) return fail(QLIN_ERR_ARG, "X/Xq/a is NULL");
+  if (nO > 0 && M > 0 && (!s || !XqO)) return fail(QLIN_ERR_ARG, "s/XqO is NULL with n_outlier=%d", nO);
+  if (!(gamma >= 0.f && gamma <= 1.f)) return fail(QLIN_ERR_ARG, "gamma=%g outside [0, 1]", double(gamma));
+  if ((X && !aligned16(X)) || (Xq && !aligned16(Xq)) || (a && !aligned16(a)) || (s && !aligned16(s)) ||
+      (XqO && !aligned16(XqO)))
+    return fail(QLIN_ERR_ALIGN, "an activation buffer is not 16-byte aligned");
+  if (M == 0) return QLIN_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  unsigned* scratch = nullptr;
+  if (update_momentum && nO > 0) {
+    st = noalloc_scratch(&scratch);
+    if (st != QLIN_OK) return st;
+    // The scratch keeps whatever the previous call left: clear the maxima
+    // and the counter (they must start at zero) before this call uses them.
+    QLIN_CUDA_TRY(cudaMemsetAsync(scratch, 0, (size_t(nO) + 1) * sizeof(unsigned), stream));
+  }
+  return launch_quant(X, M, w, s, gamma, update_momentum, Xq, a, XqO, nullptr, scratch, stream);
 }
 
 qlin_status qlin_outlier_colmax(const uint16_t* X, int32_t M, const qlin_weights* w, float* cmax, void* stream_) {

@@ -28,7 +28,7 @@ EXPORTED = [
     "qlin_status_string", "qlin_last_error", "qlin_weights_bytes", "qlin_weights_bind",
     "qlin_pack_weights", "qlin_quant_act_workspace", "qlin_quant_act", "qlin_outlier_colmax",
     "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
-    "qlin_forward", "qlin_poll_device_status",
+    "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc",
 ]
 
 
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "qlin_forward_workspace": [I32, W, ctypes.POINTER(SZ)],
             "qlin_forward": [P, I32, W, P, F32, I32, P, P, SZ, P],
             "qlin_poll_device_status": [P],
+            "qlin_quant_act_noalloc": [P, I32, W, P, F32, I32, P, P, P, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -146,6 +147,16 @@ def qlin_quant_act(X, M: int, w: qlin_weights, s, gamma: float, update_momentum:
     _check(lib().qlin_quant_act(_ptr(X), M, ctypes.byref(w), _ptr(s), float(gamma), int(bool(update_momentum)),
                                 _ptr(Xq), _ptr(a), _ptr(XqO), _ptr(workspace), ws_bytes, _stream(stream)),
            "qlin_quant_act")
+
+
+def qlin_quant_act_noalloc(X, M: int, w: qlin_weights, s, gamma: float, update_momentum: bool, Xq, a, XqO,
+                           stream=None):
+    """qlin_quant_act with the library's fixed internal scratch instead of a
+    caller workspace (for callers that cannot allocate device memory; at most
+    1024 outlier channels; calls that overlap on the GPU race)."""
+    _check(lib().qlin_quant_act_noalloc(_ptr(X), M, ctypes.byref(w), _ptr(s), float(gamma),
+                                        int(bool(update_momentum)), _ptr(Xq), _ptr(a), _ptr(XqO), _stream(stream)),
+           "qlin_quant_act_noalloc")
 
 
 def qlin_outlier_colmax(X, M: int, w: qlin_weights, cmax, stream=None):
