@@ -199,6 +199,40 @@ def build_problem(wl, copies, device):
     return layers, meta, inputs
 
 
+def run_profile_case(args, wl):
+    """A few qlin_forward calls on one linear of the workload (one weight
+    copy), launched eagerly so a profiler sees every kernel: W warm-up
+    calls, then K calls timed with CUDA events."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    name, m = args.profile_case.split(":")
+    M = int(m)
+    si = [n for n, _, _ in wl.shapes].index(name)
+    _, K, N = wl.shapes[si]
+    L = synth.layer(wl, si, M=M)
+    layer = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).cuda(), L["O"], wl.fmt)
+    X = torch.from_numpy(L["X"]).cuda()
+    s = torch.ones(max(len(L["O"]), 1), dtype=torch.float32, device="cuda")
+    Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    nws = qlin.qlin_forward_workspace(M, layer.w)
+    ws = qlin.empty_workspace(nws)
+    for _ in range(args.warmup):
+        qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
+    e1.record()
+    torch.cuda.synchronize()
+    qlin.qlin_poll_device_status()
+    us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
+    print(json.dumps({"profile_case": args.profile_case, "workload": wl.name, "K": K, "N": N, "M": M,
+                      "us_per_forward_eager": us}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -207,11 +241,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_w4_decode")
     ap.add_argument("--copies", type=int, default=4)
+    ap.add_argument("--profile-case", default=None,
+                    help="NAME:M -- run only that linear of the workload at M tokens (for ncu captures)")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
 
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.profile_case:
+        return run_profile_case(args, wl)
 
     import torch
     from quantized_linear_layers_token_b200 import qlin

@@ -327,7 +327,11 @@ def forward(X_bits: np.ndarray, W_bits: np.ndarray, packed: dict, s: np.ndarray,
     M = Xq.shape[0]
     if rows is None:
         rows = np.arange(M, dtype=np.int32)
-    acc, ovf = int_gemm_rows(Xq, packed["B"], rows)
-    assert not ovf
-    y = dequant(acc, a, packed["cscale"], XqO, s1, W_bits, O, rows)
+    if len(rows):
+        acc, ovf = int_gemm_rows(Xq, packed["B"], rows)
+        assert not ovf
+        y = dequant(acc, a, packed["cscale"], XqO, s1, W_bits, O, rows)
+    else:
+        acc = np.zeros((0, packed["N"]), np.int64)
+        y = np.zeros((0, packed["N"]), np.float64)
     return {"s": s1, "Xq": Xq, "a": a, "XqO": XqO, "acc": acc, "y": y, "rows": rows}

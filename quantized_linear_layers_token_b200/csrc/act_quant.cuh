@@ -27,6 +27,8 @@ namespace qlin {
 
 constexpr int kColmaxRows = 32;   // rows per CTA of colmax_kernel
 constexpr int kQuantThreads = 256;
+constexpr int kFusedMomentumMaxM = 64;  // up to this many tokens the update runs inside quant_kernel
+
 
 __device__ __forceinline__ float block_max_256(float v, float* red /* >= 8 floats */) {
 #pragma unroll
@@ -60,6 +62,8 @@ __global__ void colmax_kernel(const uint16_t* __restrict__ X, int M, int K, cons
   int* sO = reinterpret_cast<int*>(colmax_smem);
   unsigned* scm = reinterpret_cast<unsigned*>(sO + nO);
   __shared__ int is_last;
+  griddep_launch_dependents();
+  griddep_wait();
   for (int i = threadIdx.x; i < nO; i += blockDim.x) {
     sO[i] = O[i];
     scm[i] = 0u;
@@ -123,24 +127,47 @@ __device__ __forceinline__ uint2 comp_split(int q, float s) {
   return make_uint2(__half_as_ushort(hi), __half_as_ushort(lo));
 }
 
+struct MomentumArgs {
+  const float* wmaxO;  // [nO]
+  float gamma;
+  unsigned* counter;   // completion counter (zero on entry, left zero)
+  int M;               // rows of X (all of them feed the column maxima)
+};
+
 // One CTA per token row.  VPT = 8-element vectors per thread (K <= 2048*VPT).
-template <int VPT>
+// FUSED: every CTA also computes the outlier column maxima over all M rows
+// and the momentum update itself (identical in every CTA, cheap for small
+// M); the last CTA to finish writes the new state back, after every CTA has
+// read the old one.
+template <int VPT, bool FUSED>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ O, int nO,
-             const float* __restrict__ s, int8_t* __restrict__ Xq, float* __restrict__ a,
-             int8_t* __restrict__ XqO, uint16_t* __restrict__ U, int nOp) {
+             float* __restrict__ s, int8_t* __restrict__ Xq, float* __restrict__ a,
+             int8_t* __restrict__ XqO, uint16_t* __restrict__ U, int nOp, MomentumArgs mom) {
   extern __shared__ unsigned char quant_smem[];
   int* sO = reinterpret_cast<int*>(quant_smem);
   float* sS = reinterpret_cast<float*>(sO + nO);
   unsigned* mask = reinterpret_cast<unsigned*>(sS + nO);
   __shared__ float red[kQuantThreads / 32];
+  __shared__ int is_last;
 
+  griddep_launch_dependents();
+  griddep_wait();  // X (and s) may come from the previous kernel
   const int m = blockIdx.x;
   const int nmask = K >> 5;
   for (int w = threadIdx.x; w < nmask; w += kQuantThreads) mask[w] = 0u;
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
     sO[i] = O[i];
-    sS[i] = s[i];
+    float si = s[i];
+    if (FUSED) {
+      float cm = 0.f;
+      for (int r = 0; r < mom.M; ++r) {
+        const float v = fabsf(h2f(X[static_cast<size_t>(r) * K + sO[i]]));
+        cm = v > cm ? v : cm;
+      }
+      si = momentum_step(si, mom.gamma, cm, mom.wmaxO[i]);
+    }
+    sS[i] = si;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) atomicOr(&mask[sO[i] >> 5], 1u << (sO[i] & 31));
@@ -210,6 +237,15 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     } else if (U) {
       U[static_cast<size_t>(m) * nOp + i] = 0;
       U[lo_off + static_cast<size_t>(m) * nOp + i] = 0;
+    }
+  }
+  if (FUSED) {
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomicAdd(mom.counter, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (is_last) {
+      for (int i = threadIdx.x; i < nO; i += kQuantThreads) s[i] = sS[i];
+      if (threadIdx.x == 0) *mom.counter = 0u;
     }
   }
 }

@@ -127,13 +127,98 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
   return QLIN_OK;
 }
 
+// ---------------------------------------------------------------- launches
+// Kernels are launched with programmatic dependent launch, so each may start
+// its prologue (and the GEMM its weight stream) while the previous kernel in
+// the stream finishes; every kernel waits on the grid dependency before it
+// reads what the previous one wrote.  QLIN_NO_PDL=1 turns this off.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("QLIN_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+int pick_bt(int M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
+}
+
+// Work decomposition of one GEMM call (same on the host for workspace sizes
+// and for the launch).
+struct GemmPlan {
+  int bt, tiles_n, tiles_m, nk, nc, ncs, T, grid, split;
+  size_t u_off, acc_off, comp_off, cnt_off, total;
+};
+
+GemmPlan plan_gemm(int M, const qlin_weights* w) {
+  GemmPlan p{};
+  p.bt = pick_bt(M);
+  p.tiles_n = (w->N + 127) / 128;
+  p.tiles_m = (M + p.bt - 1) / p.bt;
+  p.nk = (w->K + 127) / 128;
+  p.ncs = w->n_outlier > 0 ? (w->n_outlier + 63) / 64 : 0;
+  p.nc = (p.bt <= 64) ? p.ncs : 2 * p.ncs;
+  p.T = p.nk + p.nc;
+  const int sms = sm_count();
+  const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
+  p.split = tiles < 4LL * sms ? 1 : 0;
+  const long long units = p.split ? tiles * p.T : tiles;
+  const int cap = sms < kMaxGrid ? sms : kMaxGrid;
+  p.grid = static_cast<int>(units < cap ? units : cap);
+  if (p.grid < 1) p.grid = 1;
+  size_t off = 0;
+  p.u_off = off;
+  off = round_up(off + (w->n_outlier > 0 ? size_t(2) * M * w->n_outlier_pad * 2 : 0), kAlign);
+  const size_t slot_bytes = size_t(p.bt) * 128 * 4;
+  p.acc_off = off;
+  off = round_up(off + (p.split ? size_t(2) * p.grid * slot_bytes : 0), kAlign);
+  p.comp_off = off;
+  off = round_up(off + (p.split && w->n_outlier > 0 ? size_t(2) * p.grid * slot_bytes : 0), kAlign);
+  p.cnt_off = off;
+  off = round_up(off + (p.split ? size_t(p.grid) * 4 : 0), kAlign);
+  p.total = off;
+  return p;
+}
+
 // ---------------------------------------------------------------- GEMM launch
 template <int FMT, int BT>
-qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_t* U, const GemmArgs& args,
+qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_t* U, GemmArgs args,
                           cudaStream_t stream) {
   using C = GemmCfg<FMT, BT>;
-  constexpr int NCW = (FMT == kFmtW4G128) ? 8 : 4;
-  auto kern = gemm_kernel<FMT, BT, NCW>;
+  auto kern = gemm_kernel<FMT, BT>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
@@ -166,40 +251,58 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != QLIN_OK) return st;
   }
-  dim3 grid((N + C::kBN - 1) / C::kBN, (M + BT - 1) / BT);
-  kern<<<grid, 64 + 32 * NCW, C::kSmemBytes, stream>>>(tmW, tmX, tmR, tmWO, tmU, args);
-  QLIN_LAUNCH_CHECK("gemm_kernel");
+  cudaError_t e = launch_k(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, tmW, tmX, tmR, tmWO,
+                           tmU, args);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
 }
 
 template <int FMT>
-qlin_status launch_gemm_fmt(const qlin_weights* w, const int8_t* Xq, const uint16_t* U, const GemmArgs& args,
+qlin_status launch_gemm_fmt(int bt, const qlin_weights* w, const int8_t* Xq, const uint16_t* U, const GemmArgs& args,
                             cudaStream_t stream) {
-  const int M = args.M;
-  if (M <= 16) return launch_gemm_t<FMT, 16>(w, Xq, U, args, stream);
-  if (M <= 32) return launch_gemm_t<FMT, 32>(w, Xq, U, args, stream);
-  if (M <= 64) return launch_gemm_t<FMT, 64>(w, Xq, U, args, stream);
-  if (M <= 128) return launch_gemm_t<FMT, 128>(w, Xq, U, args, stream);
-  return launch_gemm_t<FMT, 256>(w, Xq, U, args, stream);
+  switch (bt) {
+    case 16: return launch_gemm_t<FMT, 16>(w, Xq, U, args, stream);
+    case 32: return launch_gemm_t<FMT, 32>(w, Xq, U, args, stream);
+    case 64: return launch_gemm_t<FMT, 64>(w, Xq, U, args, stream);
+    case 128: return launch_gemm_t<FMT, 128>(w, Xq, U, args, stream);
+    default: return launch_gemm_t<FMT, 256>(w, Xq, U, args, stream);
+  }
 }
 
-qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, const uint16_t* U, int M,
-                        uint16_t* Y, int32_t* acc_debug, cudaStream_t stream) {
+// `gws` is the GEMM scratch laid out by plan_gemm (U first).
+qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, int M, uint16_t* Y,
+                        int32_t* acc_debug, char* gws, cudaStream_t stream) {
   qlin_status st = get_encoder();
   if (st != QLIN_OK) return st;
+  const GemmPlan p = plan_gemm(M, w);
   GemmArgs args;
   args.cscale = w->chan_scale;
   args.a = a;
   args.Y = Y;
   args.acc_debug = acc_debug;
+  args.ws_acc = reinterpret_cast<int32_t*>(gws + p.acc_off);
+  args.ws_comp = reinterpret_cast<float*>(gws + p.comp_off);
+  args.ws_cnt = reinterpret_cast<unsigned*>(gws + p.cnt_off);
   args.M = M;
   args.N = w->N;
   args.K = w->K;
   args.nO = w->n_outlier;
+  args.tiles_n = p.tiles_n;
+  args.tiles_m = p.tiles_m;
+  args.nk = p.nk;
+  args.nc = p.nc;
+  args.ncs = p.ncs;
+  args.T = p.T;
+  args.grid = p.grid;
+  args.split = p.split;
+  const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
+  if (tiles * p.T >= (1LL << 31)) return fail(QLIN_ERR_SHAPE, "problem too large (%lld tile iterations)", tiles * p.T);
+  for (int c = 0; c <= p.grid; ++c) args.bnd[c] = gemm_boundary(c, tiles, p.T, p.nk, p.grid, p.split);
+  const uint16_t* U = reinterpret_cast<const uint16_t*>(gws + p.u_off);
   switch (w->fmt) {
-    case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC>(w, Xq, U, args, stream);
-    case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128>(w, Xq, U, args, stream);
-    default: return launch_gemm_fmt<kFmtW8>(w, Xq, U, args, stream);
+    case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC>(p.bt, w, Xq, U, args, stream);
+    case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128>(p.bt, w, Xq, U, args, stream);
+    default: return launch_gemm_fmt<kFmtW8>(p.bt, w, Xq, U, args, stream);
   }
 }
 
@@ -212,39 +315,44 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
                          int8_t* Xq, float* a, int8_t* XqO, uint16_t* U, void* act_ws, cudaStream_t stream) {
   const int K = w->K, nO = w->n_outlier;
   if (M == 0) return QLIN_OK;
-  if (update && nO > 0) {
-    unsigned* cmax = static_cast<unsigned*>(act_ws);
-    unsigned* counter = cmax + nO;
+  unsigned* cmax = static_cast<unsigned*>(act_ws);
+  MomentumArgs mom{w->wmax_O, gamma, cmax + nO, M};
+  const bool do_update = update && nO > 0;
+  const bool fused = do_update && M <= kFusedMomentumMaxM;
+  if (do_update && !fused) {
     const int grid = (M + kColmaxRows - 1) / kColmaxRows;
-    colmax_kernel<<<grid, 256, size_t(nO) * 8, stream>>>(X, M, K, w->outlier_idx, nO, cmax, 1, w->wmax_O, s, gamma,
-                                                          counter);
-    QLIN_LAUNCH_CHECK("colmax_kernel");
+    cudaError_t e = launch_k(colmax_kernel, dim3(grid), dim3(256), size_t(nO) * 8, stream, X, M, K,
+                             static_cast<const int32_t*>(w->outlier_idx), nO, cmax, 1,
+                             static_cast<const float*>(w->wmax_O), s, gamma, cmax + nO);
+    if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "colmax_kernel launch failed: %s", cudaGetErrorString(e));
   }
   const int nvec = K / 8;
   const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
   const size_t smem = size_t(nO) * 8 + size_t(K / 32) * 4;
   const int nOp = w->n_outlier_pad;
-#define QLIN_QUANT_CASE(V)                                                                                \
-  quant_kernel<V><<<M, kQuantThreads, smem, stream>>>(X, K, w->outlier_idx, nO, s, Xq, a, XqO, U, nOp); \
-  QLIN_LAUNCH_CHECK("quant_kernel");                                                                      \
-  return QLIN_OK;
+  cudaError_t e = cudaSuccess;
+#define QLIN_QUANT_CASE(V)                                                                               \
+  e = fused ? launch_k(quant_kernel<V, true>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,         \
+                       static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom)     \
+            : launch_k(quant_kernel<V, false>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,        \
+                       static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom);
   if (vpt <= 1) { QLIN_QUANT_CASE(1) }
-  if (vpt <= 2) { QLIN_QUANT_CASE(2) }
-  if (vpt <= 4) { QLIN_QUANT_CASE(4) }
-  if (vpt <= 8) { QLIN_QUANT_CASE(8) }
-  if (vpt <= 16) { QLIN_QUANT_CASE(16) }
-  if (vpt <= 32) { QLIN_QUANT_CASE(32) }
-  if (vpt <= 64) { QLIN_QUANT_CASE(64) }
+  else if (vpt <= 2) { QLIN_QUANT_CASE(2) }
+  else if (vpt <= 4) { QLIN_QUANT_CASE(4) }
+  else if (vpt <= 8) { QLIN_QUANT_CASE(8) }
+  else if (vpt <= 16) { QLIN_QUANT_CASE(16) }
+  else if (vpt <= 32) { QLIN_QUANT_CASE(32) }
+  else if (vpt <= 64) { QLIN_QUANT_CASE(64) }
+  else return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", K);
 #undef QLIN_QUANT_CASE
-  return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", K);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "quant_kernel launch failed: %s", cudaGetErrorString(e));
+  return QLIN_OK;
 }
 
-size_t gemm_ws_bytes(int M, const qlin_weights* w) {
-  return w->n_outlier > 0 ? round_up(size_t(2) * M * w->n_outlier_pad * 2, kAlign) : 0;
-}
+size_t gemm_ws_bytes(int M, const qlin_weights* w) { return M > 0 ? plan_gemm(M, w).total : 0; }
 
 struct FwdLayout {
-  size_t act, xq, a, xqo, u, total;
+  size_t act, xq, a, xqo, gemm, total;
 };
 
 FwdLayout forward_layout(int M, const qlin_weights* w) {
@@ -254,7 +362,7 @@ FwdLayout forward_layout(int M, const qlin_weights* w) {
   L.xq = off; off = round_up(off + size_t(M) * w->K, kAlign);
   L.a = off; off = round_up(off + size_t(M) * 4, kAlign);
   L.xqo = off; off = round_up(off + size_t(M) * w->n_outlier, kAlign);
-  L.u = off; off = round_up(off + gemm_ws_bytes(M, w), kAlign);
+  L.gemm = off; off = round_up(off + gemm_ws_bytes(M, w), kAlign);
   L.total = off;
   return L;
 }
@@ -498,17 +606,18 @@ qlin_status qlin_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, c
     return fail(QLIN_ERR_ALIGN, "a GEMM buffer is not 16-byte aligned");
   const size_t need = gemm_ws_bytes(M, w);
   if (ws_bytes < need || (need && !workspace)) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, need);
-  if (need && !aligned16(workspace)) return fail(QLIN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  if (need && reinterpret_cast<uintptr_t>(workspace) % kAlign)
+    return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  uint16_t* U = nullptr;
+  char* gws = static_cast<char*>(workspace);
   if (nO > 0) {
-    U = static_cast<uint16_t*>(workspace);
+    uint16_t* U = reinterpret_cast<uint16_t*>(gws + plan_gemm(M, w).u_off);
     const size_t total = size_t(M) * w->n_outlier_pad;
     comp_operand_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(XqO, s, M, nO,
                                                                                        w->n_outlier_pad, U);
     QLIN_LAUNCH_CHECK("comp_operand_kernel");
   }
-  return launch_gemm(w, Xq, a, U, M, Y, acc_debug, stream);
+  return launch_gemm(w, Xq, a, M, Y, acc_debug, gws, stream);
 }
 
 qlin_status qlin_forward_workspace(int32_t M, const qlin_weights* w, size_t* bytes) {
@@ -538,12 +647,21 @@ qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weights* w, fl
   int8_t* Xq = reinterpret_cast<int8_t*>(ws + L.xq);
   float* a = reinterpret_cast<float*>(ws + L.a);
   int8_t* XqO = nO > 0 ? reinterpret_cast<int8_t*>(ws + L.xqo) : nullptr;
-  uint16_t* U = nO > 0 ? reinterpret_cast<uint16_t*>(ws + L.u) : nullptr;
+  char* gws = ws + L.gemm;
+  uint16_t* U = nO > 0 ? reinterpret_cast<uint16_t*>(gws + plan_gemm(M, w).u_off) : nullptr;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   st = launch_quant(X, M, w, s, gamma, update_momentum, Xq, a, XqO, U, ws + L.act, stream);
   if (st != QLIN_OK) return st;
-  return launch_gemm(w, Xq, a, U, M, Y, nullptr, stream);
+  return launch_gemm(w, Xq, a, M, Y, nullptr, gws, stream);
 }
+
+#ifdef QLIN_TRACE
+// Diagnostic builds only: point the GEMM's phase stamps at a device buffer
+// of [grid][16] int64 (NULL turns them off).
+QLIN_API int qlin_trace_set(long long* p) {
+  return static_cast<int>(cudaMemcpyToSymbol(qlin::g_trace, &p, sizeof(p)));
+}
+#endif
 
 qlin_status qlin_poll_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
