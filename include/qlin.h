@@ -34,7 +34,7 @@
  *     is enqueued and leave all buffers untouched.
  *   - Matrices are row-major with dense rows (no padding) unless stated.
  *   - Device pointers must be 16-byte aligned (QLIN_ERR_ALIGN otherwise).
- *   - Shapes: K % 32 == 0, N % 16 == 0, 1 <= K < 131072, N >= 16; for the
+ *   - Shapes: K % 32 == 0, N % 16 == 0, 32 <= K <= 65536, N >= 16; for the
  *     g128 format K % 128 == 0; 0 <= n_outlier <= min(K, 4096).
  *   - Workspaces: buffers whose size comes from the matching *_workspace
  *     call.  A workspace must be zero-filled before its first use (for
@@ -81,21 +81,32 @@ typedef enum {
  * Plain descriptor: every pointer is device memory owned by the caller, and
  * qlin_weights_bind() can carve all of them out of one allocation.
  *
- *   codes        W4 formats: uint8 [N][K/2].  For the 32-bit little-endian
- *                word of row n that covers input channels k0..k0+7, byte b
- *                (0..3) holds q[k0+b] in its low nibble and q[k0+4+b] in its
- *                high nibble (two's complement).  Then (word << 4) & 0xF0F0F0F0
- *                holds the INT8 lanes 16*q[k0..k0+3] and word & 0xF0F0F0F0
- *                the lanes 16*q[k0+4..k0+7].
- *                W8 format: int8 [N][K] (row n = output channel n).
+ *   codes        Tile-major, one contiguous block per (channel tile tn,
+ *                input tile kb) of 128 output channels x 128 input channels,
+ *                blocks ordered tn-major: block (tn, kb) starts at
+ *                (tn * ceil(K/128) + kb) * block_bytes.  Row r of a block is
+ *                channel 128*tn + r; channels >= N and inputs >= K are zero.
+ *                W4 formats: 8192-byte blocks, 64 bytes per row.  In the
+ *                32-bit little-endian word of a row that covers inputs
+ *                k0..k0+7, byte b (0..3) holds q[k0+b] in its low nibble and
+ *                q[k0+4+b] in its high nibble (two's complement); then
+ *                (word << 4) & 0xF0F0F0F0 holds the INT8 lanes 16*q[k0..k0+3]
+ *                and word & 0xF0F0F0F0 the lanes 16*q[k0+4..k0+7].
+ *                W8 format: 16384-byte blocks, 128 bytes per row, stored with
+ *                the tensor core's 128-byte swizzle: the 16-byte chunk c
+ *                (inputs 16c..16c+15 of the tile) of row r sits at chunk
+ *                c ^ (r % 8) of that row.
  *   chan_scale   c_n, fp32 [N].  Per-channel formats: c_n = max_k|W[k][n]| / qmax
  *                (qmax = 7 or 127).  g128: c_n = 7 * max_j g[j][n] / 127.
  *   group_scale  g128 only: g[j][n] = fp16(max_{k in group j}|W[k][n]| / 7), fp16 [K/128][N].
  *   fold_ratio   g128 only: r[j][n] = fp16(g[j][n] / c_n), fp16 [K/128][N].
  *   outlier_idx  O, int32 [n_outlier], strictly increasing, in [0, K).
- *   W_Ot         fp16 [N][n_outlier_pad]: W_Ot[n][i] = W[O_i][n]; columns
- *                n_outlier .. n_outlier_pad-1 are zero.  The outlier rows of
- *                W kept in full precision.
+ *   W_Ot         The outlier rows of W kept in fp16 ("full precision"),
+ *                transposed and tiled: one 16384-byte block per (channel
+ *                tile tn, outlier tile ib) of 128 channels x 64 outliers,
+ *                ordered tn-major; row r holds W[O_i][128*tn + r] for
+ *                i = 64*ib .. 64*ib+63 (128 bytes) with the same 128-byte
+ *                swizzle as the W8 codes; padding is zero.
  *   wmax_O       fp32 [n_outlier]: max_n |W[O_i][n]| (the weight side of beta).
  */
 typedef struct {
@@ -104,7 +115,8 @@ typedef struct {
   int32_t fmt;           /* qlin_wfmt */
   int32_t group;         /* 128 for QLIN_W4_G128, else 0 */
   int32_t n_outlier;     /* |O| */
-  int32_t n_outlier_pad; /* n_outlier rounded up to a multiple of 8 */
+  int32_t n_outlier_pad; /* n_outlier rounded up to a multiple of 8 (row stride of the
+                            compensation operand in the GEMM workspace) */
   void* codes;
   float* chan_scale;
   uint16_t* group_scale;

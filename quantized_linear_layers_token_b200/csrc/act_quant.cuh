@@ -139,13 +139,16 @@ struct MomentumArgs {
 // and the momentum update itself (identical in every CTA, cheap for small
 // M); the last CTA to finish writes the new state back, after every CTA has
 // read the old one.
+// Latency: the row is requested first (independent of O), then staged in
+// shared memory so every outlier lookup is a shared-memory read.
 template <int VPT, bool FUSED>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ O, int nO,
              float* __restrict__ s, int8_t* __restrict__ Xq, float* __restrict__ a,
              int8_t* __restrict__ XqO, uint16_t* __restrict__ U, int nOp, MomentumArgs mom) {
-  extern __shared__ unsigned char quant_smem[];
-  int* sO = reinterpret_cast<int*>(quant_smem);
+  extern __shared__ __align__(16) unsigned char quant_smem[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(quant_smem);          // [K] this row
+  int* sO = reinterpret_cast<int*>(quant_smem + static_cast<size_t>(K) * 2);
   float* sS = reinterpret_cast<float*>(sO + nO);
   unsigned* mask = reinterpret_cast<unsigned*>(sS + nO);
   __shared__ float red[kQuantThreads / 32];
@@ -154,35 +157,46 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
   griddep_launch_dependents();
   griddep_wait();  // X (and s) may come from the previous kernel
   const int m = blockIdx.x;
-  const int nmask = K >> 5;
-  for (int w = threadIdx.x; w < nmask; w += kQuantThreads) mask[w] = 0u;
-  for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
-    sO[i] = O[i];
-    float si = s[i];
-    if (FUSED) {
-      float cm = 0.f;
-      for (int r = 0; r < mom.M; ++r) {
-        const float v = fabsf(h2f(X[static_cast<size_t>(r) * K + sO[i]]));
-        cm = v > cm ? v : cm;
-      }
-      si = momentum_step(si, mom.gamma, cm, mom.wmaxO[i]);
-    }
-    sS[i] = si;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < nO; i += kQuantThreads) atomicOr(&mask[sO[i] >> 5], 1u << (sO[i] & 31));
-  __syncthreads();
-
   const uint16_t* xrow = X + static_cast<size_t>(m) * K;
   const uint4* xv = reinterpret_cast<const uint4*>(xrow);
   const int nvec = K >> 3;
   uint4 v[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int vi = threadIdx.x + j * kQuantThreads;
+    if (vi < nvec) v[j] = __ldg(xv + vi);
+  }
+  const int nmask = K >> 5;
+  for (int w = threadIdx.x; w < nmask; w += kQuantThreads) mask[w] = 0u;
+  for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
+    sO[i] = O[i];
+    sS[i] = s[i];
+  }
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int vi = threadIdx.x + j * kQuantThreads;
+    if (vi < nvec) reinterpret_cast<uint4*>(xs)[vi] = v[j];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
+    const int col = sO[i];
+    atomicOr(&mask[col >> 5], 1u << (col & 31));
+    if (FUSED) {
+      float cm = 0.f;
+      for (int r = 0; r < mom.M; ++r) {
+        const float xv_r = fabsf(h2f(r == m ? xs[col] : X[static_cast<size_t>(r) * K + col]));
+        cm = xv_r > cm ? xv_r : cm;
+      }
+      sS[i] = momentum_step(sS[i], mom.gamma, cm, mom.wmaxO[i]);
+    }
+  }
+  __syncthreads();
+
   float lmax = 0.f;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int vi = threadIdx.x + j * kQuantThreads;
     if (vi < nvec) {
-      v[j] = __ldg(xv + vi);
       const unsigned mb = (mask[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
       const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
@@ -194,8 +208,7 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     }
   }
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
-    const float xh = __fdiv_rn(h2f(xrow[sO[i]]), sS[i]);
-    const float f = fabsf(xh);
+    const float f = fabsf(__fdiv_rn(h2f(xs[sO[i]]), sS[i]));
     lmax = f > lmax ? f : lmax;
   }
   const float amax = block_max_256(lmax, red);
@@ -226,7 +239,7 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
   const size_t lo_off = static_cast<size_t>(gridDim.x) * nOp;  // U holds [2][M][nOp]: hi rows, then lo rows
   for (int i = threadIdx.x; i < nOp; i += kQuantThreads) {
     if (i < nO) {
-      const float xh = __fdiv_rn(h2f(xrow[sO[i]]), sS[i]);
+      const float xh = __fdiv_rn(h2f(xs[sO[i]]), sS[i]);
       const int q = quant_code(xh, inv);
       XqO[static_cast<size_t>(m) * nO + i] = static_cast<int8_t>(q);
       if (U) {

@@ -19,22 +19,23 @@
 // exactly one CTA computes it.  When tiles are plentiful the split points
 // snap to whole tiles and no scratch is used.
 //
-// Pipeline: two shared-memory rings.  The staging ring (INT4 formats) holds
-// packed weight tiles straight from TMA and is released as soon as the
-// converters have read a slot, so many of them can be in flight; the operand
-// ring holds what the tensor core reads (the INT8 weight operand written by
-// the converters, or by TMA for the INT8 format, and the activation or
-// compensation tiles) and is released by tcgen05.commit.
+// Pipeline: three shared-memory rings, each with its own producer, so no
+// load waits behind another: the staging ring (INT4 formats) takes packed
+// weight blocks straight from bulk copies and is released as soon as the
+// converters have read a slot; the A ring holds the tensor core's weight
+// operand (written by the converters, or copied for the INT8 format and for
+// W_O^T) and the X ring its activation (or compensation) operand; both are
+// released by tcgen05.commit.
 //
 // Warp roles:
-//   warp 0        operand producer: activation tiles (after the grid
-//                 dependency on the previous kernel), INT8 weight tiles,
-//                 compensation operands (W_O^T tile, U hi/lo tiles).
+//   warp 0        X producer: activation tiles (TMA, after the grid
+//                 dependency on the previous kernel) and the compensation
+//                 operands U hi/lo.
 //   warp 1        allocates TMEM (two accumulator buffers when they fit); one
 //                 lane issues tcgen05.mma and commits.
-//   warp 2        staging producer (INT4 formats): packed weights and the
-//                 g128 ratio row; starts at once (weights do not depend on
-//                 the previous kernel).
+//   warp 2        weight producer: packed INT4 blocks into the staging ring,
+//                 INT8 blocks and W_O^T blocks into the A ring; starts at once
+//                 (weights do not depend on the previous kernel).
 //   warps 3..     converters (INT4 formats): unpack the staged INT4 codes into
 //                 the 128-byte-swizzled K-major INT8 operand (QQQ review,
 //                 per-channel GEMM: INT4 -> INT8 by a left shift of 4;
@@ -57,17 +58,39 @@ constexpr int kMaxGrid = 256;  // persistent CTAs per GEMM (>= SMs per GPU)
 // Diagnostic builds (-DQLIN_TRACE) record per-CTA clock64 stamps at the
 // phase boundaries below into g_trace[cta][16]; normal builds compile the
 // stamps away.
+// QLIN_STEP(g, k) records per-step events of CTA 0 into g_steps[g][8].  The
+// buffer pointers are read once into registers (QLIN_TRACE_INIT) so a stamp
+// costs a clock read and a store, not a global load.
 #ifdef QLIN_TRACE
 __device__ long long* g_trace = nullptr;
-#define QLIN_STAMP(k)                                                            \
-  do {                                                                           \
-    if (g_trace) g_trace[blockIdx.x * 16 + (k)] = static_cast<long long>(clock64()); \
+__device__ long long* g_steps = nullptr;
+#define QLIN_TRACE_INIT                           \
+  long long* const qlin_tr = g_trace;             \
+  long long* const qlin_st = blockIdx.x == 0 ? g_steps : nullptr;
+#define QLIN_STAMP(k)                                                                \
+  do {                                                                               \
+    if (qlin_tr) qlin_tr[blockIdx.x * 32 + (k)] = static_cast<long long>(clock64()); \
+  } while (0)
+#define QLIN_STEP(g, k)                                                                       \
+  do {                                                                                        \
+    if (qlin_st && (g) < 64) qlin_st[(g) * 8 + (k)] = static_cast<long long>(clock64());      \
+  } while (0)
+// finisher phases of any CTA into g_steps[63][k] (last writer wins)
+#define QLIN_FIN(k)                                                                           \
+  do {                                                                                        \
+    if (g_steps) g_steps[63 * 8 + (k)] = static_cast<long long>(clock64());                   \
   } while (0)
 #else
+#define QLIN_FIN(k) do { } while (0)
+#define QLIN_TRACE_INIT
 #define QLIN_STAMP(k) do { } while (0)
+#define QLIN_STEP(g, k) do { } while (0)
 #endif
 
 struct GemmArgs {
+  const uint8_t* codes;     // tiled packed codes (INT4: 8 KiB blocks, INT8: 16 KiB swizzled blocks)
+  const uint16_t* rfold;    // g128 ratios r [K/128][N] fp16
+  const uint16_t* wot;      // tiled W_O^T (16 KiB swizzled blocks of 128 channels x 64 outliers)
   const float* cscale;  // c_n [N]
   const float* a;       // a_m [M]
   uint16_t* Y;          // [M][N] fp16
@@ -77,7 +100,8 @@ struct GemmArgs {
   unsigned* ws_cnt;     // [grid] iteration counters (zero on entry, left zero)
   int M, N, K, nO;
   int tiles_n, tiles_m;
-  int nk;               // main K-steps per tile
+  int kb;               // 128-wide K-blocks per tile (ceil(K / 128))
+  int nk;               // main K-steps per tile (ceil(kb / KS))
   int nc;               // compensation steps per tile
   int ncs;              // 64-wide outlier slices
   int T;                // iterations per tile = nk + nc
@@ -89,41 +113,52 @@ struct GemmArgs {
   unsigned bnd[kMaxGrid + 1];
 };
 
+// K-blocks of 128 INT8 codes per pipeline step for a token tile of BT.
+__host__ __device__ constexpr int gemm_ks(int BT) { return BT <= 16 ? 4 : (BT <= 64 ? 2 : 1); }
+
 template <int FMT, int BT>
 struct GemmCfg {
   static constexpr int kBN = 128;                    // output channels per tile (MMA M)
-  static constexpr int kBK = 128;                    // INT8 elements of K per stage (one swizzle row)
+  // K-blocks of 128 INT8 codes per pipeline step.  Each step costs a few
+  // hundred cycles of bookkeeping in the MMA and converter threads whatever
+  // its size, so small token tiles (HBM-bound decode) move four blocks per
+  // step; large ones are tensor-bound and move one.
+  static constexpr int KS = gemm_ks(BT);
   static constexpr bool kW4 = FMT != kFmtW8;
-  static constexpr int kNCW = FMT == kFmtW4G128 ? 8 : 4;  // converter warps (>= 4: epilogue)
+  // converter warps (>= 4: the first four are the epilogue); two per SM
+  // sub-partition for the INT4 formats so unpacking is not latency-bound
+  static constexpr int kNCW = kW4 ? 8 : 4;
   static constexpr int kThreads = 96 + 32 * kNCW;
-  // Small token tiles load the hi and lo compensation operands in one stage
-  // (one W_O^T tile feeds both); large ones use two passes.
+  // Small token tiles load the hi and lo compensation operands in one step
+  // (one W_O^T block feeds both); large ones use two passes.
   static constexpr bool kCompFused = BT <= 64;
-  // operand slot: A (128 x 128 B), B (BT x 128 B), B2 (U lo, fused compensation)
-  static constexpr int kOffA = 0;
-  static constexpr int kOffB = 16384;
-  static constexpr int kOffB2 = kOffB + BT * 128;
-  static constexpr int kOpBytes = (kOffB2 + (kCompFused ? BT * 128 : 0) + 1023) / 1024 * 1024;
-  // staging slot: packed INT4 (128 x 64 B) + g128 ratios (128 fp16)
-  static constexpr int kStgBytes = kW4 ? 8192 + (FMT == kFmtW4G128 ? 256 : 0) : 0;
-  static constexpr int kSmemLimit = 232448;   // 227 KB per CTA
-  static constexpr int kReserve = 1024 + 768; // alignment slack + barriers
+  static constexpr int kABytes = KS * 16384;                             // KS x (128 x 128 B)
+  static constexpr int kXTile = BT * 128;                                // BT x 128 B per K-block
+  static constexpr int kXTiles = KS > (kCompFused ? 2 : 1) ? KS : (kCompFused ? 2 : 1);
+  static constexpr int kXBytes = (kXTile * kXTiles + 1023) / 1024 * 1024;
+  static constexpr int kStgRatio = KS * 8192;                            // g128 ratio rows follow the codes
+  static constexpr int kStgBytes = kW4 ? KS * 8192 + (FMT == kFmtW4G128 ? KS * 256 : 0) : 0;
+  static constexpr int kSmemLimit = 232448;          // 227 KB per CTA
+  static constexpr int kReserve = 1024 + 1024 + 1024;  // alignment slack, barriers, token scales
   static constexpr int kBudget = kSmemLimit - kReserve;
-  static constexpr int kOpSlotsFit = kBudget / kOpBytes;
-  static constexpr int kOpSlots = kW4 ? (BT <= 128 ? 4 : 3) : (kOpSlotsFit > 8 ? 8 : kOpSlotsFit);
-  static constexpr int kStgSlotsFit = kW4 ? (kBudget - kOpSlots * kOpBytes) / kStgBytes : 0;
+  static constexpr int kXSlots = KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 ? 4 : 3));
+  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes) / kABytes;
+  static constexpr int kASlots = kW4 ? (KS == 4 ? 2 : (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)))
+                                     : (kASlotsW8 > 8 ? 8 : kASlotsW8);
+  static constexpr int kStgSlotsFit = kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes) / kStgBytes : 0;
   static constexpr int kStgSlots = kStgSlotsFit > 16 ? 16 : kStgSlotsFit;
-  static constexpr int kOffStg = kOpSlots * kOpBytes;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffX = kASlots * kABytes;
+  static constexpr int kOffStg = kOffX + kXSlots * kXBytes;
   static constexpr int kOffBar = kOffStg + kStgSlots * kStgBytes;
+  static constexpr int kOffScale = kOffBar + 1024;   // BT token scales for the finisher
   static constexpr int kSmemBytes = kReserve + kOffBar;
-  // TMA transaction bytes
-  static constexpr uint32_t kTxStg = kW4 ? kStgBytes : 0;
-  static constexpr uint32_t kTxMainOp = (kW4 ? 0 : 16384) + BT * 128;
-  static constexpr uint32_t kTxComp = 16384 + (kCompFused ? 2 : 1) * BT * 128;
-  static_assert(kOpSlots >= 2, "operand ring too small");
-  static_assert(!kW4 || kStgSlots >= 2, "staging ring too small");
+  static constexpr uint32_t kTxX = BT * 128;
+  static constexpr uint32_t kTxU = (kCompFused ? 2 : 1) * BT * 128;
+  static_assert(kASlots >= 2 && kASlots <= 8, "A ring");
+  static_assert(kXSlots >= 2 && kXSlots <= 8, "X ring");
+  static_assert(!kW4 || (kStgSlots >= 2 && kStgSlots <= 16), "staging ring");
   static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N must be 16..256 in steps of 16");
-  static_assert(kOpSlots <= 8 && kStgSlots <= 16, "barrier area");
 };
 
 // TMEM columns per accumulator buffer and the number of buffers.
@@ -227,32 +262,37 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int slots, int issued
   for (int t = issued - 1; t >= 0 && t >= issued - slots; --t) {
     const int s = t % slots;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(&full[s], static_cast<uint32_t>(t / slots) & 1u) && globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+    while (!mbar_try_wait_sleep(&full[s], static_cast<uint32_t>(t / slots) & 1u, 1000000u) &&
+           globaltimer_ns() - t0 < QLIN_WAIT_NS) {
     }
   }
 }
 
 template <int FMT, int BT>
 __global__ void __launch_bounds__(GemmCfg<FMT, BT>::kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-            const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmWO,
-            const __grid_constant__ CUtensorMap tmU, const __grid_constant__ GemmArgs args) {
+gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmU,
+            const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<FMT, BT>;
-  constexpr int P = C::kOpSlots;
-  constexpr int LS = C::kStgSlots;
+  constexpr int P = C::kASlots;
+  constexpr int XS = C::kXSlots;
+  constexpr int LS = C::kStgSlots > 0 ? C::kStgSlots : 1;
   constexpr int kConvThreads = 32 * C::kNCW;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* ofull = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* oconv = ofull + 8;
-  uint64_t* oempty = oconv + 8;
-  uint64_t* sfull = oempty + 8;
+  uint64_t* sfull = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* sempty = sfull + 16;
-  uint64_t* acc_full = sempty + 16;   // [2]
+  uint64_t* afull = sempty + 16;
+  uint64_t* aconv = afull + 8;
+  uint64_t* aempty = aconv + 8;
+  uint64_t* xfull = aempty + 8;
+  uint64_t* xempty = xfull + 8;
+  uint64_t* acc_full = xempty + 8;    // [2]
   uint64_t* acc_empty = acc_full + 2; // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* fin_bar = acc_empty + 2;  // finisher's bulk loads of partials
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;  // [2]
+  float* sa = reinterpret_cast<float*>(smem + C::kOffScale);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -262,39 +302,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
   const uint32_t tcols = tmem_alloc_cols(BT, comp);
   const unsigned it0 = args.bnd[blockIdx.x];
   const unsigned it1 = args.bnd[blockIdx.x + 1];
+  QLIN_TRACE_INIT
 #ifdef QLIN_TRACE
-  if (threadIdx.x == 0 && g_trace) g_trace[blockIdx.x * 16 + 15] = static_cast<long long>(globaltimer_ns());
+  if (threadIdx.x == 0 && qlin_tr) qlin_tr[blockIdx.x * 32 + 31] = static_cast<long long>(globaltimer_ns());
 #endif
   if (threadIdx.x == 0) QLIN_STAMP(0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < P; ++s) {
-      mbar_init(&ofull[s], 1);
-      mbar_init(&oconv[s], kConvThreads);
-      mbar_init(&oempty[s], 1);
+    for (int i = 0; i < 16; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], kConvThreads);
     }
-    for (int s = 0; s < LS; ++s) {
-      mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], kConvThreads);
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(&afull[i], 1);
+      mbar_init(&aconv[i], kConvThreads);
+      mbar_init(&aempty[i], 1);
+      mbar_init(&xfull[i], 1);
+      mbar_init(&xempty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    mbar_init(fin_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmX);
-    if (!C::kW4) tma_prefetch_desc(&tmW);
-    if (comp) {
-      tma_prefetch_desc(&tmWO);
-      tma_prefetch_desc(&tmU);
-    }
-  }
-  if (warp == 2 && lane == 0 && C::kW4) {
-    tma_prefetch_desc(&tmW);
-    if (FMT == kFmtW4G128) tma_prefetch_desc(&tmR);
+    if (comp) tma_prefetch_desc(&tmU);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, tcols);
@@ -310,100 +346,116 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
   griddep_launch_dependents();
 
   if (warp == 0) {
-    // ------------------------------------------------------------ operand producer
+    // ------------------------------------------------------------ X producer
     if (lane == 0) {
-      const uint64_t pol_stream = policy_evict_first();
-      // part 0: expect the slot's bytes and load the weight side (INT8
-      // weights or W_O^T); part 1: the activation side; 2: both.
-      auto issue = [&](const Segment& sg, int r, int p, int part) {
-        unsigned char* op = smem + p * C::kOpBytes;
-        const int tn = static_cast<int>(sg.tile % args.tiles_n);
-        const int tm = static_cast<int>(sg.tile / args.tiles_n);
-        const int n0 = tn * C::kBN, m0 = tm * BT;
-        if (r < args.nk) {
-          const int k0 = r * C::kBK;
-          if (part != 1) {
-            mbar_arrive_expect_tx(&ofull[p], C::kTxMainOp);
-            if (!C::kW4) tma_load_2d_hint(op + C::kOffA, &tmW, &ofull[p], k0, n0, pol_stream);
-          }
-          if (part != 0) tma_load_2d(op + C::kOffB, &tmX, &ofull[p], k0, m0);
-        } else {
-          const int j = r - args.nk;
-          int i0, y;
-          if (C::kCompFused) {
-            i0 = j * 64;
-            y = m0;
-          } else {
-            const int lo = j >= args.ncs ? 1 : 0;  // U rows [0, M) hold hi, [M, 2M) hold lo
-            i0 = (j - lo * args.ncs) * 64;
-            y = lo * args.M + m0;
-          }
-          if (part != 1) {
-            mbar_arrive_expect_tx(&ofull[p], C::kTxComp);
-            tma_load_2d(op + C::kOffA, &tmWO, &ofull[p], i0, n0);
-          }
-          if (part != 0) {
-            tma_load_2d(op + C::kOffB, &tmU, &ofull[p], i0, y);
-            if (C::kCompFused) tma_load_2d(op + C::kOffB2, &tmU, &ofull[p], i0, args.M + m0);
-          }
-        }
-      };
-      // pass 1: weight side of the first P iterations (independent of the
-      // previous kernel), then wait for the grid dependency.
-      int pre = 0;
-      {
-        unsigned ita = it0;
-        Segment sa;
-        while (pre < P && next_segment(ita, it1, args, sa))
-          for (int r = sa.r0; r < sa.r1 && pre < P; ++r, ++pre) issue(sa, r, pre, 0);
-      }
-      griddep_wait();
+      griddep_wait();  // activations come from the previous kernel
       QLIN_STAMP(4);
       unsigned it = it0;
       Segment sg;
       int g = 0;
       bool ok = true;
       while (ok && next_segment(it, it1, args, sg)) {
+        const int m0 = static_cast<int>(sg.tile / args.tiles_n) * BT;
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
-          const int p = g % P;
-          if (g < P) {
-            issue(sg, r, p, 1);
+          const int x = g % XS;
+          if (g >= XS && !mbar_wait(&xempty[x], static_cast<uint32_t>(g / XS - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          unsigned char* xb = smem + C::kOffX + x * C::kXBytes;
+          QLIN_STEP(g, 0);
+          if (r < args.nk) {
+            const int kb0 = r * C::KS;
+            const int nkb = min(C::KS, args.kb - kb0);
+            mbar_arrive_expect_tx(&xfull[x], static_cast<uint32_t>(nkb) * C::kTxX);
+            for (int i = 0; i < nkb; ++i) tma_load_2d(xb + i * C::kXTile, &tmX, &xfull[x], (kb0 + i) * 128, m0);
           } else {
-            if (!mbar_wait(&oempty[p], static_cast<uint32_t>(g / P - 1) & 1u, abort_flag)) { ok = false; break; }
-            issue(sg, r, p, 2);
+            const int j = r - args.nk;
+            mbar_arrive_expect_tx(&xfull[x], C::kTxU);
+            if (C::kCompFused) {
+              tma_load_2d(xb, &tmU, &xfull[x], j * 64, m0);                          // hi rows
+              tma_load_2d(xb + C::kXTile, &tmU, &xfull[x], j * 64, args.M + m0);     // lo rows
+            } else {
+              const int lo = j >= args.ncs ? 1 : 0;  // U rows [0, M) hold hi, [M, 2M) hold lo
+              tma_load_2d(xb, &tmU, &xfull[x], (j - lo * args.ncs) * 64, lo * args.M + m0);
+            }
           }
         }
       }
       QLIN_STAMP(5);
-      drain_ring(ofull, P, g > pre ? g : pre);
+      drain_ring(xfull, XS, g);
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ------------------------------------------------------------ staging producer
-    if (lane == 0 && C::kW4) {
+    // ------------------------------------------------------------ weight producer
+    if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();
+      uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // loads issued into each A slot
       unsigned it = it0;
       Segment sg;
-      int gs = 0;
+      int g = 0, gs = 0;
       bool ok = true;
       while (ok && next_segment(it, it1, args, sg)) {
-        const int n0 = static_cast<int>(sg.tile % args.tiles_n) * C::kBN;
-        const int rend = sg.r1 < args.nk ? sg.r1 : args.nk;
-        for (int r = sg.r0; r < rend; ++r, ++gs) {
-          const int ls = gs % LS;
-          if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
-            ok = false;
-            break;
+        const int tn = static_cast<int>(sg.tile % args.tiles_n);
+        const int n0 = tn * C::kBN;
+        const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(min(C::kBN, args.N - n0)) * 2u : 0u;
+        for (int r = sg.r0; r < sg.r1; ++r, ++g) {
+          if (r < args.nk && C::kW4) {
+            const int ls = gs % LS;
+            if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
+            QLIN_STEP(g, 1);
+            const int kb0 = r * C::KS;
+            const int nkb = min(C::KS, args.kb - kb0);
+            mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nkb) * (8192u + rb));
+            bulk_load_hint(st, args.codes + (static_cast<size_t>(tn) * args.kb + kb0) * 8192,
+                           static_cast<uint32_t>(nkb) * 8192u, &sfull[ls], pol_stream);
+            if (FMT == kFmtW4G128)
+              for (int i = 0; i < nkb; ++i)
+                bulk_load(st + C::kStgRatio + i * 256, args.rfold + static_cast<size_t>(kb0 + i) * args.N + n0, rb,
+                          &sfull[ls]);
+            if (gs == 0) QLIN_STAMP(2);
+            ++gs;
+          } else if (!C::kW4) {
+            // INT8 weights and W_O^T blocks into the A ring.  This thread
+            // waits on every A slot in order, so a parity wait never runs
+            // more than one phase ahead of the ring.  (For the INT4 formats
+            // the converters, which move in step with the A ring, issue the
+            // W_O^T copies instead.)
+            const int p = g % P;
+            if (g >= P && !mbar_wait(&aempty[p], static_cast<uint32_t>(g / P - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            unsigned char* ab = smem + C::kOffA + p * C::kABytes;
+            if (r < args.nk) {
+              const int kb0 = r * C::KS;
+              const int nkb = min(C::KS, args.kb - kb0);
+              mbar_arrive_expect_tx(&afull[p], static_cast<uint32_t>(nkb) * 16384u);
+              bulk_load_hint(ab, args.codes + (static_cast<size_t>(tn) * args.kb + kb0) * 16384,
+                             static_cast<uint32_t>(nkb) * 16384u, &afull[p], pol_stream);
+            } else {
+              const int j = r - args.nk;
+              const int ib = C::kCompFused ? j : (j >= args.ncs ? j - args.ncs : j);
+              mbar_arrive_expect_tx(&afull[p], 16384u);
+              bulk_load(ab, args.wot + (static_cast<size_t>(tn) * args.ncs + ib) * 8192, 16384, &afull[p]);
+            }
+            ++a_issues[p];
           }
-          unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
-          mbar_arrive_expect_tx(&sfull[ls], C::kTxStg);
-          tma_load_2d_hint(st, &tmW, &sfull[ls], r * (C::kBK / 2), n0, pol_stream);
-          if (FMT == kFmtW4G128) tma_load_2d(st + 8192, &tmR, &sfull[ls], n0, r);
-          if (gs == 0) QLIN_STAMP(2);
         }
       }
       QLIN_STAMP(3);
-      drain_ring(sfull, LS, gs);
+      if (C::kW4) drain_ring(sfull, LS, gs);
+      for (int p = 0; p < P; ++p) {  // outstanding A-ring copies
+        if (!a_issues[p]) continue;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(&afull[p], (a_issues[p] - 1) & 1u, 1000000u) &&
+               globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+        }
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -411,7 +463,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
     if (lane == 0) {
       constexpr uint32_t idesc_main = idesc_s8_s32(128, BT);
       constexpr uint32_t idesc_comp = idesc_f16_f32(128, BT);
-      uint32_t conv_phase = 0;  // one parity bit per operand slot
+      // Descriptors of ring slot 0; the start-address field counts 16-byte
+      // units, so slot i adds i * slot_bytes / 16 and a 32-byte K-slice adds
+      // 2 (shared addresses stay below 2^18, so the field never carries).
+      const uint64_t adesc0 = sdesc_k_sw128(smem_u32(smem + C::kOffA));
+      const uint64_t xdesc0 = sdesc_k_sw128(smem_u32(smem + C::kOffX));
+      uint32_t conv_phase = 0;  // per A slot: parity of the next converter phase
+      uint32_t full_phase = 0;  // per A slot: parity of the next copy phase
       unsigned it = it0;
       Segment sg;
       int g = 0, seg = 0;
@@ -425,35 +483,54 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
         const uint32_t dcomp = dmain + BT;
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
           const int p = g % P;
+          const int x = g % XS;
           const bool main_step = r < args.nk;
-          if (!mbar_wait(&ofull[p], static_cast<uint32_t>(g / P) & 1u, abort_flag)) { ok = false; break; }
-          if (g == 0) QLIN_STAMP(8);
+          if (!mbar_wait(&xfull[x], static_cast<uint32_t>(g / XS) & 1u, abort_flag)) { ok = false; break; }
+          QLIN_STEP(g, 5);
           if (main_step && C::kW4) {
-            if (!mbar_wait(&oconv[p], (conv_phase >> p) & 1u, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&aconv[p], (conv_phase >> p) & 1u, abort_flag)) { ok = false; break; }
             conv_phase ^= 1u << p;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + p * C::kOpBytes + C::kOffA);
-          const uint32_t b_addr = smem_u32(smem + p * C::kOpBytes + C::kOffB);
-          if (main_step) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_i8(dmain, sdesc_k_sw128(a_addr + 32 * kk), sdesc_k_sw128(b_addr + 32 * kk), idesc_main,
-                     (r > sg.r0 || kk > 0) ? 1u : 0u);
           } else {
-            const bool first = (r == args.nk) || (r == sg.r0);
+            if (!mbar_wait(&afull[p], (full_phase >> p) & 1u, abort_flag)) { ok = false; break; }
+            full_phase ^= 1u << p;
+          }
+          if (g == 0) QLIN_STAMP(8);
+          QLIN_STEP(g, 6);
+          tc_fence_after();
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(p * (C::kABytes >> 4));
+          const uint64_t bd = xdesc0 + static_cast<uint64_t>(x * (C::kXBytes >> 4));
+          if (main_step) {
+            const int nkb = min(C::KS, args.kb - r * C::KS);
+            mma_i8(dmain, ad, bd, idesc_main, r > sg.r0 ? 1u : 0u);
+            mma_i8(dmain, ad + 2, bd + 2, idesc_main, 1u);
+            mma_i8(dmain, ad + 4, bd + 4, idesc_main, 1u);
+            mma_i8(dmain, ad + 6, bd + 6, idesc_main, 1u);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(dcomp, sdesc_k_sw128(a_addr + 32 * kk), sdesc_k_sw128(b_addr + 32 * kk), idesc_comp,
-                      (!first || kk > 0) ? 1u : 0u);
+            for (int i = 1; i < C::KS; ++i) {
+              if (i < nkb) {
+                const uint64_t ai = ad + static_cast<uint64_t>(i * 1024);
+                const uint64_t bi = bd + static_cast<uint64_t>(i * (C::kXTile >> 4));
+                mma_i8(dmain, ai, bi, idesc_main, 1u);
+                mma_i8(dmain, ai + 2, bi + 2, idesc_main, 1u);
+                mma_i8(dmain, ai + 4, bi + 4, idesc_main, 1u);
+                mma_i8(dmain, ai + 6, bi + 6, idesc_main, 1u);
+              }
+            }
+          } else {
+            const uint32_t acc0 = ((r == args.nk) || (r == sg.r0)) ? 0u : 1u;
+            mma_f16(dcomp, ad, bd, idesc_comp, acc0);
+            mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
+            mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
+            mma_f16(dcomp, ad + 6, bd + 6, idesc_comp, 1u);
             if (C::kCompFused) {
-              const uint32_t b2_addr = smem_u32(smem + p * C::kOpBytes + C::kOffB2);
+              const uint64_t bd2 = bd + (C::kXTile >> 4);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_f16(dcomp, sdesc_k_sw128(a_addr + 32 * kk), sdesc_k_sw128(b2_addr + 32 * kk), idesc_comp, 1u);
+              for (int kk = 0; kk < 4; ++kk) mma_f16(dcomp, ad + 2 * kk, bd2 + 2 * kk, idesc_comp, 1u);
             }
           }
-          mma_commit(&oempty[p]);
+          mma_commit(&aempty[p]);
+          mma_commit(&xempty[x]);
+          QLIN_STEP(g, 7);
         }
         if (!ok) break;
         mma_commit(&acc_full[buf]);
@@ -466,31 +543,54 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
     const int ctid = threadIdx.x - 96;
     // ------------------------------------------------------------ converters
     if (C::kW4) {
+      uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // W_O^T copies issued into each A slot (ctid 0)
       unsigned it = it0;
       Segment sg;
       int g = 0, gs = 0;
       bool ok = true;
       while (ok && next_segment(it, it1, args, sg)) {
+        const int tn = static_cast<int>(sg.tile % args.tiles_n);
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
-          if (r >= args.nk) continue;
           const int p = g % P;
+          if (r >= args.nk) {
+            // compensation step: the W_O^T block goes into the A slot once
+            // the tensor core has released it
+            if (g >= P && !mbar_wait(&aempty[p], static_cast<uint32_t>(g / P - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (ctid == 0) {
+              const int j = r - args.nk;
+              const int ib = C::kCompFused ? j : (j >= args.ncs ? j - args.ncs : j);
+              mbar_arrive_expect_tx(&afull[p], 16384u);
+              bulk_load(smem + C::kOffA + p * C::kABytes, args.wot + (static_cast<size_t>(tn) * args.ncs + ib) * 8192,
+                        16384, &afull[p]);
+              ++a_issues[p];
+            }
+            continue;
+          }
           const int ls = gs % LS;
           if (!mbar_wait(&sfull[ls], static_cast<uint32_t>(gs / LS) & 1u, abort_flag)) { ok = false; break; }
           if (gs == 0 && ctid == 0) QLIN_STAMP(6);
-          if (g >= P && !mbar_wait(&oempty[p], static_cast<uint32_t>(g / P - 1) & 1u, abort_flag)) { ok = false; break; }
+          if (ctid == 0) QLIN_STEP(g, 2);
+          if (g >= P && !mbar_wait(&aempty[p], static_cast<uint32_t>(g / P - 1) & 1u, abort_flag)) { ok = false; break; }
+          if (ctid == 0) QLIN_STEP(g, 3);
           const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
-          unsigned char* A = smem + p * C::kOpBytes + C::kOffA;
+          unsigned char* A0 = smem + C::kOffA + p * C::kABytes;
+          const int nchunk = min(C::KS, args.kb - r * C::KS) * 512;  // 16-byte packed chunks this step
 #pragma unroll 2
-          for (int c = ctid; c < 512; c += kConvThreads) {
-            const int row = c >> 2;
+          for (int c = ctid; c < nchunk; c += kConvThreads) {
+            const int blk = c >> 9;       // K-block within the step
+            const int row = (c >> 2) & 127;
             const int part = c & 3;
+            unsigned char* A = A0 + blk * 16384;
             const uint4 w = *reinterpret_cast<const uint4*>(stg + c * 16);
             uint4 o0, o1;
             if (FMT == kFmtW4PC) {
               unpack_w4pc(w, o0, o1);
             } else {
-              const uint16_t rb = reinterpret_cast<const uint16_t*>(stg + 8192)[row];
-              const __half2 r1 = __half2half2(__ushort_as_half(rb));
+              const uint16_t rbits = reinterpret_cast<const uint16_t*>(stg + C::kStgRatio + blk * 256)[row];
+              const __half2 r1 = __half2half2(__ushort_as_half(rbits));
               const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
               const uint2 a0 = requant_g128(w.x, r1, r16);
               const uint2 a1 = requant_g128(w.y, r1, r16);
@@ -505,11 +605,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
           }
           mbar_arrive(&sempty[ls]);  // staging slot consumed
           fence_proxy_async_smem();
-          mbar_arrive(&oconv[p]);
+          mbar_arrive(&aconv[p]);
+          if (ctid == 0) QLIN_STEP(g, 4);
           ++gs;
         }
       }
-      if (ctid == 0) QLIN_STAMP(7);
+      if (ctid == 0) {
+        QLIN_STAMP(7);
+        for (int p = 0; p < P; ++p) {  // outstanding W_O^T copies
+          if (!a_issues[p]) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait_sleep(&afull[p], (a_issues[p] - 1) & 1u, 1000000u) &&
+                 globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+          }
+        }
+      }
     }
     // ------------------------------------------------------------ epilogue
     if (warp < 7) {
@@ -601,53 +711,109 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUt
         }
         named_bar_sync(1, 128);
         if (nl == 0) QLIN_STAMP(12);
+        uint32_t fin_phase = 0;
         for (int q = 0; q < npend; ++q) {
           if (!last_flag[q]) continue;
-          __threadfence();
           const unsigned tile = pend_tile[q];
           const unsigned first_it = tile * static_cast<unsigned>(args.T);
           const int c_lo = owner_cta(first_it, args);
           const int c_hi = owner_cta(first_it + args.T - 1, args);
+          int nctr = 0;
+          for (int c = c_lo; c <= c_hi; ++c) nctr += args.bnd[c] != args.bnd[c + 1] ? 1 : 0;
           const int tn = static_cast<int>(tile % args.tiles_n);
           const int tm = static_cast<int>(tile / args.tiles_n);
           const int n = tn * C::kBN + nl;
           const int m0 = tm * BT;
           const int mvalid = min(BT, args.M - m0);
           const float cn = n < args.N ? (FMT == kFmtW4PC ? __fmul_rn(args.cscale[n], 0.0625f) : args.cscale[n]) : 0.f;
-          const float* ccmp = args.ws_comp + static_cast<size_t>(partial_slot(c_hi, tile, args)) * BT * 128;
-          // rows in groups of 8, contributors in groups of 4: 32 independent loads in flight
-          for (int j0 = 0; j0 < mvalid; j0 += 8) {
-            int32_t av[8];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) av[r] = 0;
-            for (int cb = c_lo; cb <= c_hi; cb += 4) {
-              int32_t v[4][8];
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                const int c = cb + cc;
-                const bool live = c <= c_hi && args.bnd[c] != args.bnd[c + 1];
-                const int32_t* src = args.ws_acc + static_cast<size_t>(live ? partial_slot(c, tile, args) : 0) * BT * 128;
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-                  v[cc][r] = (live && j0 + r < mvalid) ? __ldcg(src + static_cast<size_t>(j0 + r) * 128 + nl) : 0;
+          for (int j = nl; j < mvalid; j += 128) sa[j] = args.a[m0 + j];
+          // The rings are idle now: bulk-copy every contributor's rows of
+          // partial sums (and the compensation block) into shared memory,
+          // all copies in flight at once, then reduce from there.
+          const int blocks = nctr + (comp ? 1 : 0);
+          // all three rings are free by now: partial blocks, then an fp16
+          // staging tile (256 bytes per row) for coalesced stores of Y
+          int rows = (C::kOffBar / (blocks * 512 + 256));
+          rows = rows > 16 ? rows & ~15 : rows;
+          rows = rows < mvalid ? rows : mvalid;
+          int32_t* fin = reinterpret_cast<int32_t*>(smem);
+          for (int j0 = 0; j0 < mvalid; j0 += rows) {
+            const int rr = min(rows, mvalid - j0);
+            uint16_t* ystage = reinterpret_cast<uint16_t*>(fin + static_cast<size_t>(blocks) * rr * 128);
+            const uint32_t blk_bytes = static_cast<uint32_t>(rr) * 512u;
+            if (nl == 0) {
+              QLIN_STAMP(16 + 4 * q);
+              QLIN_FIN(0);
+              __threadfence();
+              fence_proxy_async_global();
+              QLIN_FIN(1);
+              mbar_arrive_expect_tx(fin_bar, blk_bytes * blocks);
+              int qq = 0;
+              for (int c = c_lo; c <= c_hi; ++c) {
+                if (args.bnd[c] == args.bnd[c + 1]) continue;
+                bulk_load(fin + static_cast<size_t>(qq) * rr * 128,
+                          args.ws_acc + (static_cast<size_t>(partial_slot(c, tile, args)) * BT + j0) * 128, blk_bytes,
+                          fin_bar);
+                ++qq;
               }
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-                for (int r = 0; r < 8; ++r) av[r] += v[cc][r];
+              if (comp)
+                bulk_load(fin + static_cast<size_t>(nctr) * rr * 128,
+                          args.ws_comp + (static_cast<size_t>(partial_slot(c_hi, tile, args)) * BT + j0) * 128,
+                          blk_bytes, fin_bar);
             }
+            if (nl == 0) QLIN_FIN(2);
+            mbar_wait(fin_bar, fin_phase, abort_flag);
+            fin_phase ^= 1u;
+            if (nl == 0) QLIN_FIN(3);
+            if (nl == 0) QLIN_STAMP(17 + 4 * q);
+            named_bar_sync(1, 128);  // token scales staged
+            // Thread t reduces channels 4*(t % 32) .. +3 of rows t/32, t/32 + 4,
+            // ... with 16-byte shared-memory loads (four partial sums per load).
+            {
+              const int cg = nl & 31;
+              const int n4 = tn * C::kBN + 4 * cg;
+              float c4[4];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-              const int j = j0 + r;
-              if (j < mvalid && n < args.N) {
-                const int m = m0 + j;
-                float vv = __fmul_rn(cn, static_cast<float>(av[r]));
-                if (comp) vv = __fadd_rn(vv, __ldcg(ccmp + static_cast<size_t>(j) * 128 + nl));
-                const float y = __fmul_rn(args.a[m], vv);
-                args.Y[static_cast<size_t>(m) * args.N + n] = __half_as_ushort(__float2half_rn(y));
-                if (args.acc_debug) args.acc_debug[static_cast<size_t>(m) * args.N + n] = av[r];
+              for (int i = 0; i < 4; ++i) {
+                const int nn = n4 + i;
+                c4[i] = nn < args.N ? (FMT == kFmtW4PC ? __fmul_rn(args.cscale[nn], 0.0625f) : args.cscale[nn]) : 0.f;
+              }
+              for (int j = nl >> 5; j < rr; j += 4) {
+                int4 sum = make_int4(0, 0, 0, 0);
+                for (int qq = 0; qq < nctr; ++qq) {
+                  const int4 v = *reinterpret_cast<const int4*>(fin + (static_cast<size_t>(qq) * rr + j) * 128 + 4 * cg);
+                  sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+                }
+                float4 cp = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (comp) cp = *reinterpret_cast<const float4*>(fin + (static_cast<size_t>(nctr) * rr + j) * 128 + 4 * cg);
+                const float am = sa[j0 + j];
+                const float y0 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[0], static_cast<float>(sum.x)), cp.x) : __fmul_rn(c4[0], static_cast<float>(sum.x)));
+                const float y1 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[1], static_cast<float>(sum.y)), cp.y) : __fmul_rn(c4[1], static_cast<float>(sum.y)));
+                const float y2 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[2], static_cast<float>(sum.z)), cp.z) : __fmul_rn(c4[2], static_cast<float>(sum.z)));
+                const float y3 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[3], static_cast<float>(sum.w)), cp.w) : __fmul_rn(c4[3], static_cast<float>(sum.w)));
+                uint2 hv;
+                hv.x = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y0))) |
+                       (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y1))) << 16);
+                hv.y = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y2))) |
+                       (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y3))) << 16);
+                *reinterpret_cast<uint2*>(ystage + j * 128 + 4 * cg) = hv;
+                if (args.acc_debug && n4 < args.N)
+                  *reinterpret_cast<int4*>(args.acc_debug + static_cast<size_t>(m0 + j0 + j) * args.N + n4) = sum;
               }
             }
+            named_bar_sync(1, 128);  // staged tile complete
+            // 16-byte coalesced stores: 16 per 128-channel row
+            for (int idx = nl; idx < rr * 16; idx += 128) {
+              const int j = idx >> 4;
+              const int n8 = tn * C::kBN + (idx & 15) * 8;
+              if (n8 < args.N)
+                *reinterpret_cast<uint4*>(args.Y + static_cast<size_t>(m0 + j0 + j) * args.N + n8) =
+                    *reinterpret_cast<const uint4*>(ystage + j * 128 + (idx & 15) * 8);
+            }
+            if (nl == 0) QLIN_FIN(4);
+            if (nl == 0) QLIN_STAMP(18 + 4 * q);
+            named_bar_sync(1, 128);  // the buffer is reused by the next chunk
+            if (nl == 0) QLIN_FIN(5);
           }
           if (nl == 0) args.ws_cnt[c_lo] = 0u;
           if (nl == 0) QLIN_STAMP(13);

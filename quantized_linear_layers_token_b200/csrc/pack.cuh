@@ -9,6 +9,14 @@
 // One thread owns one output channel n and walks its K inputs twice (scale
 // pass, code pass); reads of W[k][*] are coalesced across the threads of a
 // warp.  Packing runs once per layer and is not on the timed path.
+//
+// Packed codes are tile-major so that the GEMM fetches each 128-channel x
+// 128-input block with one contiguous bulk copy: block (tn, kb) holds
+// channels 128*tn .. +127 (rows) and inputs 128*kb .. +127.  INT4 blocks are
+// 128 rows x 64 bytes (8 KiB); INT8 blocks are 128 rows x 128 bytes (16 KiB)
+// stored with the tensor core's 128-byte swizzle already applied (16-byte
+// chunk c of row r sits at chunk c ^ (r % 8)).  Padding rows and inputs are
+// zero.
 #pragma once
 
 #include "sm100.cuh"
@@ -46,6 +54,18 @@ __device__ __forceinline__ uint2 pack8_bytes(const int (&q)[8]) {
   return o;
 }
 
+// Byte offset of the 8 codes k0..k0+7 of channel n in the tiled layouts.
+__device__ __forceinline__ size_t w4_tile_offset(int n, int k0, int KB) {
+  const size_t blk = static_cast<size_t>(n >> 7) * KB + (k0 >> 7);
+  return (blk * 128 + (n & 127)) * 64 + ((k0 & 127) >> 1);
+}
+__device__ __forceinline__ size_t w8_tile_offset(int n, int k0, int KB) {
+  const size_t blk = static_cast<size_t>(n >> 7) * KB + (k0 >> 7);
+  const int r = n & 127;
+  const int chunk = (k0 & 127) >> 4;
+  return (blk * 128 + r) * 128 + ((chunk ^ (r & 7)) << 4) + (k0 & 15);
+}
+
 // Symmetric per-output-channel quantization:
 //   c_n = wmax_n / qmax,  q = clamp(rne(w * (qmax / wmax_n)), -qmax, qmax)   (fp32)
 template <int QMAX, bool W4>
@@ -65,10 +85,11 @@ __global__ void pack_per_channel_kernel(const uint16_t* __restrict__ W, int K, i
     int q[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) q[j] = rne_clamp(__fmul_rn(h2f(W[static_cast<size_t>(k0 + j) * N + n]), inv), QMAX);
+    const int KB = (K + 127) >> 7;
     if (W4) {
-      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (K / 2) + k0 / 2) = pack8_nibbles(q);
+      *reinterpret_cast<uint32_t*>(codes + w4_tile_offset(n, k0, KB)) = pack8_nibbles(q);
     } else {
-      *reinterpret_cast<uint2*>(codes + static_cast<size_t>(n) * K + k0) = pack8_bytes(q);
+      *reinterpret_cast<uint2*>(codes + w8_tile_offset(n, k0, KB)) = pack8_bytes(q);
     }
   }
 }
@@ -107,24 +128,35 @@ __global__ void pack_group_kernel(const uint16_t* __restrict__ W, int K, int N,
         const float w = h2f(W[static_cast<size_t>(k0 + t) * N + n]);
         q[t] = ghf > 0.f ? rne_clamp(__fdiv_rn(w, ghf), 7) : 0;
       }
-      *reinterpret_cast<uint32_t*>(codes + static_cast<size_t>(n) * (K / 2) + k0 / 2) = pack8_nibbles(q);
+      *reinterpret_cast<uint32_t*>(codes + w4_tile_offset(n, k0, K >> 7)) = pack8_nibbles(q);
     }
   }
 }
 
-// Outlier rows: W_Ot[n][i] = W[O_i][n] (transposed so the compensation
-// operand is K-major for the tensor core), wmax_O[i] = max_n |W[O_i][n]|.
-// One CTA per outlier channel; the padding columns are cleared beforehand.
+// Outlier rows: W_Ot holds W[O_i][n] transposed (channel n, outlier i) so
+// the compensation operand is K-major for the tensor core, tiled like the
+// INT8 codes: block (tn, ib) is channels 128*tn .. +127 by outliers
+// 64*ib .. +63 in fp16, 128 bytes per row, 128-byte swizzle applied.
+// wmax_O[i] = max_n |W[O_i][n]|.  One CTA per outlier channel; the padding
+// is cleared beforehand.
+__device__ __forceinline__ size_t wot_tile_index(int n, int i, int IB) {
+  const size_t blk = static_cast<size_t>(n >> 7) * IB + (i >> 6);
+  const int r = n & 127;
+  const int byte = (i & 63) * 2;
+  return ((blk * 128 + r) * 128 + (((byte >> 4) ^ (r & 7)) << 4) + (byte & 15)) >> 1;
+}
+
 __global__ void pack_outliers_kernel(const uint16_t* __restrict__ W, int N, const int32_t* __restrict__ O,
-                                     int nOp, uint16_t* __restrict__ W_Ot, float* __restrict__ wmaxO) {
+                                     int nO, uint16_t* __restrict__ W_Ot, float* __restrict__ wmaxO) {
   const int i = blockIdx.x;
+  const int IB = (nO + 63) >> 6;
   const uint16_t* row = W + static_cast<size_t>(O[i]) * N;
   float m = 0.f;
   for (int n = threadIdx.x; n < N; n += blockDim.x) {
     const uint16_t v = row[n];
     const float f = fabsf(h2f(v));
     m = f > m ? f : m;
-    W_Ot[static_cast<size_t>(n) * nOp + i] = v;
+    W_Ot[wot_tile_index(n, i, IB)] = v;
   }
   __shared__ float red[32];
 #pragma unroll

@@ -52,7 +52,7 @@ qlin_status check_shape(int32_t K, int32_t N, int32_t fmt, int32_t nO) {
   if (fmt != QLIN_W4_PERCHANNEL && fmt != QLIN_W4_G128 && fmt != QLIN_W8_PERCHANNEL)
     return fail(QLIN_ERR_ARG, "unknown weight format %d", fmt);
   if (K <= 0 || N <= 0 || nO < 0) return fail(QLIN_ERR_ARG, "negative or zero size K=%d N=%d n_outlier=%d", K, N, nO);
-  if (K % 32 != 0 || K >= 131072) return fail(QLIN_ERR_SHAPE, "K=%d must be a multiple of 32 below 131072", K);
+  if (K % 32 != 0 || K > 65536) return fail(QLIN_ERR_SHAPE, "K=%d must be a multiple of 32, at most 65536", K);
   if (N % 16 != 0) return fail(QLIN_ERR_SHAPE, "N=%d must be a multiple of 16", N);
   if (fmt == QLIN_W4_G128 && K % 128 != 0) return fail(QLIN_ERR_SHAPE, "g128 needs K %% 128 == 0 (K=%d)", K);
   if (nO > K || nO > 4096) return fail(QLIN_ERR_SHAPE, "n_outlier=%d must be <= min(K, 4096)", nO);
@@ -66,14 +66,15 @@ struct Layout {
 Layout weights_layout(int32_t K, int32_t N, int32_t fmt, int32_t nO) {
   Layout L{};
   size_t off = 0;
-  const size_t codes_b = (fmt == QLIN_W8_PERCHANNEL) ? size_t(K) * N : size_t(K) * N / 2;
+  const size_t tiles_n = (N + 127) / 128, kb = (K + 127) / 128, ib = (nO + 63) / 64;
+  const size_t codes_b = tiles_n * kb * ((fmt == QLIN_W8_PERCHANNEL) ? 16384 : 8192);
   L.codes = off; off = round_up(off + codes_b, kAlign);
   L.chan = off; off = round_up(off + size_t(N) * 4, kAlign);
   const size_t gb = (fmt == QLIN_W4_G128) ? size_t(K / 128) * N * 2 : 0;
   L.group = off; off = round_up(off + gb, kAlign);
   L.fold = off; off = round_up(off + gb, kAlign);
   L.oidx = off; off = round_up(off + size_t(nO) * 4, kAlign);
-  L.wot = off; off = round_up(off + size_t(N) * pad8(nO) * 2, kAlign);
+  L.wot = off; off = round_up(off + tiles_n * ib * 16384, kAlign);
   L.wmax = off; off = round_up(off + size_t(nO) * 4, kAlign);
   L.total = off;
   return L;
@@ -179,7 +180,7 @@ int pick_bt(int M) {
 // Work decomposition of one GEMM call (same on the host for workspace sizes
 // and for the launch).
 struct GemmPlan {
-  int bt, tiles_n, tiles_m, nk, nc, ncs, T, grid, split;
+  int bt, tiles_n, tiles_m, kb, nk, nc, ncs, T, grid, split;
   size_t u_off, acc_off, comp_off, cnt_off, total;
 };
 
@@ -188,7 +189,9 @@ GemmPlan plan_gemm(int M, const qlin_weights* w) {
   p.bt = pick_bt(M);
   p.tiles_n = (w->N + 127) / 128;
   p.tiles_m = (M + p.bt - 1) / p.bt;
-  p.nk = (w->K + 127) / 128;
+  p.kb = (w->K + 127) / 128;
+  const int ks = gemm_ks(p.bt);
+  p.nk = (p.kb + ks - 1) / ks;
   p.ncs = w->n_outlier > 0 ? (w->n_outlier + 63) / 64 : 0;
   p.nc = (p.bt <= 64) ? p.ncs : 2 * p.ncs;
   p.T = p.nk + p.nc;
@@ -226,33 +229,17 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
   });
   if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
 
-  CUtensorMap tmW, tmX, tmR, tmWO, tmU;
-  memset(&tmR, 0, sizeof(tmR));
-  memset(&tmWO, 0, sizeof(tmWO));
+  CUtensorMap tmX, tmU;
   memset(&tmU, 0, sizeof(tmU));
-  qlin_status st;
-  const int K = w->K, N = w->N, M = args.M;
-  if (FMT == kFmtW8)
-    st = make_map(&tmW, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  else
-    st = make_map(&tmW, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  const int K = w->K, M = args.M;
+  qlin_status st = make_map(&tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, BT, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != QLIN_OK) return st;
-  st = make_map(&tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, BT, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != QLIN_OK) return st;
-  if (FMT == kFmtW4G128) {
-    st = make_map(&tmR, w->fold_ratio, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, K / 128, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != QLIN_OK) return st;
-  }
   if (w->n_outlier > 0) {
-    const int nOp = w->n_outlier_pad;
-    st = make_map(&tmWO, w->W_Ot, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, nOp, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != QLIN_OK) return st;
-    st = make_map(&tmU, U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, nOp, 2 * static_cast<uint64_t>(M), 64, BT,
+    st = make_map(&tmU, U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->n_outlier_pad, 2 * static_cast<uint64_t>(M), 64, BT,
                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != QLIN_OK) return st;
   }
-  cudaError_t e = launch_k(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, tmW, tmX, tmR, tmWO,
-                           tmU, args);
+  cudaError_t e = launch_k(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, tmX, tmU, args);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
 }
@@ -276,6 +263,9 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
   if (st != QLIN_OK) return st;
   const GemmPlan p = plan_gemm(M, w);
   GemmArgs args;
+  args.codes = static_cast<const uint8_t*>(w->codes);
+  args.rfold = w->fold_ratio;
+  args.wot = w->W_Ot;
   args.cscale = w->chan_scale;
   args.a = a;
   args.Y = Y;
@@ -289,6 +279,7 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
   args.nO = w->n_outlier;
   args.tiles_n = p.tiles_n;
   args.tiles_m = p.tiles_m;
+  args.kb = p.kb;
   args.nk = p.nk;
   args.nc = p.nc;
   args.ncs = p.ncs;
@@ -328,13 +319,20 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   }
   const int nvec = K / 8;
   const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
-  const size_t smem = size_t(nO) * 8 + size_t(K / 32) * 4;
+  const size_t smem = size_t(K) * 2 + size_t(nO) * 8 + size_t(K / 32) * 4;
   const int nOp = w->n_outlier_pad;
   cudaError_t e = cudaSuccess;
-#define QLIN_QUANT_CASE(V)                                                                               \
-  e = fused ? launch_k(quant_kernel<V, true>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,         \
-                       static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom)     \
-            : launch_k(quant_kernel<V, false>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,        \
+#define QLIN_QUANT_CASE(V)                                                                                   \
+  {                                                                                                          \
+    static std::once_flag once_##V;                                                                          \
+    std::call_once(once_##V, [] {                                                                            \
+      cudaFuncSetAttribute(quant_kernel<V, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);  \
+      cudaFuncSetAttribute(quant_kernel<V, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024); \
+    });                                                                                                      \
+  }                                                                                                          \
+  e = fused ? launch_k(quant_kernel<V, true>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,             \
+                       static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom)         \
+            : launch_k(quant_kernel<V, false>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,            \
                        static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom);
   if (vpt <= 1) { QLIN_QUANT_CASE(1) }
   else if (vpt <= 2) { QLIN_QUANT_CASE(2) }
@@ -342,7 +340,6 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   else if (vpt <= 8) { QLIN_QUANT_CASE(8) }
   else if (vpt <= 16) { QLIN_QUANT_CASE(16) }
   else if (vpt <= 32) { QLIN_QUANT_CASE(32) }
-  else if (vpt <= 64) { QLIN_QUANT_CASE(64) }
   else return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", K);
 #undef QLIN_QUANT_CASE
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "quant_kernel launch failed: %s", cudaGetErrorString(e));
@@ -477,6 +474,8 @@ qlin_status qlin_pack_weights(const uint16_t* W, const int32_t* O_host, const ql
   const int threads = 128;
   const int blocks = (N + threads - 1) / threads;
   uint8_t* codes = static_cast<uint8_t*>(w->codes);
+  const Layout L = weights_layout(K, N, w->fmt, nO);
+  QLIN_CUDA_TRY(cudaMemsetAsync(codes, 0, L.chan - L.codes, stream));  // tile padding is zero
   switch (w->fmt) {
     case QLIN_W4_PERCHANNEL:
       pack_per_channel_kernel<7, true><<<blocks, threads, 0, stream>>>(W, K, N, codes, w->chan_scale);
@@ -491,8 +490,8 @@ qlin_status qlin_pack_weights(const uint16_t* W, const int32_t* O_host, const ql
   QLIN_LAUNCH_CHECK("pack kernel");
   if (nO > 0) {
     QLIN_CUDA_TRY(cudaMemcpyAsync(w->outlier_idx, O_host, size_t(nO) * 4, cudaMemcpyHostToDevice, stream));
-    QLIN_CUDA_TRY(cudaMemsetAsync(w->W_Ot, 0, size_t(N) * w->n_outlier_pad * 2, stream));
-    pack_outliers_kernel<<<nO, 256, 0, stream>>>(W, N, w->outlier_idx, w->n_outlier_pad, w->W_Ot, w->wmax_O);
+    QLIN_CUDA_TRY(cudaMemsetAsync(w->W_Ot, 0, L.wmax - L.wot, stream));
+    pack_outliers_kernel<<<nO, 256, 0, stream>>>(W, N, w->outlier_idx, nO, w->W_Ot, w->wmax_O);
     QLIN_LAUNCH_CHECK("pack_outliers_kernel");
   }
   return QLIN_OK;
@@ -657,9 +656,12 @@ qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weights* w, fl
 
 #ifdef QLIN_TRACE
 // Diagnostic builds only: point the GEMM's phase stamps at a device buffer
-// of [grid][16] int64 (NULL turns them off).
+// of [grid][32] int64 (NULL turns them off).
 QLIN_API int qlin_trace_set(long long* p) {
   return static_cast<int>(cudaMemcpyToSymbol(qlin::g_trace, &p, sizeof(p)));
+}
+QLIN_API int qlin_steps_set(long long* p) {
+  return static_cast<int>(cudaMemcpyToSymbol(qlin::g_steps, &p, sizeof(p)));
 }
 #endif
 

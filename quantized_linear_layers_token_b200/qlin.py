@@ -228,14 +228,16 @@ class PackedLayer:
         """Typed view of one packed sub-buffer (for parity checks)."""
         w = self.w
         base = self.buffer.data_ptr()
-        K, N, nO, nOp = w.K, w.N, w.n_outlier, w.n_outlier_pad
+        K, N, nO = w.K, w.N, w.n_outlier
+        TN, KB, IB = -(-N // 128), -(-K // 128), -(-nO // 64)
+        block = 16384 if self.fmt == QLIN_W8_PERCHANNEL else 8192
         spec = {
-            "codes": (w.codes, torch.uint8, (N, K // 2) if self.fmt != QLIN_W8_PERCHANNEL else (N, K)),
+            "codes": (w.codes, torch.uint8, (TN * KB * block,)),       # tile-major (include/qlin.h)
             "chan_scale": (w.chan_scale, torch.float32, (N,)),
             "group_scale": (w.group_scale, torch.int16, (K // 128, N)),
             "fold_ratio": (w.fold_ratio, torch.int16, (K // 128, N)),
             "outlier_idx": (w.outlier_idx, torch.int32, (nO,)),
-            "W_Ot": (w.W_Ot, torch.int16, (N, nOp)),
+            "W_Ot": (w.W_Ot, torch.int16, (TN * IB * 8192,)),           # tiled, swizzled fp16
             "wmax_O": (w.wmax_O, torch.float32, (nO,)),
         }[name]
         ptr, dtype, shape = spec

@@ -42,7 +42,9 @@ def test_bench_workload_sampled(q, oracle, wl_name, shape_idx, ms):
     O = L0["O"]
     layer = q.PackedLayer.pack(torch.from_numpy(W).cuda(), O, wl.fmt)
     pk = oracle.pack_layer(bits(W), O, wl.fmt)
-    np.testing.assert_array_equal(layer.view("codes").cpu().numpy(), pk["packed"])
+    from layouts import tile_w4
+    K, N = W.shape
+    np.testing.assert_array_equal(layer.view("codes").cpu().numpy(), tile_w4(pk["packed"], N, K))
     np.testing.assert_array_equal(layer.view("chan_scale").cpu().numpy().view(np.uint32), pk["c"].view(np.uint32))
     for M in ms:
         L = synth.layer(wl, shape_idx, M=M, with_weights=False)
@@ -107,7 +109,8 @@ def test_split_k_accumulators_exact(q, oracle, fmt, M):
     up = lambda v: -(-v // 256) * 256
     bt = 16 if M <= 16 else (32 if M <= 32 else 64)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    T = -(-K // 128) + -(-nO // 64)
+    ks = 4 if bt <= 16 else 2  # K-blocks per pipeline step for this token tile
+    T = -(-(-(-K // 128)) // ks) + -(-nO // 64)
     grid = min(sms, -(-N // 128) * -(-M // bt) * T)
     u_bytes = up(2 * M * ((nO + 7) // 8 * 8) * 2)
     slots = up(2 * grid * bt * 128 * 4)

@@ -74,11 +74,13 @@ def run_gpu(q, L, s0, gamma, update=True, with_forward=True):
 
 
 def check_pack(oracle, L, g):
+    from layouts import tile_w4, tile_w8, tile_wot
     fmt = L["fmt"]
+    K, N = L["W"].shape
     pk = oracle.pack_layer(bits(L["W"]), L["O"], fmt)
     layer = g["layer"]
-    np.testing.assert_array_equal(layer.view("codes").cpu().numpy(), pk["packed"].view(np.uint8)
-                                  if fmt != synth.W8_PERCHANNEL else pk["packed"].view(np.uint8))
+    want = tile_w8(pk["packed"], N, K) if fmt == synth.W8_PERCHANNEL else tile_w4(pk["packed"], N, K)
+    np.testing.assert_array_equal(layer.view("codes").cpu().numpy(), want)
     np.testing.assert_array_equal(layer.view("chan_scale").cpu().numpy().view(np.uint32), pk["c"].view(np.uint32))
     if fmt == synth.W4_G128:
         np.testing.assert_array_equal(layer.view("group_scale").cpu().numpy().view(np.uint16), pk["g_h"])
@@ -86,8 +88,7 @@ def check_pack(oracle, L, g):
     nO = len(L["O"])
     if nO:
         wot = layer.view("W_Ot").cpu().numpy().view(np.uint16)
-        np.testing.assert_array_equal(wot[:, :nO], bits(L["W"])[L["O"], :].T)
-        assert not wot[:, nO:].any()
+        np.testing.assert_array_equal(wot, tile_wot(bits(L["W"])[L["O"], :].T, N, nO))
         np.testing.assert_array_equal(layer.view("wmax_O").cpu().numpy().view(np.uint32),
                                       pk["wmaxO"].view(np.uint32))
         np.testing.assert_array_equal(layer.view("outlier_idx").cpu().numpy(), L["O"])
