@@ -30,7 +30,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -69,50 +68,69 @@ def read_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
-    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+    """SM clocks and clock-event reasons sampled through NVML by a host
+    thread every few milliseconds while the timed region runs (reading only;
+    no setting of the GPU is changed).  The device is found by its UUID so
+    CUDA_VISIBLE_DEVICES remapping does not matter."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.device_index = device_index
+        self.period = period_s
+        self.samples = []
+        self.error = None
+        self._stop = None
+        self._thread = None
+
+    def _run(self, ready):
+        import pynvml as nv
+        try:
+            import torch
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+            h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            while True:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((mhz, [n for n, m in masks if bits & m]))
+                ready.set()
+                if self._stop.wait(self.period):
+                    break
+        except Exception as e:  # sampling is evidence, never a reason to fail the run
+            self.error = f"{type(e).__name__}: {e}"
+        finally:
+            ready.set()
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+        import threading
+        self._stop = threading.Event()
+        ready = threading.Event()
+        self._thread = threading.Thread(target=self._run, args=(ready,), daemon=True)
+        self._thread.start()
+        ready.wait(10.0)
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        self._thread.join(5.0)
         return False
 
     def summary(self):
-        rows = []
-        for line in (self.out or "").strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable: " + str(self.error)],
+                    "samples": 0}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
 
 
 # ---------------------------------------------------------------------------
@@ -236,7 +254,7 @@ def run_profile_case(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_w4_decode")
@@ -460,8 +478,9 @@ def main():
         cpu = {"value": sample.bytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": sample.describe(t)}
 
-    launches_per_forward = {sl["si"]: (3 if len(meta[sl["si"]]["O"]) else 2) for sl in slots}
-    gpu_launches = args.steps * sum(launches_per_forward[sl["si"]] for sl in slots)
+    # per forward: quantization (+ the column-max kernel when the momentum
+    # update is not fused, M > 64) and the GEMM
+    gpu_launches = args.steps * sum(2 + (1 if len(meta[sl["si"]]["O"]) and sl["M"] > 64 else 0) for sl in slots)
 
     if rank == 0:
         line = {
@@ -480,7 +499,7 @@ def main():
                        "timing": "CUDA graph of one step, CUDA events on the launch stream"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                       "reasons": clocks["reasons"]},
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

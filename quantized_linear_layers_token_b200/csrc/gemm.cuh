@@ -139,7 +139,7 @@ struct GemmCfg {
   static constexpr int kStgRatio = KS * 8192;                            // g128 ratio rows follow the codes
   static constexpr int kStgBytes = kW4 ? KS * 8192 + (FMT == kFmtW4G128 ? KS * 256 : 0) : 0;
   static constexpr int kSmemLimit = 232448;          // 227 KB per CTA
-  static constexpr int kReserve = 1024 + 1024 + 1024;  // alignment slack, barriers, token scales
+  static constexpr int kReserve = 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table
   static constexpr int kBudget = kSmemLimit - kReserve;
   static constexpr int kXSlots = KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 ? 4 : 3));
   static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes) / kABytes;
@@ -151,7 +151,7 @@ struct GemmCfg {
   static constexpr int kOffX = kASlots * kABytes;
   static constexpr int kOffStg = kOffX + kXSlots * kXBytes;
   static constexpr int kOffBar = kOffStg + kStgSlots * kStgBytes;
-  static constexpr int kOffScale = kOffBar + 1024;   // BT token scales for the finisher
+  static constexpr int kOffBnd = kOffBar + 1024;     // stream-K boundary table (<= 256 entries)
   static constexpr int kSmemBytes = kReserve + kOffBar;
   static constexpr uint32_t kTxX = BT * 128;
   static constexpr uint32_t kTxU = (kCompFused ? 2 : 1) * BT * 128;
@@ -184,20 +184,26 @@ inline unsigned gemm_boundary(int c, long long tiles, int T, int nk, int grid, i
   return static_cast<unsigned>(b);
 }
 
+// The boundary table is copied into shared memory at kernel start (entries
+// 0 .. grid-1; entry grid is the total iteration count).
+__device__ __forceinline__ unsigned bnd_s(int c, const unsigned* sbnd, const GemmArgs& g) {
+  return c < g.grid ? sbnd[c] : static_cast<unsigned>(g.tiles_n * g.tiles_m * g.T);
+}
+
 // The CTA whose range contains iteration `it` (binary search of the table).
-__device__ __forceinline__ int owner_cta(unsigned it, const GemmArgs& g) {
+__device__ __forceinline__ int owner_cta_s(unsigned it, const unsigned* sbnd, const GemmArgs& g) {
   int lo = 0, hi = g.grid - 1;  // invariant: bnd[lo] <= it < bnd[hi + 1]
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (g.bnd[mid] <= it) lo = mid; else hi = mid - 1;
+    if (sbnd[mid] <= it) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
 // Scratch slot holding CTA c's partial of split tile `tile`: its first
 // segment if its range starts inside the tile, else its last segment.
-__device__ __forceinline__ int partial_slot(int c, unsigned tile, const GemmArgs& g) {
-  return 2 * c + (g.bnd[c] < tile * static_cast<unsigned>(g.T) ? 1 : 0);
+__device__ __forceinline__ int partial_slot_s(int c, unsigned tile, const unsigned* sbnd, const GemmArgs& g) {
+  return 2 * c + (sbnd[c] < tile * static_cast<unsigned>(g.T) ? 1 : 0);
 }
 
 struct Segment {
@@ -288,11 +294,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   uint64_t* xempty = xfull + 8;
   uint64_t* acc_full = xempty + 8;    // [2]
   uint64_t* acc_empty = acc_full + 2; // [2]
-  uint64_t* fin_bar = acc_empty + 2;  // finisher's bulk loads of partials
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin_bar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;  // [2]
-  float* sa = reinterpret_cast<float*>(smem + C::kOffScale);
+  unsigned* sbnd = reinterpret_cast<unsigned*>(smem + C::kOffBnd);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -324,7 +329,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
-    mbar_init(fin_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -541,6 +545,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     __syncwarp();
   } else {
     const int ctid = threadIdx.x - 96;
+    // The epilogue threads keep the boundary table in shared memory (read
+    // after the epilogue's first named barrier).
+    if (warp < 7)
+      for (int i = ctid; i < args.grid; i += 128) sbnd[i] = args.bnd[i];
     // ------------------------------------------------------------ converters
     if (C::kW4) {
       uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // W_O^T copies issued into each A slot (ctid 0)
@@ -652,7 +660,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         const bool whole = sg.r0 == 0 && sg.r1 == args.T;
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * bcols);
         const float cn = n < args.N ? (FMT == kFmtW4PC ? __fmul_rn(args.cscale[n], 0.0625f) : args.cscale[n]) : 0.f;
-        const int my_slot = whole ? 0 : partial_slot(static_cast<int>(blockIdx.x), sg.tile, args);
+        const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tile * static_cast<unsigned>(args.T) ? 1 : 0);
         int32_t* pacc = args.ws_acc + static_cast<size_t>(my_slot) * BT * 128;
         float* pcmp = args.ws_comp + static_cast<size_t>(my_slot) * BT * 128;
 #pragma unroll 1
@@ -700,124 +708,136 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       }
       if (nl == 0) QLIN_STAMP(11);
       if (npend > 0) {
-        __threadfence();
+        // Count this CTA's contributions (CTA barrier, then one thread's
+        // acq_rel fence and atomic: the release covers every epilogue
+        // thread's partial stores).  The CTA whose addition completes a
+        // tile's T iterations finishes it.
         named_bar_sync(1, 128);
         if (nl == 0) {
+          fence_acq_rel_gpu();
+          bool any = false;
           for (int q = 0; q < npend; ++q) {
-            const int c_lo = owner_cta(pend_tile[q] * static_cast<unsigned>(args.T), args);
-            const unsigned old = atomicAdd(&args.ws_cnt[c_lo], static_cast<unsigned>(pend_add[q]));
-            last_flag[q] = (old + static_cast<unsigned>(pend_add[q]) == static_cast<unsigned>(args.T)) ? 1 : 0;
+            const int c_lo = owner_cta_s(pend_tile[q] * static_cast<unsigned>(args.T), sbnd, args);
+            const unsigned old = atom_add_relaxed_gpu(&args.ws_cnt[c_lo], static_cast<unsigned>(pend_add[q]));
+            const bool last = old + static_cast<unsigned>(pend_add[q]) == static_cast<unsigned>(args.T);
+            last_flag[q] = last ? 1 : 0;
+            any = any || last;
           }
+          if (any) fence_acq_rel_gpu();  // acquire the other contributors' partials
         }
         named_bar_sync(1, 128);
         if (nl == 0) QLIN_STAMP(12);
-        uint32_t fin_phase = 0;
         for (int q = 0; q < npend; ++q) {
           if (!last_flag[q]) continue;
           const unsigned tile = pend_tile[q];
           const unsigned first_it = tile * static_cast<unsigned>(args.T);
-          const int c_lo = owner_cta(first_it, args);
-          const int c_hi = owner_cta(first_it + args.T - 1, args);
-          int nctr = 0;
-          for (int c = c_lo; c <= c_hi; ++c) nctr += args.bnd[c] != args.bnd[c + 1] ? 1 : 0;
+          const int c_lo = owner_cta_s(first_it, sbnd, args);
+          const int c_hi = owner_cta_s(first_it + args.T - 1, sbnd, args);
           const int tn = static_cast<int>(tile % args.tiles_n);
           const int tm = static_cast<int>(tile / args.tiles_n);
-          const int n = tn * C::kBN + nl;
           const int m0 = tm * BT;
           const int mvalid = min(BT, args.M - m0);
-          const float cn = n < args.N ? (FMT == kFmtW4PC ? __fmul_rn(args.cscale[n], 0.0625f) : args.cscale[n]) : 0.f;
-          for (int j = nl; j < mvalid; j += 128) sa[j] = args.a[m0 + j];
-          // The rings are idle now: bulk-copy every contributor's rows of
-          // partial sums (and the compensation block) into shared memory,
-          // all copies in flight at once, then reduce from there.
+          if (nl == 0) QLIN_STAMP(16 + 4 * q);
+          // Thread t owns channels 4*(t % 32) .. +3, so a warp covers one
+          // 128-channel row of the tile; warp w takes rows w, w + 4, ...
+          // Every partial of those rows (and the token scales) is gathered
+          // into the idle rings with cp.async, all copies in flight at once;
+          // each thread then reduces exactly the elements it copied, and the
+          // finished row goes out as one 256-byte store per warp.
+          const int cg = nl & 31;
+          const int wq = nl >> 5;
+          const int n4 = tn * C::kBN + 4 * cg;
+          const bool live = n4 < args.N;
+          float c4[4] = {0.f, 0.f, 0.f, 0.f};
+          if (live) {
+            const float4 cs = *reinterpret_cast<const float4*>(args.cscale + n4);
+            c4[0] = cs.x; c4[1] = cs.y; c4[2] = cs.z; c4[3] = cs.w;
+            if (FMT == kFmtW4PC) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) c4[i] = __fmul_rn(c4[i], 0.0625f);
+            }
+          }
+          int nctr = 0;
+          for (int c = c_lo; c <= c_hi; ++c) nctr += bnd_s(c, sbnd, args) != bnd_s(c + 1, sbnd, args) ? 1 : 0;
           const int blocks = nctr + (comp ? 1 : 0);
-          // all three rings are free by now: partial blocks, then an fp16
-          // staging tile (256 bytes per row) for coalesced stores of Y
-          int rows = (C::kOffBar / (blocks * 512 + 256));
-          rows = rows > 16 ? rows & ~15 : rows;
-          rows = rows < mvalid ? rows : mvalid;
+          int rows = C::kOffBar / (blocks * 512 + 4);
+          rows = rows > 4 ? rows & ~3 : rows;
           int32_t* fin = reinterpret_cast<int32_t*>(smem);
+          // kernel parameters used per row, held in registers (the stores
+          // below would otherwise force reloads of the parameter block)
+          uint16_t* const Yp = args.Y;
+          int32_t* const accd = args.acc_debug;
+          const size_t ldy = static_cast<size_t>(args.N);
           for (int j0 = 0; j0 < mvalid; j0 += rows) {
             const int rr = min(rows, mvalid - j0);
-            uint16_t* ystage = reinterpret_cast<uint16_t*>(fin + static_cast<size_t>(blocks) * rr * 128);
-            const uint32_t blk_bytes = static_cast<uint32_t>(rr) * 512u;
-            if (nl == 0) {
-              QLIN_STAMP(16 + 4 * q);
-              QLIN_FIN(0);
-              __threadfence();
-              fence_proxy_async_global();
-              QLIN_FIN(1);
-              mbar_arrive_expect_tx(fin_bar, blk_bytes * blocks);
-              int qq = 0;
-              for (int c = c_lo; c <= c_hi; ++c) {
-                if (args.bnd[c] == args.bnd[c + 1]) continue;
-                bulk_load(fin + static_cast<size_t>(qq) * rr * 128,
-                          args.ws_acc + (static_cast<size_t>(partial_slot(c, tile, args)) * BT + j0) * 128, blk_bytes,
-                          fin_bar);
-                ++qq;
-              }
-              if (comp)
-                bulk_load(fin + static_cast<size_t>(nctr) * rr * 128,
-                          args.ws_comp + (static_cast<size_t>(partial_slot(c_hi, tile, args)) * BT + j0) * 128,
-                          blk_bytes, fin_bar);
+            float* fa = reinterpret_cast<float*>(fin + static_cast<size_t>(blocks) * rr * 128);
+            int qq = 0;
+            for (int c = c_lo; c <= c_hi; ++c) {
+              if (bnd_s(c, sbnd, args) == bnd_s(c + 1, sbnd, args)) continue;
+              const int32_t* src = args.ws_acc + (static_cast<size_t>(partial_slot_s(c, tile, sbnd, args)) * BT + j0) * 128 + 4 * cg;
+              for (int j = wq; j < rr; j += 4) cp_async16(fin + (static_cast<size_t>(qq) * rr + j) * 128 + 4 * cg, src + j * 128);
+              ++qq;
             }
-            if (nl == 0) QLIN_FIN(2);
-            mbar_wait(fin_bar, fin_phase, abort_flag);
-            fin_phase ^= 1u;
-            if (nl == 0) QLIN_FIN(3);
-            if (nl == 0) QLIN_STAMP(17 + 4 * q);
-            named_bar_sync(1, 128);  // token scales staged
-            // Thread t reduces channels 4*(t % 32) .. +3 of rows t/32, t/32 + 4,
-            // ... with 16-byte shared-memory loads (four partial sums per load).
-            {
-              const int cg = nl & 31;
-              const int n4 = tn * C::kBN + 4 * cg;
-              float c4[4];
+            if (comp) {
+              const float* src = args.ws_comp + (static_cast<size_t>(partial_slot_s(c_hi, tile, sbnd, args)) * BT + j0) * 128 + 4 * cg;
+              for (int j = wq; j < rr; j += 4) cp_async16(fin + (static_cast<size_t>(nctr) * rr + j) * 128 + 4 * cg, src + j * 128);
+            }
+            if (cg == 0)
+              for (int j = wq; j < rr; j += 4) cp_async4(fa + j, args.a + m0 + j0 + j);
+            cp_async_wait_all();
+            __syncwarp();  // lane 0's token scales
+            if (nl == 0 && j0 == 0) QLIN_STAMP(17 + 4 * q);
+            // four rows per thread at a time, contributors unrolled, so the
+            // shared-memory loads are independent of one another
+            for (int jb = wq; jb < rr; jb += 16) {
+              int4 sum[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) sum[i] = make_int4(0, 0, 0, 0);
+#pragma unroll 2
+              for (int k = 0; k < nctr; ++k) {
+                const int32_t* blk = fin + static_cast<size_t>(k) * rr * 128 + 4 * cg;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  if (jb + 4 * i < rr) {
+                    const int4 v = *reinterpret_cast<const int4*>(blk + (jb + 4 * i) * 128);
+                    sum[i].x += v.x; sum[i].y += v.y; sum[i].z += v.z; sum[i].w += v.w;
+                  }
+                }
+              }
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const int nn = n4 + i;
-                c4[i] = nn < args.N ? (FMT == kFmtW4PC ? __fmul_rn(args.cscale[nn], 0.0625f) : args.cscale[nn]) : 0.f;
-              }
-              for (int j = nl >> 5; j < rr; j += 4) {
-                int4 sum = make_int4(0, 0, 0, 0);
-                for (int qq = 0; qq < nctr; ++qq) {
-                  const int4 v = *reinterpret_cast<const int4*>(fin + (static_cast<size_t>(qq) * rr + j) * 128 + 4 * cg);
-                  sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-                }
+                const int j = jb + 4 * i;
+                if (j >= rr) break;
                 float4 cp = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (comp) cp = *reinterpret_cast<const float4*>(fin + (static_cast<size_t>(nctr) * rr + j) * 128 + 4 * cg);
-                const float am = sa[j0 + j];
-                const float y0 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[0], static_cast<float>(sum.x)), cp.x) : __fmul_rn(c4[0], static_cast<float>(sum.x)));
-                const float y1 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[1], static_cast<float>(sum.y)), cp.y) : __fmul_rn(c4[1], static_cast<float>(sum.y)));
-                const float y2 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[2], static_cast<float>(sum.z)), cp.z) : __fmul_rn(c4[2], static_cast<float>(sum.z)));
-                const float y3 = __fmul_rn(am, comp ? __fadd_rn(__fmul_rn(c4[3], static_cast<float>(sum.w)), cp.w) : __fmul_rn(c4[3], static_cast<float>(sum.w)));
-                uint2 hv;
-                hv.x = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y0))) |
-                       (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y1))) << 16);
-                hv.y = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y2))) |
-                       (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y3))) << 16);
-                *reinterpret_cast<uint2*>(ystage + j * 128 + 4 * cg) = hv;
-                if (args.acc_debug && n4 < args.N)
-                  *reinterpret_cast<int4*>(args.acc_debug + static_cast<size_t>(m0 + j0 + j) * args.N + n4) = sum;
+                const float am = fa[j];
+                const int s4[4] = {sum[i].x, sum[i].y, sum[i].z, sum[i].w};
+                const float p4[4] = {cp.x, cp.y, cp.z, cp.w};
+                float y[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  float v = __fmul_rn(c4[e], static_cast<float>(s4[e]));
+                  if (comp) v = __fadd_rn(v, p4[e]);
+                  y[e] = __fmul_rn(am, v);
+                }
+                if (live) {
+                  uint2 hv;
+                  hv.x = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[0]))) |
+                         (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[1]))) << 16);
+                  hv.y = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[2]))) |
+                         (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y[3]))) << 16);
+                  *reinterpret_cast<uint2*>(Yp + static_cast<size_t>(m0 + j0 + j) * ldy + n4) = hv;
+                  if (accd) *reinterpret_cast<int4*>(accd + static_cast<size_t>(m0 + j0 + j) * ldy + n4) = sum[i];
+                }
               }
+              if (nl == 0 && q == 0 && j0 == 0 && jb < 112) QLIN_STAMP(24 + jb / 16);
             }
-            named_bar_sync(1, 128);  // staged tile complete
-            // 16-byte coalesced stores: 16 per 128-channel row
-            for (int idx = nl; idx < rr * 16; idx += 128) {
-              const int j = idx >> 4;
-              const int n8 = tn * C::kBN + (idx & 15) * 8;
-              if (n8 < args.N)
-                *reinterpret_cast<uint4*>(args.Y + static_cast<size_t>(m0 + j0 + j) * args.N + n8) =
-                    *reinterpret_cast<const uint4*>(ystage + j * 128 + (idx & 15) * 8);
-            }
-            if (nl == 0) QLIN_FIN(4);
-            if (nl == 0) QLIN_STAMP(18 + 4 * q);
-            named_bar_sync(1, 128);  // the buffer is reused by the next chunk
-            if (nl == 0) QLIN_FIN(5);
+            __syncwarp();  // the warp's shared rows are reused by the next chunk
           }
           if (nl == 0) args.ws_cnt[c_lo] = 0u;
-          if (nl == 0) QLIN_STAMP(13);
+          if (nl == 0) QLIN_STAMP(18 + 4 * q);
         }
+        if (nl == 0) QLIN_STAMP(13);
       }
     }
   }

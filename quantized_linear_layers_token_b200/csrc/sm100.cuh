@@ -152,6 +152,28 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// GPU-scope acquire-release fence; with a CTA barrier in front of it, it
+// releases every thread's earlier global stores (and, after an atomic that
+// observed the last arrival, acquires the other CTAs' stores for the whole
+// CTA once the barrier behind it is passed).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned atom_add_relaxed_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Asynchronous global -> shared copies (L2 only for the 16-byte form);
+// the issuing thread sees the data after cp_async_wait_all().
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Generic-proxy smem writes must be made visible to the async proxy (the
 // tensor core reads operands through it) before signalling the MMA warp.
 __device__ __forceinline__ void fence_proxy_async_smem() {
