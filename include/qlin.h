@@ -91,7 +91,11 @@ typedef enum {
  *                k0..k0+7, byte b (0..3) holds q[k0+b] in its low nibble and
  *                q[k0+4+b] in its high nibble (two's complement); then
  *                (word << 4) & 0xF0F0F0F0 holds the INT8 lanes 16*q[k0..k0+3]
- *                and word & 0xF0F0F0F0 the lanes 16*q[k0+4..k0+7].
+ *                and word & 0xF0F0F0F0 the lanes 16*q[k0+4..k0+7].  The
+ *                16-byte chunk c (inputs 32c..32c+31 of the tile) of row r
+ *                sits at chunk c ^ ((r / 2) % 4) of that row, so one thread
+ *                per row can read a block without shared-memory bank
+ *                conflicts.
  *                W8 format: 16384-byte blocks, 128 bytes per row, stored with
  *                the tensor core's 128-byte swizzle: the 16-byte chunk c
  *                (inputs 16c..16c+15 of the tile) of row r sits at chunk

@@ -125,36 +125,51 @@ struct GemmCfg {
   // step; large ones are tensor-bound and move one.
   static constexpr int KS = gemm_ks(BT);
   static constexpr bool kW4 = FMT != kFmtW8;
-  // converter warps (>= 4: the first four are the epilogue); two per SM
-  // sub-partition for the INT4 formats so unpacking is not latency-bound
-  static constexpr int kNCW = kW4 ? 8 : 4;
-  static constexpr int kThreads = 96 + 32 * kNCW;
+  // INT4 formats: eight converter warps (two per SM sub-partition, so
+  // unpacking is not latency-bound) and four epilogue warps of their own,
+  // so accumulators drain while later segments are still being converted.
+  // INT8: the four warps after the first three are the epilogue.
+  static constexpr int kNCW = kW4 ? 8 : 4;          // arrivals on the converter barriers
+  static constexpr int kEpiWarp0 = kW4 ? 3 + kNCW : 3;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
   // Small token tiles load the hi and lo compensation operands in one step
   // (one W_O^T block feeds both); large ones use two passes.
   static constexpr bool kCompFused = BT <= 64;
-  static constexpr int kABytes = KS * 16384;                             // KS x (128 x 128 B)
+  // INT4 formats with token tiles up to 64 keep the converted INT8 weight
+  // operand in tensor memory (tcgen05.st by the converters, MMA with A in
+  // TMEM): no shared-memory round trip for the 16 KiB of INT8 per K-block.
+  static constexpr bool kTA = kW4 && BT <= 64;
+  static constexpr int kACols = KS * 32;                                 // TMEM columns per A slot
+  static constexpr int kABytes = kTA ? 0 : KS * 16384;                   // smem per A slot: KS x (128 x 128 B)
   static constexpr int kXTile = BT * 128;                                // BT x 128 B per K-block
   static constexpr int kXTiles = KS > (kCompFused ? 2 : 1) ? KS : (kCompFused ? 2 : 1);
   static constexpr int kXBytes = (kXTile * kXTiles + 1023) / 1024 * 1024;
   static constexpr int kStgRatio = KS * 8192;                            // g128 ratio rows follow the codes
   static constexpr int kStgBytes = kW4 ? KS * 8192 + (FMT == kFmtW4G128 ? KS * 256 : 0) : 0;
+  static constexpr int kCompSlots = kTA ? 2 : 0;                         // W_O^T ring (16 KiB slots)
   static constexpr int kSmemLimit = 232448;          // 227 KB per CTA
   static constexpr int kReserve = 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table
   static constexpr int kBudget = kSmemLimit - kReserve;
   static constexpr int kXSlots = KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 ? 4 : 3));
-  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes) / kABytes;
-  static constexpr int kASlots = kW4 ? (KS == 4 ? 2 : (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)))
-                                     : (kASlotsW8 > 8 ? 8 : kASlotsW8);
-  static constexpr int kStgSlotsFit = kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes) / kStgBytes : 0;
+  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes) / (KS * 16384);
+  static constexpr int kASlots = kTA ? (BT <= 16 ? 3 : 4)
+                                     : (kW4 ? (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)) : (kASlotsW8 > 8 ? 8 : kASlotsW8));
+  static constexpr int kStgSlotsFit =
+      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384) / kStgBytes : 0;
   static constexpr int kStgSlots = kStgSlotsFit > 16 ? 16 : kStgSlotsFit;
   static constexpr int kOffA = 0;
   static constexpr int kOffX = kASlots * kABytes;
-  static constexpr int kOffStg = kOffX + kXSlots * kXBytes;
+  static constexpr int kOffComp = kOffX + kXSlots * kXBytes;
+  static constexpr int kOffStg = kOffComp + kCompSlots * 16384;
   static constexpr int kOffBar = kOffStg + kStgSlots * kStgBytes;
   static constexpr int kOffBnd = kOffBar + 1024;     // stream-K boundary table (<= 256 entries)
   static constexpr int kSmemBytes = kReserve + kOffBar;
   static constexpr uint32_t kTxX = BT * 128;
   static constexpr uint32_t kTxU = (kCompFused ? 2 : 1) * BT * 128;
+  // TMEM: accumulators (two buffers of main + compensation columns), then
+  // the A slots
+  static_assert(!kTA || 2 * 2 * BT + kASlots * kACols <= 512, "TMEM budget");
+  static_assert(!kTA || kCompFused, "the TMEM-A variant loads hi and lo compensation rows together");
   static_assert(kASlots >= 2 && kASlots <= 8, "A ring");
   static_assert(kXSlots >= 2 && kXSlots <= 8, "X ring");
   static_assert(!kW4 || (kStgSlots >= 2 && kStgSlots <= 16), "staging ring");
@@ -164,8 +179,9 @@ struct GemmCfg {
 // TMEM columns per accumulator buffer and the number of buffers.
 __host__ __device__ inline int tmem_buf_cols(int BT, bool comp) { return comp ? 2 * BT : BT; }
 __host__ __device__ inline int tmem_nbuf(int BT, bool comp) { return 2 * tmem_buf_cols(BT, comp) <= 512 ? 2 : 1; }
-__host__ __device__ inline uint32_t tmem_alloc_cols(int BT, bool comp) {
-  const int need = tmem_nbuf(BT, comp) * tmem_buf_cols(BT, comp);
+// Columns to allocate: the accumulator buffers plus `extra` (A slots).
+__host__ __device__ inline uint32_t tmem_alloc_cols(int BT, bool comp, int extra) {
+  const int need = tmem_nbuf(BT, comp) * tmem_buf_cols(BT, comp) + extra;
   uint32_t c = 32;
   while (c < static_cast<uint32_t>(need)) c <<= 1;
   return c;
@@ -294,7 +310,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   uint64_t* xempty = xfull + 8;
   uint64_t* acc_full = xempty + 8;    // [2]
   uint64_t* acc_empty = acc_full + 2; // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 3);
+  uint64_t* cfull = acc_empty + 2;    // [2] W_O^T ring (TMEM-A variant)
+  uint64_t* cempty = cfull + 2;       // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;  // [2]
   unsigned* sbnd = reinterpret_cast<unsigned*>(smem + C::kOffBnd);
@@ -304,7 +322,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   const bool comp = args.nO > 0;
   const int bcols = tmem_buf_cols(BT, comp);
   const int nbuf = tmem_nbuf(BT, comp);
-  const uint32_t tcols = tmem_alloc_cols(BT, comp);
+  const uint32_t tcols = tmem_alloc_cols(BT, comp, C::kTA ? P * C::kACols : 0);
+  const uint32_t a_col0 = static_cast<uint32_t>(nbuf * bcols);  // first TMEM column of the A slots
   const unsigned it0 = args.bnd[blockIdx.x];
   const unsigned it1 = args.bnd[blockIdx.x + 1];
   QLIN_TRACE_INIT
@@ -316,11 +335,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   if (threadIdx.x == 0) {
     for (int i = 0; i < 16; ++i) {
       mbar_init(&sfull[i], 1);
-      mbar_init(&sempty[i], kConvThreads);
+      mbar_init(&sempty[i], C::kNCW);  // one arrival per converter warp
     }
     for (int i = 0; i < 8; ++i) {
       mbar_init(&afull[i], 1);
-      mbar_init(&aconv[i], kConvThreads);
+      mbar_init(&aconv[i], C::kNCW);
       mbar_init(&aempty[i], 1);
       mbar_init(&xfull[i], 1);
       mbar_init(&xempty[i], 1);
@@ -328,6 +347,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
+      mbar_init(&cfull[b], 1);
+      mbar_init(&cempty[b], 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -397,7 +418,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // loads issued into each A slot
       unsigned it = it0;
       Segment sg;
-      int g = 0, gs = 0;
+      int g = 0, gs = 0, gc = 0;
       bool ok = true;
       while (ok && next_segment(it, it1, args, sg)) {
         const int tn = static_cast<int>(sg.tile % args.tiles_n);
@@ -423,6 +444,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                           &sfull[ls]);
             if (gs == 0) QLIN_STAMP(2);
             ++gs;
+          } else if (C::kTA) {
+            // W_O^T block of a compensation step into its own ring, as soon
+            // as a slot is free (well ahead of its use)
+            const int cs = gc & 1;
+            if (gc >= 2 && !mbar_wait(&cempty[cs], static_cast<uint32_t>(gc / 2 - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int j = r - args.nk;
+            const int ib = C::kCompFused ? j : (j >= args.ncs ? j - args.ncs : j);
+            mbar_arrive_expect_tx(&cfull[cs], 16384u);
+            bulk_load(smem + C::kOffComp + cs * 16384, args.wot + (static_cast<size_t>(tn) * args.ncs + ib) * 8192,
+                      16384, &cfull[cs]);
+            ++gc;
           } else if (!C::kW4) {
             // INT8 weights and W_O^T blocks into the A ring.  This thread
             // waits on every A slot in order, so a parity wait never runs
@@ -453,6 +488,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       }
       QLIN_STAMP(3);
       if (C::kW4) drain_ring(sfull, LS, gs);
+      if (C::kTA) drain_ring(cfull, 2, gc);
       for (int p = 0; p < P; ++p) {  // outstanding A-ring copies
         if (!a_issues[p]) continue;
         const uint64_t t0 = globaltimer_ns();
@@ -472,6 +508,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       // 2 (shared addresses stay below 2^18, so the field never carries).
       const uint64_t adesc0 = sdesc_k_sw128(smem_u32(smem + C::kOffA));
       const uint64_t xdesc0 = sdesc_k_sw128(smem_u32(smem + C::kOffX));
+      const uint64_t cdesc0 = sdesc_k_sw128(smem_u32(smem + C::kOffComp));
+      int gm = 0, gc = 0;       // TMEM-A variant: main steps (A ring) and compensation steps (W_O^T ring)
       uint32_t conv_phase = 0;  // per A slot: parity of the next converter phase
       uint32_t full_phase = 0;  // per A slot: parity of the next copy phase
       unsigned it = it0;
@@ -491,6 +529,55 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           const bool main_step = r < args.nk;
           if (!mbar_wait(&xfull[x], static_cast<uint32_t>(g / XS) & 1u, abort_flag)) { ok = false; break; }
           QLIN_STEP(g, 5);
+          if (C::kTA) {
+            const uint64_t bd = xdesc0 + static_cast<uint64_t>(x * (C::kXBytes >> 4));
+            if (main_step) {
+              const int pa = gm % P;
+              if (!mbar_wait(&aconv[pa], static_cast<uint32_t>(gm / P) & 1u, abort_flag)) { ok = false; break; }
+              if (g == 0) QLIN_STAMP(8);
+              QLIN_STEP(g, 6);
+              tc_fence_after();
+              const uint32_t at = tmem + a_col0 + static_cast<uint32_t>(pa * C::kACols);
+              const int nkb = min(C::KS, args.kb - r * C::KS);
+              mma_i8_ta(dmain, at, bd, idesc_main, r > sg.r0 ? 1u : 0u);
+              mma_i8_ta(dmain, at + 8, bd + 2, idesc_main, 1u);
+              mma_i8_ta(dmain, at + 16, bd + 4, idesc_main, 1u);
+              mma_i8_ta(dmain, at + 24, bd + 6, idesc_main, 1u);
+#pragma unroll
+              for (int i = 1; i < C::KS; ++i) {
+                if (i < nkb) {
+                  const uint32_t ai = at + static_cast<uint32_t>(i * 32);
+                  const uint64_t bi = bd + static_cast<uint64_t>(i * (C::kXTile >> 4));
+                  mma_i8_ta(dmain, ai, bi, idesc_main, 1u);
+                  mma_i8_ta(dmain, ai + 8, bi + 2, idesc_main, 1u);
+                  mma_i8_ta(dmain, ai + 16, bi + 4, idesc_main, 1u);
+                  mma_i8_ta(dmain, ai + 24, bi + 6, idesc_main, 1u);
+                }
+              }
+              mma_commit(&aempty[pa]);
+              ++gm;
+            } else {
+              const int cs = gc & 1;
+              if (!mbar_wait(&cfull[cs], static_cast<uint32_t>(gc / 2) & 1u, abort_flag)) { ok = false; break; }
+              if (g == 0) QLIN_STAMP(8);
+              QLIN_STEP(g, 6);
+              tc_fence_after();
+              const uint64_t ad = cdesc0 + static_cast<uint64_t>(cs * (16384 >> 4));
+              const uint32_t acc0 = ((r == args.nk) || (r == sg.r0)) ? 0u : 1u;
+              mma_f16(dcomp, ad, bd, idesc_comp, acc0);
+              mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
+              mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
+              mma_f16(dcomp, ad + 6, bd + 6, idesc_comp, 1u);
+              const uint64_t bd2 = bd + (C::kXTile >> 4);  // lo rows (fused hi + lo)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) mma_f16(dcomp, ad + 2 * kk, bd2 + 2 * kk, idesc_comp, 1u);
+              mma_commit(&cempty[cs]);
+              ++gc;
+            }
+            mma_commit(&xempty[x]);
+            QLIN_STEP(g, 7);
+            continue;
+          }
           if (main_step && C::kW4) {
             if (!mbar_wait(&aconv[p], (conv_phase >> p) & 1u, abort_flag)) { ok = false; break; }
             conv_phase ^= 1u << p;
@@ -545,12 +632,83 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     __syncwarp();
   } else {
     const int ctid = threadIdx.x - 96;
+    const bool epi = warp >= C::kEpiWarp0;
     // The epilogue threads keep the boundary table in shared memory (read
     // after the epilogue's first named barrier).
-    if (warp < 7)
-      for (int i = ctid; i < args.grid; i += 128) sbnd[i] = args.bnd[i];
+    if (epi)
+      for (int i = threadIdx.x - 32 * C::kEpiWarp0; i < args.grid; i += 128) sbnd[i] = args.bnd[i];
     // ------------------------------------------------------------ converters
-    if (C::kW4) {
+    if (C::kTA && !epi) {
+      // One thread per weight row: warp w may only reach TMEM lanes
+      // 32*(w % 4) .. +31, so the two warps of a lane quarter split the
+      // step's K-blocks (even / odd).  Each thread reads its row's 64 packed
+      // bytes of a block (swizzled chunks: conflict-free), widens them to
+      // 128 INT8 codes in registers and stores 32 TMEM columns.
+      const int qd = warp & 3;
+      const int half = (warp - 3) >> 2;
+      const int row = qd * 32 + lane;
+      const int sw = (row >> 1) & 3;
+      const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16) + a_col0;
+      unsigned it = it0;
+      Segment sg;
+      int gm = 0, gs = 0;
+      bool ok = true;
+      while (ok && next_segment(it, it1, args, sg)) {
+        for (int r = sg.r0; r < sg.r1 && r < args.nk; ++r) {
+          const int ls = gs % LS;
+          if (!mbar_wait(&sfull[ls], static_cast<uint32_t>(gs / LS) & 1u, abort_flag)) { ok = false; break; }
+          if (gs == 0 && ctid == 0) QLIN_STAMP(6);
+          const int pa = gm % P;
+          if (gm >= P && !mbar_wait(&aempty[pa], static_cast<uint32_t>(gm / P - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
+          const int nkb = min(C::KS, args.kb - r * C::KS);
+          for (int blk = half; blk < nkb; blk += 2) {
+            const unsigned char* src = stg + blk * 8192 + row * 64;
+            uint32_t o[32];
+            if (FMT == kFmtW4PC) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+                uint4 o0, o1;
+                unpack_w4pc(w, o0, o1);
+                o[8 * c + 0] = o0.x; o[8 * c + 1] = o0.y; o[8 * c + 2] = o0.z; o[8 * c + 3] = o0.w;
+                o[8 * c + 4] = o1.x; o[8 * c + 5] = o1.y; o[8 * c + 6] = o1.z; o[8 * c + 7] = o1.w;
+              }
+            } else {
+              const uint16_t rbits = reinterpret_cast<const uint16_t*>(stg + C::kStgRatio + blk * 256)[row];
+              const __half2 r1 = __half2half2(__ushort_as_half(rbits));
+              const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+                const uint2 a0 = requant_g128(w.x, r1, r16);
+                const uint2 a1 = requant_g128(w.y, r1, r16);
+                const uint2 a2 = requant_g128(w.z, r1, r16);
+                const uint2 a3 = requant_g128(w.w, r1, r16);
+                o[8 * c + 0] = a0.x; o[8 * c + 1] = a0.y; o[8 * c + 2] = a1.x; o[8 * c + 3] = a1.y;
+                o[8 * c + 4] = a2.x; o[8 * c + 5] = a2.y; o[8 * c + 6] = a3.x; o[8 * c + 7] = a3.y;
+              }
+            }
+            tmem_st32(tlane + static_cast<uint32_t>(pa * C::kACols + blk * 32), o);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sempty[ls]);  // staging slot consumed
+            mbar_arrive(&aconv[pa]);   // A slot written
+          }
+          if (ctid == 0) QLIN_STEP(gs, 4);
+          ++gm;
+          ++gs;
+        }
+      }
+      if (ctid == 0) QLIN_STAMP(7);
+    } else if (C::kW4 && !epi) {
       uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // W_O^T copies issued into each A slot (ctid 0)
       unsigned it = it0;
       Segment sg;
@@ -590,7 +748,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           for (int c = ctid; c < nchunk; c += kConvThreads) {
             const int blk = c >> 9;       // K-block within the step
             const int row = (c >> 2) & 127;
-            const int part = c & 3;
+            const int part = (c & 3) ^ ((row >> 1) & 3);  // staged chunks are swizzled by row
             unsigned char* A = A0 + blk * 16384;
             const uint4 w = *reinterpret_cast<const uint4*>(stg + c * 16);
             uint4 o0, o1;
@@ -611,9 +769,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             *reinterpret_cast<uint4*>(A + row * 128 + (((2 * part) ^ sw) << 4)) = o0;
             *reinterpret_cast<uint4*>(A + row * 128 + (((2 * part + 1) ^ sw) << 4)) = o1;
           }
-          mbar_arrive(&sempty[ls]);  // staging slot consumed
           fence_proxy_async_smem();
-          mbar_arrive(&aconv[p]);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sempty[ls]);  // staging slot consumed
+            mbar_arrive(&aconv[p]);    // A slot written
+          }
           if (ctid == 0) QLIN_STEP(g, 4);
           ++gs;
         }
@@ -630,7 +791,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       }
     }
     // ------------------------------------------------------------ epilogue
-    if (warp < 7) {
+    if (epi) {
       const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
       const int nl = quad * 32 + lane;
       griddep_wait();  // a[] comes from the previous kernel

@@ -13,10 +13,10 @@
 // Packed codes are tile-major so that the GEMM fetches each 128-channel x
 // 128-input block with one contiguous bulk copy: block (tn, kb) holds
 // channels 128*tn .. +127 (rows) and inputs 128*kb .. +127.  INT4 blocks are
-// 128 rows x 64 bytes (8 KiB); INT8 blocks are 128 rows x 128 bytes (16 KiB)
-// stored with the tensor core's 128-byte swizzle already applied (16-byte
-// chunk c of row r sits at chunk c ^ (r % 8)).  Padding rows and inputs are
-// zero.
+// 128 rows x 64 bytes (8 KiB), 16-byte chunk c of row r at chunk
+// c ^ ((r / 2) % 4); INT8 blocks are 128 rows x 128 bytes (16 KiB) stored
+// with the tensor core's 128-byte swizzle already applied (16-byte chunk c
+// of row r sits at chunk c ^ (r % 8)).  Padding rows and inputs are zero.
 #pragma once
 
 #include "sm100.cuh"
@@ -55,9 +55,13 @@ __device__ __forceinline__ uint2 pack8_bytes(const int (&q)[8]) {
 }
 
 // Byte offset of the 8 codes k0..k0+7 of channel n in the tiled layouts.
+// INT4 rows are 64 bytes; the 16-byte chunk c of row r sits at chunk
+// c ^ ((r >> 1) & 3) (conflict-free reads with one thread per row).
 __device__ __forceinline__ size_t w4_tile_offset(int n, int k0, int KB) {
   const size_t blk = static_cast<size_t>(n >> 7) * KB + (k0 >> 7);
-  return (blk * 128 + (n & 127)) * 64 + ((k0 & 127) >> 1);
+  const int r = n & 127;
+  const int byte = (k0 & 127) >> 1;
+  return (blk * 128 + r) * 64 + ((((byte >> 4) ^ ((r >> 1) & 3))) << 4) + (byte & 15);
 }
 __device__ __forceinline__ size_t w8_tile_offset(int n, int k0, int KB) {
   const size_t blk = static_cast<size_t>(n >> 7) * KB + (k0 >> 7);

@@ -18,12 +18,19 @@ def _swizzle_rows(block: np.ndarray) -> np.ndarray:
 
 
 def tile_w4(packed: np.ndarray, N: int, K: int) -> np.ndarray:
-    """packed: uint8 [N][K/2] (row n = channel n) -> tiled uint8 bytes."""
+    """packed: uint8 [N][K/2] (row n = channel n) -> tiled uint8 bytes; the
+    16-byte chunk c of row r of a block moves to chunk c ^ ((r // 2) % 4)."""
     TN, KB = -(-N // 128), -(-K // 128)
     full = np.zeros((TN * 128, KB * 64), np.uint8)
     full[:N, :K // 2] = packed
-    t = full.reshape(TN, 128, KB, 64).transpose(0, 2, 1, 3)
-    return np.ascontiguousarray(t).reshape(-1)
+    t = np.ascontiguousarray(full.reshape(TN, 128, KB, 64).transpose(0, 2, 1, 3))
+    out = np.empty_like(t)
+    src = t.reshape(TN, KB, 128, 4, 16)
+    dst = out.reshape(TN, KB, 128, 4, 16)
+    for r in range(128):
+        for c in range(4):
+            dst[:, :, r, c ^ ((r // 2) % 4)] = src[:, :, r, c]
+    return out.reshape(-1)
 
 
 def tile_w8(q_nk: np.ndarray, N: int, K: int) -> np.ndarray:
