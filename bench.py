@@ -302,13 +302,9 @@ def main():
                               "nws": nws})
     stream = torch.cuda.Stream(device)
 
-    # DP exchange buffers (N > 1): all outlier column maxima of a step in one vector
-    offs = []
-    tot = 0
-    for sl in slots:
-        offs.append(tot)
-        tot += len(meta[sl["si"]]["O"])
-    cmax_all = torch.zeros(max(tot, 1), dtype=torch.float32, device=device)
+    # DP exchange (N > 1): all outlier column maxima of a step in one vector
+    from quantized_linear_layers_token_b200.dp import ColmaxExchange
+    xchg = ColmaxExchange([len(meta[sl["si"]]["O"]) for sl in slots], device)
 
     def step_single():
         for sl in slots:
@@ -316,21 +312,18 @@ def main():
                               sl["nws"], stream)
 
     def step_dp():
-        for sl, o in zip(slots, offs):
-            nO = len(meta[sl["si"]]["O"])
-            if nO:
-                qlin.qlin_outlier_colmax(sl["X"], sl["M"], sl["layer"].w, cmax_all[o:o + nO], stream)
+        for j, sl in enumerate(slots):
+            if xchg.n_outliers[j]:
+                qlin.qlin_outlier_colmax(sl["X"], sl["M"], sl["layer"].w, xchg.view(j), stream)
         with torch.cuda.stream(stream):
-            dist.all_reduce(cmax_all, op=dist.ReduceOp.MAX)
-        for sl, o in zip(slots, offs):
-            nO = len(meta[sl["si"]]["O"])
+            xchg.allreduce()
+        for j, sl in enumerate(slots):
             lay = sl["layer"]
-            if nO:
-                qlin.qlin_momentum_update(lay.w, cmax_all[o:o + nO], sl["s"], wl.gamma, stream)
-            ws = sl["ws"]
-            # quant_act(update=0) + gemm through the split entry points
-            M, K = sl["M"], meta[sl["si"]]["K"]
-            qlin.qlin_forward(sl["X"], M, lay.w, sl["s"], wl.gamma, False, sl["Y"], ws, sl["nws"], stream)
+            if xchg.n_outliers[j]:
+                qlin.qlin_momentum_update(lay.w, xchg.view(j), sl["s"], wl.gamma, stream)
+            # quantization with the already-updated state, then the GEMM
+            qlin.qlin_forward(sl["X"], sl["M"], lay.w, sl["s"], wl.gamma, False, sl["Y"], sl["ws"], sl["nws"],
+                              stream)
 
     step = step_single if world == 1 else step_dp
 
@@ -479,8 +472,14 @@ def main():
                "sample": sample.describe(t)}
 
     # per forward: quantization (+ the column-max kernel when the momentum
-    # update is not fused, M > 64) and the GEMM
-    gpu_launches = args.steps * sum(2 + (1 if len(meta[sl["si"]]["O"]) and sl["M"] > 64 else 0) for sl in slots)
+    # update is not fused, M > 64) and the GEMM; data-parallel steps run the
+    # column-max and momentum kernels separately around the all-reduce
+    def forward_launches(sl):
+        has_o = len(meta[sl["si"]]["O"]) > 0
+        if world > 1:
+            return 2 + (2 if has_o else 0)
+        return 2 + (1 if has_o and sl["M"] > 64 else 0)
+    gpu_launches = args.steps * sum(forward_launches(sl) for sl in slots)
 
     if rank == 0:
         line = {
