@@ -151,6 +151,7 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
   int* sO = reinterpret_cast<int*>(quant_smem + static_cast<size_t>(K) * 2);
   float* sS = reinterpret_cast<float*>(sO + nO);
   unsigned* mask = reinterpret_cast<unsigned*>(sS + nO);
+  unsigned* cmx = mask + (K >> 5);  // [nO] fused column maxima (fp32 bits)
   __shared__ float red[kQuantThreads / 32];
   __shared__ int is_last;
 
@@ -181,14 +182,37 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
     const int col = sO[i];
     atomicOr(&mask[col >> 5], 1u << (col & 31));
-    if (FUSED) {
-      float cm = 0.f;
-      for (int r = 0; r < mom.M; ++r) {
-        const float xv_r = fabsf(h2f(r == m ? xs[col] : X[static_cast<size_t>(r) * K + col]));
-        cm = xv_r > cm ? xv_r : cm;
+    if (FUSED) cmx[i] = 0u;
+  }
+  if (FUSED) {
+    // column maxima of |X[:, O]| over all M rows: the M * nO gathers are
+    // spread over the whole CTA, eight independent loads per thread in
+    // flight, merged with shared-memory atomicMax on the fp32 bit patterns
+    // (non-negative, so ordered like unsigned integers)
+    __syncthreads();
+    const int pairs = mom.M * nO;
+    for (int p0 = threadIdx.x; p0 < pairs; p0 += 8 * kQuantThreads) {
+      uint16_t hv[8];
+      int ii[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u * kQuantThreads;
+        ii[u] = -1;
+        hv[u] = 0;
+        if (p < pairs) {
+          const int r = p / nO;
+          const int i = p - r * nO;
+          ii[u] = i;
+          hv[u] = X[static_cast<size_t>(r) * K + sO[i]];
+        }
       }
-      sS[i] = momentum_step(sS[i], mom.gamma, cm, mom.wmaxO[i]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (ii[u] >= 0) atomicMax(&cmx[ii[u]], __float_as_uint(fabsf(h2f(hv[u]))));
     }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nO; i += kQuantThreads)
+      sS[i] = momentum_step(sS[i], mom.gamma, __uint_as_float(cmx[i]), mom.wmaxO[i]);
   }
   __syncthreads();
 

@@ -107,6 +107,14 @@ struct GemmArgs {
   int T;                // iterations per tile = nk + nc
   int grid;             // persistent CTAs (<= kMaxGrid)
   int split;            // 1: stream-K split points; 0: whole tiles per CTA
+  // Cluster split-K (cs > 1): the grid is ncl clusters of cs CTAs; cluster c
+  // takes tiles c, c + ncl, ...; cluster rank r computes iterations
+  // [cb[r], cb[r+1]) of each (cb[cs] = T, the compensation run never cut),
+  // and the partials are reduced through distributed shared memory: rank q
+  // owns channels [q * 128/cs, (q+1) * 128/cs) of the tile.
+  int cs;
+  int ncl;
+  int cb[9];
   // bnd[c] = first iteration of CTA c, bnd[grid] = tiles * T (computed on
   // the host by gemm_boundary(); kernel parameters, read from the constant
   // cache).
@@ -147,21 +155,31 @@ struct GemmCfg {
   static constexpr int kStgRatio = KS * 8192;                            // g128 ratio rows follow the codes
   static constexpr int kStgBytes = kW4 ? KS * 8192 + (FMT == kFmtW4G128 ? KS * 256 : 0) : 0;
   static constexpr int kCompSlots = kTA ? 2 : 0;                         // W_O^T ring (16 KiB slots)
+  // Cluster split-K receive buffer (token tiles up to 64): INT32 partials of
+  // the owned channel slice from every rank, [rank][channel][kRecvLd], and the
+  // fp32 compensation of the slice from the rank that ran it; rows padded by
+  // 4 words so 16-byte reads of consecutive channels hit distinct banks.
+  static constexpr bool kCluster = BT <= 64;
+  static constexpr int kRecvLd = BT + 4;
+  static constexpr int kRecvMain = kCluster ? 128 * kRecvLd * 4 : 0;
+  static constexpr int kRecvComp = kCluster ? 64 * kRecvLd * 4 : 0;  // slice <= 64 channels (cs >= 2)
+  static constexpr int kRecvBytes = kRecvMain + kRecvComp;
   static constexpr int kSmemLimit = 232448;          // 227 KB per CTA
   static constexpr int kReserve = 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table
   static constexpr int kBudget = kSmemLimit - kReserve;
   static constexpr int kXSlots = KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 ? 4 : 3));
-  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes) / (KS * 16384);
+  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes - kRecvBytes) / (KS * 16384);
   static constexpr int kASlots = kTA ? (BT <= 16 ? 3 : 4)
                                      : (kW4 ? (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)) : (kASlotsW8 > 8 ? 8 : kASlotsW8));
   static constexpr int kStgSlotsFit =
-      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384) / kStgBytes : 0;
+      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384 - kRecvBytes) / kStgBytes : 0;
   static constexpr int kStgSlots = kStgSlotsFit > 16 ? 16 : kStgSlotsFit;
   static constexpr int kOffA = 0;
   static constexpr int kOffX = kASlots * kABytes;
   static constexpr int kOffComp = kOffX + kXSlots * kXBytes;
   static constexpr int kOffStg = kOffComp + kCompSlots * 16384;
-  static constexpr int kOffBar = kOffStg + kStgSlots * kStgBytes;
+  static constexpr int kOffRecv = kOffStg + kStgSlots * kStgBytes;
+  static constexpr int kOffBar = kOffRecv + kRecvBytes;
   static constexpr int kOffBnd = kOffBar + 1024;     // stream-K boundary table (<= 256 entries)
   static constexpr int kSmemBytes = kReserve + kOffBar;
   static constexpr uint32_t kTxX = BT * 128;
@@ -200,6 +218,22 @@ inline unsigned gemm_boundary(int c, long long tiles, int T, int nk, int grid, i
   return static_cast<unsigned>(b);
 }
 
+// Cluster split-K rank ranges of one tile's T iterations: an even cut, with
+// any cut inside the compensation run (iterations nk .. T-1) moved to its
+// start so one rank runs all of it.  Returns false when a rank would get no
+// iterations.
+inline bool cluster_bounds(int T, int nk, int cs, int* cb) {
+  for (int r = 0; r < cs; ++r) {
+    int b = static_cast<int>((static_cast<long long>(T) * r) / cs);
+    if (b > nk) b = nk;
+    cb[r] = b;
+  }
+  cb[cs] = T;
+  for (int r = 0; r < cs; ++r)
+    if (cb[r + 1] <= cb[r]) return false;
+  return true;
+}
+
 // The boundary table is copied into shared memory at kernel start (entries
 // 0 .. grid-1; entry grid is the total iteration count).
 __device__ __forceinline__ unsigned bnd_s(int c, const unsigned* sbnd, const GemmArgs& g) {
@@ -227,14 +261,50 @@ struct Segment {
   int r0, r1;  // iterations [r0, r1) of the tile
 };
 
-__device__ __forceinline__ bool next_segment(unsigned& it, unsigned it1, const GemmArgs& g, Segment& sg) {
-  if (it >= it1) return false;
-  const unsigned T = static_cast<unsigned>(g.T);
-  sg.tile = it / T;
-  sg.r0 = static_cast<int>(it - sg.tile * T);
-  const unsigned left = it1 - it;
-  sg.r1 = static_cast<int>(left < T - sg.r0 ? sg.r0 + left : T);
-  it += sg.r1 - sg.r0;
+// Segments of one CTA, in order: a stream-K range of the flat iteration
+// space, or (cluster split-K) the same rank range of every cluster tile.
+// The fields come from the CTA plan staged in shared memory at start-up, so
+// no role waits on kernel-parameter loads for its first segment.
+struct SegGen {
+  unsigned it, it1, T;
+  int u, cid, ncl, ntiles, r0, r1;
+  bool cl;
+};
+
+// CTA plan (shared memory, written once during setup).
+enum : int { kPlanIt0 = 0, kPlanIt1, kPlanT, kPlanR0, kPlanR1, kPlanNcl, kPlanTiles, kPlanWords };
+
+__device__ __forceinline__ SegGen seg_begin(const int* plan, int cid, bool cl) {
+  SegGen s;
+  s.it = static_cast<unsigned>(plan[kPlanIt0]);
+  s.it1 = static_cast<unsigned>(plan[kPlanIt1]);
+  s.T = static_cast<unsigned>(plan[kPlanT]);
+  s.u = 0;
+  s.cid = cid;
+  s.ncl = plan[kPlanNcl];
+  s.ntiles = plan[kPlanTiles];
+  s.r0 = plan[kPlanR0];
+  s.r1 = plan[kPlanR1];
+  s.cl = cl;
+  return s;
+}
+
+__device__ __forceinline__ bool seg_next(SegGen& s, Segment& sg) {
+  if (s.cl) {
+    const int t = s.cid + s.u * s.ncl;
+    if (t >= s.ntiles) return false;
+    sg.tile = static_cast<unsigned>(t);
+    sg.r0 = s.r0;
+    sg.r1 = s.r1;
+    ++s.u;
+    return true;
+  }
+  if (s.it >= s.it1) return false;
+  sg.tile = s.it / s.T;
+  sg.r0 = static_cast<int>(s.it - sg.tile * s.T);
+  const unsigned left = s.it1 - s.it;
+  sg.r1 = static_cast<int>(left < s.T - sg.r0 ? sg.r0 + left : s.T);
+  s.it += sg.r1 - sg.r0;
   return true;
 }
 
@@ -312,9 +382,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   uint64_t* acc_empty = acc_full + 2; // [2]
   uint64_t* cfull = acc_empty + 2;    // [2] W_O^T ring (TMEM-A variant)
   uint64_t* cempty = cfull + 2;       // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + 2);
+  uint64_t* recv_full = cempty + 2;   // cluster split-K: this CTA's receive buffer is complete
+  uint64_t* recv_free = recv_full + 1; // every owner has read this CTA's previous partials
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;  // [2]
+  int* plan = const_cast<int*>(last_flag + 2);  // [kPlanWords]
   unsigned* sbnd = reinterpret_cast<unsigned*>(smem + C::kOffBnd);
 
   const int warp = threadIdx.x >> 5;
@@ -324,38 +397,61 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   const int nbuf = tmem_nbuf(BT, comp);
   const uint32_t tcols = tmem_alloc_cols(BT, comp, C::kTA ? P * C::kACols : 0);
   const uint32_t a_col0 = static_cast<uint32_t>(nbuf * bcols);  // first TMEM column of the A slots
-  const unsigned it0 = args.bnd[blockIdx.x];
-  const unsigned it1 = args.bnd[blockIdx.x + 1];
+  const bool cl = args.cs > 1;
+  const int crk = cl ? static_cast<int>(cluster_ctarank()) : 0;
+  const int cid = cl ? static_cast<int>(cluster_id_x()) : 0;
+  // it0 of this CTA's stream-K range (read once more by the epilogue)
+  const unsigned it0 = cl ? 0u : args.bnd[blockIdx.x];
+  const int slice = 128 / args.cs;  // channels owned per cluster rank
+  // bytes arriving in a receive buffer per round: every rank's INT32 slice,
+  // plus the compensation slice when the layer has outliers
+  const uint32_t recv_bytes =
+      static_cast<uint32_t>(128 * BT * 4 + (args.nO > 0 ? slice * BT * 4 : 0));
   QLIN_TRACE_INIT
 #ifdef QLIN_TRACE
   if (threadIdx.x == 0 && qlin_tr) qlin_tr[blockIdx.x * 32 + 31] = static_cast<long long>(globaltimer_ns());
 #endif
   if (threadIdx.x == 0) QLIN_STAMP(0);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 16; ++i) {
-      mbar_init(&sfull[i], 1);
-      mbar_init(&sempty[i], C::kNCW);  // one arrival per converter warp
-    }
-    for (int i = 0; i < 8; ++i) {
+  // warp 0 initialises the barriers, one per lane
+  if (warp == 0) {
+    if (lane < 16) {
+      mbar_init(&sfull[lane], 1);
+      mbar_init(&sempty[lane], C::kNCW);  // one arrival per converter warp
+    } else if (lane < 24) {
+      const int i = lane - 16;
       mbar_init(&afull[i], 1);
       mbar_init(&aconv[i], C::kNCW);
       mbar_init(&aempty[i], 1);
       mbar_init(&xfull[i], 1);
       mbar_init(&xempty[i], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
+    } else if (lane < 26) {
+      const int b = lane - 24;
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
       mbar_init(&cfull[b], 1);
       mbar_init(&cempty[b], 1);
+    } else if (lane == 26) {
+      mbar_init(recv_full, 1);
+      mbar_init(recv_free, static_cast<uint32_t>(args.cs));
+      *abort_flag = 0;
     }
-    *abort_flag = 0;
     fence_barrier_init();
+    __syncwarp();
+    if (lane == 26 && cl) mbar_arrive_expect_tx(recv_full, recv_bytes);  // round 0
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmX);
     if (comp) tma_prefetch_desc(&tmU);
+  }
+  if (warp == 3 && lane == 0) {
+    plan[kPlanIt0] = cl ? 0 : static_cast<int>(it0);
+    plan[kPlanIt1] = cl ? 0 : static_cast<int>(args.bnd[blockIdx.x + 1]);
+    plan[kPlanT] = args.T;
+    plan[kPlanR0] = cl ? args.cb[crk] : 0;
+    plan[kPlanR1] = cl ? args.cb[crk + 1] : 0;
+    plan[kPlanNcl] = args.ncl;
+    plan[kPlanTiles] = args.tiles_n * args.tiles_m;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, tcols);
@@ -364,6 +460,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Peers' barriers must be initialised before any remote access: arrive
+  // now, wait just before the first one (epilogue) or at the end.
+  if (cl) cluster_arrive();
+  bool cl_waited = false;
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) QLIN_STAMP(1);
   // Let the next kernel in the stream start its prologue; it waits for this
@@ -375,11 +475,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     if (lane == 0) {
       griddep_wait();  // activations come from the previous kernel
       QLIN_STAMP(4);
-      unsigned it = it0;
+      bool first_x = true;
+      SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int g = 0;
       bool ok = true;
-      while (ok && next_segment(it, it1, args, sg)) {
+      while (ok && seg_next(gen, sg)) {
         const int m0 = static_cast<int>(sg.tile / args.tiles_n) * BT;
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
           const int x = g % XS;
@@ -389,11 +490,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           }
           unsigned char* xb = smem + C::kOffX + x * C::kXBytes;
           QLIN_STEP(g, 0);
+          if (first_x) QLIN_STAMP(28);
           if (r < args.nk) {
             const int kb0 = r * C::KS;
             const int nkb = min(C::KS, args.kb - kb0);
             mbar_arrive_expect_tx(&xfull[x], static_cast<uint32_t>(nkb) * C::kTxX);
-            for (int i = 0; i < nkb; ++i) tma_load_2d(xb + i * C::kXTile, &tmX, &xfull[x], (kb0 + i) * 128, m0);
+            if (first_x) QLIN_STAMP(29);
+            for (int i = 0; i < nkb; ++i) {
+              tma_load_2d(xb + i * C::kXTile, &tmX, &xfull[x], (kb0 + i) * 128, m0);
+              if (first_x && i == 0) QLIN_STAMP(30);
+            }
+            first_x = false;
+            if (g == 0) QLIN_STAMP(19);
           } else {
             const int j = r - args.nk;
             mbar_arrive_expect_tx(&xfull[x], C::kTxU);
@@ -414,13 +522,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   } else if (warp == 2) {
     // ------------------------------------------------------------ weight producer
     if (lane == 0) {
+      QLIN_STAMP(25);
       const uint64_t pol_stream = policy_evict_first();
       uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // loads issued into each A slot
-      unsigned it = it0;
+      SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int g = 0, gs = 0, gc = 0;
       bool ok = true;
-      while (ok && next_segment(it, it1, args, sg)) {
+      while (ok && seg_next(gen, sg)) {
+        if (g == 0) QLIN_STAMP(26);
         const int tn = static_cast<int>(sg.tile % args.tiles_n);
         const int n0 = tn * C::kBN;
         const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(min(C::kBN, args.N - n0)) * 2u : 0u;
@@ -435,6 +545,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             QLIN_STEP(g, 1);
             const int kb0 = r * C::KS;
             const int nkb = min(C::KS, args.kb - kb0);
+            if (gs == 0) QLIN_STAMP(15);
             mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nkb) * (8192u + rb));
             bulk_load_hint(st, args.codes + (static_cast<size_t>(tn) * args.kb + kb0) * 8192,
                            static_cast<uint32_t>(nkb) * 8192u, &sfull[ls], pol_stream);
@@ -512,11 +623,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       int gm = 0, gc = 0;       // TMEM-A variant: main steps (A ring) and compensation steps (W_O^T ring)
       uint32_t conv_phase = 0;  // per A slot: parity of the next converter phase
       uint32_t full_phase = 0;  // per A slot: parity of the next copy phase
-      unsigned it = it0;
+      SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int g = 0, seg = 0;
       bool ok = true;
-      while (ok && next_segment(it, it1, args, sg)) {
+      while (ok && seg_next(gen, sg)) {
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
         if (use > 0 && !mbar_wait(&acc_empty[buf], static_cast<uint32_t>(use - 1) & 1u, abort_flag)) break;
@@ -635,7 +746,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     const bool epi = warp >= C::kEpiWarp0;
     // The epilogue threads keep the boundary table in shared memory (read
     // after the epilogue's first named barrier).
-    if (epi)
+    if (epi && !cl)
       for (int i = threadIdx.x - 32 * C::kEpiWarp0; i < args.grid; i += 128) sbnd[i] = args.bnd[i];
     // ------------------------------------------------------------ converters
     if (C::kTA && !epi) {
@@ -649,11 +760,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       const int row = qd * 32 + lane;
       const int sw = (row >> 1) & 3;
       const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16) + a_col0;
-      unsigned it = it0;
+      SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int gm = 0, gs = 0;
       bool ok = true;
-      while (ok && next_segment(it, it1, args, sg)) {
+      while (ok && seg_next(gen, sg)) {
         for (int r = sg.r0; r < sg.r1 && r < args.nk; ++r) {
           const int ls = gs % LS;
           if (!mbar_wait(&sfull[ls], static_cast<uint32_t>(gs / LS) & 1u, abort_flag)) { ok = false; break; }
@@ -710,11 +821,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       if (ctid == 0) QLIN_STAMP(7);
     } else if (C::kW4 && !epi) {
       uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // W_O^T copies issued into each A slot (ctid 0)
-      unsigned it = it0;
+      SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int g = 0, gs = 0;
       bool ok = true;
-      while (ok && next_segment(it, it1, args, sg)) {
+      while (ok && seg_next(gen, sg)) {
         const int tn = static_cast<int>(sg.tile % args.tiles_n);
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
           const int p = g % P;
@@ -801,10 +912,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       unsigned pend_tile[2] = {0u, 0u};
       int pend_add[2] = {0, 0};
       int npend = 0;
-      unsigned it = it0;
+      SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int seg = 0;
-      while (next_segment(it, it1, args, sg)) {
+      while (seg_next(gen, sg)) {
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
         bool ok = mbar_wait(&acc_full[buf], static_cast<uint32_t>(use) & 1u, abort_flag);
@@ -824,9 +935,32 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tile * static_cast<unsigned>(args.T) ? 1 : 0);
         int32_t* pacc = args.ws_acc + static_cast<size_t>(my_slot) * BT * 128;
         float* pcmp = args.ws_comp + static_cast<size_t>(my_slot) * BT * 128;
+        // cluster split-K: channel nl goes to owner rank nl / slice
+        uint32_t r_main = 0, r_comp = 0, r_bar = 0;
+        float a_own = 0.f, cn_own = 0.f;
+        if (cl) {
+          if (!cl_waited) {
+            cluster_wait();
+            cl_waited = true;
+          }
+          // the owner's scale factors, requested before the exchange
+          {
+            const int n_own = tn * C::kBN + crk * slice + (nl % slice);
+            if (n_own < args.N) cn_own = FMT == kFmtW4PC ? __fmul_rn(args.cscale[n_own], 0.0625f) : args.cscale[n_own];
+            if (nl < mvalid) a_own = args.a[m0 + nl];
+          }
+          const int q = nl / slice;
+          const int c = nl - q * slice;
+          r_main = mapa_shared(smem_u32(smem + C::kOffRecv + ((crk * slice + c) * C::kRecvLd) * 4), q);
+          r_comp = mapa_shared(smem_u32(smem + C::kOffRecv + C::kRecvMain + (c * C::kRecvLd) * 4), q);
+          r_bar = mapa_shared(smem_u32(recv_full), q);
+          // the owners have read this CTA's previous round
+          if (seg > 0) ok = mbar_wait_cluster(recv_free, static_cast<uint32_t>(seg - 1) & 1u, abort_flag) && ok;
+          ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+        }
 #pragma unroll 1
         for (int c0 = 0; c0 < BT; c0 += 16) {
-          if (c0 >= mvalid) break;
+          if (!cl && c0 >= mvalid) break;
           uint32_t acc[16], cmp[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) { acc[j] = 0u; cmp[j] = 0u; }
@@ -835,7 +969,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             if (has_comp) tmem_ld16(trow + BT + c0, cmp);
             tmem_ld_wait();
           }
-          if (whole) {
+          if (cl) {
+            // every token column goes out (fixed byte count per round)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              st_async_v4(r_main + (c0 + 4 * i) * 4,
+                          make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]), r_bar);
+              if (has_comp && comp)
+                st_async_v4(r_comp + (c0 + 4 * i) * 4,
+                            make_uint4(cmp[4 * i], cmp[4 * i + 1], cmp[4 * i + 2], cmp[4 * i + 3]), r_bar);
+            }
+          } else if (whole) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int m = m0 + c0 + j;
@@ -860,7 +1004,50 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);  // TMEM buffer may be reused
-        if (!whole && npend < 2) {
+        if (cl) {
+          // Owner of channels [crk * slice, +slice): sum every rank's INT32
+          // partial in rank order (exact), add the compensation, dequantize.
+          // Thread t takes channel t % slice and token quads t / slice,
+          // + cs, ...
+          const int c = nl % slice;
+          const int n_own = tn * C::kBN + crk * slice + c;
+          float* sa = reinterpret_cast<float*>(smem + C::kOffBnd);  // token scales of this tile
+          if (nl < BT) sa[nl] = a_own;
+          if (nl == 0 && seg == 0) QLIN_STAMP(23);
+          ok = mbar_wait_cluster(recv_full, static_cast<uint32_t>(seg) & 1u, abort_flag) && ok;
+          if (nl == 0 && seg == 0) QLIN_STAMP(12);
+          ok = __all_sync(0xffffffffu, ok);
+          named_bar_sync(1, 128);  // token scales staged
+          const unsigned char* rb = smem + C::kOffRecv;
+          for (int jq = nl / slice; jq < BT / 4; jq += args.cs) {
+            int4 sum = make_int4(0, 0, 0, 0);
+            for (int r = 0; r < args.cs; ++r) {
+              const int4 v = *reinterpret_cast<const int4*>(rb + ((r * slice + c) * C::kRecvLd + 4 * jq) * 4);
+              sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+            }
+            float4 cp = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (comp) cp = *reinterpret_cast<const float4*>(rb + C::kRecvMain + (c * C::kRecvLd + 4 * jq) * 4);
+            const int s4[4] = {sum.x, sum.y, sum.z, sum.w};
+            const float p4[4] = {cp.x, cp.y, cp.z, cp.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int j = 4 * jq + i;
+              if (ok && j < mvalid && n_own < args.N) {
+                float v = __fmul_rn(cn_own, static_cast<float>(s4[i]));
+                if (comp) v = __fadd_rn(v, p4[i]);
+                const float y = __fmul_rn(sa[j], v);
+                args.Y[static_cast<size_t>(m0 + j) * args.N + n_own] = __half_as_ushort(__float2half_rn(y));
+                if (args.acc_debug) args.acc_debug[static_cast<size_t>(m0 + j) * args.N + n_own] = s4[i];
+              }
+            }
+          }
+          named_bar_sync(1, 128);  // every read of the receive buffer is done
+          if (nl == 0 && cid + (seg + 1) * args.ncl < args.tiles_n * args.tiles_m) {
+            mbar_arrive_expect_tx(recv_full, recv_bytes);  // next round
+            for (int r = 0; r < args.cs; ++r) mbar_arrive_remote(mapa_shared(smem_u32(recv_free), r));
+          }
+        }
+        if (!cl && !whole && npend < 2) {
           pend_tile[npend] = sg.tile;
           pend_add[npend] = sg.r1 - sg.r0;
           ++npend;
@@ -1004,6 +1191,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   }
   tc_fence_before();
   __syncthreads();
+  if (cl) {  // no CTA leaves while a peer may still touch its shared memory
+    if (!cl_waited) cluster_wait();
+    cluster_arrive();
+    cluster_wait();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tcols);

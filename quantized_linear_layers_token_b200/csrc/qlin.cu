@@ -133,6 +133,24 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 // its prologue (and the GEMM its weight stream) while the previous kernel in
 // the stream finishes; every kernel waits on the grid dependency before it
 // reads what the previous one wrote.  QLIN_NO_PDL=1 turns this off.
+// QLIN_NO_CLUSTER=1 keeps decode GEMMs on global-memory stream-K.
+bool cluster_disabled() {
+  static const bool off = [] {
+    const char* e = getenv("QLIN_NO_CLUSTER");
+    return e && e[0] == '1';
+  }();
+  return off;
+}
+
+int forced_cluster_size() {
+  static const int cs = [] {
+    const char* e = getenv("QLIN_CLUSTER_CS");
+    const int v = e ? atoi(e) : 0;
+    return (v == 2 || v == 4 || v == 8) ? v : 0;
+  }();
+  return cs;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = getenv("QLIN_NO_PDL");
@@ -141,20 +159,38 @@ bool pdl_enabled() {
   return on;
 }
 
+// `cluster` > 1 launches thread-block clusters of that many CTAs along x.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                     Args... args) {
+cudaError_t launch_kc(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, int cluster,
+                      Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args... args) {
+  return launch_kc(kern, grid, block, smem, stream, 1, args...);
 }
 
 int sm_count() {
@@ -239,7 +275,66 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != QLIN_OK) return st;
   }
-  cudaError_t e = launch_k(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, tmX, tmU, args);
+  // Token tiles up to 64 whose tiles would be split (decode): cluster
+  // split-K when it is expected to beat global-memory stream-K.  Costs in
+  // units of one pipeline step, fitted to B200 measurements of the 7B decode
+  // shapes: a cluster round costs its longest rank range plus the exchange of
+  // BT x 128 partials through distributed shared memory (about 0.5 / 2 / 7.5
+  // steps at BT = 16 / 32 / 64); stream-K costs its per-CTA iterations plus
+  // the global fixup chain (about 7 / 12 / 28 steps).  QLIN_CLUSTER_CS=n
+  // forces cluster size n when it is valid (measurement aid).
+  if (C::kCluster && args.split && !cluster_disabled()) {
+    const double xchg = BT <= 16 ? 0.5 : (BT <= 32 ? 2.0 : 7.5);
+    const double fixup = BT <= 16 ? 7.0 : (BT <= 32 ? 12.0 : 28.0);
+    const int forced = forced_cluster_size();
+    const long long iters = static_cast<long long>(args.tiles_n) * args.tiles_m * args.T;
+    const double streamk_cost = static_cast<double>((iters + args.grid - 1) / args.grid) + fixup;
+    const long long tiles = static_cast<long long>(args.tiles_n) * args.tiles_m;
+    static int max_clusters[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};  // per cluster size, this instantiation
+    int best_cs = 0, best_ncl = 0;
+    double best_cost = streamk_cost;
+    for (int cs = 2; cs <= 8; cs *= 2) {
+      int cb[9];
+      if (!cluster_bounds(args.T, args.nk, cs, cb)) continue;
+      if (max_clusters[cs] < 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(cs * ((sm_count() + cs - 1) / cs)));
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = static_cast<unsigned>(cs);
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+          cudaGetLastError();
+          n = 0;
+        }
+        max_clusters[cs] = n;
+      }
+      const int ncl = static_cast<int>(max_clusters[cs] < tiles ? max_clusters[cs] : tiles);
+      if (ncl < 1) continue;
+      int span = 0;
+      for (int r = 0; r < cs; ++r) span = cb[r + 1] - cb[r] > span ? cb[r + 1] - cb[r] : span;
+      double cost = static_cast<double>((tiles + ncl - 1) / ncl) * (span + xchg);
+      if (forced) cost = forced == cs ? -1.0 : 1e30;
+      if (cost < best_cost) {
+        best_cs = cs;
+        best_ncl = ncl;
+        best_cost = cost;
+      }
+    }
+    if (best_cs) {
+      args.cs = best_cs;
+      args.ncl = best_ncl;
+      args.grid = best_cs * best_ncl;
+      cluster_bounds(args.T, args.nk, best_cs, args.cb);
+    }
+  }
+  cudaError_t e = launch_kc(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, args.cs, tmX, tmU, args);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
 }
@@ -286,6 +381,9 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
   args.T = p.T;
   args.grid = p.grid;
   args.split = p.split;
+  args.cs = 1;
+  args.ncl = 0;
+  for (int r = 0; r < 9; ++r) args.cb[r] = 0;
   const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
   if (tiles * p.T >= (1LL << 31)) return fail(QLIN_ERR_SHAPE, "problem too large (%lld tile iterations)", tiles * p.T);
   for (int c = 0; c <= p.grid; ++c) args.bnd[c] = gemm_boundary(c, tiles, p.T, p.nk, p.grid, p.split);
@@ -298,6 +396,8 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
 }
 
 // ---------------------------------------------------------------- act quant
+constexpr int kQuantSmemMax = 232448 - 1024;  // 227 KB per CTA, less room for the kernel's static shared memory
+
 size_t act_ws_bytes(const qlin_weights* w) {
   return w->n_outlier > 0 ? round_up(size_t(w->n_outlier) * 4 + 4, kAlign) : 0;
 }
@@ -319,16 +419,24 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   }
   const int nvec = K / 8;
   const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
-  const size_t smem = size_t(K) * 2 + size_t(nO) * 8 + size_t(K / 32) * 4;
+  const size_t smem = size_t(K) * 2 + size_t(nO) * 12 + size_t(K / 32) * 4;
+  if (smem > size_t(kQuantSmemMax))
+    return fail(QLIN_ERR_SHAPE, "K=%d with %d outliers needs %zu bytes of shared memory", K, nO, smem);
   const int nOp = w->n_outlier_pad;
   cudaError_t e = cudaSuccess;
 #define QLIN_QUANT_CASE(V)                                                                                   \
   {                                                                                                          \
     static std::once_flag once_##V;                                                                          \
+    static cudaError_t attr_##V = cudaSuccess;                                                               \
     std::call_once(once_##V, [] {                                                                            \
-      cudaFuncSetAttribute(quant_kernel<V, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);  \
-      cudaFuncSetAttribute(quant_kernel<V, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024); \
+      attr_##V = cudaFuncSetAttribute(quant_kernel<V, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
+                                      kQuantSmemMax);                                                        \
+      if (attr_##V == cudaSuccess)                                                                           \
+        attr_##V = cudaFuncSetAttribute(quant_kernel<V, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                        kQuantSmemMax);                                                      \
     });                                                                                                      \
+    if (attr_##V != cudaSuccess)                                                                             \
+      return fail(QLIN_ERR_CUDA, "quant_kernel attribute: %s", cudaGetErrorString(attr_##V));               \
   }                                                                                                          \
   e = fused ? launch_k(quant_kernel<V, true>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,             \
                        static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom)         \
