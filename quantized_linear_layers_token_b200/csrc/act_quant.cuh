@@ -15,8 +15,9 @@
 //                   column; with `update` set, the last CTA to finish (a
 //                   completion counter, no spinning) applies the momentum
 //                   recurrence to s in place and clears its scratch.
-//   quant_kernel    one CTA per token: 128-bit loads of the row, warp-shuffle
-//                   + shared-memory row max, RNE codes, 64-bit stores; also
+//   quant_kernel    one CTA per token: 128-bit loads of the row staged in
+//                   shared memory, fp16 |x| row max, RNE codes, 64-bit
+//                   stores, outlier codes patched in afterwards; also
 //                   emits the compact outlier codes XqO and, when asked, the
 //                   fp16 compensation operand U = XqO * (s - 1) as hi + lo.
 #pragma once
@@ -26,11 +27,13 @@
 namespace qlin {
 
 constexpr int kColmaxRows = 32;   // rows per CTA of colmax_kernel
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 512;
 constexpr int kFusedMomentumMaxM = 64;  // up to this many tokens the update runs inside quant_kernel
 
 
-__device__ __forceinline__ float block_max_256(float v, float* red /* >= 8 floats */) {
+__device__ __forceinline__ __half2 u32_as_half2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+__device__ __forceinline__ float block_max(float v, float* red /* >= kQuantThreads / 32 floats */) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
@@ -134,62 +137,61 @@ struct MomentumArgs {
   int M;               // rows of X (all of them feed the column maxima)
 };
 
-// One CTA per token row.  VPT = 8-element vectors per thread (K <= 2048*VPT).
+// One CTA per token row.  VPT = 8-element vectors per thread
+// (K <= 8 * kQuantThreads * VPT).
 // FUSED: every CTA also computes the outlier column maxima over all M rows
 // and the momentum update itself (identical in every CTA, cheap for small
 // M); the last CTA to finish writes the new state back, after every CTA has
 // read the old one.
-// Latency: the row is requested first (independent of O), then staged in
-// shared memory so every outlier lookup is a shared-memory read.
+// The row is staged in shared memory; the outlier columns' raw values are
+// set aside and their slots zeroed, so the row maximum (fp16 |x| maxima,
+// exact) and the quantization pass run without per-element outlier checks;
+// the outlier codes x_hat = x / s are computed separately and written over
+// the zeros after a barrier.  O and max|W_O| do not depend on the previous
+// kernel and are read before the grid dependency.
 template <int VPT, bool FUSED>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ O, int nO,
              float* __restrict__ s, int8_t* __restrict__ Xq, float* __restrict__ a,
              int8_t* __restrict__ XqO, uint16_t* __restrict__ U, int nOp, MomentumArgs mom) {
   extern __shared__ __align__(16) unsigned char quant_smem[];
-  uint16_t* xs = reinterpret_cast<uint16_t*>(quant_smem);          // [K] this row
+  uint16_t* xs = reinterpret_cast<uint16_t*>(quant_smem);          // [K] this row (outliers zeroed)
   int* sO = reinterpret_cast<int*>(quant_smem + static_cast<size_t>(K) * 2);
-  float* sS = reinterpret_cast<float*>(sO + nO);
-  unsigned* mask = reinterpret_cast<unsigned*>(sS + nO);
-  unsigned* cmx = mask + (K >> 5);  // [nO] fused column maxima (fp32 bits)
+  float* sS = reinterpret_cast<float*>(sO + nO);                    // [nO] momentum state
+  float* xo = sS + nO;                                              // [nO] raw outlier values of this row
+  unsigned* cmx = reinterpret_cast<unsigned*>(xo + nO);             // [nO] fused column maxima (fp32 bits)
   __shared__ float red[kQuantThreads / 32];
   __shared__ int is_last;
 
   griddep_launch_dependents();
-  griddep_wait();  // X (and s) may come from the previous kernel
-  const int m = blockIdx.x;
-  const uint16_t* xrow = X + static_cast<size_t>(m) * K;
-  const uint4* xv = reinterpret_cast<const uint4*>(xrow);
-  const int nvec = K >> 3;
-  uint4 v[VPT];
-#pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int vi = threadIdx.x + j * kQuantThreads;
-    if (vi < nvec) v[j] = __ldg(xv + vi);
-  }
-  const int nmask = K >> 5;
-  for (int w = threadIdx.x; w < nmask; w += kQuantThreads) mask[w] = 0u;
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
     sO[i] = O[i];
-    sS[i] = s[i];
+    if (FUSED) cmx[i] = 0u;
   }
+  float wmx = 0.f;  // max|W_O| of outlier threadIdx.x (FUSED, nO <= kQuantThreads handled in the loop below)
+  if (FUSED && threadIdx.x < nO) wmx = mom.wmaxO[threadIdx.x];
+  griddep_wait();  // X (and s) may come from the previous kernel
+  const int m = blockIdx.x;
+  const uint4* xv = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
+  const int nvec = K >> 3;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int vi = threadIdx.x + j * kQuantThreads;
-    if (vi < nvec) reinterpret_cast<uint4*>(xs)[vi] = v[j];
+    if (vi < nvec) reinterpret_cast<uint4*>(xs)[vi] = __ldg(xv + vi);
   }
+  for (int i = threadIdx.x; i < nO; i += kQuantThreads) sS[i] = s[i];
   __syncthreads();
+  // set the outliers aside (each thread owns distinct columns)
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
     const int col = sO[i];
-    atomicOr(&mask[col >> 5], 1u << (col & 31));
-    if (FUSED) cmx[i] = 0u;
+    xo[i] = h2f(xs[col]);
+    xs[col] = 0;
   }
   if (FUSED) {
     // column maxima of |X[:, O]| over all M rows: the M * nO gathers are
     // spread over the whole CTA, eight independent loads per thread in
     // flight, merged with shared-memory atomicMax on the fp32 bit patterns
     // (non-negative, so ordered like unsigned integers)
-    __syncthreads();
     const int pairs = mom.M * nO;
     for (int p0 = threadIdx.x; p0 < pairs; p0 += 8 * kQuantThreads) {
       uint16_t hv[8];
@@ -212,30 +214,30 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     }
     __syncthreads();
     for (int i = threadIdx.x; i < nO; i += kQuantThreads)
-      sS[i] = momentum_step(sS[i], mom.gamma, __uint_as_float(cmx[i]), mom.wmaxO[i]);
+      sS[i] = momentum_step(sS[i], mom.gamma, __uint_as_float(cmx[i]),
+                            i == static_cast<int>(threadIdx.x) ? wmx : mom.wmaxO[i]);
   }
   __syncthreads();
 
-  float lmax = 0.f;
+  // row maximum: fp16 |x| maxima of the staged row (exact), then the
+  // outliers' |x / s| in fp32
+  __half2 hm = __float2half2_rn(0.f);
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int vi = threadIdx.x + j * kQuantThreads;
     if (vi < nvec) {
-      const unsigned mb = (mask[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
-      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint16_t hb = static_cast<uint16_t>(w4[e >> 1] >> ((e & 1) * 16));
-        const float f = fabsf(h2f(hb));
-        if (!((mb >> e) & 1u)) lmax = f > lmax ? f : lmax;
-      }
+      const uint4 w = reinterpret_cast<const uint4*>(xs)[vi];
+      const __half2 m01 = __hmax2(__habs2(u32_as_half2(w.x)), __habs2(u32_as_half2(w.y)));
+      const __half2 m23 = __hmax2(__habs2(u32_as_half2(w.z)), __habs2(u32_as_half2(w.w)));
+      hm = __hmax2(hm, __hmax2(m01, m23));
     }
   }
+  float lmax = fmaxf(__low2float(hm), __high2float(hm));
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
-    const float f = fabsf(__fdiv_rn(h2f(xs[sO[i]]), sS[i]));
+    const float f = fabsf(__fdiv_rn(xo[i], sS[i]));
     lmax = f > lmax ? f : lmax;
   }
-  const float amax = block_max_256(lmax, red);
+  const float amax = block_max(lmax, red);
   const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
   if (threadIdx.x == 0) a[m] = __fdiv_rn(amax, 127.f);
 
@@ -244,27 +246,25 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
   for (int j = 0; j < VPT; ++j) {
     const int vi = threadIdx.x + j * kQuantThreads;
     if (vi < nvec) {
-      const unsigned mb = (mask[vi >> 2] >> ((vi & 3) * 8)) & 0xFFu;
-      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+      const uint4 w = reinterpret_cast<const uint4*>(xs)[vi];
+      const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
       int q[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint16_t hb = static_cast<uint16_t>(w4[e >> 1] >> ((e & 1) * 16));
-        float xh = h2f(hb);
-        if ((mb >> e) & 1u) {
-          const int i = lower_bound_sorted(sO, nO, vi * 8 + e);
-          xh = __fdiv_rn(xh, sS[i]);
-        }
-        q[e] = quant_code(xh, inv);
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(u32_as_half2(w4[e]));
+        q[2 * e] = quant_code(f.x, inv);
+        q[2 * e + 1] = quant_code(f.y, inv);
       }
       *reinterpret_cast<uint2*>(qrow + static_cast<size_t>(vi) * 8) = pack8_bytes(q);
     }
   }
+  __syncthreads();  // the zero codes at the outlier columns are written before the patch below
   const size_t lo_off = static_cast<size_t>(gridDim.x) * nOp;  // U holds [2][M][nOp]: hi rows, then lo rows
   for (int i = threadIdx.x; i < nOp; i += kQuantThreads) {
     if (i < nO) {
-      const float xh = __fdiv_rn(h2f(xs[sO[i]]), sS[i]);
+      const float xh = __fdiv_rn(xo[i], sS[i]);
       const int q = quant_code(xh, inv);
+      qrow[sO[i]] = static_cast<int8_t>(q);
       XqO[static_cast<size_t>(m) * nO + i] = static_cast<int8_t>(q);
       if (U) {
         const uint2 hl = comp_split(q, sS[i]);
@@ -277,12 +277,16 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     }
   }
   if (FUSED) {
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = (atomicAdd(mom.counter, 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (is_last) {
+    if (gridDim.x == 1) {  // the only reader of the old state
       for (int i = threadIdx.x; i < nO; i += kQuantThreads) s[i] = sS[i];
-      if (threadIdx.x == 0) *mom.counter = 0u;
+    } else {
+      __syncthreads();
+      if (threadIdx.x == 0) is_last = (atomicAdd(mom.counter, 1u) == gridDim.x - 1);
+      __syncthreads();
+      if (is_last) {
+        for (int i = threadIdx.x; i < nO; i += kQuantThreads) s[i] = sS[i];
+        if (threadIdx.x == 0) *mom.counter = 0u;
+      }
     }
   }
 }

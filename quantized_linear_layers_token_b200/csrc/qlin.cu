@@ -419,7 +419,7 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   }
   const int nvec = K / 8;
   const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
-  const size_t smem = size_t(K) * 2 + size_t(nO) * 12 + size_t(K / 32) * 4;
+  const size_t smem = size_t(K) * 2 + size_t(nO) * 16;
   if (smem > size_t(kQuantSmemMax))
     return fail(QLIN_ERR_SHAPE, "K=%d with %d outliers needs %zu bytes of shared memory", K, nO, smem);
   const int nOp = w->n_outlier_pad;
@@ -447,7 +447,6 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   else if (vpt <= 4) { QLIN_QUANT_CASE(4) }
   else if (vpt <= 8) { QLIN_QUANT_CASE(8) }
   else if (vpt <= 16) { QLIN_QUANT_CASE(16) }
-  else if (vpt <= 32) { QLIN_QUANT_CASE(32) }
   else return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", K);
 #undef QLIN_QUANT_CASE
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "quant_kernel launch failed: %s", cudaGetErrorString(e));
