@@ -165,22 +165,27 @@ struct GemmCfg {
   static constexpr int kRecvComp = kCluster ? 64 * kRecvLd * 4 : 0;  // slice <= 64 channels (cs >= 2)
   static constexpr int kRecvBytes = kRecvMain + kRecvComp;
   static constexpr int kSmemLimit = 232448;          // 227 KB per CTA
-  static constexpr int kReserve = 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table
+  static constexpr int kReserve = 1024 + 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table, token scales
+  static constexpr int kYStage = 16 * 128 * 2;                  // one 16-token x 128-channel fp16 chunk of Y
   static constexpr int kBudget = kSmemLimit - kReserve;
   static constexpr int kXSlots = KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 ? 4 : 3));
-  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes - kRecvBytes) / (KS * 16384);
+  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes - kRecvBytes - 2 * kYStage) / (KS * 16384);
   static constexpr int kASlots = kTA ? (BT <= 16 ? 3 : 4)
                                      : (kW4 ? (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)) : (kASlotsW8 > 8 ? 8 : kASlotsW8));
   static constexpr int kStgSlotsFit =
-      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384 - kRecvBytes) / kStgBytes : 0;
+      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384 - kRecvBytes - 2 * kYStage) /
+                kStgBytes
+          : 0;
   static constexpr int kStgSlots = kStgSlotsFit > 16 ? 16 : kStgSlotsFit;
   static constexpr int kOffA = 0;
   static constexpr int kOffX = kASlots * kABytes;
   static constexpr int kOffComp = kOffX + kXSlots * kXBytes;
   static constexpr int kOffStg = kOffComp + kCompSlots * 16384;
   static constexpr int kOffRecv = kOffStg + kStgSlots * kStgBytes;
-  static constexpr int kOffBar = kOffRecv + kRecvBytes;
+  static constexpr int kOffYst = kOffRecv + kRecvBytes;              // two Y staging chunks
+  static constexpr int kOffBar = kOffYst + 2 * kYStage;
   static constexpr int kOffBnd = kOffBar + 1024;     // stream-K boundary table (<= 256 entries)
+  static constexpr int kOffSa = kOffBnd + 1024;      // token scales a[m] of the tile being finished
   static constexpr int kSmemBytes = kReserve + kOffBar;
   static constexpr uint32_t kTxX = BT * 128;
   static constexpr uint32_t kTxU = (kCompFused ? 2 : 1) * BT * 128;
@@ -363,7 +368,7 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int slots, int issued
 template <int FMT, int BT>
 __global__ void __launch_bounds__(GemmCfg<FMT, BT>::kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmU,
-            const __grid_constant__ GemmArgs args) {
+            const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmArgs args) {
   using C = GemmCfg<FMT, BT>;
   constexpr int P = C::kASlots;
   constexpr int XS = C::kXSlots;
@@ -855,19 +860,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
           unsigned char* A0 = smem + C::kOffA + p * C::kABytes;
           const int nchunk = min(C::KS, args.kb - r * C::KS) * 512;  // 16-byte packed chunks this step
-#pragma unroll 2
-          for (int c = ctid; c < nchunk; c += kConvThreads) {
-            const int blk = c >> 9;       // K-block within the step
+          // Token tiles >= 128 move one K-block per step: 512 chunks, at
+          // most two per thread.  Both chunks (and their ratios) are loaded
+          // before any operand store: the compiler cannot prove the staging
+          // and operand rings disjoint, so an interleaved load would wait for
+          // the previous store.
+          static_assert(!C::kW4 || C::kTA || C::KS == 1, "shared-memory operand path converts one K-block per step");
+          uint4 wpre[2];
+          uint16_t rpre[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = ctid + u * kConvThreads;
+            wpre[u] = c < nchunk ? *reinterpret_cast<const uint4*>(stg + c * 16) : make_uint4(0u, 0u, 0u, 0u);
+            rpre[u] = (FMT == kFmtW4G128 && c < nchunk)
+                          ? reinterpret_cast<const uint16_t*>(stg + C::kStgRatio)[(c >> 2) & 127]
+                          : static_cast<uint16_t>(0);
+          }
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = ctid + u * kConvThreads;
+            if (c >= nchunk) break;
             const int row = (c >> 2) & 127;
             const int part = (c & 3) ^ ((row >> 1) & 3);  // staged chunks are swizzled by row
-            unsigned char* A = A0 + blk * 16384;
-            const uint4 w = *reinterpret_cast<const uint4*>(stg + c * 16);
+            unsigned char* A = A0;
+            const uint4 w = wpre[u];
             uint4 o0, o1;
             if (FMT == kFmtW4PC) {
               unpack_w4pc(w, o0, o1);
             } else {
-              const uint16_t rbits = reinterpret_cast<const uint16_t*>(stg + C::kStgRatio + blk * 256)[row];
-              const __half2 r1 = __half2half2(__ushort_as_half(rbits));
+              const __half2 r1 = __half2half2(__ushort_as_half(rpre[u]));
               const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
               const uint2 a0 = requant_g128(w.x, r1, r16);
               const uint2 a1 = requant_g128(w.y, r1, r16);
@@ -915,6 +936,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       SegGen gen = seg_begin(plan, cid, cl);
       Segment sg;
       int seg = 0;
+      int ycnt = 0;  // Y chunks handed to TMA stores (two staging buffers alternate)
+      float* sa_t = reinterpret_cast<float*>(smem + C::kOffSa);
       while (seg_next(gen, sg)) {
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
@@ -958,6 +981,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           if (seg > 0) ok = mbar_wait_cluster(recv_free, static_cast<uint32_t>(seg - 1) & 1u, abort_flag) && ok;
           ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
         }
+        if (!cl && whole) {
+          // token scales of the tile, staged once
+          named_bar_sync(1, 128);
+          for (int j = nl; j < BT; j += 128) sa_t[j] = j < mvalid ? args.a[m0 + j] : 0.f;
+          named_bar_sync(1, 128);
+          if (seg == 0 && nl == 0) QLIN_STAMP(16);
+        }
 #pragma unroll 1
         for (int c0 = 0; c0 < BT; c0 += 16) {
           if (!cl && c0 >= mvalid) break;
@@ -980,17 +1010,49 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                             make_uint4(cmp[4 * i], cmp[4 * i + 1], cmp[4 * i + 2], cmp[4 * i + 3]), r_bar);
             }
           } else if (whole) {
+            // 16 tokens x 128 channels of Y, transposed through shared
+            // memory (written with thread = channel, read back with 16-byte
+            // row segments) and stored with coalesced 16-byte stores.  Two
+            // staging buffers alternate, so one barrier per chunk suffices:
+            // the next write of a buffer comes after the barrier that
+            // follows every thread's reads of it.
+            const int b = ycnt & 1;
+            uint16_t* ys = reinterpret_cast<uint16_t*>(smem + C::kOffYst + b * C::kYStage);
+            // the 16 token scales into registers before any staging store
+            // (the compiler cannot prove the two shared arrays disjoint, so
+            // interleaved loads would each wait for the previous store)
+            float sc[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 t = *reinterpret_cast<const float4*>(sa_t + c0 + 4 * q4);
+              sc[4 * q4] = t.x; sc[4 * q4 + 1] = t.y; sc[4 * q4 + 2] = t.z; sc[4 * q4 + 3] = t.w;
+            }
+            uint16_t yh[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const int m = m0 + c0 + j;
-              if (c0 + j < mvalid && n < args.N) {
-                float v = __fmul_rn(cn, static_cast<float>(static_cast<int32_t>(acc[j])));
-                if (comp) v = __fadd_rn(v, __uint_as_float(cmp[j]));
-                const float y = __fmul_rn(args.a[m], v);
-                args.Y[static_cast<size_t>(m) * args.N + n] = __half_as_ushort(__float2half_rn(y));
-                if (args.acc_debug) args.acc_debug[static_cast<size_t>(m) * args.N + n] = static_cast<int32_t>(acc[j]);
-              }
+              float v = __fmul_rn(cn, static_cast<float>(static_cast<int32_t>(acc[j])));
+              if (comp) v = __fadd_rn(v, __uint_as_float(cmp[j]));
+              yh[j] = __half_as_ushort(__float2half_rn(__fmul_rn(sc[j], v)));
             }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) ys[j * 128 + nl] = yh[j];
+            if (args.acc_debug) {
+              for (int j = 0; j < 16; ++j)
+                if (c0 + j < mvalid && n < args.N)
+                  args.acc_debug[static_cast<size_t>(m0 + c0 + j) * args.N + n] = static_cast<int32_t>(acc[j]);
+            }
+            named_bar_sync(1, 128);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int idx = nl + h * 128;  // 16 rows x 16 segments of 8 channels
+              const int j = idx >> 4;
+              const int n8 = tn * C::kBN + (idx & 15) * 8;
+              if (c0 + j < mvalid && n8 < args.N)
+                *reinterpret_cast<uint4*>(args.Y + static_cast<size_t>(m0 + c0 + j) * args.N + n8) =
+                    *reinterpret_cast<const uint4*>(ys + j * 128 + (idx & 15) * 8);
+            }
+            if (seg == 0 && nl == 0 && c0 == 0) QLIN_STAMP(17);
+            ++ycnt;
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -1002,6 +1064,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             }
           }
         }
+        if (seg == 0 && nl == 0) QLIN_STAMP(18);
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);  // TMEM buffer may be reused
         if (cl) {
@@ -1011,7 +1074,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           // + cs, ...
           const int c = nl % slice;
           const int n_own = tn * C::kBN + crk * slice + c;
-          float* sa = reinterpret_cast<float*>(smem + C::kOffBnd);  // token scales of this tile
+          float* sa = reinterpret_cast<float*>(smem + C::kOffSa);  // token scales of this tile
           if (nl < BT) sa[nl] = a_own;
           if (nl == 0 && seg == 0) QLIN_STAMP(23);
           ok = mbar_wait_cluster(recv_full, static_cast<uint32_t>(seg) & 1u, abort_flag) && ok;

@@ -265,10 +265,13 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
   });
   if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
 
-  CUtensorMap tmX, tmU;
+  CUtensorMap tmX, tmU, tmY;
   memset(&tmU, 0, sizeof(tmU));
   const int K = w->K, M = args.M;
   qlin_status st = make_map(&tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, BT, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLIN_OK) return st;
+  // Y [M][N] fp16, written in 16-token x 128-channel boxes
+  st = make_map(&tmY, args.Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w->N, M, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != QLIN_OK) return st;
   if (w->n_outlier > 0) {
     st = make_map(&tmU, U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->n_outlier_pad, 2 * static_cast<uint64_t>(M), 64, BT,
@@ -334,7 +337,8 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
       cluster_bounds(args.T, args.nk, best_cs, args.cb);
     }
   }
-  cudaError_t e = launch_kc(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, args.cs, tmX, tmU, args);
+  cudaError_t e =
+      launch_kc(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, args.cs, tmX, tmU, tmY, args);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
 }
