@@ -1082,25 +1082,47 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           ok = __all_sync(0xffffffffu, ok);
           named_bar_sync(1, 128);  // token scales staged
           const unsigned char* rb = smem + C::kOffRecv;
-          for (int jq = nl / slice; jq < BT / 4; jq += args.cs) {
-            int4 sum = make_int4(0, 0, 0, 0);
-            for (int r = 0; r < args.cs; ++r) {
-              const int4 v = *reinterpret_cast<const int4*>(rb + ((r * slice + c) * C::kRecvLd + 4 * jq) * 4);
-              sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-            }
-            float4 cp = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (comp) cp = *reinterpret_cast<const float4*>(rb + C::kRecvMain + (c * C::kRecvLd + 4 * jq) * 4);
-            const int s4[4] = {sum.x, sum.y, sum.z, sum.w};
-            const float p4[4] = {cp.x, cp.y, cp.z, cp.w};
+          // Thread t has token quads t / slice + k * cs, taken four at a
+          // time: the group's shared-memory reads all happen before its
+          // stores to Y (the compiler would otherwise order each read after
+          // the preceding stores).
+          constexpr int kG = 4;
+          for (int k0 = 0; nl / slice + k0 * args.cs < BT / 4; k0 += kG) {
+            int4 sum[kG];
+            float4 cp[kG];
+            float scl[kG][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int j = 4 * jq + i;
-              if (ok && j < mvalid && n_own < args.N) {
-                float v = __fmul_rn(cn_own, static_cast<float>(s4[i]));
-                if (comp) v = __fadd_rn(v, p4[i]);
-                const float y = __fmul_rn(sa[j], v);
-                args.Y[static_cast<size_t>(m0 + j) * args.N + n_own] = __half_as_ushort(__float2half_rn(y));
-                if (args.acc_debug) args.acc_debug[static_cast<size_t>(m0 + j) * args.N + n_own] = s4[i];
+            for (int k = 0; k < kG; ++k) {
+              sum[k] = make_int4(0, 0, 0, 0);
+              cp[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+              scl[k][0] = scl[k][1] = scl[k][2] = scl[k][3] = 0.f;
+              const int jq = nl / slice + (k0 + k) * args.cs;
+              if (jq < BT / 4) {
+                for (int r = 0; r < args.cs; ++r) {
+                  const int4 v = *reinterpret_cast<const int4*>(rb + ((r * slice + c) * C::kRecvLd + 4 * jq) * 4);
+                  sum[k].x += v.x; sum[k].y += v.y; sum[k].z += v.z; sum[k].w += v.w;
+                }
+                if (comp) cp[k] = *reinterpret_cast<const float4*>(rb + C::kRecvMain + (c * C::kRecvLd + 4 * jq) * 4);
+                const float4 t = *reinterpret_cast<const float4*>(sa + 4 * jq);
+                scl[k][0] = t.x; scl[k][1] = t.y; scl[k][2] = t.z; scl[k][3] = t.w;
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < kG; ++k) {
+              const int jq = nl / slice + (k0 + k) * args.cs;
+              if (jq >= BT / 4) break;
+              const int s4[4] = {sum[k].x, sum[k].y, sum[k].z, sum[k].w};
+              const float p4[4] = {cp[k].x, cp[k].y, cp[k].z, cp[k].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int j = 4 * jq + i;
+                if (ok && j < mvalid && n_own < args.N) {
+                  float v = __fmul_rn(cn_own, static_cast<float>(s4[i]));
+                  if (comp) v = __fadd_rn(v, p4[i]);
+                  const float y = __fmul_rn(scl[k][i], v);
+                  args.Y[static_cast<size_t>(m0 + j) * args.N + n_own] = __half_as_ushort(__float2half_rn(y));
+                  if (args.acc_debug) args.acc_debug[static_cast<size_t>(m0 + j) * args.N + n_own] = s4[i];
+                }
               }
             }
           }

@@ -205,12 +205,23 @@ int sm_count() {
   return cached[dev];
 }
 
+// QLIN_MAX_BT=128 caps the token tile (measurement aid).
+int max_bt() {
+  static const int v = [] {
+    const char* e = getenv("QLIN_MAX_BT");
+    const int x = e ? atoi(e) : 0;
+    return (x == 64 || x == 128) ? x : 256;
+  }();
+  return v;
+}
+
 int pick_bt(int M) {
-  if (M <= 16) return 16;
-  if (M <= 32) return 32;
-  if (M <= 64) return 64;
-  if (M <= 128) return 128;
-  return 256;
+  int bt = 256;
+  if (M <= 16) bt = 16;
+  else if (M <= 32) bt = 32;
+  else if (M <= 64) bt = 64;
+  else if (M <= 128) bt = 128;
+  return bt < max_bt() ? bt : max_bt();
 }
 
 // Work decomposition of one GEMM call (same on the host for workspace sizes
