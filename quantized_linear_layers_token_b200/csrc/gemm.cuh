@@ -467,7 +467,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   tc_fence_after();
   // Peers' barriers must be initialised before any remote access: arrive
   // now, wait just before the first one (epilogue) or at the end.
-  if (cl) cluster_arrive();
+  if (cl) cluster_arrive_relaxed();
   bool cl_waited = false;
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) QLIN_STAMP(1);

@@ -131,6 +131,12 @@ __device__ __forceinline__ void cluster_sync_all() {
 // thread of the cluster arrives once per phase and waits before arriving
 // again.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+// Arrive without ordering this thread's earlier memory operations (for the
+// start-up phase, whose mbarrier initialisations are published by
+// fence.mbarrier_init.release.cluster).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 
 // Bounded wait with cluster-scope acquire (phases completed by other CTAs'
