@@ -525,14 +525,15 @@ def main():
         cpu = {"value": sample.bytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": sample.describe(t)}
 
-    # per forward: quantization (+ the column-max kernel when the momentum
-    # update is not fused, M > 64) and the GEMM; data-parallel steps run the
-    # column-max and momentum kernels separately around the all-reduce
+    # per forward: quantization (+ the column-max kernel when the library
+    # does not fuse the momentum update into quantization, above 16 tokens)
+    # and the GEMM; data-parallel steps run the column-max and momentum
+    # kernels separately around the all-reduce
     def forward_launches(sl):
         has_o = len(meta[sl["si"]]["O"]) > 0
         if world > 1:
             return 2 + (2 if has_o else 0)
-        return 2 + (1 if has_o and sl["M"] > 64 else 0)
+        return 2 + (1 if has_o and sl["M"] > 16 else 0)
     gpu_launches = args.steps * sum(forward_launches(sl) for sl in slots)
 
     if rank == 0:

@@ -223,20 +223,38 @@ inline unsigned gemm_boundary(int c, long long tiles, int T, int nk, int grid, i
   return static_cast<unsigned>(b);
 }
 
-// Cluster split-K rank ranges of one tile's T iterations: an even cut, with
-// any cut inside the compensation run (iterations nk .. T-1) moved to its
-// start so one rank runs all of it.  Returns false when a rank would get no
-// iterations.
-inline bool cluster_bounds(int T, int nk, int cs, int* cb) {
-  for (int r = 0; r < cs; ++r) {
-    int b = static_cast<int>((static_cast<long long>(T) * r) / cs);
-    if (b > nk) b = nk;
-    cb[r] = b;
+// Cluster split-K rank ranges of one tile's T iterations (nk K-steps, then
+// the compensation run, which one rank runs whole: the last).  The last
+// rank also sends the compensation partial, so its load counts `ccost`
+// step-equivalents for that run; the cut gives it as many K-steps as keeps
+// the largest rank load smallest and splits the rest evenly.  Returns the
+// largest load, or a negative value when some rank would get no work.
+inline double cluster_bounds(int T, int nk, int cs, double ccost, int* cb) {
+  const int nc = T - nk;
+  int best_m = -1;
+  double best = 0.0;
+  for (int m = 0; m <= nk; ++m) {
+    const int rest = nk - m;
+    if (rest < cs - 1) break;  // every other rank needs at least one K-step
+    const double others = static_cast<double>((rest + cs - 2) / (cs - 1));
+    const double last = m + (nc > 0 ? ccost : 0.0);
+    const double load = others > last ? others : last;
+    if (nc == 0 && m == 0) continue;  // without a compensation run the last rank needs K-steps
+    if (best_m < 0 || load < best) {
+      best_m = m;
+      best = load;
+    }
   }
+  if (best_m < 0) return -1.0;
+  const int rest = nk - best_m;
+  int b = 0;
+  for (int r = 0; r < cs - 1; ++r) {
+    cb[r] = b;
+    b += rest / (cs - 1) + (r < rest % (cs - 1) ? 1 : 0);
+  }
+  cb[cs - 1] = b;  // == rest
   cb[cs] = T;
-  for (int r = 0; r < cs; ++r)
-    if (cb[r + 1] <= cb[r]) return false;
-  return true;
+  return best;
 }
 
 // The boundary table is copied into shared memory at kernel start (entries

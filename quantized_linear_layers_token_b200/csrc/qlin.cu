@@ -307,9 +307,13 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
     static int max_clusters[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};  // per cluster size, this instantiation
     int best_cs = 0, best_ncl = 0;
     double best_cost = streamk_cost;
+    // compensation run of the last rank: its steps plus sending a BT x slice
+    // fp32 partial (about BT / 32 steps at cs = 4)
     for (int cs = 2; cs <= 8; cs *= 2) {
       int cb[9];
-      if (!cluster_bounds(args.T, args.nk, cs, cb)) continue;
+      const double ccost = (args.T - args.nk) + (args.nO > 0 ? BT / 32.0 * 4.0 / cs : 0.0);
+      const double span = cluster_bounds(args.T, args.nk, cs, ccost, cb);
+      if (span < 0) continue;
       if (max_clusters[cs] < 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(cs * ((sm_count() + cs - 1) / cs)));
@@ -331,8 +335,6 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
       }
       const int ncl = static_cast<int>(max_clusters[cs] < tiles ? max_clusters[cs] : tiles);
       if (ncl < 1) continue;
-      int span = 0;
-      for (int r = 0; r < cs; ++r) span = cb[r + 1] - cb[r] > span ? cb[r + 1] - cb[r] : span;
       double cost = static_cast<double>((tiles + ncl - 1) / ncl) * (span + xchg);
       if (forced) cost = forced == cs ? -1.0 : 1e30;
       if (cost < best_cost) {
@@ -345,7 +347,8 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
       args.cs = best_cs;
       args.ncl = best_ncl;
       args.grid = best_cs * best_ncl;
-      cluster_bounds(args.T, args.nk, best_cs, args.cb);
+      cluster_bounds(args.T, args.nk, best_cs,
+                     (args.T - args.nk) + (args.nO > 0 ? BT / 32.0 * 4.0 / best_cs : 0.0), args.cb);
     }
   }
   cudaError_t e =
@@ -411,6 +414,18 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
 }
 
 // ---------------------------------------------------------------- act quant
+// Up to this many tokens the momentum update runs inside the quantization
+// kernel (every CTA gathers all rows' outlier values); above it a separate
+// column-max kernel gathers them once.  QLIN_FUSED_MAX_M overrides it
+// (measurement aid).
+int fused_momentum_max_m() {
+  static const int v = [] {
+    const char* e = getenv("QLIN_FUSED_MAX_M");
+    return e ? atoi(e) : kFusedMomentumMaxM;
+  }();
+  return v;
+}
+
 constexpr int kQuantSmemMax = 232448 - 1024;  // 227 KB per CTA, less room for the kernel's static shared memory
 
 size_t act_ws_bytes(const qlin_weights* w) {
@@ -424,7 +439,7 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   unsigned* cmax = static_cast<unsigned*>(act_ws);
   MomentumArgs mom{w->wmax_O, gamma, cmax + nO, M};
   const bool do_update = update && nO > 0;
-  const bool fused = do_update && M <= kFusedMomentumMaxM;
+  const bool fused = do_update && M <= fused_momentum_max_m();
   if (do_update && !fused) {
     const int grid = (M + kColmaxRows - 1) / kColmaxRows;
     cudaError_t e = launch_k(colmax_kernel, dim3(grid), dim3(256), size_t(nO) * 8, stream, X, M, K,
