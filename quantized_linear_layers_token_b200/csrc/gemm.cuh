@@ -168,7 +168,10 @@ struct GemmCfg {
   static constexpr int kReserve = 1024 + 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table, token scales
   static constexpr int kYStage = 16 * 128 * 2;                  // one 16-token x 128-channel fp16 chunk of Y
   static constexpr int kBudget = kSmemLimit - kReserve;
-  static constexpr int kXSlots = KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 ? 4 : 3));
+  // 256-token tiles: the INT8 format spends shared memory on activation
+  // slots (32 KiB each), the INT4 formats on packed-weight staging
+  static constexpr int kXSlots =
+      KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 || !kW4 ? 4 : 3));
   static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes - kRecvBytes - 2 * kYStage) / (KS * 16384);
   static constexpr int kASlots = kTA ? (BT <= 16 ? 3 : 4)
                                      : (kW4 ? (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)) : (kASlotsW8 > 8 ? 8 : kASlotsW8));
