@@ -92,6 +92,7 @@ struct GemmArgs {
   const uint16_t* rfold;    // g128 ratios r [K/128][N] fp16
   const uint16_t* wot;      // tiled W_O^T (16 KiB swizzled blocks of 128 channels x 64 outliers)
   const float* cscale;  // c_n [N]
+  float cmul;           // INT8 kernel: factor on c_n (1, or 1/16 for per-channel INT4 widened to 16 q)
   const float* a;       // a_m [M]
   uint16_t* Y;          // [M][N] fp16
   int32_t* acc_debug;   // [M][N] or null
@@ -287,6 +288,16 @@ struct Segment {
   int r0, r1;  // iterations [r0, r1) of the tile
 };
 
+// Dequantisation factor c'_n of output channel n: c_n / 16 for per-channel
+// INT4 (the operand holds 16 q), c_n for the other formats, times the INT8
+// kernel's factor (exact: 1 or 1/16) when it runs on widened INT4 weights.
+template <int FMT>
+__device__ __forceinline__ float chan_scale(const GemmArgs& g, int n) {
+  if (n >= g.N) return 0.f;
+  const float c = g.cscale[n];
+  return FMT == kFmtW4PC ? __fmul_rn(c, 0.0625f) : (FMT == kFmtW8 ? __fmul_rn(c, g.cmul) : c);
+}
+
 // Segments of one CTA, in order: a stream-K range of the flat iteration
 // space, or (cluster split-K) the same rank range of every cluster tile.
 // The fields come from the CTA plan staged in shared memory at start-up, so
@@ -383,6 +394,57 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int slots, int issued
     while (!mbar_try_wait_sleep(&full[s], static_cast<uint32_t>(t / slots) & 1u, 1000000u) &&
            globaltimer_ns() - t0 < QLIN_WAIT_NS) {
     }
+  }
+}
+
+// Prefill with INT4 weights: the packed blocks are widened once per call to
+// the INT8 operand layout (16 KiB blocks, 128-byte swizzle) -- the same
+// arithmetic as the converter warps (16 q for per-channel codes, the folded
+// FP16 requantisation for g128) -- and the INT8 kernel runs on them.  With
+// hundreds of token tiles per weight block this replaces a conversion per
+// token tile by one.  One CTA per 128 x 128 block, two 16-byte chunks per
+// thread.
+template <int FMT>
+__global__ void __launch_bounds__(256)
+widen_w4_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ rfold, int N, int kb,
+                uint8_t* __restrict__ out) {
+  griddep_launch_dependents();
+  const int blk = blockIdx.x;  // tn * kb + k
+  const int tn = blk / kb;
+  const int k = blk - tn * kb;
+  const uint8_t* src = codes + static_cast<size_t>(blk) * 8192;
+  uint8_t* dst = out + static_cast<size_t>(blk) * 16384;
+  uint4 w[2];
+  uint16_t rb[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int c = threadIdx.x + u * 256;
+    w[u] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+    const int n = tn * 128 + (c >> 2);
+    rb[u] = (FMT == kFmtW4G128 && n < N) ? rfold[static_cast<size_t>(k) * N + n] : static_cast<uint16_t>(0);
+  }
+  griddep_wait();  // the previous kernel in the stream may still read this workspace
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int c = threadIdx.x + u * 256;
+    const int row = c >> 2;
+    const int part = (c & 3) ^ ((row >> 1) & 3);  // packed chunks are swizzled by row pair
+    uint4 o0, o1;
+    if (FMT == kFmtW4PC) {
+      unpack_w4pc(w[u], o0, o1);
+    } else {
+      const __half2 r1 = __half2half2(__ushort_as_half(rb[u]));
+      const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
+      const uint2 a0 = requant_g128(w[u].x, r1, r16);
+      const uint2 a1 = requant_g128(w[u].y, r1, r16);
+      const uint2 a2 = requant_g128(w[u].z, r1, r16);
+      const uint2 a3 = requant_g128(w[u].w, r1, r16);
+      o0 = make_uint4(a0.x, a0.y, a1.x, a1.y);
+      o1 = make_uint4(a2.x, a2.y, a3.x, a3.y);
+    }
+    const int sw = row & 7;
+    *reinterpret_cast<uint4*>(dst + row * 128 + (((2 * part) ^ sw) << 4)) = o0;
+    *reinterpret_cast<uint4*>(dst + row * 128 + (((2 * part + 1) ^ sw) << 4)) = o1;
   }
 }
 
@@ -975,7 +1037,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         const bool has_comp = comp && sg.r1 == args.T && sg.r0 <= args.nk;
         const bool whole = sg.r0 == 0 && sg.r1 == args.T;
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * bcols);
-        const float cn = n < args.N ? (FMT == kFmtW4PC ? __fmul_rn(args.cscale[n], 0.0625f) : args.cscale[n]) : 0.f;
+        const float cn = chan_scale<FMT>(args, n);
         const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tile * static_cast<unsigned>(args.T) ? 1 : 0);
         int32_t* pacc = args.ws_acc + static_cast<size_t>(my_slot) * BT * 128;
         float* pcmp = args.ws_comp + static_cast<size_t>(my_slot) * BT * 128;
@@ -990,7 +1052,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           // the owner's scale factors, requested before the exchange
           {
             const int n_own = tn * C::kBN + crk * slice + (nl % slice);
-            if (n_own < args.N) cn_own = FMT == kFmtW4PC ? __fmul_rn(args.cscale[n_own], 0.0625f) : args.cscale[n_own];
+            cn_own = chan_scale<FMT>(args, n_own);
             if (nl < mvalid) a_own = args.a[m0 + nl];
           }
           const int q = nl / slice;
@@ -1202,15 +1264,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           const int wq = nl >> 5;
           const int n4 = tn * C::kBN + 4 * cg;
           const bool live = n4 < args.N;
-          float c4[4] = {0.f, 0.f, 0.f, 0.f};
-          if (live) {
-            const float4 cs = *reinterpret_cast<const float4*>(args.cscale + n4);
-            c4[0] = cs.x; c4[1] = cs.y; c4[2] = cs.z; c4[3] = cs.w;
-            if (FMT == kFmtW4PC) {
+          float c4[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) c4[i] = __fmul_rn(c4[i], 0.0625f);
-            }
-          }
+          for (int i = 0; i < 4; ++i) c4[i] = chan_scale<FMT>(args, n4 + i);
           int nctr = 0;
           for (int c = c_lo; c <= c_hi; ++c) nctr += bnd_s(c, sbnd, args) != bnd_s(c + 1, sbnd, args) ? 1 : 0;
           const int blocks = nctr + (comp ? 1 : 0);

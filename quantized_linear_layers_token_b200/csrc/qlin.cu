@@ -228,8 +228,19 @@ int pick_bt(int M) {
 // and for the launch).
 struct GemmPlan {
   int bt, tiles_n, tiles_m, kb, nk, nc, ncs, T, grid, split;
-  size_t u_off, acc_off, comp_off, cnt_off, total;
+  int widen;  // INT4 weights widened to INT8 once per call (prefill), then the INT8 kernel
+  size_t u_off, acc_off, comp_off, cnt_off, w8_off, total;
 };
+
+// From this many tokens the INT4 formats widen their weights once per call
+// and run the INT8 kernel (QLIN_WIDEN_MIN_M overrides it; 0 turns it off).
+int widen_min_m() {
+  static const int v = [] {
+    const char* e = getenv("QLIN_WIDEN_MIN_M");
+    return e ? atoi(e) : 1024;
+  }();
+  return v;
+}
 
 GemmPlan plan_gemm(int M, const qlin_weights* w) {
   GemmPlan p{};
@@ -259,6 +270,9 @@ GemmPlan plan_gemm(int M, const qlin_weights* w) {
   off = round_up(off + (p.split && w->n_outlier > 0 ? size_t(2) * p.grid * slot_bytes : 0), kAlign);
   p.cnt_off = off;
   off = round_up(off + (p.split ? size_t(p.grid) * 4 : 0), kAlign);
+  p.widen = (w->fmt != QLIN_W8_PERCHANNEL && p.bt == 256 && widen_min_m() > 0 && M >= widen_min_m()) ? 1 : 0;
+  p.w8_off = off;
+  off = round_up(off + (p.widen ? size_t(p.tiles_n) * p.kb * 16384 : 0), kAlign);
   p.total = off;
   return p;
 }
@@ -406,6 +420,20 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
   if (tiles * p.T >= (1LL << 31)) return fail(QLIN_ERR_SHAPE, "problem too large (%lld tile iterations)", tiles * p.T);
   for (int c = 0; c <= p.grid; ++c) args.bnd[c] = gemm_boundary(c, tiles, p.T, p.nk, p.grid, p.split);
   const uint16_t* U = reinterpret_cast<const uint16_t*>(gws + p.u_off);
+  args.cmul = 1.f;
+  if (p.widen) {
+    uint8_t* w8 = reinterpret_cast<uint8_t*>(gws + p.w8_off);
+    const unsigned nblk = static_cast<unsigned>(p.tiles_n) * static_cast<unsigned>(p.kb);
+    const uint8_t* codes = static_cast<const uint8_t*>(w->codes);
+    const uint16_t* rf = reinterpret_cast<const uint16_t*>(w->fold_ratio);
+    cudaError_t e = w->fmt == QLIN_W4_PERCHANNEL
+                        ? launch_k(widen_w4_kernel<kFmtW4PC>, dim3(nblk), dim3(256), 0, stream, codes, rf, w->N, p.kb, w8)
+                        : launch_k(widen_w4_kernel<kFmtW4G128>, dim3(nblk), dim3(256), 0, stream, codes, rf, w->N, p.kb, w8);
+    if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "widen_w4_kernel launch failed: %s", cudaGetErrorString(e));
+    args.codes = w8;
+    args.cmul = w->fmt == QLIN_W4_PERCHANNEL ? 0.0625f : 1.f;
+    return launch_gemm_fmt<kFmtW8>(p.bt, w, Xq, U, args, stream);
+  }
   switch (w->fmt) {
     case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC>(p.bt, w, Xq, U, args, stream);
     case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128>(p.bt, w, Xq, U, args, stream);

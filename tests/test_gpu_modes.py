@@ -1,5 +1,6 @@
 """The GEMM's work split is chosen per call (global stream-K, or cluster
-split-K with 2, 4 or 8 CTAs per tile) and kernels are chained with
+split-K with 2, 4 or 8 CTAs per tile), INT4 weights are widened ahead of
+the GEMM for large token counts, and kernels are chained with
 programmatic dependent launch.  The environment switches read once per
 process force each variant, so every one of them is checked against the
 oracle here: the exact INT32 accumulators of the split-K test and the
@@ -20,6 +21,8 @@ MODES = [
     {"QLIN_CLUSTER_CS": "4"},
     {"QLIN_CLUSTER_CS": "8"},
     {"QLIN_NO_PDL": "1"},       # plain stream-ordered launches
+    {"QLIN_WIDEN_MIN_M": "129"},  # INT4 weights widened once, INT8 kernel, from 129 tokens
+    {"QLIN_WIDEN_MIN_M": "0"},    # INT4 converters in the GEMM for every token count
 ]
 
 
