@@ -140,7 +140,11 @@ struct GemmCfg {
   // INT8: the four warps after the first three are the epilogue.
   static constexpr int kNCW = kW4 ? 8 : 4;          // arrivals on the converter barriers
   static constexpr int kEpiWarp0 = kW4 ? 3 + kNCW : 3;
-  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+  // INT8 with 256-token tiles (prefill): the single-buffered accumulator
+  // stalls the MMA while a tile drains, so two groups of four epilogue warps
+  // take alternate 16-token chunks of whole tiles.
+  static constexpr int kEpiGroups = (!kW4 && BT == 256) ? 2 : 1;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiGroups);
   // Small token tiles load the hi and lo compensation operands in one step
   // (one W_O^T block feeds both); large ones use two passes.
   static constexpr bool kCompFused = BT <= 64;
@@ -166,18 +170,20 @@ struct GemmCfg {
   static constexpr int kRecvComp = kCluster ? 64 * kRecvLd * 4 : 0;  // slice <= 64 channels (cs >= 2)
   static constexpr int kRecvBytes = kRecvMain + kRecvComp;
   static constexpr int kSmemLimit = 232448;          // 227 KB per CTA
-  static constexpr int kReserve = 1024 + 1024 + 1024 + 1024;  // alignment slack, barriers, boundary table, token scales
+  static constexpr int kReserve = 1024 + 1024 + 1024 + 2048;  // alignment slack, barriers, boundary table, token scales (x2)
   static constexpr int kYStage = 16 * 128 * 2;                  // one 16-token x 128-channel fp16 chunk of Y
   static constexpr int kBudget = kSmemLimit - kReserve;
   // 256-token tiles: the INT8 format spends shared memory on activation
   // slots (32 KiB each), the INT4 formats on packed-weight staging
   static constexpr int kXSlots =
       KS == 4 ? (FMT == kFmtW4G128 ? 3 : 4) : (BT <= 32 ? 8 : (BT <= 128 || !kW4 ? 4 : 3));
-  static constexpr int kASlotsW8 = (kBudget - kXSlots * kXBytes - kRecvBytes - 2 * kYStage) / (KS * 16384);
+  static constexpr int kASlotsW8 =
+      (kBudget - kXSlots * kXBytes - kRecvBytes - 2 * kEpiGroups * kYStage) / (KS * 16384);
   static constexpr int kASlots = kTA ? (BT <= 16 ? 3 : 4)
                                      : (kW4 ? (KS == 2 ? 3 : (BT <= 128 ? 4 : 3)) : (kASlotsW8 > 8 ? 8 : kASlotsW8));
   static constexpr int kStgSlotsFit =
-      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384 - kRecvBytes - 2 * kYStage) /
+      kW4 ? (kBudget - kASlots * kABytes - kXSlots * kXBytes - kCompSlots * 16384 - kRecvBytes -
+             2 * kEpiGroups * kYStage) /
                 kStgBytes
           : 0;
   static constexpr int kStgSlots = kStgSlotsFit > 16 ? 16 : kStgSlotsFit;
@@ -187,9 +193,9 @@ struct GemmCfg {
   static constexpr int kOffStg = kOffComp + kCompSlots * 16384;
   static constexpr int kOffRecv = kOffStg + kStgSlots * kStgBytes;
   static constexpr int kOffYst = kOffRecv + kRecvBytes;              // two Y staging chunks
-  static constexpr int kOffBar = kOffYst + 2 * kYStage;
+  static constexpr int kOffBar = kOffYst + 2 * kEpiGroups * kYStage;
   static constexpr int kOffBnd = kOffBar + 1024;     // stream-K boundary table (<= 256 entries)
-  static constexpr int kOffSa = kOffBnd + 1024;      // token scales a[m] of the tile being finished
+  static constexpr int kOffSa = kOffBnd + 1024;      // token scales a[m] of the tile being finished (per group)
   static constexpr int kSmemBytes = kReserve + kOffBar;
   static constexpr uint32_t kTxX = BT * 128;
   static constexpr uint32_t kTxU = (kCompFused ? 2 : 1) * BT * 128;
@@ -516,7 +522,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     } else if (lane < 26) {
       const int b = lane - 24;
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 128 * C::kEpiGroups);
       mbar_init(&cfull[b], 1);
       mbar_init(&cempty[b], 1);
     } else if (lane == 26) {
@@ -834,7 +840,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     const bool epi = warp >= C::kEpiWarp0;
     // The epilogue threads keep the boundary table in shared memory (read
     // after the epilogue's first named barrier).
-    if (epi && !cl)
+    if (epi && !cl && warp < C::kEpiWarp0 + 4)
       for (int i = threadIdx.x - 32 * C::kEpiWarp0; i < args.grid; i += 128) sbnd[i] = args.bnd[i];
     // ------------------------------------------------------------ converters
     if (C::kTA && !epi) {
@@ -1009,6 +1015,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     if (epi) {
       const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
       const int nl = quad * 32 + lane;
+      const int grp = (warp - C::kEpiWarp0) >> 2;  // epilogue group (two for 256-token INT8 tiles)
+      const int gbar = 1 + grp;                    // its named barrier
       griddep_wait();  // a[] comes from the previous kernel
       // Partially covered tiles (at most the first and the last segment):
       // their counters and the finishing work run after every segment's
@@ -1020,7 +1028,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       Segment sg;
       int seg = 0;
       int ycnt = 0;  // Y chunks handed to TMA stores (two staging buffers alternate)
-      float* sa_t = reinterpret_cast<float*>(smem + C::kOffSa);
+      float* sa_t = reinterpret_cast<float*>(smem + C::kOffSa + grp * 1024);
       while (seg_next(gen, sg)) {
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
@@ -1036,6 +1044,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         const bool has_main = sg.r0 < args.nk;
         const bool has_comp = comp && sg.r1 == args.T && sg.r0 <= args.nk;
         const bool whole = sg.r0 == 0 && sg.r1 == args.T;
+        if (grp > 0 && (cl || !whole)) {
+          // the second group only shares whole tiles
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+          ++seg;
+          continue;
+        }
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * bcols);
         const float cn = chan_scale<FMT>(args, n);
         const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tile * static_cast<unsigned>(args.T) ? 1 : 0);
@@ -1065,15 +1080,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
         }
         if (!cl && whole) {
-          // token scales of the tile, staged once
-          named_bar_sync(1, 128);
+          // token scales of the tile, staged once per group
+          named_bar_sync(gbar, 128);
           for (int j = nl; j < BT; j += 128) sa_t[j] = j < mvalid ? args.a[m0 + j] : 0.f;
-          named_bar_sync(1, 128);
+          named_bar_sync(gbar, 128);
           if (seg == 0 && nl == 0) QLIN_STAMP(16);
         }
 #pragma unroll 1
         for (int c0 = 0; c0 < BT; c0 += 16) {
           if (!cl && c0 >= mvalid) break;
+          if (C::kEpiGroups > 1 && whole && ((c0 >> 4) & 1) != grp) continue;  // the other group's chunk
           uint32_t acc[16], cmp[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) { acc[j] = 0u; cmp[j] = 0u; }
@@ -1100,7 +1116,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             // the next write of a buffer comes after the barrier that
             // follows every thread's reads of it.
             const int b = ycnt & 1;
-            uint16_t* ys = reinterpret_cast<uint16_t*>(smem + C::kOffYst + b * C::kYStage);
+            uint16_t* ys = reinterpret_cast<uint16_t*>(smem + C::kOffYst + (grp * 2 + b) * C::kYStage);
             // the 16 token scales into registers before any staging store
             // (the compiler cannot prove the two shared arrays disjoint, so
             // interleaved loads would each wait for the previous store)
@@ -1124,7 +1140,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                 if (c0 + j < mvalid && n < args.N)
                   args.acc_debug[static_cast<size_t>(m0 + c0 + j) * args.N + n] = static_cast<int32_t>(acc[j]);
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(gbar, 128);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int idx = nl + h * 128;  // 16 rows x 16 segments of 8 channels

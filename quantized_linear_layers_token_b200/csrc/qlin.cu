@@ -255,7 +255,10 @@ GemmPlan plan_gemm(int M, const qlin_weights* w) {
   p.T = p.nk + p.nc;
   const int sms = sm_count();
   const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
-  p.split = tiles < 4LL * sms ? 1 : 0;
+  // Split tiles (stream-K or cluster split-K) when whole tiles would leave
+  // SMs idle or badly balanced.  Token tiles of 128/256 have partials of
+  // 64-128 KiB, so they split only when there are fewer tiles than SMs.
+  p.split = tiles < (p.bt >= 128 ? 1LL : 4LL) * sms ? 1 : 0;
   const long long units = p.split ? tiles * p.T : tiles;
   const int cap = sms < kMaxGrid ? sms : kMaxGrid;
   p.grid = static_cast<int>(units < cap ? units : cap);
