@@ -65,6 +65,8 @@ def test_weights_bytes_and_bind(q):
     (512, 128, 7, 0, "QLIN_ERR_ARG"),      # unknown format
     (512, 128, 0, -1, "QLIN_ERR_ARG"),
     (512, 128, 0, 600, "QLIN_ERR_SHAPE"),  # more outliers than channels
+    (65568, 128, 0, 0, "QLIN_ERR_SHAPE"),  # K above the supported 65536
+    (8192, 128, 0, 4097, "QLIN_ERR_SHAPE"),  # more than 4096 outlier channels
     (0, 128, 0, 0, "QLIN_ERR_ARG"),
 ])
 def test_shape_validation(q, K, N, fmt, nO, status):

@@ -150,6 +150,18 @@ def test_shapes(q, oracle, fmt, M, K, N, nO):
     check_all(oracle, L, g, s0, 0.9)
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_maximum_k_and_outliers(q, oracle, fmt):
+    # the largest supported layer depth with the largest outlier set: the
+    # quantization row (128 KiB) and outlier tables fill the shared memory,
+    # 512 K-blocks stream through the rings, 64 compensation slices
+    L = case(fmt, 3, 65536, 128, 4096)
+    rng = np.random.default_rng(65536)
+    s0 = rng.uniform(1.0, 3.0, 4096).astype(np.float32)
+    g = run_gpu(q, L, s0, 0.9)
+    check_all(oracle, L, g, s0, 0.9)
+
+
 @pytest.mark.parametrize("fmt", [synth.W4_PERCHANNEL, synth.W8_PERCHANNEL])
 def test_ragged_k(q, oracle, fmt):
     # K a multiple of 32 but not of 128: the last K-step is zero-filled by TMA
