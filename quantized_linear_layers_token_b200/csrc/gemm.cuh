@@ -1032,10 +1032,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       while (seg_next(gen, sg)) {
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
-        bool ok = mbar_wait(&acc_full[buf], static_cast<uint32_t>(use) & 1u, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
-        if (seg == 0 && nl == 0) QLIN_STAMP(10);
-        tc_fence_after();
+        // everything that depends only on the tile is read before waiting for
+        // its accumulator (the loads complete behind the mainloop)
         const int tn = static_cast<int>(sg.tile % args.tiles_n);
         const int tm = static_cast<int>(sg.tile / args.tiles_n);
         const int n = tn * C::kBN + nl;
@@ -1044,6 +1042,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         const bool has_main = sg.r0 < args.nk;
         const bool has_comp = comp && sg.r1 == args.T && sg.r0 <= args.nk;
         const bool whole = sg.r0 == 0 && sg.r1 == args.T;
+        const float cn = chan_scale<FMT>(args, n);
+        float a_own = 0.f, cn_own = 0.f;  // cluster split-K: the owned slice's scales
+        if (cl) {
+          cn_own = chan_scale<FMT>(args, tn * C::kBN + crk * slice + (nl % slice));
+          if (nl < mvalid) a_own = args.a[m0 + nl];
+        }
+        bool ok = mbar_wait(&acc_full[buf], static_cast<uint32_t>(use) & 1u, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (seg == 0 && nl == 0) QLIN_STAMP(10);
+        tc_fence_after();
         if (grp > 0 && (cl || !whole)) {
           // the second group only shares whole tiles
           tc_fence_before();
@@ -1052,23 +1060,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           continue;
         }
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * bcols);
-        const float cn = chan_scale<FMT>(args, n);
         const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tile * static_cast<unsigned>(args.T) ? 1 : 0);
         int32_t* pacc = args.ws_acc + static_cast<size_t>(my_slot) * BT * 128;
         float* pcmp = args.ws_comp + static_cast<size_t>(my_slot) * BT * 128;
         // cluster split-K: channel nl goes to owner rank nl / slice
         uint32_t r_main = 0, r_comp = 0, r_bar = 0;
-        float a_own = 0.f, cn_own = 0.f;
         if (cl) {
           if (!cl_waited) {
             cluster_wait();
             cl_waited = true;
-          }
-          // the owner's scale factors, requested before the exchange
-          {
-            const int n_own = tn * C::kBN + crk * slice + (nl % slice);
-            cn_own = chan_scale<FMT>(args, n_own);
-            if (nl < mvalid) a_own = args.a[m0 + nl];
           }
           const int q = nl / slice;
           const int c = nl - q * slice;

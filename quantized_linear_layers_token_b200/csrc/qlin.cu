@@ -205,6 +205,16 @@ int sm_count() {
   return cached[dev];
 }
 
+// CTAs a GEMM may use at most (QLIN_MAX_CTAS, measurement aid; default all SMs).
+int gemm_cta_cap() {
+  static const int v = [] {
+    const char* e = getenv("QLIN_MAX_CTAS");
+    return e ? atoi(e) : 0;
+  }();
+  const int sms = sm_count();
+  return (v > 0 && v < sms) ? v : sms;
+}
+
 // QLIN_MAX_BT=128 caps the token tile (measurement aid).
 int max_bt() {
   static const int v = [] {
@@ -253,7 +263,7 @@ GemmPlan plan_gemm(int M, const qlin_weights* w) {
   p.ncs = w->n_outlier > 0 ? (w->n_outlier + 63) / 64 : 0;
   p.nc = (p.bt <= 64) ? p.ncs : 2 * p.ncs;
   p.T = p.nk + p.nc;
-  const int sms = sm_count();
+  const int sms = gemm_cta_cap();
   const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
   // Split tiles (stream-K or cluster split-K) when whole tiles would leave
   // SMs idle or badly balanced.  Token tiles of 128/256 have partials of
@@ -350,7 +360,8 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
         }
         max_clusters[cs] = n;
       }
-      const int ncl = static_cast<int>(max_clusters[cs] < tiles ? max_clusters[cs] : tiles);
+      int ncl = static_cast<int>(max_clusters[cs] < tiles ? max_clusters[cs] : tiles);
+      if (ncl * cs > gemm_cta_cap()) ncl = gemm_cta_cap() / cs;
       if (ncl < 1) continue;
       double cost = static_cast<double>((tiles + ncl - 1) / ncl) * (span + xchg);
       if (forced) cost = forced == cs ? -1.0 : 1e30;
