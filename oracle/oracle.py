@@ -70,6 +70,8 @@ def _declare(L):
     L.oq_outlier_wmax.restype = None
     L.oq_momentum_update.argtypes = [P, I, I, P, I, P, F, P]
     L.oq_momentum_update.restype = None
+    L.oq_backward_dx.argtypes = [P, I, I, I, P, P, P, P, I, P, P]
+    L.oq_backward_dx.restype = None
     L.oq_quant_act.argtypes = [P, I, I, P, I, P, P, P, P]
     L.oq_quant_act.restype = None
     L.oq_int_gemm.argtypes = [P, P, I, I, I, P]
@@ -290,6 +292,23 @@ def gptq_quantize(X: np.ndarray, w: np.ndarray, scale: float, qmax: int):
 FMT_W4_PERCHANNEL = 0
 FMT_W4_G128 = 1
 FMT_W8_PERCHANNEL = 2
+
+
+def backward_dx(dY_bits: np.ndarray, W_bits: np.ndarray, packed: dict, s: np.ndarray) -> np.ndarray:
+    """Input gradient under the straight-through estimator, fp64 [M][K]:
+    dX = (dY W_eff^T) / s with W_eff the dequantized weights plus the
+    compensation rows (s_i - 1) W[O_i, :]."""
+    dY_bits = _c(dY_bits, np.uint16)
+    W_bits = _c(W_bits, np.uint16)
+    M, N = dY_bits.shape
+    K = packed["K"]
+    B = _c(packed["B"], np.int8)
+    cs = _c(packed["cscale"], np.float32)
+    O = _c(packed["O"], np.int32)
+    s = _c(s if len(O) else np.zeros(1), np.float32)
+    dX = np.zeros((M, K), np.float64)
+    lib().oq_backward_dx(_p(dY_bits), M, N, K, _p(B), _p(cs), _p(W_bits), _p(O), len(O), _p(s), _p(dX))
+    return dX
 
 
 def pack_layer(W_bits: np.ndarray, O: np.ndarray, fmt: int) -> dict:

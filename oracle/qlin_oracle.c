@@ -366,6 +366,44 @@ OQ_EXPORT void oq_dequant(const int64_t* acc, const float* a, const float* cscal
 }
 
 /* ------------------------------------------------------------------------ */
+/* Input gradient for fine-tuning ([Quaff] 损失函数 / 训练策略: back-          */
+/* propagation through the standard straight-through estimator).             */
+/* Reading: under the estimator the quantizers are identities for the        */
+/* gradient, so the layer is the linear map X -> (X / s) W_eff, where W_eff   */
+/* holds the dequantized weights cscale_n * B[k][n] and, on the outlier rows  */
+/* k = O_i, also the compensation term (s_i - 1) * W[O_i][n] of the          */
+/* decoupled formula.  Its input gradient is                                 */
+/*   dX[m][k] = ( sum_n dY[m][n] * W_eff[k][n] ) / s_k,   s_k = 1 off O.      */
+/* fp64 throughout; dY is fp16 bits [M][N], B is the INT8 operand [K][N].     */
+/* ------------------------------------------------------------------------ */
+
+OQ_EXPORT void oq_backward_dx(const uint16_t* dY, int M, int N, int K, const int8_t* B, const float* cscale,
+                              const uint16_t* W, const int32_t* O, int nO, const float* s, double* dX) {
+  int* slot = (int*)malloc(sizeof(int) * (size_t)(K > 0 ? K : 1));
+  for (int k = 0; k < K; ++k) slot[k] = -1;
+  for (int i = 0; i < nO; ++i) slot[O[i]] = i;
+  double* dy = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+  for (int m = 0; m < M; ++m) {
+    for (int n = 0; n < N; ++n) dy[n] = oq_half_to_double(dY[(size_t)m * N + n]);
+    for (int k = 0; k < K; ++k) {
+      double g = 0.0;
+      for (int n = 0; n < N; ++n) g += dy[n] * ((double)cscale[n] * (double)B[(size_t)k * N + n]);
+      double sk = 1.0;
+      if (slot[k] >= 0) {
+        const int i = slot[k];
+        sk = (double)s[i];
+        double c = 0.0;
+        for (int n = 0; n < N; ++n) c += dy[n] * oq_half_to_double(W[(size_t)O[i] * N + n]);
+        g += (sk - 1.0) * c;
+      }
+      dX[(size_t)m * K + k] = g / sk;
+    }
+  }
+  free(dy);
+  free(slot);
+}
+
+/* ------------------------------------------------------------------------ */
 /* FastFP16toINT8 ([QQQ] FastFP16toINT8优化): add 128 to move the value into  */
 /* [0, 255], add 1024 so the eight bits of the UINT8 land in the low bits of */
 /* the FP16 significand, then read them out of the bit pattern.              */
