@@ -247,6 +247,28 @@ QLIN_API qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weigh
                          float gamma, int32_t update_momentum, uint16_t* Y, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* Input gradient of the layer for fine-tuning (Quaff notes, 损失函数 /
+ * 训练策略: the quantizers are passed by the standard straight-through
+ * estimator, so the gradient is that of the decoupled layer of 解耦 WAQ 公式
+ * before rounding):
+ *   dX[m][k]     = sum_n dY[m][n] Weff[k][n]
+ *   Weff[k][n]   = c'_n B[k][n]                                 k not in O
+ *   Weff[O_i][n] = (c'_n B[O_i][n] + (s_i - 1) W_O[i][n]) / s_i
+ * with B, c'_n the forward's INT8 operand and channel factor (16 q and c_n/16
+ * for per-channel INT4, the requantized q8 and c_n for g128, q and c_n for
+ * INT8) and W_O the fp16 outlier rows kept in `W_Ot`.  The frozen quantized
+ * weights get no gradient.
+ *   dY  fp16 [M][N] row-major, device.
+ *   s   fp32 [n_outlier], device: the scales of the forward pass whose
+ *       gradient this is (ignored and may be NULL when n_outlier = 0).
+ *   dX  fp16 [M][K] row-major, device, fully overwritten.
+ * Arithmetic: Weff is rounded to fp16 (the outlier rows after blending in
+ * fp32), products are summed in fp32 on the tensor cores, dX is rounded to
+ * fp16 once.  No workspace.  M = 0 is a no-op; M above 65535 * 128 returns
+ * QLIN_ERR_SHAPE; pointers must be 16-byte aligned (QLIN_ERR_ALIGN). */
+QLIN_API qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t M, const float* s,
+                                      uint16_t* dX, void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word that
  * kernels set when a bounded wait gives up: QLIN_ERR_TIMEOUT if it was set,
  * QLIN_ERR_CUDA if the stream reported an error, else QLIN_OK. */

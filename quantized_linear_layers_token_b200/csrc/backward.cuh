@@ -1,0 +1,403 @@
+// backward.cuh -- input gradient of the outlier-decoupled quantized linear
+// layer under the straight-through estimator.
+//
+// Quaff notes (损失函数 / 训练策略): fine-tuning back-propagates through the
+// quantizers with the standard straight-through estimator, so the gradient
+// that reaches X is the transpose of the linear map the forward evaluates
+// before rounding (解耦 WAQ 公式):
+//     Y = X_hat W_deq + X_hat[:, O] diag(s_O - 1) W_O,
+//     X_hat = X with the outlier columns divided by s,  W_deq[k][n] = c'_n B[k][n],
+// which is
+//     dX[m][k]     = sum_n dY[m][n] Weff[k][n]
+//     Weff[k][n]   = c'_n B[k][n]                                     (k not in O)
+//     Weff[O_i][n] = (c'_n B[O_i][n] + (s_i - 1) W[O_i][n]) / s_i.
+// B and c'_n are the forward's own INT8 operand and channel factor: 16 q with
+// c_n / 16 (per-channel INT4), the folded requantisation q8 with c_n (g128),
+// q with c_n (INT8).
+//
+// One CTA computes a 128-token x 256-input tile of dX on the tensor cores
+// (kind::f16, fp32 accumulators in TMEM), reducing over the N output
+// channels 64 at a time:
+//   A = dY tile (128 tokens x 64 channels, K-major), loaded by TMA (warp 0);
+//   B = Weff tile (256 inputs x 64 channels), written to shared memory as fp16
+//       by eight converter warps from the packed codes that warp 2 copies in.
+//       The codes of a channel row are contiguous along the inputs, so the
+//       operand is stored MN-major (inputs contiguous, 128-byte swizzle) and
+//       the conversion needs no transpose;
+//   warp 1 issues four 128 x 256 x 16 MMAs per step.
+// The outlier rows are blended into B after each step's conversion; the
+// converter warps then read the accumulators back and store fp16 dX rows.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace qlin {
+
+struct BwdArgs {
+  const uint8_t* codes;   // tiled packed codes (the weights' own layout)
+  const uint16_t* rfold;  // g128 ratios r [K/128][N] fp16
+  const uint16_t* wot;    // tiled W_O^T (16 KiB swizzled blocks of 128 channels x 64 outliers)
+  const float* cscale;    // c_n [N]
+  const int32_t* oidx;    // O [nO], strictly increasing
+  const float* s;         // s [nO]
+  uint16_t* dX;           // [M][K] fp16
+  int M, N, K, nO;
+  int kbs;     // 128-input code blocks per channel tile (ceil(K / 128))
+  int nib;     // 64-outlier blocks of W_O^T per channel tile (ceil(nO / 64))
+  int nsteps;  // 64-channel reduction steps (ceil(N / 64))
+};
+
+template <int FMT>
+struct BwdCfg {
+  static constexpr bool kW4 = FMT != kFmtW8;
+  static constexpr int kRowBytes = kW4 ? 64 : 128;  // code bytes of one channel row of a 128-input block
+  static constexpr int kBlkBytes = 128 * kRowBytes;  // one code block
+  static constexpr int kStgBlk = 64 * kRowBytes;     // the 64 rows of one step
+  static constexpr int kStgRatio = 2 * kStgBlk;      // g128: the step's ratios, 2 x 64 fp16
+  static constexpr int kStgBytes = 2 * kStgBlk + (FMT == kFmtW4G128 ? 256 : 0);
+  static constexpr int kASlots = 4;               // dY tiles
+  static constexpr int kBSlots = 3;               // Weff tiles
+  static constexpr int kLSlots = kW4 ? 4 : 3;     // code staging
+  static constexpr int kABytes = 128 * 64 * 2;    // 16 KiB
+  static constexpr int kBBytes = 256 * 64 * 2;    // 32 KiB
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kASlots * kABytes;
+  static constexpr int kOffStg = kOffB + kBSlots * kBBytes;
+  static constexpr int kOffOut = (kOffStg + kLSlots * kStgBytes + 15) / 16 * 16;
+  static constexpr int kMaxOut = 256;             // outliers among 256 inputs, at most
+  static constexpr int kOffBar = kOffOut + kMaxOut * 16;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + slack to 1024-align the base
+  static constexpr int kConvWarps = 8;
+  static constexpr int kThreads = 32 * (3 + kConvWarps);
+  static_assert(kSmemBytes <= 232448, "backward tile does not fit in shared memory");
+};
+
+// c'_n of the forward's INT8 operand (0 beyond N).
+template <int FMT>
+__device__ __forceinline__ float bwd_chan_scale(const BwdArgs& g, int n) {
+  if (n >= g.N) return 0.f;
+  const float c = g.cscale[n];
+  return FMT == kFmtW4PC ? __fmul_rn(c, 0.0625f) : c;
+}
+
+// Four INT8 lanes -> two fp16 pairs times c (exact int8 -> fp16 through the
+// significand of 1024, one rounding in the product).
+__device__ __forceinline__ void i8x4_scale_h2(uint32_t w, __half2 c2, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;  // q + 128 per byte
+  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));  // 1152
+  const __half2 f0 = __hsub2(u32_as_h2(prmt(u, 0x64646464u, 0x4140u)), bias);
+  const __half2 f1 = __hsub2(u32_as_h2(prmt(u, 0x64646464u, 0x4342u)), bias);
+  lo = h2_as_u32(__hmul2(f0, c2));
+  hi = h2_as_u32(__hmul2(f1, c2));
+}
+
+// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
+// atoms of 64 fp16 along MN x 8 rows along K (1 KiB), `lbo` bytes between
+// atoms along MN and `sbo` bytes between 8-row groups along K.
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(lbo >> 4) << 16;
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// First index i in [0, n) with a[i] >= v (n if none).
+__device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a + mid) < v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// B tile layout: 8-channel group g (K) x 64-input atom a (MN), atom (g, a) at
+// (4 g + a) KiB; within an atom, channel row (n % 8) at 128 (n % 8) and the
+// 16-byte chunk of inputs 8c..8c+7 at chunk c ^ (n % 8).
+constexpr uint32_t kBwdLbo = 1024;  // next 64 inputs
+constexpr uint32_t kBwdSbo = 4096;  // next 8 channels
+
+template <int FMT>
+__global__ void __launch_bounds__(BwdCfg<FMT>::kThreads, 1)
+backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ BwdArgs args) {
+  using C = BwdCfg<FMT>;
+  constexpr int AS = C::kASlots, BS = C::kBSlots, LS = C::kLSlots;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* afull = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* aempty = afull + AS;
+  uint64_t* bfull = aempty + AS;
+  uint64_t* bempty = bfull + BS;
+  uint64_t* sfull = bempty + BS;
+  uint64_t* sempty = sfull + LS;
+  uint64_t* acc_full = sempty + LS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float4* outl = reinterpret_cast<float4*>(smem + C::kOffOut);  // {input - k0, i, s_i - 1, 1 / s_i}
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int k0 = blockIdx.x * 256;
+  const int m0 = blockIdx.y * 128;
+  const int nsteps = args.nsteps;
+  const int nb = (2 * static_cast<int>(blockIdx.x) + 1 < args.kbs) ? 2 : 1;  // code blocks in this input tile
+
+  if (warp == 0) {
+    if (lane < AS) {
+      mbar_init(&afull[lane], 1);
+      mbar_init(&aempty[lane], 1);
+    } else if (lane >= 8 && lane < 8 + BS) {
+      mbar_init(&bfull[lane - 8], C::kConvWarps);
+      mbar_init(&bempty[lane - 8], 1);
+    } else if (lane >= 16 && lane < 16 + LS) {
+      mbar_init(&sfull[lane - 16], 1);
+      mbar_init(&sempty[lane - 16], C::kConvWarps);
+    } else if (lane == 24) {
+      mbar_init(acc_full, 1);
+      *abort_flag = 0;
+    }
+    fence_barrier_init();
+    if (lane == 0) tma_prefetch_desc(&tmDY);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- dY producer
+    if (lane == 0) {
+      griddep_wait();  // dY comes from the previous kernel
+      int issued = 0;
+      for (int j = 0; j < nsteps; ++j) {
+        const int a = j % AS;
+        if (j >= AS && !mbar_wait(&aempty[a], static_cast<uint32_t>(j / AS - 1) & 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(&afull[a], C::kABytes);
+        tma_load_2d(smem + C::kOffA + a * C::kABytes, &tmDY, &afull[a], j * 64, m0);
+        ++issued;
+      }
+      drain_ring(afull, AS, issued);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(128, 256) | (1u << 16);  // B MN-major
+      for (int j = 0; j < nsteps; ++j) {
+        const int a = j % AS;
+        const int b = j % BS;
+        if (!mbar_wait(&afull[a], static_cast<uint32_t>(j / AS) & 1u, abort_flag)) break;
+        if (!mbar_wait(&bfull[b], static_cast<uint32_t>(j / BS) & 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t abase = smem_u32(smem + C::kOffA + a * C::kABytes);
+        const uint32_t bbase = smem_u32(smem + C::kOffB + b * C::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem, sdesc_k_sw128(abase + kk * 32), sdesc_mn_sw128(bbase + kk * 2 * kBwdSbo, kBwdLbo, kBwdSbo),
+                  idesc, (j | kk) != 0 ? 1u : 0u);
+        mma_commit(&aempty[a]);
+        mma_commit(&bempty[b]);
+      }
+      // every MMA issued so far (all of them, or those before an abort)
+      mma_commit(acc_full);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait_sleep(acc_full, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------ code producer
+    if (lane == 0) {
+      int issued = 0;
+      const int kb0 = 2 * static_cast<int>(blockIdx.x);
+      for (int j = 0; j < nsteps; ++j) {
+        const int ls = j % LS;
+        if (j >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(j / LS - 1) & 1u, abort_flag)) break;
+        const int n0 = j * 64;
+        const int tn = n0 >> 7;
+        const int r0 = n0 & 127;
+        const uint32_t rbytes = FMT == kFmtW4G128 ? static_cast<uint32_t>(min(64, args.N - n0) * 2) : 0u;
+        mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nb) * (C::kStgBlk + rbytes));
+        unsigned char* dst = smem + C::kOffStg + ls * C::kStgBytes;
+        for (int b = 0; b < nb; ++b) {
+          const size_t blk = static_cast<size_t>(tn) * args.kbs + kb0 + b;
+          bulk_load(dst + b * C::kStgBlk, args.codes + blk * C::kBlkBytes + r0 * C::kRowBytes, C::kStgBlk, &sfull[ls]);
+          if (FMT == kFmtW4G128)
+            bulk_load(dst + C::kStgRatio + b * 128, args.rfold + static_cast<size_t>(kb0 + b) * args.N + n0, rbytes,
+                      &sfull[ls]);
+        }
+        ++issued;
+      }
+      drain_ring(sfull, LS, issued);
+    }
+  } else {
+    // ------------------------------------------- converters, then epilogue
+    const int cw = warp - 3;             // 0..7
+    const int ctid = threadIdx.x - 96;   // 0..255
+    griddep_wait();                      // s comes from the forward
+    int nout = 0;
+    if (args.nO > 0) {
+      const int lo = lower_bound_i32(args.oidx, args.nO, k0);
+      nout = lower_bound_i32(args.oidx, args.nO, k0 + 256) - lo;
+      if (ctid < nout) {
+        const int i = lo + ctid;
+        const float sv = args.s[i];
+        outl[ctid] = make_float4(__int_as_float(__ldg(args.oidx + i) - k0), __int_as_float(i), __fsub_rn(sv, 1.f),
+                                 __frcp_rn(sv));
+      }
+    }
+    named_bar_sync(1, 32 * C::kConvWarps);
+
+    const int nl = (cw & 1) * 32 + lane;  // channel row of the step
+    const int cq = cw >> 1;               // quarter of the row's inputs
+    const int sw = nl & 7;
+    // After a failed wait the loop keeps running, with no work, so that
+    // every converter warp reaches every named barrier.
+    bool ok = true;
+    for (int j = 0; j < nsteps; ++j) {
+      const int ls = j % LS;
+      const int b = j % BS;
+      if (ok) ok = mbar_wait(&sfull[ls], static_cast<uint32_t>(j / LS) & 1u, abort_flag);
+      if (ok && j >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(j / BS - 1) & 1u, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (nout > 0) named_bar_sync(1, 32 * C::kConvWarps);
+        continue;
+      }
+      const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
+      unsigned char* bt = smem + C::kOffB + b * C::kBBytes;
+      unsigned char* brow = bt + (nl >> 3) * kBwdSbo + sw * 128;
+      const __half2 c2 = __float2half2_rn(bwd_chan_scale<FMT>(args, j * 64 + nl));
+      if (FMT == kFmtW8) {
+        // 4 chunks of 16 inputs: inputs 64 cq .. 64 cq + 63
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int cc = cq * 4 + t;
+          const int blk = cc >> 3;
+          const int c = cc & 7;
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (blk < nb) w = *reinterpret_cast<const uint4*>(stg + blk * C::kStgBlk + nl * 128 + ((c ^ sw) << 4));
+          uint4 h0, h1;
+          i8x4_scale_h2(w.x, c2, h0.x, h0.y);
+          i8x4_scale_h2(w.y, c2, h0.z, h0.w);
+          i8x4_scale_h2(w.z, c2, h1.x, h1.y);
+          i8x4_scale_h2(w.w, c2, h1.z, h1.w);
+          const int kl = 16 * cc;  // first input of the chunk within the tile
+          unsigned char* atom = brow + (kl >> 6) * kBwdLbo;
+          const int ch = (kl & 63) >> 3;
+          *reinterpret_cast<uint4*>(atom + ((ch ^ sw) << 4)) = h0;
+          *reinterpret_cast<uint4*>(atom + (((ch + 1) ^ sw) << 4)) = h1;
+        }
+      } else {
+        // 2 chunks of 32 inputs: inputs 64 cq .. 64 cq + 63
+        const int blk = cq >> 1;  // both chunks lie in one code block
+        __half2 r1 = __half2half2(__ushort_as_half(static_cast<unsigned short>(0)));
+        __half2 r16 = r1;
+        if (FMT == kFmtW4G128 && blk < nb) {  // absent block: r = 0 makes every code 0
+          const uint16_t rbits = reinterpret_cast<const uint16_t*>(stg + C::kStgRatio + blk * 128)[nl];
+          r1 = __half2half2(__ushort_as_half(rbits));
+          r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
+        }
+        const int rsw = (nl >> 1) & 3;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int c = (cq & 1) * 2 + t;  // 32-input chunk within the block
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (blk < nb) w = *reinterpret_cast<const uint4*>(stg + blk * C::kStgBlk + nl * 64 + ((c ^ rsw) << 4));
+          uint32_t q8[8];  // INT8 lanes of inputs 4e .. 4e + 3 of the chunk
+          if (FMT == kFmtW4PC) {
+            uint4 o0, o1;
+            unpack_w4pc(w, o0, o1);
+            q8[0] = o0.x; q8[1] = o0.y; q8[2] = o0.z; q8[3] = o0.w;
+            q8[4] = o1.x; q8[5] = o1.y; q8[6] = o1.z; q8[7] = o1.w;
+          } else {
+            const uint2 a0 = requant_g128(w.x, r1, r16);
+            const uint2 a1 = requant_g128(w.y, r1, r16);
+            const uint2 a2 = requant_g128(w.z, r1, r16);
+            const uint2 a3 = requant_g128(w.w, r1, r16);
+            q8[0] = a0.x; q8[1] = a0.y; q8[2] = a1.x; q8[3] = a1.y;
+            q8[4] = a2.x; q8[5] = a2.y; q8[6] = a3.x; q8[7] = a3.y;
+          }
+          const int kl = blk * 128 + 32 * c;
+          unsigned char* atom = brow + (kl >> 6) * kBwdLbo;
+          const int ch0 = (kl & 63) >> 3;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 h;
+            i8x4_scale_h2(q8[2 * e], c2, h.x, h.y);
+            i8x4_scale_h2(q8[2 * e + 1], c2, h.z, h.w);
+            *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[ls]);  // staging slot consumed
+      if (nout > 0) {
+        // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i
+        named_bar_sync(1, 32 * C::kConvWarps);
+        for (int t = ctid; t < nout * 64; t += 32 * C::kConvWarps) {
+          const float4 o = outl[t >> 6];
+          const int q = t & 63;
+          const int kl = __float_as_int(o.x);
+          const int i = __float_as_int(o.y);
+          __half* p = reinterpret_cast<__half*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
+                                                ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
+          const int ng = j * 64 + q;
+          const int r = ng & 127;
+          const size_t wblk = static_cast<size_t>(ng >> 7) * args.nib + (i >> 6);
+          const uint16_t wbits =
+              __ldg(args.wot + wblk * 8192 + r * 64 + ((((i & 63) >> 3) ^ (r & 7)) << 3) + (i & 7));
+          const float v = __fmul_rn(__fmaf_rn(o.z, __half2float(__ushort_as_half(wbits)), __half2float(*p)), o.w);
+          *p = __float2half_rn(v);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bfull[b]);
+    }
+
+    // epilogue: TMEM lane = token, column = input
+    const bool got = ok && mbar_wait(acc_full, 0u, abort_flag);
+    if (__all_sync(0xffffffffu, got && *abort_flag == 0)) {
+      tc_fence_after();
+      const int qd = warp & 3;  // TMEM lane quadrant of this warp
+      const int half = cw >> 2;
+      const int m = m0 + qd * 32 + lane;
+#pragma unroll 1
+      for (int jj = 0; jj < 4; ++jj) {
+        const int col = half * 128 + jj * 32;
+        uint32_t v0[16], v1[16];
+        const uint32_t ta = tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(col);
+        tmem_ld16(ta, v0);
+        tmem_ld16(ta + 16, v1);
+        tmem_ld_wait();
+        const int k = k0 + col;
+        if (m < args.M && k < args.K) {
+          uint32_t hw[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            hw[e] = h2_as_u32(__floats2half2_rn(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1])));
+            hw[8 + e] = h2_as_u32(__floats2half2_rn(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1])));
+          }
+          uint4* dst = reinterpret_cast<uint4*>(args.dX + static_cast<size_t>(m) * args.K + k);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(hw[4 * e], hw[4 * e + 1], hw[4 * e + 2], hw[4 * e + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace qlin

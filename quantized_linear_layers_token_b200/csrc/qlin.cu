@@ -13,6 +13,7 @@
 #include "qlin.h"
 #include "act_quant.cuh"
 #include "gemm.cuh"
+#include "backward.cuh"
 #include "pack.cuh"
 
 using namespace qlin;
@@ -578,6 +579,23 @@ qlin_status noalloc_scratch(unsigned** out) {
   return QLIN_OK;
 }
 
+// ---------------------------------------------------------------- backward
+template <int FMT>
+qlin_status launch_backward_t(const CUtensorMap& tm, const BwdArgs& args, cudaStream_t stream) {
+  using C = BwdCfg<FMT>;
+  auto kern = backward_dx_kernel<FMT>;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+  const dim3 grid(static_cast<unsigned>((args.K + 255) / 256), static_cast<unsigned>((args.M + 127) / 128));
+  cudaError_t e = launch_k(kern, grid, dim3(C::kThreads), C::kSmemBytes, stream, tm, args);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "backward_dx_kernel launch failed: %s", cudaGetErrorString(e));
+  return QLIN_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -796,6 +814,46 @@ qlin_status qlin_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, c
     QLIN_LAUNCH_CHECK("comp_operand_kernel");
   }
   return launch_gemm(w, Xq, a, M, Y, acc_debug, gws, stream);
+}
+
+qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t M, const float* s, uint16_t* dX,
+                             void* stream_) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  if (M > 65535 * 128) return fail(QLIN_ERR_SHAPE, "M=%d exceeds %d", M, 65535 * 128);
+  if (M == 0) return QLIN_OK;
+  const int nO = w->n_outlier;
+  if (!dY || !dX) return fail(QLIN_ERR_ARG, "dY/dX is NULL");
+  if (nO > 0 && !s) return fail(QLIN_ERR_ARG, "s is NULL with n_outlier=%d", nO);
+  if (!aligned16(dY) || !aligned16(dX) || (s && !aligned16(s)))
+    return fail(QLIN_ERR_ALIGN, "a backward buffer is not 16-byte aligned");
+  st = get_encoder();
+  if (st != QLIN_OK) return st;
+  CUtensorMap tm;
+  st = make_map(&tm, dY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w->N, M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLIN_OK) return st;
+  BwdArgs args;
+  args.codes = static_cast<const uint8_t*>(w->codes);
+  args.rfold = w->fold_ratio;
+  args.wot = w->W_Ot;
+  args.cscale = w->chan_scale;
+  args.oidx = w->outlier_idx;
+  args.s = s;
+  args.dX = dX;
+  args.M = M;
+  args.N = w->N;
+  args.K = w->K;
+  args.nO = nO;
+  args.kbs = (w->K + 127) / 128;
+  args.nib = (nO + 63) / 64;
+  args.nsteps = (w->N + 63) / 64;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  switch (w->fmt) {
+    case QLIN_W4_PERCHANNEL: return launch_backward_t<kFmtW4PC>(tm, args, stream);
+    case QLIN_W4_G128: return launch_backward_t<kFmtW4G128>(tm, args, stream);
+    default: return launch_backward_t<kFmtW8>(tm, args, stream);
+  }
 }
 
 qlin_status qlin_forward_workspace(int32_t M, const qlin_weights* w, size_t* bytes) {

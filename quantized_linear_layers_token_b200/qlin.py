@@ -28,7 +28,7 @@ EXPORTED = [
     "qlin_status_string", "qlin_last_error", "qlin_weights_bytes", "qlin_weights_bind",
     "qlin_pack_weights", "qlin_quant_act_workspace", "qlin_quant_act", "qlin_outlier_colmax",
     "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
-    "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc",
+    "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc", "qlin_backward_dx",
 ]
 
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "qlin_forward": [P, I32, W, P, F32, I32, P, P, SZ, P],
             "qlin_poll_device_status": [P],
             "qlin_quant_act_noalloc": [P, I32, W, P, F32, I32, P, P, P, P],
+            "qlin_backward_dx": [W, P, I32, P, P, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -186,6 +187,11 @@ def qlin_forward(X, M: int, w: qlin_weights, s, gamma: float, update_momentum: b
                  ws_bytes: int, stream=None):
     _check(lib().qlin_forward(_ptr(X), M, ctypes.byref(w), _ptr(s), float(gamma), int(bool(update_momentum)),
                               _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)), "qlin_forward")
+
+
+def qlin_backward_dx(w: qlin_weights, dY, M: int, s, dX, stream=None):
+    _check(lib().qlin_backward_dx(ctypes.byref(w), _ptr(dY), M, _ptr(s), _ptr(dX), _stream(stream)),
+           "qlin_backward_dx")
 
 
 def qlin_poll_device_status(stream=None):

@@ -127,6 +127,20 @@ def weights(rng: np.random.Generator, K: int, N: int, std: float, spike_frac: fl
     return w.astype(np.float16)
 
 
+def grad_output(index: int, shape_idx: int, M: int, N: int, std: float = 2.0 ** -7) -> np.ndarray:
+    """Upstream gradient dY (fp16 [M][N]) for the input-gradient path:
+    N(0, std^2) i.i.d., a stand-in for the gradient a fine-tuning loss sends
+    back through the layer (draw kind 5 of the shape's sub-streams)."""
+    rng = rng_for(index, shape_idx, 5, M % 997)
+    return (rng.standard_normal((M, N), dtype=np.float32) * np.float32(std)).astype(np.float16)
+
+
+def outlier_scales(index: int, shape_idx: int, n: int, lo: float = 1.0, hi: float = 8.0) -> np.ndarray:
+    """Scales s (fp32 [n]) a forward pass left on the outlier channels: U[lo, hi]
+    (draw kind 6)."""
+    return rng_for(index, shape_idx, 6).uniform(lo, hi, size=n).astype(np.float32)
+
+
 def layer(workload: str | Workload, shape_idx: int, M: int | None = None, step: int = 0,
           K: int | None = None, N: int | None = None, n_outliers: int | None = None,
           with_weights: bool = True) -> dict:

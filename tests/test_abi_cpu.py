@@ -105,3 +105,20 @@ def test_workspace_and_alignment_errors(q):
     with pytest.raises(q.QlinError) as e:
         q.qlin_quant_act(1 << 24, M, w, 1 << 25, 1.5, True, 1 << 26, 1 << 27, 1 << 28, 1 << 29, 4096, stream=0)
     assert q.STATUS[e.value.status] == "QLIN_ERR_ARG"  # gamma outside [0, 1]
+
+
+def test_backward_argument_errors(q):
+    K, N, nO = 512, 128, 5
+    n = q.qlin_weights_bytes(K, N, 0, nO)
+    w = q.qlin_weights_bind(K, N, 0, nO, 1 << 20, n)
+    q.qlin_backward_dx(w, None, 0, None, None, stream=0)  # M = 0: nothing to do
+    for dY, M, s, status in [
+        (1 << 24, -1, 1 << 25, "QLIN_ERR_ARG"),
+        (None, 4, 1 << 25, "QLIN_ERR_ARG"),
+        (1 << 24, 4, None, "QLIN_ERR_ARG"),  # s is needed when the layer has outliers
+        ((1 << 24) + 2, 4, 1 << 25, "QLIN_ERR_ALIGN"),
+        (1 << 24, 65535 * 128 + 1, 1 << 25, "QLIN_ERR_SHAPE"),
+    ]:
+        with pytest.raises(q.QlinError) as e:
+            q.qlin_backward_dx(w, dY, M, s, 1 << 26, stream=0)
+        assert q.STATUS[e.value.status] == status
