@@ -15,17 +15,20 @@
 // c_n / 16 (per-channel INT4), the folded requantisation q8 with c_n (g128),
 // q with c_n (INT8).
 //
-// One CTA computes a 128-token x 256-input tile of dX on the tensor cores
-// (kind::f16, fp32 accumulators in TMEM), reducing over the N output
-// channels 64 at a time:
-//   A = dY tile (128 tokens x 64 channels, K-major), loaded by TMA (warp 0);
+// One CTA computes a 256-token x 256-input tile of dX on the tensor cores
+// (kind::f16, two fp32 accumulators of 128 x 256 filling TMEM), reducing over
+// the N output channels 64 at a time:
+//   A = dY tile (256 tokens x 64 channels, K-major), loaded by TMA (warp 0);
 //   B = Weff tile (256 inputs x 64 channels), written to shared memory as fp16
-//       by eight converter warps from the packed codes that warp 2 copies in.
+//       by sixteen converter warps from the packed codes (and the channel
+//       scales) that warp 2 copies in; each thread owns a 32-input window of
+//       one channel row.
 //       The codes of a channel row are contiguous along the inputs, so the
 //       operand is stored MN-major (inputs contiguous, 128-byte swizzle) and
 //       the conversion needs no transpose;
-//   warp 1 issues four 128 x 256 x 16 MMAs per step.
-// The outlier rows are blended into B after each step's conversion; the
+//   warp 1 issues eight 128 x 256 x 16 MMAs per step (each B slice serves
+//   both 128-token halves, so a code block is converted once per 256 tokens).
+// The outlier rows are blended into B by the thread that converted them; the
 // converter warps then read the accumulators back and store fp16 dX rows.
 #pragma once
 
@@ -53,12 +56,14 @@ struct BwdCfg {
   static constexpr int kRowBytes = kW4 ? 64 : 128;  // code bytes of one channel row of a 128-input block
   static constexpr int kBlkBytes = 128 * kRowBytes;  // one code block
   static constexpr int kStgBlk = 64 * kRowBytes;     // the 64 rows of one step
-  static constexpr int kStgRatio = 2 * kStgBlk;      // g128: the step's ratios, 2 x 64 fp16
-  static constexpr int kStgBytes = 2 * kStgBlk + (FMT == kFmtW4G128 ? 256 : 0);
-  static constexpr int kASlots = 4;               // dY tiles
-  static constexpr int kBSlots = 3;               // Weff tiles
-  static constexpr int kLSlots = kW4 ? 4 : 3;     // code staging
-  static constexpr int kABytes = 128 * 64 * 2;    // 16 KiB
+  static constexpr int kStgScale = 2 * kStgBlk;      // the step's 64 channel scales c_n (fp32)
+  static constexpr int kStgRatio = kStgScale + 256;  // g128: the step's ratios, 2 x 64 fp16
+  static constexpr int kStgBytes = kStgRatio + (FMT == kFmtW4G128 ? 256 : 0);
+  static constexpr int kPrefetch = 4;                // outlier-row values held in registers per thread
+  static constexpr int kASlots = 3;               // dY tiles
+  static constexpr int kBSlots = kW4 ? 3 : 2;     // Weff tiles
+  static constexpr int kLSlots = 3;               // code staging
+  static constexpr int kABytes = 256 * 64 * 2;    // 32 KiB: 256 tokens x 64 channels
   static constexpr int kBBytes = 256 * 64 * 2;    // 32 KiB
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kASlots * kABytes;
@@ -67,17 +72,16 @@ struct BwdCfg {
   static constexpr int kMaxOut = 256;             // outliers among 256 inputs, at most
   static constexpr int kOffBar = kOffOut + kMaxOut * 16;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + slack to 1024-align the base
-  static constexpr int kConvWarps = 8;
+  static constexpr int kConvWarps = 16;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
   static_assert(kSmemBytes <= 232448, "backward tile does not fit in shared memory");
 };
 
-// c'_n of the forward's INT8 operand (0 beyond N).
-template <int FMT>
-__device__ __forceinline__ float bwd_chan_scale(const BwdArgs& g, int n) {
-  if (n >= g.N) return 0.f;
-  const float c = g.cscale[n];
-  return FMT == kFmtW4PC ? __fmul_rn(c, 0.0625f) : c;
+// W_O[i][n] from the tiled, swizzled W_O^T (fp16 bits).
+__device__ __forceinline__ uint16_t wot_elem(const BwdArgs& g, int n, int i) {
+  const int r = n & 127;
+  const size_t blk = static_cast<size_t>(n >> 7) * g.nib + (i >> 6);
+  return __ldg(g.wot + blk * 8192 + r * 64 + ((((i & 63) >> 3) ^ (r & 7)) << 3) + (i & 7));
 }
 
 // Four INT8 lanes -> two fp16 pairs times c (exact int8 -> fp16 through the
@@ -104,6 +108,16 @@ __device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t lbo,
   return d;
 }
 
+// First entry of the outlier table (sorted by input) at or after input kl.
+__device__ __forceinline__ int outl_lower_bound(const float4* t, int n, int kl) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__float_as_int(t[mid].x) < kl) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
 // First index i in [0, n) with a[i] >= v (n if none).
 __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
   int lo = 0, hi = n;
@@ -119,6 +133,16 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
 // 16-byte chunk of inputs 8c..8c+7 at chunk c ^ (n % 8).
 constexpr uint32_t kBwdLbo = 1024;  // next 64 inputs
 constexpr uint32_t kBwdSbo = 4096;  // next 8 channels
+
+// Blend one outlier row element of a B tile: channel q of the step, outlier
+// entry o = {input - k0, i, s_i - 1, 1 / s_i}, w = W_O[i][n] (fp16 bits).
+__device__ __forceinline__ void patch_outlier(unsigned char* bt, const float4 o, int q, uint16_t w) {
+  const int kl = __float_as_int(o.x);
+  __half* p = reinterpret_cast<__half*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
+                                        ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
+  const float v = __fmul_rn(__fmaf_rn(o.z, __half2float(__ushort_as_half(w)), __half2float(*p)), o.w);
+  *p = __float2half_rn(v);
+}
 
 template <int FMT>
 __global__ void __launch_bounds__(BwdCfg<FMT>::kThreads, 1)
@@ -141,9 +165,13 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int k0 = blockIdx.x * 256;
-  const int m0 = blockIdx.y * 128;
+  const int m0 = blockIdx.y * 256;
+  const bool two = m0 + 128 < args.M;  // the second 128-token half holds tokens
   const int nsteps = args.nsteps;
   const int nb = (2 * static_cast<int>(blockIdx.x) + 1 < args.kbs) ? 2 : 1;  // code blocks in this input tile
+#ifdef QLIN_TRACE
+  long long* const qlin_st = (blockIdx.x == 0 && blockIdx.y == 0) ? g_steps : nullptr;
+#endif
 
   if (warp == 0) {
     if (lane < AS) {
@@ -163,7 +191,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     if (lane == 0) tma_prefetch_desc(&tmDY);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -182,6 +210,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
         if (j >= AS && !mbar_wait(&aempty[a], static_cast<uint32_t>(j / AS - 1) & 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&afull[a], C::kABytes);
         tma_load_2d(smem + C::kOffA + a * C::kABytes, &tmDY, &afull[a], j * 64, m0);
+        QLIN_STEP(j, 1);
         ++issued;
       }
       drain_ring(afull, AS, issued);
@@ -194,16 +223,22 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
         const int a = j % AS;
         const int b = j % BS;
         if (!mbar_wait(&afull[a], static_cast<uint32_t>(j / AS) & 1u, abort_flag)) break;
+        QLIN_STEP(j, 5);
         if (!mbar_wait(&bfull[b], static_cast<uint32_t>(j / BS) & 1u, abort_flag)) break;
+        QLIN_STEP(j, 6);
         tc_fence_after();
         const uint32_t abase = smem_u32(smem + C::kOffA + a * C::kABytes);
         const uint32_t bbase = smem_u32(smem + C::kOffB + b * C::kBBytes);
+        // one B tile, two 128-token halves of A into columns [0, 256) and [256, 512)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16(tmem, sdesc_k_sw128(abase + kk * 32), sdesc_mn_sw128(bbase + kk * 2 * kBwdSbo, kBwdLbo, kBwdSbo),
-                  idesc, (j | kk) != 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bdesc = sdesc_mn_sw128(bbase + kk * 2 * kBwdSbo, kBwdLbo, kBwdSbo);
+          mma_f16(tmem, sdesc_k_sw128(abase + kk * 32), bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
+          if (two) mma_f16(tmem + 256, sdesc_k_sw128(abase + 16384 + kk * 32), bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
+        }
         mma_commit(&aempty[a]);
         mma_commit(&bempty[b]);
+        QLIN_STEP(j, 7);
       }
       // every MMA issued so far (all of them, or those before an abort)
       mma_commit(acc_full);
@@ -222,9 +257,11 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
         const int n0 = j * 64;
         const int tn = n0 >> 7;
         const int r0 = n0 & 127;
-        const uint32_t rbytes = FMT == kFmtW4G128 ? static_cast<uint32_t>(min(64, args.N - n0) * 2) : 0u;
-        mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nb) * (C::kStgBlk + rbytes));
+        const uint32_t nv = static_cast<uint32_t>(min(64, args.N - n0));  // channels of this step (multiple of 16)
+        const uint32_t rbytes = FMT == kFmtW4G128 ? nv * 2 : 0u;
+        mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nb) * (C::kStgBlk + rbytes) + nv * 4);
         unsigned char* dst = smem + C::kOffStg + ls * C::kStgBytes;
+        bulk_load(dst + C::kStgScale, args.cscale + n0, nv * 4, &sfull[ls]);
         for (int b = 0; b < nb; ++b) {
           const size_t blk = static_cast<size_t>(tn) * args.kbs + kb0 + b;
           bulk_load(dst + b * C::kStgBlk, args.codes + blk * C::kBlkBytes + r0 * C::kRowBytes, C::kStgBlk, &sfull[ls]);
@@ -232,14 +269,15 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
             bulk_load(dst + C::kStgRatio + b * 128, args.rfold + static_cast<size_t>(kb0 + b) * args.N + n0, rbytes,
                       &sfull[ls]);
         }
+        QLIN_STEP(j, 0);
         ++issued;
       }
       drain_ring(sfull, LS, issued);
     }
   } else {
     // ------------------------------------------- converters, then epilogue
-    const int cw = warp - 3;             // 0..7
-    const int ctid = threadIdx.x - 96;   // 0..255
+    const int cw = warp - 3;             // 0..15
+    const int ctid = threadIdx.x - 96;   // 0..511
     griddep_wait();                      // s comes from the forward
     int nout = 0;
     if (args.nO > 0) {
@@ -254,31 +292,41 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     }
     named_bar_sync(1, 32 * C::kConvWarps);
 
+    // Each thread converts one 32-input window (inputs 32 g .. 32 g + 31 of
+    // the tile) of one channel row per step and blends the outlier rows that
+    // fall inside it, so no thread waits for another before the arrival.
     const int nl = (cw & 1) * 32 + lane;  // channel row of the step
-    const int cq = cw >> 1;               // quarter of the row's inputs
+    const int g = cw >> 1;                // window, 0..7
     const int sw = nl & 7;
-    // After a failed wait the loop keeps running, with no work, so that
-    // every converter warp reaches every named barrier.
+    const int olo = outl_lower_bound(outl, nout, 32 * g);  // the window's outlier entries
+    const int ohi = outl_lower_bound(outl, nout, 32 * g + 32);
+    uint16_t wpre[C::kPrefetch];  // W_O values of the first entries, one step ahead
+#pragma unroll
+    for (int u = 0; u < C::kPrefetch; ++u)
+      wpre[u] = olo + u < ohi ? wot_elem(args, nl, __float_as_int(outl[olo + u].y)) : uint16_t(0);
+
     bool ok = true;
     for (int j = 0; j < nsteps; ++j) {
       const int ls = j % LS;
       const int b = j % BS;
       if (ok) ok = mbar_wait(&sfull[ls], static_cast<uint32_t>(j / LS) & 1u, abort_flag);
+      if (ctid == 0) QLIN_STEP(j, 2);
       if (ok && j >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(j / BS - 1) & 1u, abort_flag);
+      if (ctid == 0) QLIN_STEP(j, 3);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (nout > 0) named_bar_sync(1, 32 * C::kConvWarps);
-        continue;
-      }
+      if (!ok) break;
       const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
       unsigned char* bt = smem + C::kOffB + b * C::kBBytes;
       unsigned char* brow = bt + (nl >> 3) * kBwdSbo + sw * 128;
-      const __half2 c2 = __float2half2_rn(bwd_chan_scale<FMT>(args, j * 64 + nl));
+      // c'_n of the forward's INT8 operand: c_n / 16 for per-channel INT4 (16 q), else c_n; 0 beyond N
+      float cn = j * 64 + nl < args.N ? reinterpret_cast<const float*>(stg + C::kStgScale)[nl] : 0.f;
+      if (FMT == kFmtW4PC) cn = __fmul_rn(cn, 0.0625f);
+      const __half2 c2 = __float2half2_rn(cn);
       if (FMT == kFmtW8) {
-        // 4 chunks of 16 inputs: inputs 64 cq .. 64 cq + 63
+        // two 16-input chunks of the code block's 128-byte row
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int cc = cq * 4 + t;
+        for (int t = 0; t < 2; ++t) {
+          const int cc = 2 * g + t;
           const int blk = cc >> 3;
           const int c = cc & 7;
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -295,8 +343,9 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           *reinterpret_cast<uint4*>(atom + (((ch + 1) ^ sw) << 4)) = h1;
         }
       } else {
-        // 2 chunks of 32 inputs: inputs 64 cq .. 64 cq + 63
-        const int blk = cq >> 1;  // both chunks lie in one code block
+        // one 32-input chunk of the code block's 64-byte row
+        const int blk = g >> 2;
+        const int c = g & 3;
         __half2 r1 = __half2half2(__ushort_as_half(static_cast<unsigned short>(0)));
         __half2 r16 = r1;
         if (FMT == kFmtW4G128 && blk < nb) {  // absent block: r = 0 makes every code 0
@@ -304,62 +353,55 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           r1 = __half2half2(__ushort_as_half(rbits));
           r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
         }
-        const int rsw = (nl >> 1) & 3;
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (blk < nb) w = *reinterpret_cast<const uint4*>(stg + blk * C::kStgBlk + nl * 64 + ((c ^ ((nl >> 1) & 3)) << 4));
+        uint32_t q8[8];  // INT8 lanes of inputs 4e .. 4e + 3 of the chunk
+        if (FMT == kFmtW4PC) {
+          uint4 o0, o1;
+          unpack_w4pc(w, o0, o1);
+          q8[0] = o0.x; q8[1] = o0.y; q8[2] = o0.z; q8[3] = o0.w;
+          q8[4] = o1.x; q8[5] = o1.y; q8[6] = o1.z; q8[7] = o1.w;
+        } else {
+          const uint2 a0 = requant_g128(w.x, r1, r16);
+          const uint2 a1 = requant_g128(w.y, r1, r16);
+          const uint2 a2 = requant_g128(w.z, r1, r16);
+          const uint2 a3 = requant_g128(w.w, r1, r16);
+          q8[0] = a0.x; q8[1] = a0.y; q8[2] = a1.x; q8[3] = a1.y;
+          q8[4] = a2.x; q8[5] = a2.y; q8[6] = a3.x; q8[7] = a3.y;
+        }
+        unsigned char* atom = brow + (g >> 1) * kBwdLbo;
+        const int ch0 = (g & 1) * 4;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int c = (cq & 1) * 2 + t;  // 32-input chunk within the block
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (blk < nb) w = *reinterpret_cast<const uint4*>(stg + blk * C::kStgBlk + nl * 64 + ((c ^ rsw) << 4));
-          uint32_t q8[8];  // INT8 lanes of inputs 4e .. 4e + 3 of the chunk
-          if (FMT == kFmtW4PC) {
-            uint4 o0, o1;
-            unpack_w4pc(w, o0, o1);
-            q8[0] = o0.x; q8[1] = o0.y; q8[2] = o0.z; q8[3] = o0.w;
-            q8[4] = o1.x; q8[5] = o1.y; q8[6] = o1.z; q8[7] = o1.w;
-          } else {
-            const uint2 a0 = requant_g128(w.x, r1, r16);
-            const uint2 a1 = requant_g128(w.y, r1, r16);
-            const uint2 a2 = requant_g128(w.z, r1, r16);
-            const uint2 a3 = requant_g128(w.w, r1, r16);
-            q8[0] = a0.x; q8[1] = a0.y; q8[2] = a1.x; q8[3] = a1.y;
-            q8[4] = a2.x; q8[5] = a2.y; q8[6] = a3.x; q8[7] = a3.y;
-          }
-          const int kl = blk * 128 + 32 * c;
-          unsigned char* atom = brow + (kl >> 6) * kBwdLbo;
-          const int ch0 = (kl & 63) >> 3;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 h;
-            i8x4_scale_h2(q8[2 * e], c2, h.x, h.y);
-            i8x4_scale_h2(q8[2 * e + 1], c2, h.z, h.w);
-            *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
-          }
+        for (int e = 0; e < 4; ++e) {
+          uint4 h;
+          i8x4_scale_h2(q8[2 * e], c2, h.x, h.y);
+          i8x4_scale_h2(q8[2 * e + 1], c2, h.z, h.w);
+          *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sempty[ls]);  // staging slot consumed
-      if (nout > 0) {
-        // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i
-        named_bar_sync(1, 32 * C::kConvWarps);
-        for (int t = ctid; t < nout * 64; t += 32 * C::kConvWarps) {
-          const float4 o = outl[t >> 6];
-          const int q = t & 63;
-          const int kl = __float_as_int(o.x);
-          const int i = __float_as_int(o.y);
-          __half* p = reinterpret_cast<__half*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
-                                                ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
-          const int ng = j * 64 + q;
-          const int r = ng & 127;
-          const size_t wblk = static_cast<size_t>(ng >> 7) * args.nib + (i >> 6);
-          const uint16_t wbits =
-              __ldg(args.wot + wblk * 8192 + r * 64 + ((((i & 63) >> 3) ^ (r & 7)) << 3) + (i & 7));
-          const float v = __fmul_rn(__fmaf_rn(o.z, __half2float(__ushort_as_half(wbits)), __half2float(*p)), o.w);
-          *p = __float2half_rn(v);
+      if (olo < ohi) {
+        // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i, on the
+        // values this thread has just stored
+#pragma unroll
+        for (int u = 0; u < C::kPrefetch; ++u)
+          if (olo + u < ohi) patch_outlier(bt, outl[olo + u], nl, wpre[u]);
+        for (int e = olo + C::kPrefetch; e < ohi; ++e) {
+          const float4 o = outl[e];
+          patch_outlier(bt, o, nl, wot_elem(args, j * 64 + nl, __float_as_int(o.y)));
+        }
+        if (j + 1 < nsteps) {
+#pragma unroll
+          for (int u = 0; u < C::kPrefetch; ++u)
+            if (olo + u < ohi) wpre[u] = wot_elem(args, (j + 1) * 64 + nl, __float_as_int(outl[olo + u].y));
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bfull[b]);
+      if (lane == 0) {
+        mbar_arrive(&sempty[ls]);  // staging slot consumed
+        mbar_arrive(&bfull[b]);    // B slot written
+      }
+      if (ctid == 0) QLIN_STEP(j, 4);
     }
 
     // epilogue: TMEM lane = token, column = input
@@ -367,13 +409,15 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     if (__all_sync(0xffffffffu, got && *abort_flag == 0)) {
       tc_fence_after();
       const int qd = warp & 3;  // TMEM lane quadrant of this warp
-      const int half = cw >> 2;
-      const int m = m0 + qd * 32 + lane;
+      const int quarter = cw >> 2;  // 64 input columns per warp, in both token halves
 #pragma unroll 1
-      for (int jj = 0; jj < 4; ++jj) {
-        const int col = half * 128 + jj * 32;
+      for (int jj = 0; jj < (two ? 4 : 2); ++jj) {
+        const int h = jj >> 1;
+        const int col = quarter * 64 + (jj & 1) * 32;
+        const int m = m0 + h * 128 + qd * 32 + lane;
         uint32_t v0[16], v1[16];
-        const uint32_t ta = tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(col);
+        const uint32_t ta =
+            tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(h * 256 + col);
         tmem_ld16(ta, v0);
         tmem_ld16(ta + 16, v1);
         tmem_ld_wait();
@@ -396,7 +440,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

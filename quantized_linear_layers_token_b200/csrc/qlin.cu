@@ -590,7 +590,7 @@ qlin_status launch_backward_t(const CUtensorMap& tm, const BwdArgs& args, cudaSt
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  const dim3 grid(static_cast<unsigned>((args.K + 255) / 256), static_cast<unsigned>((args.M + 127) / 128));
+  const dim3 grid(static_cast<unsigned>((args.K + 255) / 256), static_cast<unsigned>((args.M + 255) / 256));
   cudaError_t e = launch_k(kern, grid, dim3(C::kThreads), C::kSmemBytes, stream, tm, args);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "backward_dx_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
@@ -831,7 +831,7 @@ qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t 
   st = get_encoder();
   if (st != QLIN_OK) return st;
   CUtensorMap tm;
-  st = make_map(&tm, dY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w->N, M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  st = make_map(&tm, dY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w->N, M, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != QLIN_OK) return st;
   BwdArgs args;
   args.codes = static_cast<const uint8_t*>(w->codes);

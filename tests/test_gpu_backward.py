@@ -96,9 +96,10 @@ def check(dX, dY, W, pk, s, oracle, rows=None):
 
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M,K,N,nO", [
-    (200, 640, 208, 37),   # 2 token tiles (ragged), 3 input tiles (last half empty), ragged channel step
+    (200, 640, 208, 37),   # both 128-token halves (ragged), 3 input tiles (last half empty), ragged channel step
     (1, 256, 16, 0),       # one token, one 16-channel step, no outliers
-    (129, 1152, 400, 64),  # one token past a tile; odd number of code blocks
+    (129, 1152, 400, 64),  # one token past a 128-token half; odd number of code blocks
+    (300, 384, 96, 11),    # two 256-token tiles, the second with its first half only
 ])
 def test_backward_parity(q, oracle, fmt, M, K, N, nO):
     L = synth.layer("small", 0, M=1, K=K, N=N, n_outliers=nO)
