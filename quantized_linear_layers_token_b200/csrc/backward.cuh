@@ -20,9 +20,9 @@
 // the N output channels 64 at a time:
 //   A = dY tile (256 tokens x 64 channels, K-major), loaded by TMA (warp 0);
 //   B = Weff tile (256 inputs x 64 channels), written to shared memory as fp16
-//       by sixteen converter warps from the packed codes (and the channel
-//       scales) that warp 2 copies in; each thread owns a 32-input window of
-//       one channel row.
+//       by sixteen converter warps; each thread owns a 32-input window of one
+//       channel row and reads its codes (16 or 32 bytes), channel scale and
+//       ratio straight from global memory two steps ahead.
 //       The codes of a channel row are contiguous along the inputs, so the
 //       operand is stored MN-major (inputs contiguous, 128-byte swizzle) and
 //       the conversion needs no transpose;
@@ -53,24 +53,28 @@ struct BwdArgs {
 template <int FMT>
 struct BwdCfg {
   static constexpr bool kW4 = FMT != kFmtW8;
-  static constexpr int kRowBytes = kW4 ? 64 : 128;  // code bytes of one channel row of a 128-input block
-  static constexpr int kBlkBytes = 128 * kRowBytes;  // one code block
-  static constexpr int kStgBlk = 64 * kRowBytes;     // the 64 rows of one step
-  static constexpr int kStgScale = 2 * kStgBlk;      // the step's 64 channel scales c_n (fp32)
-  static constexpr int kStgRatio = kStgScale + 256;  // g128: the step's ratios, 2 x 64 fp16
-  static constexpr int kStgBytes = kStgRatio + (FMT == kFmtW4G128 ? 256 : 0);
-  static constexpr int kPrefetch = 4;                // outlier-row values held in registers per thread
+  // W_O ring: for each step, the W_O^T row segments (16-byte chunks) that
+  // hold the tile's first kWMax outliers, 64 channel rows of kWChunks chunks
+  static constexpr int kWR = 4;                   // steps in flight
+  static constexpr int kWMax = 32;                // outliers served from the ring
+  static constexpr int kWChunks = 5;              // chunks spanned by 32 consecutive outliers, at most
+  static constexpr int kWRow = 16 * kWChunks;     // 80 bytes per channel row
+  static constexpr int kWSlot = 64 * kWRow;
   static constexpr int kASlots = 3;               // dY tiles
-  static constexpr int kBSlots = kW4 ? 3 : 2;     // Weff tiles
-  static constexpr int kLSlots = 3;               // code staging
+  static constexpr int kBSlots = 3;               // Weff tiles
+  // A converter warp starts step j only after every warp has finished step
+  // j - kBSlots (its B slot must be free), so all warps stay within kBSlots
+  // steps of each other, and at least one warp waits for each ring fill; with
+  // more ring slots than that, arrivals for one slot never mix two steps.
+  static_assert(kWR > kBSlots, "the W_O ring must be deeper than the B ring");
   static constexpr int kABytes = 256 * 64 * 2;    // 32 KiB: 256 tokens x 64 channels
   static constexpr int kBBytes = 256 * 64 * 2;    // 32 KiB
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kASlots * kABytes;
-  static constexpr int kOffStg = kOffB + kBSlots * kBBytes;
-  static constexpr int kOffOut = (kOffStg + kLSlots * kStgBytes + 15) / 16 * 16;
+  static constexpr int kOffOut = kOffB + kBSlots * kBBytes;
   static constexpr int kMaxOut = 256;             // outliers among 256 inputs, at most
-  static constexpr int kOffBar = kOffOut + kMaxOut * 16;
+  static constexpr int kOffW = kOffOut + kMaxOut * 16;
+  static constexpr int kOffBar = kOffW + kWR * kWSlot;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + slack to 1024-align the base
   static constexpr int kConvWarps = 16;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
@@ -128,6 +132,45 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
   return lo;
 }
 
+// What one converter thread reads from global memory for one step: its code
+// chunk(s), the channel scale and (g128) the group ratio of its row.
+template <int FMT>
+struct BwdIn {
+  uint4 w[FMT == kFmtW8 ? 2 : 1];
+  float c;     // c_n, 0 beyond N
+  uint16_t r;  // g128: r[kb][n] bits, 0 for an absent block or channel
+};
+
+// Step j, channel row nl, 32-input window g of the tile whose first code
+// block is kb0 (nb blocks present).  Rows past N inside a block are zero
+// codes, so only the per-channel arrays need the bound.
+template <int FMT>
+__device__ __forceinline__ void load_step(BwdIn<FMT>& in, const BwdArgs& a, int j, int nl, int g, int kb0, int nb) {
+  const int n = j * 64 + nl;
+  const int tn = n >> 7;
+  const int r = n & 127;
+  in.c = n < a.N ? __ldg(a.cscale + n) : 0.f;
+  if (FMT == kFmtW8) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int cc = 2 * g + t;  // 16-input chunk of the tile
+      const int blk = cc >> 3;
+      const int c = cc & 7;
+      in.w[t] = blk < nb ? __ldg(reinterpret_cast<const uint4*>(
+                               a.codes + (static_cast<size_t>(tn) * a.kbs + kb0 + blk) * 16384 + r * 128 + ((c ^ (r & 7)) << 4)))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+  } else {
+    const int blk = g >> 2;
+    const int c = g & 3;  // 32-input chunk of the block
+    in.w[0] = blk < nb ? __ldg(reinterpret_cast<const uint4*>(
+                             a.codes + (static_cast<size_t>(tn) * a.kbs + kb0 + blk) * 8192 + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)))
+                       : make_uint4(0u, 0u, 0u, 0u);
+    if (FMT == kFmtW4G128)
+      in.r = (blk < nb && n < a.N) ? __ldg(a.rfold + static_cast<size_t>(kb0 + blk) * a.N + n) : uint16_t(0);
+  }
+}
+
 // B tile layout: 8-channel group g (K) x 64-input atom a (MN), atom (g, a) at
 // (4 g + a) KiB; within an atom, channel row (n % 8) at 128 (n % 8) and the
 // 16-byte chunk of inputs 8c..8c+7 at chunk c ^ (n % 8).
@@ -136,10 +179,13 @@ constexpr uint32_t kBwdSbo = 4096;  // next 8 channels
 
 // Blend one outlier row element of a B tile: channel q of the step, outlier
 // entry o = {input - k0, i, s_i - 1, 1 / s_i}, w = W_O[i][n] (fp16 bits).
+__device__ __forceinline__ __half* outlier_elem(unsigned char* bt, int kl, int q) {
+  return reinterpret_cast<__half*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
+                                   ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
+}
+
 __device__ __forceinline__ void patch_outlier(unsigned char* bt, const float4 o, int q, uint16_t w) {
-  const int kl = __float_as_int(o.x);
-  __half* p = reinterpret_cast<__half*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
-                                        ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
+  __half* p = outlier_elem(bt, __float_as_int(o.x), q);
   const float v = __fmul_rn(__fmaf_rn(o.z, __half2float(__ushort_as_half(w)), __half2float(*p)), o.w);
   *p = __float2half_rn(v);
 }
@@ -148,17 +194,17 @@ template <int FMT>
 __global__ void __launch_bounds__(BwdCfg<FMT>::kThreads, 1)
 backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ BwdArgs args) {
   using C = BwdCfg<FMT>;
-  constexpr int AS = C::kASlots, BS = C::kBSlots, LS = C::kLSlots;
+  constexpr int AS = C::kASlots, BS = C::kBSlots;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* afull = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* aempty = afull + AS;
   uint64_t* bfull = aempty + AS;
   uint64_t* bempty = bfull + BS;
-  uint64_t* sfull = bempty + BS;
-  uint64_t* sempty = sfull + LS;
-  uint64_t* acc_full = sempty + LS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = bempty + BS;
+  uint64_t* wfull = acc_full + 1;        // [kWR]
+  uint64_t* wempty = wfull + C::kWR;     // [kWR]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty + C::kWR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float4* outl = reinterpret_cast<float4*>(smem + C::kOffOut);  // {input - k0, i, s_i - 1, 1 / s_i}
 
@@ -180,12 +226,12 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     } else if (lane >= 8 && lane < 8 + BS) {
       mbar_init(&bfull[lane - 8], C::kConvWarps);
       mbar_init(&bempty[lane - 8], 1);
-    } else if (lane >= 16 && lane < 16 + LS) {
-      mbar_init(&sfull[lane - 16], 1);
-      mbar_init(&sempty[lane - 16], C::kConvWarps);
     } else if (lane == 24) {
       mbar_init(acc_full, 1);
       *abort_flag = 0;
+    } else if (lane >= 16 && lane < 16 + C::kWR) {
+      mbar_init(&wfull[lane - 16], 32);  // one cp.async arrival per producer lane
+      mbar_init(&wempty[lane - 16], C::kConvWarps);
     }
     fence_barrier_init();
     if (lane == 0) tma_prefetch_desc(&tmDY);
@@ -247,41 +293,56 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       }
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------ code producer
-    if (lane == 0) {
-      int issued = 0;
-      const int kb0 = 2 * static_cast<int>(blockIdx.x);
+    // ------------------------------------------------- W_O ring producer
+    // Outlier indices and W_O^T are weights: no dependency on the previous
+    // kernel.  The tile's outliers are the consecutive entries [lo, lo + nout).
+    int lo = 0, nout = 0;
+    if (args.nO > 0) {
+      lo = lower_bound_i32(args.oidx, args.nO, k0);
+      nout = lower_bound_i32(args.oidx, args.nO, k0 + 256) - lo;
+    }
+    const int ne = min(nout, C::kWMax);
+    if (ne > 0) {
+      const int cf = lo >> 3;                        // first 8-outlier chunk
+      const int nch = ((lo + ne - 1) >> 3) - cf + 1;  // chunks per channel row, <= kWChunks
       for (int j = 0; j < nsteps; ++j) {
-        const int ls = j % LS;
-        if (j >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(j / LS - 1) & 1u, abort_flag)) break;
-        const int n0 = j * 64;
-        const int tn = n0 >> 7;
-        const int r0 = n0 & 127;
-        const uint32_t nv = static_cast<uint32_t>(min(64, args.N - n0));  // channels of this step (multiple of 16)
-        const uint32_t rbytes = FMT == kFmtW4G128 ? nv * 2 : 0u;
-        mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nb) * (C::kStgBlk + rbytes) + nv * 4);
-        unsigned char* dst = smem + C::kOffStg + ls * C::kStgBytes;
-        bulk_load(dst + C::kStgScale, args.cscale + n0, nv * 4, &sfull[ls]);
-        for (int b = 0; b < nb; ++b) {
-          const size_t blk = static_cast<size_t>(tn) * args.kbs + kb0 + b;
-          bulk_load(dst + b * C::kStgBlk, args.codes + blk * C::kBlkBytes + r0 * C::kRowBytes, C::kStgBlk, &sfull[ls]);
-          if (FMT == kFmtW4G128)
-            bulk_load(dst + C::kStgRatio + b * 128, args.rfold + static_cast<size_t>(kb0 + b) * args.N + n0, rbytes,
-                      &sfull[ls]);
+        const int slot = j % C::kWR;
+        if (j >= C::kWR && !mbar_wait(&wempty[slot], static_cast<uint32_t>(j / C::kWR - 1) & 1u, abort_flag)) break;
+        unsigned char* dst = smem + C::kOffW + slot * C::kWSlot;
+        for (int t = lane; t < 64 * nch; t += 32) {
+          const int q = t / nch;
+          const int cix = t - q * nch;
+          const int kc = cf + cix;
+          const int n = j * 64 + q;
+          const int r = n & 127;
+          const uint16_t* src = args.wot + (static_cast<size_t>(n >> 7) * args.nib + (kc >> 3)) * 8192 + r * 64 +
+                                (((kc & 7) ^ (r & 7)) << 3);
+          cp_async16(dst + q * C::kWRow + cix * 16, src);
         }
-        QLIN_STEP(j, 0);
-        ++issued;
+        cp_async_mbar_arrive_noinc(&wfull[slot]);
       }
-      drain_ring(sfull, LS, issued);
+      cp_async_wait_all();
     }
   } else {
     // ------------------------------------------- converters, then epilogue
     const int cw = warp - 3;             // 0..15
     const int ctid = threadIdx.x - 96;   // 0..511
-    griddep_wait();                      // s comes from the forward
-    int nout = 0;
+    const int kb0 = 2 * static_cast<int>(blockIdx.x);
+    // Each thread converts one 32-input window (inputs 32 g .. 32 g + 31 of
+    // the tile) of one channel row per step and blends the outlier rows that
+    // fall inside it, so no thread waits for another before the arrival.
+    // Its codes, channel scale and ratio are loaded two steps ahead.
+    const int nl = (cw & 1) * 32 + lane;  // channel row of the step
+    const int g = cw >> 1;                // window, 0..7
+    const int sw = nl & 7;
+    BwdIn<FMT> in0, in1;
+    load_step<FMT>(in0, args, 0, nl, g, kb0, nb);
+    if (nsteps > 1) load_step<FMT>(in1, args, 1, nl, g, kb0, nb);
+
+    griddep_wait();  // s comes from the forward
+    int nout = 0, lo = 0;
     if (args.nO > 0) {
-      const int lo = lower_bound_i32(args.oidx, args.nO, k0);
+      lo = lower_bound_i32(args.oidx, args.nO, k0);
       nout = lower_bound_i32(args.oidx, args.nO, k0 + 256) - lo;
       if (ctid < nout) {
         const int i = lo + ctid;
@@ -291,52 +352,33 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       }
     }
     named_bar_sync(1, 32 * C::kConvWarps);
-
-    // Each thread converts one 32-input window (inputs 32 g .. 32 g + 31 of
-    // the tile) of one channel row per step and blends the outlier rows that
-    // fall inside it, so no thread waits for another before the arrival.
-    const int nl = (cw & 1) * 32 + lane;  // channel row of the step
-    const int g = cw >> 1;                // window, 0..7
-    const int sw = nl & 7;
     const int olo = outl_lower_bound(outl, nout, 32 * g);  // the window's outlier entries
     const int ohi = outl_lower_bound(outl, nout, 32 * g + 32);
-    uint16_t wpre[C::kPrefetch];  // W_O values of the first entries, one step ahead
-#pragma unroll
-    for (int u = 0; u < C::kPrefetch; ++u)
-      wpre[u] = olo + u < ohi ? wot_elem(args, nl, __float_as_int(outl[olo + u].y)) : uint16_t(0);
+    const int ne = min(nout, C::kWMax);  // entries served by the W_O ring
+    const int lo8 = lo & 7;              // position of entry 0 in a ring row (fp16 units)
 
     bool ok = true;
-    for (int j = 0; j < nsteps; ++j) {
-      const int ls = j % LS;
+    auto step = [&](int j, BwdIn<FMT>& in) {
       const int b = j % BS;
-      if (ok) ok = mbar_wait(&sfull[ls], static_cast<uint32_t>(j / LS) & 1u, abort_flag);
-      if (ctid == 0) QLIN_STEP(j, 2);
       if (ok && j >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(j / BS - 1) & 1u, abort_flag);
       if (ctid == 0) QLIN_STEP(j, 3);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
+      if (!ok) return;
       unsigned char* bt = smem + C::kOffB + b * C::kBBytes;
       unsigned char* brow = bt + (nl >> 3) * kBwdSbo + sw * 128;
-      // c'_n of the forward's INT8 operand: c_n / 16 for per-channel INT4 (16 q), else c_n; 0 beyond N
-      float cn = j * 64 + nl < args.N ? reinterpret_cast<const float*>(stg + C::kStgScale)[nl] : 0.f;
-      if (FMT == kFmtW4PC) cn = __fmul_rn(cn, 0.0625f);
-      const __half2 c2 = __float2half2_rn(cn);
+      // c'_n of the forward's INT8 operand: c_n / 16 for per-channel INT4 (16 q), else c_n
+      const __half2 c2 = __float2half2_rn(FMT == kFmtW4PC ? __fmul_rn(in.c, 0.0625f) : in.c);
       if (FMT == kFmtW8) {
         // two 16-input chunks of the code block's 128-byte row
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          const int cc = 2 * g + t;
-          const int blk = cc >> 3;
-          const int c = cc & 7;
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (blk < nb) w = *reinterpret_cast<const uint4*>(stg + blk * C::kStgBlk + nl * 128 + ((c ^ sw) << 4));
+          const uint4 w = in.w[t];
           uint4 h0, h1;
           i8x4_scale_h2(w.x, c2, h0.x, h0.y);
           i8x4_scale_h2(w.y, c2, h0.z, h0.w);
           i8x4_scale_h2(w.z, c2, h1.x, h1.y);
           i8x4_scale_h2(w.w, c2, h1.z, h1.w);
-          const int kl = 16 * cc;  // first input of the chunk within the tile
+          const int kl = 32 * g + 16 * t;  // first input of the chunk within the tile
           unsigned char* atom = brow + (kl >> 6) * kBwdLbo;
           const int ch = (kl & 63) >> 3;
           *reinterpret_cast<uint4*>(atom + ((ch ^ sw) << 4)) = h0;
@@ -344,17 +386,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
         }
       } else {
         // one 32-input chunk of the code block's 64-byte row
-        const int blk = g >> 2;
-        const int c = g & 3;
-        __half2 r1 = __half2half2(__ushort_as_half(static_cast<unsigned short>(0)));
-        __half2 r16 = r1;
-        if (FMT == kFmtW4G128 && blk < nb) {  // absent block: r = 0 makes every code 0
-          const uint16_t rbits = reinterpret_cast<const uint16_t*>(stg + C::kStgRatio + blk * 128)[nl];
-          r1 = __half2half2(__ushort_as_half(rbits));
-          r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));  // * 1/16
-        }
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (blk < nb) w = *reinterpret_cast<const uint4*>(stg + blk * C::kStgBlk + nl * 64 + ((c ^ ((nl >> 1) & 3)) << 4));
+        const uint4 w = in.w[0];
         uint32_t q8[8];  // INT8 lanes of inputs 4e .. 4e + 3 of the chunk
         if (FMT == kFmtW4PC) {
           uint4 o0, o1;
@@ -362,6 +394,9 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           q8[0] = o0.x; q8[1] = o0.y; q8[2] = o0.z; q8[3] = o0.w;
           q8[4] = o1.x; q8[5] = o1.y; q8[6] = o1.z; q8[7] = o1.w;
         } else {
+          // an absent block or channel has r = 0, which makes every code 0
+          const __half2 r1 = __half2half2(__ushort_as_half(in.r));
+          const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));
           const uint2 a0 = requant_g128(w.x, r1, r16);
           const uint2 a1 = requant_g128(w.y, r1, r16);
           const uint2 a2 = requant_g128(w.z, r1, r16);
@@ -379,29 +414,32 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
         }
       }
+      if (j + 2 < nsteps) load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
+      const int ws = j % C::kWR;
       if (olo < ohi) {
         // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i, on the
-        // values this thread has just stored
-#pragma unroll
-        for (int u = 0; u < C::kPrefetch; ++u)
-          if (olo + u < ohi) patch_outlier(bt, outl[olo + u], nl, wpre[u]);
-        for (int e = olo + C::kPrefetch; e < ohi; ++e) {
+        // values this thread has just stored; W from the ring (first kWMax
+        // entries of the tile) or from global memory
+        const uint16_t* wrow = reinterpret_cast<const uint16_t*>(smem + C::kOffW + ws * C::kWSlot + nl * C::kWRow);
+        if (olo < ne && !mbar_wait(&wfull[ws], static_cast<uint32_t>(j / C::kWR) & 1u, abort_flag)) ok = false;
+        const int emid = min(ohi, max(olo, ne));
+        for (int e = olo; e < emid; ++e) patch_outlier(bt, outl[e], nl, wrow[lo8 + e]);
+        for (int e = emid; e < ohi; ++e) {  // past the ring: global memory
           const float4 o = outl[e];
           patch_outlier(bt, o, nl, wot_elem(args, j * 64 + nl, __float_as_int(o.y)));
-        }
-        if (j + 1 < nsteps) {
-#pragma unroll
-          for (int u = 0; u < C::kPrefetch; ++u)
-            if (olo + u < ohi) wpre[u] = wot_elem(args, (j + 1) * 64 + nl, __float_as_int(outl[olo + u].y));
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sempty[ls]);  // staging slot consumed
-        mbar_arrive(&bfull[b]);    // B slot written
+        mbar_arrive(&bfull[b]);                  // B slot written
+        if (ne > 0) mbar_arrive(&wempty[ws]);    // ring slot read
       }
       if (ctid == 0) QLIN_STEP(j, 4);
+    };
+    for (int j = 0; j < nsteps && ok; j += 2) {
+      step(j, in0);
+      if (j + 1 < nsteps) step(j + 1, in1);
     }
 
     // epilogue: TMEM lane = token, column = input

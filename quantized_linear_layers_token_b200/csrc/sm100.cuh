@@ -263,6 +263,12 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Arrive on `bar` (asynchronously, without raising its pending count) once
+// every cp.async this thread has issued so far has completed; the barrier's
+// expected count includes one such arrival per issuing thread.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // Generic-proxy smem writes must be made visible to the async proxy (the
 // tensor core reads operands through it) before signalling the MMA warp.
