@@ -1,7 +1,7 @@
 """Throughput of the outlier-aware W4A8 quantized linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--op forward|backward] [--tokens M]
 
 One step = one pass of the whole hot path -- targeted momentum update,
 per-token INT8 quantization, tcgen05 INT8 GEMM with the fused dequant and
@@ -23,6 +23,11 @@ so every replica keeps the same momentum state.
 
 ``--impl reference`` times the CPU oracle (single thread) on a bounded
 sample of the same workload and prints the same JSON line.
+
+``--op backward`` measures the fine-tuning input gradient instead: one step
+is qlin_backward_dx on every linear of the workload (default: the Phi-3-mini
+W8A8 linears of the Quaff notes) at --tokens tokens; metric TFLOP/s
+(2 M N K per linear) against the tensor-core roofline.
 """
 from __future__ import annotations
 
@@ -280,6 +285,257 @@ def run_profile_case(args, wl):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# --op backward: the input gradient under the straight-through estimator
+# ---------------------------------------------------------------------------
+
+BWD_METRIC = "input-gradient (straight-through estimator) TFLOP/s of the quantized linear layers"
+
+
+def bwd_flops(M, shapes):
+    return sum(2 * M * K * N for _, K, N in shapes)
+
+
+class OracleBackwardSample:
+    """The oracle's dX = (dY Weff^T) on a bounded sample: every linear of
+    the workload at ``rows`` token rows (the rows are independent)."""
+
+    def __init__(self, wl, rows):
+        from oracle import oracle
+        self.o = oracle
+        self.wl = wl
+        self.rows = rows
+        self.items = []
+        for si, (name, K, N) in enumerate(wl.shapes):
+            L = synth.layer(wl, si, M=1)
+            Wb = np.ascontiguousarray(L["W"]).view(np.uint16)
+            pk = oracle.pack_layer(Wb, L["O"], wl.fmt)
+            dY = np.ascontiguousarray(synth.grad_output(wl.index, si, rows, N)).view(np.uint16)
+            s = synth.outlier_scales(wl.index, si, len(L["O"]))
+            self.items.append((dY, Wb, pk, s))
+        self.flops = bwd_flops(rows, wl.shapes)
+
+    def step(self):
+        t0 = time.perf_counter()
+        for dY, Wb, pk, s in self.items:
+            self.o.backward_dx(dY, Wb, pk, s)
+        return time.perf_counter() - t0
+
+    def describe(self, seconds):
+        return (f"oracle backward_dx (fp64, single thread) on every linear of {self.wl.name} "
+                f"({len(self.items)}) at {self.rows} token rows; {seconds:.1f} s of CPU time; "
+                f"host has {os.cpu_count()} cores")
+
+
+def run_backward_reference(args, wl):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    sample = OracleBackwardSample(wl, 2)
+    for _ in range(args.warmup):
+        sample.step()
+    t = sum(sample.step() for _ in range(args.steps))
+    v = args.steps * sample.flops / t / 1e12
+    line = {
+        "impl": "reference", "metric": BWD_METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "op": "backward", "sample": f"all {len(wl.shapes)} linears at 2 token rows",
+                   "parallelism": "single thread"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": sample.describe(t / args.steps) + " (per step)"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_backward(args, wl):
+    """One step = qlin_backward_dx on every linear of the workload at
+    ``--tokens`` tokens (the fine-tuning backward through the frozen
+    quantized weights).  N > 1: every rank runs its own token batch, no
+    collective (the input gradient has no exchange step)."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    M = args.tokens
+    if args.profile_case:
+        # one linear, eager launches, so a profiler sees each kernel
+        si = [n for n, _, _ in wl.shapes].index(args.profile_case)
+        _, K, N = wl.shapes[si]
+        L = synth.layer(wl, si, M=1)
+        lay = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).to(device), L["O"], wl.fmt)
+        dY = torch.from_numpy(synth.grad_output(wl.index, si, M, N)).to(device)
+        s = torch.from_numpy(synth.outlier_scales(wl.index, si, len(L["O"]))).to(device) if len(L["O"]) else None
+        dX = torch.empty((M, K), dtype=torch.float16, device=device)
+        for _ in range(args.warmup):
+            qlin.qlin_backward_dx(lay.w, dY, M, s, dX)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            qlin.qlin_backward_dx(lay.w, dY, M, s, dX)
+        e1.record()
+        torch.cuda.synchronize()
+        qlin.qlin_poll_device_status()
+        us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
+        print(json.dumps({"profile_case": args.profile_case, "op": "backward", "workload": wl.name, "K": K, "N": N,
+                          "M": M, "us_per_call_eager": us, "tflops": 2 * M * N * K / us / 1e6}), flush=True)
+        return 0
+    slots = []
+    for si, (name, K, N) in enumerate(wl.shapes):
+        L = synth.layer(wl, si, M=1)
+        lay = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).to(device), L["O"], wl.fmt)
+        dY_np = synth.grad_output(wl.index, si, M, N)
+        s_np = synth.outlier_scales(wl.index, si, len(L["O"]))
+        slots.append({"layer": lay, "K": K, "N": N, "nO": len(L["O"]), "dY_np": dY_np,
+                      "dY": torch.from_numpy(dY_np).to(device),
+                      "s": torch.from_numpy(s_np).to(device) if len(L["O"]) else None,
+                      "dX": torch.empty((M, K), dtype=torch.float16, device=device)})
+    stream = torch.cuda.Stream(device)
+
+    def step():
+        for sl in slots:
+            qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], stream)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            graph.replay()
+    torch.cuda.synchronize()
+    qlin.qlin_poll_device_status()
+
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms_step], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    clocks = clk.summary()
+    flops = bwd_flops(M, wl.shapes)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # the step is nothing but backward_dx_kernel launches: their average
+    # duration is the step time over the launches of a step
+    hbm, bf16, bf16_sus, peak_kind = read_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_sus, "unit": "TFLOP/s",
+                "frac": achieved / bf16_sus, "frac_of_burst": achieved / bf16, "traffic": None,
+                "peak_source": f"bf16_tflops_sustained of {peak_kind} peaks (fp16 and bf16 have the same "
+                               f"dense tensor rate; kernel timed inside a seconds-long loop)",
+                "kernel": "backward_dx_kernel, all launches of one step", "flops_per_step": flops,
+                "launches_per_step": len(slots)}
+
+    e2e = None
+    if world == 1:
+        host_dy = [torch.from_numpy(sl["dY_np"]).pin_memory() for sl in slots]
+        host_dx = [torch.empty(sl["dX"].shape, dtype=torch.float16).pin_memory() for sl in slots]
+        h2d = sum(x.numel() * 2 for x in host_dy)
+        d2h = sum(y.numel() * 2 for y in host_dx)
+        h2d_stream = torch.cuda.Stream(device)
+        d2h_stream = torch.cuda.Stream(device)
+
+        def e2e_step():
+            h2d_stream.wait_stream(stream)
+            d2h_stream.wait_stream(stream)
+            ready = []
+            with torch.cuda.stream(h2d_stream):
+                for sl, hy in zip(slots, host_dy):
+                    sl["dY"].copy_(hy, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d_stream)
+                    ready.append(ev)
+            for sl, hx, ev in zip(slots, host_dx, ready):
+                stream.wait_event(ev)
+                qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], stream)
+                done = torch.cuda.Event()
+                done.record(stream)
+                d2h_stream.wait_event(done)
+                with torch.cuda.stream(d2h_stream):
+                    hx.copy_(sl["dX"], non_blocking=True)
+            stream.wait_stream(h2d_stream)
+            stream.wait_stream(d2h_stream)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+        torch.cuda.synchronize()
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g3, stream=stream):
+            e2e_step()
+        with torch.cuda.stream(stream):
+            g3.replay()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                g3.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = ev0.elapsed_time(ev1) / args.steps
+        e2e = {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "note": "per linear: pinned host dY -> device (copy stream), qlin_backward_dx (compute stream), "
+                       "device -> pinned host dX (second copy stream); one CUDA graph per step"}
+
+    cpu = None
+    if rank == 0 and world == 1:
+        sample = OracleBackwardSample(wl, 48)
+        t = sample.step()
+        cpu = {"value": sample.flops / t / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": sample.describe(t)}
+
+    if rank == 0:
+        dy_bytes = sum(sl["dY"].numel() * 2 for sl in slots)
+        line = {
+            "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16 (f32 accumulate)", "data": "synthetic",
+            "config": {"workload": wl.name, "op": "backward", "tokens": M,
+                       "shapes": [[n, K, N] for n, K, N in wl.shapes], "outlier_frac": wl.outlier_frac,
+                       "format": "W4A8 per-channel" if wl.fmt == 0 else ("W4A8 g128" if wl.fmt == 1 else "W8A8"),
+                       "l2": f"inputs larger than L2 (dY of one step {dy_bytes / 1e6:.0f} MB)",
+                       "parallelism": f"dp{world}",
+                       "timing": "CUDA graph of one step, CUDA events on the launch stream"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * len(slots),
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                       "reasons": clocks["reasons"], "samples": clocks["samples"]},
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -288,9 +544,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_w4_decode")
     ap.add_argument("--copies", type=int, default=4)
+    ap.add_argument("--op", default="forward", choices=["forward", "backward"],
+                    help="backward: the input gradient of every linear (default workload phi3_w8_quaff)")
+    ap.add_argument("--tokens", type=int, default=4096, help="--op backward: tokens per step")
     ap.add_argument("--profile-case", default=None,
                     help="NAME:M -- run only that linear of the workload at M tokens (for ncu captures)")
     args = ap.parse_args()
+    if args.op == "backward":
+        wl = synth.WORKLOADS["phi3_w8_quaff" if args.workload == "llama7b_w4_decode" else args.workload]
+        return run_backward_reference(args, wl) if args.impl == "reference" else run_backward(args, wl)
     wl = synth.WORKLOADS[args.workload]
 
     if args.impl == "reference":
