@@ -352,8 +352,6 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       }
     }
     named_bar_sync(1, 32 * C::kConvWarps);
-    const int olo = outl_lower_bound(outl, nout, 32 * g);  // the window's outlier entries
-    const int ohi = outl_lower_bound(outl, nout, 32 * g + 32);
     const int ne = min(nout, C::kWMax);  // entries served by the W_O ring
     const int lo8 = lo & 7;              // position of entry 0 in a ring row (fp16 units)
 
@@ -363,7 +361,10 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       if (ok && j >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(j / BS - 1) & 1u, abort_flag);
       if (ctid == 0) QLIN_STEP(j, 3);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) return;
+      if (!ok) {  // keep every converter thread on the same named barriers
+        if (nout > 0) named_bar_sync(1, 32 * C::kConvWarps);
+        return;
+      }
       unsigned char* bt = smem + C::kOffB + b * C::kBBytes;
       unsigned char* brow = bt + (nl >> 3) * kBwdSbo + sw * 128;
       // c'_n of the forward's INT8 operand: c_n / 16 for per-channel INT4 (16 q), else c_n
@@ -416,17 +417,24 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       }
       if (j + 2 < nsteps) load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
       const int ws = j % C::kWR;
-      if (olo < ohi) {
+      if (nout > 0) {
         // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i, on the
-        // values this thread has just stored; W from the ring (first kWMax
-        // entries of the tile) or from global memory
-        const uint16_t* wrow = reinterpret_cast<const uint16_t*>(smem + C::kOffW + ws * C::kWSlot + nl * C::kWRow);
-        if (olo < ne && !mbar_wait(&wfull[ws], static_cast<uint32_t>(j / C::kWR) & 1u, abort_flag)) ok = false;
-        const int emid = min(ohi, max(olo, ne));
-        for (int e = olo; e < emid; ++e) patch_outlier(bt, outl[e], nl, wrow[lo8 + e]);
-        for (int e = emid; e < ohi; ++e) {  // past the ring: global memory
-          const float4 o = outl[e];
-          patch_outlier(bt, o, nl, wot_elem(args, j * 64 + nl, __float_as_int(o.y)));
+        // converted values, once every thread has stored its window; the
+        // nout x 64 elements are spread over all converter threads.  W from
+        // the ring (first kWMax entries of the tile) or from global memory.
+        if (ok) ok = mbar_wait(&wfull[ws], static_cast<uint32_t>(j / C::kWR) & 1u, abort_flag);
+        named_bar_sync(1, 32 * C::kConvWarps);
+        if (ok) {
+          const unsigned char* ring = smem + C::kOffW + ws * C::kWSlot;
+          for (int t = ctid; t < nout * 64; t += 32 * C::kConvWarps) {
+            const int e = t >> 6;
+            const int q = t & 63;
+            const float4 o = outl[e];
+            uint16_t w;
+            if (e < ne) w = reinterpret_cast<const uint16_t*>(ring + q * C::kWRow)[lo8 + e];
+            else w = wot_elem(args, j * 64 + q, __float_as_int(o.y));
+            patch_outlier(bt, o, q, w);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -437,7 +445,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       }
       if (ctid == 0) QLIN_STEP(j, 4);
     };
-    for (int j = 0; j < nsteps && ok; j += 2) {
+    for (int j = 0; j < nsteps; j += 2) {  // every step, also after a failed wait (named barriers)
       step(j, in0);
       if (j + 1 < nsteps) step(j + 1, in1);
     }
