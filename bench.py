@@ -377,14 +377,16 @@ def run_backward(args, wl):
         dY = torch.from_numpy(synth.grad_output(wl.index, si, M, N)).to(device)
         s = torch.from_numpy(synth.outlier_scales(wl.index, si, len(L["O"]))).to(device) if len(L["O"]) else None
         dX = torch.empty((M, K), dtype=torch.float16, device=device)
+        nws = qlin.qlin_backward_dx_workspace(M, lay.w)
+        ws = qlin.empty_workspace(nws) if nws else None
         for _ in range(args.warmup):
-            qlin.qlin_backward_dx(lay.w, dY, M, s, dX)
+            qlin.qlin_backward_dx(lay.w, dY, M, s, dX, ws, nws)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(args.steps):
-            qlin.qlin_backward_dx(lay.w, dY, M, s, dX)
+            qlin.qlin_backward_dx(lay.w, dY, M, s, dX, ws, nws)
         e1.record()
         torch.cuda.synchronize()
         qlin.qlin_poll_device_status()
@@ -398,7 +400,9 @@ def run_backward(args, wl):
         lay = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).to(device), L["O"], wl.fmt)
         dY_np = synth.grad_output(wl.index, si, M, N)
         s_np = synth.outlier_scales(wl.index, si, len(L["O"]))
+        nws = qlin.qlin_backward_dx_workspace(M, lay.w)
         slots.append({"layer": lay, "K": K, "N": N, "nO": len(L["O"]), "dY_np": dY_np,
+                      "ws": qlin.empty_workspace(nws) if nws else None, "nws": nws,
                       "dY": torch.from_numpy(dY_np).to(device),
                       "s": torch.from_numpy(s_np).to(device) if len(L["O"]) else None,
                       "dX": torch.empty((M, K), dtype=torch.float16, device=device)})
@@ -406,7 +410,7 @@ def run_backward(args, wl):
 
     def step():
         for sl in slots:
-            qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], stream)
+            qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], sl["ws"], sl["nws"], stream)
 
     for _ in range(max(1, args.warmup)):
         step()
@@ -475,7 +479,7 @@ def run_backward(args, wl):
                     ready.append(ev)
             for sl, hx, ev in zip(slots, host_dx, ready):
                 stream.wait_event(ev)
-                qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], stream)
+                qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], sl["ws"], sl["nws"], stream)
                 done = torch.cuda.Event()
                 done.record(stream)
                 d2h_stream.wait_event(done)

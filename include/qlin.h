@@ -262,12 +262,18 @@ QLIN_API qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weigh
  *   s   fp32 [n_outlier], device: the scales of the forward pass whose
  *       gradient this is (ignored and may be NULL when n_outlier = 0).
  *   dX  fp16 [M][K] row-major, device, fully overwritten.
+ *   workspace  optional (NULL, or smaller than qlin_backward_dx_workspace):
+ *       with it, the tiles of an incomplete last wave of SMs are split along
+ *       the reduction and their fp32 partials pass through it; it must be
+ *       zero-filled before its first use and is left that way.
  * Arithmetic: Weff is rounded to fp16 (the outlier rows after blending in
- * fp32), products are summed in fp32 on the tensor cores, dX is rounded to
- * fp16 once.  No workspace.  M = 0 is a no-op; M above 65535 * 128 returns
- * QLIN_ERR_SHAPE; pointers must be 16-byte aligned (QLIN_ERR_ALIGN). */
+ * fp32), products are summed in fp32 on the tensor cores (split tiles add
+ * their fp32 partials), dX is rounded to fp16 once.  M = 0 is a no-op; M
+ * above 65535 * 128 returns QLIN_ERR_SHAPE; pointers must be 16-byte aligned
+ * and the workspace 256-byte aligned (QLIN_ERR_ALIGN). */
+QLIN_API qlin_status qlin_backward_dx_workspace(int32_t M, const qlin_weights* w, size_t* bytes);
 QLIN_API qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t M, const float* s,
-                                      uint16_t* dX, void* stream);
+                                      uint16_t* dX, void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, then reports and clears the device error word that
  * kernels set when a bounded wait gives up: QLIN_ERR_TIMEOUT if it was set,

@@ -48,6 +48,17 @@ struct BwdArgs {
   int kbs;     // 128-input code blocks per channel tile (ceil(K / 128))
   int nib;     // 64-outlier blocks of W_O^T per channel tile (ceil(nO / 64))
   int nsteps;  // 64-channel reduction steps (ceil(N / 64))
+  // Work units (one CTA each): tiles [0, full) whole, then every remaining
+  // ("tail") tile as tsplit ranges of the reduction steps.  Tiles are
+  // numbered input tile fastest: tile t covers inputs 256 (t % ntk) and
+  // tokens 256 (t / ntk).  The last range of a tail tile adds the fp32
+  // partials of the other ranges (part, [tail][tsplit-1][256][256]) once
+  // their CTAs have counted in cnt[tail] (zero on entry, left zero).
+  int ntk;
+  int full;
+  int tsplit;
+  float* part;
+  unsigned* cnt;
 };
 
 template <int FMT>
@@ -210,11 +221,22 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int k0 = blockIdx.x * 256;
-  const int m0 = blockIdx.y * 256;
+  // this CTA's work unit: a whole tile, or reduction range sp of tail tile tt
+  int tile = static_cast<int>(blockIdx.x), sp = 0, S = 1, tt = -1;
+  if (tile >= args.full) {
+    const int u = tile - args.full;
+    S = args.tsplit;
+    tt = u / S;
+    sp = u - tt * S;
+    tile = args.full + tt;
+  }
+  const int k0 = (tile % args.ntk) * 256;
+  const int m0 = (tile / args.ntk) * 256;
   const bool two = m0 + 128 < args.M;  // the second 128-token half holds tokens
-  const int nsteps = args.nsteps;
-  const int nb = (2 * static_cast<int>(blockIdx.x) + 1 < args.kbs) ? 2 : 1;  // code blocks in this input tile
+  const int j0 = sp * args.nsteps / S;  // channel steps [j0, j0 + nst) of N / 64
+  const int nst = (sp + 1) * args.nsteps / S - j0;
+  const int kb0 = k0 >> 7;  // first code block of the tile
+  const int nb = (kb0 + 1 < args.kbs) ? 2 : 1;  // code blocks in this input tile
 #ifdef QLIN_TRACE
   long long* const qlin_st = (blockIdx.x == 0 && blockIdx.y == 0) ? g_steps : nullptr;
 #endif
@@ -251,12 +273,12 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     if (lane == 0) {
       griddep_wait();  // dY comes from the previous kernel
       int issued = 0;
-      for (int j = 0; j < nsteps; ++j) {
-        const int a = j % AS;
-        if (j >= AS && !mbar_wait(&aempty[a], static_cast<uint32_t>(j / AS - 1) & 1u, abort_flag)) break;
+      for (int jj = 0; jj < nst; ++jj) {
+        const int a = jj % AS;
+        if (jj >= AS && !mbar_wait(&aempty[a], static_cast<uint32_t>(jj / AS - 1) & 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&afull[a], C::kABytes);
-        tma_load_2d(smem + C::kOffA + a * C::kABytes, &tmDY, &afull[a], j * 64, m0);
-        QLIN_STEP(j, 1);
+        tma_load_2d(smem + C::kOffA + a * C::kABytes, &tmDY, &afull[a], (j0 + jj) * 64, m0);
+        QLIN_STEP(jj, 1);
         ++issued;
       }
       drain_ring(afull, AS, issued);
@@ -265,7 +287,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(128, 256) | (1u << 16);  // B MN-major
-      for (int j = 0; j < nsteps; ++j) {
+      for (int j = 0; j < nst; ++j) {  // j counts this CTA's steps
         const int a = j % AS;
         const int b = j % BS;
         if (!mbar_wait(&afull[a], static_cast<uint32_t>(j / AS) & 1u, abort_flag)) break;
@@ -305,15 +327,15 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     if (ne > 0) {
       const int cf = lo >> 3;                        // first 8-outlier chunk
       const int nch = ((lo + ne - 1) >> 3) - cf + 1;  // chunks per channel row, <= kWChunks
-      for (int j = 0; j < nsteps; ++j) {
-        const int slot = j % C::kWR;
-        if (j >= C::kWR && !mbar_wait(&wempty[slot], static_cast<uint32_t>(j / C::kWR - 1) & 1u, abort_flag)) break;
+      for (int jj = 0; jj < nst; ++jj) {
+        const int slot = jj % C::kWR;
+        if (jj >= C::kWR && !mbar_wait(&wempty[slot], static_cast<uint32_t>(jj / C::kWR - 1) & 1u, abort_flag)) break;
         unsigned char* dst = smem + C::kOffW + slot * C::kWSlot;
         for (int t = lane; t < 64 * nch; t += 32) {
           const int q = t / nch;
           const int cix = t - q * nch;
           const int kc = cf + cix;
-          const int n = j * 64 + q;
+          const int n = (j0 + jj) * 64 + q;
           const int r = n & 127;
           const uint16_t* src = args.wot + (static_cast<size_t>(n >> 7) * args.nib + (kc >> 3)) * 8192 + r * 64 +
                                 (((kc & 7) ^ (r & 7)) << 3);
@@ -327,7 +349,6 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     // ------------------------------------------- converters, then epilogue
     const int cw = warp - 3;             // 0..15
     const int ctid = threadIdx.x - 96;   // 0..511
-    const int kb0 = 2 * static_cast<int>(blockIdx.x);
     // Each thread converts one 32-input window (inputs 32 g .. 32 g + 31 of
     // the tile) of one channel row per step and blends the outlier rows that
     // fall inside it, so no thread waits for another before the arrival.
@@ -336,8 +357,8 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     const int g = cw >> 1;                // window, 0..7
     const int sw = nl & 7;
     BwdIn<FMT> in0, in1;
-    load_step<FMT>(in0, args, 0, nl, g, kb0, nb);
-    if (nsteps > 1) load_step<FMT>(in1, args, 1, nl, g, kb0, nb);
+    load_step<FMT>(in0, args, j0, nl, g, kb0, nb);
+    if (nst > 1) load_step<FMT>(in1, args, j0 + 1, nl, g, kb0, nb);
 
     griddep_wait();  // s comes from the forward
     int nout = 0, lo = 0;
@@ -356,10 +377,12 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     const int lo8 = lo & 7;              // position of entry 0 in a ring row (fp16 units)
 
     bool ok = true;
-    auto step = [&](int j, BwdIn<FMT>& in) {
-      const int b = j % BS;
-      if (ok && j >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(j / BS - 1) & 1u, abort_flag);
-      if (ctid == 0) QLIN_STEP(j, 3);
+    // jj counts this CTA's steps, j = j0 + jj is the channel step
+    auto step = [&](int jj, BwdIn<FMT>& in) {
+      const int j = j0 + jj;
+      const int b = jj % BS;
+      if (ok && jj >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(jj / BS - 1) & 1u, abort_flag);
+      if (ctid == 0) QLIN_STEP(jj, 3);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {  // keep every converter thread on the same named barriers
         if (nout > 0) named_bar_sync(1, 32 * C::kConvWarps);
@@ -415,14 +438,14 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
         }
       }
-      if (j + 2 < nsteps) load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
-      const int ws = j % C::kWR;
+      if (jj + 2 < nst) load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
+      const int ws = jj % C::kWR;
       if (nout > 0) {
         // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i, on the
         // converted values, once every thread has stored its window; the
         // nout x 64 elements are spread over all converter threads.  W from
         // the ring (first kWMax entries of the tile) or from global memory.
-        if (ok) ok = mbar_wait(&wfull[ws], static_cast<uint32_t>(j / C::kWR) & 1u, abort_flag);
+        if (ok) ok = mbar_wait(&wfull[ws], static_cast<uint32_t>(jj / C::kWR) & 1u, abort_flag);
         named_bar_sync(1, 32 * C::kConvWarps);
         if (ok) {
           const unsigned char* ring = smem + C::kOffW + ws * C::kWSlot;
@@ -443,43 +466,117 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
         mbar_arrive(&bfull[b]);                  // B slot written
         if (ne > 0) mbar_arrive(&wempty[ws]);    // ring slot read
       }
-      if (ctid == 0) QLIN_STEP(j, 4);
+      if (ctid == 0) QLIN_STEP(jj, 4);
     };
-    for (int j = 0; j < nsteps; j += 2) {  // every step, also after a failed wait (named barriers)
-      step(j, in0);
-      if (j + 1 < nsteps) step(j + 1, in1);
+    for (int jj = 0; jj < nst; jj += 2) {  // every step, also after a failed wait (named barriers)
+      step(jj, in0);
+      if (jj + 1 < nst) step(jj + 1, in1);
     }
 
-    // epilogue: TMEM lane = token, column = input
+    // epilogue: TMEM lane = token, column = input.  Thread (quadrant qd,
+    // lane) owns token row qd * 32 + lane of each half; warp quarter
+    // `quarter` owns 64 input columns, read in 16-column chunks.
     const bool got = ok && mbar_wait(acc_full, 0u, abort_flag);
-    if (__all_sync(0xffffffffu, got && *abort_flag == 0)) {
-      tc_fence_after();
-      const int qd = warp & 3;  // TMEM lane quadrant of this warp
-      const int quarter = cw >> 2;  // 64 input columns per warp, in both token halves
+    const bool live = __all_sync(0xffffffffu, got && *abort_flag == 0);
+    const int qd = warp & 3;  // TMEM lane quadrant of this warp
+    const int quarter = cw >> 2;
+    const int nch = two ? 8 : 4;  // 16-column chunks of this thread
+    auto chunk_of = [&](int c, int& h, int& col, int& row) {
+      h = c >> 2;
+      col = quarter * 64 + (c & 3) * 16;
+      row = h * 128 + qd * 32 + lane;  // row within the tile
+    };
+    auto load_acc = [&](int h, int col, float (&v)[16]) {
+      uint32_t r[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(h * 256 + col), r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]);
+    };
+    auto store_dx = [&](int row, int col, const float (&v)[16]) {
+      const int m = m0 + row;
+      const int k = k0 + col;
+      if (m < args.M && k < args.K) {
+        uint32_t hw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) hw[e] = h2_as_u32(__floats2half2_rn(v[2 * e], v[2 * e + 1]));
+        uint4* dst = reinterpret_cast<uint4*>(args.dX + static_cast<size_t>(m) * args.K + k);
+        dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+      }
+    };
+    if (S == 1) {
+      if (live) {
+        tc_fence_after();
 #pragma unroll 1
-      for (int jj = 0; jj < (two ? 4 : 2); ++jj) {
-        const int h = jj >> 1;
-        const int col = quarter * 64 + (jj & 1) * 32;
-        const int m = m0 + h * 128 + qd * 32 + lane;
-        uint32_t v0[16], v1[16];
-        const uint32_t ta =
-            tmem + (static_cast<uint32_t>(qd * 32) << 16) + static_cast<uint32_t>(h * 256 + col);
-        tmem_ld16(ta, v0);
-        tmem_ld16(ta + 16, v1);
-        tmem_ld_wait();
-        const int k = k0 + col;
-        if (m < args.M && k < args.K) {
-          uint32_t hw[16];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            hw[e] = h2_as_u32(__floats2half2_rn(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1])));
-            hw[8 + e] = h2_as_u32(__floats2half2_rn(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1])));
-          }
-          uint4* dst = reinterpret_cast<uint4*>(args.dX + static_cast<size_t>(m) * args.K + k);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(hw[4 * e], hw[4 * e + 1], hw[4 * e + 2], hw[4 * e + 3]);
+        for (int c = 0; c < nch; ++c) {
+          int h, col, row;
+          chunk_of(c, h, col, row);
+          float v[16];
+          load_acc(h, col, v);
+          store_dx(row, col, v);
         }
       }
+    } else if (sp < S - 1) {
+      // a leading range of a tail tile: publish the fp32 partial, then count
+      float* mine = args.part + (static_cast<size_t>(tt) * (S - 1) + sp) * 65536;
+      if (live) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+          int h, col, row;
+          chunk_of(c, h, col, row);
+          float v[16];
+          load_acc(h, col, v);
+          float4* dst = reinterpret_cast<float4*>(mine + row * 256 + col);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, 32 * C::kConvWarps);
+      if (ctid == 0 && live) atomicAdd(args.cnt + tt, 1u);
+    } else {
+      // the last range of a tail tile: wait (bounded) until the other
+      // ranges have counted, add their partials, store dX, reset the count
+      if (ctid == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(args.cnt + tt) < static_cast<unsigned>(S - 1)) {
+          if (*abort_flag || globaltimer_ns() - t0 > QLIN_WAIT_NS) {
+            *abort_flag = 1;
+            atomicExch(&g_device_error, kDevErrTimeout);
+            break;
+          }
+          __nanosleep(256);
+        }
+      }
+      named_bar_sync(1, 32 * C::kConvWarps);
+      fence_acq_rel_gpu();
+      if (live && *abort_flag == 0) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+          int h, col, row;
+          chunk_of(c, h, col, row);
+          float v[16];
+          load_acc(h, col, v);
+          for (int r = 0; r < S - 1; ++r) {
+            const float4* src =
+                reinterpret_cast<const float4*>(args.part + (static_cast<size_t>(tt) * (S - 1) + r) * 65536 + row * 256 + col);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float4 p = __ldcg(src + e);
+              v[4 * e] += p.x;
+              v[4 * e + 1] += p.y;
+              v[4 * e + 2] += p.z;
+              v[4 * e + 3] += p.w;
+            }
+          }
+          store_dx(row, col, v);
+        }
+      }
+      named_bar_sync(1, 32 * C::kConvWarps);
+      if (ctid == 0) args.cnt[tt] = 0u;
     }
   }
   tc_fence_before();

@@ -580,6 +580,45 @@ qlin_status noalloc_scratch(unsigned** out) {
 }
 
 // ---------------------------------------------------------------- backward
+// Work plan of the input gradient: whole 256 x 256 tiles fill complete
+// waves of one CTA per SM; when the grid is under two waves, the tiles of
+// the ragged last wave are split into tsplit ranges of the channel steps (at
+// most 8, at most one range per step) so that wave has as many CTAs as SMs,
+// and their fp32 partials go through the workspace.  Without a workspace
+// every tile is whole.
+struct BwdPlan {
+  int ntk, tiles, full, tsplit;
+  size_t part_off, cnt_off, bytes;
+};
+
+BwdPlan plan_backward(int M, const qlin_weights* w, bool split) {
+  BwdPlan p{};
+  p.ntk = (w->K + 255) / 256;
+  p.tiles = p.ntk * ((M + 255) / 256);
+  p.full = p.tiles;
+  p.tsplit = 1;
+  const int sms = sm_count();
+  const int nsteps = (w->N + 63) / 64;
+  const int tail = p.tiles % sms;
+  // only below two waves: with more, CTAs of different lengths already
+  // interleave across the wave boundaries and the partials cost more than
+  // the idle SMs of the last wave (measured on 3.5-wave grids)
+  if (split && tail > 0 && p.tiles < 2 * sms) {
+    int S = sms / tail;
+    if (S > 8) S = 8;
+    if (S > nsteps) S = nsteps;
+    if (S >= 2) {
+      p.full = p.tiles - tail;
+      p.tsplit = S;
+    }
+  }
+  const int ntail = p.tiles - p.full;
+  p.part_off = 0;
+  p.cnt_off = round_up(size_t(ntail) * (p.tsplit - 1) * 65536 * 4, kAlign);
+  p.bytes = ntail ? round_up(p.cnt_off + size_t(ntail) * 4, kAlign) : 0;
+  return p;
+}
+
 template <int FMT>
 qlin_status launch_backward_t(const CUtensorMap& tm, const BwdArgs& args, cudaStream_t stream) {
   using C = BwdCfg<FMT>;
@@ -590,7 +629,7 @@ qlin_status launch_backward_t(const CUtensorMap& tm, const BwdArgs& args, cudaSt
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  const dim3 grid(static_cast<unsigned>((args.K + 255) / 256), static_cast<unsigned>((args.M + 255) / 256));
+  const dim3 grid(static_cast<unsigned>(args.full + (args.ntk * ((args.M + 255) / 256) - args.full) * args.tsplit));
   cudaError_t e = launch_k(kern, grid, dim3(C::kThreads), C::kSmemBytes, stream, tm, args);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "backward_dx_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
@@ -816,13 +855,23 @@ qlin_status qlin_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, c
   return launch_gemm(w, Xq, a, M, Y, acc_debug, gws, stream);
 }
 
+qlin_status qlin_backward_dx_workspace(int32_t M, const qlin_weights* w, size_t* bytes) {
+  qlin_status st = check_weights(w);
+  if (st != QLIN_OK) return st;
+  if (!bytes || M < 0) return fail(QLIN_ERR_ARG, "bad arguments");
+  *bytes = M > 0 ? plan_backward(M, w, true).bytes : 0;
+  return QLIN_OK;
+}
+
 qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t M, const float* s, uint16_t* dX,
-                             void* stream_) {
+                             void* workspace, size_t ws_bytes, void* stream_) {
   qlin_status st = check_weights(w);
   if (st != QLIN_OK) return st;
   if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
   if (M > 65535 * 128) return fail(QLIN_ERR_SHAPE, "M=%d exceeds %d", M, 65535 * 128);
   if (M == 0) return QLIN_OK;
+  if (workspace && reinterpret_cast<uintptr_t>(workspace) % kAlign)
+    return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
   const int nO = w->n_outlier;
   if (!dY || !dX) return fail(QLIN_ERR_ARG, "dY/dX is NULL");
   if (nO > 0 && !s) return fail(QLIN_ERR_ARG, "s is NULL with n_outlier=%d", nO);
@@ -848,6 +897,15 @@ qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t 
   args.kbs = (w->K + 127) / 128;
   args.nib = (nO + 63) / 64;
   args.nsteps = (w->N + 63) / 64;
+  // the split plan needs the whole workspace it asks for; with none (or a
+  // smaller one) every tile runs whole
+  BwdPlan p = plan_backward(M, w, true);
+  if (p.bytes && (!workspace || ws_bytes < p.bytes)) p = plan_backward(M, w, false);
+  args.ntk = p.ntk;
+  args.full = p.full;
+  args.tsplit = p.tsplit;
+  args.part = p.bytes ? reinterpret_cast<float*>(static_cast<char*>(workspace) + p.part_off) : nullptr;
+  args.cnt = p.bytes ? reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + p.cnt_off) : nullptr;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   switch (w->fmt) {
     case QLIN_W4_PERCHANNEL: return launch_backward_t<kFmtW4PC>(tm, args, stream);

@@ -247,6 +247,11 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // observed the last arrival, acquires the other CTAs' stores for the whole
 // CTA once the barrier behind it is passed).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ unsigned atom_add_relaxed_gpu(unsigned* p, unsigned v) {
   unsigned old;

@@ -29,6 +29,7 @@ EXPORTED = [
     "qlin_pack_weights", "qlin_quant_act_workspace", "qlin_quant_act", "qlin_outlier_colmax",
     "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
     "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc", "qlin_backward_dx",
+    "qlin_backward_dx_workspace",
 ]
 
 
@@ -82,7 +83,8 @@ def lib() -> ctypes.CDLL:
             "qlin_forward": [P, I32, W, P, F32, I32, P, P, SZ, P],
             "qlin_poll_device_status": [P],
             "qlin_quant_act_noalloc": [P, I32, W, P, F32, I32, P, P, P, P],
-            "qlin_backward_dx": [W, P, I32, P, P, P],
+            "qlin_backward_dx": [W, P, I32, P, P, P, SZ, P],
+            "qlin_backward_dx_workspace": [I32, W, ctypes.POINTER(SZ)],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -189,9 +191,13 @@ def qlin_forward(X, M: int, w: qlin_weights, s, gamma: float, update_momentum: b
                               _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)), "qlin_forward")
 
 
-def qlin_backward_dx(w: qlin_weights, dY, M: int, s, dX, stream=None):
-    _check(lib().qlin_backward_dx(ctypes.byref(w), _ptr(dY), M, _ptr(s), _ptr(dX), _stream(stream)),
-           "qlin_backward_dx")
+def qlin_backward_dx_workspace(M: int, w: qlin_weights) -> int:
+    return _size(lib().qlin_backward_dx_workspace, M, ctypes.byref(w))
+
+
+def qlin_backward_dx(w: qlin_weights, dY, M: int, s, dX, workspace=None, ws_bytes: int = 0, stream=None):
+    _check(lib().qlin_backward_dx(ctypes.byref(w), _ptr(dY), M, _ptr(s), _ptr(dX), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "qlin_backward_dx")
 
 
 def qlin_poll_device_status(stream=None):

@@ -112,6 +112,9 @@ def test_backward_argument_errors(q):
     n = q.qlin_weights_bytes(K, N, 0, nO)
     w = q.qlin_weights_bind(K, N, 0, nO, 1 << 20, n)
     q.qlin_backward_dx(w, None, 0, None, None, stream=0)  # M = 0: nothing to do
+    assert q.qlin_backward_dx_workspace(0, w) == 0
+    # 4096 tokens x 512 inputs = 32 tiles < one wave: split, so a workspace is asked for
+    assert q.qlin_backward_dx_workspace(4096, w) > 0
     for dY, M, s, status in [
         (1 << 24, -1, 1 << 25, "QLIN_ERR_ARG"),
         (None, 4, 1 << 25, "QLIN_ERR_ARG"),
@@ -122,3 +125,6 @@ def test_backward_argument_errors(q):
         with pytest.raises(q.QlinError) as e:
             q.qlin_backward_dx(w, dY, M, s, 1 << 26, stream=0)
         assert q.STATUS[e.value.status] == status
+    with pytest.raises(q.QlinError) as e:  # a workspace off the 256-byte grid
+        q.qlin_backward_dx(w, 1 << 24, 4, 1 << 25, 1 << 26, (1 << 27) + 16, 1 << 20, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_ALIGN"

@@ -58,17 +58,49 @@ def w_eff_fp16(pk, W, s):
     return W16.astype(np.float64)
 
 
-def run(q, W, O, fmt, dY, s):
+def run(q, W, O, fmt, dY, s, workspace=False):
+    """dX from the GPU; with workspace=True the tiles of an incomplete last
+    wave are split along the reduction (fp32 partials through it), and the
+    call is made twice to check that the workspace is left ready for reuse."""
     K, N = W.shape
     M = dY.shape[0]
     layer = q.PackedLayer.pack(torch.from_numpy(W).cuda(), O, fmt)
     dYd = torch.from_numpy(dY).cuda()
     sd = torch.from_numpy(s).cuda() if len(O) else None
     dX = torch.full((M, K), float("nan"), dtype=torch.float16, device="cuda")
-    q.qlin_backward_dx(layer.w, dYd, M, sd, dX)
+    ws, nws = None, 0
+    if workspace:
+        nws = q.qlin_backward_dx_workspace(M, layer.w)
+        ws = q.empty_workspace(nws) if nws else None
+    q.qlin_backward_dx(layer.w, dYd, M, sd, dX, ws, nws)
+    if workspace:
+        first = dX.clone()
+        dX.fill_(float("nan"))
+        q.qlin_backward_dx(layer.w, dYd, M, sd, dX, ws, nws)
     q.qlin_poll_device_status()
     torch.cuda.synchronize()
+    if workspace:
+        assert torch.equal(first, dX), "second call with the same workspace differs"
+        cnt = split_counters(ws, M, K, N) if ws is not None else None
+        if cnt is not None:
+            assert not cnt.any().item(), "split-tile counters not left zeroed"
     return dX.float().cpu().numpy().astype(np.float64)
+
+
+def split_counters(ws, M, K, N):
+    """The per-tile counters of the split plan (workspace layout: fp32
+    partials of the split tiles, then one counter per split tile), or None
+    when the call splits nothing."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tiles = -(-K // 256) * -(-M // 256)
+    tail = tiles % sms
+    if tail == 0 or tiles >= 2 * sms:
+        return None
+    S = min(sms // tail, 8, -(-N // 64))
+    if S < 2:
+        return None
+    cnt_off = -(-(tail * (S - 1) * 65536 * 4) // 256) * 256
+    return ws[cnt_off:cnt_off + tail * 4]
 
 
 def check(dX, dY, W, pk, s, oracle, rows=None):
@@ -142,7 +174,7 @@ def test_backward_fullsize_sampled(q, oracle, wl_name, shape_idx):
     N = W.shape[1]
     dY = synth.grad_output(wl.index, shape_idx, M, N)
     s = synth.outlier_scales(wl.index, shape_idx, len(O))
-    dX = run(q, W, O, wl.fmt, dY, s)
+    dX = run(q, W, O, wl.fmt, dY, s, workspace=True)
     pk = oracle.pack_layer(bits(W), O, wl.fmt)
     rows = np.array([0, 127, 700, 1301, 1920, M - 1])
     check(dX, dY, W, pk, s, oracle, rows=rows)
@@ -160,6 +192,24 @@ def test_backward_maximum_k(q, oracle):
         dX = run(q, W, O, fmt, dY, s)
         pk = oracle.pack_layer(bits(W), O, fmt)
         check(dX, dY, W, pk, s, oracle, rows=np.array([0, 64, 129]))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,K,N,nO", [
+    (200, 640, 208, 37),    # 3 tiles: each split into ranges of the 4 channel steps
+    (520, 1536, 1024, 41),  # 18 tiles, 8 ranges each (with a ragged token tile)
+])
+def test_backward_split_tiles(q, oracle, fmt, M, K, N, nO):
+    """With a workspace, the tiles of an incomplete wave are split along the
+    reduction; the last range adds the others' fp32 partials."""
+    L = synth.layer("small", 0, M=1, K=K, N=N, n_outliers=nO)
+    W, O = L["W"], L["O"]
+    dY = synth.grad_output(0, 4, M, N)
+    s = synth.outlier_scales(0, 4, nO)
+    dX = run(q, W, O, fmt, dY, s, workspace=True)
+    pk = oracle.pack_layer(bits(W), O, fmt)
+    rows = np.unique(np.concatenate([np.arange(0, M, 37), [M - 1]])).astype(np.int64)
+    check(dX, dY, W, pk, s, oracle, rows=rows)
 
 
 def test_backward_zero_tokens_and_repeat(q):
