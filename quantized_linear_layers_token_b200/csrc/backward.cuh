@@ -28,8 +28,12 @@
 //       the conversion needs no transpose;
 //   warp 1 issues eight 128 x 256 x 16 MMAs per step (each B slice serves
 //   both 128-token halves, so a code block is converted once per 256 tokens).
-// The outlier rows are blended into B by the thread that converted them; the
-// converter warps then read the accumulators back and store fp16 dX rows.
+// In a tile with outliers, all converter threads then blend the outlier rows
+// into B (after one barrier per step), with the W_O values streamed into a
+// shared ring by warp 2.  The converter warps finally read the accumulators
+// back and store fp16 dX rows.  When the grid is under two waves, the tiles of
+// the last, incomplete wave are split into ranges of the channel steps whose
+// fp32 partials meet in a workspace.
 #pragma once
 
 #include "gemm.cuh"
@@ -350,9 +354,9 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     const int cw = warp - 3;             // 0..15
     const int ctid = threadIdx.x - 96;   // 0..511
     // Each thread converts one 32-input window (inputs 32 g .. 32 g + 31 of
-    // the tile) of one channel row per step and blends the outlier rows that
-    // fall inside it, so no thread waits for another before the arrival.
-    // Its codes, channel scale and ratio are loaded two steps ahead.
+    // the tile) of one channel row per step; its codes, channel scale and
+    // ratio are loaded two steps ahead.  The outlier rows are blended after
+    // the conversion by all threads together (below).
     const int nl = (cw & 1) * 32 + lane;  // channel row of the step
     const int g = cw >> 1;                // window, 0..7
     const int sw = nl & 7;
