@@ -1,0 +1,49 @@
+"""bench.py's reference arm (the CPU oracle on a bounded sample) runs without
+a GPU: its JSON line carries every field of the bench contract, for the
+forward and the input-gradient measurement."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+KEYS = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"]
+
+
+@pytest.mark.parametrize("extra,unit", [([], "GB/s"), (["--op", "backward"], "TFLOP/s")])
+def test_reference_arm_json_line(extra, unit):
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0", *extra],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in KEYS:
+        assert k in d, k
+    assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
+    assert d["higher_is_better"] is True and d["data"] == "synthetic" and "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["unit"] == unit and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_algorithmic_bytes_by_hand():
+    """The bytes each stage must move at least once, counted by hand for
+    LLaMA-2-7B q_proj at 16 tokens with 41 outlier channels."""
+    sys.path.insert(0, ROOT)
+    import bench
+    # GEMM: INT4 weights 8 MiB, c 16 KiB, W_O 41 x 4096 fp16, Xq 64 KiB,
+    # a 64 B, XqO 656 B, Y 16 x 4096 fp16
+    assert bench.algorithmic_bytes(16, 4096, 4096, 41, 0) == (
+        8388608 + 16384 + 335872 + 65536 + 64 + 656 + 131072,
+        # quantization: read X (128 KiB), write Xq, a and XqO
+        131072 + 65536 + 64 + 656)
+    # g128 adds the fp16 ratios (32 groups x 4096); INT8 weights are 16 MiB
+    g, _ = bench.algorithmic_bytes(16, 4096, 4096, 41, 1)
+    assert g == 8388608 + 16384 + 262144 + 335872 + 65536 + 64 + 656 + 131072
+    g, _ = bench.algorithmic_bytes(16, 4096, 4096, 41, 2)
+    assert g == 16777216 + 16384 + 335872 + 65536 + 64 + 656 + 131072
