@@ -548,6 +548,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_w4_decode")
     ap.add_argument("--copies", type=int, default=4)
+    ap.add_argument("--streams", type=int, default=1,
+                    help="compute streams the independent forwards of a step are spread over (N = 1)")
     ap.add_argument("--op", default="forward", choices=["forward", "backward"],
                     help="backward: the input gradient of every linear (default workload phi3_w8_quaff)")
     ap.add_argument("--tokens", type=int, default=4096, help="--op backward: tokens per step")
@@ -601,10 +603,30 @@ def main():
     from quantized_linear_layers_token_b200.dp import ColmaxExchange
     xchg = ColmaxExchange([len(meta[sl["si"]]["O"]) for sl in slots], device)
 
+    # Independent forwards of a step go round-robin to --streams compute
+    # streams forked from (and joined back into) the launch stream, so one
+    # GEMM's tail overlaps the next one's weight streaming on other SMs.
+    nstreams = max(1, args.streams) if world == 1 else 1
+    side = [torch.cuda.Stream(device) for _ in range(nstreams - 1)]
+
     def step_single():
-        for sl in slots:
+        if nstreams == 1:
+            for sl in slots:
+                qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
+                                  sl["nws"], stream)
+            return
+        streams = [stream] + side
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for st in side:
+            st.wait_event(fork)
+        for j, sl in enumerate(slots):
             qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
-                              sl["nws"], stream)
+                              sl["nws"], streams[j % nstreams])
+        for st in side:
+            done = torch.cuda.Event()
+            done.record(st)
+            stream.wait_event(done)
 
     def step_dp():
         for j, sl in enumerate(slots):
@@ -816,7 +838,8 @@ def main():
                        "outlier_frac": wl.outlier_frac, "gamma": wl.gamma, "format": "W4A8 per-channel"
                        if wl.fmt == 0 else ("W4A8 g128" if wl.fmt == 1 else "W8A8"),
                        "parallelism": f"dp{world}", "forwards_per_step": len(slots),
-                       "timing": "CUDA graph of one step, CUDA events on the launch stream"},
+                       "timing": "CUDA graph of one step, CUDA events on the launch stream",
+                       "streams": nstreams},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
