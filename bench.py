@@ -21,6 +21,12 @@ the same step on its own token batch with replicated weights; the outlier
 column maxima of all linears are combined with one all-reduce(MAX) per step
 so every replica keeps the same momentum state.
 
+The forwards of a step are independent (every linear at every token
+count), so on one GPU they are spread round-robin over --streams compute
+streams (default 4): one GEMM's tail then overlaps the next one's weight
+streaming on other SMs.  The roofline line times the GEMMs one after
+another on a single stream, so its per-launch figure is unaffected.
+
 ``--impl reference`` times the CPU oracle (single thread) on a bounded
 sample of the same workload and prints the same JSON line.
 
@@ -548,7 +554,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama7b_w4_decode")
     ap.add_argument("--copies", type=int, default=4)
-    ap.add_argument("--streams", type=int, default=1,
+    ap.add_argument("--streams", type=int, default=4,
                     help="compute streams the independent forwards of a step are spread over (N = 1)")
     ap.add_argument("--op", default="forward", choices=["forward", "backward"],
                     help="backward: the input gradient of every linear (default workload phi3_w8_quaff)")
@@ -771,15 +777,25 @@ def main():
                     ev = torch.cuda.Event()
                     ev.record(h2d_stream)
                     ready.append(ev)
-            for sl, hy, ev in zip(slots, host_y, ready):
-                stream.wait_event(ev)
+            streams = [stream] + side
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            for st in side:
+                st.wait_event(fork)
+            for j, (sl, hy, ev) in enumerate(zip(slots, host_y, ready)):
+                cs = streams[j % nstreams]
+                cs.wait_event(ev)
                 qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
-                                  sl["nws"], stream)
+                                  sl["nws"], cs)
                 done = torch.cuda.Event()
-                done.record(stream)
+                done.record(cs)
                 d2h_stream.wait_event(done)
                 with torch.cuda.stream(d2h_stream):
                     hy.copy_(sl["Y"], non_blocking=True)
+            for st in side:
+                joined = torch.cuda.Event()
+                joined.record(st)
+                stream.wait_event(joined)
             stream.wait_stream(h2d_stream)
             stream.wait_stream(d2h_stream)
 
@@ -801,9 +817,9 @@ def main():
         e2e_ms = e0.elapsed_time(e1) / args.steps
         e2e = {"value": step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "note": "per linear: pinned host X -> device (copy stream), qlin_forward (compute stream), "
-                       "device -> pinned host Y (second copy stream); copies overlap other linears' compute; "
-                       "one CUDA graph per step"}
+               "note": "per linear: pinned host X -> device (copy stream), qlin_forward (the step's compute "
+                       "streams, round-robin), device -> pinned host Y (second copy stream); copies overlap other "
+                       "linears' compute; one CUDA graph per step"}
 
     # ---------------------------------------------------------------- CPU baseline (rank 0, N = 1)
     cpu = None
