@@ -36,7 +36,11 @@ def compute() -> dict:
         Wb = np.ascontiguousarray(L["W"]).view(np.uint16)
         pk = oracle.pack_layer(Wb, L["O"], fmt)
         r = oracle.forward(Xb, Wb, pk, np.ones(len(L["O"]), np.float32), L["gamma"])
+        # input gradient with the forward's scales (straight-through estimator)
+        dY = np.ascontiguousarray(synth.grad_output(0, 0, L["M"], L["N"])).view(np.uint16)
+        dX = oracle.backward_dx(dY, Wb, pk, r["s"])
         out[tag] = {
+            "dX_00_01_10": [float(dX[0, 0]), float(dX[0, 1]), float(dX[1, 0])],
             "O": L["O"].tolist(),
             "s": [float(v) for v in r["s"]],
             "a_first4": [float(v) for v in r["a"][:4]],
@@ -45,7 +49,7 @@ def compute() -> dict:
             "sha256": {
                 "packed": digest(pk["packed"]), "B": digest(pk["B"]), "cscale": digest(pk["cscale"]),
                 "Xq": digest(r["Xq"]), "a": digest(r["a"]), "XqO": digest(r["XqO"]),
-                "acc": digest(r["acc"]), "s": digest(r["s"]),
+                "acc": digest(r["acc"]), "s": digest(r["s"]), "dX": digest(dX),
             },
         }
     return out
@@ -53,8 +57,9 @@ def compute() -> dict:
 
 if __name__ == "__main__":
     data = {"source": "CPU oracle on the seeded 'small' workload (M=16, K=N=512, 10 outlier "
-                      "channels, gamma=0.9, one momentum step, s0=1); the pages print no "
-                      "worked example, so these are regression values, not the pages'.",
+                      "channels, gamma=0.9, one momentum step, s0=1), and its input gradient for "
+                      "the seeded dY; the pages print no worked example, so these are regression "
+                      "values, not the pages'.",
             "cases": compute()}
     with open(os.path.join(HERE, "small_oracle.json"), "w") as f:
         json.dump(data, f, indent=1, sort_keys=True)
