@@ -64,10 +64,6 @@ def algorithmic_bytes(M, K, N, nO, fmt):
     return gemm, act
 
 
-def gemm_only_bytes(M, K, N, nO, fmt):
-    return algorithmic_bytes(M, K, N, nO, fmt)[0]
-
-
 GEMM_SOURCES = ["quantized_linear_layers_token_b200/csrc/gemm.cuh", "quantized_linear_layers_token_b200/csrc/sm100.cuh",
                 "quantized_linear_layers_token_b200/csrc/qlin.cu"]
 
