@@ -710,12 +710,12 @@ def main():
         naws = qlin.qlin_quant_act_workspace(M, lay.w)
         aws = qlin.empty_workspace(naws)
         qlin.qlin_quant_act(sl["X"], M, lay.w, sl["s"], wl.gamma, False, Xq, a, XqO, aws, naws, stream)
-        gemm_slots.append((sl, Xq, a, XqO))
+        gemm_slots.append((sl, Xq, a, XqO, aws, naws))
     torch.cuda.synchronize()
 
     def gemm_pass():
         # qlin_gemm = the compensation-operand kernel (when n_O > 0) + the tcgen05 GEMM kernel
-        for sl, Xq, a, XqO in gemm_slots:
+        for sl, Xq, a, XqO, _, _ in gemm_slots:
             qlin.qlin_gemm(sl["layer"].w, Xq, a, XqO, sl["s"], sl["M"], sl["Y"], None, sl["ws"], sl["nws"], stream)
 
     gemm_pass()
@@ -739,8 +739,48 @@ def main():
     gemm_ms = e0.elapsed_time(e1) / reps
     n_gemm_launches = len(gemm_slots)
 
+    # ---------------------------------------------------------------- activation quantization alone
+    # (momentum update + per-token INT8 codes, the forward's own path; one
+    # stream, CUDA graph).  Evidence only: an error is reported in the line,
+    # it does not fail the run.
+    act_quant = None
+    try:
+        def quant_pass():
+            for sl, Xq, a, XqO, aws, naws in gemm_slots:
+                qlin.qlin_quant_act(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, Xq, a, XqO, aws,
+                                    naws, stream)
+
+        quant_pass()
+        torch.cuda.synchronize()
+        g4 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g4, stream=stream):
+            quant_pass()
+        for _ in range(3):
+            with torch.cuda.stream(stream):
+                g4.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                g4.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        qlin.qlin_poll_device_status()
+        act_ms = e0.elapsed_time(e1) / reps
+        act_bytes = sum(algorithmic_bytes(sl["M"], meta[sl["si"]]["K"], meta[sl["si"]]["N"],
+                                          len(meta[sl["si"]]["O"]), wl.fmt)[1] for sl, *_ in gemm_slots)
+        act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
+        act_quant = {"bound": "hbm", "achieved": act_gbs, "unit": "GB/s", "algorithmic_bytes": act_bytes,
+                     "ms_per_step": act_ms, "calls_per_step": len(gemm_slots),
+                     "kernel": "qlin_quant_act (colmax above 16 tokens, then quant_kernel), one stream"}
+    except Exception as ex:  # evidence only
+        act_quant = {"error": f"{type(ex).__name__}: {ex}"[:300]}
+
     hbm, bf16, bf16_sus, peak_kind = read_peaks()
     achieved = gemm_bytes / (gemm_ms * 1e-3) / 1e9
+    if act_quant is not None and "achieved" in act_quant:
+        act_quant["peak"] = hbm
+        act_quant["frac"] = act_quant["achieved"] / hbm
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": recorded_traffic(wl.name, args.copies),
                 "traffic_unit": "bytes per step (all GEMM launches), ncu dram__bytes_read.sum + dram__bytes_write.sum",
@@ -852,7 +892,8 @@ def main():
                        "parallelism": f"dp{world}", "forwards_per_step": len(slots),
                        "timing": "CUDA graph of one step, CUDA events on the launch stream",
                        "streams": nstreams},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+            "roofline": roofline, "act_quant": act_quant, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": gpu_launches,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
         }
