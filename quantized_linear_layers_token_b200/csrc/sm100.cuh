@@ -189,7 +189,7 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// Tiled shared -> global store (no multicast); completion tracked by bulk
+// Tiled shared -> global store; completion tracked by bulk
 // groups of the issuing thread.  Rows or columns outside the tensor are not
 // written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
