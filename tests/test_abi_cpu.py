@@ -128,3 +128,28 @@ def test_backward_argument_errors(q):
     with pytest.raises(q.QlinError) as e:  # a workspace off the 256-byte grid
         q.qlin_backward_dx(w, 1 << 24, 4, 1 << 25, 1 << 26, (1 << 27) + 16, 1 << 20, stream=0)
     assert q.STATUS[e.value.status] == "QLIN_ERR_ALIGN"
+
+
+def test_binding_declares_every_entry_point(q):
+    """Every entry point of the header has an argument list in the ctypes
+    binding (so no call goes out with default int conversions)."""
+    L = q.lib()
+    for name in declared_entry_points():
+        if name in ("qlin_status_string", "qlin_last_error"):
+            continue
+        assert getattr(L, name).argtypes is not None, name
+
+
+def test_synthetic_inputs_are_reproducible():
+    """Both sides of every parity test draw the same arrays from the seeded
+    generator: repeated draws are identical, different shapes independent."""
+    import numpy as np
+    from quantized_linear_layers_token_b200 import synth
+    a = synth.layer("llama7b_w4_decode", 0, M=4)
+    b = synth.layer("llama7b_w4_decode", 0, M=4)
+    for k in ("X", "W", "O"):
+        assert np.array_equal(a[k], b[k])
+    c = synth.layer("llama7b_w4_decode", 1, M=4)
+    assert not np.array_equal(a["W"], c["W"])
+    assert np.array_equal(synth.grad_output(1, 0, 8, 64), synth.grad_output(1, 0, 8, 64))
+    assert np.array_equal(synth.outlier_scales(1, 0, 5), synth.outlier_scales(1, 0, 5))
