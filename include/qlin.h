@@ -191,7 +191,8 @@ QLIN_API qlin_status qlin_quant_act(const uint16_t* X, int32_t M, const qlin_wei
  * where the momentum update's scratch lives.
  * Same arguments and results as qlin_quant_act.  The scratch (outlier column
  * maxima and a completion counter) is a fixed array inside the library
- * (16.25 KiB on every GPU that loads it, held until the process exits), so:
+ * (4.25 KiB on every GPU that loads it: 1024 + 64 32-bit words, held until
+ * the process exits), so:
  *   - n_outlier must be <= 1024, else QLIN_ERR_SHAPE and nothing is enqueued;
  *   - no memory is allocated or freed; the call clears the part of the
  *     scratch it uses with cudaMemsetAsync on `stream` before its kernels;
@@ -274,6 +275,53 @@ QLIN_API qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weigh
 QLIN_API qlin_status qlin_backward_dx_workspace(int32_t M, const qlin_weights* w, size_t* bytes);
 QLIN_API qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t M, const float* s,
                                       uint16_t* dX, void* workspace, size_t ws_bytes, void* stream);
+
+/* Test and measurement hooks.  The library reads no environment variables:
+ * a process that wants a non-default work split, launch mode or wait limit
+ * (the test suite forcing each split-K variant, a measurement isolating one
+ * mechanism, a failure-detection test) sets it here.  Settings are global to
+ * the process, take effect from the next call that launches work, and are
+ * not meant for production use; the defaults are what the library is tuned
+ * and tested with.
+ *   QLIN_KNOB_PDL             1 (default): kernels are chained with
+ *                             programmatic dependent launch; 0: plain
+ *                             stream-ordered launches.
+ *   QLIN_KNOB_CLUSTER         1 (default): decode GEMMs may split tiles over
+ *                             thread-block clusters; 0: global stream-K only.
+ *   QLIN_KNOB_CLUSTER_SIZE    0 (default): cluster size from the cost model;
+ *                             2, 4 or 8: that size whenever it is valid.
+ *   QLIN_KNOB_MAX_CTAS        0 (default): one persistent GEMM CTA per SM;
+ *                             n > 0: at most n.
+ *   QLIN_KNOB_MAX_TOKEN_TILE  256 (default); 64 or 128 cap the GEMM's token tile.
+ *   QLIN_KNOB_WIDEN_MIN_M     1024 (default): from this token count INT4
+ *                             weights are widened to INT8 once per call; 0: never.
+ *   QLIN_KNOB_FUSED_MOMENTUM_MAX_M  16 (default): up to this token count the
+ *                             momentum update runs inside the quantization kernel.
+ *   QLIN_KNOB_WAIT_NS         2000000000 (default): limit in ns of every
+ *                             device-side pipeline wait, after which the kernel
+ *                             gives up, sets the device error word and unwinds
+ *                             (QLIN_ERR_TIMEOUT from qlin_poll_device_status).
+ *                             It is a device variable: set it with the device
+ *                             concerned current, between calls.  After a
+ *                             timeout, the workspaces and outputs of the calls
+ *                             that gave up are undefined; zero-fill the
+ *                             workspaces before reusing them.
+ * qlin_debug_set stores `value` (QLIN_ERR_ARG for an unknown knob or an
+ * invalid value) and, when `previous` is not NULL, returns the old value
+ * there; qlin_debug_get reads a knob. */
+typedef enum {
+  QLIN_KNOB_PDL = 0,
+  QLIN_KNOB_CLUSTER = 1,
+  QLIN_KNOB_CLUSTER_SIZE = 2,
+  QLIN_KNOB_MAX_CTAS = 3,
+  QLIN_KNOB_MAX_TOKEN_TILE = 4,
+  QLIN_KNOB_WIDEN_MIN_M = 5,
+  QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6,
+  QLIN_KNOB_WAIT_NS = 7
+} qlin_knob;
+
+QLIN_API qlin_status qlin_debug_set(int32_t knob, int64_t value, int64_t* previous);
+QLIN_API qlin_status qlin_debug_get(int32_t knob, int64_t* value);
 
 /* Synchronizes `stream`, then reports and clears the device error word that
  * kernels set when a bounded wait gives up: QLIN_ERR_TIMEOUT if it was set,

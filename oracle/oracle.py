@@ -78,6 +78,8 @@ def _declare(L):
     L.oq_int_gemm.restype = I
     L.oq_int_gemm_rows.argtypes = [P, P, I, I, P, I, P]
     L.oq_int_gemm_rows.restype = I
+    L.oq_int_gemm_rows_nk.argtypes = [P, P, I, I, P, I, P]
+    L.oq_int_gemm_rows_nk.restype = I
     L.oq_dequant.argtypes = [P, P, P, P, P, P, I, P, I, P, I, P]
     L.oq_dequant.restype = None
     L.oq_fast_fp16_to_int8_single.argtypes = [ctypes.c_uint16, P]
@@ -220,6 +222,19 @@ def int_gemm_rows(Xq: np.ndarray, B: np.ndarray, rows: np.ndarray):
     return acc, ovf
 
 
+def int_gemm_rows_nk(Xq: np.ndarray, Bt: np.ndarray, rows: np.ndarray):
+    """int_gemm_rows with the operand given transposed (Bt [N][K])."""
+    Xq = _c(Xq, np.int8)
+    Bt = _c(Bt, np.int8)
+    rows = _c(rows, np.int32)
+    M, K = Xq.shape
+    N = Bt.shape[0]
+    assert Bt.shape[1] == K
+    acc = np.zeros((len(rows), N), np.int64)
+    ovf = lib().oq_int_gemm_rows_nk(_p(Xq), _p(Bt), K, N, _p(rows), len(rows), _p(acc))
+    return acc, ovf
+
+
 def dequant(acc: np.ndarray, a: np.ndarray, cscale: np.ndarray, XqO: np.ndarray, s: np.ndarray,
             W_bits: np.ndarray, O: np.ndarray, rows: np.ndarray | None = None) -> np.ndarray:
     """fp64 y [R][N] for the rows of acc (rows[r] indexes a / XqO)."""
@@ -347,7 +362,9 @@ def forward(X_bits: np.ndarray, W_bits: np.ndarray, packed: dict, s: np.ndarray,
     if rows is None:
         rows = np.arange(M, dtype=np.int32)
     if len(rows):
-        acc, ovf = int_gemm_rows(Xq, packed["B"], rows)
+        if "Bt" not in packed:  # the operand transposed once per layer (a copy, no arithmetic)
+            packed["Bt"] = np.ascontiguousarray(packed["B"].T)
+        acc, ovf = int_gemm_rows_nk(Xq, packed["Bt"], rows)
         assert not ovf
         y = dequant(acc, a, packed["cscale"], XqO, s1, W_bits, O, rows)
     else:

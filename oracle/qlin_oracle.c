@@ -122,21 +122,28 @@ static int32_t clampi(double v, int32_t lo, int32_t hi) {
 OQ_EXPORT void oq_quant_weight_per_channel(const uint16_t* W, int K, int N, int qmax,
                                            int8_t* codes, float* scale) {
   const float fq = (float)qmax;
-  for (int n = 0; n < N; ++n) {
-    float wmax = 0.0f;
-    for (int k = 0; k < K; ++k) {
+  float* wmax = (float*)calloc((size_t)(N > 0 ? N : 1), sizeof(float));
+  float* inv = (float*)calloc((size_t)(N > 0 ? N : 1), sizeof(float));
+  /* W is walked row by row (k outer) so every access is sequential; each
+   * channel's max and codes are the same values as a channel-by-channel
+   * loop gives (max is exact in any order). */
+  for (int k = 0; k < K; ++k)
+    for (int n = 0; n < N; ++n) {
       float v = fabsf(oq_half_to_float(W[(size_t)k * N + n]));
-      if (v > wmax) wmax = v;
+      if (v > wmax[n]) wmax[n] = v;
     }
-    float sc = wmax / fq;
-    float inv = (wmax > 0.0f) ? (fq / wmax) : 0.0f;
-    scale[n] = sc;
-    for (int k = 0; k < K; ++k) {
+  for (int n = 0; n < N; ++n) {
+    scale[n] = wmax[n] / fq;
+    inv[n] = (wmax[n] > 0.0f) ? (fq / wmax[n]) : 0.0f;
+  }
+  for (int k = 0; k < K; ++k)
+    for (int n = 0; n < N; ++n) {
       float w = oq_half_to_float(W[(size_t)k * N + n]);
-      float p = w * inv;
+      float p = w * inv[n];
       codes[(size_t)k * N + n] = (int8_t)clampi(oq_rne((double)p), -qmax, qmax);
     }
-  }
+  free(wmax);
+  free(inv);
 }
 
 /* Per-group (g = 128 along K) symmetric INT4 with per-channel INT8
@@ -158,20 +165,27 @@ OQ_EXPORT int oq_quant_weight_group(const uint16_t* W, int K, int N, int group,
                                     float* c) {
   int bad = 0;
   int G = K / group;
-  for (int n = 0; n < N; ++n) {
-    float ghmax = 0.0f;
-    for (int j = 0; j < G; ++j) {
-      float gmax = 0.0f;
-      for (int k = j * group; k < (j + 1) * group; ++k) {
+  /* W is walked row by row (k outer) so every access is sequential; every
+   * (group, channel) value is the same as a channel-by-channel loop gives. */
+  float* gmax = (float*)calloc((size_t)(N > 0 ? N : 1), sizeof(float));
+  float* ghmax = (float*)calloc((size_t)(N > 0 ? N : 1), sizeof(float));
+  for (int j = 0; j < G; ++j) {
+    for (int n = 0; n < N; ++n) gmax[n] = 0.0f;
+    for (int k = j * group; k < (j + 1) * group; ++k)
+      for (int n = 0; n < N; ++n) {
         float v = fabsf(oq_half_to_float(W[(size_t)k * N + n]));
-        if (v > gmax) gmax = v;
+        if (v > gmax[n]) gmax[n] = v;
       }
-      float gs = gmax / 7.0f;
+    for (int n = 0; n < N; ++n) {
+      float gs = gmax[n] / 7.0f;
       uint16_t gh = oq_float_to_half(gs);
       g_h[(size_t)j * N + n] = gh;
       float ghf = oq_half_to_float(gh);
-      if (ghf > ghmax) ghmax = ghf;
-      for (int k = j * group; k < (j + 1) * group; ++k) {
+      if (ghf > ghmax[n]) ghmax[n] = ghf;
+    }
+    for (int k = j * group; k < (j + 1) * group; ++k)
+      for (int n = 0; n < N; ++n) {
+        float ghf = oq_half_to_float(g_h[(size_t)j * N + n]);
         float w = oq_half_to_float(W[(size_t)k * N + n]);
         int32_t q = 0;
         if (ghf > 0.0f) {
@@ -180,27 +194,32 @@ OQ_EXPORT int oq_quant_weight_group(const uint16_t* W, int K, int N, int group,
         }
         q4[(size_t)k * N + n] = (int8_t)q;
       }
-    }
-    float seven_g = 7.0f * ghmax;
-    float cn = seven_g / 127.0f;
-    c[n] = cn;
-    for (int j = 0; j < G; ++j) {
+  }
+  for (int n = 0; n < N; ++n) {
+    float seven_g = 7.0f * ghmax[n];
+    c[n] = seven_g / 127.0f;
+  }
+  for (int j = 0; j < G; ++j) {
+    for (int n = 0; n < N; ++n) {
       float ghf = oq_half_to_float(g_h[(size_t)j * N + n]);
       uint16_t rh = 0;
-      if (cn > 0.0f) {
-        float ratio = ghf / cn;
+      if (c[n] > 0.0f) {
+        float ratio = ghf / c[n];
         rh = oq_float_to_half(ratio);
       }
       r_h[(size_t)j * N + n] = rh;
-      double rf = oq_half_to_double(rh);
-      for (int k = j * group; k < (j + 1) * group; ++k) {
+    }
+    for (int k = j * group; k < (j + 1) * group; ++k)
+      for (int n = 0; n < N; ++n) {
+        double rf = oq_half_to_double(r_h[(size_t)j * N + n]);
         double prod = (double)q4[(size_t)k * N + n] * rf; /* exact in double */
         double q = oq_rne(prod);
         if (q > 127.0 || q < -127.0) bad = 1;
         q8[(size_t)k * N + n] = (int8_t)clampi(q, -127, 127);
       }
-    }
   }
+  free(gmax);
+  free(ghmax);
   return bad;
 }
 
@@ -328,6 +347,25 @@ OQ_EXPORT int oq_int_gemm_rows(const int8_t* Xq, const int8_t* B, int K, int N,
     for (int n = 0; n < N; ++n) {
       int64_t sum = 0;
       for (int k = 0; k < K; ++k) sum += (int64_t)xr[k] * (int64_t)B[(size_t)k * N + n];
+      if (sum > INT32_MAX || sum < INT32_MIN) overflow = 1;
+      acc[(size_t)r * N + n] = sum;
+    }
+  }
+  return overflow;
+}
+
+/* Same sums as oq_int_gemm_rows with the operand stored transposed,
+ * Bt[n][k] = B[k][n], so each output channel's K codes are contiguous (the
+ * same products added in the same k order; integer sums are exact). */
+OQ_EXPORT int oq_int_gemm_rows_nk(const int8_t* Xq, const int8_t* Bt, int K, int N,
+                                  const int32_t* rows, int R, int64_t* acc) {
+  int overflow = 0;
+  for (int r = 0; r < R; ++r) {
+    const int8_t* xr = Xq + (size_t)rows[r] * K;
+    for (int n = 0; n < N; ++n) {
+      const int8_t* bn = Bt + (size_t)n * K;
+      int64_t sum = 0;
+      for (int k = 0; k < K; ++k) sum += (int64_t)xr[k] * (int64_t)bn[k];
       if (sum > INT32_MAX || sum < INT32_MIN) overflow = 1;
       acc[(size_t)r * N + n] = sum;
     }

@@ -315,7 +315,7 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       // every MMA issued so far (all of them, or those before an abort)
       mma_commit(acc_full);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait_sleep(acc_full, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+      while (!mbar_try_wait_sleep(acc_full, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
       }
     }
   } else if (warp == 2) {
@@ -545,8 +545,9 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       // ranges have counted, add their partials, store dX, reset the count
       if (ctid == 0) {
         const uint64_t t0 = globaltimer_ns();
+        const uint64_t lim = *const_cast<const volatile unsigned long long*>(&g_wait_ns);
         while (ld_acquire_gpu(args.cnt + tt) < static_cast<unsigned>(S - 1)) {
-          if (*abort_flag || globaltimer_ns() - t0 > QLIN_WAIT_NS) {
+          if (*abort_flag || globaltimer_ns() - t0 > lim) {
             *abort_flag = 1;
             atomicExch(&g_device_error, kDevErrTimeout);
             break;

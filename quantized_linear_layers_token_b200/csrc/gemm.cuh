@@ -398,7 +398,7 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int slots, int issued
     const int s = t % slots;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_sleep(&full[s], static_cast<uint32_t>(t / slots) & 1u, 1000000u) &&
-           globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+           globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
     }
   }
 }
@@ -698,7 +698,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         if (!a_issues[p]) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait_sleep(&afull[p], (a_issues[p] - 1) & 1u, 1000000u) &&
-               globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+               globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
         }
       }
     }
@@ -1006,7 +1006,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           if (!a_issues[p]) continue;
           const uint64_t t0 = globaltimer_ns();
           while (!mbar_try_wait_sleep(&afull[p], (a_issues[p] - 1) & 1u, 1000000u) &&
-                 globaltimer_ns() - t0 < QLIN_WAIT_NS) {
+                 globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
           }
         }
       }

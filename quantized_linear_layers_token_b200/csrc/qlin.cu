@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "qlin.h"
@@ -130,35 +131,23 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 }
 
 // ---------------------------------------------------------------- launches
-// Kernels are launched with programmatic dependent launch, so each may start
-// its prologue (and the GEMM its weight stream) while the previous kernel in
-// the stream finishes; every kernel waits on the grid dependency before it
-// reads what the previous one wrote.  QLIN_NO_PDL=1 turns this off.
-// QLIN_NO_CLUSTER=1 keeps decode GEMMs on global-memory stream-K.
-bool cluster_disabled() {
-  static const bool off = [] {
-    const char* e = getenv("QLIN_NO_CLUSTER");
-    return e && e[0] == '1';
-  }();
-  return off;
-}
+// Test and measurement knobs (qlin_debug_set); the defaults are the tuned
+// behaviour.  Kernels are launched with programmatic dependent launch, so
+// each may start its prologue (and the GEMM its weight stream) while the
+// previous kernel in the stream finishes; every kernel waits on the grid
+// dependency before it reads what the previous one wrote.
+std::atomic<long long> g_knob[8] = {{1}, {1}, {0}, {0}, {256}, {1024}, {kFusedMomentumMaxM}, {2000000000LL}};
+
+long long knob(int k) { return g_knob[k].load(std::memory_order_relaxed); }
+
+bool cluster_disabled() { return knob(QLIN_KNOB_CLUSTER) == 0; }
 
 int forced_cluster_size() {
-  static const int cs = [] {
-    const char* e = getenv("QLIN_CLUSTER_CS");
-    const int v = e ? atoi(e) : 0;
-    return (v == 2 || v == 4 || v == 8) ? v : 0;
-  }();
-  return cs;
+  const long long v = knob(QLIN_KNOB_CLUSTER_SIZE);
+  return (v == 2 || v == 4 || v == 8) ? static_cast<int>(v) : 0;
 }
 
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("QLIN_NO_PDL");
-    return !(e && e[0] == '1');
-  }();
-  return on;
-}
+bool pdl_enabled() { return knob(QLIN_KNOB_PDL) != 0; }
 
 // `cluster` > 1 launches thread-block clusters of that many CTAs along x.
 template <typename... KArgs, typename... Args>
@@ -206,24 +195,17 @@ int sm_count() {
   return cached[dev];
 }
 
-// CTAs a GEMM may use at most (QLIN_MAX_CTAS, measurement aid; default all SMs).
+// CTAs a GEMM may use at most (QLIN_KNOB_MAX_CTAS; default all SMs).
 int gemm_cta_cap() {
-  static const int v = [] {
-    const char* e = getenv("QLIN_MAX_CTAS");
-    return e ? atoi(e) : 0;
-  }();
+  const long long v = knob(QLIN_KNOB_MAX_CTAS);
   const int sms = sm_count();
-  return (v > 0 && v < sms) ? v : sms;
+  return (v > 0 && v < sms) ? static_cast<int>(v) : sms;
 }
 
-// QLIN_MAX_BT=128 caps the token tile (measurement aid).
+// QLIN_KNOB_MAX_TOKEN_TILE = 64 or 128 caps the token tile.
 int max_bt() {
-  static const int v = [] {
-    const char* e = getenv("QLIN_MAX_BT");
-    const int x = e ? atoi(e) : 0;
-    return (x == 64 || x == 128) ? x : 256;
-  }();
-  return v;
+  const long long x = knob(QLIN_KNOB_MAX_TOKEN_TILE);
+  return (x == 64 || x == 128) ? static_cast<int>(x) : 256;
 }
 
 int pick_bt(int M) {
@@ -244,14 +226,8 @@ struct GemmPlan {
 };
 
 // From this many tokens the INT4 formats widen their weights once per call
-// and run the INT8 kernel (QLIN_WIDEN_MIN_M overrides it; 0 turns it off).
-int widen_min_m() {
-  static const int v = [] {
-    const char* e = getenv("QLIN_WIDEN_MIN_M");
-    return e ? atoi(e) : 1024;
-  }();
-  return v;
-}
+// and run the INT8 kernel (QLIN_KNOB_WIDEN_MIN_M; 0 turns it off).
+int widen_min_m() { return static_cast<int>(knob(QLIN_KNOB_WIDEN_MIN_M)); }
 
 GemmPlan plan_gemm(int M, const qlin_weights* w) {
   GemmPlan p{};
@@ -459,15 +435,8 @@ qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a,
 // ---------------------------------------------------------------- act quant
 // Up to this many tokens the momentum update runs inside the quantization
 // kernel (every CTA gathers all rows' outlier values); above it a separate
-// column-max kernel gathers them once.  QLIN_FUSED_MAX_M overrides it
-// (measurement aid).
-int fused_momentum_max_m() {
-  static const int v = [] {
-    const char* e = getenv("QLIN_FUSED_MAX_M");
-    return e ? atoi(e) : kFusedMomentumMaxM;
-  }();
-  return v;
-}
+// column-max kernel gathers them once (QLIN_KNOB_FUSED_MOMENTUM_MAX_M).
+int fused_momentum_max_m() { return static_cast<int>(knob(QLIN_KNOB_FUSED_MOMENTUM_MAX_M)); }
 
 constexpr int kQuantSmemMax = 232448 - 1024;  // 227 KB per CTA, less room for the kernel's static shared memory
 
@@ -480,7 +449,7 @@ qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float*
   const int K = w->K, nO = w->n_outlier;
   if (M == 0) return QLIN_OK;
   unsigned* cmax = static_cast<unsigned*>(act_ws);
-  MomentumArgs mom{w->wmax_O, gamma, cmax + nO, M};
+  MomentumArgs mom{w->wmax_O, gamma, cmax ? cmax + nO : nullptr, M};
   const bool do_update = update && nO > 0;
   const bool fused = do_update && M <= fused_momentum_max_m();
   if (do_update && !fused) {
@@ -549,8 +518,9 @@ FwdLayout forward_layout(int M, const qlin_weights* w) {
 // ---------------------------------------------------------------- allocation-free quantization
 // Fixed scratch for qlin_quant_act_noalloc: the outlier column maxima and the
 // completion counter of the momentum update.  It is a file-scope device
-// array, so every GPU that loads this library holds it (16.25 KiB) until the
-// process exits, and every call on a device shares the same copy.
+// array, so every GPU that loads this library holds it (4.25 KiB: 1024 + 64
+// words) until the process exits, and every call on a device shares the same
+// copy.
 #define QLIN_NOALLOC_MAX_OUTLIERS 1024
 static __device__ __align__(256) unsigned g_noalloc_scratch[QLIN_NOALLOC_MAX_OUTLIERS + 64];
 
@@ -959,6 +929,32 @@ QLIN_API int qlin_steps_set(long long* p) {
   return static_cast<int>(cudaMemcpyToSymbol(qlin::g_steps, &p, sizeof(p)));
 }
 #endif
+
+qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
+  if (k < 0 || k > QLIN_KNOB_WAIT_NS) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
+  bool ok = true;
+  switch (k) {
+    case QLIN_KNOB_PDL:
+    case QLIN_KNOB_CLUSTER: ok = value == 0 || value == 1; break;
+    case QLIN_KNOB_CLUSTER_SIZE: ok = value == 0 || value == 2 || value == 4 || value == 8; break;
+    case QLIN_KNOB_MAX_TOKEN_TILE: ok = value == 64 || value == 128 || value == 256; break;
+    default: ok = value >= 0;
+  }
+  if (!ok) return fail(QLIN_ERR_ARG, "invalid value %lld for knob %d", static_cast<long long>(value), k);
+  if (k == QLIN_KNOB_WAIT_NS) {
+    const unsigned long long v = static_cast<unsigned long long>(value);
+    QLIN_CUDA_TRY(cudaMemcpyToSymbol(qlin::g_wait_ns, &v, sizeof(v)));
+  }
+  const long long old = g_knob[k].exchange(value);
+  if (previous) *previous = old;
+  return QLIN_OK;
+}
+
+qlin_status qlin_debug_get(int32_t k, int64_t* value) {
+  if (k < 0 || k > QLIN_KNOB_WAIT_NS || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
+  *value = g_knob[k].load();
+  return QLIN_OK;
+}
 
 qlin_status qlin_poll_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

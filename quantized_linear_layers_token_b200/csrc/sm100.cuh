@@ -1,7 +1,7 @@
 // sm100.cuh -- thin wrappers over the sm_100a PTX this library uses:
 // mbarriers, TMA tile loads, tcgen05 (TMEM alloc, MMA, commit, loads) and
 // the shared-memory / instruction descriptors of the 5th-gen tensor cores.
-// Every wait is bounded: it gives up after QLIN_WAIT_NS of wall time, sets
+// Every wait is bounded: it gives up after g_wait_ns of wall time, sets
 // the device error word and reports failure to the caller, which unwinds.
 #pragma once
 
@@ -9,9 +9,10 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#ifndef QLIN_WAIT_NS
-#define QLIN_WAIT_NS 2000000000ull  // 2 s: far above any legitimate wait
-#endif
+// Limit of the waits that drain copies and tensor-core work still in flight
+// before a CTA exits (also after another wait gave up): fixed, independent of
+// the adjustable limit below.
+#define QLIN_DRAIN_NS 2000000000ull  // 2 s: far above any legitimate wait
 
 namespace qlin {
 
@@ -19,6 +20,12 @@ namespace qlin {
 // library is a single translation unit, so the definition lives here.
 __device__ int g_device_error = 0;
 enum : int { kDevErrTimeout = 1 };
+// Limit of every pipeline wait, in ns of %globaltimer: 2 s by default, far
+// above any legitimate wait.  The host changes it only through the
+// test/measurement hook of the C ABI; a limit below 1 ms also shortens the
+// suspend hint of each try, so a zero limit makes the first wait that is
+// not already complete give up.
+__device__ unsigned long long g_wait_ns = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -77,15 +84,22 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false (and raises the device error word) if it does not within
-// QLIN_WAIT_NS, or if *abort becomes nonzero (another role gave up).  The
-// clock and the abort flag are only read between sleeps.
+// g_wait_ns, or if *abort becomes nonzero (another role gave up).  The
+// clock, the limit and the abort flag are only read after a first try
+// failed.
+__device__ __forceinline__ uint32_t wait_hint_ns(uint64_t lim) {
+  return lim < 1000000ull ? static_cast<uint32_t>(lim) : 1000000u;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t lim = *const_cast<const volatile unsigned long long*>(&g_wait_ns);
+  const uint32_t hint = wait_hint_ns(lim);
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > QLIN_WAIT_NS) {
+    if (globaltimer_ns() - t0 > lim) {
       *abort = 1;
       atomicExch(&g_device_error, kDevErrTimeout);
       return false;
@@ -153,12 +167,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep_cluster(uint64_t* bar, uint3
   return ok != 0;
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_sleep_cluster(bar, parity, 1000000u)) return true;
+  if (mbar_try_wait_sleep_cluster(bar, parity, 0u)) return true;
+  const uint64_t lim = *const_cast<const volatile unsigned long long*>(&g_wait_ns);
+  const uint32_t hint = wait_hint_ns(lim);
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait_sleep_cluster(bar, parity, 1000000u)) return true;
+    if (mbar_try_wait_sleep_cluster(bar, parity, hint)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > QLIN_WAIT_NS) {
+    if (globaltimer_ns() - t0 > lim) {
       *abort = 1;
       atomicExch(&g_device_error, kDevErrTimeout);
       return false;

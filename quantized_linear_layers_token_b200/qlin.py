@@ -29,8 +29,18 @@ EXPORTED = [
     "qlin_pack_weights", "qlin_quant_act_workspace", "qlin_quant_act", "qlin_outlier_colmax",
     "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
     "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc", "qlin_backward_dx",
-    "qlin_backward_dx_workspace",
+    "qlin_backward_dx_workspace", "qlin_debug_set", "qlin_debug_get",
 ]
+
+# test / measurement knobs (qlin_debug_set, include/qlin.h)
+QLIN_KNOB_PDL = 0
+QLIN_KNOB_CLUSTER = 1
+QLIN_KNOB_CLUSTER_SIZE = 2
+QLIN_KNOB_MAX_CTAS = 3
+QLIN_KNOB_MAX_TOKEN_TILE = 4
+QLIN_KNOB_WIDEN_MIN_M = 5
+QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6
+QLIN_KNOB_WAIT_NS = 7
 
 
 class QlinError(RuntimeError):
@@ -85,6 +95,8 @@ def lib() -> ctypes.CDLL:
             "qlin_quant_act_noalloc": [P, I32, W, P, F32, I32, P, P, P, P],
             "qlin_backward_dx": [W, P, I32, P, P, P, SZ, P],
             "qlin_backward_dx_workspace": [I32, W, ctypes.POINTER(SZ)],
+            "qlin_debug_set": [I32, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)],
+            "qlin_debug_get": [I32, ctypes.POINTER(ctypes.c_int64)],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -198,6 +210,37 @@ def qlin_backward_dx_workspace(M: int, w: qlin_weights) -> int:
 def qlin_backward_dx(w: qlin_weights, dY, M: int, s, dX, workspace=None, ws_bytes: int = 0, stream=None):
     _check(lib().qlin_backward_dx(ctypes.byref(w), _ptr(dY), M, _ptr(s), _ptr(dX), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "qlin_backward_dx")
+
+
+def qlin_debug_set(knob: int, value: int) -> int:
+    """Set a test/measurement knob; returns its previous value."""
+    prev = ctypes.c_int64(0)
+    _check(lib().qlin_debug_set(knob, int(value), ctypes.byref(prev)), "qlin_debug_set")
+    return int(prev.value)
+
+
+def qlin_debug_get(knob: int) -> int:
+    v = ctypes.c_int64(0)
+    _check(lib().qlin_debug_get(knob, ctypes.byref(v)), "qlin_debug_get")
+    return int(v.value)
+
+
+class knobs:
+    """Context manager: set knobs for the duration of a block, then restore."""
+
+    def __init__(self, **settings):
+        self.settings = {globals()["QLIN_KNOB_" + k.upper()]: v for k, v in settings.items()}
+        self.saved = {}
+
+    def __enter__(self):
+        for k, v in self.settings.items():
+            self.saved[k] = qlin_debug_set(k, v)
+        return self
+
+    def __exit__(self, *exc):
+        for k, v in self.saved.items():
+            qlin_debug_set(k, v)
+        return False
 
 
 def qlin_poll_device_status(stream=None):

@@ -132,8 +132,7 @@ def test_small_workload(q, oracle, fmt):
     check_all(oracle, L, g, s0, L["gamma"])
 
 
-@pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("M,K,N,nO", [
+SHAPE_MKN = [
     (1, 512, 256, 10),      # single token (decode), BT = 16
     (4, 1024, 128, 3),
     (16, 640, 336, 13),     # ragged N tile, n_outlier not a multiple of 8
@@ -141,7 +140,12 @@ def test_small_workload(q, oracle, fmt):
     (64, 2048, 384, 0),     # no outliers: the plain QQQ path
     (200, 1152, 256, 41),   # BT = 256 with a ragged token tile
     (130, 4096, 128, 9),    # 32 K-steps: the stage ring wraps several times
-])
+]
+SHAPES = [(fmt, *mknO) for fmt in FMTS for mknO in SHAPE_MKN]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,K,N,nO", SHAPE_MKN)
 def test_shapes(q, oracle, fmt, M, K, N, nO):
     L = case(fmt, M, K, N, nO, seed_shape=0)
     rng = np.random.default_rng(M * 7 + K)

@@ -437,3 +437,21 @@ def test_oracle_regression_fixture(oracle):
         stored = json.load(f)["cases"]
     now = make_golden.compute()
     assert now == stored
+
+
+def test_int_gemm_row_forms_agree_with_numpy(oracle):
+    """The row GEMM over the transposed operand (the form the full-size
+    parity checks use) equals numpy's exact int64 matmul, and so the plain
+    form, including sums that reach the int32 range edge."""
+    rng = np.random.default_rng(77)
+    for K, N in [(64, 48), (1024, 96), (8192, 16)]:
+        Xq = rng.integers(-127, 128, (5, K)).astype(np.int8)
+        B = rng.integers(-127, 128, (K, N)).astype(np.int8)
+        Xq[0] = 127
+        B[:, 0] = 127  # the largest positive sum
+        rows = np.array([4, 0, 2], np.int32)
+        want = Xq[rows].astype(np.int64) @ B.astype(np.int64)
+        acc_kn, _ = oracle.int_gemm_rows(Xq, B, rows)
+        acc_nk, _ = oracle.int_gemm_rows_nk(Xq, np.ascontiguousarray(B.T), rows)
+        np.testing.assert_array_equal(acc_kn, want)
+        np.testing.assert_array_equal(acc_nk, want)

@@ -5,8 +5,9 @@ framework that owns every GPU buffer, or a latency-bound loop that must not
 call cudaMalloc -- so they cannot provide qlin_quant_act's workspace.  The
 no-alloc variant keeps that scratch in a fixed array inside the library.
 This file checks it through the C ABI against qlin_quant_act (with a
-workspace) on two calls in a row, which also exercises the scratch being
-reused after the first call left it.  Collected last on purpose.
+workspace) and against the CPU oracle's momentum update and quantization,
+on two calls in a row, which also exercises the scratch being reused after
+the first call left it.  Collected last on purpose.
 """
 import numpy as np
 import pytest
@@ -30,8 +31,10 @@ def q():
     (synth.W4_PERCHANNEL, 16, 512, 256, 10),
     (synth.W8_PERCHANNEL, 67, 1024, 128, 77),
 ])
-def test_noalloc_matches_workspace_path_twice(q, fmt, M, K, N, nO):
+def test_noalloc_matches_workspace_path_twice(q, oracle, fmt, M, K, N, nO):
     L0 = synth.layer("small", 0, M=M, K=K, N=N, n_outliers=nO)
+    wmaxO = oracle.outlier_wmax(np.ascontiguousarray(L0["W"]).view(np.uint16), L0["O"])
+    s_oracle = np.ones(nO, np.float32)
     layer = q.PackedLayer.pack(torch.from_numpy(L0["W"]).cuda(), L0["O"], fmt)
     s_ref = torch.ones(nO, dtype=torch.float32, device="cuda")
     s_new = torch.ones(nO, dtype=torch.float32, device="cuda")
@@ -60,6 +63,14 @@ def test_noalloc_matches_workspace_path_twice(q, fmt, M, K, N, nO):
             assert torch.equal(x.view(torch.uint8) if x.dtype == torch.int8 else x.view(torch.int32),
                                y.view(torch.uint8) if y.dtype == torch.int8 else y.view(torch.int32)), step
         assert (s_new > 1.0).all()
+        # and both equal the oracle, bit for bit
+        Xb = np.ascontiguousarray(L["X"]).view(np.uint16)
+        s_oracle = oracle.momentum_update(Xb, L0["O"], wmaxO, 0.9, s_oracle)
+        Xq_r, a_r, XqO_r = oracle.quant_act(Xb, L0["O"], s_oracle)
+        np.testing.assert_array_equal(s_new.cpu().numpy().view(np.uint32), s_oracle.view(np.uint32))
+        np.testing.assert_array_equal(outs[1][0].cpu().numpy(), Xq_r)
+        np.testing.assert_array_equal(outs[1][1].cpu().numpy().view(np.uint32), a_r.view(np.uint32))
+        np.testing.assert_array_equal(outs[1][2].cpu().numpy(), XqO_r)
 
 
 def test_noalloc_rejects_too_many_outliers(q):
