@@ -1,39 +1,47 @@
-"""Throughput of the outlier-aware W4A8 quantized linear layer on B200.
+"""Throughput of the outlier-aware W4A8 / W8A8 quantized linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--op forward|backward] [--tokens M]
+                    [--workload NAME] [--extras LIST] [--op forward|backward]
 
 One step = one pass of the whole hot path -- targeted momentum update,
 per-token INT8 quantization, tcgen05 INT8 GEMM with the fused dequant and
 outlier compensation -- over every linear of the workload at every token
-count, on NL distinct copies of the packed weights (so the weights streamed
-in one step exceed the 126 MB L2 and come from HBM).  Default workload:
-LLaMA-2-7B-shaped linears (q, k, v, o 4096x4096; gate, up 4096->11008; down
-11008->4096), W4A8 per-channel, M in {1, 4, 16, 64}, 1% outlier channels
-x100, synthetic seeded data.
+count.  Default workload: LLaMA-2-70B-shaped linears (q 8192x8192, kv
+8192->1024, up 8192->28672, down 28672->8192), W4A8 with g = 128 group
+scales, M in {1, 16, 128, 1024, 8192} tokens, 1% outlier channels x100,
+synthetic seeded data (no weights or datasets are used).
 
-metric / unit: effective GB/s = algorithmic bytes of the step / step time
-(weights K*N/2, scales 4N, W_O 2*n_O*N, X 2MK, Xq written and read 2MK,
-a 4M, outlier codes M*n_O, Y 2MN); TOPS (2MNK) are reported beside it.
+metric / unit: effective TOPS = 2 M N K of every linear of the step / step
+time.  The line also carries the step's effective GB/s over the fused
+layer's algorithmic bytes (X 2MK, packed weights, scales, W_O, Y 2MN), and
+per token count a bucket timed on its own (median of >= 20 CUDA-graph
+replays) with its roofline: the bound is whichever of HBM bytes / measured
+copy bandwidth and INT8 ops / INT8 peak takes longer (decode buckets are
+HBM-bound, prefill buckets tensor-bound).  The INT8 peak is twice the
+measured dense bf16 figure (the nominal INT8 : bf16 ratio of B200).
+
+``roofline`` is the dominant kernel's: the GEMM calls of the prefill
+buckets (INT4 widened once per call, then the INT8 tcgen05 GEMM), timed
+alone on one stream.
+
+``workloads`` holds the other workloads the layer is specified on, each
+measured the same way: the LLaMA-2-7B decode set (W4A8 per-channel, M in
+{1, 4, 16, 64}, four weight copies so weights come from HBM), the 7B
+prefill set (W4A8 g128, M in {512, 2048, 4096}), the Phi-3-mini W8A8 Quaff
+step (M = 4096, momentum update on) and the fine-tuning input gradient of
+the Phi-3-mini linears.
 
 N > 1 (torchrun): data-parallel over tokens, weak scaling: every rank runs
 the same step on its own token batch with replicated weights; the outlier
 column maxima of all linears are combined with one all-reduce(MAX) per step
 so every replica keeps the same momentum state.
 
-The forwards of a step are independent (every linear at every token
-count), so on one GPU they are spread round-robin over --streams compute
-streams (default 4): one GEMM's tail then overlaps the next one's weight
-streaming on other SMs.  The roofline line times the GEMMs one after
-another on a single stream, so its per-launch figure is unaffected.
-
 ``--impl reference`` times the CPU oracle (single thread) on a bounded
 sample of the same workload and prints the same JSON line.
 
-``--op backward`` measures the fine-tuning input gradient instead: one step
-is qlin_backward_dx on every linear of the workload (default: the Phi-3-mini
-W8A8 linears of the Quaff notes) at --tokens tokens; metric TFLOP/s
-(2 M N K per linear) against the tensor-core roofline.
+``--op backward`` measures only the fine-tuning input gradient: one step is
+qlin_backward_dx on every linear of the workload (default: the Phi-3-mini
+W8A8 linears of the Quaff notes) at --tokens tokens; metric TFLOP/s.
 """
 from __future__ import annotations
 
@@ -54,9 +62,32 @@ from quantized_linear_layers_token_b200 import synth  # noqa: E402
 METRIC = "W4A8/W8A8 quantized-linear effective TOPS, GB/s and % of INT8/HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0  # nominal dense INT8 : bf16 tensor rate of B200 (4.5 : 2.25 PFLOP/s)
+DEFAULT_WORKLOAD = "llama70b_w4g128"
+DEFAULT_EXTRAS = "llama7b_w4_decode,llama7b_w4g128_prefill,phi3_w8_quaff,backward,gptq"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def weight_bytes(K, N, nO, fmt):
+    """Packed weights a forward must read once: codes, channel scales, the
+    g128 ratios, the fp16 outlier rows W_O, wmax_O, O and the state s."""
+    codes = K * N // 2 if fmt != synth.W8_PERCHANNEL else K * N
+    ratios = 2 * (K // 128) * N if fmt == synth.W4_G128 else 0
+    return codes + 4 * N + ratios + 2 * nO * N + 4 * nO + 4 * nO + 8 * nO
+
+
+def layer_bytes(M, K, N, nO, fmt):
+    """The fused layer's algorithmic bytes: X in, packed weights, Y out."""
+    return 2 * M * K + weight_bytes(K, N, nO, fmt) + 2 * M * N
 
 
 def algorithmic_bytes(M, K, N, nO, fmt):
+    """(GEMM call, quantization call): the bytes each of the two stages must
+    move at least once when they run as separate kernels (the GEMM reads the
+    INT8 codes, token scales and outlier codes the quantization wrote)."""
     wbytes = K * N // 2 if fmt != synth.W8_PERCHANNEL else K * N
     gemm = wbytes + 4 * N + (2 * (K // 128) * N if fmt == synth.W4_G128 else 0) + 2 * nO * N \
         + M * K + 4 * M + M * nO + 2 * M * N
@@ -64,50 +95,33 @@ def algorithmic_bytes(M, K, N, nO, fmt):
     return gemm, act
 
 
-GEMM_SOURCES = ["quantized_linear_layers_token_b200/csrc/gemm.cuh", "quantized_linear_layers_token_b200/csrc/sm100.cuh",
-                "quantized_linear_layers_token_b200/csrc/qlin.cu"]
-
-
-def gemm_sources_sha256():
-    """Hash of the GEMM sources' code: comments and blank lines are dropped,
-    so a comment edit does not retire the recorded traffic."""
-    import hashlib
-    import re
-    h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
-        with open(os.path.join(ROOT, rel)) as f:
-            text = f.read()
-        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        text = re.sub(r"//[^\n]*", "", text)
-        code = "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
-        h.update(code.encode())
-    return h.hexdigest()
-
-
-def recorded_traffic(workload, copies):
-    """DRAM bytes (read + write) of the GEMM launches of one step, from the
-    ncu launch list summarised in profiles/gemm_traffic.json -- only while
-    the GEMM sources are the ones that capture was taken with."""
-    try:
-        with open(os.path.join(ROOT, "profiles", "gemm_traffic.json")) as f:
-            rec = json.load(f)
-    except Exception:
-        return None
-    if rec.get("sources_sha256") != gemm_sources_sha256():
-        return None
-    if rec.get("workload") != workload or rec.get("weight_copies") != copies:
-        return None
-    return rec.get("dram_bytes_per_step")
-
-
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+        return {"hbm": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]),
+                "bf16_sus": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "kind": "measured"}
     except Exception:
-        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+        return {"hbm": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "bf16_sus": 1400.0, "kind": "fallback"}
+
+
+def roofline_of(ops, nbytes, seconds, peaks):
+    """Roofline of work that moves `nbytes` and does `ops` INT8 operations in
+    `seconds`: the bound is whichever of the HBM time (bytes / measured copy
+    bandwidth) and the tensor time (ops / INT8 peak) is longer; frac is that
+    time over the measured one."""
+    int8 = INT8_PER_BF16 * peaks["bf16"]
+    t_hbm = nbytes / (peaks["hbm"] * 1e9)
+    t_tc = ops / (int8 * 1e12)
+    if t_hbm >= t_tc:
+        ach = nbytes / seconds / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s", "frac": ach / peaks["hbm"],
+                "peak_source": f"hbm_gbs of {peaks['kind']} peaks (copy)"}
+    ach = ops / seconds / 1e12
+    return {"bound": "tensor", "achieved": ach, "peak": int8, "unit": "TOPS", "frac": ach / int8,
+            "frac_of_sustained": ach / (INT8_PER_BF16 * peaks["bf16_sus"]),
+            "peak_source": f"INT8 = {INT8_PER_BF16:g} x bf16_tflops (burst) of {peaks['kind']} peaks"}
 
 
 class ClockSampler:
@@ -127,6 +141,7 @@ class ClockSampler:
         self.error = None
         self._stop = None
         self._thread = None
+        self.max_mhz = None
 
     def _run(self, ready):
         import pynvml as nv
@@ -176,122 +191,288 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
+def fmt_name(fmt):
+    return "W4A8 per-channel" if fmt == 0 else ("W4A8 g128" if fmt == 1 else "W8A8")
+
+
 # ---------------------------------------------------------------------------
 # reference arm: the CPU oracle on a bounded sample
 # ---------------------------------------------------------------------------
 
 class OracleSample:
-    """The CPU oracle on a bounded sample of the workload: every linear at
-    ``sample_m`` tokens (one weight copy).  Packing is offline and untimed."""
+    """The CPU oracle on a bounded sample of the workload: the linears
+    ``shape_ids`` at ``sample_m`` tokens each (one weight copy).  Packing is
+    offline and untimed."""
 
-    def __init__(self, wl, sample_m):
+    def __init__(self, wl, sample_m, shape_ids=None):
         from oracle import oracle
         self.o = oracle
         self.wl = wl
         self.m = sample_m
         self.items = []
-        for si, (name, K, N) in enumerate(wl.shapes):
+        ids = list(range(len(wl.shapes))) if shape_ids is None else shape_ids
+        for si in ids:
+            name, K, N = wl.shapes[si]
             L = synth.layer(wl, si, M=sample_m)
             Xb = np.ascontiguousarray(L["X"]).view(np.uint16)
             Wb = np.ascontiguousarray(L["W"]).view(np.uint16)
             pk = oracle.pack_layer(Wb, L["O"], wl.fmt)
-            self.items.append((Xb, Wb, pk, len(L["O"]), K, N))
-        self.bytes = sum(sum(algorithmic_bytes(sample_m, K, N, nO, wl.fmt)) for _, _, _, nO, K, N in self.items)
+            pk["Bt"] = np.ascontiguousarray(pk["B"].T)
+            self.items.append((name, Xb, Wb, pk, len(L["O"]), K, N))
+        self.bytes = sum(layer_bytes(sample_m, K, N, nO, wl.fmt) for *_, nO, K, N in self.items)
         self.ops = sum(2 * sample_m * K * N for *_, K, N in self.items)
 
     def step(self):
         t0 = time.perf_counter()
-        for Xb, Wb, pk, nO, K, N in self.items:
+        for _, Xb, Wb, pk, nO, K, N in self.items:
             self.o.forward(Xb, Wb, pk, np.ones(nO, np.float32), self.wl.gamma, update_momentum=True)
         return time.perf_counter() - t0
 
     def describe(self, seconds):
-        return (f"every linear of {self.wl.name} ({len(self.items)}) at M={self.m}, one weight copy: "
-                f"momentum update, quantization, int64 GEMM, fp64 dequant; {seconds:.1f} s of "
-                f"single-threaded CPU time; host has {os.cpu_count()} cores")
+        names = ", ".join(it[0] for it in self.items)
+        return (f"{names} of {self.wl.name} at M={self.m}, one weight copy: momentum update, quantization, "
+                f"int64 GEMM, fp64 dequant; {seconds:.2f} s of single-threaded CPU time; "
+                f"host has {os.cpu_count()} cores")
+
+
+def oracle_sample_for(wl):
+    """Bounded oracle sample of a workload (about 10-30 s of CPU time in
+    all, packing included): for the 70B set the two square-ish linears at
+    one token, else every linear at four tokens."""
+    if wl.name == "llama70b_w4g128":
+        return OracleSample(wl, 1, shape_ids=[0, 1])
+    if wl.name == "phi3_w8_quaff":
+        return OracleSample(wl, 2)
+    return OracleSample(wl, 4)
 
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sample = OracleSample(wl, 4)
+    sample = oracle_sample_for(wl)
     for _ in range(args.warmup):
         sample.step()
     t = sum(sample.step() for _ in range(args.steps))
-    gbs = args.steps * sample.bytes / t / 1e9
+    tops = args.steps * sample.ops / t / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64",
-        "data": "synthetic", "tops": args.steps * sample.ops / t / 1e12,
-        "config": {"workload": wl.name, "sample": f"all {len(wl.shapes)} linears at M={sample.m}",
+        "data": "synthetic", "gbs": args.steps * sample.bytes / t / 1e9,
+        "config": {"workload": wl.name, "sample": sample.describe(t / args.steps),
                    "parallelism": "single thread"},
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": 1, "kind": "oracle",
                          "sample": sample.describe(t / args.steps) + " (per step)"},
-        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ---------------------------------------------------------------------------
-# our arm
+# our arm: timing helpers
 # ---------------------------------------------------------------------------
 
-def build_problem(wl, copies, device):
+def graph_of(fn, stream):
     import torch
-    from quantized_linear_layers_token_b200 import qlin
-    layers = []  # per shape: list of PackedLayer copies
-    meta = []
-    for si, (name, K, N) in enumerate(wl.shapes):
-        L = synth.layer(wl, si, M=1)
-        W = torch.from_numpy(L["W"]).to(device)
-        base = qlin.PackedLayer.pack(W, L["O"], wl.fmt)
-        del W
-        cps = [base] + [base.clone() for _ in range(copies - 1)]
-        layers.append(cps)
-        meta.append({"name": name, "K": K, "N": N, "O": L["O"]})
-    inputs = {}
-    for M in wl.ms:
+    with torch.cuda.stream(stream):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def replay_median_ms(graph, stream, reps, warm=3):
+    """Median over `reps` replays, each bracketed by its own CUDA events on
+    the launch stream."""
+    import torch
+    for _ in range(warm):
+        with torch.cuda.stream(stream):
+            graph.replay()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for e0, e1 in evs:
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+
+
+class ForwardWorkload:
+    """Packed weights, inputs, outputs and workspaces of one forward workload
+    on one device: slot = (M, copy, linear)."""
+
+    GROUP_MAX_M = 64     # token counts the grouped entry point takes
+    GROUP_MAX_COUNT = 32  # problems per grouped call
+
+    def __init__(self, wl, copies, device, ms=None, grouped=True):
+        import torch
+        from quantized_linear_layers_token_b200 import qlin
+        self.q = qlin
+        self.wl = wl
+        self.copies = copies
+        self.grouped = grouped
+        self.device = device
+        self._group_ws = {}
+        self.ms = list(wl.ms if ms is None else ms)
+        self.meta = []
+        layers = []
         for si, (name, K, N) in enumerate(wl.shapes):
-            L = synth.layer(wl, si, M=M, with_weights=False)
-            inputs[(M, si)] = L["X"]
-    return layers, meta, inputs
+            L = synth.layer(wl, si, M=1)
+            W = torch.from_numpy(L["W"]).to(device)
+            base = qlin.PackedLayer.pack(W, L["O"], wl.fmt)
+            del W
+            layers.append([base] + [base.clone() for _ in range(copies - 1)])
+            self.meta.append({"name": name, "K": K, "N": N, "nO": len(L["O"])})
+        self.layers = layers
+        self.x_np = {}
+        self.slots = []
+        for M in self.ms:
+            for si, (name, K, N) in enumerate(wl.shapes):
+                self.x_np[(M, si)] = synth.layer(wl, si, M=M, with_weights=False)["X"]
+            for c in range(copies):
+                for si in range(len(wl.shapes)):
+                    lay = layers[si][c]
+                    nO = self.meta[si]["nO"]
+                    nws = qlin.qlin_forward_workspace(M, lay.w)
+                    self.slots.append({
+                        "M": M, "si": si, "c": c, "layer": lay,
+                        "X": torch.from_numpy(self.x_np[(M, si)]).to(device),
+                        "Y": torch.empty((M, self.meta[si]["N"]), dtype=torch.float16, device=device),
+                        "s": torch.ones(max(nO, 1), dtype=torch.float32, device=device),
+                        "ws": qlin.empty_workspace(nws, device), "nws": nws})
+
+    def ops(self, slots=None):
+        return sum(2 * sl["M"] * self.meta[sl["si"]]["K"] * self.meta[sl["si"]]["N"] for sl in (slots or self.slots))
+
+    def bytes(self, slots=None):
+        return sum(layer_bytes(sl["M"], self.meta[sl["si"]]["K"], self.meta[sl["si"]]["N"], self.meta[sl["si"]]["nO"],
+                               self.wl.fmt) for sl in (slots or self.slots))
+
+    def forward(self, sl, stream, update=True):
+        self.q.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], self.wl.gamma, update, sl["Y"], sl["ws"],
+                            sl["nws"], stream)
+
+    def units(self, slots):
+        """Launch units of a list of slots: decode-sized token counts go in
+        groups of up to 32 independent linears (one qlin_forward_grouped
+        call each), larger ones one qlin_forward call per linear."""
+        out, pend = [], {}
+        for sl in slots:
+            if self.grouped and sl["M"] <= self.GROUP_MAX_M:
+                pend.setdefault(sl["M"], []).append(sl)
+            else:
+                out.append([sl])
+        for M, sls in pend.items():
+            for i in range(0, len(sls), self.GROUP_MAX_COUNT):
+                out.append(sls[i:i + self.GROUP_MAX_COUNT])
+        return out
+
+    def run_unit(self, unit, stream, update=True):
+        if len(unit) == 1 and not (self.grouped and unit[0]["M"] <= self.GROUP_MAX_M):
+            self.forward(unit[0], stream, update)
+            return
+        key = tuple(id(sl) for sl in unit)
+        if key not in self._group_ws:
+            n = self.q.qlin_forward_grouped_workspace([sl["layer"].w for sl in unit], unit[0]["M"])
+            self._group_ws[key] = (n, self.q.empty_workspace(n, self.device))
+        n, ws = self._group_ws[key]
+        self.q.qlin_forward_grouped([sl["layer"].w for sl in unit], [sl["X"] for sl in unit], [sl["s"] for sl in unit],
+                                    [sl["Y"] for sl in unit], unit[0]["M"], self.wl.gamma, update, ws, n, stream)
+
+    def run(self, slots, stream, side=()):
+        """Independent launch units round-robin over the launch stream and
+        the side streams (forked from and joined back into the launch
+        stream)."""
+        import torch
+        units = self.units(slots)
+        if not side:
+            for u in units:
+                self.run_unit(u, stream)
+            return
+        streams = [stream, *side]
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for st in side:
+            st.wait_event(fork)
+        for j, u in enumerate(units):
+            self.run_unit(u, streams[j % len(streams)])
+        for st in side:
+            done = torch.cuda.Event()
+            done.record(st)
+            stream.wait_event(done)
+
+    def bucket(self, M):
+        return [sl for sl in self.slots if sl["M"] == M]
+
+    def measure_buckets(self, stream, side, reps, peaks):
+        """Per token count: the forwards of that bucket (one graph, median of
+        replays) and its GEMM calls alone on one stream."""
+        import torch
+        q = self.q
+        out = []
+        for M in self.ms:
+            sls = self.bucket(M)
+            g = graph_of(lambda: self.run(sls, stream, side), stream)
+            ms = replay_median_ms(g, stream, reps)
+            del g
+            ops, nbytes = self.ops(sls), self.bytes(sls)
+            rec = {"M": M, "forwards": len(sls), "ms": ms, "tops": ops / (ms * 1e-3) / 1e12,
+                   "gbs": nbytes / (ms * 1e-3) / 1e9, "algorithmic_bytes": nbytes, "ops": ops,
+                   "roofline": roofline_of(ops, nbytes, ms * 1e-3, peaks)}
+            # GEMM calls alone (quantized inputs prepared once, untimed)
+            gsl = []
+            for sl in sls:
+                K, nO = self.meta[sl["si"]]["K"], self.meta[sl["si"]]["nO"]
+                Xq = torch.empty((M, K), dtype=torch.int8, device=stream.device)
+                a = torch.empty(M, dtype=torch.float32, device=stream.device)
+                XqO = torch.empty((M, max(nO, 1)), dtype=torch.int8, device=stream.device)
+                naws = q.qlin_quant_act_workspace(M, sl["layer"].w)
+                aws = q.empty_workspace(naws, stream.device)
+                q.qlin_quant_act(sl["X"], M, sl["layer"].w, sl["s"], self.wl.gamma, False, Xq, a, XqO, aws, naws,
+                                 stream)
+                gsl.append((sl, Xq, a, XqO))
+
+            def gemms():
+                for sl, Xq, a, XqO in gsl:
+                    q.qlin_gemm(sl["layer"].w, Xq, a, XqO, sl["s"], M, sl["Y"], None, sl["ws"], sl["nws"], stream)
+            g = graph_of(gemms, stream)
+            gms = replay_median_ms(g, stream, reps)
+            del g
+            gbytes = sum(algorithmic_bytes(M, self.meta[sl["si"]]["K"], self.meta[sl["si"]]["N"],
+                                           self.meta[sl["si"]]["nO"], self.wl.fmt)[0] for sl, *_ in gsl)
+            rec["gemm"] = {"ms": gms, "launches": len(gsl), "algorithmic_bytes": gbytes,
+                           "roofline": roofline_of(ops, gbytes, gms * 1e-3, peaks)}
+            q.qlin_poll_device_status(stream)
+            out.append(rec)
+            del gsl
+        return out
+
+    def describe(self):
+        return {"workload": self.wl.name, "shapes": [[n, K, N] for n, K, N in self.wl.shapes], "M": self.ms,
+                "format": fmt_name(self.wl.fmt), "outlier_frac": self.wl.outlier_frac, "gamma": self.wl.gamma,
+                "weight_copies": self.copies, "forwards_per_step": len(self.slots)}
 
 
-def run_profile_case(args, wl):
-    """A few qlin_forward calls on one linear of the workload (one weight
-    copy), launched eagerly so a profiler sees every kernel: W warm-up
-    calls, then K calls timed with CUDA events."""
-    import torch
-    from quantized_linear_layers_token_b200 import qlin
-    name, m = args.profile_case.split(":")
-    M = int(m)
-    si = [n for n, _, _ in wl.shapes].index(name)
-    _, K, N = wl.shapes[si]
-    L = synth.layer(wl, si, M=M)
-    layer = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).cuda(), L["O"], wl.fmt)
-    X = torch.from_numpy(L["X"]).cuda()
-    s = torch.ones(max(len(L["O"]), 1), dtype=torch.float32, device="cuda")
-    Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
-    nws = qlin.qlin_forward_workspace(M, layer.w)
-    ws = qlin.empty_workspace(nws)
-    for _ in range(args.warmup):
-        qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
-    e1.record()
-    torch.cuda.synchronize()
-    qlin.qlin_poll_device_status()
-    us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
-    print(json.dumps({"profile_case": args.profile_case, "workload": wl.name, "K": K, "N": N, "M": M,
-                      "us_per_forward_eager": us}), flush=True)
-    return 0
+def measure_workload_record(wl, copies, device, stream, side, reps, peaks, grouped=True):
+    """Sub-record of a further workload: one step (all its forwards) as the
+    median of graph replays, and its buckets."""
+    fw = ForwardWorkload(wl, copies, device, grouped=grouped)
+    g = graph_of(lambda: fw.run(fw.slots, stream, side), stream)
+    ms = replay_median_ms(g, stream, reps)
+    del g
+    ops, nbytes = fw.ops(), fw.bytes()
+    rec = {"ms_per_step": ms, "tops": ops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
+           "roofline": roofline_of(ops, nbytes, ms * 1e-3, peaks), "config": fw.describe(),
+           "buckets": fw.measure_buckets(stream, side, reps, peaks),
+           "timing": f"median of {reps} CUDA-graph replays, CUDA events on the launch stream"}
+    fw.q.qlin_poll_device_status(stream)
+    return rec
 
 
 # ---------------------------------------------------------------------------
@@ -358,13 +539,49 @@ def run_backward_reference(args, wl):
     return 0
 
 
+class BackwardWorkload:
+    def __init__(self, wl, M, device):
+        import torch
+        from quantized_linear_layers_token_b200 import qlin
+        self.q = qlin
+        self.wl = wl
+        self.M = M
+        self.slots = []
+        for si, (name, K, N) in enumerate(wl.shapes):
+            L = synth.layer(wl, si, M=1)
+            lay = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).to(device), L["O"], wl.fmt)
+            dY_np = synth.grad_output(wl.index, si, M, N)
+            s_np = synth.outlier_scales(wl.index, si, len(L["O"]))
+            nws = qlin.qlin_backward_dx_workspace(M, lay.w)
+            self.slots.append({"layer": lay, "K": K, "N": N, "nO": len(L["O"]), "dY_np": dY_np,
+                               "ws": qlin.empty_workspace(nws, device) if nws else None, "nws": nws,
+                               "dY": torch.from_numpy(dY_np).to(device),
+                               "s": torch.from_numpy(s_np).to(device) if len(L["O"]) else None,
+                               "dX": torch.empty((M, K), dtype=torch.float16, device=device)})
+        self.flops = bwd_flops(M, wl.shapes)
+
+    def call(self, sl, stream):
+        self.q.qlin_backward_dx(sl["layer"].w, sl["dY"], self.M, sl["s"], sl["dX"], sl["ws"], sl["nws"], stream)
+
+    def step(self, stream):
+        for sl in self.slots:
+            self.call(sl, stream)
+
+
+def backward_roofline(flops, ms, peaks):
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_sus"], "frac_of_burst": achieved / peaks["bf16"], "traffic": None,
+            "peak_source": f"bf16_tflops_sustained of {peaks['kind']} peaks (fp16 and bf16 have the same "
+                           f"dense tensor rate)"}
+
+
 def run_backward(args, wl):
     """One step = qlin_backward_dx on every linear of the workload at
     ``--tokens`` tokens (the fine-tuning backward through the frozen
     quantized weights).  N > 1: every rank runs its own token batch, no
     collective (the input gradient has no exchange step)."""
     import torch
-    from quantized_linear_layers_token_b200 import qlin
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -377,61 +594,36 @@ def run_backward(args, wl):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     M = args.tokens
+    bw = BackwardWorkload(wl, M, device)
+    stream = torch.cuda.Stream(device)
     if args.profile_case:
-        # one linear, eager launches, so a profiler sees each kernel
-        si = [n for n, _, _ in wl.shapes].index(args.profile_case)
-        _, K, N = wl.shapes[si]
-        L = synth.layer(wl, si, M=1)
-        lay = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).to(device), L["O"], wl.fmt)
-        dY = torch.from_numpy(synth.grad_output(wl.index, si, M, N)).to(device)
-        s = torch.from_numpy(synth.outlier_scales(wl.index, si, len(L["O"]))).to(device) if len(L["O"]) else None
-        dX = torch.empty((M, K), dtype=torch.float16, device=device)
-        nws = qlin.qlin_backward_dx_workspace(M, lay.w)
-        ws = qlin.empty_workspace(nws) if nws else None
+        sl = bw.slots[[n for n, _, _ in wl.shapes].index(args.profile_case)]
         for _ in range(args.warmup):
-            qlin.qlin_backward_dx(lay.w, dY, M, s, dX, ws, nws)
+            bw.call(sl, stream)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
+        e0.record(stream)
         for _ in range(args.steps):
-            qlin.qlin_backward_dx(lay.w, dY, M, s, dX, ws, nws)
-        e1.record()
+            bw.call(sl, stream)
+        e1.record(stream)
         torch.cuda.synchronize()
-        qlin.qlin_poll_device_status()
+        bw.q.qlin_poll_device_status()
         us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
-        print(json.dumps({"profile_case": args.profile_case, "op": "backward", "workload": wl.name, "K": K, "N": N,
-                          "M": M, "us_per_call_eager": us, "tflops": 2 * M * N * K / us / 1e6}), flush=True)
+        print(json.dumps({"profile_case": args.profile_case, "op": "backward", "workload": wl.name, "K": sl["K"],
+                          "N": sl["N"], "M": M, "us_per_call_eager": us,
+                          "tflops": 2 * M * sl["N"] * sl["K"] / us / 1e6}), flush=True)
         return 0
-    slots = []
-    for si, (name, K, N) in enumerate(wl.shapes):
-        L = synth.layer(wl, si, M=1)
-        lay = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).to(device), L["O"], wl.fmt)
-        dY_np = synth.grad_output(wl.index, si, M, N)
-        s_np = synth.outlier_scales(wl.index, si, len(L["O"]))
-        nws = qlin.qlin_backward_dx_workspace(M, lay.w)
-        slots.append({"layer": lay, "K": K, "N": N, "nO": len(L["O"]), "dY_np": dY_np,
-                      "ws": qlin.empty_workspace(nws) if nws else None, "nws": nws,
-                      "dY": torch.from_numpy(dY_np).to(device),
-                      "s": torch.from_numpy(s_np).to(device) if len(L["O"]) else None,
-                      "dX": torch.empty((M, K), dtype=torch.float16, device=device)})
-    stream = torch.cuda.Stream(device)
-
-    def step():
-        for sl in slots:
-            qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], sl["ws"], sl["nws"], stream)
-
     for _ in range(max(1, args.warmup)):
-        step()
+        with torch.cuda.stream(stream):
+            bw.step(stream)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
+    graph = graph_of(lambda: bw.step(stream), stream)
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
             graph.replay()
     torch.cuda.synchronize()
-    qlin.qlin_poll_device_status()
+    bw.q.qlin_poll_device_status()
 
     if dist is not None:
         dist.barrier()
@@ -453,24 +645,16 @@ def run_backward(args, wl):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
     clocks = clk.summary()
-    flops = bwd_flops(M, wl.shapes)
-    value = world * flops / (ms_step * 1e-3) / 1e12
-
-    # the step is nothing but backward_dx_kernel launches: their average
-    # duration is the step time over the launches of a step
-    hbm, bf16, bf16_sus, peak_kind = read_peaks()
-    achieved = flops / (ms_step * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_sus, "unit": "TFLOP/s",
-                "frac": achieved / bf16_sus, "frac_of_burst": achieved / bf16, "traffic": None,
-                "peak_source": f"bf16_tflops_sustained of {peak_kind} peaks (fp16 and bf16 have the same "
-                               f"dense tensor rate; kernel timed inside a seconds-long loop)",
-                "kernel": "backward_dx_kernel, all launches of one step", "flops_per_step": flops,
-                "launches_per_step": len(slots)}
+    peaks = read_peaks()
+    value = world * bw.flops / (ms_step * 1e-3) / 1e12
+    roofline = backward_roofline(bw.flops, ms_step, peaks)
+    roofline.update({"kernel": "backward_dx_kernel, all launches of one step", "flops_per_step": bw.flops,
+                     "launches_per_step": len(bw.slots)})
 
     e2e = None
     if world == 1:
-        host_dy = [torch.from_numpy(sl["dY_np"]).pin_memory() for sl in slots]
-        host_dx = [torch.empty(sl["dX"].shape, dtype=torch.float16).pin_memory() for sl in slots]
+        host_dy = [torch.from_numpy(sl["dY_np"]).pin_memory() for sl in bw.slots]
+        host_dx = [torch.empty(sl["dX"].shape, dtype=torch.float16).pin_memory() for sl in bw.slots]
         h2d = sum(x.numel() * 2 for x in host_dy)
         d2h = sum(y.numel() * 2 for y in host_dx)
         h2d_stream = torch.cuda.Stream(device)
@@ -481,14 +665,14 @@ def run_backward(args, wl):
             d2h_stream.wait_stream(stream)
             ready = []
             with torch.cuda.stream(h2d_stream):
-                for sl, hy in zip(slots, host_dy):
+                for sl, hy in zip(bw.slots, host_dy):
                     sl["dY"].copy_(hy, non_blocking=True)
                     ev = torch.cuda.Event()
                     ev.record(h2d_stream)
                     ready.append(ev)
-            for sl, hx, ev in zip(slots, host_dx, ready):
+            for sl, hx, ev in zip(bw.slots, host_dx, ready):
                 stream.wait_event(ev)
-                qlin.qlin_backward_dx(sl["layer"].w, sl["dY"], M, sl["s"], sl["dX"], sl["ws"], sl["nws"], stream)
+                bw.call(sl, stream)
                 done = torch.cuda.Event()
                 done.record(stream)
                 d2h_stream.wait_event(done)
@@ -497,12 +681,7 @@ def run_backward(args, wl):
             stream.wait_stream(h2d_stream)
             stream.wait_stream(d2h_stream)
 
-        with torch.cuda.stream(stream):
-            e2e_step()
-        torch.cuda.synchronize()
-        g3 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g3, stream=stream):
-            e2e_step()
+        g3 = graph_of(e2e_step, stream)
         with torch.cuda.stream(stream):
             g3.replay()
         torch.cuda.synchronize()
@@ -513,7 +692,7 @@ def run_backward(args, wl):
         ev1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = ev0.elapsed_time(ev1) / args.steps
-        e2e = {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": bw.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "note": "per linear: pinned host dY -> device (copy stream), qlin_backward_dx (compute stream), "
                        "device -> pinned host dX (second copy stream); one CUDA graph per step"}
@@ -526,19 +705,19 @@ def run_backward(args, wl):
                "sample": sample.describe(t)}
 
     if rank == 0:
-        dy_bytes = sum(sl["dY"].numel() * 2 for sl in slots)
+        dy_bytes = sum(sl["dY"].numel() * 2 for sl in bw.slots)
         line = {
             "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16 (f32 accumulate)", "data": "synthetic",
             "config": {"workload": wl.name, "op": "backward", "tokens": M,
                        "shapes": [[n, K, N] for n, K, N in wl.shapes], "outlier_frac": wl.outlier_frac,
-                       "format": "W4A8 per-channel" if wl.fmt == 0 else ("W4A8 g128" if wl.fmt == 1 else "W8A8"),
+                       "format": fmt_name(wl.fmt),
                        "l2": f"inputs larger than L2 (dY of one step {dy_bytes / 1e6:.0f} MB)",
                        "parallelism": f"dp{world}",
                        "timing": "CUDA graph of one step, CUDA events on the launch stream"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * len(slots),
+            "gpu_launches": args.steps * len(bw.slots),
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
         }
@@ -549,34 +728,118 @@ def run_backward(args, wl):
     return 0
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama7b_w4_decode")
-    ap.add_argument("--copies", type=int, default=4)
-    ap.add_argument("--streams", type=int, default=4,
-                    help="compute streams the independent forwards of a step are spread over (N = 1)")
-    ap.add_argument("--op", default="forward", choices=["forward", "backward"],
-                    help="backward: the input gradient of every linear (default workload phi3_w8_quaff)")
-    ap.add_argument("--tokens", type=int, default=4096, help="--op backward: tokens per step")
-    ap.add_argument("--profile-case", default=None,
-                    help="NAME:M -- run only that linear of the workload at M tokens (for ncu captures)")
-    args = ap.parse_args()
-    if args.op == "backward":
-        wl = synth.WORKLOADS["phi3_w8_quaff" if args.workload == "llama7b_w4_decode" else args.workload]
-        return run_backward_reference(args, wl) if args.impl == "reference" else run_backward(args, wl)
-    wl = synth.WORKLOADS[args.workload]
+def gptq_bytes(K, N):
+    """Bytes the Hessian-compensated quantization must move at least once
+    per step of its three phases, fp64: the Gauss-Jordan step c reads and
+    writes the K x (K - c) active part of the eliminated matrix and all of
+    the inverse; the compensation step i reads and writes the N x (K - i - 1)
+    not-yet-quantized weights and the (K - i - 1)^2 remaining inverse."""
+    gj = sum(16 * K * ((K - c) + K) for c in range(K))
+    steps = sum(16 * (N * (K - i - 1) + (K - i - 1) ** 2) for i in range(K))
+    return gj, steps
 
-    if args.impl == "reference":
-        return run_reference(args, wl)
-    if args.profile_case:
-        return run_profile_case(args, wl)
 
+def gptq_record(device, stream, peaks, K=4096, N=4096, ns=8192, reps=2):
+    """Hessian-compensated quantization of a 7B q_proj-shaped layer (K = N =
+    4096, INT4 grid, per-channel steps) from 8192 synthetic calibration
+    tokens: H = 2 X^T X, Gauss-Jordan inverse, column-sequential
+    compensation.  HBM-bound streaming kernels (fp64)."""
     import torch
     from quantized_linear_layers_token_b200 import qlin
+    rng = synth.rng_for(9, 0)
+    X = torch.from_numpy(rng.standard_normal((ns, K))).to(device)
+    W0 = torch.from_numpy(rng.standard_normal((K, N)) * 0.02).to(device)
+    scale = (W0.abs().amax(dim=0) / 7).contiguous()
+    W = torch.empty_like(W0)
+    codes = torch.empty((K, N), dtype=torch.int8, device=device)
+    Hinv = torch.empty((K, K), dtype=torch.float64, device=device)
+    sing = torch.zeros(1, dtype=torch.int32, device=device)
+    n = qlin.qlin_gptq_workspace(K, N)
+    ws = qlin.empty_workspace(n, device)
+    times = []
+    for r in range(reps + 1):
+        W.copy_(W0)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        qlin.qlin_gptq_quantize(X, ns, K, N, W, scale, 7, codes, Hinv, sing, ws, n, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if r:
+            times.append(e0.elapsed_time(e1))
+    qlin.qlin_poll_device_status(stream)
+    ms = statistics.median(times)
+    gj, st = gptq_bytes(K, N)
+    nbytes = gj + st + 8 * ns * K + 16 * K * N
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"op": "gptq", "K": K, "N": N, "calibration_tokens": ns, "ms": ms, "singular": int(sing.item()),
+            "hessian_flops": 2 * ns * K * K, "launches": 4 * K + 3,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm"], "algorithmic_bytes": nbytes,
+                         "peak_source": f"hbm_gbs of {peaks['kind']} peaks (copy)"},
+            "timing": f"median of {reps} calls, CUDA events on the launch stream"}
+
+
+def backward_record(device, stream, reps, peaks):
+    import torch  # noqa: F401
+    wl = synth.WORKLOADS["phi3_w8_quaff"]
+    bw = BackwardWorkload(wl, 4096, device)
+    g = graph_of(lambda: bw.step(stream), stream)
+    ms = replay_median_ms(g, stream, reps)
+    del g
+    bw.q.qlin_poll_device_status(stream)
+    return {"op": "backward", "workload": wl.name, "tokens": bw.M, "ms_per_step": ms,
+            "tflops": bw.flops / (ms * 1e-3) / 1e12, "roofline": backward_roofline(bw.flops, ms, peaks),
+            "launches_per_step": len(bw.slots),
+            "timing": f"median of {reps} CUDA-graph replays of qlin_backward_dx on every linear"}
+
+
+# ---------------------------------------------------------------------------
+# --profile-case: one linear, eager launches (for ncu)
+# ---------------------------------------------------------------------------
+
+def run_profile_case(args, wl):
+    """A few qlin_forward calls on one linear of the workload (one weight
+    copy), launched eagerly so a profiler sees every kernel: W warm-up
+    calls, then K calls timed with CUDA events."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    name, m = args.profile_case.split(":")
+    M = int(m)
+    si = [n for n, _, _ in wl.shapes].index(name)
+    _, K, N = wl.shapes[si]
+    L = synth.layer(wl, si, M=M)
+    layer = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).cuda(), L["O"], wl.fmt)
+    X = torch.from_numpy(L["X"]).cuda()
+    s = torch.ones(max(len(L["O"]), 1), dtype=torch.float32, device="cuda")
+    Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    nws = qlin.qlin_forward_workspace(M, layer.w)
+    ws = qlin.empty_workspace(nws)
+    for _ in range(args.warmup):
+        qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
+    e1.record()
+    torch.cuda.synchronize()
+    qlin.qlin_poll_device_status()
+    us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
+    print(json.dumps({"profile_case": args.profile_case, "workload": wl.name, "K": K, "N": N, "M": M,
+                      "us_per_forward_eager": us}), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm: the forward step
+# ---------------------------------------------------------------------------
+
+def run_forward(args, wl):
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    from quantized_linear_layers_token_b200.dp import ColmaxExchange
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -588,94 +851,52 @@ def main():
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    layers, meta, inputs_np = build_problem(wl, args.copies, device)
-    ms = wl.ms
-    nshape = len(wl.shapes)
-
-    # per (M, shape, copy): device input, output, momentum state, workspace
-    slots = []
-    for M in ms:
-        for c in range(args.copies):
-            for si in range(nshape):
-                lay = layers[si][c]
-                X = torch.from_numpy(inputs_np[(M, si)]).to(device)
-                Y = torch.empty((M, meta[si]["N"]), dtype=torch.float16, device=device)
-                s = torch.ones(max(len(meta[si]["O"]), 1), dtype=torch.float32, device=device)
-                nws = qlin.qlin_forward_workspace(M, lay.w)
-                ws = qlin.empty_workspace(nws)
-                slots.append({"M": M, "si": si, "c": c, "layer": lay, "X": X, "Y": Y, "s": s, "ws": ws,
-                              "nws": nws})
+    peaks = read_peaks()
+    copies = args.copies if args.copies else (4 if wl.name == "llama7b_w4_decode" else 1)
+    fw = ForwardWorkload(wl, copies, device, grouped=bool(args.grouped))
+    meta = fw.meta
     stream = torch.cuda.Stream(device)
-
-    # DP exchange (N > 1): all outlier column maxima of a step in one vector
-    from quantized_linear_layers_token_b200.dp import ColmaxExchange
-    xchg = ColmaxExchange([len(meta[sl["si"]]["O"]) for sl in slots], device)
-
-    # Independent forwards of a step go round-robin to --streams compute
-    # streams forked from (and joined back into) the launch stream, so one
-    # GEMM's tail overlaps the next one's weight streaming on other SMs.
+    xchg = ColmaxExchange([meta[sl["si"]]["nO"] for sl in fw.slots], device)
     nstreams = max(1, args.streams) if world == 1 else 1
     side = [torch.cuda.Stream(device) for _ in range(nstreams - 1)]
 
     def step_single():
-        if nstreams == 1:
-            for sl in slots:
-                qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
-                                  sl["nws"], stream)
-            return
-        streams = [stream] + side
-        fork = torch.cuda.Event()
-        fork.record(stream)
-        for st in side:
-            st.wait_event(fork)
-        for j, sl in enumerate(slots):
-            qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
-                              sl["nws"], streams[j % nstreams])
-        for st in side:
-            done = torch.cuda.Event()
-            done.record(st)
-            stream.wait_event(done)
+        fw.run(fw.slots, stream, side)
 
     def step_dp():
-        for j, sl in enumerate(slots):
+        for j, sl in enumerate(fw.slots):
             if xchg.n_outliers[j]:
                 qlin.qlin_outlier_colmax(sl["X"], sl["M"], sl["layer"].w, xchg.view(j), stream)
         with torch.cuda.stream(stream):
             xchg.allreduce()
-        for j, sl in enumerate(slots):
+        for j, sl in enumerate(fw.slots):
             lay = sl["layer"]
             if xchg.n_outliers[j]:
                 qlin.qlin_momentum_update(lay.w, xchg.view(j), sl["s"], wl.gamma, stream)
-            # quantization with the already-updated state, then the GEMM
-            qlin.qlin_forward(sl["X"], sl["M"], lay.w, sl["s"], wl.gamma, False, sl["Y"], sl["ws"], sl["nws"],
-                              stream)
+            fw.forward(sl, stream, update=False)  # quantize with the already-updated state, then the GEMM
 
     step = step_single if world == 1 else step_dp
-
-    # warm-up (eager; sets kernel attributes and resolves the driver entry point)
     for _ in range(max(1, args.warmup)):
-        step()
+        with torch.cuda.stream(stream):
+            step()
     torch.cuda.synchronize()
-
     graph = None
     if world == 1:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            step()
+        graph = graph_of(step, stream)
         for _ in range(args.warmup):
-            graph.replay()
+            with torch.cuda.stream(stream):
+                graph.replay()
         torch.cuda.synchronize()
 
     def run_steps(k):
         for _ in range(k):
-            if graph is not None:
-                with torch.cuda.stream(stream):
+            with torch.cuda.stream(stream):
+                if graph is not None:
                     graph.replay()
-            else:
-                step()
+                else:
+                    step()
 
-    # ---------------------------------------------------------------- timed region
+    # ------------------------------------------------------------ timed region
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -694,221 +915,191 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
     clocks = clk.summary()
+    qlin.qlin_poll_device_status(stream)
+    step_ops, step_bytes = fw.ops(), fw.bytes()
+    value = world * step_ops / (ms_step * 1e-3) / 1e12
 
-    step_bytes = 0
-    step_ops = 0
-    gemm_bytes = 0
-    for sl in slots:
-        m = meta[sl["si"]]
-        g, a = algorithmic_bytes(sl["M"], m["K"], m["N"], len(m["O"]), wl.fmt)
-        step_bytes += g + a
-        gemm_bytes += g
-        step_ops += 2 * sl["M"] * m["K"] * m["N"]
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    line = None
+    if rank == 0:
+        reps = max(20, args.reps)
+        buckets = fw.measure_buckets(stream, side, reps, peaks) if world == 1 else None
+        # the dominant kernel: the GEMM calls of the tensor-bound buckets
+        roofline = None
+        if buckets:
+            tb = [b for b in buckets if b["gemm"]["roofline"]["bound"] == "tensor"] or buckets
+            g_ms = sum(b["gemm"]["ms"] for b in tb)
+            g_ops = sum(b["ops"] for b in tb)
+            g_bytes = sum(b["gemm"]["algorithmic_bytes"] for b in tb)
+            roofline = roofline_of(g_ops, g_bytes, g_ms * 1e-3, peaks)
+            roofline.update({
+                "kernel": "qlin_gemm (INT4 widened once per call, then the tcgen05 INT8 GEMM with the fused "
+                          "dequant and compensation), all calls of the buckets M in "
+                          f"{[b['M'] for b in tb]}, one stream",
+                "ms": g_ms, "launches": sum(b["gemm"]["launches"] for b in tb),
+                "ops": g_ops, "algorithmic_bytes": g_bytes, "traffic": None,
+                "timing": f"sum over the buckets of the median of {reps} CUDA-graph replays"})
 
-    # ---------------------------------------------------------------- GEMM-only timing (roofline)
-    gemm_slots = []
-    for sl in slots:
-        M, lay = sl["M"], sl["layer"]
-        K, nO = meta[sl["si"]]["K"], len(meta[sl["si"]]["O"])
-        Xq = torch.empty((M, K), dtype=torch.int8, device=device)
-        a = torch.empty(M, dtype=torch.float32, device=device)
-        XqO = torch.empty((M, max(nO, 1)), dtype=torch.int8, device=device)
-        naws = qlin.qlin_quant_act_workspace(M, lay.w)
-        aws = qlin.empty_workspace(naws)
-        qlin.qlin_quant_act(sl["X"], M, lay.w, sl["s"], wl.gamma, False, Xq, a, XqO, aws, naws, stream)
-        gemm_slots.append((sl, Xq, a, XqO, aws, naws))
-    torch.cuda.synchronize()
+        # ------------------------------------------------------------ end to end through the API
+        e2e = None
+        if world == 1:
+            host_x = [torch.from_numpy(fw.x_np[(sl["M"], sl["si"])]).pin_memory() for sl in fw.slots]
+            host_y = [torch.empty(sl["Y"].shape, dtype=torch.float16).pin_memory() for sl in fw.slots]
+            h2d = sum(x.numel() * 2 for x in host_x)
+            d2h = sum(y.numel() * 2 for y in host_y)
+            h2d_stream = torch.cuda.Stream(device)
+            d2h_stream = torch.cuda.Stream(device)
 
-    def gemm_pass():
-        # qlin_gemm = the compensation-operand kernel (when n_O > 0) + the tcgen05 GEMM kernel
-        for sl, Xq, a, XqO, _, _ in gemm_slots:
-            qlin.qlin_gemm(sl["layer"].w, Xq, a, XqO, sl["s"], sl["M"], sl["Y"], None, sl["ws"], sl["nws"], stream)
+            hx_of = {id(sl): hx for sl, hx in zip(fw.slots, host_x)}
+            hy_of = {id(sl): hy for sl, hy in zip(fw.slots, host_y)}
+            units = fw.units(fw.slots)
 
-    gemm_pass()
-    torch.cuda.synchronize()
-    g2 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g2, stream=stream):
-        gemm_pass()
-    for _ in range(3):
-        with torch.cuda.stream(stream):
-            g2.replay()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    reps = max(5, args.steps)
-    e0.record(stream)
-    for _ in range(reps):
-        with torch.cuda.stream(stream):
-            g2.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    gemm_ms = e0.elapsed_time(e1) / reps
-    n_gemm_launches = len(gemm_slots)
+            def e2e_step():
+                h2d_stream.wait_stream(stream)
+                d2h_stream.wait_stream(stream)
+                ready = []
+                with torch.cuda.stream(h2d_stream):
+                    for u in units:
+                        for sl in u:
+                            sl["X"].copy_(hx_of[id(sl)], non_blocking=True)
+                        ev = torch.cuda.Event()
+                        ev.record(h2d_stream)
+                        ready.append(ev)
+                streams = [stream, *side]
+                fork = torch.cuda.Event()
+                fork.record(stream)
+                for st in side:
+                    st.wait_event(fork)
+                for j, (u, ev) in enumerate(zip(units, ready)):
+                    cs = streams[j % len(streams)]
+                    cs.wait_event(ev)
+                    fw.run_unit(u, cs)
+                    done = torch.cuda.Event()
+                    done.record(cs)
+                    d2h_stream.wait_event(done)
+                    with torch.cuda.stream(d2h_stream):
+                        for sl in u:
+                            hy_of[id(sl)].copy_(sl["Y"], non_blocking=True)
+                for st in side:
+                    joined = torch.cuda.Event()
+                    joined.record(st)
+                    stream.wait_event(joined)
+                stream.wait_stream(h2d_stream)
+                stream.wait_stream(d2h_stream)
 
-    # ---------------------------------------------------------------- activation quantization alone
-    # (momentum update + per-token INT8 codes, the forward's own path; one
-    # stream, CUDA graph).  Evidence only: an error is reported in the line,
-    # it does not fail the run.
-    act_quant = None
-    try:
-        def quant_pass():
-            for sl, Xq, a, XqO, aws, naws in gemm_slots:
-                qlin.qlin_quant_act(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, Xq, a, XqO, aws,
-                                    naws, stream)
-
-        quant_pass()
-        torch.cuda.synchronize()
-        g4 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g4, stream=stream):
-            quant_pass()
-        for _ in range(3):
-            with torch.cuda.stream(stream):
-                g4.replay()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(reps):
-            with torch.cuda.stream(stream):
-                g4.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        qlin.qlin_poll_device_status()
-        act_ms = e0.elapsed_time(e1) / reps
-        act_bytes = sum(algorithmic_bytes(sl["M"], meta[sl["si"]]["K"], meta[sl["si"]]["N"],
-                                          len(meta[sl["si"]]["O"]), wl.fmt)[1] for sl, *_ in gemm_slots)
-        act_gbs = act_bytes / (act_ms * 1e-3) / 1e9
-        act_quant = {"bound": "hbm", "achieved": act_gbs, "unit": "GB/s", "algorithmic_bytes": act_bytes,
-                     "ms_per_step": act_ms, "calls_per_step": len(gemm_slots),
-                     "kernel": "qlin_quant_act (colmax above 16 tokens, then quant_kernel), one stream"}
-    except Exception as ex:  # evidence only
-        act_quant = {"error": f"{type(ex).__name__}: {ex}"[:300]}
-
-    hbm, bf16, bf16_sus, peak_kind = read_peaks()
-    achieved = gemm_bytes / (gemm_ms * 1e-3) / 1e9
-    if act_quant is not None and "achieved" in act_quant:
-        act_quant["peak"] = hbm
-        act_quant["frac"] = act_quant["achieved"] / hbm
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": recorded_traffic(wl.name, args.copies),
-                "traffic_unit": "bytes per step (all GEMM launches), ncu dram__bytes_read.sum + dram__bytes_write.sum",
-                "algorithmic_bytes": gemm_bytes,
-                "peak_source": f"hbm_gbs of {peak_kind} peaks (copy burst)",
-                "kernel": "qlin_gemm (comp operand + tcgen05 GEMM), all launches of one step",
-                "ms_per_step": gemm_ms, "launches_per_step": n_gemm_launches}
-
-    # ---------------------------------------------------------------- end to end through the API
-    e2e = None
-    if world == 1:
-        host_x = [torch.from_numpy(inputs_np[(sl["M"], sl["si"])]).pin_memory() for sl in slots]
-        host_y = [torch.empty(sl["Y"].shape, dtype=torch.float16).pin_memory() for sl in slots]
-        h2d = sum(x.numel() * 2 for x in host_x)
-        d2h = sum(y.numel() * 2 for y in host_y)
-
-        # copies overlap compute: every X goes up on its own stream, each
-        # forward waits only for its own input, each Y comes down on a third
-        # stream as soon as its forward has finished
-        h2d_stream = torch.cuda.Stream(device)
-        d2h_stream = torch.cuda.Stream(device)
-
-        def e2e_step():
-            h2d_stream.wait_stream(stream)
-            d2h_stream.wait_stream(stream)
-            ready = []
-            with torch.cuda.stream(h2d_stream):
-                for sl, hx in zip(slots, host_x):
-                    sl["X"].copy_(hx, non_blocking=True)
-                    ev = torch.cuda.Event()
-                    ev.record(h2d_stream)
-                    ready.append(ev)
-            streams = [stream] + side
-            fork = torch.cuda.Event()
-            fork.record(stream)
-            for st in side:
-                st.wait_event(fork)
-            for j, (sl, hy, ev) in enumerate(zip(slots, host_y, ready)):
-                cs = streams[j % nstreams]
-                cs.wait_event(ev)
-                qlin.qlin_forward(sl["X"], sl["M"], sl["layer"].w, sl["s"], wl.gamma, True, sl["Y"], sl["ws"],
-                                  sl["nws"], cs)
-                done = torch.cuda.Event()
-                done.record(cs)
-                d2h_stream.wait_event(done)
-                with torch.cuda.stream(d2h_stream):
-                    hy.copy_(sl["Y"], non_blocking=True)
-            for st in side:
-                joined = torch.cuda.Event()
-                joined.record(st)
-                stream.wait_event(joined)
-            stream.wait_stream(h2d_stream)
-            stream.wait_stream(d2h_stream)
-
-        with torch.cuda.stream(stream):
-            e2e_step()
-        torch.cuda.synchronize()
-        g3 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g3, stream=stream):
-            e2e_step()
-        with torch.cuda.stream(stream):
-            g3.replay()
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(args.steps):
+            g3 = graph_of(e2e_step, stream)
             with torch.cuda.stream(stream):
                 g3.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        e2e = {"value": step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "note": "per linear: pinned host X -> device (copy stream), qlin_forward (the step's compute "
-                       "streams, round-robin), device -> pinned host Y (second copy stream); copies overlap other "
-                       "linears' compute; one CUDA graph per step"}
+            torch.cuda.synchronize()
+            e2e_steps = max(3, min(args.steps, 10))
+            ev0.record(stream)
+            for _ in range(e2e_steps):
+                with torch.cuda.stream(stream):
+                    g3.replay()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            e2e_ms = ev0.elapsed_time(ev1) / e2e_steps
+            del g3
+            e2e = {"value": step_ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+                   "note": "per linear: pinned host X -> device (copy stream), qlin_forward (the step's compute "
+                           "streams), device -> pinned host Y (second copy stream); one CUDA graph per step"}
 
-    # ---------------------------------------------------------------- CPU baseline (rank 0, N = 1)
-    cpu = None
-    if rank == 0 and world == 1:
-        sample = OracleSample(wl, 16)
-        t = sample.step()
-        cpu = {"value": sample.bytes / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": sample.describe(t)}
+        # ------------------------------------------------------------ further workloads
+        workloads = {}
+        if world == 1 and args.extras:
+            for name in [x for x in args.extras.split(",") if x and x != wl.name]:
+                try:
+                    if name == "backward":
+                        workloads[name] = backward_record(device, stream, reps, peaks)
+                    elif name == "gptq":
+                        workloads[name] = gptq_record(device, stream, peaks)
+                    else:
+                        w2 = synth.WORKLOADS[name]
+                        workloads[name] = measure_workload_record(w2, 4 if name == "llama7b_w4_decode" else 1,
+                                                                  device, stream, side, reps, peaks,
+                                                                  grouped=bool(args.grouped))
+                except Exception as ex:  # evidence only: recorded, the headline stands
+                    workloads[name] = {"error": f"{type(ex).__name__}: {ex}"[:400]}
+                torch.cuda.empty_cache()
 
-    # per forward: quantization (+ the column-max kernel when the library
-    # does not fuse the momentum update into quantization, above 16 tokens)
-    # and the GEMM; data-parallel steps run the column-max and momentum
-    # kernels separately around the all-reduce
-    def forward_launches(sl):
-        has_o = len(meta[sl["si"]]["O"]) > 0
-        if world > 1:
-            return 2 + (2 if has_o else 0)
-        return 2 + (1 if has_o and sl["M"] > 16 else 0)
-    gpu_launches = args.steps * sum(forward_launches(sl) for sl in slots)
+        # ------------------------------------------------------------ CPU baseline
+        cpu = None
+        if world == 1:
+            sample = oracle_sample_for(wl)
+            t = sample.step()
+            cpu = {"value": sample.ops / t / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+                   "gbs": sample.bytes / t / 1e9, "sample": sample.describe(t)}
 
-    if rank == 0:
+        def unit_launches(u):
+            M = u[0]["M"]
+            if world > 1:  # colmax + momentum per linear, then quant + GEMM per linear
+                return sum(2 + (2 if meta[sl["si"]]["nO"] > 0 else 0) +
+                           (1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 1024) else 0) for sl in u)
+            colmax = sum(1 for sl in u if meta[sl["si"]]["nO"] > 0 and M > 16)
+            if len(u) > 1 or (fw.grouped and M <= fw.GROUP_MAX_M):
+                return 2 + colmax  # one quantization launch, one GEMM launch for the group
+            widen = 1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 1024) else 0
+            return 2 + widen + colmax
+
         line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "tops": world * step_ops / (ms_step * 1e-3) / 1e12,
-            "config": {"workload": wl.name, "shapes": [[n, K, N] for n, K, N in wl.shapes], "M": ms,
-                       "weight_copies": args.copies,
-                       "weight_bytes_per_step": int(sum(layers[si][0].nbytes for si in range(nshape)) * args.copies
-                                                    * len(ms)),
-                       "l2": "inputs larger than L2 (distinct packed-weight copies rotated each step)",
-                       "outlier_frac": wl.outlier_frac, "gamma": wl.gamma, "format": "W4A8 per-channel"
-                       if wl.fmt == 0 else ("W4A8 g128" if wl.fmt == 1 else "W8A8"),
-                       "parallelism": f"dp{world}", "forwards_per_step": len(slots),
+            "gbs": world * step_bytes / (ms_step * 1e-3) / 1e9, "algorithmic_bytes_per_step": step_bytes,
+            "ops_per_step": step_ops,
+            "config": {**fw.describe(), "parallelism": f"dp{world}", "streams": nstreams,
+                       "l2": "inputs larger than L2 (one step streams "
+                             f"{sum(l[0].nbytes for l in fw.layers) * copies / 1e6:.0f} MB of packed weights and "
+                             f"{sum(x.nbytes for x in fw.x_np.values()) / 1e6:.0f} MB of activations)",
                        "timing": "CUDA graph of one step, CUDA events on the launch stream",
-                       "streams": nstreams},
-            "roofline": roofline, "act_quant": act_quant, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": gpu_launches,
+                       "grouped": "decode token counts (<= 64): the step's linears at that count go through "
+                                  "qlin_forward_grouped, up to 32 per call" if args.grouped else "off"},
+            "roofline": roofline, "buckets": buckets, "workloads": workloads, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * sum(unit_launches(u) for u in (fw.units(fw.slots) if world == 1 else
+                                                                          [[sl] for sl in fw.slots])),
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                        "reasons": clocks["reasons"], "samples": clocks["samples"]},
         }
+    if line is not None:
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--extras", default=DEFAULT_EXTRAS,
+                    help="further workloads measured into the line's `workloads` (comma list; '' for none)")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="distinct packed-weight copies per linear (0: 4 for the 7B decode set, else 1)")
+    ap.add_argument("--streams", type=int, default=4,
+                    help="compute streams the independent forwards of a step are spread over (N = 1)")
+    ap.add_argument("--reps", type=int, default=20, help="graph replays per bucket (median)")
+    ap.add_argument("--grouped", type=int, default=1,
+                    help="1: decode-sized token counts (<= 64) run the step's linears through qlin_forward_grouped "
+                         "(up to 32 per call); 0: one qlin_forward per linear")
+    ap.add_argument("--op", default="forward", choices=["forward", "backward"],
+                    help="backward: the input gradient of every linear (default workload phi3_w8_quaff)")
+    ap.add_argument("--tokens", type=int, default=4096, help="--op backward: tokens per step")
+    ap.add_argument("--profile-case", default=None,
+                    help="NAME:M -- run only that linear of the workload at M tokens (for ncu captures)")
+    args = ap.parse_args()
+    if args.op == "backward":
+        wl = synth.WORKLOADS["phi3_w8_quaff" if args.workload == DEFAULT_WORKLOAD else args.workload]
+        return run_backward_reference(args, wl) if args.impl == "reference" else run_backward(args, wl)
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    if args.profile_case:
+        return run_profile_case(args, wl)
+    return run_forward(args, wl)
 
 
 if __name__ == "__main__":

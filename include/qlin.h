@@ -248,6 +248,31 @@ QLIN_API qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weigh
                          float gamma, int32_t update_momentum, uint16_t* Y, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* Several independent layers in one pass: stage 1 of every problem in one
+ * quantization launch, then stages 2 and 3 of every problem in one
+ * persistent GEMM launch whose CTAs stream the problems' weights back to
+ * back, so the per-launch start-up, the first weight bytes' latency and
+ * each problem's split-K reduction and epilogue overlap the other problems'
+ * weight streaming.  For decode-sized token counts, where a single layer's
+ * weights take a few microseconds to stream: independent projections of
+ * one input (q / k / v, gate / up), or many adapters or experts.  Problem q
+ * computes exactly what qlin_forward(X[q], M, w[q], s[q], gamma,
+ * update_momentum, Y[q], ...) computes (the same arithmetic, bit for bit).
+ *   count     1 .. 32 problems; every w[q] has the same format.
+ *   w, X, s, Y  host arrays of `count` pointers: packed weights, device X
+ *             fp16 [M][K_q], device momentum state fp32 [n_outlier_q] (may
+ *             be NULL for a problem without outliers), device Y fp16
+ *             [M][N_q]; distinct Y buffers.
+ *   M         0 .. 64 tokens, the same for every problem (QLIN_ERR_SHAPE above).
+ *   workspace one buffer for the group, of qlin_forward_grouped_workspace
+ *             bytes, 256-byte aligned, zero-filled before its first use
+ *             and left that way. */
+QLIN_API qlin_status qlin_forward_grouped_workspace(int32_t count, const qlin_weights* const* w, int32_t M,
+                                                    size_t* bytes);
+QLIN_API qlin_status qlin_forward_grouped(int32_t count, const qlin_weights* const* w, const uint16_t* const* X,
+                                          float* const* s, uint16_t* const* Y, int32_t M, float gamma,
+                                          int32_t update_momentum, void* workspace, size_t ws_bytes, void* stream);
+
 /* Input gradient of the layer for fine-tuning (Quaff notes, 损失函数 /
  * 训练策略: the quantizers are passed by the standard straight-through
  * estimator, so the gradient is that of the decoupled layer of 解耦 WAQ 公式
@@ -275,6 +300,38 @@ QLIN_API qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weigh
 QLIN_API qlin_status qlin_backward_dx_workspace(int32_t M, const qlin_weights* w, size_t* bytes);
 QLIN_API qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t M, const float* s,
                                       uint16_t* dX, void* workspace, size_t ws_bytes, void* stream);
+
+/* Hessian-compensated quantization of a layer's weights (offline, before
+ * packing; "QQQ: Quality Quattuor-Bit Quantization for Large Language
+ * Models", section 三 技术架构 -> Hessian补偿): with H = 2 X^T X over the
+ * calibration activations, the input channels i = 0 .. K-1 are quantized in
+ * order and each one's rounding error is compensated on the channels not
+ * yet quantized,
+ *   q_n      = clamp(rne(W[i][n] / scale[n]), -qmax, qmax) * scale[n]
+ *   W[j][n] += -(W[i][n] - q_n) / [H^-1]_ii * [H^-1]_ji     (j > i)
+ *   W[i][n]  = q_n,
+ * after which H^-1 loses row and column i by the rank-one downdate
+ * H^-1 <- H^-1 - H^-1[:, i] H^-1[i, :] / [H^-1]_ii.  H^-1 is H's inverse by
+ * Gauss-Jordan elimination with partial pivoting (the first row of largest
+ * magnitude).  Every step is an fp64 operation rounded to nearest, in this
+ * order, without fused multiply-adds, so the results do not depend on the
+ * GPU's work split.
+ *   X        device fp64 [ns][K] calibration activations (ns >= 1).
+ *   W        device fp64 [K][N] (input channel i is row i), overwritten with
+ *            the quantized values codes * scale.
+ *   scale    device fp64 [N] grid step of each output channel.
+ *   qmax     1 .. 127 (7 for INT4, 127 for INT8).
+ *   codes    device int8 [K][N]: clamp(rne(w / scale)) of each step.
+ *   Hinv     device fp64 [K][K]: H^-1 before any downdate.
+ *   singular device int32 (may be NULL): 1 if a pivot of H was zero (H is
+ *            singular; W, codes and Hinv are then undefined), else 0.
+ *   workspace  qlin_gptq_workspace bytes (one K x K fp64 matrix and a
+ *            little scratch), 256-byte aligned; no zero-fill needed.
+ * K <= 16384.  The call enqueues 4 K + 3 small kernels on `stream`. */
+QLIN_API qlin_status qlin_gptq_workspace(int32_t K, int32_t N, size_t* bytes);
+QLIN_API qlin_status qlin_gptq_quantize(const double* X, int32_t ns, int32_t K, int32_t N, double* W,
+                                        const double* scale, int32_t qmax, int8_t* codes, double* Hinv,
+                                        int32_t* singular, void* workspace, size_t ws_bytes, void* stream);
 
 /* Test and measurement hooks.  The library reads no environment variables:
  * a process that wants a non-default work split, launch mode or wait limit

@@ -94,6 +94,10 @@ def _declare(L):
     L.oq_gptq_downdate.restype = None
     L.oq_gptq_quantize.argtypes = [P, I, I, P, D, I, P, P]
     L.oq_gptq_quantize.restype = I
+    L.oq_gptq_quantize_layer.argtypes = [P, I, I, I, P, P, I, P, P]
+    L.oq_gptq_quantize_layer.restype = I
+    L.oq_smooth_search.argtypes = [P, I, I, P, I, I, P]
+    L.oq_smooth_search.restype = I
     L.oq_invert.argtypes = [P, I, P]
     L.oq_invert.restype = I
 
@@ -300,6 +304,37 @@ def gptq_quantize(X: np.ndarray, w: np.ndarray, scale: float, qmax: int):
     if r:
         raise ValueError("Hessian is singular")
     return w2, Hinv, deltas
+
+
+def gptq_quantize_layer(X: np.ndarray, W: np.ndarray, scale: np.ndarray, qmax: int):
+    """Hessian-compensated quantization of a layer W [d][N] (fp64): every
+    output channel n is oq_gptq_quantize's w with grid step scale[n].
+    Returns (W after compensation = the grid values, codes int8 [d][N],
+    inverse Hessian)."""
+    X = _c(X, np.float64)
+    ns, d = X.shape
+    W2 = np.array(W, dtype=np.float64, copy=True, order="C")
+    assert W2.shape[0] == d
+    N = W2.shape[1]
+    scale = _c(scale, np.float64)
+    codes = np.zeros((d, N), np.int8)
+    Hinv = np.zeros((d, d), np.float64)
+    r = lib().oq_gptq_quantize_layer(_p(X), ns, d, N, _p(W2), _p(scale), int(qmax), _p(codes), _p(Hinv))
+    if r:
+        raise ValueError("Hessian is singular")
+    return W2, codes, Hinv
+
+
+def smooth_search(X_bits: np.ndarray, W_bits: np.ndarray, G: int):
+    """QQQ adaptive smoothing threshold search (readings in qlin_oracle.c):
+    returns (loss fp64 [G], index of the least loss)."""
+    X_bits = _c(X_bits, np.uint16)
+    W_bits = _c(W_bits, np.uint16)
+    M, K = X_bits.shape
+    N = W_bits.shape[1]
+    loss = np.zeros(G, np.float64)
+    best = lib().oq_smooth_search(_p(X_bits), M, K, _p(W_bits), N, int(G), _p(loss))
+    return loss, int(best)
 
 
 # --- whole layer, composed from the steps above ------------------------------

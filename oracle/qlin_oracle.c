@@ -575,6 +575,120 @@ OQ_EXPORT int oq_gptq_quantize(const double* X, int ns, int d, double* w, double
   return 0;
 }
 
+/* The same compensation for a whole layer: W is [d][N] (input channel i is
+ * row i, output channel n is column n) and every output channel is the
+ * weight vector w of oq_gptq_quantize with its own grid step scale[n].  H,
+ * its inverse and the downdate sequence do not depend on w, so they are
+ * computed once and shared; each column goes through exactly the steps of
+ * oq_gptq_quantize (quantize column i, delta from column i of the current
+ * inverse, update the not-yet-quantized entries, keep the grid value).
+ * codes[i][n] receives the integer grid index clamp(rne(w_i / scale_n)).
+ * Returns nonzero if H is singular. */
+OQ_EXPORT int oq_gptq_quantize_layer(const double* X, int ns, int d, int N, double* W, const double* scale,
+                                     int qmax, int8_t* codes, double* Hinv_out) {
+  double* H = (double*)malloc(sizeof(double) * d * d);
+  double* Hinv = (double*)malloc(sizeof(double) * d * d);
+  double* w = (double*)malloc(sizeof(double) * d);
+  double* delta = (double*)malloc(sizeof(double) * d);
+  oq_gptq_hessian(X, ns, d, H);
+  if (invert_sym(H, d, Hinv)) {
+    free(H); free(Hinv); free(w); free(delta);
+    return 1;
+  }
+  if (Hinv_out) memcpy(Hinv_out, Hinv, sizeof(double) * d * d);
+  for (int i = 0; i < d; ++i) {
+    for (int n = 0; n < N; ++n) {
+      for (int j = 0; j < d; ++j) w[j] = W[(size_t)j * N + n];
+      int32_t c = clampi(oq_rne(w[i] / scale[n]), -qmax, qmax);
+      double q = (double)c * scale[n];
+      oq_gptq_delta(w, Hinv, d, i, q, delta);
+      for (int j = i; j < d; ++j) W[(size_t)j * N + n] = w[j] + delta[j];
+      W[(size_t)i * N + n] = q;
+      codes[(size_t)i * N + n] = (int8_t)c;
+    }
+    oq_gptq_downdate(Hinv, d, i);
+  }
+  free(H); free(Hinv); free(w); free(delta);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* QQQ adaptive smoothing ([QQQ] 自适应平滑), the threshold search.          */
+/* Readings (the page's formulas are partly garbled):                       */
+/*  - the smoothed channels are T(sigma) = { t : max_m |X[m,t]| > sigma }    */
+/*    (only channels with significant outliers are smoothed);               */
+/*  - s_t = sqrt(max_m|X[m,t]| / max_n|W[t,n]|) on T, 1 elsewhere (the       */
+/*    migration strength 1/2; 1 when a maximum is 0);                        */
+/*  - the smoothed tensors are rounded to fp16 before quantization:          */
+/*    Xh[m,t] = fp16(X[m,t] / s_t), Wh[t,n] = fp16(W[t,n] * s_t) on T, and   */
+/*    0 off T, so Q(X_T / s) and Q(W_T * s) are the layer's own quantizers   */
+/*    (per-token INT8, per-channel INT4) applied to the T parts;            */
+/*  - loss(sigma) = sum_{m,n} ( a_m c'_n acc[m][n] - (X_T W_T)[m][n] )^2     */
+/*    in fp64, acc the integer product of the codes;                         */
+/*  - sigma_j = max|X| * j / G for j = 0 .. G-1 (the grid over               */
+/*    [0, max|X|]); the search returns the first j of least loss.            */
+/* X fp16 [M][K], W fp16 [K][N]; loss [G]; returns the best index.           */
+/* ------------------------------------------------------------------------ */
+OQ_EXPORT int oq_smooth_search(const uint16_t* X, int M, int K, const uint16_t* W, int N, int G, double* loss) {
+  float* cmax = (float*)calloc((size_t)K, sizeof(float));
+  float* wmax = (float*)calloc((size_t)K, sizeof(float));
+  float* sv = (float*)malloc(sizeof(float) * (size_t)K);
+  uint16_t* Xh = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)M * K);
+  uint16_t* Wh = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)K * N);
+  int8_t* xq = (int8_t*)malloc((size_t)M * K);
+  float* a = (float*)malloc(sizeof(float) * (size_t)M);
+  int8_t* wq = (int8_t*)malloc((size_t)K * N);
+  float* c = (float*)malloc(sizeof(float) * (size_t)N);
+  float xall = 0.0f;
+  for (int m = 0; m < M; ++m)
+    for (int t = 0; t < K; ++t) {
+      float v = fabsf(oq_half_to_float(X[(size_t)m * K + t]));
+      if (v > cmax[t]) cmax[t] = v;
+      if (v > xall) xall = v;
+    }
+  for (int t = 0; t < K; ++t)
+    for (int n = 0; n < N; ++n) {
+      float v = fabsf(oq_half_to_float(W[(size_t)t * N + n]));
+      if (v > wmax[t]) wmax[t] = v;
+    }
+  int best = 0;
+  for (int j = 0; j < G; ++j) {
+    float sigma = xall * (float)j / (float)G;
+    for (int t = 0; t < K; ++t) {
+      int in_t = cmax[t] > sigma;
+      float st = 1.0f;
+      if (in_t && cmax[t] > 0.0f && wmax[t] > 0.0f) st = sqrtf(cmax[t] / wmax[t]);
+      sv[t] = in_t ? st : 0.0f;  /* 0 marks a channel outside T */
+    }
+    for (int m = 0; m < M; ++m)
+      for (int t = 0; t < K; ++t)
+        Xh[(size_t)m * K + t] = sv[t] > 0.0f ? oq_float_to_half(oq_half_to_float(X[(size_t)m * K + t]) / sv[t]) : 0;
+    for (int t = 0; t < K; ++t)
+      for (int n = 0; n < N; ++n)
+        Wh[(size_t)t * N + n] = sv[t] > 0.0f ? oq_float_to_half(oq_half_to_float(W[(size_t)t * N + n]) * sv[t]) : 0;
+    oq_quant_act(Xh, M, K, NULL, 0, NULL, xq, a, NULL);
+    oq_quant_weight_per_channel(Wh, K, N, 7, wq, c);
+    double L = 0.0;
+    for (int m = 0; m < M; ++m)
+      for (int n = 0; n < N; ++n) {
+        int64_t acc = 0;
+        double ref = 0.0;
+        for (int t = 0; t < K; ++t) {
+          acc += (int64_t)xq[(size_t)m * K + t] * (int64_t)(16 * wq[(size_t)t * N + n]);
+          if (sv[t] > 0.0f)
+            ref += oq_half_to_double(X[(size_t)m * K + t]) * oq_half_to_double(W[(size_t)t * N + n]);
+        }
+        double y = (double)acc * (double)a[m] * ((double)c[n] / 16.0);
+        double d = y - ref;
+        L += d * d;
+      }
+    loss[j] = L;
+    if (L < loss[best]) best = j;
+  }
+  free(cmax); free(wmax); free(sv); free(Xh); free(Wh); free(xq); free(a); free(wq); free(c);
+  return best;
+}
+
 OQ_EXPORT int oq_invert(const double* A, int d, double* inv) {
   double* a = (double*)malloc(sizeof(double) * d * d);
   memcpy(a, A, sizeof(double) * d * d);

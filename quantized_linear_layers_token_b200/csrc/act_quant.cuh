@@ -130,38 +130,63 @@ __device__ __forceinline__ uint2 comp_split(int q, float s) {
   return make_uint2(__half_as_ushort(hi), __half_as_ushort(lo));
 }
 
-struct MomentumArgs {
-  const float* wmaxO;  // [nO]
+// One quantization problem (a layer's activations at M tokens).  A launch
+// quantizes one problem or a group of independent problems
+// (qlin_forward_grouped); CTA b works on row b - row0 of the problem whose
+// rows [row0, row0 + M) contain it.
+struct QuantProb {
+  const uint16_t* X;     // [M][K] fp16
+  const int32_t* O;      // [nO]
+  float* s;              // [nO] momentum state
+  int8_t* Xq;            // [M][K]
+  float* a;              // [M]
+  int8_t* XqO;           // [M][nO]
+  uint16_t* U;           // [2][M][nOp] compensation operand (hi rows, then lo rows), or null
+  const float* wmaxO;    // [nO]
+  unsigned* counter;     // completion counter of the fused update (zero on entry, left zero)
+  int K, nO, nOp, M, row0;
+};
+
+template <int MAXP>
+struct QuantGroup {
   float gamma;
-  unsigned* counter;   // completion counter (zero on entry, left zero)
-  int M;               // rows of X (all of them feed the column maxima)
+  int nprob;
+  QuantProb pr[MAXP];
 };
 
 // One CTA per token row.  VPT = 8-element vectors per thread
 // (K <= 8 * kQuantThreads * VPT).
 // FUSED: every CTA also computes the outlier column maxima over all M rows
-// and the momentum update itself (identical in every CTA, cheap for small
-// M); the last CTA to finish writes the new state back, after every CTA has
-// read the old one.
+// of its problem and the momentum update itself (identical in every CTA,
+// cheap for small M); the last CTA of the problem to finish writes the new
+// state back, after every CTA has read the old one.
 // The row is staged in shared memory; the outlier columns' raw values are
 // set aside and their slots zeroed, so the row maximum (fp16 |x| maxima,
 // exact) and the quantization pass run without per-element outlier checks;
 // the outlier codes x_hat = x / s are computed separately and written over
 // the zeros after a barrier.  O and max|W_O| do not depend on the previous
 // kernel and are read before the grid dependency.
-template <int VPT, bool FUSED>
+template <int VPT, bool FUSED, int MAXP>
 __global__ void __launch_bounds__(kQuantThreads)
-quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ O, int nO,
-             float* __restrict__ s, int8_t* __restrict__ Xq, float* __restrict__ a,
-             int8_t* __restrict__ XqO, uint16_t* __restrict__ U, int nOp, MomentumArgs mom) {
+quant_kernel(const __grid_constant__ QuantGroup<MAXP> qg) {
   extern __shared__ __align__(16) unsigned char quant_smem[];
+  __shared__ float red[kQuantThreads / 32];
+  __shared__ int is_last;
+  int pi = 0;
+  if (MAXP > 1)
+    while (pi + 1 < qg.nprob && static_cast<int>(blockIdx.x) >= qg.pr[pi + 1].row0) ++pi;
+  const QuantProb& qp = qg.pr[pi];
+  const uint16_t* __restrict__ X = qp.X;
+  const int K = qp.K, nO = qp.nO, nOp = qp.nOp, M = qp.M;
+  const int32_t* __restrict__ O = qp.O;
+  float* __restrict__ s = qp.s;
+  int8_t* __restrict__ XqO = qp.XqO;
+  uint16_t* __restrict__ U = qp.U;
   uint16_t* xs = reinterpret_cast<uint16_t*>(quant_smem);          // [K] this row (outliers zeroed)
   int* sO = reinterpret_cast<int*>(quant_smem + static_cast<size_t>(K) * 2);
   float* sS = reinterpret_cast<float*>(sO + nO);                    // [nO] momentum state
   float* xo = sS + nO;                                              // [nO] raw outlier values of this row
   unsigned* cmx = reinterpret_cast<unsigned*>(xo + nO);             // [nO] fused column maxima (fp32 bits)
-  __shared__ float red[kQuantThreads / 32];
-  __shared__ int is_last;
 
   griddep_launch_dependents();
   for (int i = threadIdx.x; i < nO; i += kQuantThreads) {
@@ -169,9 +194,9 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     if (FUSED) cmx[i] = 0u;
   }
   float wmx = 0.f;  // max|W_O| of outlier threadIdx.x (FUSED, nO <= kQuantThreads handled in the loop below)
-  if (FUSED && threadIdx.x < nO) wmx = mom.wmaxO[threadIdx.x];
+  if (FUSED && static_cast<int>(threadIdx.x) < nO) wmx = qp.wmaxO[threadIdx.x];
   griddep_wait();  // X (and s) may come from the previous kernel
-  const int m = blockIdx.x;
+  const int m = static_cast<int>(blockIdx.x) - qp.row0;
   const uint4* xv = reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K);
   const int nvec = K >> 3;
 #pragma unroll
@@ -192,7 +217,7 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     // spread over the whole CTA, eight independent loads per thread in
     // flight, merged with shared-memory atomicMax on the fp32 bit patterns
     // (non-negative, so ordered like unsigned integers)
-    const int pairs = mom.M * nO;
+    const int pairs = M * nO;
     for (int p0 = threadIdx.x; p0 < pairs; p0 += 8 * kQuantThreads) {
       uint16_t hv[8];
       int ii[8];
@@ -214,8 +239,8 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     }
     __syncthreads();
     for (int i = threadIdx.x; i < nO; i += kQuantThreads)
-      sS[i] = momentum_step(sS[i], mom.gamma, __uint_as_float(cmx[i]),
-                            i == static_cast<int>(threadIdx.x) ? wmx : mom.wmaxO[i]);
+      sS[i] = momentum_step(sS[i], qg.gamma, __uint_as_float(cmx[i]),
+                            i == static_cast<int>(threadIdx.x) ? wmx : qp.wmaxO[i]);
   }
   __syncthreads();
 
@@ -239,9 +264,9 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
   }
   const float amax = block_max(lmax, red);
   const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
-  if (threadIdx.x == 0) a[m] = __fdiv_rn(amax, 127.f);
+  if (threadIdx.x == 0) qp.a[m] = __fdiv_rn(amax, 127.f);
 
-  int8_t* qrow = Xq + static_cast<size_t>(m) * K;
+  int8_t* qrow = qp.Xq + static_cast<size_t>(m) * K;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
     const int vi = threadIdx.x + j * kQuantThreads;
@@ -259,7 +284,7 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
     }
   }
   __syncthreads();  // the zero codes at the outlier columns are written before the patch below
-  const size_t lo_off = static_cast<size_t>(gridDim.x) * nOp;  // U holds [2][M][nOp]: hi rows, then lo rows
+  const size_t lo_off = static_cast<size_t>(M) * nOp;  // U holds [2][M][nOp]: hi rows, then lo rows
   for (int i = threadIdx.x; i < nOp; i += kQuantThreads) {
     if (i < nO) {
       const float xh = __fdiv_rn(xo[i], sS[i]);
@@ -276,16 +301,16 @@ quant_kernel(const uint16_t* __restrict__ X, int K, const int32_t* __restrict__ 
       U[lo_off + static_cast<size_t>(m) * nOp + i] = 0;
     }
   }
-  if (FUSED) {
-    if (gridDim.x == 1) {  // the only reader of the old state
+  if (FUSED && nO > 0) {
+    if (M == 1) {  // the only reader of the old state
       for (int i = threadIdx.x; i < nO; i += kQuantThreads) s[i] = sS[i];
     } else {
       __syncthreads();
-      if (threadIdx.x == 0) is_last = (atomicAdd(mom.counter, 1u) == gridDim.x - 1);
+      if (threadIdx.x == 0) is_last = (atomicAdd(qp.counter, 1u) == static_cast<unsigned>(M - 1));
       __syncthreads();
       if (is_last) {
         for (int i = threadIdx.x; i < nO; i += kQuantThreads) s[i] = sS[i];
-        if (threadIdx.x == 0) *mom.counter = 0u;
+        if (threadIdx.x == 0) *qp.counter = 0u;
       }
     }
   }

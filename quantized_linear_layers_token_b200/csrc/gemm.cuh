@@ -58,7 +58,7 @@ constexpr int kMaxGrid = 256;  // persistent CTAs per GEMM (>= SMs per GPU)
 // Diagnostic builds (-DQLIN_TRACE) record per-CTA clock64 stamps at the
 // phase boundaries below into g_trace[cta][16]; normal builds compile the
 // stamps away.
-// QLIN_STEP(g, k) records per-step events of CTA 0 into g_steps[g][8].  The
+// QLIN_STEP(g, k) records per-step events of CTA 0 into g_steps[g][8] (g < 255).  The
 // buffer pointers are read once into registers (QLIN_TRACE_INIT) so a stamp
 // costs a clock read and a store, not a global load.
 #ifdef QLIN_TRACE
@@ -73,12 +73,12 @@ __device__ long long* g_steps = nullptr;
   } while (0)
 #define QLIN_STEP(g, k)                                                                       \
   do {                                                                                        \
-    if (qlin_st && (g) < 64) qlin_st[(g) * 8 + (k)] = static_cast<long long>(clock64());      \
+    if (qlin_st && (g) < 255) qlin_st[(g) * 8 + (k)] = static_cast<long long>(clock64());     \
   } while (0)
-// finisher phases of any CTA into g_steps[63][k] (last writer wins)
+// finisher phases of any CTA into g_steps[255][k] (last writer wins)
 #define QLIN_FIN(k)                                                                           \
   do {                                                                                        \
-    if (g_steps) g_steps[63 * 8 + (k)] = static_cast<long long>(clock64());                   \
+    if (g_steps) g_steps[255 * 8 + (k)] = static_cast<long long>(clock64());                  \
   } while (0)
 #else
 #define QLIN_FIN(k) do { } while (0)
@@ -87,39 +87,79 @@ __device__ long long* g_steps = nullptr;
 #define QLIN_STEP(g, k) do { } while (0)
 #endif
 
-struct GemmArgs {
+// One GEMM problem of a launch (a linear layer at M tokens).  A launch runs
+// one problem (qlin_gemm / qlin_forward) or a group of independent problems
+// with the same token tile (qlin_forward_grouped): their tiles' iterations
+// are concatenated into one space that the persistent CTAs split.
+struct GemmProb {
   const uint8_t* codes;     // tiled packed codes (INT4: 8 KiB blocks, INT8: 16 KiB swizzled blocks)
   const uint16_t* rfold;    // g128 ratios r [K/128][N] fp16
   const uint16_t* wot;      // tiled W_O^T (16 KiB swizzled blocks of 128 channels x 64 outliers)
-  const float* cscale;  // c_n [N]
-  float cmul;           // INT8 kernel: factor on c_n (1, or 1/16 for per-channel INT4 widened to 16 q)
-  const float* a;       // a_m [M]
-  uint16_t* Y;          // [M][N] fp16
-  int32_t* acc_debug;   // [M][N] or null
+  const float* cscale;      // c_n [N]
+  const float* a;           // a_m [M]
+  uint16_t* Y;              // [M][N] fp16
+  int32_t* acc_debug;       // [M][N] or null
+  float cmul;               // INT8 kernel: factor on c_n (1, or 1/16 for per-channel INT4 widened to 16 q)
+  int M, N, K, nO;
+  int tiles_n, tiles_m;
+  int kb;                   // 128-wide K-blocks per tile (ceil(K / 128))
+  int nk;                   // main K-steps per tile (ceil(kb / KS))
+  int nc;                   // compensation steps per tile
+  int ncs;                  // 64-wide outlier slices
+  int T;                    // iterations per tile = nk + nc
+  int gm;                   // token tiles per raster group (see tile_coords)
+  unsigned it0;             // first iteration of this problem in the launch's iteration space
+};
+
+// Tile t of a problem -> (channel tile tn, token tile tm).  Token tiles are
+// visited in groups of gm, the token tile varying fastest within a group, so
+// the CTAs that run at the same time share weight tiles (one HBM read, the
+// rest L2 hits) and the group's activations stay in L2.  gm = 1 is the
+// channel-tile-fastest order.
+__host__ __device__ __forceinline__ void tile_coords(const GemmProb& pr, unsigned t, int& tn, int& tm) {
+  const unsigned per = static_cast<unsigned>(pr.gm) * static_cast<unsigned>(pr.tiles_n);
+  const unsigned grp = t / per;
+  const unsigned w = t - grp * per;
+  const int g0 = static_cast<int>(grp) * pr.gm;
+  const int gs = pr.tiles_m - g0 < pr.gm ? pr.tiles_m - g0 : pr.gm;
+  tm = g0 + static_cast<int>(w % static_cast<unsigned>(gs));
+  tn = static_cast<int>(w / static_cast<unsigned>(gs));
+}
+
+// Launch-wide arguments.
+struct GemmArgs {
   int32_t* ws_acc;      // [2*grid][BT][128] INT32 partial sums of split tiles
   float* ws_comp;       // [2*grid][BT][128] fp32 compensation of split tiles
   unsigned* ws_cnt;     // [grid] iteration counters (zero on entry, left zero)
-  int M, N, K, nO;
-  int tiles_n, tiles_m;
-  int kb;               // 128-wide K-blocks per tile (ceil(K / 128))
-  int nk;               // main K-steps per tile (ceil(kb / KS))
-  int nc;               // compensation steps per tile
-  int ncs;              // 64-wide outlier slices
-  int T;                // iterations per tile = nk + nc
+  int nprob;            // problems in the launch
   int grid;             // persistent CTAs (<= kMaxGrid)
   int split;            // 1: stream-K split points; 0: whole tiles per CTA
-  // Cluster split-K (cs > 1): the grid is ncl clusters of cs CTAs; cluster c
-  // takes tiles c, c + ncl, ...; cluster rank r computes iterations
-  // [cb[r], cb[r+1]) of each (cb[cs] = T, the compensation run never cut),
-  // and the partials are reduced through distributed shared memory: rank q
-  // owns channels [q * 128/cs, (q+1) * 128/cs) of the tile.
+  unsigned total;       // iterations of every problem's tiles
+  // Cluster split-K (cs > 1, single-problem launches only): the grid is ncl
+  // clusters of cs CTAs; cluster c takes tiles c, c + ncl, ...; cluster rank
+  // r computes iterations [cb[r], cb[r+1]) of each (cb[cs] = T, the
+  // compensation run never cut), and the partials are reduced through
+  // distributed shared memory: rank q owns channels [q * 128/cs, (q+1) *
+  // 128/cs) of the tile.
   int cs;
   int ncl;
   int cb[9];
-  // bnd[c] = first iteration of CTA c, bnd[grid] = tiles * T (computed on
-  // the host by gemm_boundary(); kernel parameters, read from the constant
+  // bnd[c] = first iteration of CTA c, bnd[grid] = total (computed on the
+  // host by gemm_boundaries(); kernel parameters, read from the constant
   // cache).
   unsigned bnd[kMaxGrid + 1];
+};
+
+constexpr int kMaxProbs = 32;  // problems per grouped launch
+
+// Kernel parameters: the TMA maps of every problem's activation (Xq) and
+// compensation (U) operands, the launch-wide arguments and the problems.
+template <int MAXP>
+struct alignas(64) GemmParams {
+  CUtensorMap tmX[MAXP];
+  CUtensorMap tmU[MAXP];
+  GemmArgs g;
+  GemmProb pr[MAXP];
 };
 
 // K-blocks of 128 INT8 codes per pipeline step for a token tile of BT.
@@ -220,17 +260,32 @@ __host__ __device__ inline uint32_t tmem_alloc_cols(int BT, bool comp, int extra
   return c;
 }
 
-// First iteration owned by CTA c (host side; c == grid gives the total).
-// Split points never fall strictly inside a tile's compensation run.
-inline unsigned gemm_boundary(int c, long long tiles, int T, int nk, int grid, int split) {
-  const long long I = tiles * T;
-  if (c <= 0) return 0;
-  if (c >= grid) return static_cast<unsigned>(I);
-  if (!split) return static_cast<unsigned>(((tiles * c) / grid) * T);
-  long long b = (I * c) / grid;
-  const long long r = b % T;
-  if (r > nk) b += T - r;
-  return static_cast<unsigned>(b);
+// First iteration of every CTA (host side; bnd[grid] = total).  Split
+// points never fall strictly inside a tile's compensation run; without
+// splitting they snap to the nearest tile start.
+inline void gemm_boundaries(const GemmProb* pr, int nprob, int grid, int split, unsigned* bnd) {
+  long long total = 0;
+  for (int p = 0; p < nprob; ++p) total += static_cast<long long>(pr[p].tiles_n) * pr[p].tiles_m * pr[p].T;
+  int p = 0;
+  for (int c = 0; c <= grid; ++c) {
+    if (c == 0 || c == grid) {
+      bnd[c] = c == 0 ? 0u : static_cast<unsigned>(total);
+      continue;
+    }
+    long long b = (total * c) / grid;
+    while (p + 1 < nprob && b >= static_cast<long long>(pr[p + 1].it0)) ++p;
+    const long long T = pr[p].T;
+    const long long r = (b - pr[p].it0) % T;
+    if (!split) {
+      if (r) b += 2 * r >= T ? T - r : -r;  // the nearest tile start
+    } else if (r > pr[p].nk) {
+      b += T - r;
+    }
+    if (b > total) b = total;
+    bnd[c] = static_cast<unsigned>(b);
+  }
+  for (int c = 1; c <= grid; ++c)  // monotone after snapping
+    if (bnd[c] < bnd[c - 1]) bnd[c] = bnd[c - 1];
 }
 
 // Cluster split-K rank ranges of one tile's T iterations (nk K-steps, then
@@ -270,7 +325,7 @@ inline double cluster_bounds(int T, int nk, int cs, double ccost, int* cb) {
 // The boundary table is copied into shared memory at kernel start (entries
 // 0 .. grid-1; entry grid is the total iteration count).
 __device__ __forceinline__ unsigned bnd_s(int c, const unsigned* sbnd, const GemmArgs& g) {
-  return c < g.grid ? sbnd[c] : static_cast<unsigned>(g.tiles_n * g.tiles_m * g.T);
+  return c < g.grid ? sbnd[c] : g.total;
 }
 
 // The CTA whose range contains iteration `it` (binary search of the table).
@@ -283,45 +338,49 @@ __device__ __forceinline__ int owner_cta_s(unsigned it, const unsigned* sbnd, co
   return lo;
 }
 
-// Scratch slot holding CTA c's partial of split tile `tile`: its first
-// segment if its range starts inside the tile, else its last segment.
-__device__ __forceinline__ int partial_slot_s(int c, unsigned tile, const unsigned* sbnd, const GemmArgs& g) {
-  return 2 * c + (sbnd[c] < tile * static_cast<unsigned>(g.T) ? 1 : 0);
+// Scratch slot holding CTA c's partial of the split tile whose first
+// iteration is `tfirst`: its first segment if its range starts inside the
+// tile, else its last segment.
+__device__ __forceinline__ int partial_slot_s(int c, unsigned tfirst, const unsigned* sbnd) {
+  return 2 * c + (sbnd[c] < tfirst ? 1 : 0);
 }
 
 struct Segment {
-  unsigned tile;
-  int r0, r1;  // iterations [r0, r1) of the tile
+  int p;            // problem
+  unsigned tile;    // tile within the problem (tn + tiles_n * tm)
+  unsigned tfirst;  // first iteration of the tile in the launch's iteration space
+  int r0, r1;       // iterations [r0, r1) of the tile
 };
 
 // Dequantisation factor c'_n of output channel n: c_n / 16 for per-channel
 // INT4 (the operand holds 16 q), c_n for the other formats, times the INT8
 // kernel's factor (exact: 1 or 1/16) when it runs on widened INT4 weights.
 template <int FMT>
-__device__ __forceinline__ float chan_scale(const GemmArgs& g, int n) {
+__device__ __forceinline__ float chan_scale(const GemmProb& g, int n) {
   if (n >= g.N) return 0.f;
   const float c = g.cscale[n];
   return FMT == kFmtW4PC ? __fmul_rn(c, 0.0625f) : (FMT == kFmtW8 ? __fmul_rn(c, g.cmul) : c);
 }
 
-// Segments of one CTA, in order: a stream-K range of the flat iteration
-// space, or (cluster split-K) the same rank range of every cluster tile.
-// The fields come from the CTA plan staged in shared memory at start-up, so
-// no role waits on kernel-parameter loads for its first segment.
+// Segments of one CTA, in order: a stream-K range of the launch's iteration
+// space (crossing problems), or (cluster split-K) the same rank range of
+// every cluster tile of the single problem.  The range comes from the CTA
+// plan staged in shared memory at start-up, so no role waits on
+// kernel-parameter loads for its first segment.
 struct SegGen {
-  unsigned it, it1, T;
-  int u, cid, ncl, ntiles, r0, r1;
+  unsigned it, it1;
+  int p, u, cid, ncl, ntiles, r0, r1;
   bool cl;
 };
 
 // CTA plan (shared memory, written once during setup).
-enum : int { kPlanIt0 = 0, kPlanIt1, kPlanT, kPlanR0, kPlanR1, kPlanNcl, kPlanTiles, kPlanWords };
+enum : int { kPlanIt0 = 0, kPlanIt1, kPlanR0, kPlanR1, kPlanNcl, kPlanTiles, kPlanWords };
 
 __device__ __forceinline__ SegGen seg_begin(const int* plan, int cid, bool cl) {
   SegGen s;
   s.it = static_cast<unsigned>(plan[kPlanIt0]);
   s.it1 = static_cast<unsigned>(plan[kPlanIt1]);
-  s.T = static_cast<unsigned>(plan[kPlanT]);
+  s.p = 0;
   s.u = 0;
   s.cid = cid;
   s.ncl = plan[kPlanNcl];
@@ -332,21 +391,28 @@ __device__ __forceinline__ SegGen seg_begin(const int* plan, int cid, bool cl) {
   return s;
 }
 
-__device__ __forceinline__ bool seg_next(SegGen& s, Segment& sg) {
+__device__ __forceinline__ bool seg_next(SegGen& s, Segment& sg, const GemmProb* pr, int nprob) {
   if (s.cl) {
     const int t = s.cid + s.u * s.ncl;
     if (t >= s.ntiles) return false;
+    sg.p = 0;
     sg.tile = static_cast<unsigned>(t);
+    sg.tfirst = static_cast<unsigned>(t) * static_cast<unsigned>(pr[0].T);
     sg.r0 = s.r0;
     sg.r1 = s.r1;
     ++s.u;
     return true;
   }
   if (s.it >= s.it1) return false;
-  sg.tile = s.it / s.T;
-  sg.r0 = static_cast<int>(s.it - sg.tile * s.T);
+  while (s.p + 1 < nprob && s.it >= pr[s.p + 1].it0) ++s.p;
+  const unsigned T = static_cast<unsigned>(pr[s.p].T);
+  const unsigned local = s.it - pr[s.p].it0;
+  sg.p = s.p;
+  sg.tile = local / T;
+  sg.r0 = static_cast<int>(local - sg.tile * T);
+  sg.tfirst = pr[s.p].it0 + sg.tile * T;
   const unsigned left = s.it1 - s.it;
-  sg.r1 = static_cast<int>(left < s.T - sg.r0 ? sg.r0 + left : s.T);
+  sg.r1 = static_cast<int>(left < T - sg.r0 ? sg.r0 + left : T);
   s.it += sg.r1 - sg.r0;
   return true;
 }
@@ -454,11 +520,13 @@ widen_w4_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ 
   }
 }
 
-template <int FMT, int BT>
+template <int FMT, int BT, int MAXP>
 __global__ void __launch_bounds__(GemmCfg<FMT, BT>::kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmU,
-            const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmArgs args) {
+gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
   using C = GemmCfg<FMT, BT>;
+  const GemmArgs& args = prm.g;
+  const GemmProb* const probs = prm.pr;
+  const int nprob = MAXP == 1 ? 1 : args.nprob;
   constexpr int P = C::kASlots;
   constexpr int XS = C::kXSlots;
   constexpr int LS = C::kStgSlots > 0 ? C::kStgSlots : 1;
@@ -478,7 +546,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   uint64_t* cempty = cfull + 2;       // [2]
   uint64_t* recv_full = cempty + 2;   // cluster split-K: this CTA's receive buffer is complete
   uint64_t* recv_free = recv_full + 1; // every owner has read this CTA's previous partials
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_free + 1);
+  uint64_t* mma_done = recv_free + 1;   // every tensor-core op the issuer started has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;  // [2]
   int* plan = const_cast<int*>(last_flag + 2);  // [kPlanWords]
@@ -486,7 +555,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const bool comp = args.nO > 0;
+  // Compensation accumulators are allocated when any problem has outliers.
+  bool comp = false;
+  for (int q = 0; q < nprob; ++q) comp = comp || probs[q].nO > 0;
   const int bcols = tmem_buf_cols(BT, comp);
   const int nbuf = tmem_nbuf(BT, comp);
   const uint32_t tcols = tmem_alloc_cols(BT, comp, C::kTA ? P * C::kACols : 0);
@@ -500,7 +571,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   // bytes arriving in a receive buffer per round: every rank's INT32 slice,
   // plus the compensation slice when the layer has outliers
   const uint32_t recv_bytes =
-      static_cast<uint32_t>(128 * BT * 4 + (args.nO > 0 ? slice * BT * 4 : 0));
+      static_cast<uint32_t>(128 * BT * 4 + (probs[0].nO > 0 ? slice * BT * 4 : 0));
   QLIN_TRACE_INIT
 #ifdef QLIN_TRACE
   if (threadIdx.x == 0 && qlin_tr) qlin_tr[blockIdx.x * 32 + 31] = static_cast<long long>(globaltimer_ns());
@@ -528,24 +599,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     } else if (lane == 26) {
       mbar_init(recv_full, 1);
       mbar_init(recv_free, static_cast<uint32_t>(args.cs));
+      mbar_init(mma_done, 1);
       *abort_flag = 0;
     }
     fence_barrier_init();
     __syncwarp();
     if (lane == 26 && cl) mbar_arrive_expect_tx(recv_full, recv_bytes);  // round 0
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmX);
-    if (comp) tma_prefetch_desc(&tmU);
+  if (warp == 0 && lane < nprob) {
+    tma_prefetch_desc(&prm.tmX[lane]);
+    if (probs[lane].nO > 0) tma_prefetch_desc(&prm.tmU[lane]);
   }
   if (warp == 3 && lane == 0) {
     plan[kPlanIt0] = cl ? 0 : static_cast<int>(it0);
     plan[kPlanIt1] = cl ? 0 : static_cast<int>(args.bnd[blockIdx.x + 1]);
-    plan[kPlanT] = args.T;
     plan[kPlanR0] = cl ? args.cb[crk] : 0;
     plan[kPlanR1] = cl ? args.cb[crk + 1] : 0;
     plan[kPlanNcl] = args.ncl;
-    plan[kPlanTiles] = args.tiles_n * args.tiles_m;
+    plan[kPlanTiles] = probs[0].tiles_n * probs[0].tiles_m;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, tcols);
@@ -574,8 +645,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       Segment sg;
       int g = 0;
       bool ok = true;
-      while (ok && seg_next(gen, sg)) {
-        const int m0 = static_cast<int>(sg.tile / args.tiles_n) * BT;
+      while (ok && seg_next(gen, sg, probs, nprob)) {
+        const GemmProb& pr = probs[sg.p];
+        const CUtensorMap* tmX = &prm.tmX[sg.p];
+        const CUtensorMap* tmU = &prm.tmU[sg.p];
+        int tn_, tm_;
+        tile_coords(pr, sg.tile, tn_, tm_);
+        const int m0 = tm_ * BT;
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
           const int x = g % XS;
           if (g >= XS && !mbar_wait(&xempty[x], static_cast<uint32_t>(g / XS - 1) & 1u, abort_flag)) {
@@ -585,26 +661,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           unsigned char* xb = smem + C::kOffX + x * C::kXBytes;
           QLIN_STEP(g, 0);
           if (first_x) QLIN_STAMP(28);
-          if (r < args.nk) {
+          if (r < pr.nk) {
             const int kb0 = r * C::KS;
-            const int nkb = min(C::KS, args.kb - kb0);
+            const int nkb = min(C::KS, pr.kb - kb0);
             mbar_arrive_expect_tx(&xfull[x], static_cast<uint32_t>(nkb) * C::kTxX);
             if (first_x) QLIN_STAMP(29);
             for (int i = 0; i < nkb; ++i) {
-              tma_load_2d(xb + i * C::kXTile, &tmX, &xfull[x], (kb0 + i) * 128, m0);
+              tma_load_2d(xb + i * C::kXTile, tmX, &xfull[x], (kb0 + i) * 128, m0);
               if (first_x && i == 0) QLIN_STAMP(30);
             }
             first_x = false;
             if (g == 0) QLIN_STAMP(19);
           } else {
-            const int j = r - args.nk;
+            const int j = r - pr.nk;
             mbar_arrive_expect_tx(&xfull[x], C::kTxU);
             if (C::kCompFused) {
-              tma_load_2d(xb, &tmU, &xfull[x], j * 64, m0);                          // hi rows
-              tma_load_2d(xb + C::kXTile, &tmU, &xfull[x], j * 64, args.M + m0);     // lo rows
+              tma_load_2d(xb, tmU, &xfull[x], j * 64, m0);                          // hi rows
+              tma_load_2d(xb + C::kXTile, tmU, &xfull[x], j * 64, pr.M + m0);     // lo rows
             } else {
-              const int lo = j >= args.ncs ? 1 : 0;  // U rows [0, M) hold hi, [M, 2M) hold lo
-              tma_load_2d(xb, &tmU, &xfull[x], (j - lo * args.ncs) * 64, lo * args.M + m0);
+              const int lo = j >= pr.ncs ? 1 : 0;  // U rows [0, M) hold hi, [M, 2M) hold lo
+              tma_load_2d(xb, tmU, &xfull[x], (j - lo * pr.ncs) * 64, lo * pr.M + m0);
             }
           }
         }
@@ -623,13 +699,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       Segment sg;
       int g = 0, gs = 0, gc = 0;
       bool ok = true;
-      while (ok && seg_next(gen, sg)) {
+      while (ok && seg_next(gen, sg, probs, nprob)) {
         if (g == 0) QLIN_STAMP(26);
-        const int tn = static_cast<int>(sg.tile % args.tiles_n);
+        const GemmProb& pr = probs[sg.p];
+        int tn, tm_;
+        tile_coords(pr, sg.tile, tn, tm_);
         const int n0 = tn * C::kBN;
-        const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(min(C::kBN, args.N - n0)) * 2u : 0u;
+        const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(min(C::kBN, pr.N - n0)) * 2u : 0u;
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
-          if (r < args.nk && C::kW4) {
+          if (r < pr.nk && C::kW4) {
             const int ls = gs % LS;
             if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
               ok = false;
@@ -638,14 +716,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
             QLIN_STEP(g, 1);
             const int kb0 = r * C::KS;
-            const int nkb = min(C::KS, args.kb - kb0);
+            const int nkb = min(C::KS, pr.kb - kb0);
             if (gs == 0) QLIN_STAMP(15);
             mbar_arrive_expect_tx(&sfull[ls], static_cast<uint32_t>(nkb) * (8192u + rb));
-            bulk_load_hint(st, args.codes + (static_cast<size_t>(tn) * args.kb + kb0) * 8192,
+            bulk_load_hint(st, pr.codes + (static_cast<size_t>(tn) * pr.kb + kb0) * 8192,
                            static_cast<uint32_t>(nkb) * 8192u, &sfull[ls], pol_stream);
             if (FMT == kFmtW4G128)
               for (int i = 0; i < nkb; ++i)
-                bulk_load(st + C::kStgRatio + i * 256, args.rfold + static_cast<size_t>(kb0 + i) * args.N + n0, rb,
+                bulk_load(st + C::kStgRatio + i * 256, pr.rfold + static_cast<size_t>(kb0 + i) * pr.N + n0, rb,
                           &sfull[ls]);
             if (gs == 0) QLIN_STAMP(2);
             ++gs;
@@ -657,10 +735,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               ok = false;
               break;
             }
-            const int j = r - args.nk;
-            const int ib = C::kCompFused ? j : (j >= args.ncs ? j - args.ncs : j);
+            const int j = r - pr.nk;
+            const int ib = C::kCompFused ? j : (j >= pr.ncs ? j - pr.ncs : j);
             mbar_arrive_expect_tx(&cfull[cs], 16384u);
-            bulk_load(smem + C::kOffComp + cs * 16384, args.wot + (static_cast<size_t>(tn) * args.ncs + ib) * 8192,
+            bulk_load(smem + C::kOffComp + cs * 16384, pr.wot + (static_cast<size_t>(tn) * pr.ncs + ib) * 8192,
                       16384, &cfull[cs]);
             ++gc;
           } else if (!C::kW4) {
@@ -675,17 +753,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               break;
             }
             unsigned char* ab = smem + C::kOffA + p * C::kABytes;
-            if (r < args.nk) {
+            QLIN_STEP(g, 1);
+            if (r < pr.nk) {
               const int kb0 = r * C::KS;
-              const int nkb = min(C::KS, args.kb - kb0);
+              const int nkb = min(C::KS, pr.kb - kb0);
               mbar_arrive_expect_tx(&afull[p], static_cast<uint32_t>(nkb) * 16384u);
-              bulk_load_hint(ab, args.codes + (static_cast<size_t>(tn) * args.kb + kb0) * 16384,
+              bulk_load_hint(ab, pr.codes + (static_cast<size_t>(tn) * pr.kb + kb0) * 16384,
                              static_cast<uint32_t>(nkb) * 16384u, &afull[p], pol_stream);
             } else {
-              const int j = r - args.nk;
-              const int ib = C::kCompFused ? j : (j >= args.ncs ? j - args.ncs : j);
+              const int j = r - pr.nk;
+              const int ib = C::kCompFused ? j : (j >= pr.ncs ? j - pr.ncs : j);
               mbar_arrive_expect_tx(&afull[p], 16384u);
-              bulk_load(ab, args.wot + (static_cast<size_t>(tn) * args.ncs + ib) * 8192, 16384, &afull[p]);
+              bulk_load(ab, pr.wot + (static_cast<size_t>(tn) * pr.ncs + ib) * 8192, 16384, &afull[p]);
             }
             ++a_issues[p];
           }
@@ -721,17 +800,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       Segment sg;
       int g = 0, seg = 0;
       bool ok = true;
-      while (ok && seg_next(gen, sg)) {
+      bool issued = false;  // any tcgen05.mma started (drained before TMEM is freed)
+      while (ok && seg_next(gen, sg, probs, nprob)) {
+        const GemmProb& pr = probs[sg.p];
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
-        if (use > 0 && !mbar_wait(&acc_empty[buf], static_cast<uint32_t>(use - 1) & 1u, abort_flag)) break;
+        if (use > 0 && !mbar_wait(&acc_empty[buf], static_cast<uint32_t>(use - 1) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t dmain = tmem + static_cast<uint32_t>(buf * bcols);
         const uint32_t dcomp = dmain + BT;
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
           const int p = g % P;
           const int x = g % XS;
-          const bool main_step = r < args.nk;
+          const bool main_step = r < pr.nk;
           if (!mbar_wait(&xfull[x], static_cast<uint32_t>(g / XS) & 1u, abort_flag)) { ok = false; break; }
           QLIN_STEP(g, 5);
           if (C::kTA) {
@@ -742,8 +826,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               if (g == 0) QLIN_STAMP(8);
               QLIN_STEP(g, 6);
               tc_fence_after();
+              issued = true;
               const uint32_t at = tmem + a_col0 + static_cast<uint32_t>(pa * C::kACols);
-              const int nkb = min(C::KS, args.kb - r * C::KS);
+              const int nkb = min(C::KS, pr.kb - r * C::KS);
               mma_i8_ta(dmain, at, bd, idesc_main, r > sg.r0 ? 1u : 0u);
               mma_i8_ta(dmain, at + 8, bd + 2, idesc_main, 1u);
               mma_i8_ta(dmain, at + 16, bd + 4, idesc_main, 1u);
@@ -767,8 +852,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               if (g == 0) QLIN_STAMP(8);
               QLIN_STEP(g, 6);
               tc_fence_after();
+              issued = true;
               const uint64_t ad = cdesc0 + static_cast<uint64_t>(cs * (16384 >> 4));
-              const uint32_t acc0 = ((r == args.nk) || (r == sg.r0)) ? 0u : 1u;
+              const uint32_t acc0 = ((r == pr.nk) || (r == sg.r0)) ? 0u : 1u;
               mma_f16(dcomp, ad, bd, idesc_comp, acc0);
               mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
               mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
@@ -793,10 +879,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           if (g == 0) QLIN_STAMP(8);
           QLIN_STEP(g, 6);
           tc_fence_after();
+          issued = true;
           const uint64_t ad = adesc0 + static_cast<uint64_t>(p * (C::kABytes >> 4));
           const uint64_t bd = xdesc0 + static_cast<uint64_t>(x * (C::kXBytes >> 4));
           if (main_step) {
-            const int nkb = min(C::KS, args.kb - r * C::KS);
+            const int nkb = min(C::KS, pr.kb - r * C::KS);
             mma_i8(dmain, ad, bd, idesc_main, r > sg.r0 ? 1u : 0u);
             mma_i8(dmain, ad + 2, bd + 2, idesc_main, 1u);
             mma_i8(dmain, ad + 4, bd + 4, idesc_main, 1u);
@@ -813,7 +900,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               }
             }
           } else {
-            const uint32_t acc0 = ((r == args.nk) || (r == sg.r0)) ? 0u : 1u;
+            const uint32_t acc0 = ((r == pr.nk) || (r == sg.r0)) ? 0u : 1u;
             mma_f16(dcomp, ad, bd, idesc_comp, acc0);
             mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
             mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
@@ -833,6 +920,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         ++seg;
       }
       QLIN_STAMP(9);
+      // Every MMA issued has completed before TMEM is freed: normally the
+      // epilogue's accumulator waits already saw that, but after a wait gave
+      // up nothing else does, so wait here (fixed limit) either way.
+      if (issued) {
+        mma_commit(mma_done);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(mma_done, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
+        }
+      }
     }
     __syncwarp();
   } else {
@@ -858,8 +954,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       Segment sg;
       int gm = 0, gs = 0;
       bool ok = true;
-      while (ok && seg_next(gen, sg)) {
-        for (int r = sg.r0; r < sg.r1 && r < args.nk; ++r) {
+      while (ok && seg_next(gen, sg, probs, nprob)) {
+        const GemmProb& pr = probs[sg.p];
+        for (int r = sg.r0; r < sg.r1 && r < pr.nk; ++r) {
           const int ls = gs % LS;
           if (!mbar_wait(&sfull[ls], static_cast<uint32_t>(gs / LS) & 1u, abort_flag)) { ok = false; break; }
           if (gs == 0 && ctid == 0) QLIN_STAMP(6);
@@ -870,7 +967,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           }
           tc_fence_after();
           const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
-          const int nkb = min(C::KS, args.kb - r * C::KS);
+          const int nkb = min(C::KS, pr.kb - r * C::KS);
           for (int blk = half; blk < nkb; blk += 2) {
             const unsigned char* src = stg + blk * 8192 + row * 64;
             uint32_t o[32];
@@ -919,11 +1016,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       Segment sg;
       int g = 0, gs = 0;
       bool ok = true;
-      while (ok && seg_next(gen, sg)) {
-        const int tn = static_cast<int>(sg.tile % args.tiles_n);
+      while (ok && seg_next(gen, sg, probs, nprob)) {
+        const GemmProb& pr = probs[sg.p];
+        int tn, tm_;
+        tile_coords(pr, sg.tile, tn, tm_);
         for (int r = sg.r0; r < sg.r1; ++r, ++g) {
           const int p = g % P;
-          if (r >= args.nk) {
+          if (r >= pr.nk) {
             // compensation step: the W_O^T block goes into the A slot once
             // the tensor core has released it
             if (g >= P && !mbar_wait(&aempty[p], static_cast<uint32_t>(g / P - 1) & 1u, abort_flag)) {
@@ -931,10 +1030,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               break;
             }
             if (ctid == 0) {
-              const int j = r - args.nk;
-              const int ib = C::kCompFused ? j : (j >= args.ncs ? j - args.ncs : j);
+              const int j = r - pr.nk;
+              const int ib = C::kCompFused ? j : (j >= pr.ncs ? j - pr.ncs : j);
               mbar_arrive_expect_tx(&afull[p], 16384u);
-              bulk_load(smem + C::kOffA + p * C::kABytes, args.wot + (static_cast<size_t>(tn) * args.ncs + ib) * 8192,
+              bulk_load(smem + C::kOffA + p * C::kABytes, pr.wot + (static_cast<size_t>(tn) * pr.ncs + ib) * 8192,
                         16384, &afull[p]);
               ++a_issues[p];
             }
@@ -948,7 +1047,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           if (ctid == 0) QLIN_STEP(g, 3);
           const unsigned char* stg = smem + C::kOffStg + ls * C::kStgBytes;
           unsigned char* A0 = smem + C::kOffA + p * C::kABytes;
-          const int nchunk = min(C::KS, args.kb - r * C::KS) * 512;  // 16-byte packed chunks this step
+          const int nchunk = min(C::KS, pr.kb - r * C::KS) * 512;  // 16-byte packed chunks this step
           // Token tiles >= 128 move one K-block per step: 512 chunks, at
           // most two per thread.  Both chunks (and their ratios) are loaded
           // before any operand store: the compiler cannot prove the staging
@@ -1021,7 +1120,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       // Partially covered tiles (at most the first and the last segment):
       // their counters and the finishing work run after every segment's
       // TMEM has been drained, so the mainloop never waits on them.
-      unsigned pend_tile[2] = {0u, 0u};
+      unsigned pend_tile[2] = {0u, 0u};  // first iteration of each pending tile
+      int pend_prob[2] = {0, 0};
+      unsigned pend_loc[2] = {0u, 0u};   // its index within its problem
       int pend_add[2] = {0, 0};
       int npend = 0;
       SegGen gen = seg_begin(plan, cid, cl);
@@ -1029,24 +1130,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       int seg = 0;
       int ycnt = 0;  // Y chunks handed to TMA stores (two staging buffers alternate)
       float* sa_t = reinterpret_cast<float*>(smem + C::kOffSa + grp * 1024);
-      while (seg_next(gen, sg)) {
+      while (seg_next(gen, sg, probs, nprob)) {
+        const GemmProb& pr = probs[sg.p];
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
         // everything that depends only on the tile is read before waiting for
         // its accumulator (the loads complete behind the mainloop)
-        const int tn = static_cast<int>(sg.tile % args.tiles_n);
-        const int tm = static_cast<int>(sg.tile / args.tiles_n);
+        int tn, tm;
+        tile_coords(pr, sg.tile, tn, tm);
         const int n = tn * C::kBN + nl;
         const int m0 = tm * BT;
-        const int mvalid = min(BT, args.M - m0);
-        const bool has_main = sg.r0 < args.nk;
-        const bool has_comp = comp && sg.r1 == args.T && sg.r0 <= args.nk;
-        const bool whole = sg.r0 == 0 && sg.r1 == args.T;
-        const float cn = chan_scale<FMT>(args, n);
+        const int mvalid = min(BT, pr.M - m0);
+        const bool pcomp = pr.nO > 0;  // this problem has outliers
+        const bool has_main = sg.r0 < pr.nk;
+        const bool has_comp = pcomp && sg.r1 == pr.T && sg.r0 <= pr.nk;
+        const bool whole = sg.r0 == 0 && sg.r1 == pr.T;
+        const float cn = chan_scale<FMT>(pr, n);
         float a_own = 0.f, cn_own = 0.f;  // cluster split-K: the owned slice's scales
         if (cl) {
-          cn_own = chan_scale<FMT>(args, tn * C::kBN + crk * slice + (nl % slice));
-          if (nl < mvalid) a_own = args.a[m0 + nl];
+          cn_own = chan_scale<FMT>(pr, tn * C::kBN + crk * slice + (nl % slice));
+          if (nl < mvalid) a_own = pr.a[m0 + nl];
         }
         bool ok = mbar_wait(&acc_full[buf], static_cast<uint32_t>(use) & 1u, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
@@ -1060,7 +1163,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           continue;
         }
         const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * bcols);
-        const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tile * static_cast<unsigned>(args.T) ? 1 : 0);
+        const int my_slot = whole ? 0 : 2 * static_cast<int>(blockIdx.x) + (it0 < sg.tfirst ? 1 : 0);
         int32_t* pacc = args.ws_acc + static_cast<size_t>(my_slot) * BT * 128;
         float* pcmp = args.ws_comp + static_cast<size_t>(my_slot) * BT * 128;
         // cluster split-K: channel nl goes to owner rank nl / slice
@@ -1082,7 +1185,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         if (!cl && whole) {
           // token scales of the tile, staged once per group
           named_bar_sync(gbar, 128);
-          for (int j = nl; j < BT; j += 128) sa_t[j] = j < mvalid ? args.a[m0 + j] : 0.f;
+          for (int j = nl; j < BT; j += 128) sa_t[j] = j < mvalid ? pr.a[m0 + j] : 0.f;
           named_bar_sync(gbar, 128);
           if (seg == 0 && nl == 0) QLIN_STAMP(16);
         }
@@ -1104,7 +1207,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
             for (int i = 0; i < 4; ++i) {
               st_async_v4(r_main + (c0 + 4 * i) * 4,
                           make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]), r_bar);
-              if (has_comp && comp)
+              if (has_comp)
                 st_async_v4(r_comp + (c0 + 4 * i) * 4,
                             make_uint4(cmp[4 * i], cmp[4 * i + 1], cmp[4 * i + 2], cmp[4 * i + 3]), r_bar);
             }
@@ -1130,15 +1233,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               float v = __fmul_rn(cn, static_cast<float>(static_cast<int32_t>(acc[j])));
-              if (comp) v = __fadd_rn(v, __uint_as_float(cmp[j]));
+              if (pcomp) v = __fadd_rn(v, __uint_as_float(cmp[j]));
               yh[j] = __half_as_ushort(__float2half_rn(__fmul_rn(sc[j], v)));
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) ys[j * 128 + nl] = yh[j];
-            if (args.acc_debug) {
+            if (pr.acc_debug) {
               for (int j = 0; j < 16; ++j)
-                if (c0 + j < mvalid && n < args.N)
-                  args.acc_debug[static_cast<size_t>(m0 + c0 + j) * args.N + n] = static_cast<int32_t>(acc[j]);
+                if (c0 + j < mvalid && n < pr.N)
+                  pr.acc_debug[static_cast<size_t>(m0 + c0 + j) * pr.N + n] = static_cast<int32_t>(acc[j]);
             }
             named_bar_sync(gbar, 128);
 #pragma unroll
@@ -1146,8 +1249,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
               const int idx = nl + h * 128;  // 16 rows x 16 segments of 8 channels
               const int j = idx >> 4;
               const int n8 = tn * C::kBN + (idx & 15) * 8;
-              if (c0 + j < mvalid && n8 < args.N)
-                *reinterpret_cast<uint4*>(args.Y + static_cast<size_t>(m0 + c0 + j) * args.N + n8) =
+              if (c0 + j < mvalid && n8 < pr.N)
+                *reinterpret_cast<uint4*>(pr.Y + static_cast<size_t>(m0 + c0 + j) * pr.N + n8) =
                     *reinterpret_cast<const uint4*>(ys + j * 128 + (idx & 15) * 8);
             }
             if (seg == 0 && nl == 0 && c0 == 0) QLIN_STAMP(17);
@@ -1201,7 +1304,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                   const int4 v = *reinterpret_cast<const int4*>(rb + ((r * slice + c) * C::kRecvLd + 4 * jq) * 4);
                   sum[k].x += v.x; sum[k].y += v.y; sum[k].z += v.z; sum[k].w += v.w;
                 }
-                if (comp) cp[k] = *reinterpret_cast<const float4*>(rb + C::kRecvMain + (c * C::kRecvLd + 4 * jq) * 4);
+                if (pcomp) cp[k] = *reinterpret_cast<const float4*>(rb + C::kRecvMain + (c * C::kRecvLd + 4 * jq) * 4);
                 const float4 t = *reinterpret_cast<const float4*>(sa + 4 * jq);
                 scl[k][0] = t.x; scl[k][1] = t.y; scl[k][2] = t.z; scl[k][3] = t.w;
               }
@@ -1215,24 +1318,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const int j = 4 * jq + i;
-                if (ok && j < mvalid && n_own < args.N) {
+                if (ok && j < mvalid && n_own < pr.N) {
                   float v = __fmul_rn(cn_own, static_cast<float>(s4[i]));
-                  if (comp) v = __fadd_rn(v, p4[i]);
+                  if (pcomp) v = __fadd_rn(v, p4[i]);
                   const float y = __fmul_rn(scl[k][i], v);
-                  args.Y[static_cast<size_t>(m0 + j) * args.N + n_own] = __half_as_ushort(__float2half_rn(y));
-                  if (args.acc_debug) args.acc_debug[static_cast<size_t>(m0 + j) * args.N + n_own] = s4[i];
+                  pr.Y[static_cast<size_t>(m0 + j) * pr.N + n_own] = __half_as_ushort(__float2half_rn(y));
+                  if (pr.acc_debug) pr.acc_debug[static_cast<size_t>(m0 + j) * pr.N + n_own] = s4[i];
                 }
               }
             }
           }
           named_bar_sync(1, 128);  // every read of the receive buffer is done
-          if (nl == 0 && cid + (seg + 1) * args.ncl < args.tiles_n * args.tiles_m) {
+          if (nl == 0 && cid + (seg + 1) * args.ncl < pr.tiles_n * pr.tiles_m) {
             mbar_arrive_expect_tx(recv_full, recv_bytes);  // next round
             for (int r = 0; r < args.cs; ++r) mbar_arrive_remote(mapa_shared(smem_u32(recv_free), r));
           }
         }
         if (!cl && !whole && npend < 2) {
-          pend_tile[npend] = sg.tile;
+          pend_tile[npend] = sg.tfirst;
+          pend_prob[npend] = sg.p;
+          pend_loc[npend] = sg.tile;
           pend_add[npend] = sg.r1 - sg.r0;
           ++npend;
         }
@@ -1249,9 +1354,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           fence_acq_rel_gpu();
           bool any = false;
           for (int q = 0; q < npend; ++q) {
-            const int c_lo = owner_cta_s(pend_tile[q] * static_cast<unsigned>(args.T), sbnd, args);
+            const int c_lo = owner_cta_s(pend_tile[q], sbnd, args);
             const unsigned old = atom_add_relaxed_gpu(&args.ws_cnt[c_lo], static_cast<unsigned>(pend_add[q]));
-            const bool last = old + static_cast<unsigned>(pend_add[q]) == static_cast<unsigned>(args.T);
+            const bool last = old + static_cast<unsigned>(pend_add[q]) == static_cast<unsigned>(probs[pend_prob[q]].T);
             last_flag[q] = last ? 1 : 0;
             any = any || last;
           }
@@ -1261,14 +1366,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
         if (nl == 0) QLIN_STAMP(12);
         for (int q = 0; q < npend; ++q) {
           if (!last_flag[q]) continue;
-          const unsigned tile = pend_tile[q];
-          const unsigned first_it = tile * static_cast<unsigned>(args.T);
+          const GemmProb& pr = probs[pend_prob[q]];
+          const bool pcomp = pr.nO > 0;
+          const unsigned tile = pend_loc[q];
+          const unsigned first_it = pend_tile[q];
           const int c_lo = owner_cta_s(first_it, sbnd, args);
-          const int c_hi = owner_cta_s(first_it + args.T - 1, sbnd, args);
-          const int tn = static_cast<int>(tile % args.tiles_n);
-          const int tm = static_cast<int>(tile / args.tiles_n);
+          const int c_hi = owner_cta_s(first_it + pr.T - 1, sbnd, args);
+          int tn, tm;
+          tile_coords(pr, tile, tn, tm);
           const int m0 = tm * BT;
-          const int mvalid = min(BT, args.M - m0);
+          const int mvalid = min(BT, pr.M - m0);
           if (nl == 0) QLIN_STAMP(16 + 4 * q);
           // Thread t owns channels 4*(t % 32) .. +3, so a warp covers one
           // 128-channel row of the tile; warp w takes rows w, w + 4, ...
@@ -1279,37 +1386,37 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
           const int cg = nl & 31;
           const int wq = nl >> 5;
           const int n4 = tn * C::kBN + 4 * cg;
-          const bool live = n4 < args.N;
+          const bool live = n4 < pr.N;
           float c4[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) c4[i] = chan_scale<FMT>(args, n4 + i);
+          for (int i = 0; i < 4; ++i) c4[i] = chan_scale<FMT>(pr, n4 + i);
           int nctr = 0;
           for (int c = c_lo; c <= c_hi; ++c) nctr += bnd_s(c, sbnd, args) != bnd_s(c + 1, sbnd, args) ? 1 : 0;
-          const int blocks = nctr + (comp ? 1 : 0);
+          const int blocks = nctr + (pcomp ? 1 : 0);
           int rows = C::kOffBar / (blocks * 512 + 4);
           rows = rows > 4 ? rows & ~3 : rows;
           int32_t* fin = reinterpret_cast<int32_t*>(smem);
           // kernel parameters used per row, held in registers (the stores
           // below would otherwise force reloads of the parameter block)
-          uint16_t* const Yp = args.Y;
-          int32_t* const accd = args.acc_debug;
-          const size_t ldy = static_cast<size_t>(args.N);
+          uint16_t* const Yp = pr.Y;
+          int32_t* const accd = pr.acc_debug;
+          const size_t ldy = static_cast<size_t>(pr.N);
           for (int j0 = 0; j0 < mvalid; j0 += rows) {
             const int rr = min(rows, mvalid - j0);
             float* fa = reinterpret_cast<float*>(fin + static_cast<size_t>(blocks) * rr * 128);
             int qq = 0;
             for (int c = c_lo; c <= c_hi; ++c) {
               if (bnd_s(c, sbnd, args) == bnd_s(c + 1, sbnd, args)) continue;
-              const int32_t* src = args.ws_acc + (static_cast<size_t>(partial_slot_s(c, tile, sbnd, args)) * BT + j0) * 128 + 4 * cg;
+              const int32_t* src = args.ws_acc + (static_cast<size_t>(partial_slot_s(c, first_it, sbnd)) * BT + j0) * 128 + 4 * cg;
               for (int j = wq; j < rr; j += 4) cp_async16(fin + (static_cast<size_t>(qq) * rr + j) * 128 + 4 * cg, src + j * 128);
               ++qq;
             }
-            if (comp) {
-              const float* src = args.ws_comp + (static_cast<size_t>(partial_slot_s(c_hi, tile, sbnd, args)) * BT + j0) * 128 + 4 * cg;
+            if (pcomp) {
+              const float* src = args.ws_comp + (static_cast<size_t>(partial_slot_s(c_hi, first_it, sbnd)) * BT + j0) * 128 + 4 * cg;
               for (int j = wq; j < rr; j += 4) cp_async16(fin + (static_cast<size_t>(nctr) * rr + j) * 128 + 4 * cg, src + j * 128);
             }
             if (cg == 0)
-              for (int j = wq; j < rr; j += 4) cp_async4(fa + j, args.a + m0 + j0 + j);
+              for (int j = wq; j < rr; j += 4) cp_async4(fa + j, pr.a + m0 + j0 + j);
             cp_async_wait_all();
             __syncwarp();  // lane 0's token scales
             if (nl == 0 && j0 == 0) QLIN_STAMP(17 + 4 * q);
@@ -1335,7 +1442,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
                 const int j = jb + 4 * i;
                 if (j >= rr) break;
                 float4 cp = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (comp) cp = *reinterpret_cast<const float4*>(fin + (static_cast<size_t>(nctr) * rr + j) * 128 + 4 * cg);
+                if (pcomp) cp = *reinterpret_cast<const float4*>(fin + (static_cast<size_t>(nctr) * rr + j) * 128 + 4 * cg);
                 const float am = fa[j];
                 const int s4[4] = {sum[i].x, sum[i].y, sum[i].z, sum[i].w};
                 const float p4[4] = {cp.x, cp.y, cp.z, cp.w};
@@ -1343,7 +1450,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   float v = __fmul_rn(c4[e], static_cast<float>(s4[e]));
-                  if (comp) v = __fadd_rn(v, p4[e]);
+                  if (pcomp) v = __fadd_rn(v, p4[e]);
                   y[e] = __fmul_rn(am, v);
                 }
                 if (live) {

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -15,6 +16,7 @@
 #include "act_quant.cuh"
 #include "gemm.cuh"
 #include "backward.cuh"
+#include "gptq.cuh"
 #include "pack.cuh"
 
 using namespace qlin;
@@ -217,97 +219,127 @@ int pick_bt(int M) {
   return bt < max_bt() ? bt : max_bt();
 }
 
-// Work decomposition of one GEMM call (same on the host for workspace sizes
-// and for the launch).
+// Work decomposition of one GEMM launch over one or more problems that
+// share the token count M (same on the host for workspace sizes and for the
+// launch).
 struct GemmPlan {
-  int bt, tiles_n, tiles_m, kb, nk, nc, ncs, T, grid, split;
-  int widen;  // INT4 weights widened to INT8 once per call (prefill), then the INT8 kernel
-  size_t u_off, acc_off, comp_off, cnt_off, w8_off, total;
+  int bt, grid, split, widen, nprob;
+  long long tiles;         // tiles of every problem
+  GemmProb pr[kMaxProbs];  // per problem: shape, tiles and iteration offsets (pointers unset)
+  size_t acc_off, comp_off, cnt_off, w8_off, total;  // shared scratch (after the problems' U operands)
+  size_t u_off[kMaxProbs];                           // each problem's compensation operand U
 };
 
 // From this many tokens the INT4 formats widen their weights once per call
 // and run the INT8 kernel (QLIN_KNOB_WIDEN_MIN_M; 0 turns it off).
 int widen_min_m() { return static_cast<int>(knob(QLIN_KNOB_WIDEN_MIN_M)); }
 
-GemmPlan plan_gemm(int M, const qlin_weights* w) {
+GemmPlan plan_gemm_group(int M, const qlin_weights* const* ws, int n) {
   GemmPlan p{};
+  p.nprob = n;
   p.bt = pick_bt(M);
-  p.tiles_n = (w->N + 127) / 128;
-  p.tiles_m = (M + p.bt - 1) / p.bt;
-  p.kb = (w->K + 127) / 128;
   const int ks = gemm_ks(p.bt);
-  p.nk = (p.kb + ks - 1) / ks;
-  p.ncs = w->n_outlier > 0 ? (w->n_outlier + 63) / 64 : 0;
-  p.nc = (p.bt <= 64) ? p.ncs : 2 * p.ncs;
-  p.T = p.nk + p.nc;
+  bool any_outliers = false;
+  unsigned it = 0;
+  for (int q = 0; q < n; ++q) {
+    const qlin_weights* w = ws[q];
+    GemmProb& g = p.pr[q];
+    g.M = M;
+    g.N = w->N;
+    g.K = w->K;
+    g.nO = w->n_outlier;
+    g.tiles_n = (w->N + 127) / 128;
+    g.tiles_m = (M + p.bt - 1) / p.bt;
+    g.kb = (w->K + 127) / 128;
+    g.nk = (g.kb + ks - 1) / ks;
+    g.ncs = w->n_outlier > 0 ? (w->n_outlier + 63) / 64 : 0;
+    g.nc = (p.bt <= 64) ? g.ncs : 2 * g.ncs;
+    g.T = g.nk + g.nc;
+    g.gm = 1;
+    g.it0 = it;
+    it += static_cast<unsigned>(static_cast<long long>(g.tiles_n) * g.tiles_m * g.T);
+    p.tiles += static_cast<long long>(g.tiles_n) * g.tiles_m;
+    any_outliers = any_outliers || w->n_outlier > 0;
+  }
+  long long iters = 0;
+  for (int q = 0; q < n; ++q) iters += static_cast<long long>(p.pr[q].tiles_n) * p.pr[q].tiles_m * p.pr[q].T;
   const int sms = gemm_cta_cap();
-  const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
   // Split tiles (stream-K or cluster split-K) when whole tiles would leave
   // SMs idle or badly balanced.  Token tiles of 128/256 have partials of
   // 64-128 KiB, so they split only when there are fewer tiles than SMs.
-  p.split = tiles < (p.bt >= 128 ? 1LL : 4LL) * sms ? 1 : 0;
-  const long long units = p.split ? tiles * p.T : tiles;
+  // Groups of decode problems split too: their tiles differ in length (K),
+  // and only split points give every CTA the same number of iterations.
+  p.split = (p.tiles < (p.bt >= 128 ? 1LL : 4LL) * sms || (n > 1 && p.bt <= 64)) ? 1 : 0;
+  const long long units = p.split ? iters : p.tiles;
   const int cap = sms < kMaxGrid ? sms : kMaxGrid;
   p.grid = static_cast<int>(units < cap ? units : cap);
   if (p.grid < 1) p.grid = 1;
+  // Raster order of many-token problems: the CTAs running at once should
+  // share weight tiles and reuse activation tiles from L2.  All token tiles
+  // in one group when the INT8 activations (M x K) fit well inside L2, else
+  // groups of about sqrt(grid * 128 / BT) token tiles (the size that
+  // minimises the activation bytes plus the weight bytes one wave of CTAs
+  // touches).
+  for (int q = 0; q < n; ++q) {
+    GemmProb& g = p.pr[q];
+    if (g.tiles_m <= 1) continue;
+    const double x_bytes = static_cast<double>(M) * g.K;
+    int gm = static_cast<int>(std::lround(std::sqrt(static_cast<double>(p.grid) * 128.0 / p.bt)));
+    if (x_bytes <= 48.0 * 1024 * 1024) gm = g.tiles_m;
+    g.gm = gm < 1 ? 1 : (gm > g.tiles_m ? g.tiles_m : gm);
+  }
   size_t off = 0;
-  p.u_off = off;
-  off = round_up(off + (w->n_outlier > 0 ? size_t(2) * M * w->n_outlier_pad * 2 : 0), kAlign);
+  for (int q = 0; q < n; ++q) {
+    p.u_off[q] = off;
+    off = round_up(off + (ws[q]->n_outlier > 0 ? size_t(2) * M * ws[q]->n_outlier_pad * 2 : 0), kAlign);
+  }
   const size_t slot_bytes = size_t(p.bt) * 128 * 4;
   p.acc_off = off;
   off = round_up(off + (p.split ? size_t(2) * p.grid * slot_bytes : 0), kAlign);
   p.comp_off = off;
-  off = round_up(off + (p.split && w->n_outlier > 0 ? size_t(2) * p.grid * slot_bytes : 0), kAlign);
+  off = round_up(off + (p.split && any_outliers ? size_t(2) * p.grid * slot_bytes : 0), kAlign);
   p.cnt_off = off;
   off = round_up(off + (p.split ? size_t(p.grid) * 4 : 0), kAlign);
-  p.widen = (w->fmt != QLIN_W8_PERCHANNEL && p.bt == 256 && widen_min_m() > 0 && M >= widen_min_m()) ? 1 : 0;
+  p.widen = (n == 1 && ws[0]->fmt != QLIN_W8_PERCHANNEL && p.bt == 256 && widen_min_m() > 0 && M >= widen_min_m())
+                ? 1 : 0;
   p.w8_off = off;
-  off = round_up(off + (p.widen ? size_t(p.tiles_n) * p.kb * 16384 : 0), kAlign);
+  off = round_up(off + (p.widen ? size_t(p.pr[0].tiles_n) * p.pr[0].kb * 16384 : 0), kAlign);
   p.total = off;
   return p;
 }
 
+GemmPlan plan_gemm(int M, const qlin_weights* w) { return plan_gemm_group(M, &w, 1); }
+
+constexpr int kGroupMaxM = 64;  // token counts a grouped launch takes (decode-sized tiles)
+
 // ---------------------------------------------------------------- GEMM launch
-template <int FMT, int BT>
-qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_t* U, GemmArgs args,
-                          cudaStream_t stream) {
+template <int FMT, int BT, int MAXP>
+qlin_status launch_gemm_t(GemmParams<MAXP>& prm, cudaStream_t stream) {
   using C = GemmCfg<FMT, BT>;
-  auto kern = gemm_kernel<FMT, BT>;
+  auto kern = gemm_kernel<FMT, BT, MAXP>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return fail(QLIN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-
-  CUtensorMap tmX, tmU, tmY;
-  memset(&tmU, 0, sizeof(tmU));
-  const int K = w->K, M = args.M;
-  qlin_status st = make_map(&tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, BT, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != QLIN_OK) return st;
-  // Y [M][N] fp16, written in 16-token x 128-channel boxes
-  st = make_map(&tmY, args.Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w->N, M, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (st != QLIN_OK) return st;
-  if (w->n_outlier > 0) {
-    st = make_map(&tmU, U, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->n_outlier_pad, 2 * static_cast<uint64_t>(M), 64, BT,
-                  CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != QLIN_OK) return st;
-  }
-  // Token tiles up to 64 whose tiles would be split (decode): cluster
-  // split-K when it is expected to beat global-memory stream-K.  Costs in
-  // units of one pipeline step, fitted to B200 measurements of the 7B decode
-  // shapes: a cluster round costs its longest rank range plus the exchange of
-  // BT x 128 partials through distributed shared memory (about 0.5 / 2 / 7.5
-  // steps at BT = 16 / 32 / 64); stream-K costs its per-CTA iterations plus
-  // the global fixup chain (about 7 / 12 / 28 steps).  QLIN_CLUSTER_CS=n
-  // forces cluster size n when it is valid (measurement aid).
-  if (C::kCluster && args.split && !cluster_disabled()) {
+  GemmArgs& args = prm.g;
+  // Single-problem launches whose token tiles (up to 64) would be split
+  // (decode): cluster split-K when it is expected to beat global-memory
+  // stream-K.  Costs in units of one pipeline step, fitted to B200
+  // measurements of the 7B decode shapes: a cluster round costs its longest
+  // rank range plus the exchange of BT x 128 partials through distributed
+  // shared memory (about 0.5 / 2 / 7.5 steps at BT = 16 / 32 / 64);
+  // stream-K costs its per-CTA iterations plus the global fixup chain
+  // (about 7 / 12 / 28 steps).  QLIN_KNOB_CLUSTER_SIZE forces a size.
+  if (MAXP == 1 && C::kCluster && args.split && !cluster_disabled()) {
+    const GemmProb& g0 = prm.pr[0];
     const double xchg = BT <= 16 ? 0.5 : (BT <= 32 ? 2.0 : 7.5);
     const double fixup = BT <= 16 ? 7.0 : (BT <= 32 ? 12.0 : 28.0);
     const int forced = forced_cluster_size();
-    const long long iters = static_cast<long long>(args.tiles_n) * args.tiles_m * args.T;
+    const long long iters = static_cast<long long>(g0.tiles_n) * g0.tiles_m * g0.T;
     const double streamk_cost = static_cast<double>((iters + args.grid - 1) / args.grid) + fixup;
-    const long long tiles = static_cast<long long>(args.tiles_n) * args.tiles_m;
+    const long long tiles = static_cast<long long>(g0.tiles_n) * g0.tiles_m;
     static int max_clusters[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};  // per cluster size, this instantiation
     int best_cs = 0, best_ncl = 0;
     double best_cost = streamk_cost;
@@ -315,8 +347,8 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
     // fp32 partial (about BT / 32 steps at cs = 4)
     for (int cs = 2; cs <= 8; cs *= 2) {
       int cb[9];
-      const double ccost = (args.T - args.nk) + (args.nO > 0 ? BT / 32.0 * 4.0 / cs : 0.0);
-      const double span = cluster_bounds(args.T, args.nk, cs, ccost, cb);
+      const double ccost = (g0.T - g0.nk) + (g0.nO > 0 ? BT / 32.0 * 4.0 / cs : 0.0);
+      const double span = cluster_bounds(g0.T, g0.nk, cs, ccost, cb);
       if (span < 0) continue;
       if (max_clusters[cs] < 0) {
         cudaLaunchConfig_t cfg = {};
@@ -352,84 +384,110 @@ qlin_status launch_gemm_t(const qlin_weights* w, const int8_t* Xq, const uint16_
       args.cs = best_cs;
       args.ncl = best_ncl;
       args.grid = best_cs * best_ncl;
-      cluster_bounds(args.T, args.nk, best_cs,
-                     (args.T - args.nk) + (args.nO > 0 ? BT / 32.0 * 4.0 / best_cs : 0.0), args.cb);
+      cluster_bounds(g0.T, g0.nk, best_cs,
+                     (g0.T - g0.nk) + (g0.nO > 0 ? BT / 32.0 * 4.0 / best_cs : 0.0), args.cb);
     }
   }
-  cudaError_t e =
-      launch_kc(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, args.cs, tmX, tmU, tmY, args);
+  cudaError_t e = launch_kc(kern, dim3(args.grid), dim3(C::kThreads), C::kSmemBytes, stream, args.cs, prm);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
 }
 
-template <int FMT>
-qlin_status launch_gemm_fmt(int bt, const qlin_weights* w, const int8_t* Xq, const uint16_t* U, const GemmArgs& args,
-                            cudaStream_t stream) {
+// Grouped launches (MAXP > 1) take decode-sized token tiles only (<= 64).
+template <int FMT, int MAXP>
+qlin_status launch_gemm_fmt(int bt, GemmParams<MAXP>& prm, cudaStream_t stream) {
   switch (bt) {
-    case 16: return launch_gemm_t<FMT, 16>(w, Xq, U, args, stream);
-    case 32: return launch_gemm_t<FMT, 32>(w, Xq, U, args, stream);
-    case 64: return launch_gemm_t<FMT, 64>(w, Xq, U, args, stream);
-    case 128: return launch_gemm_t<FMT, 128>(w, Xq, U, args, stream);
-    default: return launch_gemm_t<FMT, 256>(w, Xq, U, args, stream);
+    case 16: return launch_gemm_t<FMT, 16, MAXP>(prm, stream);
+    case 32: return launch_gemm_t<FMT, 32, MAXP>(prm, stream);
+    case 64: return launch_gemm_t<FMT, 64, MAXP>(prm, stream);
+    default:
+      if constexpr (MAXP == 1) {
+        if (bt == 128) return launch_gemm_t<FMT, 128, 1>(prm, stream);
+        return launch_gemm_t<FMT, 256, 1>(prm, stream);
+      } else {
+        return fail(QLIN_ERR_SHAPE, "grouped GEMMs take at most %d tokens", kGroupMaxM);
+      }
   }
 }
 
-// `gws` is the GEMM scratch laid out by plan_gemm (U first).
-qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, int M, uint16_t* Y,
-                        int32_t* acc_debug, char* gws, cudaStream_t stream) {
+// One GEMM launch over the problems of a plan.  Per problem q: weights
+// ws[q], the INT8 activations Xq[q], token scales a[q], output Y[q] and
+// (optional) acc_debug[q]; `gws` is the scratch laid out by the plan (each
+// problem's U, then the shared split-K slots and counters).
+template <int MAXP>
+qlin_status launch_gemm_group(const GemmPlan& p, const qlin_weights* const* ws, const int8_t* const* Xq,
+                              const float* const* a, uint16_t* const* Y, int32_t* const* acc_debug, char* gws,
+                              cudaStream_t stream) {
   qlin_status st = get_encoder();
   if (st != QLIN_OK) return st;
-  const GemmPlan p = plan_gemm(M, w);
-  GemmArgs args;
-  args.codes = static_cast<const uint8_t*>(w->codes);
-  args.rfold = w->fold_ratio;
-  args.wot = w->W_Ot;
-  args.cscale = w->chan_scale;
-  args.a = a;
-  args.Y = Y;
-  args.acc_debug = acc_debug;
+  static_assert(sizeof(GemmParams<MAXP>) <= 32000, "kernel parameter space");
+  GemmParams<MAXP> prm;
+  memset(&prm, 0, sizeof(prm));
+  GemmArgs& args = prm.g;
+  const int M = p.pr[0].M;
+  long long iters = 0;
+  for (int q = 0; q < p.nprob; ++q) {
+    const qlin_weights* w = ws[q];
+    GemmProb& g = prm.pr[q];
+    g = p.pr[q];
+    g.codes = static_cast<const uint8_t*>(w->codes);
+    g.rfold = w->fold_ratio;
+    g.wot = w->W_Ot;
+    g.cscale = w->chan_scale;
+    g.a = a[q];
+    g.Y = Y[q];
+    g.acc_debug = acc_debug ? acc_debug[q] : nullptr;
+    g.cmul = 1.f;
+    iters += static_cast<long long>(g.tiles_n) * g.tiles_m * g.T;
+    st = make_map(&prm.tmX[q], Xq[q], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K, M, 128, p.bt,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QLIN_OK) return st;
+    if (w->n_outlier > 0) {
+      st = make_map(&prm.tmU[q], gws + p.u_off[q], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->n_outlier_pad,
+                    2 * static_cast<uint64_t>(M), 64, p.bt, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (st != QLIN_OK) return st;
+    }
+  }
+  if (iters >= (1LL << 31)) return fail(QLIN_ERR_SHAPE, "problem too large (%lld tile iterations)", iters);
   args.ws_acc = reinterpret_cast<int32_t*>(gws + p.acc_off);
   args.ws_comp = reinterpret_cast<float*>(gws + p.comp_off);
   args.ws_cnt = reinterpret_cast<unsigned*>(gws + p.cnt_off);
-  args.M = M;
-  args.N = w->N;
-  args.K = w->K;
-  args.nO = w->n_outlier;
-  args.tiles_n = p.tiles_n;
-  args.tiles_m = p.tiles_m;
-  args.kb = p.kb;
-  args.nk = p.nk;
-  args.nc = p.nc;
-  args.ncs = p.ncs;
-  args.T = p.T;
+  args.nprob = p.nprob;
   args.grid = p.grid;
   args.split = p.split;
+  args.total = static_cast<unsigned>(iters);
   args.cs = 1;
   args.ncl = 0;
-  for (int r = 0; r < 9; ++r) args.cb[r] = 0;
-  const long long tiles = static_cast<long long>(p.tiles_n) * p.tiles_m;
-  if (tiles * p.T >= (1LL << 31)) return fail(QLIN_ERR_SHAPE, "problem too large (%lld tile iterations)", tiles * p.T);
-  for (int c = 0; c <= p.grid; ++c) args.bnd[c] = gemm_boundary(c, tiles, p.T, p.nk, p.grid, p.split);
-  const uint16_t* U = reinterpret_cast<const uint16_t*>(gws + p.u_off);
-  args.cmul = 1.f;
+  gemm_boundaries(prm.pr, p.nprob, p.grid, p.split, args.bnd);
+  const int fmt = ws[0]->fmt;
   if (p.widen) {
+    const qlin_weights* w = ws[0];
     uint8_t* w8 = reinterpret_cast<uint8_t*>(gws + p.w8_off);
-    const unsigned nblk = static_cast<unsigned>(p.tiles_n) * static_cast<unsigned>(p.kb);
+    const unsigned nblk = static_cast<unsigned>(p.pr[0].tiles_n) * static_cast<unsigned>(p.pr[0].kb);
     const uint8_t* codes = static_cast<const uint8_t*>(w->codes);
     const uint16_t* rf = reinterpret_cast<const uint16_t*>(w->fold_ratio);
-    cudaError_t e = w->fmt == QLIN_W4_PERCHANNEL
-                        ? launch_k(widen_w4_kernel<kFmtW4PC>, dim3(nblk), dim3(256), 0, stream, codes, rf, w->N, p.kb, w8)
-                        : launch_k(widen_w4_kernel<kFmtW4G128>, dim3(nblk), dim3(256), 0, stream, codes, rf, w->N, p.kb, w8);
+    cudaError_t e = fmt == QLIN_W4_PERCHANNEL
+                        ? launch_k(widen_w4_kernel<kFmtW4PC>, dim3(nblk), dim3(256), 0, stream, codes, rf, w->N,
+                                   p.pr[0].kb, w8)
+                        : launch_k(widen_w4_kernel<kFmtW4G128>, dim3(nblk), dim3(256), 0, stream, codes, rf, w->N,
+                                   p.pr[0].kb, w8);
     if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "widen_w4_kernel launch failed: %s", cudaGetErrorString(e));
-    args.codes = w8;
-    args.cmul = w->fmt == QLIN_W4_PERCHANNEL ? 0.0625f : 1.f;
-    return launch_gemm_fmt<kFmtW8>(p.bt, w, Xq, U, args, stream);
+    prm.pr[0].codes = w8;
+    prm.pr[0].cmul = fmt == QLIN_W4_PERCHANNEL ? 0.0625f : 1.f;
+    return launch_gemm_fmt<kFmtW8, MAXP>(p.bt, prm, stream);
   }
-  switch (w->fmt) {
-    case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC>(p.bt, w, Xq, U, args, stream);
-    case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128>(p.bt, w, Xq, U, args, stream);
-    default: return launch_gemm_fmt<kFmtW8>(p.bt, w, Xq, U, args, stream);
+  switch (fmt) {
+    case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC, MAXP>(p.bt, prm, stream);
+    case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128, MAXP>(p.bt, prm, stream);
+    default: return launch_gemm_fmt<kFmtW8, MAXP>(p.bt, prm, stream);
   }
+}
+
+// Single-problem GEMM launch.
+qlin_status launch_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, int M, uint16_t* Y,
+                        int32_t* acc_debug, char* gws, cudaStream_t stream) {
+  const GemmPlan p = plan_gemm(M, w);
+  return launch_gemm_group<1>(p, &w, &Xq, &a, &Y, acc_debug ? &acc_debug : nullptr, gws, stream);
 }
 
 // ---------------------------------------------------------------- act quant
@@ -444,55 +502,105 @@ size_t act_ws_bytes(const qlin_weights* w) {
   return w->n_outlier > 0 ? round_up(size_t(w->n_outlier) * 4 + 4, kAlign) : 0;
 }
 
-qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float* s, float gamma, int update,
-                         int8_t* Xq, float* a, int8_t* XqO, uint16_t* U, void* act_ws, cudaStream_t stream) {
-  const int K = w->K, nO = w->n_outlier;
-  if (M == 0) return QLIN_OK;
-  unsigned* cmax = static_cast<unsigned*>(act_ws);
-  MomentumArgs mom{w->wmax_O, gamma, cmax ? cmax + nO : nullptr, M};
-  const bool do_update = update && nO > 0;
-  const bool fused = do_update && M <= fused_momentum_max_m();
-  if (do_update && !fused) {
-    const int grid = (M + kColmaxRows - 1) / kColmaxRows;
-    cudaError_t e = launch_k(colmax_kernel, dim3(grid), dim3(256), size_t(nO) * 8, stream, X, M, K,
-                             static_cast<const int32_t*>(w->outlier_idx), nO, cmax, 1,
-                             static_cast<const float*>(w->wmax_O), s, gamma, cmax + nO);
-    if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "colmax_kernel launch failed: %s", cudaGetErrorString(e));
-  }
-  const int nvec = K / 8;
-  const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
-  const size_t smem = size_t(K) * 2 + size_t(nO) * 16;
-  if (smem > size_t(kQuantSmemMax))
-    return fail(QLIN_ERR_SHAPE, "K=%d with %d outliers needs %zu bytes of shared memory", K, nO, smem);
-  const int nOp = w->n_outlier_pad;
-  cudaError_t e = cudaSuccess;
-#define QLIN_QUANT_CASE(V)                                                                                   \
-  {                                                                                                          \
-    static std::once_flag once_##V;                                                                          \
-    static cudaError_t attr_##V = cudaSuccess;                                                               \
-    std::call_once(once_##V, [] {                                                                            \
-      attr_##V = cudaFuncSetAttribute(quant_kernel<V, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,     \
-                                      kQuantSmemMax);                                                        \
-      if (attr_##V == cudaSuccess)                                                                           \
-        attr_##V = cudaFuncSetAttribute(quant_kernel<V, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                        kQuantSmemMax);                                                      \
-    });                                                                                                      \
-    if (attr_##V != cudaSuccess)                                                                             \
-      return fail(QLIN_ERR_CUDA, "quant_kernel attribute: %s", cudaGetErrorString(attr_##V));               \
-  }                                                                                                          \
-  e = fused ? launch_k(quant_kernel<V, true>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,             \
-                       static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom)         \
-            : launch_k(quant_kernel<V, false>, dim3(M), dim3(kQuantThreads), smem, stream, X, K,            \
-                       static_cast<const int32_t*>(w->outlier_idx), nO, s, Xq, a, XqO, U, nOp, mom);
-  if (vpt <= 1) { QLIN_QUANT_CASE(1) }
-  else if (vpt <= 2) { QLIN_QUANT_CASE(2) }
-  else if (vpt <= 4) { QLIN_QUANT_CASE(4) }
-  else if (vpt <= 8) { QLIN_QUANT_CASE(8) }
-  else if (vpt <= 16) { QLIN_QUANT_CASE(16) }
-  else return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", K);
-#undef QLIN_QUANT_CASE
+// Activations of one quantization problem (outputs and scratch per problem).
+struct QuantIO {
+  const uint16_t* X;
+  float* s;
+  int8_t* Xq;
+  float* a;
+  int8_t* XqO;
+  uint16_t* U;   // compensation operand (qlin_forward), or null
+  void* act_ws;  // outlier column maxima + completion counter (update only)
+};
+
+template <int VPT, bool FUSED, int MAXP>
+qlin_status launch_quant_v(const QuantGroup<MAXP>& qg, int rows, size_t smem, cudaStream_t stream) {
+  auto kern = quant_kernel<VPT, FUSED, MAXP>;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmemMax); });
+  if (attr != cudaSuccess) return fail(QLIN_ERR_CUDA, "quant_kernel attribute: %s", cudaGetErrorString(attr));
+  cudaError_t e = launch_k(kern, dim3(rows), dim3(kQuantThreads), smem, stream, qg);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "quant_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
+}
+
+template <bool FUSED, int MAXP>
+qlin_status launch_quant_f(const QuantGroup<MAXP>& qg, int rows, int vpt, size_t smem, cudaStream_t stream) {
+  if (vpt <= 1) return launch_quant_v<1, FUSED, MAXP>(qg, rows, smem, stream);
+  if (vpt <= 2) return launch_quant_v<2, FUSED, MAXP>(qg, rows, smem, stream);
+  if (vpt <= 4) return launch_quant_v<4, FUSED, MAXP>(qg, rows, smem, stream);
+  if (vpt <= 8) return launch_quant_v<8, FUSED, MAXP>(qg, rows, smem, stream);
+  return launch_quant_v<16, FUSED, MAXP>(qg, rows, smem, stream);
+}
+
+// Stage 1 for one problem or a group (same M): the momentum update (fused
+// into the quantization kernel up to the fused-momentum token count, else a
+// column-max kernel per problem first), then one quantization launch with a
+// CTA per token row of every problem.
+template <int MAXP>
+qlin_status launch_quant_group(const qlin_weights* const* ws, const QuantIO* io, int n, int M, float gamma,
+                               int update, cudaStream_t stream) {
+  if (M == 0) return QLIN_OK;
+  QuantGroup<MAXP> qg;
+  memset(&qg, 0, sizeof(qg));
+  qg.gamma = gamma;
+  qg.nprob = n;
+  bool any_update = false;
+  int maxK = 0;
+  size_t smem = 0;
+  for (int q = 0; q < n; ++q) {
+    const qlin_weights* w = ws[q];
+    const int K = w->K, nO = w->n_outlier;
+    QuantProb& p = qg.pr[q];
+    unsigned* cmax = static_cast<unsigned*>(io[q].act_ws);
+    p.X = io[q].X;
+    p.O = static_cast<const int32_t*>(w->outlier_idx);
+    p.s = io[q].s;
+    p.Xq = io[q].Xq;
+    p.a = io[q].a;
+    p.XqO = io[q].XqO;
+    p.U = io[q].U;
+    p.wmaxO = w->wmax_O;
+    p.counter = cmax ? cmax + nO : nullptr;
+    p.K = K;
+    p.nO = nO;
+    p.nOp = w->n_outlier_pad;
+    p.M = M;
+    p.row0 = q * M;
+    any_update = any_update || (update && nO > 0);
+    if (K > maxK) maxK = K;
+    const size_t sm = size_t(K) * 2 + size_t(nO) * 16;
+    if (sm > smem) smem = sm;
+  }
+  if (smem > size_t(kQuantSmemMax))
+    return fail(QLIN_ERR_SHAPE, "K=%d with its outliers needs %zu bytes of shared memory", maxK, smem);
+  const int nvec = maxK / 8;
+  const int vpt = (nvec + kQuantThreads - 1) / kQuantThreads;
+  if (vpt > 16) return fail(QLIN_ERR_SHAPE, "K=%d too large for the quantization kernel", maxK);
+  const bool fused = any_update && M <= fused_momentum_max_m();
+  if (any_update && !fused) {
+    for (int q = 0; q < n; ++q) {
+      const qlin_weights* w = ws[q];
+      const int nO = w->n_outlier;
+      if (nO == 0) continue;
+      unsigned* cmax = static_cast<unsigned*>(io[q].act_ws);
+      const int grid = (M + kColmaxRows - 1) / kColmaxRows;
+      cudaError_t e = launch_k(colmax_kernel, dim3(grid), dim3(256), size_t(nO) * 8, stream, io[q].X, M, w->K,
+                               static_cast<const int32_t*>(w->outlier_idx), nO, cmax, 1,
+                               static_cast<const float*>(w->wmax_O), io[q].s, gamma, cmax + nO);
+      if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "colmax_kernel launch failed: %s", cudaGetErrorString(e));
+    }
+  }
+  const int rows = n * M;
+  return fused ? launch_quant_f<true, MAXP>(qg, rows, vpt, smem, stream)
+               : launch_quant_f<false, MAXP>(qg, rows, vpt, smem, stream);
+}
+
+qlin_status launch_quant(const uint16_t* X, int M, const qlin_weights* w, float* s, float gamma, int update,
+                         int8_t* Xq, float* a, int8_t* XqO, uint16_t* U, void* act_ws, cudaStream_t stream) {
+  const QuantIO io{X, s, Xq, a, XqO, U, act_ws};
+  return launch_quant_group<1>(&w, &io, 1, M, gamma, update, stream);
 }
 
 size_t gemm_ws_bytes(int M, const qlin_weights* w) { return M > 0 ? plan_gemm(M, w).total : 0; }
@@ -511,6 +619,45 @@ FwdLayout forward_layout(int M, const qlin_weights* w) {
   L.gemm = off; off = round_up(off + gemm_ws_bytes(M, w), kAlign);
   L.total = off;
   return L;
+}
+
+// Workspace of a grouped forward: per problem the quantization scratch, Xq,
+// a and XqO, then the GEMM launch's scratch (every problem's U and the
+// shared split-K slots and counters).
+struct GroupLayout {
+  size_t act[kMaxProbs], xq[kMaxProbs], a[kMaxProbs], xqo[kMaxProbs];
+  size_t gemm, total;
+  GemmPlan plan;
+};
+
+GroupLayout group_layout(int M, const qlin_weights* const* ws, int n) {
+  GroupLayout L{};
+  size_t off = 0;
+  for (int q = 0; q < n; ++q) {
+    const qlin_weights* w = ws[q];
+    L.act[q] = off; off = round_up(off + act_ws_bytes(w), kAlign);
+    L.xq[q] = off; off = round_up(off + size_t(M) * w->K, kAlign);
+    L.a[q] = off; off = round_up(off + size_t(M) * 4, kAlign);
+    L.xqo[q] = off; off = round_up(off + size_t(M) * w->n_outlier, kAlign);
+  }
+  L.plan = plan_gemm_group(M > 0 ? M : 1, ws, n);
+  L.gemm = off;
+  off = round_up(off + (M > 0 ? L.plan.total : 0), kAlign);
+  L.total = off;
+  return L;
+}
+
+qlin_status check_group(int32_t count, const qlin_weights* const* w, int32_t M) {
+  if (count < 1 || count > kMaxProbs) return fail(QLIN_ERR_SHAPE, "count=%d must be in [1, %d]", count, kMaxProbs);
+  if (!w) return fail(QLIN_ERR_ARG, "weights array is NULL");
+  if (M < 0) return fail(QLIN_ERR_ARG, "M=%d is negative", M);
+  if (M > kGroupMaxM) return fail(QLIN_ERR_SHAPE, "M=%d: grouped forwards take at most %d tokens", M, kGroupMaxM);
+  for (int q = 0; q < count; ++q) {
+    qlin_status st = check_weights(w[q]);
+    if (st != QLIN_OK) return fail(st, "problem %d: %s", q, t_last_error);
+    if (w[q]->fmt != w[0]->fmt) return fail(QLIN_ERR_ARG, "problem %d: every problem must have the same format", q);
+  }
+  return QLIN_OK;
 }
 
 }  // namespace
@@ -816,7 +963,7 @@ qlin_status qlin_gemm(const qlin_weights* w, const int8_t* Xq, const float* a, c
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char* gws = static_cast<char*>(workspace);
   if (nO > 0) {
-    uint16_t* U = reinterpret_cast<uint16_t*>(gws + plan_gemm(M, w).u_off);
+    uint16_t* U = reinterpret_cast<uint16_t*>(gws + plan_gemm(M, w).u_off[0]);
     const size_t total = size_t(M) * w->n_outlier_pad;
     comp_operand_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(XqO, s, M, nO,
                                                                                        w->n_outlier_pad, U);
@@ -912,7 +1059,7 @@ qlin_status qlin_forward(const uint16_t* X, int32_t M, const qlin_weights* w, fl
   float* a = reinterpret_cast<float*>(ws + L.a);
   int8_t* XqO = nO > 0 ? reinterpret_cast<int8_t*>(ws + L.xqo) : nullptr;
   char* gws = ws + L.gemm;
-  uint16_t* U = nO > 0 ? reinterpret_cast<uint16_t*>(gws + plan_gemm(M, w).u_off) : nullptr;
+  uint16_t* U = nO > 0 ? reinterpret_cast<uint16_t*>(gws + plan_gemm(M, w).u_off[0]) : nullptr;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   st = launch_quant(X, M, w, s, gamma, update_momentum, Xq, a, XqO, U, ws + L.act, stream);
   if (st != QLIN_OK) return st;
@@ -929,6 +1076,135 @@ QLIN_API int qlin_steps_set(long long* p) {
   return static_cast<int>(cudaMemcpyToSymbol(qlin::g_steps, &p, sizeof(p)));
 }
 #endif
+
+qlin_status qlin_forward_grouped_workspace(int32_t count, const qlin_weights* const* w, int32_t M, size_t* bytes) {
+  qlin_status st = check_group(count, w, M);
+  if (st != QLIN_OK) return st;
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  *bytes = group_layout(M, w, count).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_forward_grouped(int32_t count, const qlin_weights* const* w, const uint16_t* const* X,
+                                 float* const* s, uint16_t* const* Y, int32_t M, float gamma,
+                                 int32_t update_momentum, void* workspace, size_t ws_bytes, void* stream_) {
+  qlin_status st = check_group(count, w, M);
+  if (st != QLIN_OK) return st;
+  if (!(gamma >= 0.f && gamma <= 1.f)) return fail(QLIN_ERR_ARG, "gamma=%g outside [0, 1]", double(gamma));
+  if (M == 0) return QLIN_OK;
+  if (!X || !Y || !s) return fail(QLIN_ERR_ARG, "X/Y/s array is NULL");
+  for (int q = 0; q < count; ++q) {
+    if (!X[q] || !Y[q]) return fail(QLIN_ERR_ARG, "problem %d: X/Y is NULL", q);
+    if (w[q]->n_outlier > 0 && !s[q]) return fail(QLIN_ERR_ARG, "problem %d: s is NULL with n_outlier=%d", q,
+                                                  w[q]->n_outlier);
+    if (!aligned16(X[q]) || !aligned16(Y[q]) || (s[q] && !aligned16(s[q])))
+      return fail(QLIN_ERR_ALIGN, "problem %d: X/Y/s is not 16-byte aligned", q);
+    for (int r = 0; r < q; ++r)
+      if (Y[r] == Y[q]) return fail(QLIN_ERR_ARG, "problems %d and %d write the same Y", r, q);
+  }
+  const GroupLayout L = group_layout(M, w, count);
+  if (ws_bytes < L.total || !workspace) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, L.total);
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
+  char* ws = static_cast<char*>(workspace);
+  char* gws = ws + L.gemm;
+  QuantIO io[kMaxProbs];
+  const int8_t* xq[kMaxProbs];
+  const float* av[kMaxProbs];
+  uint16_t* yv[kMaxProbs];
+  for (int q = 0; q < count; ++q) {
+    const bool o = w[q]->n_outlier > 0;
+    io[q] = QuantIO{X[q], s[q], reinterpret_cast<int8_t*>(ws + L.xq[q]), reinterpret_cast<float*>(ws + L.a[q]),
+                    o ? reinterpret_cast<int8_t*>(ws + L.xqo[q]) : nullptr,
+                    o ? reinterpret_cast<uint16_t*>(gws + L.plan.u_off[q]) : nullptr, ws + L.act[q]};
+    xq[q] = io[q].Xq;
+    av[q] = io[q].a;
+    yv[q] = Y[q];
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  st = launch_quant_group<kMaxProbs>(w, io, count, M, gamma, update_momentum, stream);
+  if (st != QLIN_OK) return st;
+  return launch_gemm_group<kMaxProbs>(L.plan, w, xq, av, yv, nullptr, gws, stream);
+}
+
+namespace {
+struct GptqLayout {
+  size_t st, f, a, total;
+};
+GptqLayout gptq_layout(int K) {
+  GptqLayout L{};
+  L.st = 0;
+  L.f = round_up(sizeof(GjScratch), kAlign);
+  L.a = round_up(L.f + size_t(K) * 8, kAlign);
+  L.total = round_up(L.a + size_t(K) * K * 8, kAlign);
+  return L;
+}
+qlin_status check_gptq_shape(int32_t K, int32_t N) {
+  if (K < 1 || N < 1) return fail(QLIN_ERR_ARG, "K=%d N=%d must be positive", K, N);
+  if (K > 16384) return fail(QLIN_ERR_SHAPE, "K=%d exceeds 16384", K);
+  return QLIN_OK;
+}
+}  // namespace
+
+qlin_status qlin_gptq_workspace(int32_t K, int32_t N, size_t* bytes) {
+  qlin_status st = check_gptq_shape(K, N);
+  if (st != QLIN_OK) return st;
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  *bytes = gptq_layout(K).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_gptq_quantize(const double* X, int32_t ns, int32_t K, int32_t N, double* W, const double* scale,
+                               int32_t qmax, int8_t* codes, double* Hinv, int32_t* singular, void* workspace,
+                               size_t ws_bytes, void* stream_) {
+  qlin_status st = check_gptq_shape(K, N);
+  if (st != QLIN_OK) return st;
+  if (ns < 1) return fail(QLIN_ERR_ARG, "ns=%d must be positive", ns);
+  if (qmax < 1 || qmax > 127) return fail(QLIN_ERR_ARG, "qmax=%d outside [1, 127]", qmax);
+  if (!X || !W || !scale || !codes || !Hinv || !workspace) return fail(QLIN_ERR_ARG, "a GPTQ buffer is NULL");
+  if ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(scale) |
+       reinterpret_cast<uintptr_t>(Hinv)) & 7u)
+    return fail(QLIN_ERR_ALIGN, "fp64 buffers must be 8-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const GptqLayout L = gptq_layout(K);
+  if (ws_bytes < L.total) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, L.total);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  char* ws = static_cast<char*>(workspace);
+  GjScratch* scr = reinterpret_cast<GjScratch*>(ws + L.st);
+  double* f = reinterpret_cast<double*>(ws + L.f);
+  double* a = reinterpret_cast<double*>(ws + L.a);
+  QLIN_CUDA_TRY(cudaMemsetAsync(scr, 0, sizeof(GjScratch), stream));
+  // H = 2 X^T X into the working matrix; the inverse starts as the identity
+  const unsigned th = static_cast<unsigned>((K + kHessTile - 1) / kHessTile);
+  gptq_hessian_kernel<<<dim3(th, th), 256, 0, stream>>>(X, ns, K, a);
+  QLIN_LAUNCH_CHECK("gptq_hessian_kernel");
+  const size_t kk = size_t(K) * K;
+  gptq_identity_kernel<<<static_cast<unsigned>((kk + 255) / 256), 256, 0, stream>>>(Hinv, K);
+  QLIN_LAUNCH_CHECK("gptq_identity_kernel");
+  // Gauss-Jordan elimination with partial pivoting: a -> I, Hinv -> H^-1
+  const unsigned cb = static_cast<unsigned>((K + 255) / 256);
+  const unsigned ex = cb < 4 ? cb : 4;
+  for (int c = 0; c < K; ++c) {
+    gj_pivot_kernel<<<1, 1024, 0, stream>>>(a, K, c, scr, f);
+    gj_swap_scale_kernel<<<cb, 256, 0, stream>>>(a, Hinv, K, c, scr);
+    gj_eliminate_kernel<<<dim3(ex, static_cast<unsigned>(K)), 256, 0, stream>>>(a, Hinv, K, c, scr, f);
+  }
+  QLIN_LAUNCH_CHECK("Gauss-Jordan kernels");
+  // column-sequential quantization with compensation on a working copy of H^-1
+  QLIN_CUDA_TRY(cudaMemcpyAsync(a, Hinv, kk * 8, cudaMemcpyDeviceToDevice, stream));
+  constexpr int kRows = 64;
+  for (int i = 0; i < K; ++i) {
+    const int rem = K - i - 1;
+    const int yw = rem > 0 ? (rem + kRows - 1) / kRows : 1;
+    const int yd = rem > 0 ? (rem + kRows - 1) / kRows : 0;
+    const int xa = (N + 255) / 256, xd = (rem + 255) / 256;
+    const unsigned gx = static_cast<unsigned>(xa > xd ? xa : xd);
+    gptq_step_kernel<<<dim3(gx, static_cast<unsigned>(yw + yd)), 256, 0, stream>>>(W, codes, scale, a, K, N, i, qmax,
+                                                                                  kRows, yw, scr);
+  }
+  QLIN_LAUNCH_CHECK("gptq_step_kernel");
+  if (singular) QLIN_CUDA_TRY(cudaMemcpyAsync(singular, &scr->singular, 4, cudaMemcpyDeviceToDevice, stream));
+  return QLIN_OK;
+}
 
 qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
   if (k < 0 || k > QLIN_KNOB_WAIT_NS) return fail(QLIN_ERR_ARG, "unknown knob %d", k);

@@ -29,7 +29,8 @@ EXPORTED = [
     "qlin_pack_weights", "qlin_quant_act_workspace", "qlin_quant_act", "qlin_outlier_colmax",
     "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
     "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc", "qlin_backward_dx",
-    "qlin_backward_dx_workspace", "qlin_debug_set", "qlin_debug_get",
+    "qlin_backward_dx_workspace", "qlin_debug_set", "qlin_debug_get", "qlin_forward_grouped_workspace",
+    "qlin_forward_grouped", "qlin_gptq_workspace", "qlin_gptq_quantize",
 ]
 
 # test / measurement knobs (qlin_debug_set, include/qlin.h)
@@ -96,6 +97,10 @@ def lib() -> ctypes.CDLL:
             "qlin_backward_dx": [W, P, I32, P, P, P, SZ, P],
             "qlin_backward_dx_workspace": [I32, W, ctypes.POINTER(SZ)],
             "qlin_debug_set": [I32, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)],
+            "qlin_forward_grouped_workspace": [I32, P, I32, ctypes.POINTER(SZ)],
+            "qlin_forward_grouped": [I32, P, P, P, P, I32, F32, I32, P, SZ, P],
+            "qlin_gptq_workspace": [I32, I32, ctypes.POINTER(SZ)],
+            "qlin_gptq_quantize": [P, I32, I32, I32, P, P, I32, P, P, P, P, SZ, P],
             "qlin_debug_get": [I32, ctypes.POINTER(ctypes.c_int64)],
         }
         for name, argt in sigs.items():
@@ -201,6 +206,44 @@ def qlin_forward(X, M: int, w: qlin_weights, s, gamma: float, update_momentum: b
                  ws_bytes: int, stream=None):
     _check(lib().qlin_forward(_ptr(X), M, ctypes.byref(w), _ptr(s), float(gamma), int(bool(update_momentum)),
                               _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)), "qlin_forward")
+
+
+def _weights_array(ws):
+    arr = (ctypes.POINTER(qlin_weights) * len(ws))(*[ctypes.pointer(w) for w in ws])
+    return arr
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+
+
+def qlin_forward_grouped_workspace(ws, M: int) -> int:
+    arr = _weights_array(ws)
+    return _size(lib().qlin_forward_grouped_workspace, len(ws), ctypes.cast(arr, P), M)
+
+
+def qlin_forward_grouped(ws, Xs, ss, Ys, M: int, gamma: float, update_momentum: bool, workspace, ws_bytes: int,
+                         stream=None):
+    """Independent forwards of len(ws) layers at the same token count in one
+    quantization launch and one GEMM launch (C ABI qlin_forward_grouped)."""
+    n = len(ws)
+    assert len(Xs) == n and len(ss) == n and len(Ys) == n
+    arr = _weights_array(ws)
+    xa, sa, ya = _ptr_array(Xs), _ptr_array(ss), _ptr_array(Ys)
+    _check(lib().qlin_forward_grouped(n, ctypes.cast(arr, P), ctypes.cast(xa, P), ctypes.cast(sa, P),
+                                      ctypes.cast(ya, P), M, float(gamma), int(bool(update_momentum)),
+                                      _ptr(workspace), ws_bytes, _stream(stream)), "qlin_forward_grouped")
+
+
+def qlin_gptq_workspace(K: int, N: int) -> int:
+    return _size(lib().qlin_gptq_workspace, K, N)
+
+
+def qlin_gptq_quantize(X, ns: int, K: int, N: int, W, scale, qmax: int, codes, Hinv, singular, workspace,
+                       ws_bytes: int, stream=None):
+    _check(lib().qlin_gptq_quantize(_ptr(X), ns, K, N, _ptr(W), _ptr(scale), qmax, _ptr(codes), _ptr(Hinv),
+                                    _ptr(singular), _ptr(workspace), ws_bytes, _stream(stream)),
+           "qlin_gptq_quantize")
 
 
 def qlin_backward_dx_workspace(M: int, w: qlin_weights) -> int:

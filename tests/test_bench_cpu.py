@@ -14,7 +14,7 @@ KEYS = ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "
         "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"]
 
 
-@pytest.mark.parametrize("extra,unit", [([], "GB/s"), (["--op", "backward"], "TFLOP/s")])
+@pytest.mark.parametrize("extra,unit", [([], "TOPS"), (["--op", "backward"], "TFLOP/s")])
 def test_reference_arm_json_line(extra, unit):
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0", *extra],
                        cwd=ROOT, capture_output=True, text=True, timeout=600)
@@ -47,3 +47,31 @@ def test_algorithmic_bytes_by_hand():
     assert g == 8388608 + 16384 + 262144 + 335872 + 65536 + 64 + 656 + 131072
     g, _ = bench.algorithmic_bytes(16, 4096, 4096, 41, 2)
     assert g == 16777216 + 16384 + 335872 + 65536 + 64 + 656 + 131072
+
+
+def test_layer_bytes_by_hand():
+    """The fused layer's algorithmic bytes (no INT8 round trip between the
+    two kernels): X, packed weights with their scales and outlier rows, Y."""
+    sys.path.insert(0, ROOT)
+    import bench
+    # 70B up_proj at one token, g128, 82 outliers
+    K, N, nO = 8192, 28672, 82
+    want = 2 * K + K * N // 2 + 4 * N + 2 * (K // 128) * N + 2 * nO * N + 16 * nO + 2 * N
+    assert bench.layer_bytes(1, K, N, nO, 1) == want
+
+
+def test_roofline_bound_follows_arithmetic_intensity():
+    """Decode buckets are bound by HBM, prefill buckets by the INT8 tensor
+    peak (twice the measured bf16 figure); the fraction is the roofline time
+    over the measured time."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"hbm": 6551.0, "bf16": 1666.8, "bf16_sus": 1391.0, "kind": "measured"}
+    K, N, nO = 8192, 28672, 82
+    for M, bound in [(1, "hbm"), (16, "hbm"), (1024, "tensor"), (8192, "tensor")]:
+        ops, nb = 2 * M * K * N, bench.layer_bytes(M, K, N, nO, 1)
+        t_roof = max(nb / 6551e9, ops / (2 * 1666.8e12))
+        r = bench.roofline_of(ops, nb, 2 * t_roof, peaks)
+        assert r["bound"] == bound, M
+        assert abs(r["frac"] - 0.5) < 1e-9
+        assert r["peak"] == (6551.0 if bound == "hbm" else 2 * 1666.8)

@@ -8,8 +8,8 @@ sweep, with the knob set for the duration of the test only."""
 import pytest
 import torch
 
-from test_gpu_fullsize import test_split_k_accumulators_exact
-from test_gpu_parity import test_shapes, SHAPES
+from test_gpu_fullsize import test_split_k_accumulators_exact as _split_k_case
+from test_gpu_parity import test_shapes as _shape_case, SHAPES
 
 pytestmark = pytest.mark.gpu
 
@@ -35,10 +35,9 @@ def q():
 
 @pytest.mark.parametrize("mode", MODES, ids=lambda e: ",".join(f"{k}={v}" for k, v in e.items()))
 def test_forced_split_mode(q, oracle, mode):
-    from test_gpu_fullsize import TOL  # noqa: F401
     with q.knobs(**mode):
         for fmt in (0, 1, 2):
             for M in (1, 16, 48):
-                test_split_k_accumulators_exact(q, oracle, fmt, M)
+                _split_k_case(q, oracle, fmt, M)
         for args in SHAPES:
-            test_shapes(q, oracle, *args)
+            _shape_case(q, oracle, *args)

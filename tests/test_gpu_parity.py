@@ -140,6 +140,7 @@ SHAPE_MKN = [
     (64, 2048, 384, 0),     # no outliers: the plain QQQ path
     (200, 1152, 256, 41),   # BT = 256 with a ragged token tile
     (130, 4096, 128, 9),    # 32 K-steps: the stage ring wraps several times
+    (700, 512, 384, 17),    # 3 x 3 tiles of 256 tokens: token-tile-fastest raster order, ragged last token tile
 ]
 SHAPES = [(fmt, *mknO) for fmt in FMTS for mknO in SHAPE_MKN]
 

@@ -455,3 +455,26 @@ def test_int_gemm_row_forms_agree_with_numpy(oracle):
         acc_nk, _ = oracle.int_gemm_rows_nk(Xq, np.ascontiguousarray(B.T), rows)
         np.testing.assert_array_equal(acc_kn, want)
         np.testing.assert_array_equal(acc_nk, want)
+
+
+def test_gptq_layer_equals_row_by_row(oracle):
+    """The layer form of the Hessian compensation (one shared inverse and
+    downdate sequence) gives, column for column, exactly what the pinned
+    single-vector form gives, and codes * scale are the grid values."""
+    rng = np.random.default_rng(9)
+    ns, d, N, qmax = 40, 24, 7, 7
+    X = rng.standard_normal((ns, d))
+    W = rng.standard_normal((d, N)) * 0.1
+    scale = np.abs(W).max(axis=0) / qmax
+    Wq, codes, Hinv = oracle.gptq_quantize_layer(X, W, scale, qmax)
+    for n in range(N):
+        w_row, Hinv_row, _ = oracle.gptq_quantize(X, W[:, n], float(scale[n]), qmax)
+        np.testing.assert_array_equal(Wq[:, n], w_row)
+        np.testing.assert_array_equal(Hinv, Hinv_row)
+    np.testing.assert_array_equal(codes.astype(np.float64) * scale[None, :], Wq)
+    assert np.abs(codes).max() <= qmax
+    # the compensation lowers the layer's output error against plain rounding
+    plain = np.clip(np.rint(W / scale), -qmax, qmax) * scale
+    err_gptq = np.linalg.norm(X @ (Wq - W))
+    err_plain = np.linalg.norm(X @ (plain - W))
+    assert err_gptq < err_plain
