@@ -64,7 +64,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense INT8 : bf16 tensor rate of B200 (4.5 : 2.25 PFLOP/s)
 DEFAULT_WORKLOAD = "llama70b_w4g128"
-DEFAULT_EXTRAS = "llama7b_w4_decode,llama7b_w4g128_prefill,phi3_w8_quaff,backward,gptq"
+DEFAULT_EXTRAS = "llama7b_w4_decode,llama7b_w4g128_prefill,phi3_w8_quaff,backward,gptq,smooth_search"
 
 
 # ---------------------------------------------------------------------------
@@ -780,6 +780,50 @@ def gptq_record(device, stream, peaks, K=4096, N=4096, ns=8192, reps=2):
             "timing": f"median of {reps} calls, CUDA events on the launch stream"}
 
 
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 148 SMs x 128 FP32 lanes x FMA x max SM clock
+
+
+def smooth_record(device, stream, peaks, M=512, G=10, reps=3):
+    """QQQ adaptive-smoothing threshold search on a 7B q_proj-shaped layer
+    (K = N = 4096, W4A8 per-channel) with 512 calibration tokens of the 7B
+    recipe (1% outlier channels x100), 10 thresholds.  Per candidate: the
+    smoothed tensors, the layer's packer, quantization and tcgen05 GEMM, the
+    fp32 reference product on the smoothed channels and the loss.  The
+    reference product (CUDA-core fp32 FMA) dominates: reported against the
+    FP32 FMA peak from the unit counts and the maximum clock."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    wl = synth.WORKLOADS["llama7b_w4_decode"]
+    L = synth.layer(wl, 0, M=M)
+    K, N = L["K"], L["N"]
+    X = torch.from_numpy(L["X"]).to(device)
+    W = torch.from_numpy(L["W"]).to(device)
+    loss = torch.zeros(G, dtype=torch.float64, device=device)
+    best = torch.zeros(1, dtype=torch.int32, device=device)
+    n = qlin.qlin_smooth_search_workspace(M, K, N, G)
+    ws = qlin.empty_workspace(n, device)
+    times = []
+    for r in range(reps + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        qlin.qlin_smooth_search(X, M, K, W, N, G, loss, best, None, ws, n, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if r:
+            times.append(e0.elapsed_time(e1))
+    qlin.qlin_poll_device_status(stream)
+    ms = statistics.median(times)
+    ref_flops = 2 * M * N * K * G
+    ach = ref_flops / (ms * 1e-3) / 1e12
+    return {"op": "smooth_search", "M": M, "K": K, "N": N, "candidates": G, "ms": ms, "best": int(best.item()),
+            "int8_ops": 2 * M * N * K * G,
+            "roofline": {"bound": "alu", "achieved": ach, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": ach / FP32_PEAK_TFLOPS,
+                         "peak_source": "148 SMs x 128 FP32 lanes x 2 (FMA) x 1.965 GHz (unit counts x max clock)",
+                         "note": "the whole call's time against the fp32 reference product's FLOPs"},
+            "timing": f"median of {reps} calls, CUDA events on the launch stream"}
+
+
 def backward_record(device, stream, reps, peaks):
     import torch  # noqa: F401
     wl = synth.WORKLOADS["phi3_w8_quaff"]
@@ -1013,6 +1057,8 @@ def run_forward(args, wl):
                         workloads[name] = backward_record(device, stream, reps, peaks)
                     elif name == "gptq":
                         workloads[name] = gptq_record(device, stream, peaks)
+                    elif name == "smooth_search":
+                        workloads[name] = smooth_record(device, stream, peaks)
                     else:
                         w2 = synth.WORKLOADS[name]
                         workloads[name] = measure_workload_record(w2, 4 if name == "llama7b_w4_decode" else 1,

@@ -333,6 +333,33 @@ QLIN_API qlin_status qlin_gptq_quantize(const double* X, int32_t ns, int32_t K, 
                                         const double* scale, int32_t qmax, int8_t* codes, double* Hinv,
                                         int32_t* singular, void* workspace, size_t ws_bytes, void* stream);
 
+/* QQQ adaptive smoothing, the threshold search (offline calibration; "QQQ:
+ * Quality Quattuor-Bit Quantization for Large Language Models", section 三
+ * 技术架构 -> 自适应平滑): only activation channels with significant
+ * outliers are smoothed, and the threshold sigma comes from a grid search
+ * over [0, max|X|] minimising the quantized product's error on those
+ * channels.  For j = 0 .. G-1, sigma_j = max|X| * j / G (fp32) and
+ *   T      = { t : max_m |X[m][t]| > sigma_j }
+ *   s_t    = sqrt(max_m |X[m][t]| / max_n |W[t][n]|) on T (1 if a maximum is 0)
+ *   Xh     = fp16(X / s), Wh = fp16(W * s) on T, 0 elsewhere
+ *   loss_j = sum_{m,n} (a_m (c_n / 16) acc[m][n] - sum_{t in T} X[m][t] W[t][n])^2
+ * where (Xq, a) = qlin_quant_act of Xh (no outliers), (q, c) = the W4A8
+ * per-channel packing of Wh and acc = Xq . 16 q exactly (qlin_gemm); the
+ * reference product is summed in fp32, the loss in fp64 (its summation
+ * order is not fixed: repeated calls may differ in the last bits).
+ *   X       device fp16 [M][K] calibration activations; W device fp16 [K][N].
+ *   loss    device fp64 [G], overwritten.
+ *   best    device int32 (may be NULL): the first j of least loss.
+ *   s_best  device fp32 [K] (may be NULL): s of that candidate, 1 off T.
+ *   workspace  qlin_smooth_search_workspace bytes, 256-byte aligned (no
+ *           zero-fill needed).
+ * Shapes: as the W4A8 per-channel layer (K % 32 == 0, N % 16 == 0), M >= 1,
+ * 1 <= G <= 64. */
+QLIN_API qlin_status qlin_smooth_search_workspace(int32_t M, int32_t K, int32_t N, int32_t G, size_t* bytes);
+QLIN_API qlin_status qlin_smooth_search(const uint16_t* X, int32_t M, int32_t K, const uint16_t* W, int32_t N,
+                                        int32_t G, double* loss, int32_t* best, float* s_best, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
 /* Test and measurement hooks.  The library reads no environment variables:
  * a process that wants a non-default work split, launch mode or wait limit
  * (the test suite forcing each split-K variant, a measurement isolating one
@@ -354,6 +381,10 @@ QLIN_API qlin_status qlin_gptq_quantize(const double* X, int32_t ns, int32_t K, 
  *                             weights are widened to INT8 once per call; 0: never.
  *   QLIN_KNOB_FUSED_MOMENTUM_MAX_M  16 (default): up to this token count the
  *                             momentum update runs inside the quantization kernel.
+ *   QLIN_KNOB_PAIR_MMA        1 (default): 256-token tiles with INT8 operands run
+ *                             on CTA pairs (one 256-row tensor-core operation
+ *                             per pair) when there is a full wave of 256 x 256
+ *                             tiles; 0: never; 2: whenever the operands allow.
  *   QLIN_KNOB_WAIT_NS         2000000000 (default): limit in ns of every
  *                             device-side pipeline wait, after which the kernel
  *                             gives up, sets the device error word and unwinds
@@ -374,7 +405,8 @@ typedef enum {
   QLIN_KNOB_MAX_TOKEN_TILE = 4,
   QLIN_KNOB_WIDEN_MIN_M = 5,
   QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6,
-  QLIN_KNOB_WAIT_NS = 7
+  QLIN_KNOB_WAIT_NS = 7,
+  QLIN_KNOB_PAIR_MMA = 8
 } qlin_knob;
 
 QLIN_API qlin_status qlin_debug_set(int32_t knob, int64_t value, int64_t* previous);

@@ -1,0 +1,314 @@
+// gemm_pair.cuh -- stages 2 and 3 for many-token calls on two SMs at a time.
+//
+// The INT8 contraction of a 256-channel x 256-token tile is one tensor-core
+// operation of 256 rows shared by a pair of CTAs (a 2-CTA cluster,
+// tcgen05 cta_group::2): each CTA loads its own 128 weight rows and its own
+// 128 tokens of every K-block into its shared memory, the even CTA issues
+// tcgen05.mma.cta_group::2 over both halves, and each CTA's tensor memory
+// receives the accumulator of its 128 channels for all 256 tokens.  Per SM
+// and K-block that is 16 KB of weights and 16 KB of activations (against
+// 16 + 32 KB when one CTA computes a 128 x 256 tile alone), which is what
+// bounds the single-CTA kernel on many-token calls: the operand stream from
+// L2 into each SM.  No load is multicast: every CTA loads its own halves.
+//
+// Operands are INT8: the INT8 weight format, or INT4 weights widened once
+// per call (16 q per-channel, q8 for g128; gemm.cuh).  The compensation of
+// the outlier channels (the Quaff term X_hat[:,O] (s_O - 1) W_O) runs
+// after the K-blocks of a tile as kind::f16 pair operations of W_O^T x U
+// (hi and lo passes) into a second accumulator; the epilogue computes
+// Y = fp16(a_m (c'_n acc + comp)) exactly as the single-CTA kernel does.
+//
+// Roles per CTA (both CTAs of a pair run all of them, the MMA only in the
+// even CTA):
+//   warp 0        producer: per step one TMA load of the weight (or W_O^T)
+//                 block rows and one of the activation (or U) rows, both
+//                 counted on the even CTA's full barrier; waits for its own
+//                 empty barrier (released by the pair's MMA commit).
+//   warp 1        tensor memory allocation (both CTAs, cta_group::2); in the
+//                 even CTA one lane issues the pair MMAs and commits.
+//   warps 2..9    epilogue, two groups of four warps taking alternate
+//                 16-token chunks of the CTA's 128 x 256 accumulator; each
+//                 warp then arrives on the even CTA's accumulator-empty
+//                 barrier.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace qlin {
+
+constexpr int kPairStages = 6;
+constexpr int kPairStage = 32768;  // per CTA and step: 16 KB weight rows + 16 KB token rows
+constexpr int kPairYStage = 16 * 128 * 2;
+constexpr int kPairOffY = kPairStages * kPairStage;
+constexpr int kPairOffBar = kPairOffY + 4 * kPairYStage;
+constexpr int kPairOffSa = kPairOffBar + 1024;
+constexpr int kPairSmem = kPairOffSa + 2048 + 1024;  // + alignment slack
+constexpr int kPairThreads = 32 * (2 + 8);
+constexpr int kPairEpiWarps = 8;
+
+struct PairArgs {
+  const float* cscale;
+  float cmul;         // factor on c_n (1, or 1/16 for per-channel INT4 widened to 16 q)
+  const float* a;
+  uint16_t* Y;
+  int32_t* acc_debug;
+  int M, N, nO;
+  int kb;             // 128-wide K-blocks
+  int ntn;            // 128-channel tiles of the weights
+  int ncs;            // 64-wide outlier slices
+  int T;              // steps per tile: kb + 2 ncs
+  int tiles_n2;       // 256-channel pair tiles
+  int tiles_m;        // 256-token tiles
+  int gm;             // raster group of token tiles
+  int tiles;          // tiles_n2 * tiles_m
+  int ncl;            // clusters (pairs) in the grid
+};
+
+struct alignas(64) PairParams {
+  CUtensorMap tmA;   // weight blocks as rows of 128 bytes: [ntn * kb * 128][128]
+  CUtensorMap tmX;   // Xq int8 [M][K], 128 x 128 boxes, 128-byte swizzle
+  CUtensorMap tmU;   // U fp16 [2M][nOp], 64 x 128 boxes, 128-byte swizzle
+  CUtensorMap tmWo;  // W_O^T blocks as rows of 128 bytes: [ntn * ncs * 128][128]
+  PairArgs g;
+};
+
+__device__ __forceinline__ void pair_tile_coords(const PairArgs& g, int t, int& tn2, int& tm) {
+  const int per = g.gm * g.tiles_n2;
+  const int grp = t / per;
+  const int w = t - grp * per;
+  const int g0 = grp * g.gm;
+  const int gs = g.tiles_m - g0 < g.gm ? g.tiles_m - g0 : g.gm;
+  tm = g0 + w % gs;
+  tn2 = w / gs;
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid_constant__ PairParams prm) {
+  const PairArgs& g = prm.g;
+  constexpr int S = kPairStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairOffBar);  // [S] (the even CTA's are used)
+  uint64_t* empty = full + S;                                         // [S] (each CTA's own)
+  uint64_t* acc_full = empty + S;                                     // each CTA's own
+  uint64_t* acc_empty = acc_full + 1;                                 // the even CTA's
+  uint64_t* mma_done = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int crk = static_cast<int>(cluster_ctarank());
+  const int cid = static_cast<int>(cluster_id_x());
+  const bool leader = crk == 0;
+  const bool comp = g.nO > 0;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * kPairEpiWarps);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 1) {
+    tma_prefetch_desc(&prm.tmA);
+    tma_prefetch_desc(&prm.tmX);
+    if (comp) {
+      tma_prefetch_desc(&prm.tmU);
+      tma_prefetch_desc(&prm.tmWo);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync_all();  // both CTAs' barriers exist before either touches the other's
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      griddep_wait();  // Xq, U and widened weights come from the previous kernels
+      const uint32_t lfull0 = mapa_shared(smem_u32(&full[0]), 0);
+      int gi = 0;
+      bool ok = true;
+      for (int t = cid; ok && t < g.tiles; t += g.ncl) {
+        int tn2, tm;
+        pair_tile_coords(g, t, tn2, tm);
+        const int ctile = 2 * tn2 + crk;    // this CTA's 128 channels
+        const int m0 = tm * 256 + crk * 128;  // this CTA's 128 tokens
+        for (int r = 0; r < g.T; ++r, ++gi) {
+          const int s = gi % S;
+          if (gi >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2u * kPairStage);
+          unsigned char* A = smem + s * kPairStage;
+          unsigned char* X = A + 16384;
+          const uint32_t lb = lfull0 + static_cast<uint32_t>(8 * s);
+          if (r < g.kb) {
+            tma_load_2d_pair(A, &prm.tmA, lb, 0, (ctile * g.kb + r) * 128);
+            tma_load_2d_pair(X, &prm.tmX, lb, r * 128, m0);
+          } else {
+            const int j = r - g.kb;
+            const int lo = j >= g.ncs ? 1 : 0;  // U rows [0, M) hold hi, [M, 2M) hold lo
+            const int ib = j - lo * g.ncs;
+            tma_load_2d_pair(A, &prm.tmWo, lb, 0, (ctile * g.ncs + ib) * 128);
+            tma_load_2d_pair(X, &prm.tmU, lb, ib * 64, lo * g.M + m0);
+          }
+        }
+      }
+      // every stage this CTA filled has been consumed by the pair's MMAs (so
+      // its copies have landed) before the CTA can leave
+      for (int t = gi - 1; t >= 0 && t >= gi - S; --t) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(&empty[t % S], static_cast<uint32_t>(t / S) & 1u, 1000000u) &&
+               globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ pair MMA (even CTA)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc_main = idesc_s8_s32(256, 256);
+      constexpr uint32_t idesc_comp = idesc_f16_f32(256, 256);
+      const uint64_t adesc0 = sdesc_k_sw128(smem_u32(smem));
+      const uint64_t bdesc0 = sdesc_k_sw128(smem_u32(smem + 16384));
+      int gi = 0, ti = 0;
+      bool ok = true, issued = false;
+      for (int t = cid; ok && t < g.tiles; t += g.ncl, ++ti) {
+        if (ti > 0 && !mbar_wait_cluster(acc_empty, static_cast<uint32_t>(ti - 1) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int r = 0; r < g.T; ++r, ++gi) {
+          const int s = gi % S;
+          if (!mbar_wait(&full[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issued = true;
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kPairStage >> 4));
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (kPairStage >> 4));
+          if (r < g.kb) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_i8_pair(tmem, ad + 2 * k, bd + 2 * k, idesc_main, (r > 0 || k > 0) ? 1u : 0u);
+          } else {
+            const int j = r - g.kb;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma_f16_pair(tmem + 256, ad + 2 * k, bd + 2 * k, idesc_comp, (j > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[s], 0x3);
+        }
+        if (!ok) break;
+        mma_commit_pair(acc_full, 0x3);
+      }
+      // every pair MMA has completed before tensor memory can be freed
+      if (issued) {
+        mma_commit_pair(mma_done, 0x1);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait_sleep(mma_done, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ep = warp - 2;
+    const int grp = ep >> 2;
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. +31
+    const int nl = quad * 32 + lane;
+    const int gbar = 1 + grp;
+    float* sa_t = reinterpret_cast<float*>(smem + kPairOffSa + grp * 1024);
+    const uint32_t lempty = mapa_shared(smem_u32(acc_empty), 0);
+    griddep_wait();  // a[] comes from the previous kernel
+    int ycnt = 0, ti = 0;
+    for (int t = cid; t < g.tiles; t += g.ncl, ++ti) {
+      int tn2, tm;
+      pair_tile_coords(g, t, tn2, tm);
+      const int ctile = 2 * tn2 + crk;
+      const int n = ctile * 128 + nl;
+      const int m0 = tm * 256;
+      const int mvalid = min(256, g.M - m0);
+      float cn = 0.f;
+      if (n < g.N) cn = __fmul_rn(g.cscale[n], g.cmul);
+      bool ok = mbar_wait(acc_full, static_cast<uint32_t>(ti) & 1u, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      named_bar_sync(gbar, 128);
+      for (int j = nl; j < 256; j += 128) sa_t[j] = j < mvalid ? g.a[m0 + j] : 0.f;
+      named_bar_sync(gbar, 128);
+      const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 16) {
+        if (c0 >= mvalid) break;
+        if (((c0 >> 4) & 1) != grp) continue;
+        uint32_t acc[16], cmp[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) { acc[j] = 0u; cmp[j] = 0u; }
+        if (ok) {
+          tmem_ld16(trow + c0, acc);
+          if (comp) tmem_ld16(trow + 256 + c0, cmp);
+          tmem_ld_wait();
+        }
+        const int b = ycnt & 1;
+        uint16_t* ys = reinterpret_cast<uint16_t*>(smem + kPairOffY + (grp * 2 + b) * kPairYStage);
+        float sc[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float4 v = *reinterpret_cast<const float4*>(sa_t + c0 + 4 * q4);
+          sc[4 * q4] = v.x; sc[4 * q4 + 1] = v.y; sc[4 * q4 + 2] = v.z; sc[4 * q4 + 3] = v.w;
+        }
+        uint16_t yh[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float v = __fmul_rn(cn, static_cast<float>(static_cast<int32_t>(acc[j])));
+          if (comp) v = __fadd_rn(v, __uint_as_float(cmp[j]));
+          yh[j] = __half_as_ushort(__float2half_rn(__fmul_rn(sc[j], v)));
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ys[j * 128 + nl] = yh[j];
+        if (g.acc_debug && n < g.N)
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < mvalid) g.acc_debug[static_cast<size_t>(m0 + c0 + j) * g.N + n] = static_cast<int32_t>(acc[j]);
+        named_bar_sync(gbar, 128);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int idx = nl + h * 128;  // 16 rows x 16 segments of 8 channels
+          const int j = idx >> 4;
+          const int n8 = ctile * 128 + (idx & 15) * 8;
+          if (c0 + j < mvalid && n8 < g.N)
+            *reinterpret_cast<uint4*>(g.Y + static_cast<size_t>(m0 + c0 + j) * g.N + n8) =
+                *reinterpret_cast<const uint4*>(ys + j * 128 + (idx & 15) * 8);
+        }
+        ++ycnt;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader) mbar_arrive(acc_empty);
+        else mbar_arrive_remote(lempty);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its pair may still signal or read it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+}  // namespace qlin

@@ -15,9 +15,11 @@
 #include "qlin.h"
 #include "act_quant.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "backward.cuh"
 #include "gptq.cuh"
 #include "pack.cuh"
+#include "smooth.cuh"
 
 using namespace qlin;
 
@@ -138,7 +140,7 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 // each may start its prologue (and the GEMM its weight stream) while the
 // previous kernel in the stream finishes; every kernel waits on the grid
 // dependency before it reads what the previous one wrote.
-std::atomic<long long> g_knob[8] = {{1}, {1}, {0}, {0}, {256}, {1024}, {kFusedMomentumMaxM}, {2000000000LL}};
+std::atomic<long long> g_knob[9] = {{1}, {1}, {0}, {0}, {256}, {1024}, {kFusedMomentumMaxM}, {2000000000LL}, {1}};
 
 long long knob(int k) { return g_knob[k].load(std::memory_order_relaxed); }
 
@@ -410,6 +412,98 @@ qlin_status launch_gemm_fmt(int bt, GemmParams<MAXP>& prm, cudaStream_t stream) 
   }
 }
 
+// ---------------------------------------------------------------- CTA-pair GEMM (many tokens)
+int pair_max_clusters() {
+  static int n = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+      return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * ((sm_count() + 1) / 2)));
+    cfg.blockDim = dim3(kPairThreads);
+    cfg.dynamicSmemBytes = kPairSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      c = 0;
+    }
+    n = c;
+  });
+  return n;
+}
+
+// Whether a single-problem launch runs on CTA pairs: 256-token tiles with
+// INT8 operands (the INT8 format, or INT4 widened once per call) and at
+// least one full wave of 256 x 256 pair tiles (QLIN_KNOB_PAIR_MMA: 0 never,
+// 2 whenever the operands allow).
+bool use_pair(const GemmPlan& p, const qlin_weights* w) {
+  const long long mode = knob(QLIN_KNOB_PAIR_MMA);
+  if (mode == 0 || p.nprob != 1 || p.bt != 256) return false;
+  if (!(w->fmt == QLIN_W8_PERCHANNEL || p.widen)) return false;
+  const int ncl = pair_max_clusters();
+  if (ncl < 1) return false;
+  const long long tiles = static_cast<long long>((p.pr[0].tiles_n + 1) / 2) * p.pr[0].tiles_m;
+  return mode == 2 ? tiles >= 1 : tiles >= ncl;
+}
+
+qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int8_t* Xq, const float* a, uint16_t* Y,
+                             int32_t* acc_debug, char* gws, const uint8_t* codes8, float cmul, cudaStream_t stream) {
+  PairParams prm;
+  memset(&prm, 0, sizeof(prm));
+  PairArgs& g = prm.g;
+  const GemmProb& q = p.pr[0];
+  const int M = q.M;
+  g.cscale = w->chan_scale;
+  g.cmul = cmul;
+  g.a = a;
+  g.Y = Y;
+  g.acc_debug = acc_debug;
+  g.M = M;
+  g.N = w->N;
+  g.nO = w->n_outlier;
+  g.kb = q.kb;
+  g.ntn = q.tiles_n;
+  g.ncs = q.ncs;
+  g.T = q.kb + 2 * q.ncs;
+  g.tiles_n2 = (q.tiles_n + 1) / 2;
+  g.tiles_m = q.tiles_m;
+  g.tiles = g.tiles_n2 * g.tiles_m;
+  const double x_bytes = static_cast<double>(M) * w->K;
+  int gm = static_cast<int>(std::lround(std::sqrt(static_cast<double>(pair_max_clusters()) * 256.0 / 256.0)));
+  if (x_bytes <= 48.0 * 1024 * 1024) gm = g.tiles_m;
+  g.gm = gm < 1 ? 1 : (gm > g.tiles_m ? g.tiles_m : gm);
+  const int maxc = pair_max_clusters();
+  g.ncl = g.tiles < maxc ? g.tiles : maxc;
+  qlin_status st = make_map(&prm.tmA, codes8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128,
+                            static_cast<uint64_t>(q.tiles_n) * q.kb * 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != QLIN_OK) return st;
+  st = make_map(&prm.tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K, M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLIN_OK) return st;
+  if (w->n_outlier > 0) {
+    st = make_map(&prm.tmU, gws + p.u_off[0], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->n_outlier_pad,
+                  2 * static_cast<uint64_t>(M), 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != QLIN_OK) return st;
+    st = make_map(&prm.tmWo, w->W_Ot, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128,
+                  static_cast<uint64_t>(q.tiles_n) * q.ncs * 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != QLIN_OK) return st;
+  }
+  cudaError_t e = launch_kc(gemm_pair_kernel, dim3(static_cast<unsigned>(2 * g.ncl)), dim3(kPairThreads), kPairSmem,
+                            stream, 2, prm);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_pair_kernel launch failed: %s", cudaGetErrorString(e));
+  return QLIN_OK;
+}
+
 // One GEMM launch over the problems of a plan.  Per problem q: weights
 // ws[q], the INT8 activations Xq[q], token scales a[q], output Y[q] and
 // (optional) acc_debug[q]; `gws` is the scratch laid out by the plan (each
@@ -474,8 +568,14 @@ qlin_status launch_gemm_group(const GemmPlan& p, const qlin_weights* const* ws, 
     if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "widen_w4_kernel launch failed: %s", cudaGetErrorString(e));
     prm.pr[0].codes = w8;
     prm.pr[0].cmul = fmt == QLIN_W4_PERCHANNEL ? 0.0625f : 1.f;
+    if (MAXP == 1 && use_pair(p, w))
+      return launch_gemm_pair(p, w, Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws, w8, prm.pr[0].cmul,
+                              stream);
     return launch_gemm_fmt<kFmtW8, MAXP>(p.bt, prm, stream);
   }
+  if (MAXP == 1 && fmt == QLIN_W8_PERCHANNEL && use_pair(p, ws[0]))
+    return launch_gemm_pair(p, ws[0], Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws,
+                            static_cast<const uint8_t*>(ws[0]->codes), 1.f, stream);
   switch (fmt) {
     case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC, MAXP>(p.bt, prm, stream);
     case QLIN_W4_G128: return launch_gemm_fmt<kFmtW4G128, MAXP>(p.bt, prm, stream);
@@ -1206,14 +1306,114 @@ qlin_status qlin_gptq_quantize(const double* X, int32_t ns, int32_t K, int32_t N
   return QLIN_OK;
 }
 
+namespace {
+struct SmoothLayout {
+  size_t cmax, wmax, xall, sv, xh, wh, packed, xq, a, gemm, y, acc, ref, total;
+  Layout wl;
+};
+SmoothLayout smooth_layout(int M, int K, int N) {
+  SmoothLayout L{};
+  size_t off = 0;
+  L.cmax = off; off = round_up(off + size_t(K) * 4, kAlign);
+  L.wmax = off; off = round_up(off + size_t(K) * 4, kAlign);
+  L.xall = off; off = round_up(off + 16, kAlign);
+  L.sv = off; off = round_up(off + size_t(K) * 4, kAlign);
+  L.xh = off; off = round_up(off + size_t(M) * K * 2, kAlign);
+  L.wh = off; off = round_up(off + size_t(K) * N * 2, kAlign);
+  L.wl = weights_layout(K, N, QLIN_W4_PERCHANNEL, 0);
+  L.packed = off; off = round_up(off + L.wl.total, kAlign);
+  L.xq = off; off = round_up(off + size_t(M) * K, kAlign);
+  L.a = off; off = round_up(off + size_t(M) * 4, kAlign);
+  qlin_weights w{};
+  w.K = K; w.N = N; w.fmt = QLIN_W4_PERCHANNEL; w.n_outlier = 0; w.n_outlier_pad = 0;
+  L.gemm = off; off = round_up(off + gemm_ws_bytes(M, &w), kAlign);
+  L.y = off; off = round_up(off + size_t(M) * N * 2, kAlign);
+  L.acc = off; off = round_up(off + size_t(M) * N * 4, kAlign);
+  L.ref = off; off = round_up(off + size_t(M) * N * 4, kAlign);
+  L.total = off;
+  return L;
+}
+qlin_status check_smooth(int32_t M, int32_t K, int32_t N, int32_t G) {
+  if (M < 1 || G < 1 || G > 64) return fail(QLIN_ERR_ARG, "M=%d must be >= 1 and G=%d in [1, 64]", M, G);
+  return check_shape(K, N, QLIN_W4_PERCHANNEL, 0);
+}
+}  // namespace
+
+qlin_status qlin_smooth_search_workspace(int32_t M, int32_t K, int32_t N, int32_t G, size_t* bytes) {
+  qlin_status st = check_smooth(M, K, N, G);
+  if (st != QLIN_OK) return st;
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  *bytes = smooth_layout(M, K, N).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_smooth_search(const uint16_t* X, int32_t M, int32_t K, const uint16_t* W, int32_t N, int32_t G,
+                               double* loss, int32_t* best, float* s_best, void* workspace, size_t ws_bytes,
+                               void* stream_) {
+  qlin_status st = check_smooth(M, K, N, G);
+  if (st != QLIN_OK) return st;
+  if (!X || !W || !loss || !workspace) return fail(QLIN_ERR_ARG, "X/W/loss/workspace is NULL");
+  if (!aligned16(X) || !aligned16(W) || (reinterpret_cast<uintptr_t>(loss) & 7u) ||
+      (s_best && (reinterpret_cast<uintptr_t>(s_best) & 3u)) || (best && (reinterpret_cast<uintptr_t>(best) & 3u)))
+    return fail(QLIN_ERR_ALIGN, "X/W must be 16-byte aligned, loss 8, best and s_best 4");
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const SmoothLayout L = smooth_layout(M, K, N);
+  if (ws_bytes < L.total) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, L.total);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  char* ws = static_cast<char*>(workspace);
+  unsigned* cmax = reinterpret_cast<unsigned*>(ws + L.cmax);
+  float* wmax = reinterpret_cast<float*>(ws + L.wmax);
+  float* xall = reinterpret_cast<float*>(ws + L.xall);
+  float* sv = reinterpret_cast<float*>(ws + L.sv);
+  uint16_t* Xh = reinterpret_cast<uint16_t*>(ws + L.xh);
+  uint16_t* Wh = reinterpret_cast<uint16_t*>(ws + L.wh);
+  int8_t* Xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* a = reinterpret_cast<float*>(ws + L.a);
+  uint16_t* Y = reinterpret_cast<uint16_t*>(ws + L.y);
+  int32_t* acc = reinterpret_cast<int32_t*>(ws + L.acc);
+  float* ref = reinterpret_cast<float*>(ws + L.ref);
+  qlin_weights w{};
+  st = qlin_weights_bind(&w, K, N, QLIN_W4_PERCHANNEL, 0, ws + L.packed, L.wl.total);
+  if (st != QLIN_OK) return st;
+  QLIN_CUDA_TRY(cudaMemsetAsync(cmax, 0, size_t(K) * 4, stream));
+  QLIN_CUDA_TRY(cudaMemsetAsync(ws + L.gemm, 0, L.y - L.gemm, stream));  // split-K counters start at zero
+  QLIN_CUDA_TRY(cudaMemsetAsync(loss, 0, size_t(G) * 8, stream));
+  smooth_colmax_kernel<<<dim3((K + 255) / 256, (M + 63) / 64), 256, 0, stream>>>(X, M, K, cmax);
+  smooth_rowmax_kernel<<<K, 256, 0, stream>>>(W, N, wmax);
+  smooth_allmax_kernel<<<1, 1024, 0, stream>>>(cmax, K, xall);
+  QLIN_LAUNCH_CHECK("smoothing maxima");
+  const size_t mk = size_t(M) * K, kn = size_t(K) * N, mn = size_t(M) * N;
+  for (int j = 0; j < G; ++j) {
+    smooth_factors_kernel<<<(K + 255) / 256, 256, 0, stream>>>(cmax, wmax, xall, K, j, G, sv);
+    smooth_apply_x_kernel<<<static_cast<unsigned>((mk + 255) / 256), 256, 0, stream>>>(X, sv, M, K, Xh);
+    smooth_apply_w_kernel<<<static_cast<unsigned>((kn + 255) / 256), 256, 0, stream>>>(W, sv, K, N, Wh);
+    QLIN_LAUNCH_CHECK("smoothing kernels");
+    // the layer's quantizers and integer product on the smoothed tensors
+    st = qlin_pack_weights(Wh, nullptr, &w, stream);
+    if (st != QLIN_OK) return st;
+    st = launch_quant(Xh, M, &w, nullptr, 0.f, 0, Xq, a, nullptr, nullptr, nullptr, stream);
+    if (st != QLIN_OK) return st;
+    st = launch_gemm(&w, Xq, a, M, Y, acc, ws + L.gemm, stream);
+    if (st != QLIN_OK) return st;
+    smooth_ref_kernel<<<dim3((N + 63) / 64, (M + 63) / 64), 256, 0, stream>>>(X, W, sv, M, K, N, ref);
+    smooth_loss_kernel<<<static_cast<unsigned>((mn + 255) / 256), 256, 0, stream>>>(acc, a, w.chan_scale, ref, M,
+                                                                                    N, loss + j);
+    QLIN_LAUNCH_CHECK("smoothing loss");
+  }
+  smooth_pick_kernel<<<1, 256, 0, stream>>>(loss, G, cmax, wmax, xall, K, best, s_best);
+  QLIN_LAUNCH_CHECK("smooth_pick_kernel");
+  return QLIN_OK;
+}
+
 qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
-  if (k < 0 || k > QLIN_KNOB_WAIT_NS) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
+  if (k < 0 || k > QLIN_KNOB_PAIR_MMA) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
   bool ok = true;
   switch (k) {
     case QLIN_KNOB_PDL:
     case QLIN_KNOB_CLUSTER: ok = value == 0 || value == 1; break;
     case QLIN_KNOB_CLUSTER_SIZE: ok = value == 0 || value == 2 || value == 4 || value == 8; break;
     case QLIN_KNOB_MAX_TOKEN_TILE: ok = value == 64 || value == 128 || value == 256; break;
+    case QLIN_KNOB_PAIR_MMA: ok = value >= 0 && value <= 2; break;
     default: ok = value >= 0;
   }
   if (!ok) return fail(QLIN_ERR_ARG, "invalid value %lld for knob %d", static_cast<long long>(value), k);
@@ -1227,7 +1427,7 @@ qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
 }
 
 qlin_status qlin_debug_get(int32_t k, int64_t* value) {
-  if (k < 0 || k > QLIN_KNOB_WAIT_NS || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
+  if (k < 0 || k > QLIN_KNOB_PAIR_MMA || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
   *value = g_knob[k].load();
   return QLIN_OK;
 }

@@ -30,7 +30,8 @@ EXPORTED = [
     "qlin_momentum_update", "qlin_gemm_workspace", "qlin_gemm", "qlin_forward_workspace",
     "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc", "qlin_backward_dx",
     "qlin_backward_dx_workspace", "qlin_debug_set", "qlin_debug_get", "qlin_forward_grouped_workspace",
-    "qlin_forward_grouped", "qlin_gptq_workspace", "qlin_gptq_quantize",
+    "qlin_forward_grouped", "qlin_gptq_workspace", "qlin_gptq_quantize", "qlin_smooth_search_workspace",
+    "qlin_smooth_search",
 ]
 
 # test / measurement knobs (qlin_debug_set, include/qlin.h)
@@ -42,6 +43,7 @@ QLIN_KNOB_MAX_TOKEN_TILE = 4
 QLIN_KNOB_WIDEN_MIN_M = 5
 QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6
 QLIN_KNOB_WAIT_NS = 7
+QLIN_KNOB_PAIR_MMA = 8
 
 
 class QlinError(RuntimeError):
@@ -101,6 +103,8 @@ def lib() -> ctypes.CDLL:
             "qlin_forward_grouped": [I32, P, P, P, P, I32, F32, I32, P, SZ, P],
             "qlin_gptq_workspace": [I32, I32, ctypes.POINTER(SZ)],
             "qlin_gptq_quantize": [P, I32, I32, I32, P, P, I32, P, P, P, P, SZ, P],
+            "qlin_smooth_search_workspace": [I32, I32, I32, I32, ctypes.POINTER(SZ)],
+            "qlin_smooth_search": [P, I32, I32, P, I32, I32, P, P, P, P, SZ, P],
             "qlin_debug_get": [I32, ctypes.POINTER(ctypes.c_int64)],
         }
         for name, argt in sigs.items():
@@ -244,6 +248,16 @@ def qlin_gptq_quantize(X, ns: int, K: int, N: int, W, scale, qmax: int, codes, H
     _check(lib().qlin_gptq_quantize(_ptr(X), ns, K, N, _ptr(W), _ptr(scale), qmax, _ptr(codes), _ptr(Hinv),
                                     _ptr(singular), _ptr(workspace), ws_bytes, _stream(stream)),
            "qlin_gptq_quantize")
+
+
+def qlin_smooth_search_workspace(M: int, K: int, N: int, G: int) -> int:
+    return _size(lib().qlin_smooth_search_workspace, M, K, N, G)
+
+
+def qlin_smooth_search(X, M: int, K: int, W, N: int, G: int, loss, best, s_best, workspace, ws_bytes: int,
+                       stream=None):
+    _check(lib().qlin_smooth_search(_ptr(X), M, K, _ptr(W), N, G, _ptr(loss), _ptr(best), _ptr(s_best),
+                                    _ptr(workspace), ws_bytes, _stream(stream)), "qlin_smooth_search")
 
 
 def qlin_backward_dx_workspace(M: int, w: qlin_weights) -> int:

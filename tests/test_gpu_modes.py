@@ -1,7 +1,7 @@
 """The GEMM's work split is chosen per call (global stream-K, or cluster
 split-K with 2, 4 or 8 CTAs per tile), INT4 weights are widened ahead of
-the GEMM for large token counts, and kernels are chained with
-programmatic dependent launch.  The library's test knobs (qlin_debug_set)
+the GEMM for large token counts, many-token tiles run on CTA pairs, and
+kernels are chained with programmatic dependent launch.  The library's test knobs (qlin_debug_set)
 force each variant, so every one of them is checked against the oracle
 here: the exact INT32 accumulators of the split-K test and the ragged-shape
 sweep, with the knob set for the duration of the test only."""
@@ -21,6 +21,8 @@ MODES = [
     {"pdl": 0},                # plain stream-ordered launches
     {"widen_min_m": 129},      # INT4 weights widened once, INT8 kernel, from 129 tokens
     {"widen_min_m": 0},        # INT4 converters in the GEMM for every token count
+    {"pair_mma": 2, "widen_min_m": 129},  # CTA-pair GEMM for every 256-token tile with INT8 operands
+    {"pair_mma": 0},           # one CTA per tile everywhere
 ]
 
 

@@ -478,3 +478,53 @@ def test_gptq_layer_equals_row_by_row(oracle):
     err_gptq = np.linalg.norm(X @ (Wq - W))
     err_plain = np.linalg.norm(X @ (plain - W))
     assert err_gptq < err_plain
+
+
+def _smooth_case(M, K, N, seed):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    X[:, rng.choice(K, max(2, K // 50), replace=False)] *= rng.uniform(20, 80)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    return X.astype(np.float16), W.astype(np.float16)
+
+
+def test_smooth_search_composes_pinned_quantizers(oracle):
+    """Each candidate's loss equals the same steps assembled from the pinned
+    quantizers (per-token INT8, per-channel INT4), numpy's exact integer
+    matmul and an fp64 reference on the smoothed channel set; the search
+    returns the first least loss."""
+    X, W = _smooth_case(12, 64, 24, 3)
+    G = 6
+    loss, best = oracle.smooth_search(X.view(np.uint16), W.view(np.uint16), G)
+    assert best == int(np.argmin(loss)) and (loss >= 0).all()
+    x32, w32 = X.astype(np.float32), W.astype(np.float32)
+    cmax = np.abs(x32).max(axis=0)
+    wmax = np.abs(w32).max(axis=1)
+    xall = np.float32(cmax.max())
+    for j in range(G):
+        sigma = np.float32(np.float32(xall * np.float32(j)) / np.float32(G))
+        inT = cmax > sigma
+        s = np.where(inT & (cmax > 0) & (wmax > 0), np.sqrt(cmax / np.where(wmax > 0, wmax, 1)), np.float32(1))
+        s = s.astype(np.float32)
+        Xh = np.where(inT[None, :], x32 / s[None, :], 0).astype(np.float16)
+        Wh = np.where(inT[:, None], w32 * s[:, None], 0).astype(np.float16)
+        xq, a, _ = oracle.quant_act(Xh.view(np.uint16), np.zeros(0, np.int32), np.zeros(0, np.float32))
+        q, c = oracle.quant_weight_per_channel(Wh.view(np.uint16), 7)
+        acc = xq.astype(np.int64) @ (16 * q.astype(np.int64))
+        y = acc.astype(np.float64) * a.astype(np.float64)[:, None] * (c.astype(np.float64) / 16.0)[None, :]
+        ref = X.astype(np.float64)[:, inT] @ W.astype(np.float64)[inT, :]
+        want = float(((y - ref) ** 2).sum())
+        assert abs(loss[j] - want) <= 1e-12 * want, (j, loss[j], want)
+
+
+def test_smooth_search_channel_permutation_invariant(oracle):
+    """Relabelling the input channels (columns of X with the rows of W) does
+    not change any candidate's loss: a mixed-up index (a column maximum taken
+    over the wrong axis, a factor applied to the wrong channel) would."""
+    X, W = _smooth_case(10, 96, 16, 8)
+    perm = np.random.default_rng(1).permutation(96)
+    l1, b1 = oracle.smooth_search(X.view(np.uint16), W.view(np.uint16), 5)
+    l2, b2 = oracle.smooth_search(np.ascontiguousarray(X[:, perm]).view(np.uint16),
+                                  np.ascontiguousarray(W[perm, :]).view(np.uint16), 5)
+    np.testing.assert_allclose(l1, l2, rtol=1e-12)
+    assert b1 == b2
