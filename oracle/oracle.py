@@ -98,6 +98,16 @@ def _declare(L):
     L.oq_gptq_quantize_layer.restype = I
     L.oq_smooth_search.argtypes = [P, I, I, P, I, I, P]
     L.oq_smooth_search.restype = I
+    L.oq_offq_transform.argtypes = [P, I, I, P, P]
+    L.oq_offq_transform.restype = None
+    L.oq_offq_quant_act.argtypes = [P, I, I, P, P, P, P]
+    L.oq_offq_quant_act.restype = None
+    L.oq_offq_rotate_weights.argtypes = [P, I, I, P, P]
+    L.oq_offq_rotate_weights.restype = None
+    L.oq_quant_weight_per_channel_f32.argtypes = [P, I, I, I, P, P]
+    L.oq_quant_weight_per_channel_f32.restype = None
+    L.oq_offq_gemm_rows.argtypes = [P, P, P, P, P, I, I, P, I, P]
+    L.oq_offq_gemm_rows.restype = None
     L.oq_invert.argtypes = [P, I, P]
     L.oq_invert.restype = I
 
@@ -335,6 +345,55 @@ def smooth_search(X_bits: np.ndarray, W_bits: np.ndarray, G: int):
     loss = np.zeros(G, np.float64)
     best = lib().oq_smooth_search(_p(X_bits), M, K, _p(W_bits), N, int(G), _p(loss))
     return loss, int(best)
+
+
+def offq_transform(X_bits: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """y = x (D H) per 128-channel group, fp64 [M][K] (unnormalised)."""
+    X_bits = _c(X_bits, np.uint16)
+    M, K = X_bits.shape
+    y = np.zeros((M, K), np.float64)
+    lib().oq_offq_transform(_p(X_bits), M, K, _p(_c(signs, np.int8)), _p(y))
+    return y
+
+
+def offq_quant_act(X_bits: np.ndarray, signs: np.ndarray):
+    """OffQ activations: (q int8 [M][K] in 0..15, scale fp32 [M][K/128], offset fp32 [M][K/128]);
+    the dequantized value is q * scale + offset."""
+    X_bits = _c(X_bits, np.uint16)
+    M, K = X_bits.shape
+    G = K // 128
+    Xq = np.zeros((M, K), np.int8)
+    sc = np.zeros((M, G), np.float32)
+    off = np.zeros((M, G), np.float32)
+    lib().oq_offq_quant_act(_p(X_bits), M, K, _p(_c(signs, np.int8)), _p(Xq), _p(sc), _p(off))
+    return Xq, sc, off
+
+
+def offq_pack_layer(W_bits: np.ndarray, signs: np.ndarray) -> dict:
+    """OffQ weights: W' = (1/128) H D W per group (fp32), then per-channel INT4."""
+    W_bits = _c(W_bits, np.uint16)
+    K, N = W_bits.shape
+    Wr = np.zeros((K, N), np.float32)
+    lib().oq_offq_rotate_weights(_p(W_bits), K, N, _p(_c(signs, np.int8)), _p(Wr))
+    q = np.zeros((K, N), np.int8)
+    c = np.zeros(N, np.float32)
+    lib().oq_quant_weight_per_channel_f32(_p(Wr), K, N, 7, _p(q), _p(c))
+    B = (q.astype(np.int16) * 16).astype(np.int8)
+    return {"K": K, "N": N, "Wr": Wr, "q": q, "c": c, "B": B, "Bt": np.ascontiguousarray(B.T),
+            "cscale": (c / np.float32(16.0)).astype(np.float32), "packed": pack_nibbles(q)}
+
+
+def offq_gemm_rows(Xq: np.ndarray, scale: np.ndarray, offset: np.ndarray, packed: dict,
+                   rows: np.ndarray) -> np.ndarray:
+    Xq = _c(Xq, np.int8)
+    scale = _c(scale, np.float32)
+    offset = _c(offset, np.float32)
+    rows = _c(rows, np.int32)
+    K, N = packed["K"], packed["N"]
+    y = np.zeros((len(rows), N), np.float64)
+    lib().oq_offq_gemm_rows(_p(Xq), _p(scale), _p(offset), _p(packed["Bt"]), _p(_c(packed["cscale"], np.float32)),
+                            K, N, _p(rows), len(rows), _p(y))
+    return y
 
 
 # --- whole layer, composed from the steps above ------------------------------

@@ -689,6 +689,118 @@ OQ_EXPORT int oq_smooth_search(const uint16_t* X, int M, int K, const uint16_t* 
   return best;
 }
 
+/* ------------------------------------------------------------------------ */
+/* OffQ: outliers absorbed as an offset ([OffQ] 方法: 通过偏移量进行吸收     */
+/* (Hadamard 旋转), 分组实现).  Readings (the pages fix no precision or      */
+/* normalisation):                                                          */
+/*  - groups of 128 consecutive channels (K % 128 == 0); the activations    */
+/*    are taken after the offline top-1 PCA rotation, the outlier of a      */
+/*    group in its first channel;                                           */
+/*  - the partially random Hadamard matrix is D H, H the 128 x 128 Sylvester */
+/*    matrix h(i, j) = (-1)^popcount(i & j) and D = diag(d) with d_0 = 1     */
+/*    and d_i = +-1 given (seeded): its first row is all ones, so a value   */
+/*    in channel 0 adds the same amount to every transformed channel;       */
+/*  - y_g = x_g (D H) for each token and group, unnormalised (exact in fp64: */
+/*    sums of +-fp16 values); the 1/128 of the inverse goes to the weights;  */
+/*  - per (token, group) asymmetric INT4 with the group minimum as the     */
+/*    offset ("absorbed into the zero point"): lo = min y, hi = max y,      */
+/*    sd = (hi - lo) / 15, q = clamp(rne((y - lo) / sd), 0, 15), all in      */
+/*    fp64, so y ~ q sd + lo; stored: q (0..15), fp32(sd) and fp32(lo); a    */
+/*    constant group (hi == lo) gets sd = 0 and q = 0;                       */
+/*  - weights: W'_g = (1/128) H D W_g (so y_g W'_g = x_g W_g), fp64 then     */
+/*    fp32, quantized per output channel to INT4 like the W4A8 layer, with  */
+/*    the operand B = 16 q and its per-group column sums kept for the        */
+/*    offset term: y_m W' = sum_g c'_n (sd acc_g + lo colsum_g).             */
+/* ------------------------------------------------------------------------ */
+static int hsign(int i, int j) { return __builtin_popcount((unsigned)(i & j)) & 1 ? -1 : 1; }
+
+OQ_EXPORT void oq_offq_transform(const uint16_t* X, int M, int K, const int8_t* d, double* Y) {
+  for (int m = 0; m < M; ++m)
+    for (int g = 0; g < K / 128; ++g)
+      for (int j = 0; j < 128; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < 128; ++i)
+          acc += oq_half_to_double(X[(size_t)m * K + g * 128 + i]) * (double)d[i] * (double)hsign(i, j);
+        Y[(size_t)m * K + g * 128 + j] = acc;
+      }
+}
+
+OQ_EXPORT void oq_offq_quant_act(const uint16_t* X, int M, int K, const int8_t* d, int8_t* Xq, float* scale,
+                                 float* offset) {
+  const int G = K / 128;
+  double* y = (double*)malloc(sizeof(double) * (size_t)M * K);
+  oq_offq_transform(X, M, K, d, y);
+  for (int m = 0; m < M; ++m)
+    for (int g = 0; g < G; ++g) {
+      const double* yg = y + (size_t)m * K + g * 128;
+      double lo = yg[0], hi = yg[0];
+      for (int j = 1; j < 128; ++j) {
+        if (yg[j] < lo) lo = yg[j];
+        if (yg[j] > hi) hi = yg[j];
+      }
+      const double sd = (hi - lo) / 15.0;
+      scale[(size_t)m * G + g] = (float)sd;
+      offset[(size_t)m * G + g] = (float)lo;
+      for (int j = 0; j < 128; ++j)
+        Xq[(size_t)m * K + g * 128 + j] = (int8_t)(sd > 0.0 ? clampi(oq_rne((yg[j] - lo) / sd), 0, 15) : 0);
+    }
+  free(y);
+}
+
+OQ_EXPORT void oq_offq_rotate_weights(const uint16_t* W, int K, int N, const int8_t* d, float* Wr) {
+  for (int g = 0; g < K / 128; ++g)
+    for (int n = 0; n < N; ++n)
+      for (int j = 0; j < 128; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < 128; ++i)
+          acc += (double)hsign(j, i) * (double)d[i] * oq_half_to_double(W[(size_t)(g * 128 + i) * N + n]);
+        Wr[(size_t)(g * 128 + j) * N + n] = (float)(acc / 128.0);
+      }
+}
+
+/* Per-output-channel symmetric quantization of fp32 weights (the rule of
+ * oq_quant_weight_per_channel on fp32 input). */
+OQ_EXPORT void oq_quant_weight_per_channel_f32(const float* W, int K, int N, int qmax, int8_t* codes, float* scale) {
+  const float fq = (float)qmax;
+  float* wmax = (float*)calloc((size_t)(N > 0 ? N : 1), sizeof(float));
+  for (int k = 0; k < K; ++k)
+    for (int n = 0; n < N; ++n) {
+      float v = fabsf(W[(size_t)k * N + n]);
+      if (v > wmax[n]) wmax[n] = v;
+    }
+  for (int n = 0; n < N; ++n) scale[n] = wmax[n] / fq;
+  for (int k = 0; k < K; ++k)
+    for (int n = 0; n < N; ++n) {
+      float inv = (wmax[n] > 0.0f) ? (fq / wmax[n]) : 0.0f;
+      float p = W[(size_t)k * N + n] * inv;
+      codes[(size_t)k * N + n] = (int8_t)clampi(oq_rne((double)p), -qmax, qmax);
+    }
+  free(wmax);
+}
+
+/* y[r][n] = cscale[n] * sum_g (scale[m][g] * acc_g[m][n] + offset[m][g] *
+ * colsum_g[n]) in fp64, acc_g = sum_{k in g} Xq[m][k] Bt[n][k] and colsum_g
+ * = sum_{k in g} Bt[n][k] exact (int64); m = rows[r]. */
+OQ_EXPORT void oq_offq_gemm_rows(const int8_t* Xq, const float* scale, const float* offset, const int8_t* Bt,
+                                 const float* cscale, int K, int N, const int32_t* rows, int R, double* y) {
+  const int G = K / 128;
+  for (int r = 0; r < R; ++r) {
+    const int m = rows[r];
+    for (int n = 0; n < N; ++n) {
+      double sum = 0.0;
+      for (int g = 0; g < G; ++g) {
+        int64_t acc = 0, cs = 0;
+        for (int k = g * 128; k < (g + 1) * 128; ++k) {
+          acc += (int64_t)Xq[(size_t)m * K + k] * (int64_t)Bt[(size_t)n * K + k];
+          cs += (int64_t)Bt[(size_t)n * K + k];
+        }
+        sum += (double)scale[(size_t)m * G + g] * (double)acc + (double)offset[(size_t)m * G + g] * (double)cs;
+      }
+      y[(size_t)r * N + n] = sum * (double)cscale[n];
+    }
+  }
+}
+
 OQ_EXPORT int oq_invert(const double* A, int d, double* inv) {
   double* a = (double*)malloc(sizeof(double) * d * d);
   memcpy(a, A, sizeof(double) * d * d);

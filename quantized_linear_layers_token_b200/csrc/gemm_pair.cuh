@@ -100,6 +100,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
   const int cid = static_cast<int>(cluster_id_x());
   const bool leader = crk == 0;
   const bool comp = g.nO > 0;
+  QLIN_TRACE_INIT
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < S; ++s) {
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
             break;
           }
           if (leader) mbar_arrive_expect_tx(&full[s], 2u * kPairStage);
+          QLIN_STEP(gi, 0);
           unsigned char* A = smem + s * kPairStage;
           unsigned char* X = A + 16384;
           const uint32_t lb = lfull0 + static_cast<uint32_t>(8 * s);
@@ -196,6 +198,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
             ok = false;
             break;
           }
+          QLIN_STEP(gi, 5);
           tc_fence_after();
           issued = true;
           const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kPairStage >> 4));
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
               mma_f16_pair(tmem + 256, ad + 2 * k, bd + 2 * k, idesc_comp, (j > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit_pair(&empty[s], 0x3);
+          QLIN_STEP(gi, 7);
         }
         if (!ok) break;
         mma_commit_pair(acc_full, 0x3);

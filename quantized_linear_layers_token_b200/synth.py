@@ -127,6 +127,27 @@ def weights(rng: np.random.Generator, K: int, N: int, std: float, spike_frac: fl
     return w.astype(np.float16)
 
 
+def offq_signs(seed: int = 0) -> np.ndarray:
+    """Signs d (int8 [128]) of the partially random Hadamard matrix D H of
+    the OffQ transform: d_0 = +1 (so the matrix's first row is all ones),
+    the other 127 seeded +-1 (draw kind 7)."""
+    d = np.where(rng_for(5, seed, 7).random(128) < 0.5, -1, 1).astype(np.int8)
+    d[0] = 1
+    return d
+
+
+def offq_activations(M: int, K: int, seed: int = 0, outlier_mult: tuple = (20.0, 60.0)) -> np.ndarray:
+    """X fp16 [M][K] for the OffQ layer: N(0, 1), with the first channel of
+    every 128-channel group scaled by U[20, 60] per group -- the layout the
+    offline top-1 PCA rotation leaves (each group's outlier energy in its
+    first channel)."""
+    rng = rng_for(5, seed, 8, M % 997)
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    mult = rng.uniform(outlier_mult[0], outlier_mult[1], size=K // 128).astype(np.float32)
+    x[:, 0::128] *= mult[None, :]
+    return x.astype(np.float16)
+
+
 def grad_output(index: int, shape_idx: int, M: int, N: int, std: float = 2.0 ** -7) -> np.ndarray:
     """Upstream gradient dY (fp16 [M][N]) for the input-gradient path:
     N(0, std^2) i.i.d., a stand-in for the gradient a fine-tuning loss sends
