@@ -64,7 +64,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0  # nominal dense INT8 : bf16 tensor rate of B200 (4.5 : 2.25 PFLOP/s)
 DEFAULT_WORKLOAD = "llama70b_w4g128"
-DEFAULT_EXTRAS = "llama7b_w4_decode,llama7b_w4g128_prefill,phi3_w8_quaff,backward,gptq,smooth_search"
+DEFAULT_EXTRAS = "llama7b_w4_decode,llama7b_w4g128_prefill,phi3_w8_quaff,backward,gptq,smooth_search,offq"
 
 
 # ---------------------------------------------------------------------------
@@ -824,6 +824,88 @@ def smooth_record(device, stream, peaks, M=512, G=10, reps=3):
             "timing": f"median of {reps} calls, CUDA events on the launch stream"}
 
 
+# OffQ reports on Llama-3-8B; its linears (hidden 4096, 8 KV heads of 128,
+# intermediate 14336) at 4096 prefill tokens.
+OFFQ_LAYERS = (("q_proj", 4096, 4096), ("k_proj", 4096, 1024), ("v_proj", 4096, 1024), ("o_proj", 4096, 4096),
+               ("gate_proj", 4096, 14336), ("up_proj", 4096, 14336), ("down_proj", 14336, 4096))
+
+
+def offq_bytes(M, K, N):
+    """(quantization, GEMM) algorithmic bytes of one OffQ linear: X fp16 in,
+    one code byte per value and two fp32 per (token, group) out; then the
+    codes and group scales in, the packed INT4 weights, channel scales and
+    per-group column sums, and Y fp16 out."""
+    G = K // 128
+    quant = 2 * M * K + M * K + 8 * M * G
+    gemm = M * K + 8 * M * G + K * N // 2 + 4 * N + 4 * G * N + 2 * M * N
+    return quant, gemm
+
+
+def offq_record(device, stream, peaks, reps, M=4096):
+    """OffQ W4A4 prefill (Hadamard offset, per-group asymmetric INT4
+    activations, per-channel INT4 rotated weights) on the Llama-3-8B linears
+    at 4096 tokens: qlin_offq_forward per linear, and its two stages timed
+    apart.  Synthetic inputs of the OffQ recipe (each group's outlier energy
+    in its first channel, x U[20, 60])."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    d = synth.offq_signs(0)
+    xs, layers = {}, []
+    for i, (name, K, N) in enumerate(OFFQ_LAYERS):
+        if K not in xs:
+            xs[K] = torch.from_numpy(synth.offq_activations(M, K, seed=K).view(np.uint16)).to(device)
+        W = torch.from_numpy(synth.offq_weights(K, N, seed=i).view(np.uint16)).to(device)
+        codes = torch.zeros(qlin.qlin_offq_codes_bytes(K, N), dtype=torch.uint8, device=device)
+        cs = torch.zeros(N, dtype=torch.float32, device=device)
+        colsum = torch.zeros((K // 128, N), dtype=torch.float32, device=device)
+        Wr = torch.empty((K, N), dtype=torch.float32, device=device)
+        qlin.qlin_offq_pack(W, K, N, d, codes, cs, colsum, Wr, stream)
+        del Wr, W
+        nf = qlin.qlin_offq_forward_workspace(M, K, N)
+        ng = qlin.qlin_offq_gemm_workspace(M, K, N)
+        layers.append({"K": K, "N": N, "codes": codes, "cs": cs, "colsum": colsum,
+                       "Y": torch.empty((M, N), dtype=torch.int16, device=device),
+                       "Xq": torch.empty((M, K), dtype=torch.int8, device=device),
+                       "sc": torch.empty((M, K // 128), dtype=torch.float32, device=device),
+                       "off": torch.empty((M, K // 128), dtype=torch.float32, device=device),
+                       "nf": nf, "wsf": qlin.empty_workspace(nf, device), "ng": ng,
+                       "wsg": qlin.empty_workspace(ng, device)})
+
+    def fwd():
+        for L in layers:
+            qlin.qlin_offq_forward(xs[L["K"]], M, L["K"], L["N"], d, L["codes"], L["cs"], L["colsum"], L["Y"],
+                                   L["wsf"], L["nf"], stream)
+
+    def quant():
+        for L in layers:
+            qlin.qlin_offq_quant_act(xs[L["K"]], M, L["K"], d, L["Xq"], L["sc"], L["off"], stream)
+
+    def gemm():
+        for L in layers:
+            qlin.qlin_offq_gemm(L["Xq"], L["sc"], L["off"], M, L["K"], L["N"], L["codes"], L["cs"], L["colsum"],
+                                L["Y"], L["wsg"], L["ng"], stream)
+    times = {}
+    for key, fn in (("forward", fwd), ("quant", quant), ("gemm", gemm)):
+        g = graph_of(fn, stream)
+        times[key] = replay_median_ms(g, stream, reps)
+        del g
+    qlin.qlin_poll_device_status(stream)
+    ops = sum(2 * M * K * N for _, K, N in OFFQ_LAYERS)
+    qb = sum(offq_bytes(M, K, N)[0] for _, K, N in OFFQ_LAYERS)
+    gb = sum(offq_bytes(M, K, N)[1] for _, K, N in OFFQ_LAYERS)
+    fb = sum(2 * M * K + K * N // 2 + 4 * N + 4 * (K // 128) * N + 2 * M * N for _, K, N in OFFQ_LAYERS)
+    ms = times["forward"]
+    return {"op": "offq_forward", "model": "llama3_8b linears (q, k, v, o, gate, up, down)", "tokens": M,
+            "ms_per_step": ms, "tops": ops / (ms * 1e-3) / 1e12,
+            "roofline": roofline_of(ops, fb, ms * 1e-3, peaks),
+            "quant": {"ms": times["quant"], "roofline": roofline_of(0, qb, times["quant"] * 1e-3, peaks)},
+            "gemm": {"ms": times["gemm"], "tops": ops / (times["gemm"] * 1e-3) / 1e12,
+                     "roofline": roofline_of(ops, gb, times["gemm"] * 1e-3, peaks),
+                     "note": "includes the per-call widening of the INT4 codes to INT8"},
+            "launches_per_step": 3 * len(OFFQ_LAYERS),
+            "timing": f"median of {reps} CUDA-graph replays of the 7 linears"}
+
+
 def backward_record(device, stream, reps, peaks):
     import torch  # noqa: F401
     wl = synth.WORKLOADS["phi3_w8_quaff"]
@@ -1059,6 +1141,8 @@ def run_forward(args, wl):
                         workloads[name] = gptq_record(device, stream, peaks)
                     elif name == "smooth_search":
                         workloads[name] = smooth_record(device, stream, peaks)
+                    elif name == "offq":
+                        workloads[name] = offq_record(device, stream, peaks, reps)
                     else:
                         w2 = synth.WORKLOADS[name]
                         workloads[name] = measure_workload_record(w2, 4 if name == "llama7b_w4_decode" else 1,
@@ -1080,11 +1164,11 @@ def run_forward(args, wl):
             M = u[0]["M"]
             if world > 1:  # colmax + momentum per linear, then quant + GEMM per linear
                 return sum(2 + (2 if meta[sl["si"]]["nO"] > 0 else 0) +
-                           (1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 1024) else 0) for sl in u)
+                           (1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 512) else 0) for sl in u)
             colmax = sum(1 for sl in u if meta[sl["si"]]["nO"] > 0 and M > 16)
             if len(u) > 1 or (fw.grouped and M <= fw.GROUP_MAX_M):
                 return 2 + colmax  # one quantization launch, one GEMM launch for the group
-            widen = 1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 1024) else 0
+            widen = 1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 512) else 0
             return 2 + widen + colmax
 
         line = {

@@ -360,6 +360,73 @@ QLIN_API qlin_status qlin_smooth_search(const uint16_t* X, int32_t M, int32_t K,
                                         int32_t G, double* loss, int32_t* best, float* s_best, void* workspace,
                                         size_t ws_bytes, void* stream);
 
+/* OffQ: W4A4 with per-group asymmetric activations whose offset absorbs the
+ * structured outliers ("OffQ: Taming Structured Outliers in LLM Quantization
+ * by Offsetting", technical summary, 方法论: 通过偏移量进行吸收 (Hadamard
+ * 旋转) and its grouped implementation).  After the offline top-1 PCA step
+ * has concentrated a group's outlier energy in one channel, the rotation
+ * D H (first row all ones) spreads it as one constant over the group, and
+ * that constant becomes the group's offset (zero point).  The readings this
+ * library takes where the summaries are silent:
+ *   - groups of 128 consecutive input channels (K % 128 == 0);
+ *   - H the 128 x 128 Sylvester matrix h(i,j) = (-1)^popcount(i & j),
+ *     D = diag(signs), signs[i] = +1 or -1 with signs[0] = +1 (host int8
+ *     [128], read during the call; QLIN_ERR_ARG otherwise);
+ *   - activations, per token m and group g: y = x_g D H unnormalised and
+ *     exact (fp64), lo = min y, hi = max y, sd = (hi - lo) / 15,
+ *     q = clamp(rne((y - lo) / sd), 0, 15) taken in fp64 (q = 0 when
+ *     sd == 0); so y ~ q sd + lo;
+ *   - weights, per group: W' = (1/128) H D W_g in fp64 then fp32, then
+ *     symmetric INT4 per output channel in fp32: c_n = max_k|W'[k][n]| / 7,
+ *     q_w = clamp(rne(W' * (7 / max)), -7, 7);
+ *   - output: Y[m][n] = fp16( (c_n / 16) * sum_g ( sd[m][g] acc_g[m][n]
+ *     + lo[m][g] colsum_g[n] ) ), acc_g = sum_{k in g} q[m][k] 16 q_w[k][n]
+ *     (exact INT32 per K-block on the tensor cores) and colsum_g[n] =
+ *     sum_{k in g} 16 q_w[k][n]; the sum over groups is fp32 (two fused
+ *     multiply-adds per group, in group order).
+ * Shapes: 128 <= K <= 65536 with K % 128 == 0; N % 16 == 0; M >= 0 (M == 0
+ * enqueues nothing).  Non-finite activations give unspecified codes. */
+
+/* Bytes of the packed OffQ codes of a K x N layer: the W4 per-channel tile
+ * layout of qlin_weights.codes (ceil(N/128) * K/128 blocks of 8 KiB). */
+QLIN_API qlin_status qlin_offq_codes_bytes(int32_t K, int32_t N, size_t* bytes);
+
+/* Wr = the rotated weights, fp32 [K][N] (device), from W fp16 [K][N]
+ * (device): Wr[128g + j][n] = fp32((1/128) sum_i h(j,i) signs[i] W[128g + i][n]),
+ * bit-exact (the sums are exact in fp64). */
+QLIN_API qlin_status qlin_offq_rotate_weights(const uint16_t* W, int32_t K, int32_t N, const int8_t* signs,
+                                              float* Wr, void* stream);
+
+/* Offline packing: rotates W into Wr (device fp32 [K][N], caller-owned
+ * scratch that keeps the rotated weights) and quantizes it.
+ *   codes       device, qlin_offq_codes_bytes bytes (cleared, then written).
+ *   chan_scale  device fp32 [N]: c_n.
+ *   colsum      device fp32 [K/128][N]: colsum_g[n] (integers, exact). */
+QLIN_API qlin_status qlin_offq_pack(const uint16_t* W, int32_t K, int32_t N, const int8_t* signs, uint8_t* codes,
+                                    float* chan_scale, float* colsum, float* Wr, void* stream);
+
+/* Activation side: X device fp16 [M][K] -> Xq device int8 [M][K] (codes
+ * 0..15, one per byte), scale = fp32(sd) and offset = fp32(lo), device fp32
+ * [M][K/128].  Bit-exact. */
+QLIN_API qlin_status qlin_offq_quant_act(const uint16_t* X, int32_t M, int32_t K, const int8_t* signs, int8_t* Xq,
+                                         float* scale, float* offset, void* stream);
+
+/* The GEMM from quantized activations: Y device fp16 [M][N] as above.  The
+ * workspace (qlin_offq_gemm_workspace bytes, 256-byte aligned, no
+ * zero-fill needed) receives the codes widened to INT8 (16 q_w) once per
+ * call. */
+QLIN_API qlin_status qlin_offq_gemm_workspace(int32_t M, int32_t K, int32_t N, size_t* bytes);
+QLIN_API qlin_status qlin_offq_gemm(const int8_t* Xq, const float* scale, const float* offset, int32_t M, int32_t K,
+                                    int32_t N, const uint8_t* codes, const float* chan_scale, const float* colsum,
+                                    uint16_t* Y, void* workspace, size_t ws_bytes, void* stream);
+
+/* qlin_offq_quant_act then qlin_offq_gemm, the intermediates in the
+ * workspace (qlin_offq_forward_workspace bytes, 256-byte aligned). */
+QLIN_API qlin_status qlin_offq_forward_workspace(int32_t M, int32_t K, int32_t N, size_t* bytes);
+QLIN_API qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, int32_t N, const int8_t* signs,
+                                       const uint8_t* codes, const float* chan_scale, const float* colsum,
+                                       uint16_t* Y, void* workspace, size_t ws_bytes, void* stream);
+
 /* Test and measurement hooks.  The library reads no environment variables:
  * a process that wants a non-default work split, launch mode or wait limit
  * (the test suite forcing each split-K variant, a measurement isolating one
@@ -377,14 +444,15 @@ QLIN_API qlin_status qlin_smooth_search(const uint16_t* X, int32_t M, int32_t K,
  *   QLIN_KNOB_MAX_CTAS        0 (default): one persistent GEMM CTA per SM;
  *                             n > 0: at most n.
  *   QLIN_KNOB_MAX_TOKEN_TILE  256 (default); 64 or 128 cap the GEMM's token tile.
- *   QLIN_KNOB_WIDEN_MIN_M     1024 (default): from this token count INT4
+ *   QLIN_KNOB_WIDEN_MIN_M     512 (default): from this token count INT4
  *                             weights are widened to INT8 once per call; 0: never.
  *   QLIN_KNOB_FUSED_MOMENTUM_MAX_M  16 (default): up to this token count the
  *                             momentum update runs inside the quantization kernel.
- *   QLIN_KNOB_PAIR_MMA        1 (default): 256-token tiles with INT8 operands run
+ *   QLIN_KNOB_PAIR_MMA        2 (default): 256-token tiles with INT8 operands run
  *                             on CTA pairs (one 256-row tensor-core operation
- *                             per pair) when there is a full wave of 256 x 256
- *                             tiles; 0: never; 2: whenever the operands allow.
+ *                             per pair) whenever the operands allow; 1: only
+ *                             when there is a full wave of 256 x 256 tiles;
+ *                             0: never.
  *   QLIN_KNOB_WAIT_NS         2000000000 (default): limit in ns of every
  *                             device-side pipeline wait, after which the kernel
  *                             gives up, sets the device error word and unwinds

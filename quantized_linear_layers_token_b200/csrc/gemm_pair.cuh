@@ -27,22 +27,24 @@
 //   warp 1        tensor memory allocation (both CTAs, cta_group::2); in the
 //                 even CTA one lane issues the pair MMAs and commits.
 //   warps 2..9    epilogue, two groups of four warps taking alternate
-//                 16-token chunks of the CTA's 128 x 256 accumulator; each
-//                 warp then arrives on the even CTA's accumulator-empty
-//                 barrier.
+//                 16-token chunks of the CTA's 128 x 256 accumulator into an
+//                 fp16 output tile in shared memory; each warp then arrives
+//                 on the even CTA's accumulator-empty barrier (so the next
+//                 tile's products start), and one thread writes the output
+//                 tile with a TMA store that runs under them.
 #pragma once
 
 #include "gemm.cuh"
 
 namespace qlin {
 
-constexpr int kPairStages = 6;
+constexpr int kPairStages = 5;
 constexpr int kPairStage = 32768;  // per CTA and step: 16 KB weight rows + 16 KB token rows
-constexpr int kPairYStage = 16 * 128 * 2;
-constexpr int kPairOffY = kPairStages * kPairStage;
-constexpr int kPairOffBar = kPairOffY + 4 * kPairYStage;
-constexpr int kPairOffSa = kPairOffBar + 1024;
-constexpr int kPairSmem = kPairOffSa + 2048 + 1024;  // + alignment slack
+constexpr int kPairOffY = kPairStages * kPairStage;  // the tile's output, fp16 [256 tokens][128 channels]
+constexpr int kPairOffBar = kPairOffY + 256 * 128 * 2;
+constexpr int kPairOffSa = kPairOffBar + 256;
+constexpr int kPairSmem = kPairOffSa + 1024 + 1024;  // + alignment slack
+static_assert(kPairSmem <= 232448, "pair kernel shared memory above 227 KB");
 constexpr int kPairThreads = 32 * (2 + 8);
 constexpr int kPairEpiWarps = 8;
 
@@ -69,6 +71,7 @@ struct alignas(64) PairParams {
   CUtensorMap tmX;   // Xq int8 [M][K], 128 x 128 boxes, 128-byte swizzle
   CUtensorMap tmU;   // U fp16 [2M][nOp], 64 x 128 boxes, 128-byte swizzle
   CUtensorMap tmWo;  // W_O^T blocks as rows of 128 bytes: [ntn * ncs * 128][128]
+  CUtensorMap tmY;   // Y fp16 [M][N], 128 x 256 boxes (stores)
   PairArgs g;
 };
 
@@ -229,15 +232,20 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // Each tile's output goes to shared memory first; the accumulator is
+    // released as soon as it has been read, and one TMA store per tile
+    // writes the output while the next tile's products run.
     const int ep = warp - 2;
     const int grp = ep >> 2;
     const int quad = warp & 3;  // TMEM lanes 32*quad .. +31
     const int nl = quad * 32 + lane;
-    const int gbar = 1 + grp;
-    float* sa_t = reinterpret_cast<float*>(smem + kPairOffSa + grp * 1024);
+    const bool issuer = ep == 0 && lane == 0;
+    float* sa = reinterpret_cast<float*>(smem + kPairOffSa);       // a_m of the tile's 256 tokens
+    uint16_t* ys = reinterpret_cast<uint16_t*>(smem + kPairOffY);  // [256 tokens][128 channels]
     const uint32_t lempty = mapa_shared(smem_u32(acc_empty), 0);
     griddep_wait();  // a[] comes from the previous kernel
-    int ycnt = 0, ti = 0;
+    int ti = 0;
+    bool ok = true;
     for (int t = cid; t < g.tiles; t += g.ncl, ++ti) {
       int tn2, tm;
       pair_tile_coords(g, t, tn2, tm);
@@ -247,17 +255,19 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
       const int mvalid = min(256, g.M - m0);
       float cn = 0.f;
       if (n < g.N) cn = __fmul_rn(g.cscale[n], g.cmul);
-      bool ok = mbar_wait(acc_full, static_cast<uint32_t>(ti) & 1u, abort_flag);
+      if (issuer) bulk_wait_group_read0();  // the previous tile's store has read the output buffer
+      named_bar_sync(1, 256);
+      {
+        const int j = ep * 32 + lane;
+        sa[j] = j < mvalid ? g.a[m0 + j] : 0.f;
+      }
+      named_bar_sync(1, 256);
+      if (ok) ok = mbar_wait(acc_full, static_cast<uint32_t>(ti) & 1u, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      named_bar_sync(gbar, 128);
-      for (int j = nl; j < 256; j += 128) sa_t[j] = j < mvalid ? g.a[m0 + j] : 0.f;
-      named_bar_sync(gbar, 128);
       const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
 #pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 16) {
-        if (c0 >= mvalid) break;
-        if (((c0 >> 4) & 1) != grp) continue;
+      for (int c0 = grp * 16; c0 < mvalid; c0 += 32) {
         uint32_t acc[16], cmp[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) { acc[j] = 0u; cmp[j] = 0u; }
@@ -266,37 +276,21 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
           if (comp) tmem_ld16(trow + 256 + c0, cmp);
           tmem_ld_wait();
         }
-        const int b = ycnt & 1;
-        uint16_t* ys = reinterpret_cast<uint16_t*>(smem + kPairOffY + (grp * 2 + b) * kPairYStage);
         float sc[16];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const float4 v = *reinterpret_cast<const float4*>(sa_t + c0 + 4 * q4);
+          const float4 v = *reinterpret_cast<const float4*>(sa + c0 + 4 * q4);
           sc[4 * q4] = v.x; sc[4 * q4 + 1] = v.y; sc[4 * q4 + 2] = v.z; sc[4 * q4 + 3] = v.w;
         }
-        uint16_t yh[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           float v = __fmul_rn(cn, static_cast<float>(static_cast<int32_t>(acc[j])));
           if (comp) v = __fadd_rn(v, __uint_as_float(cmp[j]));
-          yh[j] = __half_as_ushort(__float2half_rn(__fmul_rn(sc[j], v)));
+          ys[(c0 + j) * 128 + nl] = __half_as_ushort(__float2half_rn(__fmul_rn(sc[j], v)));
         }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ys[j * 128 + nl] = yh[j];
         if (g.acc_debug && n < g.N)
           for (int j = 0; j < 16; ++j)
             if (c0 + j < mvalid) g.acc_debug[static_cast<size_t>(m0 + c0 + j) * g.N + n] = static_cast<int32_t>(acc[j]);
-        named_bar_sync(gbar, 128);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int idx = nl + h * 128;  // 16 rows x 16 segments of 8 channels
-          const int j = idx >> 4;
-          const int n8 = ctile * 128 + (idx & 15) * 8;
-          if (c0 + j < mvalid && n8 < g.N)
-            *reinterpret_cast<uint4*>(g.Y + static_cast<size_t>(m0 + c0 + j) * g.N + n8) =
-                *reinterpret_cast<const uint4*>(ys + j * 128 + (idx & 15) * 8);
-        }
-        ++ycnt;
       }
       tc_fence_before();
       __syncwarp();
@@ -304,7 +298,14 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
         if (leader) mbar_arrive(acc_empty);
         else mbar_arrive_remote(lempty);
       }
+      fence_proxy_async_smem();  // the output rows are read by the bulk copy next
+      named_bar_sync(1, 256);
+      if (issuer && ctile * 128 < g.N) {
+        tma_store_2d(&prm.tmY, ys, ctile * 128, m0);
+        bulk_commit_group();
+      }
     }
+    if (issuer) bulk_wait_group_all();
   }
   tc_fence_before();
   __syncthreads();

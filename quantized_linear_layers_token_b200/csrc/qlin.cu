@@ -18,6 +18,7 @@
 #include "gemm_pair.cuh"
 #include "backward.cuh"
 #include "gptq.cuh"
+#include "offq.cuh"
 #include "pack.cuh"
 #include "smooth.cuh"
 
@@ -140,7 +141,7 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 // each may start its prologue (and the GEMM its weight stream) while the
 // previous kernel in the stream finishes; every kernel waits on the grid
 // dependency before it reads what the previous one wrote.
-std::atomic<long long> g_knob[9] = {{1}, {1}, {0}, {0}, {256}, {1024}, {kFusedMomentumMaxM}, {2000000000LL}, {1}};
+std::atomic<long long> g_knob[9] = {{1}, {1}, {0}, {0}, {256}, {512}, {kFusedMomentumMaxM}, {2000000000LL}, {2}};
 
 long long knob(int k) { return g_knob[k].load(std::memory_order_relaxed); }
 
@@ -444,9 +445,9 @@ int pair_max_clusters() {
 }
 
 // Whether a single-problem launch runs on CTA pairs: 256-token tiles with
-// INT8 operands (the INT8 format, or INT4 widened once per call) and at
-// least one full wave of 256 x 256 pair tiles (QLIN_KNOB_PAIR_MMA: 0 never,
-// 2 whenever the operands allow).
+// INT8 operands (the INT8 format, or INT4 widened once per call); by default
+// whenever the operands allow, even with fewer 256 x 256 pair tiles than
+// pairs on the GPU (QLIN_KNOB_PAIR_MMA: 0 never, 1 only from one full wave).
 bool use_pair(const GemmPlan& p, const qlin_weights* w) {
   const long long mode = knob(QLIN_KNOB_PAIR_MMA);
   if (mode == 0 || p.nprob != 1 || p.bt != 256) return false;
@@ -498,6 +499,8 @@ qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int
                   static_cast<uint64_t>(q.tiles_n) * q.ncs * 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != QLIN_OK) return st;
   }
+  st = make_map(&prm.tmY, Y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->N, M, 128, 256, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != QLIN_OK) return st;
   cudaError_t e = launch_kc(gemm_pair_kernel, dim3(static_cast<unsigned>(2 * g.ncl)), dim3(kPairThreads), kPairSmem,
                             stream, 2, prm);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_pair_kernel launch failed: %s", cudaGetErrorString(e));
@@ -1403,6 +1406,221 @@ qlin_status qlin_smooth_search(const uint16_t* X, int32_t M, int32_t K, const ui
   smooth_pick_kernel<<<1, 256, 0, stream>>>(loss, G, cmax, wmax, xall, K, best, s_best);
   QLIN_LAUNCH_CHECK("smooth_pick_kernel");
   return QLIN_OK;
+}
+
+// ---------------------------------------------------------------- OffQ
+namespace {
+// d (+1/-1, d_0 = +1) as a bit mask: bit i set when d_i = -1.
+qlin_status offq_signs(const int8_t* d, uint4* out) {
+  if (!d) return fail(QLIN_ERR_ARG, "signs is NULL");
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  for (int i = 0; i < 128; ++i) {
+    if (d[i] != 1 && d[i] != -1) return fail(QLIN_ERR_ARG, "signs[%d] = %d is not +1 or -1", i, int(d[i]));
+    if (d[i] < 0) w[i >> 5] |= 1u << (i & 31);
+  }
+  if (w[0] & 1u) return fail(QLIN_ERR_ARG, "signs[0] must be +1 (row 0 of D H is all ones)");
+  *out = make_uint4(w[0], w[1], w[2], w[3]);
+  return QLIN_OK;
+}
+
+qlin_status check_offq_shape(int32_t M, int32_t K, int32_t N) {
+  if (M < 0 || K <= 0 || N <= 0) return fail(QLIN_ERR_ARG, "bad sizes M=%d K=%d N=%d", M, K, N);
+  if (K % 128 || K > 65536) return fail(QLIN_ERR_SHAPE, "OffQ needs K %% 128 == 0 and K <= 65536 (K=%d)", K);
+  if (N % 16 || N > 1048576) return fail(QLIN_ERR_SHAPE, "N=%d must be a multiple of 16 and <= 2^20", N);
+  return QLIN_OK;
+}
+
+size_t offq_codes_size(int32_t K, int32_t N) { return size_t((N + 127) / 128) * (K / 128) * 8192; }
+size_t offq_wide_size(int32_t K, int32_t N) { return size_t((N + 127) / 128) * (K / 128) * 16384; }
+
+struct OffqLayout {
+  size_t xq = 0, scale = 0, offset = 0, wide = 0, total = 0;
+};
+OffqLayout offq_layout(int32_t M, int32_t K, int32_t N, bool with_act) {
+  OffqLayout L;
+  size_t o = 0;
+  if (with_act) {
+    L.xq = o;
+    o = round_up(o + size_t(M) * K, kAlign);
+    L.scale = o;
+    o = round_up(o + size_t(M) * (K / 128) * 4, kAlign);
+    L.offset = o;
+    o = round_up(o + size_t(M) * (K / 128) * 4, kAlign);
+  }
+  L.wide = o;
+  L.total = round_up(o + offq_wide_size(K, N), kAlign);
+  return L;
+}
+
+int offq_gemm_smem_ok() {
+  static int ok = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    ok = cudaFuncSetAttribute(offq_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOffqSmem) ==
+         cudaSuccess;
+    if (!ok) cudaGetLastError();
+  });
+  return ok;
+}
+
+qlin_status launch_offq_quant(const uint16_t* X, int32_t M, int32_t K, uint4 sg, int8_t* Xq, float* scale,
+                              float* offset, cudaStream_t stream) {
+  const long long units = static_cast<long long>(M) * (K / 128);
+  const long long blocks = (units + kOffqQuantThreads / 4 - 1) / (kOffqQuantThreads / 4);
+  if (blocks > 0x7fffffffLL) return fail(QLIN_ERR_SHAPE, "M * K too large");
+  cudaError_t e = launch_k(offq_quant_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kOffqQuantThreads), 0,
+                           stream, X, M, K, sg, Xq, scale, offset);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "offq_quant_kernel launch failed: %s", cudaGetErrorString(e));
+  return QLIN_OK;
+}
+
+qlin_status launch_offq_gemm(const int8_t* Xq, const float* scale, const float* offset, int32_t M, int32_t K,
+                             int32_t N, const uint8_t* codes, const float* chan_scale, const float* colsum,
+                             uint16_t* Y, uint8_t* wide, cudaStream_t stream) {
+  qlin_status st = get_encoder();
+  if (st != QLIN_OK) return st;
+  if (!offq_gemm_smem_ok()) return fail(QLIN_ERR_CUDA, "offq_gemm_kernel: shared memory attribute refused");
+  const int kb = K / 128;
+  const int tiles_n = (N + 127) / 128;
+  const unsigned nblk = static_cast<unsigned>(tiles_n) * static_cast<unsigned>(kb);
+  cudaError_t e = launch_k(widen_w4_kernel<kFmtW4PC>, dim3(nblk), dim3(256), 0, stream, codes,
+                           static_cast<const uint16_t*>(nullptr), N, kb, wide);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "widen_w4_kernel launch failed: %s", cudaGetErrorString(e));
+  OffqParams prm;
+  memset(&prm, 0, sizeof(prm));
+  OffqArgs& g = prm.g;
+  g.scale = scale;
+  g.offset = offset;
+  g.colsum = colsum;
+  g.cscale = chan_scale;
+  g.wide = wide;
+  g.Y = Y;
+  g.M = M;
+  g.N = N;
+  g.G = kb;
+  g.tiles_m = (M + 127) / 128;
+  g.tiles = g.tiles_m * tiles_n;
+  st = make_map(&prm.tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QLIN_OK) return st;
+  const int cap = gemm_cta_cap();
+  const int grid = g.tiles < cap ? g.tiles : cap;
+  e = launch_k(offq_gemm_kernel<0>, dim3(static_cast<unsigned>(grid)), dim3(kOffqThreads), kOffqSmem, stream, prm);
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "offq_gemm_kernel launch failed: %s", cudaGetErrorString(e));
+  return QLIN_OK;
+}
+}  // namespace
+
+qlin_status qlin_offq_codes_bytes(int32_t K, int32_t N, size_t* bytes) {
+  qlin_status st = check_offq_shape(0, K, N);
+  if (st != QLIN_OK) return st;
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  *bytes = offq_codes_size(K, N);
+  return QLIN_OK;
+}
+
+qlin_status qlin_offq_rotate_weights(const uint16_t* W, int32_t K, int32_t N, const int8_t* signs, float* Wr,
+                                     void* stream_) {
+  qlin_status st = check_offq_shape(0, K, N);
+  if (st != QLIN_OK) return st;
+  uint4 sg;
+  st = offq_signs(signs, &sg);
+  if (st != QLIN_OK) return st;
+  if (!W || !Wr) return fail(QLIN_ERR_ARG, "W/Wr is NULL");
+  if (!aligned16(W) || !aligned16(Wr)) return fail(QLIN_ERR_ALIGN, "W/Wr is not 16-byte aligned");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  offq_rotate_kernel<<<dim3((N + 31) / 32, K / 128), 256, 0, stream>>>(W, K, N, sg, Wr);
+  QLIN_LAUNCH_CHECK("offq_rotate_kernel");
+  return QLIN_OK;
+}
+
+qlin_status qlin_offq_pack(const uint16_t* W, int32_t K, int32_t N, const int8_t* signs, uint8_t* codes,
+                           float* chan_scale, float* colsum, float* Wr, void* stream_) {
+  qlin_status st = qlin_offq_rotate_weights(W, K, N, signs, Wr, stream_);
+  if (st != QLIN_OK) return st;
+  if (!codes || !chan_scale || !colsum) return fail(QLIN_ERR_ARG, "codes/chan_scale/colsum is NULL");
+  if (!aligned16(codes) || !aligned16(chan_scale) || !aligned16(colsum))
+    return fail(QLIN_ERR_ALIGN, "codes/chan_scale/colsum is not 16-byte aligned");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  QLIN_CUDA_TRY(cudaMemsetAsync(codes, 0, offq_codes_size(K, N), stream));  // padding channels stay zero
+  offq_pack_kernel<<<(N + 127) / 128, 128, 0, stream>>>(Wr, K, N, codes, chan_scale, colsum);
+  QLIN_LAUNCH_CHECK("offq_pack_kernel");
+  return QLIN_OK;
+}
+
+qlin_status qlin_offq_quant_act(const uint16_t* X, int32_t M, int32_t K, const int8_t* signs, int8_t* Xq,
+                                float* scale, float* offset, void* stream_) {
+  qlin_status st = check_offq_shape(M, K, 16);
+  if (st != QLIN_OK) return st;
+  uint4 sg;
+  st = offq_signs(signs, &sg);
+  if (st != QLIN_OK) return st;
+  if (M == 0) return QLIN_OK;
+  if (!X || !Xq || !scale || !offset) return fail(QLIN_ERR_ARG, "X/Xq/scale/offset is NULL");
+  if (!aligned16(X) || !aligned16(Xq) || (reinterpret_cast<uintptr_t>(scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(offset) & 3u))
+    return fail(QLIN_ERR_ALIGN, "X/Xq must be 16-byte aligned, scale/offset 4");
+  return launch_offq_quant(X, M, K, sg, Xq, scale, offset, static_cast<cudaStream_t>(stream_));
+}
+
+qlin_status qlin_offq_gemm_workspace(int32_t M, int32_t K, int32_t N, size_t* bytes) {
+  qlin_status st = check_offq_shape(M, K, N);
+  if (st != QLIN_OK) return st;
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  *bytes = offq_layout(M, K, N, false).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_offq_gemm(const int8_t* Xq, const float* scale, const float* offset, int32_t M, int32_t K,
+                           int32_t N, const uint8_t* codes, const float* chan_scale, const float* colsum, uint16_t* Y,
+                           void* workspace, size_t ws_bytes, void* stream_) {
+  qlin_status st = check_offq_shape(M, K, N);
+  if (st != QLIN_OK) return st;
+  if (M == 0) return QLIN_OK;
+  if (!Xq || !scale || !offset || !codes || !chan_scale || !colsum || !Y || !workspace)
+    return fail(QLIN_ERR_ARG, "a pointer argument is NULL");
+  if (!aligned16(Xq) || !aligned16(codes) || !aligned16(chan_scale) || !aligned16(colsum) || !aligned16(Y) ||
+      (reinterpret_cast<uintptr_t>(scale) & 3u) || (reinterpret_cast<uintptr_t>(offset) & 3u))
+    return fail(QLIN_ERR_ALIGN, "Xq/codes/chan_scale/colsum/Y must be 16-byte aligned, scale/offset 4");
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const OffqLayout L = offq_layout(M, K, N, false);
+  if (ws_bytes < L.total) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, L.total);
+  uint8_t* wide = static_cast<uint8_t*>(workspace) + L.wide;
+  return launch_offq_gemm(Xq, scale, offset, M, K, N, codes, chan_scale, colsum, Y, wide,
+                          static_cast<cudaStream_t>(stream_));
+}
+
+qlin_status qlin_offq_forward_workspace(int32_t M, int32_t K, int32_t N, size_t* bytes) {
+  qlin_status st = check_offq_shape(M, K, N);
+  if (st != QLIN_OK) return st;
+  if (!bytes) return fail(QLIN_ERR_ARG, "bytes is NULL");
+  *bytes = offq_layout(M, K, N, true).total;
+  return QLIN_OK;
+}
+
+qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, int32_t N, const int8_t* signs,
+                              const uint8_t* codes, const float* chan_scale, const float* colsum, uint16_t* Y,
+                              void* workspace, size_t ws_bytes, void* stream_) {
+  qlin_status st = check_offq_shape(M, K, N);
+  if (st != QLIN_OK) return st;
+  uint4 sg;
+  st = offq_signs(signs, &sg);
+  if (st != QLIN_OK) return st;
+  if (M == 0) return QLIN_OK;
+  if (!X || !codes || !chan_scale || !colsum || !Y || !workspace) return fail(QLIN_ERR_ARG, "a pointer argument is NULL");
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(chan_scale) || !aligned16(colsum) || !aligned16(Y))
+    return fail(QLIN_ERR_ALIGN, "X/codes/chan_scale/colsum/Y is not 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return fail(QLIN_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const OffqLayout L = offq_layout(M, K, N, true);
+  if (ws_bytes < L.total) return fail(QLIN_ERR_WORKSPACE, "workspace %zu < %zu", ws_bytes, L.total);
+  char* ws = static_cast<char*>(workspace);
+  int8_t* Xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* scale = reinterpret_cast<float*>(ws + L.scale);
+  float* offset = reinterpret_cast<float*>(ws + L.offset);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  st = launch_offq_quant(X, M, K, sg, Xq, scale, offset, stream);
+  if (st != QLIN_OK) return st;
+  return launch_offq_gemm(Xq, scale, offset, M, K, N, codes, chan_scale, colsum, Y,
+                          reinterpret_cast<uint8_t*>(ws + L.wide), stream);
 }
 
 qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {

@@ -31,7 +31,9 @@ EXPORTED = [
     "qlin_forward", "qlin_poll_device_status", "qlin_quant_act_noalloc", "qlin_backward_dx",
     "qlin_backward_dx_workspace", "qlin_debug_set", "qlin_debug_get", "qlin_forward_grouped_workspace",
     "qlin_forward_grouped", "qlin_gptq_workspace", "qlin_gptq_quantize", "qlin_smooth_search_workspace",
-    "qlin_smooth_search",
+    "qlin_smooth_search", "qlin_offq_codes_bytes", "qlin_offq_rotate_weights", "qlin_offq_pack",
+    "qlin_offq_quant_act", "qlin_offq_gemm_workspace", "qlin_offq_gemm", "qlin_offq_forward_workspace",
+    "qlin_offq_forward",
 ]
 
 # test / measurement knobs (qlin_debug_set, include/qlin.h)
@@ -106,6 +108,14 @@ def lib() -> ctypes.CDLL:
             "qlin_smooth_search_workspace": [I32, I32, I32, I32, ctypes.POINTER(SZ)],
             "qlin_smooth_search": [P, I32, I32, P, I32, I32, P, P, P, P, SZ, P],
             "qlin_debug_get": [I32, ctypes.POINTER(ctypes.c_int64)],
+            "qlin_offq_codes_bytes": [I32, I32, ctypes.POINTER(SZ)],
+            "qlin_offq_rotate_weights": [P, I32, I32, P, P, P],
+            "qlin_offq_pack": [P, I32, I32, P, P, P, P, P, P],
+            "qlin_offq_quant_act": [P, I32, I32, P, P, P, P, P],
+            "qlin_offq_gemm_workspace": [I32, I32, I32, ctypes.POINTER(SZ)],
+            "qlin_offq_gemm": [P, P, P, I32, I32, I32, P, P, P, P, P, SZ, P],
+            "qlin_offq_forward_workspace": [I32, I32, I32, ctypes.POINTER(SZ)],
+            "qlin_offq_forward": [P, I32, I32, I32, P, P, P, P, P, P, SZ, P],
         }
         for name, argt in sigs.items():
             fn = getattr(L, name)
@@ -258,6 +268,58 @@ def qlin_smooth_search(X, M: int, K: int, W, N: int, G: int, loss, best, s_best,
                        stream=None):
     _check(lib().qlin_smooth_search(_ptr(X), M, K, _ptr(W), N, G, _ptr(loss), _ptr(best), _ptr(s_best),
                                     _ptr(workspace), ws_bytes, _stream(stream)), "qlin_smooth_search")
+
+
+def _signs(signs) -> tuple:
+    """Host int8 [128] copy of the OffQ signs d (kept alive by the caller's frame)."""
+    arr = np.ascontiguousarray(np.asarray(signs, dtype=np.int8))
+    if arr.shape != (128,):
+        raise ValueError(f"signs must have 128 entries, got shape {arr.shape}")
+    return arr, arr.ctypes.data
+
+
+def qlin_offq_codes_bytes(K: int, N: int) -> int:
+    return _size(lib().qlin_offq_codes_bytes, K, N)
+
+
+def qlin_offq_rotate_weights(W, K: int, N: int, signs, Wr, stream=None):
+    arr, sp = _signs(signs)
+    _check(lib().qlin_offq_rotate_weights(_ptr(W), K, N, sp, _ptr(Wr), _stream(stream)),
+           "qlin_offq_rotate_weights")
+
+
+def qlin_offq_pack(W, K: int, N: int, signs, codes, chan_scale, colsum, Wr, stream=None):
+    arr, sp = _signs(signs)
+    _check(lib().qlin_offq_pack(_ptr(W), K, N, sp, _ptr(codes), _ptr(chan_scale), _ptr(colsum), _ptr(Wr),
+                                _stream(stream)), "qlin_offq_pack")
+
+
+def qlin_offq_quant_act(X, M: int, K: int, signs, Xq, scale, offset, stream=None):
+    arr, sp = _signs(signs)
+    _check(lib().qlin_offq_quant_act(_ptr(X), M, K, sp, _ptr(Xq), _ptr(scale), _ptr(offset), _stream(stream)),
+           "qlin_offq_quant_act")
+
+
+def qlin_offq_gemm_workspace(M: int, K: int, N: int) -> int:
+    return _size(lib().qlin_offq_gemm_workspace, M, K, N)
+
+
+def qlin_offq_gemm(Xq, scale, offset, M: int, K: int, N: int, codes, chan_scale, colsum, Y, workspace,
+                   ws_bytes: int, stream=None):
+    _check(lib().qlin_offq_gemm(_ptr(Xq), _ptr(scale), _ptr(offset), M, K, N, _ptr(codes), _ptr(chan_scale),
+                                _ptr(colsum), _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "qlin_offq_gemm")
+
+
+def qlin_offq_forward_workspace(M: int, K: int, N: int) -> int:
+    return _size(lib().qlin_offq_forward_workspace, M, K, N)
+
+
+def qlin_offq_forward(X, M: int, K: int, N: int, signs, codes, chan_scale, colsum, Y, workspace, ws_bytes: int,
+                      stream=None):
+    arr, sp = _signs(signs)
+    _check(lib().qlin_offq_forward(_ptr(X), M, K, N, sp, _ptr(codes), _ptr(chan_scale), _ptr(colsum), _ptr(Y),
+                                   _ptr(workspace), ws_bytes, _stream(stream)), "qlin_offq_forward")
 
 
 def qlin_backward_dx_workspace(M: int, w: qlin_weights) -> int:

@@ -148,6 +148,12 @@ def offq_activations(M: int, K: int, seed: int = 0, outlier_mult: tuple = (20.0,
     return x.astype(np.float16)
 
 
+def offq_weights(K: int, N: int, seed: int = 0, std: float = 0.02) -> np.ndarray:
+    """W fp16 [K][N] for the OffQ layer: N(0, std^2) i.i.d. (draw kind 9)."""
+    rng = rng_for(5, seed, 9, N % 997)
+    return (rng.standard_normal((K, N), dtype=np.float32) * np.float32(std)).astype(np.float16)
+
+
 def grad_output(index: int, shape_idx: int, M: int, N: int, std: float = 2.0 ** -7) -> np.ndarray:
     """Upstream gradient dY (fp16 [M][N]) for the input-gradient path:
     N(0, std^2) i.i.d., a stand-in for the gradient a fine-tuning loss sends

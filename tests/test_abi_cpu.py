@@ -130,6 +130,40 @@ def test_backward_argument_errors(q):
     assert q.STATUS[e.value.status] == "QLIN_ERR_ALIGN"
 
 
+def test_offq_argument_errors(q):
+    """OffQ shapes, signs and sizes are checked on the host before anything
+    is enqueued."""
+    import numpy as np
+    from quantized_linear_layers_token_b200 import synth
+    d = synth.offq_signs(0)
+    assert q.qlin_offq_codes_bytes(256, 160) == 2 * 2 * 8192
+    assert q.qlin_offq_gemm_workspace(7, 256, 160) == 2 * 2 * 16384
+    assert q.qlin_offq_forward_workspace(7, 256, 160) > q.qlin_offq_gemm_workspace(7, 256, 160)
+    q.qlin_offq_quant_act(None, 0, 256, d, None, None, None, stream=0)  # M = 0: nothing to do
+    for K, N, status in [(200, 128, "QLIN_ERR_SHAPE"), (256, 120, "QLIN_ERR_SHAPE"), (0, 128, "QLIN_ERR_ARG"),
+                         (65536 + 128, 128, "QLIN_ERR_SHAPE")]:
+        with pytest.raises(q.QlinError) as e:
+            q.qlin_offq_codes_bytes(K, N)
+        assert q.STATUS[e.value.status] == status
+    bad = d.copy()
+    bad[0] = -1  # row 0 of D H must be all ones
+    half = d.copy()
+    half[5] = 0
+    for signs in (bad, half):
+        with pytest.raises(q.QlinError) as e:
+            q.qlin_offq_quant_act(1 << 24, 4, 256, signs, 1 << 25, 1 << 26, 1 << 27, stream=0)
+        assert q.STATUS[e.value.status] == "QLIN_ERR_ARG"
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_offq_quant_act((1 << 24) + 8, 4, 256, d, 1 << 25, 1 << 26, 1 << 27, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_ALIGN"
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_offq_gemm(1 << 24, 1 << 25, 1 << 26, 4, 256, 160, 1 << 27, 1 << 28, 1 << 29, 1 << 30, 1 << 31,
+                         16, stream=0)
+    assert q.STATUS[e.value.status] == "QLIN_ERR_WORKSPACE"
+    with pytest.raises(ValueError):
+        q.qlin_offq_quant_act(1 << 24, 4, 256, np.ones(64, np.int8), 1 << 25, 1 << 26, 1 << 27, stream=0)
+
+
 def test_binding_declares_every_entry_point(q):
     """Every entry point of the header has an argument list in the ctypes
     binding (so no call goes out with default int conversions)."""

@@ -22,6 +22,7 @@ MODES = [
     {"widen_min_m": 129},      # INT4 weights widened once, INT8 kernel, from 129 tokens
     {"widen_min_m": 0},        # INT4 converters in the GEMM for every token count
     {"pair_mma": 2, "widen_min_m": 129},  # CTA-pair GEMM for every 256-token tile with INT8 operands
+    {"pair_mma": 1, "widen_min_m": 1024},  # CTA pairs only from a full wave of pair tiles
     {"pair_mma": 0},           # one CTA per tile everywhere
 ]
 
