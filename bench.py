@@ -958,6 +958,79 @@ def run_profile_case(args, wl):
     return 0
 
 
+def run_profile_grouped(args, wl):
+    """grouped:M -- every linear of the workload (one weight copy) as one
+    qlin_forward_grouped call at M <= 64 tokens, launched eagerly (for ncu)."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    M = int(args.profile_case.split(":")[1])
+    layers, Xs, ss, Ys = [], [], [], []
+    for si, (_, K, N) in enumerate(wl.shapes):
+        L = synth.layer(wl, si, M=M)
+        layers.append(qlin.PackedLayer.pack(torch.from_numpy(L["W"]).cuda(), L["O"], wl.fmt))
+        Xs.append(torch.from_numpy(L["X"]).cuda())
+        ss.append(torch.ones(max(len(L["O"]), 1), dtype=torch.float32, device="cuda"))
+        Ys.append(torch.empty((M, N), dtype=torch.float16, device="cuda"))
+    ws = [l.w for l in layers]
+    n = qlin.qlin_forward_grouped_workspace(ws, M)
+    wsp = qlin.empty_workspace(n)
+    for _ in range(args.warmup):
+        qlin.qlin_forward_grouped(ws, Xs, ss, Ys, M, wl.gamma, True, wsp, n)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        qlin.qlin_forward_grouped(ws, Xs, ss, Ys, M, wl.gamma, True, wsp, n)
+    e1.record()
+    torch.cuda.synchronize()
+    qlin.qlin_poll_device_status()
+    us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
+    nbytes = sum(layer_bytes(M, K, N, l.n_outlier, wl.fmt) for (_, K, N), l in zip(wl.shapes, layers))
+    print(json.dumps({"profile_case": args.profile_case, "workload": wl.name, "M": M, "problems": len(ws),
+                      "us_per_call_eager": us, "algorithmic_bytes": nbytes,
+                      "gbs": nbytes / (us * 1e-6) / 1e9}), flush=True)
+    return 0
+
+
+def run_profile_offq(args):
+    """offq:NAME:M -- W warm-up and K timed qlin_offq_forward calls on one
+    Llama-3-8B linear, launched eagerly (for ncu)."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    _, name, m = args.profile_case.split(":")
+    M = int(m)
+    i = [n for n, _, _ in OFFQ_LAYERS].index(name)
+    _, K, N = OFFQ_LAYERS[i]
+    d = synth.offq_signs(0)
+    X = torch.from_numpy(synth.offq_activations(M, K, seed=K).view(np.uint16)).cuda()
+    W = torch.from_numpy(synth.offq_weights(K, N, seed=i).view(np.uint16)).cuda()
+    codes = torch.zeros(qlin.qlin_offq_codes_bytes(K, N), dtype=torch.uint8, device="cuda")
+    cs = torch.zeros(N, dtype=torch.float32, device="cuda")
+    colsum = torch.zeros((K // 128, N), dtype=torch.float32, device="cuda")
+    Wr = torch.empty((K, N), dtype=torch.float32, device="cuda")
+    qlin.qlin_offq_pack(W, K, N, d, codes, cs, colsum, Wr)
+    del Wr
+    Y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    n = qlin.qlin_offq_forward_workspace(M, K, N)
+    ws = qlin.empty_workspace(n)
+    for _ in range(args.warmup):
+        qlin.qlin_offq_forward(X, M, K, N, d, codes, cs, colsum, Y, ws, n)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        qlin.qlin_offq_forward(X, M, K, N, d, codes, cs, colsum, Y, ws, n)
+    e1.record()
+    torch.cuda.synchronize()
+    qlin.qlin_poll_device_status()
+    us = e0.elapsed_time(e1) * 1e3 / max(args.steps, 1)
+    print(json.dumps({"profile_case": args.profile_case, "K": K, "N": N, "M": M, "us_per_forward_eager": us,
+                      "tops": 2 * M * K * N / (us * 1e-6) / 1e12}), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------------------
 # our arm: the forward step
 # ---------------------------------------------------------------------------
@@ -1219,7 +1292,8 @@ def main():
                     help="backward: the input gradient of every linear (default workload phi3_w8_quaff)")
     ap.add_argument("--tokens", type=int, default=4096, help="--op backward: tokens per step")
     ap.add_argument("--profile-case", default=None,
-                    help="NAME:M -- run only that linear of the workload at M tokens (for ncu captures)")
+                    help="NAME:M -- run only that linear of the workload at M tokens (for ncu captures); "
+                         "offq:NAME:M -- one OffQ linear of the Llama-3-8B set")
     args = ap.parse_args()
     if args.op == "backward":
         wl = synth.WORKLOADS["phi3_w8_quaff" if args.workload == DEFAULT_WORKLOAD else args.workload]
@@ -1227,6 +1301,10 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.profile_case and args.profile_case.startswith("offq:"):
+        return run_profile_offq(args)
+    if args.profile_case and args.profile_case.startswith("grouped:"):
+        return run_profile_grouped(args, wl)
     if args.profile_case:
         return run_profile_case(args, wl)
     return run_forward(args, wl)

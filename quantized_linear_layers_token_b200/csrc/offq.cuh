@@ -47,7 +47,11 @@
 //                        product per 128-wide K-block into its own tensor-memory
 //                        accumulator (four in flight); the epilogue promotes
 //                        each block with the group's token scale and offset
-//                        into fp32 registers, then applies c_n / 16.
+//                        into fp32 registers, then applies c_n / 16.  Each
+//                        epilogue warp streams its 64 column sums per block
+//                        through a private three-slot cp.async ring and
+//                        loads the token scales and offsets two blocks ahead,
+//                        so no promotion waits on a global load.
 #pragma once
 
 #include "gemm.cuh"
@@ -214,7 +218,9 @@ constexpr int kOffqStage = 32768;  // 16 KB token rows (A) + 16 KB weight rows (
 constexpr int kOffqAccBufs = 4;    // 128-column accumulators in tensor memory
 constexpr int kOffqEpiWarps = 8;
 constexpr int kOffqThreads = 32 * (2 + kOffqEpiWarps);
-constexpr int kOffqOffBar = kOffqStages * kOffqStage;
+constexpr int kOffqCsSlots = 3;  // per epilogue warp: column sums of 64 channels per K-block
+constexpr int kOffqOffCs = kOffqStages * kOffqStage;
+constexpr int kOffqOffBar = kOffqOffCs + kOffqEpiWarps * kOffqCsSlots * 256;
 constexpr int kOffqSmem = kOffqOffBar + 256 + 1024;  // barriers + alignment slack
 
 struct OffqArgs {
@@ -233,14 +239,6 @@ struct alignas(64) OffqParams {
   OffqArgs g;
 };
 
-// Exact int32 -> fp32 for |v| < 2^22: the integer lands in the mantissa of
-// 1.5 * 2^23, and subtracting that constant is exact.  The accumulators of
-// one K-block stay below 128 * 15 * 112 = 215040 in magnitude.
-__device__ __forceinline__ float small_int_to_float(uint32_t v) {
-  return __fsub_rn(__int_as_float(static_cast<int>(v) + 0x4B400000), 12582912.f);
-}
-
-template <int CVT>
 __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid_constant__ OffqParams prm) {
   const OffqArgs& g = prm.g;
   constexpr int S = kOffqStages;
@@ -348,6 +346,7 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
     const int quad = warp & 3;         // tensor-memory lanes 32*quad .. +31
     const int row = quad * 32 + lane;  // token within the tile
     const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(half * 64);
+    float* csr = reinterpret_cast<float*>(smem + kOffqOffCs + ep * kOffqCsSlots * 256);  // this warp's ring
     griddep_wait();
     int it = 0;
     bool ok = true;
@@ -356,18 +355,33 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
       const int m = tm * 128 + row;
       const bool mv = m < g.M;
       const int nb = tn * 128 + half * 64;
+      // column sums of K-block kb into ring slot kb % 3: 16 lanes x 16 bytes
+      // (a lane past N reads an in-range chunk; those columns are not stored)
+      const int cn = min(nb + 4 * (lane & 15), g.N - 4);
+      auto fetch_cs = [&](int kb) {
+        if (kb < g.G && lane < 16)
+          cp_async16(csr + (kb % kOffqCsSlots) * 64 + 4 * lane, g.colsum + static_cast<size_t>(kb) * g.N + cn);
+        cp_async_commit();
+      };
+      fetch_cs(0);
+      fetch_cs(1);
       const float* sdp = g.scale + static_cast<size_t>(mv ? m : 0) * g.G;
       const float* lop = g.offset + static_cast<size_t>(mv ? m : 0) * g.G;
       float sum[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) sum[j] = 0.f;
-      float sd_n = mv ? __ldg(sdp) : 0.f, lo_n = mv ? __ldg(lop) : 0.f;
+      // token scale and offset two K-blocks ahead
+      float sd1 = mv ? __ldg(sdp) : 0.f, lo1 = mv ? __ldg(lop) : 0.f;
+      float sd2 = (mv && g.G > 1) ? __ldg(sdp + 1) : 0.f, lo2 = (mv && g.G > 1) ? __ldg(lop + 1) : 0.f;
       for (int kb = 0; kb < g.G; ++kb, ++it) {
-        const float sd = sd_n, lo = lo_n;
-        if (mv && kb + 1 < g.G) {
-          sd_n = __ldg(sdp + kb + 1);
-          lo_n = __ldg(lop + kb + 1);
+        const float sd = sd1, lo = lo1;
+        sd1 = sd2;
+        lo1 = lo2;
+        if (mv && kb + 2 < g.G) {
+          sd2 = __ldg(sdp + kb + 2);
+          lo2 = __ldg(lop + kb + 2);
         }
+        fetch_cs(kb + 2);
         const int b = it % B;
         ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], static_cast<uint32_t>(it / B) & 1u, abort_flag));
         if (!ok) break;
@@ -377,21 +391,24 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
         tmem_ld32(trow + 128u * b + 32u, v + 32);
         tmem_ld_wait();
         tc_fence_before();
+        cp_async_wait_group<2>();  // this K-block's column sums have landed
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        const float4* csp = reinterpret_cast<const float4*>(g.colsum + static_cast<size_t>(kb) * g.N + nb);
+        const float4* cs4 = reinterpret_cast<const float4*>(csr + (kb % kOffqCsSlots) * 64);
 #pragma unroll
         for (int j4 = 0; j4 < 16; ++j4) {
-          const float4 c4 = nb + 4 * j4 < g.N ? __ldg(csp + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 c4 = cs4[j4];
           const float cs[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = 4 * j4 + e;
-            const float a = CVT == 0 ? small_int_to_float(v[j]) : __int2float_rn(static_cast<int>(v[j]));
-            sum[j] = __fmaf_rn(sd, a, __fmaf_rn(lo, cs[e], sum[j]));
+            sum[j] = __fmaf_rn(sd, __int2float_rn(static_cast<int>(v[j])), __fmaf_rn(lo, cs[e], sum[j]));
           }
         }
+        __syncwarp();  // every lane has read the slot before it is refilled
       }
+      cp_async_wait_all();
+      __syncwarp();
       if (!ok) break;
       if (mv) {
 #pragma unroll
@@ -400,12 +417,12 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
           if (n < g.N) {
             const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.cscale + n));
             const float4 c1 = __ldg(reinterpret_cast<const float4*>(g.cscale + n) + 1);
-            const float cn[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const float cnv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
             uint32_t h[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float y0 = __fmul_rn(__fmul_rn(cn[2 * e], 0.0625f), sum[8 * j8 + 2 * e]);
-              const float y1 = __fmul_rn(__fmul_rn(cn[2 * e + 1], 0.0625f), sum[8 * j8 + 2 * e + 1]);
+              const float y0 = __fmul_rn(__fmul_rn(cnv[2 * e], 0.0625f), sum[8 * j8 + 2 * e]);
+              const float y1 = __fmul_rn(__fmul_rn(cnv[2 * e + 1], 0.0625f), sum[8 * j8 + 2 * e + 1]);
               h[e] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y0))) |
                      (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(y1))) << 16);
             }
@@ -414,6 +431,7 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
         }
       }
     }
+    cp_async_wait_all();
   }
   tc_fence_before();
   __syncthreads();
