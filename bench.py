@@ -95,6 +95,40 @@ def algorithmic_bytes(M, K, N, nO, fmt):
     return gemm, act
 
 
+TRAFFIC_SOURCES = ("quantized_linear_layers_token_b200/csrc/gemm.cuh",
+                   "quantized_linear_layers_token_b200/csrc/gemm_pair.cuh",
+                   "quantized_linear_layers_token_b200/csrc/sm100.cuh",
+                   "quantized_linear_layers_token_b200/csrc/qlin.cu")
+
+
+def gemm_sources_sha256():
+    """sha256 of the GEMM sources with // comments and blank lines removed, so
+    a recorded DRAM-traffic figure is used only while the code it was taken
+    on is unchanged."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel)) as f:
+            for line in f:
+                line = re.sub(r"//.*", "", line).rstrip()
+                if line:
+                    h.update(line.encode() + b"\n")
+    return h.hexdigest()
+
+
+def recorded_traffic(workload):
+    """DRAM bytes of the headline roofline's launch set from the ncu capture
+    recorded under profiles/, or None if there is none for these sources."""
+    p = os.path.join(ROOT, "profiles", f"gemm_traffic_{workload}.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d if d.get("sources_sha256") == gemm_sources_sha256() else None
+    except Exception:
+        return None
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -958,6 +992,35 @@ def run_profile_case(args, wl):
     return 0
 
 
+def run_profile_tensor_buckets(args, wl):
+    """tensor-buckets -- one qlin_forward per linear at each token count of
+    the workload's tensor-bound buckets (the launch set of the headline
+    roofline), eager and in order, for an ncu DRAM-traffic capture."""
+    import torch
+    from quantized_linear_layers_token_b200 import qlin
+    peaks = read_peaks()
+    ms = [M for M in wl.ms if roofline_of(2 * M * sum(K * N for _, K, N in wl.shapes),
+                                          sum(layer_bytes(M, K, N, 0, wl.fmt) for _, K, N in wl.shapes),
+                                          1.0, peaks)["bound"] == "tensor"]
+    for M in ms:
+        for si, (name, K, N) in enumerate(wl.shapes):
+            L = synth.layer(wl, si, M=M)
+            layer = qlin.PackedLayer.pack(torch.from_numpy(L["W"]).cuda(), L["O"], wl.fmt)
+            X = torch.from_numpy(L["X"]).cuda()
+            s = torch.ones(max(len(L["O"]), 1), dtype=torch.float32, device="cuda")
+            Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            nws = qlin.qlin_forward_workspace(M, layer.w)
+            ws = qlin.empty_workspace(nws)
+            qlin.qlin_forward(X, M, layer.w, s, wl.gamma, True, Y, ws, nws)
+            torch.cuda.synchronize()
+            del layer, X, Y, ws
+            torch.cuda.empty_cache()
+    qlin.qlin_poll_device_status()
+    print(json.dumps({"profile_case": "tensor-buckets", "workload": wl.name, "M": ms,
+                      "linears": [n for n, _, _ in wl.shapes]}), flush=True)
+    return 0
+
+
 def run_profile_grouped(args, wl):
     """grouped:M -- every linear of the workload (one weight copy) as one
     qlin_forward_grouped call at M <= 64 tokens, launched eagerly (for ncu)."""
@@ -1130,12 +1193,15 @@ def run_forward(args, wl):
             g_ops = sum(b["ops"] for b in tb)
             g_bytes = sum(b["gemm"]["algorithmic_bytes"] for b in tb)
             roofline = roofline_of(g_ops, g_bytes, g_ms * 1e-3, peaks)
+            tr = recorded_traffic(wl.name)
             roofline.update({
                 "kernel": "qlin_gemm (INT4 widened once per call, then the tcgen05 INT8 GEMM with the fused "
                           "dequant and compensation), all calls of the buckets M in "
                           f"{[b['M'] for b in tb]}, one stream",
                 "ms": g_ms, "launches": sum(b["gemm"]["launches"] for b in tb),
-                "ops": g_ops, "algorithmic_bytes": g_bytes, "traffic": None,
+                "ops": g_ops, "algorithmic_bytes": g_bytes,
+                "traffic": tr["dram_bytes"] if tr else None,
+                "traffic_source": tr["how"] if tr else "no capture recorded for these GEMM sources",
                 "timing": f"sum over the buckets of the median of {reps} CUDA-graph replays"})
 
         # ------------------------------------------------------------ end to end through the API
@@ -1305,6 +1371,8 @@ def main():
         return run_profile_offq(args)
     if args.profile_case and args.profile_case.startswith("grouped:"):
         return run_profile_grouped(args, wl)
+    if args.profile_case and args.profile_case.startswith("tensor-buckets"):
+        return run_profile_tensor_buckets(args, wl)
     if args.profile_case:
         return run_profile_case(args, wl)
     return run_forward(args, wl)

@@ -140,11 +140,14 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
 
 // What one converter thread reads from global memory for one step: its code
 // chunk(s), the channel scale and (g128) the group ratio of its row.
+constexpr int kBwdOvPre = 8;  // outlier inputs per window whose blended values are loaded ahead
+
 template <int FMT>
 struct BwdIn {
   uint4 w[FMT == kFmtW8 ? 2 : 1];
   float c;     // c_n, 0 beyond N
   uint16_t r;  // g128: r[kb][n] bits, 0 for an absent block or channel
+  uint32_t ov[kBwdOvPre / 2];  // blended rows of the window's first outlier inputs (fp16 pairs)
 };
 
 // Step j, channel row nl, 32-input window g of the tile whose first code
@@ -369,6 +372,21 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       wb0 += kl < 32 * g ? 1 : 0;
       wb1 += kl < 32 * g + 32 ? 1 : 0;
     }
+    // the blended values of the window's first outlier inputs for step j
+    auto load_ov = [&](BwdIn<FMT>& in, int j) {
+      const int n = j * 64 + nl;
+#pragma unroll
+      for (int u = 0; u < kBwdOvPre; u += 2) {
+        uint32_t lo16 = 0u, hi16 = 0u;
+        if (n < args.N && wb0 + u < wb1)
+          lo16 = __ldg(args.weffo + static_cast<size_t>(lo + wb0 + u) * args.N + n);
+        if (n < args.N && wb0 + u + 1 < wb1)
+          hi16 = __ldg(args.weffo + static_cast<size_t>(lo + wb0 + u + 1) * args.N + n);
+        in.ov[u >> 1] = lo16 | (hi16 << 16);
+      }
+    };
+    load_ov(in0, j0);
+    if (nst > 1) load_ov(in1, j0 + 1);
 
     bool ok = true;
     // jj counts this CTA's steps, j = j0 + jj is the channel step
@@ -429,13 +447,22 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
         }
       }
-      if (jj + 2 < nst) load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
       const int n = j * 64 + nl;
       if (wb1 > wb0 && n < args.N) {
-        // outlier inputs of this window: Weff[O_i][n] from the blended rows
-        // (every lane of the warp has the same entries: no divergence)
+        // outlier inputs of this window: Weff[O_i][n] from the blended rows,
+        // the first kBwdOvPre loaded two steps ahead (every lane of the warp
+        // has the same entries: no divergence)
+#pragma unroll
+        for (int u = 0; u < kBwdOvPre; ++u)
+          if (wb0 + u < wb1)
+            *outlier_elem(bt, outl[wb0 + u], nl) = static_cast<uint16_t>(in.ov[u >> 1] >> (16 * (u & 1)));
         const uint16_t* src = args.weffo + static_cast<size_t>(lo) * args.N + n;
-        for (int e = wb0; e < wb1; ++e) *outlier_elem(bt, outl[e], nl) = __ldg(src + static_cast<size_t>(e) * args.N);
+        for (int e = wb0 + kBwdOvPre; e < wb1; ++e)
+          *outlier_elem(bt, outl[e], nl) = __ldg(src + static_cast<size_t>(e) * args.N);
+      }
+      if (jj + 2 < nst) {
+        load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
+        load_ov(in, j + 2);
       }
       fence_proxy_async_smem();
       __syncwarp();

@@ -47,8 +47,9 @@
 //                        product per 128-wide K-block into its own tensor-memory
 //                        accumulator (four in flight); the epilogue promotes
 //                        each block with the group's token scale and offset
-//                        into fp32 registers, then applies c_n / 16.  Each
-//                        epilogue warp streams its 64 column sums per block
+//                        into fp32 registers, then applies c_n / 16 (sixteen
+//                        epilogue warps, 32 columns each).  Each
+//                        epilogue warp streams its column sums per block
 //                        through a private three-slot cp.async ring and
 //                        loads the token scales and offsets two blocks ahead,
 //                        so no promotion waits on a global load.
@@ -216,11 +217,12 @@ __global__ void offq_pack_kernel(const float* __restrict__ Wr, int K, int N, uin
 constexpr int kOffqStages = 6;
 constexpr int kOffqStage = 32768;  // 16 KB token rows (A) + 16 KB weight rows (B)
 constexpr int kOffqAccBufs = 4;    // 128-column accumulators in tensor memory
-constexpr int kOffqEpiWarps = 8;
+constexpr int kOffqEpiWarps = 16;  // four per TMEM lane quarter, 32 columns each
+constexpr int kOffqCols = 128 / (kOffqEpiWarps / 4);
 constexpr int kOffqThreads = 32 * (2 + kOffqEpiWarps);
 constexpr int kOffqCsSlots = 3;  // per epilogue warp: column sums of 64 channels per K-block
 constexpr int kOffqOffCs = kOffqStages * kOffqStage;
-constexpr int kOffqOffBar = kOffqOffCs + kOffqEpiWarps * kOffqCsSlots * 256;
+constexpr int kOffqOffBar = kOffqOffCs + kOffqEpiWarps * kOffqCsSlots * kOffqCols * 4;
 constexpr int kOffqSmem = kOffqOffBar + 256 + 1024;  // barriers + alignment slack
 
 struct OffqArgs {
@@ -342,11 +344,12 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
   } else {
     // ------------------------------------------------------------ epilogue
     const int ep = warp - 2;
-    const int half = ep >> 2;          // columns 64*half .. +63 of each accumulator
+    constexpr int C = kOffqCols;
+    const int part = ep >> 2;          // columns C*part .. +C-1 of each accumulator
     const int quad = warp & 3;         // tensor-memory lanes 32*quad .. +31
     const int row = quad * 32 + lane;  // token within the tile
-    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(half * 64);
-    float* csr = reinterpret_cast<float*>(smem + kOffqOffCs + ep * kOffqCsSlots * 256);  // this warp's ring
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(part * C);
+    float* csr = reinterpret_cast<float*>(smem + kOffqOffCs + ep * kOffqCsSlots * C * 4);  // this warp's ring
     griddep_wait();
     int it = 0;
     bool ok = true;
@@ -354,22 +357,23 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
       const int tm = t % g.tiles_m, tn = t / g.tiles_m;
       const int m = tm * 128 + row;
       const bool mv = m < g.M;
-      const int nb = tn * 128 + half * 64;
-      // column sums of K-block kb into ring slot kb % 3: 16 lanes x 16 bytes
-      // (a lane past N reads an in-range chunk; those columns are not stored)
-      const int cn = min(nb + 4 * (lane & 15), g.N - 4);
+      const int nb = tn * 128 + part * C;
+      // column sums of K-block kb into ring slot kb % 3: C / 4 lanes x 16
+      // bytes (a lane past N reads an in-range chunk; those columns are not
+      // stored)
+      const int cn = min(nb + 4 * (lane % (C / 4)), g.N - 4);
       auto fetch_cs = [&](int kb) {
-        if (kb < g.G && lane < 16)
-          cp_async16(csr + (kb % kOffqCsSlots) * 64 + 4 * lane, g.colsum + static_cast<size_t>(kb) * g.N + cn);
+        if (kb < g.G && lane < C / 4)
+          cp_async16(csr + (kb % kOffqCsSlots) * C + 4 * lane, g.colsum + static_cast<size_t>(kb) * g.N + cn);
         cp_async_commit();
       };
       fetch_cs(0);
       fetch_cs(1);
       const float* sdp = g.scale + static_cast<size_t>(mv ? m : 0) * g.G;
       const float* lop = g.offset + static_cast<size_t>(mv ? m : 0) * g.G;
-      float sum[64];
+      float sum[C];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) sum[j] = 0.f;
+      for (int j = 0; j < C; ++j) sum[j] = 0.f;
       // token scale and offset two K-blocks ahead
       float sd1 = mv ? __ldg(sdp) : 0.f, lo1 = mv ? __ldg(lop) : 0.f;
       float sd2 = (mv && g.G > 1) ? __ldg(sdp + 1) : 0.f, lo2 = (mv && g.G > 1) ? __ldg(lop + 1) : 0.f;
@@ -386,17 +390,17 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
         ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], static_cast<uint32_t>(it / B) & 1u, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        uint32_t v[64];
-        tmem_ld32(trow + 128u * b, v);
-        tmem_ld32(trow + 128u * b + 32u, v + 32);
+        uint32_t v[C];
+#pragma unroll
+        for (int c = 0; c < C; c += 32) tmem_ld32(trow + 128u * b + c, v + c);
         tmem_ld_wait();
         tc_fence_before();
         cp_async_wait_group<2>();  // this K-block's column sums have landed
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        const float4* cs4 = reinterpret_cast<const float4*>(csr + (kb % kOffqCsSlots) * 64);
+        const float4* cs4 = reinterpret_cast<const float4*>(csr + (kb % kOffqCsSlots) * C);
 #pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
+        for (int j4 = 0; j4 < C / 4; ++j4) {
           const float4 c4 = cs4[j4];
           const float cs[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
@@ -412,7 +416,7 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
       if (!ok) break;
       if (mv) {
 #pragma unroll
-        for (int j8 = 0; j8 < 8; ++j8) {
+        for (int j8 = 0; j8 < C / 8; ++j8) {
           const int n = nb + 8 * j8;
           if (n < g.N) {
             const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.cscale + n));
