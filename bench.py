@@ -480,7 +480,11 @@ class ForwardWorkload:
             del g
             gbytes = sum(algorithmic_bytes(M, self.meta[sl["si"]]["K"], self.meta[sl["si"]]["N"],
                                            self.meta[sl["si"]]["nO"], self.wl.fmt)[0] for sl, *_ in gsl)
-            rec["gemm"] = {"ms": gms, "launches": len(gsl), "algorithmic_bytes": gbytes,
+            # qlin_gemm: the compensation operand (layers with outliers), the
+            # widening of INT4 weights (from 512 tokens), the GEMM
+            widen = 1 if (self.wl.fmt != synth.W8_PERCHANNEL and M >= 512) else 0
+            nl = sum(1 + widen + (1 if self.meta[sl["si"]]["nO"] > 0 else 0) for sl, *_ in gsl)
+            rec["gemm"] = {"ms": gms, "calls": len(gsl), "launches": nl, "algorithmic_bytes": gbytes,
                            "roofline": roofline_of(ops, gbytes, gms * 1e-3, peaks)}
             q.qlin_poll_device_status(stream)
             out.append(rec)

@@ -47,9 +47,10 @@
 //                        product per 128-wide K-block into its own tensor-memory
 //                        accumulator (four in flight); the epilogue promotes
 //                        each block with the group's token scale and offset
-//                        into fp32 registers, then applies c_n / 16 (sixteen
-//                        epilogue warps, 32 columns each).  Each
-//                        epilogue warp streams its column sums per block
+//                        into fp32 registers, then applies c_n / 16 (eight
+//                        epilogue warps of 64 columns, read as two halves
+//                        whose loads overlap the other half's promotion).
+//                        Each epilogue warp streams its column sums per block
 //                        through a private three-slot cp.async ring and
 //                        loads the token scales and offsets two blocks ahead,
 //                        so no promotion waits on a global load.
@@ -217,7 +218,7 @@ __global__ void offq_pack_kernel(const float* __restrict__ Wr, int K, int N, uin
 constexpr int kOffqStages = 6;
 constexpr int kOffqStage = 32768;  // 16 KB token rows (A) + 16 KB weight rows (B)
 constexpr int kOffqAccBufs = 4;    // 128-column accumulators in tensor memory
-constexpr int kOffqEpiWarps = 16;  // four per TMEM lane quarter, 32 columns each
+constexpr int kOffqEpiWarps = 8;  // two per TMEM lane quarter, 64 columns each
 constexpr int kOffqCols = 128 / (kOffqEpiWarps / 4);
 constexpr int kOffqThreads = 32 * (2 + kOffqEpiWarps);
 constexpr int kOffqCsSlots = 3;  // per epilogue warp: column sums of 64 channels per K-block
@@ -235,6 +236,23 @@ struct OffqArgs {
   int M, N, G;
   int tiles_m, tiles;
 };
+
+// sum[J0 + j] += sd * acc[j] + lo * colsum[j] for 32 columns (fp32, the
+// offset term first, both fused multiply-adds rounded once).
+template <int J0>
+__device__ __forceinline__ void offq_promote(const uint32_t (&v)[32], float (&sum)[64], float sd, float lo,
+                                             const float4* cs4) {
+#pragma unroll
+  for (int j4 = 0; j4 < 8; ++j4) {
+    const float4 c4 = cs4[j4];
+    const float cs[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * j4 + e;
+      sum[J0 + j] = __fmaf_rn(sd, __int2float_rn(static_cast<int>(v[j])), __fmaf_rn(lo, cs[e], sum[J0 + j]));
+    }
+  }
+}
 
 struct alignas(64) OffqParams {
   CUtensorMap tmX;  // q int8 [M][K], 128 x 128 boxes, 128-byte swizzle
@@ -343,13 +361,16 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // Per K-block the two 32-column halves of this warp's accumulator slice
+    // are read alternately with their promotion: the load of one half (or of
+    // the next block's first half) is in flight while the other is promoted.
+    static_assert(kOffqCols == 64, "the epilogue reads 64 columns as two halves");
     const int ep = warp - 2;
-    constexpr int C = kOffqCols;
-    const int part = ep >> 2;          // columns C*part .. +C-1 of each accumulator
+    const int part = ep >> 2;          // columns 64*part .. +63 of each accumulator
     const int quad = warp & 3;         // tensor-memory lanes 32*quad .. +31
     const int row = quad * 32 + lane;  // token within the tile
-    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(part * C);
-    float* csr = reinterpret_cast<float*>(smem + kOffqOffCs + ep * kOffqCsSlots * C * 4);  // this warp's ring
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(part * 64);
+    float* csr = reinterpret_cast<float*>(smem + kOffqOffCs + ep * kOffqCsSlots * 256);  // this warp's ring
     griddep_wait();
     int it = 0;
     bool ok = true;
@@ -357,27 +378,33 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
       const int tm = t % g.tiles_m, tn = t / g.tiles_m;
       const int m = tm * 128 + row;
       const bool mv = m < g.M;
-      const int nb = tn * 128 + part * C;
-      // column sums of K-block kb into ring slot kb % 3: C / 4 lanes x 16
-      // bytes (a lane past N reads an in-range chunk; those columns are not
-      // stored)
-      const int cn = min(nb + 4 * (lane % (C / 4)), g.N - 4);
-      auto fetch_cs = [&](int kb) {
-        if (kb < g.G && lane < C / 4)
-          cp_async16(csr + (kb % kOffqCsSlots) * C + 4 * lane, g.colsum + static_cast<size_t>(kb) * g.N + cn);
-        cp_async_commit();
-      };
-      fetch_cs(0);
-      fetch_cs(1);
+      const int nb = tn * 128 + part * 64;
+      // column sums of K-block kb into ring slot kb % 3: 16 lanes x 16 bytes
+      // (a lane past N reads an in-range chunk; those columns are not stored)
+      const float* csrc = g.colsum + min(nb + 4 * (lane & 15), g.N - 4);
+      if (lane < 16) cp_async16(csr + 4 * lane, csrc);
+      cp_async_commit();
+      if (lane < 16 && g.G > 1) cp_async16(csr + 64 + 4 * lane, csrc + g.N);
+      cp_async_commit();
       const float* sdp = g.scale + static_cast<size_t>(mv ? m : 0) * g.G;
       const float* lop = g.offset + static_cast<size_t>(mv ? m : 0) * g.G;
-      float sum[C];
+      float sum[64];
 #pragma unroll
-      for (int j = 0; j < C; ++j) sum[j] = 0.f;
+      for (int j = 0; j < 64; ++j) sum[j] = 0.f;
       // token scale and offset two K-blocks ahead
       float sd1 = mv ? __ldg(sdp) : 0.f, lo1 = mv ? __ldg(lop) : 0.f;
       float sd2 = (mv && g.G > 1) ? __ldg(sdp + 1) : 0.f, lo2 = (mv && g.G > 1) ? __ldg(lop + 1) : 0.f;
+      uint32_t v0[32], v1[32];
+      {
+        const int b = it % B;
+        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], static_cast<uint32_t>(it / B) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld32(trow + 128u * b, v0);
+        tmem_ld_wait();
+      }
       for (int kb = 0; kb < g.G; ++kb, ++it) {
+        const int b = it % B;
         const float sd = sd1, lo = lo1;
         sd1 = sd2;
         lo1 = lo2;
@@ -385,38 +412,39 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
           sd2 = __ldg(sdp + kb + 2);
           lo2 = __ldg(lop + kb + 2);
         }
-        fetch_cs(kb + 2);
-        const int b = it % B;
-        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], static_cast<uint32_t>(it / B) & 1u, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t v[C];
-#pragma unroll
-        for (int c = 0; c < C; c += 32) tmem_ld32(trow + 128u * b + c, v + c);
-        tmem_ld_wait();
+        if (lane < 16 && kb + 2 < g.G)
+          cp_async16(csr + ((kb + 2) % kOffqCsSlots) * 64 + 4 * lane, csrc + static_cast<size_t>(kb + 2) * g.N);
+        cp_async_commit();
+        tmem_ld32(trow + 128u * b + 32u, v1);  // second half of this block
+        cp_async_wait_group<2>();              // this block's column sums have landed
+        __syncwarp();
+        const float4* cs4 = reinterpret_cast<const float4*>(csr + (kb % kOffqCsSlots) * 64);
+        offq_promote<0>(v0, sum, sd, lo, cs4);
+        tmem_ld_wait();  // the block is read: release its accumulator
         tc_fence_before();
-        cp_async_wait_group<2>();  // this K-block's column sums have landed
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
-        const float4* cs4 = reinterpret_cast<const float4*>(csr + (kb % kOffqCsSlots) * C);
-#pragma unroll
-        for (int j4 = 0; j4 < C / 4; ++j4) {
-          const float4 c4 = cs4[j4];
-          const float cs[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * j4 + e;
-            sum[j] = __fmaf_rn(sd, __int2float_rn(static_cast<int>(v[j])), __fmaf_rn(lo, cs[e], sum[j]));
+        const bool more = kb + 1 < g.G;
+        if (more) {
+          const int b1 = (it + 1) % B;
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&acc_full[b1], static_cast<uint32_t>((it + 1) / B) & 1u, abort_flag));
+          if (ok) {
+            tc_fence_after();
+            tmem_ld32(trow + 128u * b1, v0);  // the next block's first half
           }
         }
-        __syncwarp();  // every lane has read the slot before it is refilled
+        offq_promote<32>(v1, sum, sd, lo, cs4 + 8);
+        if (more && ok) tmem_ld_wait();
+        __syncwarp();  // every lane has read the ring slot before it is refilled
+        if (!ok) break;
       }
       cp_async_wait_all();
       __syncwarp();
       if (!ok) break;
       if (mv) {
 #pragma unroll
-        for (int j8 = 0; j8 < C / 8; ++j8) {
+        for (int j8 = 0; j8 < 8; ++j8) {
           const int n = nb + 8 * j8;
           if (n < g.N) {
             const float4 c0 = __ldg(reinterpret_cast<const float4*>(g.cscale + n));
