@@ -288,19 +288,13 @@ QLIN_API qlin_status qlin_forward_grouped(int32_t count, const qlin_weights* con
  *   s   fp32 [n_outlier], device: the scales of the forward pass whose
  *       gradient this is (ignored and may be NULL when n_outlier = 0).
  *   dX  fp16 [M][K] row-major, device, fully overwritten.
- *   workspace  256-byte aligned; it starts with the blended outlier rows
- *       of Weff (fp16 [n_outlier][N], computed once per call from s), so a
- *       layer with outliers needs at least 2 * n_outlier * N bytes rounded
- *       up to a multiple of 256 (QLIN_ERR_WORKSPACE otherwise); a layer
- *       without outliers may pass NULL.  With the whole
- *       qlin_backward_dx_workspace size, the tiles of an incomplete last
- *       wave of SMs are also split along the reduction and their fp32
- *       partials pass through it; it must then be zero-filled before its
- *       first use and is left that way.
+ *   workspace  optional (NULL, or smaller than qlin_backward_dx_workspace):
+ *       with it, the tiles of an incomplete last wave of SMs are split along
+ *       the reduction and their fp32 partials pass through it; it must be
+ *       zero-filled before its first use and is left that way.
  * Arithmetic: Weff is rounded to fp16 (the outlier rows after blending in
- * fp32: fma(s_i - 1, W_O, fp16(c'_n B)) * rcp(s_i)), products are summed in
- * fp32 on the tensor cores (split tiles add their fp32 partials), dX is
- * rounded to fp16 once.  M = 0 is a no-op; M
+ * fp32), products are summed in fp32 on the tensor cores (split tiles add
+ * their fp32 partials), dX is rounded to fp16 once.  M = 0 is a no-op; M
  * above 65535 * 128 returns QLIN_ERR_SHAPE; pointers must be 16-byte aligned
  * and the workspace 256-byte aligned (QLIN_ERR_ALIGN). */
 QLIN_API qlin_status qlin_backward_dx_workspace(int32_t M, const qlin_weights* w, size_t* bytes);

@@ -28,18 +28,15 @@
 //       the conversion needs no transpose;
 //   warp 1 issues eight 128 x 256 x 16 MMAs per step (each B slice serves
 //   both 128-token halves, so a code block is converted once per 256 tokens).
-// The blended outlier rows of Weff depend on s only, not on the tokens:
-// outlier_rows_kernel computes them once per call, [n_O][N] fp16 in the
-// workspace, with exactly the converters' roundings; a converter thread whose
-// window holds outlier inputs overwrites those elements of its own row with
-// them (no barrier: the thread's own stores).  The converter warps finally
-// read the accumulators back and store fp16 dX rows.  When the grid is under two waves, the tiles of
+// In a tile with outliers, all converter threads then blend the outlier rows
+// into B (after one barrier per step), with the W_O values streamed into a
+// shared ring by warp 2.  The converter warps finally read the accumulators
+// back and store fp16 dX rows.  When the grid is under two waves, the tiles of
 // the last, incomplete wave are split into ranges of the channel steps whose
 // fp32 partials meet in a workspace.
 #pragma once
 
 #include "gemm.cuh"
-#include "pack.cuh"
 
 namespace qlin {
 
@@ -47,7 +44,6 @@ struct BwdArgs {
   const uint8_t* codes;   // tiled packed codes (the weights' own layout)
   const uint16_t* rfold;  // g128 ratios r [K/128][N] fp16
   const uint16_t* wot;    // tiled W_O^T (16 KiB swizzled blocks of 128 channels x 64 outliers)
-  const uint16_t* weffo;  // blended outlier rows of Weff, fp16 [nO][N] (outlier_rows_kernel)
   const float* cscale;    // c_n [N]
   const int32_t* oidx;    // O [nO], strictly increasing
   const float* s;         // s [nO]
@@ -72,15 +68,28 @@ struct BwdArgs {
 template <int FMT>
 struct BwdCfg {
   static constexpr bool kW4 = FMT != kFmtW8;
+  // W_O ring: for each step, the W_O^T row segments (16-byte chunks) that
+  // hold the tile's first kWMax outliers, 64 channel rows of kWChunks chunks
+  static constexpr int kWR = 4;                   // steps in flight
+  static constexpr int kWMax = 32;                // outliers served from the ring
+  static constexpr int kWChunks = 5;              // chunks spanned by 32 consecutive outliers, at most
+  static constexpr int kWRow = 16 * kWChunks;     // 80 bytes per channel row
+  static constexpr int kWSlot = 64 * kWRow;
   static constexpr int kASlots = 3;               // dY tiles
   static constexpr int kBSlots = 3;               // Weff tiles
+  // A converter warp starts step j only after every warp has finished step
+  // j - kBSlots (its B slot must be free), so all warps stay within kBSlots
+  // steps of each other, and at least one warp waits for each ring fill; with
+  // more ring slots than that, arrivals for one slot never mix two steps.
+  static_assert(kWR > kBSlots, "the W_O ring must be deeper than the B ring");
   static constexpr int kABytes = 256 * 64 * 2;    // 32 KiB: 256 tokens x 64 channels
   static constexpr int kBBytes = 256 * 64 * 2;    // 32 KiB
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kASlots * kABytes;
   static constexpr int kOffOut = kOffB + kBSlots * kBBytes;
   static constexpr int kMaxOut = 256;             // outliers among 256 inputs, at most
-  static constexpr int kOffBar = kOffOut + kMaxOut * 16;
+  static constexpr int kOffW = kOffOut + kMaxOut * 16;
+  static constexpr int kOffBar = kOffW + kWR * kWSlot;
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + slack to 1024-align the base
   static constexpr int kConvWarps = 16;
   static constexpr int kThreads = 32 * (3 + kConvWarps);
@@ -140,14 +149,11 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int v) {
 
 // What one converter thread reads from global memory for one step: its code
 // chunk(s), the channel scale and (g128) the group ratio of its row.
-constexpr int kBwdOvPre = 8;  // outlier inputs per window whose blended values are loaded ahead
-
 template <int FMT>
 struct BwdIn {
   uint4 w[FMT == kFmtW8 ? 2 : 1];
   float c;     // c_n, 0 beyond N
   uint16_t r;  // g128: r[kb][n] bits, 0 for an absent block or channel
-  uint32_t ov[kBwdOvPre / 2];  // blended rows of the window's first outlier inputs (fp16 pairs)
 };
 
 // Step j, channel row nl, 32-input window g of the tile whose first code
@@ -186,50 +192,17 @@ __device__ __forceinline__ void load_step(BwdIn<FMT>& in, const BwdArgs& a, int 
 constexpr uint32_t kBwdLbo = 1024;  // next 64 inputs
 constexpr uint32_t kBwdSbo = 4096;  // next 8 channels
 
-// Element (input kl of the tile, channel q of the step) of a B tile.
-__device__ __forceinline__ uint16_t* outlier_elem(unsigned char* bt, int kl, int q) {
-  return reinterpret_cast<uint16_t*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
-                                     ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
+// Blend one outlier row element of a B tile: channel q of the step, outlier
+// entry o = {input - k0, i, s_i - 1, 1 / s_i}, w = W_O[i][n] (fp16 bits).
+__device__ __forceinline__ __half* outlier_elem(unsigned char* bt, int kl, int q) {
+  return reinterpret_cast<__half*>(bt + (q >> 3) * kBwdSbo + (kl >> 6) * kBwdLbo + (q & 7) * 128 +
+                                   ((((kl & 63) >> 3) ^ (q & 7)) << 4) + (kl & 7) * 2);
 }
 
-// Weff[O_i][n] = fp16((c'_n B[O_i][n] + (s_i - 1) W_O[i][n]) / s_i), with
-// c'_n B[O_i][n] the fp16 value the converters produce (the same unpacking,
-// requantisation and i8x4_scale_h2 rounding), the blend in fp32 as
-// fma(s_i - 1, W_O, that value) * rcp(s_i).  grid (ceil(N / 256), nO).
-template <int FMT>
-__global__ void __launch_bounds__(256) outlier_rows_kernel(const BwdArgs args, uint16_t* __restrict__ weffo) {
-  griddep_launch_dependents();
-  const int n = blockIdx.x * 256 + threadIdx.x;
-  const int i = blockIdx.y;
-  if (n >= args.N) return;
-  const int k = __ldg(args.oidx + i);
-  const int k8 = k & ~7;
-  const float c = __ldg(args.cscale + n);
-  const __half2 c2 = __float2half2_rn(FMT == kFmtW4PC ? __fmul_rn(c, 0.0625f) : c);
-  uint32_t lanes;  // the INT8 operand of inputs (k & ~3) .. +3
-  if (FMT == kFmtW8) {
-    lanes = __ldg(reinterpret_cast<const uint32_t*>(args.codes + w8_tile_offset(n, k8, args.kbs) + (k & 4)));
-  } else {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(args.codes + w4_tile_offset(n, k8, args.kbs)));
-    if (FMT == kFmtW4PC) {
-      lanes = (k & 4) ? (w & 0xF0F0F0F0u) : ((w << 4) & 0xF0F0F0F0u);
-    } else {
-      const __half2 r1 = __half2half2(__ushort_as_half(__ldg(args.rfold + static_cast<size_t>(k >> 7) * args.N + n)));
-      const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));
-      const uint2 q = requant_g128(w, r1, r16);
-      lanes = (k & 4) ? q.y : q.x;
-    }
-  }
-  uint32_t h01, h23;
-  i8x4_scale_h2(lanes, c2, h01, h23);
-  const uint16_t base = static_cast<uint16_t>(((k & 2) ? h23 : h01) >> (16 * (k & 1)));
-  const uint16_t wo = wot_elem(args, n, i);
-  griddep_wait();  // s comes from the forward; the previous call may still read this workspace
-  const float sv = args.s[i];
-  const float v = __fmul_rn(__fmaf_rn(__fsub_rn(sv, 1.f), __half2float(__ushort_as_half(wo)),
-                                      __half2float(__ushort_as_half(base))),
-                            __frcp_rn(sv));
-  weffo[static_cast<size_t>(i) * args.N + n] = __half_as_ushort(__float2half_rn(v));
+__device__ __forceinline__ void patch_outlier(unsigned char* bt, const float4 o, int q, uint16_t w) {
+  __half* p = outlier_elem(bt, __float_as_int(o.x), q);
+  const float v = __fmul_rn(__fmaf_rn(o.z, __half2float(__ushort_as_half(w)), __half2float(*p)), o.w);
+  *p = __float2half_rn(v);
 }
 
 template <int FMT>
@@ -244,9 +217,11 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
   uint64_t* bfull = aempty + AS;
   uint64_t* bempty = bfull + BS;
   uint64_t* acc_full = bempty + BS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* wfull = acc_full + 1;        // [kWR]
+  uint64_t* wempty = wfull + C::kWR;     // [kWR]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wempty + C::kWR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* outl = reinterpret_cast<int*>(smem + C::kOffOut);  // input - k0 of the tile's outliers, in order
+  float4* outl = reinterpret_cast<float4*>(smem + C::kOffOut);  // {input - k0, i, s_i - 1, 1 / s_i}
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -280,6 +255,9 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     } else if (lane == 24) {
       mbar_init(acc_full, 1);
       *abort_flag = 0;
+    } else if (lane >= 16 && lane < 16 + C::kWR) {
+      mbar_init(&wfull[lane - 16], 32);  // one cp.async arrival per producer lane
+      mbar_init(&wempty[lane - 16], C::kConvWarps);
     }
     fence_barrier_init();
     if (lane == 0) tma_prefetch_desc(&tmDY);
@@ -341,15 +319,44 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       }
     }
   } else if (warp == 2) {
-    // idle: the outlier rows come precomputed from the workspace
+    // ------------------------------------------------- W_O ring producer
+    // Outlier indices and W_O^T are weights: no dependency on the previous
+    // kernel.  The tile's outliers are the consecutive entries [lo, lo + nout).
+    int lo = 0, nout = 0;
+    if (args.nO > 0) {
+      lo = lower_bound_i32(args.oidx, args.nO, k0);
+      nout = lower_bound_i32(args.oidx, args.nO, k0 + 256) - lo;
+    }
+    const int ne = min(nout, C::kWMax);
+    if (ne > 0) {
+      const int cf = lo >> 3;                        // first 8-outlier chunk
+      const int nch = ((lo + ne - 1) >> 3) - cf + 1;  // chunks per channel row, <= kWChunks
+      for (int jj = 0; jj < nst; ++jj) {
+        const int slot = jj % C::kWR;
+        if (jj >= C::kWR && !mbar_wait(&wempty[slot], static_cast<uint32_t>(jj / C::kWR - 1) & 1u, abort_flag)) break;
+        unsigned char* dst = smem + C::kOffW + slot * C::kWSlot;
+        for (int t = lane; t < 64 * nch; t += 32) {
+          const int q = t / nch;
+          const int cix = t - q * nch;
+          const int kc = cf + cix;
+          const int n = (j0 + jj) * 64 + q;
+          const int r = n & 127;
+          const uint16_t* src = args.wot + (static_cast<size_t>(n >> 7) * args.nib + (kc >> 3)) * 8192 + r * 64 +
+                                (((kc & 7) ^ (r & 7)) << 3);
+          cp_async16(dst + q * C::kWRow + cix * 16, src);
+        }
+        cp_async_mbar_arrive_noinc(&wfull[slot]);
+      }
+      cp_async_wait_all();
+    }
   } else {
     // ------------------------------------------- converters, then epilogue
     const int cw = warp - 3;             // 0..15
     const int ctid = threadIdx.x - 96;   // 0..511
     // Each thread converts one 32-input window (inputs 32 g .. 32 g + 31 of
     // the tile) of one channel row per step; its codes, channel scale and
-    // ratio are loaded two steps ahead.  Outlier inputs of the window are
-    // then overwritten with the precomputed blended rows.
+    // ratio are loaded two steps ahead.  The outlier rows are blended after
+    // the conversion by all threads together (below).
     const int nl = (cw & 1) * 32 + lane;  // channel row of the step
     const int g = cw >> 1;                // window, 0..7
     const int sw = nl & 7;
@@ -357,36 +364,21 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     load_step<FMT>(in0, args, j0, nl, g, kb0, nb);
     if (nst > 1) load_step<FMT>(in1, args, j0 + 1, nl, g, kb0, nb);
 
-    griddep_wait();  // the blended outlier rows come from the previous kernel
+    griddep_wait();  // s comes from the forward
     int nout = 0, lo = 0;
     if (args.nO > 0) {
       lo = lower_bound_i32(args.oidx, args.nO, k0);
       nout = lower_bound_i32(args.oidx, args.nO, k0 + 256) - lo;
-      if (ctid < nout) outl[ctid] = __ldg(args.oidx + lo + ctid) - k0;
+      if (ctid < nout) {
+        const int i = lo + ctid;
+        const float sv = args.s[i];
+        outl[ctid] = make_float4(__int_as_float(__ldg(args.oidx + i) - k0), __int_as_float(i), __fsub_rn(sv, 1.f),
+                                 __frcp_rn(sv));
+      }
     }
     named_bar_sync(1, 32 * C::kConvWarps);
-    // this window's entries of the tile's outlier table: [wb0, wb1)
-    int wb0 = 0, wb1 = 0;
-    for (int e = 0; e < nout; ++e) {
-      const int kl = outl[e];
-      wb0 += kl < 32 * g ? 1 : 0;
-      wb1 += kl < 32 * g + 32 ? 1 : 0;
-    }
-    // the blended values of the window's first outlier inputs for step j
-    auto load_ov = [&](BwdIn<FMT>& in, int j) {
-      const int n = j * 64 + nl;
-#pragma unroll
-      for (int u = 0; u < kBwdOvPre; u += 2) {
-        uint32_t lo16 = 0u, hi16 = 0u;
-        if (n < args.N && wb0 + u < wb1)
-          lo16 = __ldg(args.weffo + static_cast<size_t>(lo + wb0 + u) * args.N + n);
-        if (n < args.N && wb0 + u + 1 < wb1)
-          hi16 = __ldg(args.weffo + static_cast<size_t>(lo + wb0 + u + 1) * args.N + n);
-        in.ov[u >> 1] = lo16 | (hi16 << 16);
-      }
-    };
-    load_ov(in0, j0);
-    if (nst > 1) load_ov(in1, j0 + 1);
+    const int ne = min(nout, C::kWMax);  // entries served by the W_O ring
+    const int lo8 = lo & 7;              // position of entry 0 in a ring row (fp16 units)
 
     bool ok = true;
     // jj counts this CTA's steps, j = j0 + jj is the channel step
@@ -396,7 +388,10 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
       if (ok && jj >= BS) ok = mbar_wait(&bempty[b], static_cast<uint32_t>(jj / BS - 1) & 1u, abort_flag);
       if (ctid == 0) QLIN_STEP(jj, 3);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) return;
+      if (!ok) {  // keep every converter thread on the same named barriers
+        if (nout > 0) named_bar_sync(1, 32 * C::kConvWarps);
+        return;
+      }
       unsigned char* bt = smem + C::kOffB + b * C::kBBytes;
       unsigned char* brow = bt + (nl >> 3) * kBwdSbo + sw * 128;
       // c'_n of the forward's INT8 operand: c_n / 16 for per-channel INT4 (16 q), else c_n
@@ -447,26 +442,34 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
           *reinterpret_cast<uint4*>(atom + (((ch0 + e) ^ sw) << 4)) = h;
         }
       }
-      const int n = j * 64 + nl;
-      if (wb1 > wb0 && n < args.N) {
-        // outlier inputs of this window: Weff[O_i][n] from the blended rows,
-        // the first kBwdOvPre loaded two steps ahead (every lane of the warp
-        // has the same entries: no divergence)
-#pragma unroll
-        for (int u = 0; u < kBwdOvPre; ++u)
-          if (wb0 + u < wb1)
-            *outlier_elem(bt, outl[wb0 + u], nl) = static_cast<uint16_t>(in.ov[u >> 1] >> (16 * (u & 1)));
-        const uint16_t* src = args.weffo + static_cast<size_t>(lo) * args.N + n;
-        for (int e = wb0 + kBwdOvPre; e < wb1; ++e)
-          *outlier_elem(bt, outl[e], nl) = __ldg(src + static_cast<size_t>(e) * args.N);
-      }
-      if (jj + 2 < nst) {
-        load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
-        load_ov(in, j + 2);
+      if (jj + 2 < nst) load_step<FMT>(in, args, j + 2, nl, g, kb0, nb);
+      const int ws = jj % C::kWR;
+      if (nout > 0) {
+        // outlier rows: Weff = (c'_n B + (s_i - 1) W[O_i][n]) / s_i, on the
+        // converted values, once every thread has stored its window; the
+        // nout x 64 elements are spread over all converter threads.  W from
+        // the ring (first kWMax entries of the tile) or from global memory.
+        if (ok) ok = mbar_wait(&wfull[ws], static_cast<uint32_t>(jj / C::kWR) & 1u, abort_flag);
+        named_bar_sync(1, 32 * C::kConvWarps);
+        if (ok) {
+          const unsigned char* ring = smem + C::kOffW + ws * C::kWSlot;
+          for (int t = ctid; t < nout * 64; t += 32 * C::kConvWarps) {
+            const int e = t >> 6;
+            const int q = t & 63;
+            const float4 o = outl[e];
+            uint16_t w;
+            if (e < ne) w = reinterpret_cast<const uint16_t*>(ring + q * C::kWRow)[lo8 + e];
+            else w = wot_elem(args, j * 64 + q, __float_as_int(o.y));
+            patch_outlier(bt, o, q, w);
+          }
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bfull[b]);  // B slot written
+      if (lane == 0) {
+        mbar_arrive(&bfull[b]);                  // B slot written
+        if (ne > 0) mbar_arrive(&wempty[ws]);    // ring slot read
+      }
       if (ctid == 0) QLIN_STEP(jj, 4);
     };
     for (int jj = 0; jj < nst; jj += 2) {  // every step, also after a failed wait (named barriers)

@@ -804,15 +804,12 @@ qlin_status noalloc_scratch(unsigned** out) {
 // waves of one CTA per SM; when the grid is under two waves, the tiles of
 // the ragged last wave are split into tsplit ranges of the channel steps (at
 // most 8, at most one range per step) so that wave has as many CTAs as SMs,
-// and their fp32 partials go through the workspace.  Without room for them
-// every tile is whole.  The workspace starts with the blended outlier rows
-// ([n_O][N] fp16), which a layer with outliers always needs.
+// and their fp32 partials go through the workspace.  Without a workspace
+// every tile is whole.
 struct BwdPlan {
   int ntk, tiles, full, tsplit;
   size_t part_off, cnt_off, bytes;
 };
-
-size_t bwd_rows_bytes(const qlin_weights* w) { return round_up(size_t(w->n_outlier) * w->N * 2, kAlign); }
 
 BwdPlan plan_backward(int M, const qlin_weights* w, bool split) {
   BwdPlan p{};
@@ -836,23 +833,16 @@ BwdPlan plan_backward(int M, const qlin_weights* w, bool split) {
     }
   }
   const int ntail = p.tiles - p.full;
-  const size_t rows = bwd_rows_bytes(w);
-  p.part_off = rows;
-  p.cnt_off = rows + round_up(size_t(ntail) * (p.tsplit - 1) * 65536 * 4, kAlign);
-  p.bytes = ntail ? round_up(p.cnt_off + size_t(ntail) * 4, kAlign) : rows;
+  p.part_off = 0;
+  p.cnt_off = round_up(size_t(ntail) * (p.tsplit - 1) * 65536 * 4, kAlign);
+  p.bytes = ntail ? round_up(p.cnt_off + size_t(ntail) * 4, kAlign) : 0;
   return p;
 }
 
 template <int FMT>
-qlin_status launch_backward_t(const CUtensorMap& tm, const BwdArgs& args, uint16_t* weffo, cudaStream_t stream) {
+qlin_status launch_backward_t(const CUtensorMap& tm, const BwdArgs& args, cudaStream_t stream) {
   using C = BwdCfg<FMT>;
   auto kern = backward_dx_kernel<FMT>;
-  if (args.nO > 0) {
-    cudaError_t e = launch_k(outlier_rows_kernel<FMT>, dim3(static_cast<unsigned>((args.N + 255) / 256),
-                                                            static_cast<unsigned>(args.nO)),
-                             dim3(256), 0, stream, args, weffo);
-    if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "outlier_rows_kernel launch failed: %s", cudaGetErrorString(e));
-  }
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [&] {
@@ -1089,7 +1079,7 @@ qlin_status qlin_backward_dx_workspace(int32_t M, const qlin_weights* w, size_t*
   qlin_status st = check_weights(w);
   if (st != QLIN_OK) return st;
   if (!bytes || M < 0) return fail(QLIN_ERR_ARG, "bad arguments");
-  *bytes = M > 0 ? plan_backward(M, w, true).bytes : 0;  // the outlier rows, then the split partials
+  *bytes = M > 0 ? plan_backward(M, w, true).bytes : 0;
   return QLIN_OK;
 }
 
@@ -1127,27 +1117,20 @@ qlin_status qlin_backward_dx(const qlin_weights* w, const uint16_t* dY, int32_t 
   args.kbs = (w->K + 127) / 128;
   args.nib = (nO + 63) / 64;
   args.nsteps = (w->N + 63) / 64;
-  // the outlier rows need their part of the workspace; the split plan needs
-  // the whole workspace it asks for, and with a smaller one every tile runs
-  // whole
-  const size_t rows = bwd_rows_bytes(w);
-  if (nO > 0 && (!workspace || ws_bytes < rows))
-    return fail(QLIN_ERR_WORKSPACE, "a layer with outliers needs a workspace of at least %zu bytes", rows);
+  // the split plan needs the whole workspace it asks for; with none (or a
+  // smaller one) every tile runs whole
   BwdPlan p = plan_backward(M, w, true);
-  if (p.bytes > rows && (!workspace || ws_bytes < p.bytes)) p = plan_backward(M, w, false);
-  uint16_t* weffo = nO > 0 ? static_cast<uint16_t*>(workspace) : nullptr;
-  args.weffo = weffo;
+  if (p.bytes && (!workspace || ws_bytes < p.bytes)) p = plan_backward(M, w, false);
   args.ntk = p.ntk;
   args.full = p.full;
   args.tsplit = p.tsplit;
-  const bool split = p.full < p.tiles;
-  args.part = split ? reinterpret_cast<float*>(static_cast<char*>(workspace) + p.part_off) : nullptr;
-  args.cnt = split ? reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + p.cnt_off) : nullptr;
+  args.part = p.bytes ? reinterpret_cast<float*>(static_cast<char*>(workspace) + p.part_off) : nullptr;
+  args.cnt = p.bytes ? reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + p.cnt_off) : nullptr;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   switch (w->fmt) {
-    case QLIN_W4_PERCHANNEL: return launch_backward_t<kFmtW4PC>(tm, args, weffo, stream);
-    case QLIN_W4_G128: return launch_backward_t<kFmtW4G128>(tm, args, weffo, stream);
-    default: return launch_backward_t<kFmtW8>(tm, args, weffo, stream);
+    case QLIN_W4_PERCHANNEL: return launch_backward_t<kFmtW4PC>(tm, args, stream);
+    case QLIN_W4_G128: return launch_backward_t<kFmtW4G128>(tm, args, stream);
+    default: return launch_backward_t<kFmtW8>(tm, args, stream);
   }
 }
 

@@ -72,9 +72,6 @@ def run(q, W, O, fmt, dY, s, workspace=False):
     if workspace:
         nws = q.qlin_backward_dx_workspace(M, layer.w)
         ws = q.empty_workspace(nws) if nws else None
-    elif len(O):  # the blended outlier rows only: every tile runs whole
-        nws = rows_bytes(len(O), N)
-        ws = q.empty_workspace(nws)
     q.qlin_backward_dx(layer.w, dYd, M, sd, dX, ws, nws)
     if workspace:
         first = dX.clone()
@@ -84,22 +81,16 @@ def run(q, W, O, fmt, dY, s, workspace=False):
     torch.cuda.synchronize()
     if workspace:
         assert torch.equal(first, dX), "second call with the same workspace differs"
-        cnt = split_counters(ws, M, K, N, len(O)) if ws is not None else None
+        cnt = split_counters(ws, M, K, N) if ws is not None else None
         if cnt is not None:
             assert not cnt.any().item(), "split-tile counters not left zeroed"
     return dX.float().cpu().numpy().astype(np.float64)
 
 
-def rows_bytes(nO, N):
-    """Workspace bytes of the blended outlier rows (fp16 [nO][N], 256-byte
-    multiple), the part every call on a layer with outliers needs."""
-    return -(-(2 * nO * N) // 256) * 256
-
-
-def split_counters(ws, M, K, N, nO=0):
-    """The per-tile counters of the split plan (workspace layout: the
-    blended outlier rows, the fp32 partials of the split tiles, then one
-    counter per split tile), or None when the call splits nothing."""
+def split_counters(ws, M, K, N):
+    """The per-tile counters of the split plan (workspace layout: fp32
+    partials of the split tiles, then one counter per split tile), or None
+    when the call splits nothing."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles = -(-K // 256) * -(-M // 256)
     tail = tiles % sms
@@ -108,7 +99,7 @@ def split_counters(ws, M, K, N, nO=0):
     S = min(sms // tail, 8, -(-N // 64))
     if S < 2:
         return None
-    cnt_off = rows_bytes(nO, N) + -(-(tail * (S - 1) * 65536 * 4) // 256) * 256
+    cnt_off = -(-(tail * (S - 1) * 65536 * 4) // 256) * 256
     return ws[cnt_off:cnt_off + tail * 4]
 
 
@@ -233,13 +224,8 @@ def test_backward_zero_tokens_and_repeat(q):
     q.qlin_backward_dx(layer.w, dY, 0, s, dX)
     torch.cuda.synchronize()
     assert bool((dX == 7.0).all())
-    with pytest.raises(q.QlinError) as e:  # the outlier rows need a workspace
-        q.qlin_backward_dx(layer.w, dY, 64, s, dX)
-    assert q.STATUS[e.value.status] == "QLIN_ERR_WORKSPACE"
-    nws = q.qlin_backward_dx_workspace(64, layer.w)
-    ws = q.empty_workspace(nws)
-    q.qlin_backward_dx(layer.w, dY, 64, s, dX, ws, nws)
+    q.qlin_backward_dx(layer.w, dY, 64, s, dX)
     a = dX.clone()
-    q.qlin_backward_dx(layer.w, dY, 64, s, dX, ws, nws)
+    q.qlin_backward_dx(layer.w, dY, 64, s, dX)
     q.qlin_poll_device_status()
     assert torch.equal(a, dX)
