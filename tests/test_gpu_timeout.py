@@ -5,7 +5,9 @@ its copies and tensor-core work and frees its tensor memory, and
 qlin_poll_device_status reports QLIN_ERR_TIMEOUT.  Afterwards, with the
 default limit back, a normal forward on a zero-filled workspace matches the
 oracle: the context and the library recovered.  No fault is provoked: the
-wait runs out on data that would have arrived."""
+wait runs out on data that would have arrived.  The layer is sized, and
+the GEMM held to one persistent CTA, so that a wait is certainly pending
+when it is first tested."""
 import numpy as np
 import pytest
 import torch
@@ -26,7 +28,9 @@ def q():
 
 
 def test_zero_wait_limit_reports_timeout_then_recovers(q, oracle):
-    L = synth.layer("small", 0)  # M = 16, K = N = 512, 10 outlier channels
+    # one persistent CTA walks a long K loop, so its pipeline waits cannot all
+    # be complete at their first test (a short loop can finish inside it)
+    L = synth.layer("small", 0, M=16, K=16384, N=256, n_outliers=10)
     M, K, N, O = L["M"], L["K"], L["N"], L["O"]
     layer = q.PackedLayer.pack(torch.from_numpy(L["W"]).cuda(), O, synth.W4_PERCHANNEL)
     X = torch.from_numpy(L["X"]).cuda()
@@ -35,7 +39,7 @@ def test_zero_wait_limit_reports_timeout_then_recovers(q, oracle):
     ws = q.empty_workspace(n)
     s = torch.ones(len(O), dtype=torch.float32, device="cuda")
     q.qlin_poll_device_status()  # nothing pending
-    with q.knobs(wait_ns=0, cluster=0):
+    with q.knobs(wait_ns=0, cluster=0, max_ctas=1):
         q.qlin_forward(X, M, layer.w, s, L["gamma"], True, Y, ws, n)
         with pytest.raises(q.QlinError) as e:
             q.qlin_poll_device_status()
