@@ -144,6 +144,9 @@ struct GemmArgs {
   int cs;
   int ncl;
   int cb[9];
+  // 1: the weight blocks were written by the previous kernel (INT4 widened
+  // once per call), so the weight producer waits on the grid dependency too
+  int wdep;
   // bnd[c] = first iteration of CTA c, bnd[grid] = total (computed on the
   // host by gemm_boundaries(); kernel parameters, read from the constant
   // cache).
@@ -693,6 +696,7 @@ gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
     // ------------------------------------------------------------ weight producer
     if (lane == 0) {
       QLIN_STAMP(25);
+      if (args.wdep) griddep_wait();  // widened weights come from the previous kernel
       const uint64_t pol_stream = policy_evict_first();
       uint32_t a_issues[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // loads issued into each A slot
       SegGen gen = seg_begin(plan, cid, cl);

@@ -555,6 +555,7 @@ qlin_status launch_gemm_group(const GemmPlan& p, const qlin_weights* const* ws, 
   args.total = static_cast<unsigned>(iters);
   args.cs = 1;
   args.ncl = 0;
+  args.wdep = p.widen ? 1 : 0;
   gemm_boundaries(prm.pr, p.nprob, p.grid, p.split, args.bnd);
   const int fmt = ws[0]->fmt;
   if (p.widen) {
