@@ -448,6 +448,10 @@ QLIN_API qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, 
  *                             weights are widened to INT8 once per call; 0: never.
  *   QLIN_KNOB_FUSED_MOMENTUM_MAX_M  16 (default): up to this token count the
  *                             momentum update runs inside the quantization kernel.
+ *   QLIN_KNOB_CONVERT_MAX_M   0 (default): INT4 layers on CTA pairs up to this
+ *                             token count convert their codes inside the GEMM
+ *                             (eight converter warps per CTA) instead of
+ *                             widening them to INT8 ahead of it; 0: always widen.
  *   QLIN_KNOB_PAIR_MMA        2 (default): 256-token tiles with INT8 operands run
  *                             on CTA pairs (one 256-row tensor-core operation
  *                             per pair) whenever the operands allow; 1: only
@@ -474,7 +478,8 @@ typedef enum {
   QLIN_KNOB_WIDEN_MIN_M = 5,
   QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6,
   QLIN_KNOB_WAIT_NS = 7,
-  QLIN_KNOB_PAIR_MMA = 8
+  QLIN_KNOB_PAIR_MMA = 8,
+  QLIN_KNOB_CONVERT_MAX_M = 9
 } qlin_knob;
 
 QLIN_API qlin_status qlin_debug_set(int32_t knob, int64_t value, int64_t* previous);

@@ -38,17 +38,32 @@
 
 namespace qlin {
 
-constexpr int kPairStages = 5;
 constexpr int kPairStage = 32768;  // per CTA and step: 16 KB weight rows + 16 KB token rows
-constexpr int kPairOffY = kPairStages * kPairStage;  // the tile's output, fp16 [256 tokens][128 channels]
-constexpr int kPairOffBar = kPairOffY + 256 * 128 * 2;
-constexpr int kPairOffSa = kPairOffBar + 256;
-constexpr int kPairSmem = kPairOffSa + 1024 + 1024;  // + alignment slack
-static_assert(kPairSmem <= 232448, "pair kernel shared memory above 227 KB");
-constexpr int kPairThreads = 32 * (2 + 8);
 constexpr int kPairEpiWarps = 8;
 
+// FMT = kFmtW8: the INT8 weight rows arrive by TMA (the INT8 format, or INT4
+// widened ahead of the GEMM).  FMT = kFmtW4PC / kFmtW4G128: the packed INT4
+// blocks arrive in a staging ring and eight converter warps per CTA widen
+// them into the stage's weight rows (the arithmetic of widen_w4_kernel).
+template <int FMT>
+struct PairCfg {
+  static constexpr bool kConv = FMT != kFmtW8;
+  static constexpr int S = kConv ? 4 : 5;             // stages of weight + token rows
+  static constexpr int LS = kConv ? 3 : 0;            // staging slots of packed blocks
+  static constexpr int kStgBytes = 8192 + 256;        // packed block + the g128 ratio row
+  static constexpr int kOffStg = S * kPairStage;
+  static constexpr int kOffY = kOffStg + (LS * kStgBytes + 1023) / 1024 * 1024;  // output tile
+  static constexpr int kOffBar = kOffY + 256 * 128 * 2;
+  static constexpr int kOffSa = kOffBar + 256;
+  static constexpr int kSmem = kOffSa + 1024 + 1024;  // + alignment slack
+  static constexpr int kConvWarps = kConv ? 8 : 0;
+  static constexpr int kThreads = 32 * (2 + kPairEpiWarps + kConvWarps);
+  static_assert(kSmem <= 232448, "pair kernel shared memory above 227 KB");
+};
+
 struct PairArgs {
+  const uint8_t* codes;      // packed INT4 blocks (converting kernels)
+  const uint16_t* rfold;     // g128 ratios r [K/128][N]
   const float* cscale;
   float cmul;         // factor on c_n (1, or 1/16 for per-channel INT4 widened to 16 q)
   const float* a;
@@ -85,15 +100,21 @@ __device__ __forceinline__ void pair_tile_coords(const PairArgs& g, int t, int& 
   tn2 = w / gs;
 }
 
-__global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid_constant__ PairParams prm) {
+template <int FMT>
+__global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(const __grid_constant__ PairParams prm) {
+  using C = PairCfg<FMT>;
   const PairArgs& g = prm.g;
-  constexpr int S = kPairStages;
+  constexpr int S = C::S;
+  constexpr int LS = C::LS > 0 ? C::LS : 1;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairOffBar);  // [S] (the even CTA's are used)
-  uint64_t* empty = full + S;                                         // [S] (each CTA's own)
-  uint64_t* acc_full = empty + S;                                     // each CTA's own
-  uint64_t* acc_empty = acc_full + 1;                                 // the even CTA's
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);  // [S] (the even CTA's are used)
+  uint64_t* empty = full + S;                                        // [S] (each CTA's own)
+  uint64_t* aready = empty + S;                                      // [S] converted rows (the even CTA's)
+  uint64_t* sfull = aready + S;                                      // [LS] staging (each CTA's own)
+  uint64_t* sempty = sfull + LS;                                     // [LS]
+  uint64_t* acc_full = sempty + LS;                                  // each CTA's own
+  uint64_t* acc_empty = acc_full + 1;                                // the even CTA's
   uint64_t* mma_done = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -109,6 +130,11 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&aready[s], 2 * C::kConvWarps);
+    }
+    for (int s = 0; s < C::LS; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], C::kConvWarps);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kPairEpiWarps);
@@ -117,7 +143,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
     fence_barrier_init();
   }
   if (warp == 0 && lane == 1) {
-    tma_prefetch_desc(&prm.tmA);
+    if (!C::kConv) tma_prefetch_desc(&prm.tmA);
     tma_prefetch_desc(&prm.tmX);
     if (comp) {
       tma_prefetch_desc(&prm.tmU);
@@ -140,25 +166,47 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
     if (lane == 0) {
       griddep_wait();  // Xq, U and widened weights come from the previous kernels
       const uint32_t lfull0 = mapa_shared(smem_u32(&full[0]), 0);
-      int gi = 0;
+      int gi = 0, gs = 0;
       bool ok = true;
       for (int t = cid; ok && t < g.tiles; t += g.ncl) {
         int tn2, tm;
         pair_tile_coords(g, t, tn2, tm);
         const int ctile = 2 * tn2 + crk;    // this CTA's 128 channels
         const int m0 = tm * 256 + crk * 128;  // this CTA's 128 tokens
+        const int n0 = ctile * 128;
+        const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(max(0, min(128, g.N - n0))) * 2u : 0u;
         for (int r = 0; r < g.T; ++r, ++gi) {
           const int s = gi % S;
           if (gi >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag)) {
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[s], 2u * kPairStage);
+          const bool conv = C::kConv && r < g.kb;  // weight rows from the converters
+          if (leader) mbar_arrive_expect_tx(&full[s], conv ? 2u * 16384u : 2u * kPairStage);
           QLIN_STEP(gi, 0);
           unsigned char* A = smem + s * kPairStage;
           unsigned char* X = A + 16384;
           const uint32_t lb = lfull0 + static_cast<uint32_t>(8 * s);
-          if (r < g.kb) {
+          if (conv) {
+            // the packed block (and its ratio row) into the staging ring
+            const int ls = gs % LS;
+            if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
+            // the odd CTA of the last pair tile may lie past the weights
+            // (an odd number of channel tiles): nothing to load, its rows
+            // are never stored
+            const bool have = ctile < g.ntn;
+            mbar_arrive_expect_tx(&sfull[ls], have ? 8192u + rb : 0u);
+            if (have) {
+              bulk_load(st, g.codes + (static_cast<size_t>(ctile) * g.kb + r) * 8192, 8192u, &sfull[ls]);
+              if (rb) bulk_load(st + 8192, g.rfold + static_cast<size_t>(r) * g.N + n0, rb, &sfull[ls]);
+            }
+            ++gs;
+            tma_load_2d_pair(X, &prm.tmX, lb, r * 128, m0);
+          } else if (r < g.kb) {
             tma_load_2d_pair(A, &prm.tmA, lb, 0, (ctile * g.kb + r) * 128);
             tma_load_2d_pair(X, &prm.tmX, lb, r * 128, m0);
           } else {
@@ -178,6 +226,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
                globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
         }
       }
+      if (C::kConv) drain_ring(sfull, LS, gs);  // staging copies (the converters consume them unless aborted)
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -198,6 +247,10 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
         for (int r = 0; r < g.T; ++r, ++gi) {
           const int s = gi % S;
           if (!mbar_wait(&full[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (C::kConv && !mbar_wait_cluster(&aready[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
             ok = false;
             break;
           }
@@ -230,6 +283,67 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
       }
     }
     __syncwarp();
+  } else if (warp >= 2 + kPairEpiWarps) {
+    // ------------------------------------------------------------ converters
+    // Thread ct widens half a weight row per step: packed chunks 2h, 2h+1
+    // (64 inputs) of row ct / 2 into INT8 chunks 4h .. 4h+3 of the stage's
+    // weight rows (128-byte swizzle), then every warp arrives on the even
+    // CTA's converted-rows barrier of the stage.  Compensation steps carry
+    // W_O^T rows from TMA: the warps only arrive.
+    if (C::kConv) {
+      const int ct = threadIdx.x - 32 * (2 + kPairEpiWarps);
+      const int row = ct >> 1, hh = ct & 1;
+      const uint32_t lready0 = mapa_shared(smem_u32(&aready[0]), 0);
+      int gi = 0, gs = 0;
+      bool ok = true;
+      for (int t = cid; ok && t < g.tiles; t += g.ncl) {
+        int tn2, tm;
+        pair_tile_coords(g, t, tn2, tm);
+        const int n = (2 * tn2 + crk) * 128 + row;
+        for (int r = 0; r < g.T; ++r, ++gi) {
+          const int s = gi % S;
+          if (gi >= S) ok = mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          if (r < g.kb) {
+            const int ls = gs % LS;
+            ok = __all_sync(0xffffffffu, mbar_wait(&sfull[ls], static_cast<uint32_t>(gs / LS) & 1u, abort_flag));
+            if (!ok) break;
+            const unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
+            const int sw4 = (row >> 1) & 3;  // packed chunks are swizzled by row pair
+            const uint4 w0 = *reinterpret_cast<const uint4*>(st + row * 64 + (((2 * hh) ^ sw4) << 4));
+            const uint4 w1 = *reinterpret_cast<const uint4*>(st + row * 64 + (((2 * hh + 1) ^ sw4) << 4));
+            uint4 o[4];
+            if (FMT == kFmtW4PC) {
+              unpack_w4pc(w0, o[0], o[1]);
+              unpack_w4pc(w1, o[2], o[3]);
+            } else {
+              // a channel past N has zero codes and no ratio loaded: ratio 0
+              const uint16_t rbits = n < g.N ? reinterpret_cast<const uint16_t*>(st + 8192)[row] : uint16_t(0);
+              const __half2 r1 = __half2half2(__ushort_as_half(rbits));
+              const __half2 r16 = __hmul2(r1, __half2half2(__ushort_as_half(static_cast<unsigned short>(0x2C00))));
+              const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              uint2 a[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) a[i] = requant_g128(wv[i], r1, r16);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) o[i] = make_uint4(a[2 * i].x, a[2 * i].y, a[2 * i + 1].x, a[2 * i + 1].y);
+            }
+            unsigned char* A = smem + s * kPairStage;
+            const int sw = row & 7;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(A + row * 128 + (((4 * hh + i) ^ sw) << 4)) = o[i];
+            fence_proxy_async_smem();  // the tensor core reads these rows next
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[ls]);
+            ++gs;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(lready0 + static_cast<uint32_t>(8 * s));
+        }
+      }
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     // Each tile's output goes to shared memory first; the accumulator is
@@ -240,8 +354,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemm_pair_kernel(const __grid
     const int quad = warp & 3;  // TMEM lanes 32*quad .. +31
     const int nl = quad * 32 + lane;
     const bool issuer = ep == 0 && lane == 0;
-    float* sa = reinterpret_cast<float*>(smem + kPairOffSa);       // a_m of the tile's 256 tokens
-    uint16_t* ys = reinterpret_cast<uint16_t*>(smem + kPairOffY);  // [256 tokens][128 channels]
+    float* sa = reinterpret_cast<float*>(smem + C::kOffSa);       // a_m of the tile's 256 tokens
+    uint16_t* ys = reinterpret_cast<uint16_t*>(smem + C::kOffY);  // [256 tokens][128 channels]
     const uint32_t lempty = mapa_shared(smem_u32(acc_empty), 0);
     griddep_wait();  // a[] comes from the previous kernel
     int ti = 0;

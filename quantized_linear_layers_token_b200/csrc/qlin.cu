@@ -141,7 +141,7 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 // each may start its prologue (and the GEMM its weight stream) while the
 // previous kernel in the stream finishes; every kernel waits on the grid
 // dependency before it reads what the previous one wrote.
-std::atomic<long long> g_knob[9] = {{1}, {1}, {0}, {0}, {256}, {512}, {kFusedMomentumMaxM}, {2000000000LL}, {2}};
+std::atomic<long long> g_knob[10] = {{1}, {1}, {0}, {0}, {256}, {512}, {kFusedMomentumMaxM}, {2000000000LL}, {2}, {0}};
 
 long long knob(int k) { return g_knob[k].load(std::memory_order_relaxed); }
 
@@ -206,6 +206,10 @@ int gemm_cta_cap() {
   const int sms = sm_count();
   return (v > 0 && v < sms) ? static_cast<int>(v) : sms;
 }
+
+// INT4 layers on CTA pairs up to this many tokens convert their codes inside
+// the GEMM instead of widening them ahead (QLIN_KNOB_CONVERT_MAX_M; 0 never).
+long long convert_max_m() { return knob(QLIN_KNOB_CONVERT_MAX_M); }
 
 // QLIN_KNOB_MAX_TOKEN_TILE = 64 or 128 caps the token tile.
 int max_bt() {
@@ -414,19 +418,21 @@ qlin_status launch_gemm_fmt(int bt, GemmParams<MAXP>& prm, cudaStream_t stream) 
 }
 
 // ---------------------------------------------------------------- CTA-pair GEMM (many tokens)
+template <int FMT>
 int pair_max_clusters() {
   static int n = -1;
   static std::once_flag once;
   std::call_once(once, [] {
-    if (cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem) != cudaSuccess) {
+    if (cudaFuncSetAttribute(gemm_pair_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairCfg<FMT>::kSmem) != cudaSuccess) {
       cudaGetLastError();
       n = 0;
       return;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * ((sm_count() + 1) / 2)));
-    cfg.blockDim = dim3(kPairThreads);
-    cfg.dynamicSmemBytes = kPairSmem;
+    cfg.blockDim = dim3(PairCfg<FMT>::kThreads);
+    cfg.dynamicSmemBytes = PairCfg<FMT>::kSmem;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 2;
@@ -435,7 +441,7 @@ int pair_max_clusters() {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&c, gemm_pair_kernel<FMT>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       c = 0;
     }
@@ -452,12 +458,16 @@ bool use_pair(const GemmPlan& p, const qlin_weights* w) {
   const long long mode = knob(QLIN_KNOB_PAIR_MMA);
   if (mode == 0 || p.nprob != 1 || p.bt != 256) return false;
   if (!(w->fmt == QLIN_W8_PERCHANNEL || p.widen)) return false;
-  const int ncl = pair_max_clusters();
+  const int ncl = pair_max_clusters<kFmtW8>();
   if (ncl < 1) return false;
   const long long tiles = static_cast<long long>((p.pr[0].tiles_n + 1) / 2) * p.pr[0].tiles_m;
   return mode == 2 ? tiles >= 1 : tiles >= ncl;
 }
 
+// FMT = kFmtW8: INT8 weight rows by TMA from `codes8` (the INT8 format, or
+// INT4 widened ahead); kFmtW4PC / kFmtW4G128: the layer's packed INT4 codes,
+// converted inside the kernel.
+template <int FMT>
 qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int8_t* Xq, const float* a, uint16_t* Y,
                              int32_t* acc_debug, char* gws, const uint8_t* codes8, float cmul, cudaStream_t stream) {
   PairParams prm;
@@ -465,6 +475,8 @@ qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int
   PairArgs& g = prm.g;
   const GemmProb& q = p.pr[0];
   const int M = q.M;
+  g.codes = static_cast<const uint8_t*>(w->codes);
+  g.rfold = w->fold_ratio;
   g.cscale = w->chan_scale;
   g.cmul = cmul;
   g.a = a;
@@ -481,14 +493,18 @@ qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int
   g.tiles_m = q.tiles_m;
   g.tiles = g.tiles_n2 * g.tiles_m;
   const double x_bytes = static_cast<double>(M) * w->K;
-  int gm = static_cast<int>(std::lround(std::sqrt(static_cast<double>(pair_max_clusters()) * 256.0 / 256.0)));
+  const int maxc = pair_max_clusters<FMT>();
+  if (maxc < 1) return fail(QLIN_ERR_CUDA, "gemm_pair_kernel: no 2-CTA cluster fits");
+  int gm = static_cast<int>(std::lround(std::sqrt(static_cast<double>(maxc) * 256.0 / 256.0)));
   if (x_bytes <= 48.0 * 1024 * 1024) gm = g.tiles_m;
   g.gm = gm < 1 ? 1 : (gm > g.tiles_m ? g.tiles_m : gm);
-  const int maxc = pair_max_clusters();
   g.ncl = g.tiles < maxc ? g.tiles : maxc;
-  qlin_status st = make_map(&prm.tmA, codes8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128,
-                            static_cast<uint64_t>(q.tiles_n) * q.kb * 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (st != QLIN_OK) return st;
+  qlin_status st = QLIN_OK;
+  if (FMT == kFmtW8) {
+    st = make_map(&prm.tmA, codes8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128,
+                  static_cast<uint64_t>(q.tiles_n) * q.kb * 128, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != QLIN_OK) return st;
+  }
   st = make_map(&prm.tmX, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K, M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != QLIN_OK) return st;
   if (w->n_outlier > 0) {
@@ -501,8 +517,8 @@ qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int
   }
   st = make_map(&prm.tmY, Y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w->N, M, 128, 256, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != QLIN_OK) return st;
-  cudaError_t e = launch_kc(gemm_pair_kernel, dim3(static_cast<unsigned>(2 * g.ncl)), dim3(kPairThreads), kPairSmem,
-                            stream, 2, prm);
+  cudaError_t e = launch_kc(gemm_pair_kernel<FMT>, dim3(static_cast<unsigned>(2 * g.ncl)),
+                            dim3(PairCfg<FMT>::kThreads), PairCfg<FMT>::kSmem, stream, 2, prm);
   if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "gemm_pair_kernel launch failed: %s", cudaGetErrorString(e));
   return QLIN_OK;
 }
@@ -558,6 +574,16 @@ qlin_status launch_gemm_group(const GemmPlan& p, const qlin_weights* const* ws, 
   args.wdep = p.widen ? 1 : 0;
   gemm_boundaries(prm.pr, p.nprob, p.grid, p.split, args.bnd);
   const int fmt = ws[0]->fmt;
+  if (p.widen && MAXP == 1 && use_pair(p, ws[0]) && p.pr[0].M <= convert_max_m()) {
+    // INT4 on CTA pairs, converted inside the kernel (no widening pass)
+    const qlin_weights* w = ws[0];
+    const float cm = fmt == QLIN_W4_PERCHANNEL ? 0.0625f : 1.f;
+    return fmt == QLIN_W4_PERCHANNEL
+               ? launch_gemm_pair<kFmtW4PC>(p, w, Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws, nullptr,
+                                            cm, stream)
+               : launch_gemm_pair<kFmtW4G128>(p, w, Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws,
+                                              nullptr, cm, stream);
+  }
   if (p.widen) {
     const qlin_weights* w = ws[0];
     uint8_t* w8 = reinterpret_cast<uint8_t*>(gws + p.w8_off);
@@ -573,12 +599,12 @@ qlin_status launch_gemm_group(const GemmPlan& p, const qlin_weights* const* ws, 
     prm.pr[0].codes = w8;
     prm.pr[0].cmul = fmt == QLIN_W4_PERCHANNEL ? 0.0625f : 1.f;
     if (MAXP == 1 && use_pair(p, w))
-      return launch_gemm_pair(p, w, Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws, w8, prm.pr[0].cmul,
-                              stream);
+      return launch_gemm_pair<kFmtW8>(p, w, Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws, w8,
+                                      prm.pr[0].cmul, stream);
     return launch_gemm_fmt<kFmtW8, MAXP>(p.bt, prm, stream);
   }
   if (MAXP == 1 && fmt == QLIN_W8_PERCHANNEL && use_pair(p, ws[0]))
-    return launch_gemm_pair(p, ws[0], Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws,
+    return launch_gemm_pair<kFmtW8>(p, ws[0], Xq[0], a[0], Y[0], acc_debug ? acc_debug[0] : nullptr, gws,
                             static_cast<const uint8_t*>(ws[0]->codes), 1.f, stream);
   switch (fmt) {
     case QLIN_W4_PERCHANNEL: return launch_gemm_fmt<kFmtW4PC, MAXP>(p.bt, prm, stream);
@@ -1625,7 +1651,7 @@ qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, int32_t N
 }
 
 qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
-  if (k < 0 || k > QLIN_KNOB_PAIR_MMA) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
+  if (k < 0 || k > QLIN_KNOB_CONVERT_MAX_M) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
   bool ok = true;
   switch (k) {
     case QLIN_KNOB_PDL:
@@ -1646,7 +1672,7 @@ qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
 }
 
 qlin_status qlin_debug_get(int32_t k, int64_t* value) {
-  if (k < 0 || k > QLIN_KNOB_PAIR_MMA || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
+  if (k < 0 || k > QLIN_KNOB_CONVERT_MAX_M || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
   *value = g_knob[k].load();
   return QLIN_OK;
 }

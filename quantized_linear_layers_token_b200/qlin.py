@@ -46,6 +46,7 @@ QLIN_KNOB_WIDEN_MIN_M = 5
 QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6
 QLIN_KNOB_WAIT_NS = 7
 QLIN_KNOB_PAIR_MMA = 8
+QLIN_KNOB_CONVERT_MAX_M = 9
 
 
 class QlinError(RuntimeError):

@@ -8,6 +8,8 @@ sweep, with the knob set for the duration of the test only."""
 import pytest
 import torch
 
+from quantized_linear_layers_token_b200 import synth
+from test_gpu_fullsize import run_full_forward as _run_full_forward
 from test_gpu_fullsize import test_split_k_accumulators_exact as _split_k_case
 from test_gpu_parity import test_shapes as _shape_case, SHAPES
 
@@ -24,6 +26,7 @@ MODES = [
     {"pair_mma": 2, "widen_min_m": 129},  # CTA-pair GEMM for every 256-token tile with INT8 operands
     {"pair_mma": 1, "widen_min_m": 1024},  # CTA pairs only from a full wave of pair tiles
     {"pair_mma": 0},           # one CTA per tile everywhere
+    {"convert_max_m": 1 << 20, "widen_min_m": 129},  # INT4 on CTA pairs, converted inside the GEMM
 ]
 
 
@@ -44,3 +47,15 @@ def test_forced_split_mode(q, oracle, mode):
                 _split_k_case(q, oracle, fmt, M)
         for args in SHAPES:
             _shape_case(q, oracle, *args)
+
+
+@pytest.mark.parametrize("wl_name,shape_idx,ms", [
+    ("llama70b_w4g128", 2, [1024]),       # up_proj 8192 -> 28672
+    ("llama7b_w4g128_prefill", 6, [512]),  # down_proj 11008 -> 4096
+    ("llama7b_w4_decode", 4, [512]),       # per-channel INT4, gate_proj 4096 -> 11008 (86 channel tiles)
+])
+def test_pair_convert_full_size(q, oracle, wl_name, shape_idx, ms):
+    """INT4 layers on CTA pairs with the codes converted inside the GEMM, at
+    bench sizes: codes, scales and accumulators bit-exact on sampled rows."""
+    with q.knobs(convert_max_m=1 << 20):
+        _run_full_forward(q, oracle, synth.WORKLOADS[wl_name], shape_idx, ms)
