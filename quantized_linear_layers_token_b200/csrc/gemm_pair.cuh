@@ -166,15 +166,13 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
     if (lane == 0) {
       griddep_wait();  // Xq, U and widened weights come from the previous kernels
       const uint32_t lfull0 = mapa_shared(smem_u32(&full[0]), 0);
-      int gi = 0, gs = 0;
+      int gi = 0;
       bool ok = true;
       for (int t = cid; ok && t < g.tiles; t += g.ncl) {
         int tn2, tm;
         pair_tile_coords(g, t, tn2, tm);
         const int ctile = 2 * tn2 + crk;    // this CTA's 128 channels
         const int m0 = tm * 256 + crk * 128;  // this CTA's 128 tokens
-        const int n0 = ctile * 128;
-        const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(max(0, min(128, g.N - n0))) * 2u : 0u;
         for (int r = 0; r < g.T; ++r, ++gi) {
           const int s = gi % S;
           if (gi >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag)) {
@@ -188,24 +186,7 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
           unsigned char* X = A + 16384;
           const uint32_t lb = lfull0 + static_cast<uint32_t>(8 * s);
           if (conv) {
-            // the packed block (and its ratio row) into the staging ring
-            const int ls = gs % LS;
-            if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
-              ok = false;
-              break;
-            }
-            unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
-            // the odd CTA of the last pair tile may lie past the weights
-            // (an odd number of channel tiles): nothing to load, its rows
-            // are never stored
-            const bool have = ctile < g.ntn;
-            mbar_arrive_expect_tx(&sfull[ls], have ? 8192u + rb : 0u);
-            if (have) {
-              bulk_load(st, g.codes + (static_cast<size_t>(ctile) * g.kb + r) * 8192, 8192u, &sfull[ls]);
-              if (rb) bulk_load(st + 8192, g.rfold + static_cast<size_t>(r) * g.N + n0, rb, &sfull[ls]);
-            }
-            ++gs;
-            tma_load_2d_pair(X, &prm.tmX, lb, r * 128, m0);
+            tma_load_2d_pair(X, &prm.tmX, lb, r * 128, m0);  // weight rows: converters
           } else if (r < g.kb) {
             tma_load_2d_pair(A, &prm.tmA, lb, 0, (ctile * g.kb + r) * 128);
             tma_load_2d_pair(X, &prm.tmX, lb, r * 128, m0);
@@ -226,7 +207,36 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
                globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
         }
       }
-      if (C::kConv) drain_ring(sfull, LS, gs);  // staging copies (the converters consume them unless aborted)
+    } else if (C::kConv && lane == 1) {
+      // staging producer: the packed blocks (and g128 ratio rows) of the
+      // main steps, as far ahead as the staging ring allows, independent of
+      // the stage ring (lane 0)
+      int gs = 0;
+      bool ok = true;
+      for (int t = cid; ok && t < g.tiles; t += g.ncl) {
+        int tn2, tm;
+        pair_tile_coords(g, t, tn2, tm);
+        const int ctile = 2 * tn2 + crk;
+        const int n0 = ctile * 128;
+        const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(max(0, min(128, g.N - n0))) * 2u : 0u;
+        // the odd CTA of the last pair tile may lie past the weights (an odd
+        // number of channel tiles): nothing to load, its rows are never stored
+        const bool have = ctile < g.ntn;
+        for (int r = 0; r < g.kb; ++r, ++gs) {
+          const int ls = gs % LS;
+          if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
+          mbar_arrive_expect_tx(&sfull[ls], have ? 8192u + rb : 0u);
+          if (have) {
+            bulk_load(st, g.codes + (static_cast<size_t>(ctile) * g.kb + r) * 8192, 8192u, &sfull[ls]);
+            if (rb) bulk_load(st + 8192, g.rfold + static_cast<size_t>(r) * g.N + n0, rb, &sfull[ls]);
+          }
+        }
+      }
+      drain_ring(sfull, LS, gs);  // the converters consume every copy unless aborted
     }
     __syncwarp();
   } else if (warp == 1) {
