@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
             ok = false;
             break;
           }
-          if (C::kConv && !mbar_wait_cluster(&aready[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
+          QLIN_STEP(gi, 1);
+          if (C::kConv && !mbar_wait_cluster_poll(&aready[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
             ok = false;
             break;
           }
@@ -315,10 +316,12 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
           if (gi >= S) ok = mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
+          if (ct == 0) QLIN_STEP(gi, 2);
           if (r < g.kb) {
             const int ls = gs % LS;
             ok = __all_sync(0xffffffffu, mbar_wait(&sfull[ls], static_cast<uint32_t>(gs / LS) & 1u, abort_flag));
             if (!ok) break;
+            if (ct == 0) QLIN_STEP(gi, 3);
             const unsigned char* st = smem + C::kOffStg + ls * C::kStgBytes;
             const int sw4 = (row >> 1) & 3;  // packed chunks are swizzled by row pair
             const uint4 w0 = *reinterpret_cast<const uint4*>(st + row * 64 + (((2 * hh) ^ sw4) << 4));
@@ -346,6 +349,7 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
             fence_proxy_async_smem();  // the tensor core reads these rows next
             __syncwarp();
             if (lane == 0) mbar_arrive(&sempty[ls]);
+            if (ct == 0) QLIN_STEP(gi, 4);
             ++gs;
           }
           __syncwarp();

@@ -182,6 +182,25 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// The same wait polling without a suspend hint: for phases completed by
+// another CTA's arrivals, where a suspended waiter may not be woken at once.
+__device__ __forceinline__ bool mbar_wait_cluster_poll(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait_sleep_cluster(bar, parity, 0u)) return true;
+  const uint64_t lim = *const_cast<const volatile unsigned long long*>(&g_wait_ns);
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_sleep_cluster(bar, parity, 0u)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > lim) {
+        *abort = 1;
+        atomicExch(&g_device_error, kDevErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
