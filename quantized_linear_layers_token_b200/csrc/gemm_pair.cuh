@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&aready[s], 2 * C::kConvWarps);
+      if (C::kConv) mbar_init(&aready[s], 2 * C::kConvWarps);
     }
     for (int s = 0; s < C::LS; ++s) {
       mbar_init(&sfull[s], 1);

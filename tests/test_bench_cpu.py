@@ -60,6 +60,19 @@ def test_layer_bytes_by_hand():
     assert bench.layer_bytes(1, K, N, nO, 1) == want
 
 
+def test_offq_bytes_by_hand():
+    """OffQ: the quantization reads X and writes one code byte per value and
+    an fp32 scale and offset per (token, group); the GEMM reads those, the
+    packed INT4 weights, the channel scales and per-group column sums, and
+    writes Y.  Llama-3-8B k_proj at 4096 tokens."""
+    sys.path.insert(0, ROOT)
+    import bench
+    M, K, N = 4096, 4096, 1024
+    G = K // 128
+    assert bench.offq_bytes(M, K, N) == (2 * M * K + M * K + 8 * M * G,
+                                         M * K + 8 * M * G + K * N // 2 + 4 * N + 4 * G * N + 2 * M * N)
+
+
 def test_roofline_bound_follows_arithmetic_intensity():
     """Decode buckets are bound by HBM, prefill buckets by the INT8 tensor
     peak (twice the measured bf16 figure); the fraction is the roofline time
