@@ -1308,7 +1308,7 @@ def run_forward(args, wl):
             if world > 1:  # colmax + momentum per linear, then quant + GEMM per linear
                 return sum(2 + (2 if meta[sl["si"]]["nO"] > 0 else 0) +
                            (1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 512) else 0) for sl in u)
-            colmax = sum(1 for sl in u if meta[sl["si"]]["nO"] > 0 and M > 16)
+            colmax = sum(1 for sl in u if meta[sl["si"]]["nO"] > 0 and M > 64)
             if len(u) > 1 or (fw.grouped and M <= fw.GROUP_MAX_M):
                 return 2 + colmax  # one quantization launch, one GEMM launch for the group
             widen = 1 if (wl.fmt != synth.W8_PERCHANNEL and M >= 512) else 0

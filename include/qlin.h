@@ -446,8 +446,11 @@ QLIN_API qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, 
  *   QLIN_KNOB_MAX_TOKEN_TILE  256 (default); 64 or 128 cap the GEMM's token tile.
  *   QLIN_KNOB_WIDEN_MIN_M     512 (default): from this token count INT4
  *                             weights are widened to INT8 once per call; 0: never.
- *   QLIN_KNOB_FUSED_MOMENTUM_MAX_M  16 (default): up to this token count the
- *                             momentum update runs inside the quantization kernel.
+ *   QLIN_KNOB_FUSED_MOMENTUM_MAX_M  64 (default): up to this token count the
+ *                             momentum update runs inside the quantization kernel
+ *                             (every CTA gathers the outlier columns of all rows);
+ *                             above it one column-maximum launch per problem
+ *                             precedes the quantization.
  *   QLIN_KNOB_CONVERT_MAX_M   0 (default): INT4 layers on CTA pairs up to this
  *                             token count convert their codes inside the GEMM
  *                             (eight converter warps per CTA) instead of

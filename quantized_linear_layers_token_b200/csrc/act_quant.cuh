@@ -28,7 +28,7 @@ namespace qlin {
 
 constexpr int kColmaxRows = 32;   // rows per CTA of colmax_kernel
 constexpr int kQuantThreads = 512;
-constexpr int kFusedMomentumMaxM = 16;  // up to this many tokens the update runs inside quant_kernel
+constexpr int kFusedMomentumMaxM = 64;  // up to this many tokens the update runs inside quant_kernel
 
 
 __device__ __forceinline__ __half2 u32_as_half2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
