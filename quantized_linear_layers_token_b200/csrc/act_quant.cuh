@@ -75,11 +75,26 @@ __global__ void colmax_kernel(const uint16_t* __restrict__ X, int M, int K, cons
   const int r0 = blockIdx.x * kColmaxRows;
   const int r1 = min(M, r0 + kColmaxRows);
   const int total = (r1 - r0) * nO;
-  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-    const int m = r0 + idx / nO;
-    const int i = idx - (idx / nO) * nO;
-    const float v = fabsf(h2f(X[static_cast<size_t>(m) * K + sO[i]]));
-    atomicMax(&scm[i], __float_as_uint(v));
+  // eight independent gathers per thread in flight before the merges
+  const int stride = static_cast<int>(blockDim.x);
+  for (int idx0 = threadIdx.x; idx0 < total; idx0 += 8 * stride) {
+    uint16_t hv[8];
+    int ii[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int idx = idx0 + u * stride;
+      ii[u] = -1;
+      hv[u] = 0;
+      if (idx < total) {
+        const int r = idx / nO;
+        const int i = idx - r * nO;
+        ii[u] = i;
+        hv[u] = X[static_cast<size_t>(r0 + r) * K + sO[i]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (ii[u] >= 0) atomicMax(&scm[ii[u]], __float_as_uint(fabsf(h2f(hv[u]))));
   }
   __syncthreads();
   for (int i = threadIdx.x; i < nO; i += blockDim.x)
