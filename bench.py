@@ -95,10 +95,12 @@ def algorithmic_bytes(M, K, N, nO, fmt):
     return gemm, act
 
 
+# The GEMM kernels' sources, and the part of the host file that plans and
+# launches them (between its "TMA maps" and "act quant" section markers).
 TRAFFIC_SOURCES = ("quantized_linear_layers_token_b200/csrc/gemm.cuh",
                    "quantized_linear_layers_token_b200/csrc/gemm_pair.cuh",
                    "quantized_linear_layers_token_b200/csrc/sm100.cuh",
-                   "quantized_linear_layers_token_b200/csrc/qlin.cu")
+                   "quantized_linear_layers_token_b200/csrc/qlin.cu:TMA maps:act quant")
 
 
 def gemm_sources_sha256():
@@ -108,12 +110,18 @@ def gemm_sources_sha256():
     import hashlib
     import re
     h = hashlib.sha256()
-    for rel in TRAFFIC_SOURCES:
+    for spec in TRAFFIC_SOURCES:
+        rel, *section = spec.split(":")
         with open(os.path.join(ROOT, rel)) as f:
-            for line in f:
-                line = re.sub(r"//.*", "", line).rstrip()
-                if line:
-                    h.update(line.encode() + b"\n")
+            lines = f.readlines()
+        if section:
+            start = next(i for i, l in enumerate(lines) if l.startswith("// ---") and l.rstrip().endswith(section[0]))
+            end = next(i for i, l in enumerate(lines) if l.startswith("// ---") and l.rstrip().endswith(section[1]))
+            lines = lines[start:end]
+        for line in lines:
+            line = re.sub(r"//.*", "", line).rstrip()
+            if line:
+                h.update(line.encode() + b"\n")
     return h.hexdigest()
 
 
