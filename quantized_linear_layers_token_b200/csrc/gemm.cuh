@@ -788,7 +788,11 @@ gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and its waits; one elected lane issues
+    // each step's tensor-core instructions and commits (issued from a
+    // converged warp, a narrow MMA costs about a third of the cycles it
+    // costs from a lone lane).
+    {
       constexpr uint32_t idesc_main = idesc_s8_s32(128, BT);
       constexpr uint32_t idesc_comp = idesc_f16_f32(128, BT);
       // Descriptors of ring slot 0; the start-address field counts 16-byte
@@ -809,7 +813,7 @@ gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
         const GemmProb& pr = probs[sg.p];
         const int buf = seg % nbuf;
         const int use = seg / nbuf;
-        if (use > 0 && !mbar_wait(&acc_empty[buf], static_cast<uint32_t>(use - 1) & 1u, abort_flag)) {
+        if (use > 0 && !warp_wait(&acc_empty[buf], static_cast<uint32_t>(use - 1) & 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -820,64 +824,71 @@ gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
           const int p = g % P;
           const int x = g % XS;
           const bool main_step = r < pr.nk;
-          if (!mbar_wait(&xfull[x], static_cast<uint32_t>(g / XS) & 1u, abort_flag)) { ok = false; break; }
+          if (!warp_wait(&xfull[x], static_cast<uint32_t>(g / XS) & 1u, abort_flag)) { ok = false; break; }
           QLIN_STEP(g, 5);
           if (C::kTA) {
             const uint64_t bd = xdesc0 + static_cast<uint64_t>(x * (C::kXBytes >> 4));
             if (main_step) {
               const int pa = gm % P;
-              if (!mbar_wait(&aconv[pa], static_cast<uint32_t>(gm / P) & 1u, abort_flag)) { ok = false; break; }
+              if (!warp_wait(&aconv[pa], static_cast<uint32_t>(gm / P) & 1u, abort_flag)) { ok = false; break; }
               if (g == 0) QLIN_STAMP(8);
               QLIN_STEP(g, 6);
               tc_fence_after();
               issued = true;
               const uint32_t at = tmem + a_col0 + static_cast<uint32_t>(pa * C::kACols);
               const int nkb = min(C::KS, pr.kb - r * C::KS);
-              mma_i8_ta(dmain, at, bd, idesc_main, r > sg.r0 ? 1u : 0u);
-              mma_i8_ta(dmain, at + 8, bd + 2, idesc_main, 1u);
-              mma_i8_ta(dmain, at + 16, bd + 4, idesc_main, 1u);
-              mma_i8_ta(dmain, at + 24, bd + 6, idesc_main, 1u);
+              if (elect_one()) {
+                mma_i8_ta(dmain, at, bd, idesc_main, r > sg.r0 ? 1u : 0u);
+                mma_i8_ta(dmain, at + 8, bd + 2, idesc_main, 1u);
+                mma_i8_ta(dmain, at + 16, bd + 4, idesc_main, 1u);
+                mma_i8_ta(dmain, at + 24, bd + 6, idesc_main, 1u);
 #pragma unroll
-              for (int i = 1; i < C::KS; ++i) {
-                if (i < nkb) {
-                  const uint32_t ai = at + static_cast<uint32_t>(i * 32);
-                  const uint64_t bi = bd + static_cast<uint64_t>(i * (C::kXTile >> 4));
-                  mma_i8_ta(dmain, ai, bi, idesc_main, 1u);
-                  mma_i8_ta(dmain, ai + 8, bi + 2, idesc_main, 1u);
-                  mma_i8_ta(dmain, ai + 16, bi + 4, idesc_main, 1u);
-                  mma_i8_ta(dmain, ai + 24, bi + 6, idesc_main, 1u);
+                for (int i = 1; i < C::KS; ++i) {
+                  if (i < nkb) {
+                    const uint32_t ai = at + static_cast<uint32_t>(i * 32);
+                    const uint64_t bi = bd + static_cast<uint64_t>(i * (C::kXTile >> 4));
+                    mma_i8_ta(dmain, ai, bi, idesc_main, 1u);
+                    mma_i8_ta(dmain, ai + 8, bi + 2, idesc_main, 1u);
+                    mma_i8_ta(dmain, ai + 16, bi + 4, idesc_main, 1u);
+                    mma_i8_ta(dmain, ai + 24, bi + 6, idesc_main, 1u);
+                  }
                 }
+                mma_commit(&aempty[pa]);
               }
-              mma_commit(&aempty[pa]);
+              __syncwarp();
               ++gm;
             } else {
               const int cs = gc & 1;
-              if (!mbar_wait(&cfull[cs], static_cast<uint32_t>(gc / 2) & 1u, abort_flag)) { ok = false; break; }
+              if (!warp_wait(&cfull[cs], static_cast<uint32_t>(gc / 2) & 1u, abort_flag)) { ok = false; break; }
               if (g == 0) QLIN_STAMP(8);
               QLIN_STEP(g, 6);
               tc_fence_after();
               issued = true;
               const uint64_t ad = cdesc0 + static_cast<uint64_t>(cs * (16384 >> 4));
               const uint32_t acc0 = ((r == pr.nk) || (r == sg.r0)) ? 0u : 1u;
-              mma_f16(dcomp, ad, bd, idesc_comp, acc0);
-              mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
-              mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
-              mma_f16(dcomp, ad + 6, bd + 6, idesc_comp, 1u);
-              const uint64_t bd2 = bd + (C::kXTile >> 4);  // lo rows (fused hi + lo)
+              if (elect_one()) {
+                mma_f16(dcomp, ad, bd, idesc_comp, acc0);
+                mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
+                mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
+                mma_f16(dcomp, ad + 6, bd + 6, idesc_comp, 1u);
+                const uint64_t bd2 = bd + (C::kXTile >> 4);  // lo rows (fused hi + lo)
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) mma_f16(dcomp, ad + 2 * kk, bd2 + 2 * kk, idesc_comp, 1u);
-              mma_commit(&cempty[cs]);
+                for (int kk = 0; kk < 4; ++kk) mma_f16(dcomp, ad + 2 * kk, bd2 + 2 * kk, idesc_comp, 1u);
+                mma_commit(&cempty[cs]);
+              }
+              __syncwarp();
               ++gc;
             }
-            mma_commit(&xempty[x]);
+            if (elect_one()) mma_commit(&xempty[x]);
+            __syncwarp();
             QLIN_STEP(g, 7);
             continue;
           }
           if (main_step && C::kW4) {
-            if (!mbar_wait(&aconv[p], (conv_phase >> p) & 1u, abort_flag)) { ok = false; break; }
+            if (!warp_wait(&aconv[p], (conv_phase >> p) & 1u, abort_flag)) { ok = false; break; }
             conv_phase ^= 1u << p;
           } else {
-            if (!mbar_wait(&afull[p], (full_phase >> p) & 1u, abort_flag)) { ok = false; break; }
+            if (!warp_wait(&afull[p], (full_phase >> p) & 1u, abort_flag)) { ok = false; break; }
             full_phase ^= 1u << p;
           }
           if (g == 0) QLIN_STAMP(8);
@@ -886,41 +897,45 @@ gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
           issued = true;
           const uint64_t ad = adesc0 + static_cast<uint64_t>(p * (C::kABytes >> 4));
           const uint64_t bd = xdesc0 + static_cast<uint64_t>(x * (C::kXBytes >> 4));
-          if (main_step) {
-            const int nkb = min(C::KS, pr.kb - r * C::KS);
-            mma_i8(dmain, ad, bd, idesc_main, r > sg.r0 ? 1u : 0u);
-            mma_i8(dmain, ad + 2, bd + 2, idesc_main, 1u);
-            mma_i8(dmain, ad + 4, bd + 4, idesc_main, 1u);
-            mma_i8(dmain, ad + 6, bd + 6, idesc_main, 1u);
+          if (elect_one()) {
+            if (main_step) {
+              const int nkb = min(C::KS, pr.kb - r * C::KS);
+              mma_i8(dmain, ad, bd, idesc_main, r > sg.r0 ? 1u : 0u);
+              mma_i8(dmain, ad + 2, bd + 2, idesc_main, 1u);
+              mma_i8(dmain, ad + 4, bd + 4, idesc_main, 1u);
+              mma_i8(dmain, ad + 6, bd + 6, idesc_main, 1u);
 #pragma unroll
-            for (int i = 1; i < C::KS; ++i) {
-              if (i < nkb) {
-                const uint64_t ai = ad + static_cast<uint64_t>(i * 1024);
-                const uint64_t bi = bd + static_cast<uint64_t>(i * (C::kXTile >> 4));
-                mma_i8(dmain, ai, bi, idesc_main, 1u);
-                mma_i8(dmain, ai + 2, bi + 2, idesc_main, 1u);
-                mma_i8(dmain, ai + 4, bi + 4, idesc_main, 1u);
-                mma_i8(dmain, ai + 6, bi + 6, idesc_main, 1u);
+              for (int i = 1; i < C::KS; ++i) {
+                if (i < nkb) {
+                  const uint64_t ai = ad + static_cast<uint64_t>(i * 1024);
+                  const uint64_t bi = bd + static_cast<uint64_t>(i * (C::kXTile >> 4));
+                  mma_i8(dmain, ai, bi, idesc_main, 1u);
+                  mma_i8(dmain, ai + 2, bi + 2, idesc_main, 1u);
+                  mma_i8(dmain, ai + 4, bi + 4, idesc_main, 1u);
+                  mma_i8(dmain, ai + 6, bi + 6, idesc_main, 1u);
+                }
+              }
+            } else {
+              const uint32_t acc0 = ((r == pr.nk) || (r == sg.r0)) ? 0u : 1u;
+              mma_f16(dcomp, ad, bd, idesc_comp, acc0);
+              mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
+              mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
+              mma_f16(dcomp, ad + 6, bd + 6, idesc_comp, 1u);
+              if (C::kCompFused) {
+                const uint64_t bd2 = bd + (C::kXTile >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) mma_f16(dcomp, ad + 2 * kk, bd2 + 2 * kk, idesc_comp, 1u);
               }
             }
-          } else {
-            const uint32_t acc0 = ((r == pr.nk) || (r == sg.r0)) ? 0u : 1u;
-            mma_f16(dcomp, ad, bd, idesc_comp, acc0);
-            mma_f16(dcomp, ad + 2, bd + 2, idesc_comp, 1u);
-            mma_f16(dcomp, ad + 4, bd + 4, idesc_comp, 1u);
-            mma_f16(dcomp, ad + 6, bd + 6, idesc_comp, 1u);
-            if (C::kCompFused) {
-              const uint64_t bd2 = bd + (C::kXTile >> 4);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) mma_f16(dcomp, ad + 2 * kk, bd2 + 2 * kk, idesc_comp, 1u);
-            }
+            mma_commit(&aempty[p]);
+            mma_commit(&xempty[x]);
           }
-          mma_commit(&aempty[p]);
-          mma_commit(&xempty[x]);
+          __syncwarp();
           QLIN_STEP(g, 7);
         }
         if (!ok) break;
-        mma_commit(&acc_full[buf]);
+        if (elect_one()) mma_commit(&acc_full[buf]);
+        __syncwarp();
         ++seg;
       }
       QLIN_STAMP(9);
@@ -928,7 +943,8 @@ gemm_kernel(const __grid_constant__ GemmParams<MAXP> prm) {
       // epilogue's accumulator waits already saw that, but after a wait gave
       // up nothing else does, so wait here (fixed limit) either way.
       if (issued) {
-        mma_commit(mma_done);
+        if (elect_one()) mma_commit(mma_done);
+        __syncwarp();
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait_sleep(mma_done, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
         }

@@ -107,6 +107,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same wait made by every lane of a converged warp; the warp agrees on
+// the outcome (a lane that saw the limit pass makes the whole warp give up).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort)) != 0;
+}
+
+// One lane of a converged warp (elect.sync over the full mask: the lowest
+// active lane, so repeated calls in a converged warp pick the same lane).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- clusters
 // Distributed shared memory between the CTAs of a thread-block cluster:
 // `mapa` turns a local shared address into the same offset in CTA `rank`;
