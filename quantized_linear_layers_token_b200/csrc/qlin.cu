@@ -1425,7 +1425,8 @@ qlin_status qlin_smooth_search(const uint16_t* X, int32_t M, int32_t K, const ui
     if (st != QLIN_OK) return st;
     st = launch_gemm(&w, Xq, a, M, Y, acc, ws + L.gemm, stream);
     if (st != QLIN_OK) return st;
-    smooth_ref_kernel<<<dim3((N + 63) / 64, (M + 63) / 64), 256, 0, stream>>>(X, W, sv, M, K, N, ref);
+    smooth_ref_kernel<<<dim3((N + kRefTile - 1) / kRefTile, (M + kRefTile - 1) / kRefTile), 256, 0, stream>>>(
+        X, W, sv, M, K, N, ref);
     smooth_loss_kernel<<<static_cast<unsigned>((mn + 255) / 256), 256, 0, stream>>>(acc, a, w.chan_scale, ref, M,
                                                                                     N, loss + j);
     QLIN_LAUNCH_CHECK("smoothing loss");

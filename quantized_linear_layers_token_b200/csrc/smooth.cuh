@@ -100,47 +100,89 @@ __global__ void smooth_apply_w_kernel(const uint16_t* __restrict__ W, const floa
   Wh[idx] = s > 0.f ? __half_as_ushort(__float2half_rn(__fmul_rn(half_bits_to_float(W[idx]), s))) : 0;
 }
 
-// ref[m][n] = sum over t in T of X[m][t] * W[t][n] (fp32 FMA; 64 x 64 tiles,
-// 256 threads of 4 x 4 outputs, K staged 16 at a time).
+// ref[m][n] = sum over t in T of X[m][t] * W[t][n] (fp32 FMA in input
+// order): 128 x 128 tiles, 256 threads of 8 x 8 outputs, 16 inputs per
+// stage; the next stage's 16-byte loads go to registers while the current
+// stage (shared memory, double-buffered) is used.  K % 32 == 0, N % 16 == 0.
+constexpr int kRefTile = 128;
+constexpr int kRefK = 16;
+
 __global__ void __launch_bounds__(256)
-smooth_ref_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ W, const float* __restrict__ sv, int M,
-                  int K, int N, float* __restrict__ ref) {
-  __shared__ float xs[16][64 + 1];
-  __shared__ float ws[16][64];
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  float acc[4][4] = {};
-  for (int t0 = 0; t0 < K; t0 += 16) {
-    for (int e = threadIdx.x; e < 16 * 64; e += 256) {
-      const int tt = e % 16, mm = e / 16;  // X tile: 64 rows x 16 inputs
-      const int t = t0 + tt, m = m0 + mm;
-      xs[tt][mm] = (m < M && t < K && sv[t] > 0.f) ? half_bits_to_float(X[static_cast<size_t>(m) * K + t]) : 0.f;
-      const int nn = e % 64, tw = e / 64;  // W tile: 16 inputs x 64 outputs
-      const int t2 = t0 + tw, n = n0 + nn;
-      ws[tw][nn] = (n < N && t2 < K) ? half_bits_to_float(W[static_cast<size_t>(t2) * N + n]) : 0.f;
+smooth_ref_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ W, const float* __restrict__ sv,
+                  int M, int K, int N, float* __restrict__ ref) {
+  __shared__ __align__(16) float xs[2][kRefK][kRefTile];  // [input][token]
+  __shared__ __align__(16) float ws[2][kRefK][kRefTile];  // [input][channel]
+  const int m0 = blockIdx.y * kRefTile, n0 = blockIdx.x * kRefTile;
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;         // 8 tokens x 8 channels each
+  const int xr = tid >> 1, xk = (tid & 1) * 8;    // loader: token row, 8 inputs
+  const int wk = tid >> 4, wn = (tid & 15) * 8;   // loader: input row, 8 channels
+  float xa[8], wb[8];
+  auto load = [&](int t0) {
+    const int m = m0 + xr;
+    const int t = t0 + xk;  // 8 inputs, inside K (K % 16 == 0)
+    uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+    if (m < M) xv = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(m) * K + t));
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(sv + t));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(sv + t) + 1);
+    const float sm[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      xa[j] = sm[j] > 0.f ? half_bits_to_float(static_cast<uint16_t>(xw[j >> 1] >> (16 * (j & 1)))) : 0.f;
+    const int n = n0 + wn;
+    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
+    if (n < N) wv = __ldg(reinterpret_cast<const uint4*>(W + static_cast<size_t>(t0 + wk) * N + n));
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wb[j] = half_bits_to_float(static_cast<uint16_t>(ww[j >> 1] >> (16 * (j & 1))));
+  };
+  auto store = [&](int b) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xs[b][xk + j][xr] = xa[j];
+    *reinterpret_cast<float4*>(&ws[b][wk][wn]) = make_float4(wb[0], wb[1], wb[2], wb[3]);
+    *reinterpret_cast<float4*>(&ws[b][wk][wn + 4]) = make_float4(wb[4], wb[5], wb[6], wb[7]);
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int t0 = 0; t0 < K; t0 += kRefK) {
+    const int cur = (t0 / kRefK) & 1;
+    const bool more = t0 + kRefK < K;
+    if (more) load(t0 + kRefK);
+#pragma unroll
+    for (int k = 0; k < kRefK; ++k) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[cur][k][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[cur][k][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&ws[cur][k][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&ws[cur][k][tx * 8 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
     }
-    __syncthreads();
-#pragma unroll
-    for (int tt = 0; tt < 16; ++tt) {
-      float a4[4], b4[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) a4[a] = xs[tt][ty * 4 + a];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) b4[b] = ws[tt][tx * 4 + b];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(a4[a], b4[b], acc[a][b]);
-    }
+    if (more) store(cur ^ 1);
     __syncthreads();
   }
+  const int n = n0 + tx * 8;
+  if (n < N) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int m = m0 + ty * 4 + a, n = n0 + tx * 4 + b;
-      if (m < M && n < N) ref[static_cast<size_t>(m) * N + n] = acc[a][b];
+    for (int a = 0; a < 8; ++a) {
+      const int m = m0 + ty * 8 + a;
+      if (m < M) {
+        float* dst = ref + static_cast<size_t>(m) * N + n;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+      }
     }
+  }
 }
 
 // loss[j] += sum of (a_m (c_n / 16) acc - ref)^2 in fp64 (zero on entry).
