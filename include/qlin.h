@@ -460,6 +460,15 @@ QLIN_API qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, 
  *                             per pair) whenever the operands allow; 1: only
  *                             when there is a full wave of 256 x 256 tiles;
  *                             0: never.
+ *   QLIN_KNOB_PAIR_SPLIT      0 (default): launches on CTA pairs take whole
+ *                             tiles; 1: when such a launch would leave its
+ *                             last wave of tiles partly empty (and has fewer
+ *                             than eight full waves), its last full wave and
+ *                             the remainder are divided by K-steps across all
+ *                             pairs, and the pairs that share a tile sum their
+ *                             INT32 partials in the workspace (exact: the
+ *                             result does not depend on the split; measured
+ *                             slower than whole tiles on the bench shapes).
  *   QLIN_KNOB_WAIT_NS         2000000000 (default): limit in ns of every
  *                             device-side pipeline wait, after which the kernel
  *                             gives up, sets the device error word and unwinds
@@ -482,7 +491,8 @@ typedef enum {
   QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6,
   QLIN_KNOB_WAIT_NS = 7,
   QLIN_KNOB_PAIR_MMA = 8,
-  QLIN_KNOB_CONVERT_MAX_M = 9
+  QLIN_KNOB_CONVERT_MAX_M = 9,
+  QLIN_KNOB_PAIR_SPLIT = 10
 } qlin_knob;
 
 QLIN_API qlin_status qlin_debug_set(int32_t knob, int64_t value, int64_t* previous);

@@ -289,31 +289,37 @@ backward_dx_kernel(const __grid_constant__ CUtensorMap tmDY, const __grid_consta
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the loop and its waits; an elected lane issues.
+    {
       constexpr uint32_t idesc = idesc_f16_f32(128, 256) | (1u << 16);  // B MN-major
       for (int j = 0; j < nst; ++j) {  // j counts this CTA's steps
         const int a = j % AS;
         const int b = j % BS;
-        if (!mbar_wait(&afull[a], static_cast<uint32_t>(j / AS) & 1u, abort_flag)) break;
+        if (!warp_wait(&afull[a], static_cast<uint32_t>(j / AS) & 1u, abort_flag)) break;
         QLIN_STEP(j, 5);
-        if (!mbar_wait(&bfull[b], static_cast<uint32_t>(j / BS) & 1u, abort_flag)) break;
+        if (!warp_wait(&bfull[b], static_cast<uint32_t>(j / BS) & 1u, abort_flag)) break;
         QLIN_STEP(j, 6);
         tc_fence_after();
         const uint32_t abase = smem_u32(smem + C::kOffA + a * C::kABytes);
         const uint32_t bbase = smem_u32(smem + C::kOffB + b * C::kBBytes);
         // one B tile, two 128-token halves of A into columns [0, 256) and [256, 512)
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bdesc = sdesc_mn_sw128(bbase + kk * 2 * kBwdSbo, kBwdLbo, kBwdSbo);
-          mma_f16(tmem, sdesc_k_sw128(abase + kk * 32), bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
-          if (two) mma_f16(tmem + 256, sdesc_k_sw128(abase + 16384 + kk * 32), bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = sdesc_mn_sw128(bbase + kk * 2 * kBwdSbo, kBwdLbo, kBwdSbo);
+            mma_f16(tmem, sdesc_k_sw128(abase + kk * 32), bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
+            if (two)
+              mma_f16(tmem + 256, sdesc_k_sw128(abase + 16384 + kk * 32), bdesc, idesc, (j | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&aempty[a]);
+          mma_commit(&bempty[b]);
         }
-        mma_commit(&aempty[a]);
-        mma_commit(&bempty[b]);
+        __syncwarp();
         QLIN_STEP(j, 7);
       }
       // every MMA issued so far (all of them, or those before an abort)
-      mma_commit(acc_full);
+      if (elect_one()) mma_commit(acc_full);
+      __syncwarp();
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait_sleep(acc_full, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
       }

@@ -40,6 +40,7 @@ namespace qlin {
 
 constexpr int kPairStage = 32768;  // per CTA and step: 16 KB weight rows + 16 KB token rows
 constexpr int kPairEpiWarps = 8;
+constexpr int kMaxPairs = 128;     // pairs in one launch (stream-K boundary table)
 
 // FMT = kFmtW8: the INT8 weight rows arrive by TMA (the INT8 format, or INT4
 // widened ahead of the GEMM).  FMT = kFmtW4PC / kFmtW4G128: the packed INT4
@@ -79,6 +80,21 @@ struct PairArgs {
   int gm;             // raster group of token tiles
   int tiles;          // tiles_n2 * tiles_m
   int ncl;            // clusters (pairs) in the grid
+  // Stream-K tail: tiles [0, dp) are whole tiles, pair c taking c, c + ncl,
+  // ...; the steps of tiles [dp, tiles) are split in contiguous ranges,
+  // pair c taking [bnd[c], bnd[c + 1]) of them (bnd[ncl] = their total).
+  // Tiles split across pairs leave INT32 partials in ws_acc slots
+  // [2 * pair + (first segment of its range ? 0 : 1)][CTA][256 tokens][128
+  // channels], and the range holding a tile's compensation steps (never
+  // split, always the first segment of that range) leaves it, fp32, in
+  // ws_comp [pair][CTA][256][128]; ws_cnt counts each split tile's finished
+  // steps per CTA, and the range whose steps complete the count sums the
+  // partials and writes Y.
+  int dp;
+  int32_t* ws_acc;
+  float* ws_comp;
+  unsigned* ws_cnt;   // [tiles - dp][2], zero between launches
+  unsigned bnd[kMaxPairs + 1];
 };
 
 struct alignas(64) PairParams {
@@ -100,6 +116,58 @@ __device__ __forceinline__ void pair_tile_coords(const PairArgs& g, int t, int& 
   tn2 = w / gs;
 }
 
+// One unit of a pair's work: steps [r0, r1) of tile t.
+struct PairSeg {
+  int t;
+  int r0, r1;
+  int slot;  // partial slot, or -1 for a whole tile
+  int sk;    // index of the tile among the split tail (t - dp), -1 for whole tiles before it
+};
+struct PairGen {
+  int t;
+  unsigned it, it1;
+};
+__device__ __forceinline__ PairGen pair_begin(const PairArgs& g, int cid) {
+  PairGen s;
+  s.t = cid;
+  s.it = g.bnd[cid];
+  s.it1 = g.bnd[cid + 1];
+  return s;
+}
+__device__ __forceinline__ bool pair_next(const PairArgs& g, int cid, PairGen& s, PairSeg& w) {
+  if (s.t < g.dp) {
+    w.t = s.t;
+    w.r0 = 0;
+    w.r1 = g.T;
+    w.slot = -1;
+    w.sk = -1;
+    s.t += g.ncl;
+    return true;
+  }
+  if (s.it >= s.it1) return false;
+  const unsigned T = static_cast<unsigned>(g.T);
+  const unsigned i = s.it / T;
+  const unsigned r0 = s.it - i * T;
+  const unsigned left = s.it1 - s.it;
+  const unsigned r1 = left < T - r0 ? r0 + left : T;
+  w.t = g.dp + static_cast<int>(i);
+  w.r0 = static_cast<int>(r0);
+  w.r1 = static_cast<int>(r1);
+  w.sk = static_cast<int>(i);
+  w.slot = (r0 == 0 && r1 == T) ? -1 : 2 * cid + (s.it == g.bnd[cid] ? 0 : 1);
+  s.it += r1 - r0;
+  return true;
+}
+// Pair whose range holds step `it` of the split tail (bnd[c] <= it < bnd[c + 1]).
+__device__ __forceinline__ int pair_owner(const PairArgs& g, unsigned it) {
+  int lo = 0, hi = g.ncl - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (g.bnd[mid] <= it) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(const __grid_constant__ PairParams prm) {
   using C = PairCfg<FMT>;
@@ -118,6 +186,7 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
   uint64_t* mma_done = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* fin_flag = abort_flag + 1;  // epilogue: this CTA completes the split tile
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int crk = static_cast<int>(cluster_ctarank());
@@ -168,12 +237,14 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
       const uint32_t lfull0 = mapa_shared(smem_u32(&full[0]), 0);
       int gi = 0;
       bool ok = true;
-      for (int t = cid; ok && t < g.tiles; t += g.ncl) {
+      PairGen gen = pair_begin(g, cid);
+      PairSeg sg;
+      while (ok && pair_next(g, cid, gen, sg)) {
         int tn2, tm;
-        pair_tile_coords(g, t, tn2, tm);
+        pair_tile_coords(g, sg.t, tn2, tm);
         const int ctile = 2 * tn2 + crk;    // this CTA's 128 channels
         const int m0 = tm * 256 + crk * 128;  // this CTA's 128 tokens
-        for (int r = 0; r < g.T; ++r, ++gi) {
+        for (int r = sg.r0; r < sg.r1; ++r, ++gi) {
           const int s = gi % S;
           if (gi >= S && !mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag)) {
             ok = false;
@@ -213,16 +284,19 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
       // the stage ring (lane 0)
       int gs = 0;
       bool ok = true;
-      for (int t = cid; ok && t < g.tiles; t += g.ncl) {
+      PairGen gen = pair_begin(g, cid);
+      PairSeg sg;
+      while (ok && pair_next(g, cid, gen, sg)) {
         int tn2, tm;
-        pair_tile_coords(g, t, tn2, tm);
+        pair_tile_coords(g, sg.t, tn2, tm);
         const int ctile = 2 * tn2 + crk;
         const int n0 = ctile * 128;
         const uint32_t rb = FMT == kFmtW4G128 ? static_cast<uint32_t>(max(0, min(128, g.N - n0))) * 2u : 0u;
         // the odd CTA of the last pair tile may lie past the weights (an odd
         // number of channel tiles): nothing to load, its rows are never stored
         const bool have = ctile < g.ntn;
-        for (int r = 0; r < g.kb; ++r, ++gs) {
+        const int r1 = min(sg.r1, g.kb);
+        for (int r = sg.r0; r < r1; ++r, ++gs) {
           const int ls = gs % LS;
           if (gs >= LS && !mbar_wait(&sempty[ls], static_cast<uint32_t>(gs / LS - 1) & 1u, abort_flag)) {
             ok = false;
@@ -241,27 +315,31 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ pair MMA (even CTA)
-    if (leader && lane == 0) {
+    // The leader's whole warp runs the loop and its waits; an elected lane
+    // issues the pair instructions and commits.
+    if (leader) {
       constexpr uint32_t idesc_main = idesc_s8_s32(256, 256);
       constexpr uint32_t idesc_comp = idesc_f16_f32(256, 256);
       const uint64_t adesc0 = sdesc_k_sw128(smem_u32(smem));
       const uint64_t bdesc0 = sdesc_k_sw128(smem_u32(smem + 16384));
       int gi = 0, ti = 0;
       bool ok = true, issued = false;
-      for (int t = cid; ok && t < g.tiles; t += g.ncl, ++ti) {
-        if (ti > 0 && !mbar_wait_cluster(acc_empty, static_cast<uint32_t>(ti - 1) & 1u, abort_flag)) {
+      PairGen gen = pair_begin(g, cid);
+      PairSeg sg;
+      for (; ok && pair_next(g, cid, gen, sg); ++ti) {
+        if (ti > 0 && !warp_agree(mbar_wait_cluster(acc_empty, static_cast<uint32_t>(ti - 1) & 1u, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int r = 0; r < g.T; ++r, ++gi) {
+        for (int r = sg.r0; r < sg.r1; ++r, ++gi) {
           const int s = gi % S;
-          if (!mbar_wait(&full[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
+          if (!warp_wait(&full[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
             ok = false;
             break;
           }
           QLIN_STEP(gi, 1);
-          if (C::kConv && !mbar_wait_cluster_poll(&aready[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag)) {
+          if (C::kConv && !warp_agree(mbar_wait_cluster_poll(&aready[s], static_cast<uint32_t>(gi / S) & 1u, abort_flag))) {
             ok = false;
             break;
           }
@@ -270,24 +348,30 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
           issued = true;
           const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kPairStage >> 4));
           const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (kPairStage >> 4));
-          if (r < g.kb) {
+          if (elect_one()) {
+            if (r < g.kb) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mma_i8_pair(tmem, ad + 2 * k, bd + 2 * k, idesc_main, (r > 0 || k > 0) ? 1u : 0u);
-          } else {
-            const int j = r - g.kb;
+              for (int k = 0; k < 4; ++k)
+                mma_i8_pair(tmem, ad + 2 * k, bd + 2 * k, idesc_main, (r > sg.r0 || k > 0) ? 1u : 0u);
+            } else {
+              const int j = r - g.kb;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_f16_pair(tmem + 256, ad + 2 * k, bd + 2 * k, idesc_comp, (j > 0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                mma_f16_pair(tmem + 256, ad + 2 * k, bd + 2 * k, idesc_comp, (j > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit_pair(&empty[s], 0x3);
           }
-          mma_commit_pair(&empty[s], 0x3);
+          __syncwarp();
           QLIN_STEP(gi, 7);
         }
         if (!ok) break;
-        mma_commit_pair(acc_full, 0x3);
+        if (elect_one()) mma_commit_pair(acc_full, 0x3);
+        __syncwarp();
       }
       // every pair MMA has completed before tensor memory can be freed
       if (issued) {
-        mma_commit_pair(mma_done, 0x1);
+        if (elect_one()) mma_commit_pair(mma_done, 0x1);
+        __syncwarp();
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait_sleep(mma_done, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
         }
@@ -307,11 +391,13 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
       const uint32_t lready0 = mapa_shared(smem_u32(&aready[0]), 0);
       int gi = 0, gs = 0;
       bool ok = true;
-      for (int t = cid; ok && t < g.tiles; t += g.ncl) {
+      PairGen gen = pair_begin(g, cid);
+      PairSeg sg;
+      while (ok && pair_next(g, cid, gen, sg)) {
         int tn2, tm;
-        pair_tile_coords(g, t, tn2, tm);
+        pair_tile_coords(g, sg.t, tn2, tm);
         const int n = (2 * tn2 + crk) * 128 + row;
-        for (int r = 0; r < g.T; ++r, ++gi) {
+        for (int r = sg.r0; r < sg.r1; ++r, ++gi) {
           const int s = gi % S;
           if (gi >= S) ok = mbar_wait(&empty[s], static_cast<uint32_t>(gi / S - 1) & 1u, abort_flag);
           ok = __all_sync(0xffffffffu, ok);
@@ -374,13 +460,18 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
     griddep_wait();  // a[] comes from the previous kernel
     int ti = 0;
     bool ok = true;
-    for (int t = cid; t < g.tiles; t += g.ncl, ++ti) {
+    PairGen gen = pair_begin(g, cid);
+    PairSeg sg;
+    for (; pair_next(g, cid, gen, sg); ++ti) {
       int tn2, tm;
-      pair_tile_coords(g, t, tn2, tm);
+      pair_tile_coords(g, sg.t, tn2, tm);
       const int ctile = 2 * tn2 + crk;
       const int n = ctile * 128 + nl;
       const int m0 = tm * 256;
       const int mvalid = min(256, g.M - m0);
+      const bool part = sg.slot >= 0;
+      const bool has_main = sg.r0 < g.kb;           // the range holds K-blocks of the tile
+      const bool has_comp = comp && sg.r1 == g.T;  // ... and its compensation (never split)
       float cn = 0.f;
       if (n < g.N) cn = __fmul_rn(g.cscale[n], g.cmul);
       if (issuer) bulk_wait_group_read0();  // the previous tile's store has read the output buffer
@@ -394,15 +485,28 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       const uint32_t trow = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+      // partial of a split tile: this CTA's slot, [token][channel]
+      const size_t pslot = part ? (static_cast<size_t>(sg.slot) * 2 + crk) * 256 * 128 : 0;
 #pragma unroll 1
       for (int c0 = grp * 16; c0 < mvalid; c0 += 32) {
         uint32_t acc[16], cmp[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) { acc[j] = 0u; cmp[j] = 0u; }
         if (ok) {
-          tmem_ld16(trow + c0, acc);
-          if (comp) tmem_ld16(trow + 256 + c0, cmp);
+          if (has_main) tmem_ld16(trow + c0, acc);
+          if (has_comp) tmem_ld16(trow + 256 + c0, cmp);
           tmem_ld_wait();
+        }
+        if (part) {
+          int32_t* pa = g.ws_acc + pslot + static_cast<size_t>(c0) * 128 + nl;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pa[j * 128] = static_cast<int32_t>(acc[j]);
+          if (has_comp) {  // only a range's first segment can hold a compensation: one slot per pair
+            float* pc = g.ws_comp + (static_cast<size_t>(cid) * 2 + crk) * 256 * 128 + static_cast<size_t>(c0) * 128 + nl;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pc[j * 128] = __uint_as_float(cmp[j]);
+          }
+          continue;
         }
         float sc[16];
 #pragma unroll
@@ -425,6 +529,65 @@ __global__ void __launch_bounds__(PairCfg<FMT>::kThreads, 1) gemm_pair_kernel(co
       if (lane == 0) {
         if (leader) mbar_arrive(acc_empty);
         else mbar_arrive_remote(lempty);
+      }
+      if (part) {
+        // Count this CTA's steps of the split tile (CTA barrier, then one
+        // thread's release fence and atomic: the release covers every
+        // epilogue thread's partial stores); the range whose steps complete
+        // the tile sums every contributor's partial and writes the output.
+        named_bar_sync(1, 256);
+        if (ep == 0 && lane == 0) {
+          fence_acq_rel_gpu();
+          const unsigned add = static_cast<unsigned>(sg.r1 - sg.r0);
+          const unsigned old = atom_add_relaxed_gpu(&g.ws_cnt[sg.sk * 2 + crk], add);
+          const bool last = old + add == static_cast<unsigned>(g.T);
+          if (last) fence_acq_rel_gpu();  // acquire the other contributors' partials
+          *fin_flag = last ? 1 : 0;
+        }
+        named_bar_sync(1, 256);
+        if (!*fin_flag) continue;
+        const unsigned ts = static_cast<unsigned>(sg.sk) * static_cast<unsigned>(g.T);
+        const int c_lo = pair_owner(g, ts);
+        const int c_hi = pair_owner(g, ts + static_cast<unsigned>(g.T) - 1u);
+#pragma unroll 1
+        for (int c0 = grp * 16; c0 < mvalid; c0 += 32) {
+          int32_t sum[16];
+          float cp[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) { sum[j] = 0; cp[j] = 0.f; }
+          for (int c = c_lo; c <= c_hi; ++c) {
+            if (g.bnd[c] == g.bnd[c + 1]) continue;  // an empty range
+            const int slot = 2 * c + (g.bnd[c] < ts ? 1 : 0);
+            const int32_t* src = g.ws_acc + (static_cast<size_t>(slot) * 2 + crk) * 256 * 128 + static_cast<size_t>(c0) * 128 + nl;
+            int32_t v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + j * 128);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) sum[j] += v[j];
+          }
+          if (comp) {
+            // the range holding the tile's last step holds its whole compensation
+            const float* src = g.ws_comp + (static_cast<size_t>(c_hi) * 2 + crk) * 256 * 128 + static_cast<size_t>(c0) * 128 + nl;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) cp[j] = __ldcg(src + j * 128);
+          }
+          float sc[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 v = *reinterpret_cast<const float4*>(sa + c0 + 4 * q4);
+            sc[4 * q4] = v.x; sc[4 * q4 + 1] = v.y; sc[4 * q4 + 2] = v.z; sc[4 * q4 + 3] = v.w;
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float v = __fmul_rn(cn, static_cast<float>(sum[j]));
+            if (comp) v = __fadd_rn(v, cp[j]);
+            ys[(c0 + j) * 128 + nl] = __half_as_ushort(__float2half_rn(__fmul_rn(sc[j], v)));
+          }
+          if (g.acc_debug && n < g.N)
+            for (int j = 0; j < 16; ++j)
+              if (c0 + j < mvalid) g.acc_debug[static_cast<size_t>(m0 + c0 + j) * g.N + n] = sum[j];
+        }
+        if (ep == 0 && lane == 0) g.ws_cnt[sg.sk * 2 + crk] = 0u;  // zero for the next launch
       }
       fence_proxy_async_smem();  // the output rows are read by the bulk copy next
       named_bar_sync(1, 256);

@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and its waits; an elected lane issues.
+    {
       constexpr uint32_t idesc = idesc_s8_s32(128, 128);
       const uint64_t adesc0 = sdesc_k_sw128(smem_u32(smem));
       const uint64_t bdesc0 = sdesc_k_sw128(smem_u32(smem + 16384));
@@ -333,11 +334,11 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
       for (int t = blockIdx.x; ok && t < g.tiles; t += gridDim.x) {
         for (int kb = 0; kb < g.G; ++kb, ++it) {
           const int s = it % S, b = it % B;
-          if (it >= B && !mbar_wait(&acc_empty[b], static_cast<uint32_t>(it / B - 1) & 1u, abort_flag)) {
+          if (it >= B && !warp_wait(&acc_empty[b], static_cast<uint32_t>(it / B - 1) & 1u, abort_flag)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(&full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag)) {
+          if (!warp_wait(&full[s], static_cast<uint32_t>(it / S) & 1u, abort_flag)) {
             ok = false;
             break;
           }
@@ -345,14 +346,18 @@ __global__ void __launch_bounds__(kOffqThreads, 1) offq_gemm_kernel(const __grid
           issued = true;
           const uint64_t ad = adesc0 + static_cast<uint64_t>(s * (kOffqStage >> 4));
           const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (kOffqStage >> 4));
+          if (elect_one()) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mma_i8(tmem + 128u * b, ad + 2 * k, bd + 2 * k, idesc, k > 0 ? 1u : 0u);
-          mma_commit(&empty[s]);
-          mma_commit(&acc_full[b]);
+            for (int k = 0; k < 4; ++k) mma_i8(tmem + 128u * b, ad + 2 * k, bd + 2 * k, idesc, k > 0 ? 1u : 0u);
+            mma_commit(&empty[s]);
+            mma_commit(&acc_full[b]);
+          }
+          __syncwarp();
         }
       }
       if (issued) {  // every tensor-core op has completed before tensor memory is freed
-        mma_commit(mma_done);
+        if (elect_one()) mma_commit(mma_done);
+        __syncwarp();
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait_sleep(mma_done, 0u, 1000000u) && globaltimer_ns() - t0 < QLIN_DRAIN_NS) {
         }

@@ -141,7 +141,7 @@ qlin_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
 // each may start its prologue (and the GEMM its weight stream) while the
 // previous kernel in the stream finishes; every kernel waits on the grid
 // dependency before it reads what the previous one wrote.
-std::atomic<long long> g_knob[10] = {{1}, {1}, {0}, {0}, {256}, {512}, {kFusedMomentumMaxM}, {2000000000LL}, {2}, {0}};
+std::atomic<long long> g_knob[11] = {{1}, {1}, {0}, {0}, {256}, {512}, {kFusedMomentumMaxM}, {2000000000LL}, {2}, {0}, {0}};
 
 long long knob(int k) { return g_knob[k].load(std::memory_order_relaxed); }
 
@@ -235,7 +235,52 @@ struct GemmPlan {
   GemmProb pr[kMaxProbs];  // per problem: shape, tiles and iteration offsets (pointers unset)
   size_t acc_off, comp_off, cnt_off, w8_off, total;  // shared scratch (after the problems' U operands)
   size_t u_off[kMaxProbs];                           // each problem's compensation operand U
+  // CTA-pair launch (one problem, 256 x 256 tiles): pairs, whole tiles and
+  // the stream-K tail's step boundaries, partial slots and tile counters
+  int pair_ncl, pair_dp;
+  long long pair_sk_tiles;
+  size_t pacc_off, pcomp_off, pcnt_off;
+  unsigned pair_bnd[kMaxPairs + 1];
 };
+
+bool use_pair(const GemmPlan& p, const qlin_weights* w);
+template <int FMT>
+int pair_max_clusters();
+
+// Work split of a launch on CTA pairs over `tiles` tiles of T steps (the
+// last T - kb of them the outlier compensation, never split).  Whole tiles
+// in raster order while they fill whole waves; when the last wave would be
+// partly empty, the last full wave and the remainder are instead divided by
+// steps into one contiguous range per pair (stream-K), so every pair ends
+// at about the same time.  With eight or more full waves the empty part of
+// the last one is small and tiles stay whole.
+void pair_split(GemmPlan& p, long long tiles, int T, int kb, int maxc) {
+  if (maxc > kMaxPairs) maxc = kMaxPairs;
+  p.pair_sk_tiles = 0;
+  for (int c = 0; c <= kMaxPairs; ++c) p.pair_bnd[c] = 0u;
+  const long long full = tiles / maxc, rem = tiles % maxc;
+  if (knob(QLIN_KNOB_PAIR_SPLIT) == 0 || rem == 0 || full >= 8 || maxc < 2) {
+    p.pair_ncl = static_cast<int>(tiles < maxc ? tiles : maxc);
+    p.pair_dp = static_cast<int>(tiles);
+    return;
+  }
+  p.pair_ncl = maxc;
+  p.pair_dp = static_cast<int>(full >= 1 ? (full - 1) * maxc : 0);
+  p.pair_sk_tiles = tiles - p.pair_dp;
+  const unsigned long long total = static_cast<unsigned long long>(p.pair_sk_tiles) * T;
+  unsigned prev = 0;
+  for (int c = 0; c <= p.pair_ncl; ++c) {
+    unsigned long long b = total * c / p.pair_ncl;
+    const unsigned long long r = b % T;
+    if (r > static_cast<unsigned long long>(kb) && r < static_cast<unsigned long long>(T))
+      b = (r - kb <= T - r) ? b - (r - kb) : b + (T - r);  // not inside a compensation run
+    if (c == p.pair_ncl) b = total;
+    unsigned v = static_cast<unsigned>(b);
+    if (v < prev) v = prev;
+    p.pair_bnd[c] = v;
+    prev = v;
+  }
+}
 
 // From this many tokens the INT4 formats widen their weights once per call
 // and run the INT8 kernel (QLIN_KNOB_WIDEN_MIN_M; 0 turns it off).
@@ -311,6 +356,27 @@ GemmPlan plan_gemm_group(int M, const qlin_weights* const* ws, int n) {
                 ? 1 : 0;
   p.w8_off = off;
   off = round_up(off + (p.widen ? size_t(p.pr[0].tiles_n) * p.pr[0].kb * 16384 : 0), kAlign);
+  p.pair_ncl = 0;
+  p.pair_dp = 0;
+  p.pair_sk_tiles = 0;
+  p.pacc_off = p.pcomp_off = p.pcnt_off = off;
+  if (n == 1 && use_pair(p, ws[0])) {
+    const GemmProb& q = p.pr[0];
+    const bool conv = p.widen && M <= convert_max_m();
+    const int maxc = !conv ? pair_max_clusters<kFmtW8>()
+                           : (ws[0]->fmt == QLIN_W4_PERCHANNEL ? pair_max_clusters<kFmtW4PC>()
+                                                                : pair_max_clusters<kFmtW4G128>());
+    const long long tiles = static_cast<long long>((q.tiles_n + 1) / 2) * q.tiles_m;
+    pair_split(p, tiles, q.kb + 2 * q.ncs, q.kb, maxc > 0 ? maxc : 1);
+    if (p.pair_sk_tiles > 0) {
+      const size_t part = size_t(2) * 256 * 128 * 4;  // one slot: both CTAs' 128 channels x 256 tokens
+      off = round_up(off + size_t(2) * p.pair_ncl * part, kAlign);
+      p.pcomp_off = off;
+      off = round_up(off + (ws[0]->n_outlier > 0 ? size_t(p.pair_ncl) * part : 0), kAlign);
+      p.pcnt_off = off;
+      off = round_up(off + size_t(p.pair_sk_tiles) * 2 * 4, kAlign);
+    }
+  }
   p.total = off;
   return p;
 }
@@ -498,7 +564,13 @@ qlin_status launch_gemm_pair(const GemmPlan& p, const qlin_weights* w, const int
   int gm = static_cast<int>(std::lround(std::sqrt(static_cast<double>(maxc) * 256.0 / 256.0)));
   if (x_bytes <= 48.0 * 1024 * 1024) gm = g.tiles_m;
   g.gm = gm < 1 ? 1 : (gm > g.tiles_m ? g.tiles_m : gm);
-  g.ncl = g.tiles < maxc ? g.tiles : maxc;
+  if (p.pair_ncl < 1 || p.pair_ncl > maxc) return fail(QLIN_ERR_CUDA, "gemm_pair_kernel: plan of %d pairs, %d fit", p.pair_ncl, maxc);
+  g.ncl = p.pair_ncl;
+  g.dp = p.pair_dp;
+  for (int c = 0; c <= kMaxPairs; ++c) g.bnd[c] = p.pair_bnd[c];
+  g.ws_acc = reinterpret_cast<int32_t*>(gws + p.pacc_off);
+  g.ws_comp = reinterpret_cast<float*>(gws + p.pcomp_off);
+  g.ws_cnt = reinterpret_cast<unsigned*>(gws + p.pcnt_off);
   qlin_status st = QLIN_OK;
   if (FMT == kFmtW8) {
     st = make_map(&prm.tmA, codes8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128,
@@ -1652,11 +1724,12 @@ qlin_status qlin_offq_forward(const uint16_t* X, int32_t M, int32_t K, int32_t N
 }
 
 qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
-  if (k < 0 || k > QLIN_KNOB_CONVERT_MAX_M) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
+  if (k < 0 || k > QLIN_KNOB_PAIR_SPLIT) return fail(QLIN_ERR_ARG, "unknown knob %d", k);
   bool ok = true;
   switch (k) {
     case QLIN_KNOB_PDL:
-    case QLIN_KNOB_CLUSTER: ok = value == 0 || value == 1; break;
+    case QLIN_KNOB_CLUSTER:
+    case QLIN_KNOB_PAIR_SPLIT: ok = value == 0 || value == 1; break;
     case QLIN_KNOB_CLUSTER_SIZE: ok = value == 0 || value == 2 || value == 4 || value == 8; break;
     case QLIN_KNOB_MAX_TOKEN_TILE: ok = value == 64 || value == 128 || value == 256; break;
     case QLIN_KNOB_PAIR_MMA: ok = value >= 0 && value <= 2; break;
@@ -1673,7 +1746,7 @@ qlin_status qlin_debug_set(int32_t k, int64_t value, int64_t* previous) {
 }
 
 qlin_status qlin_debug_get(int32_t k, int64_t* value) {
-  if (k < 0 || k > QLIN_KNOB_CONVERT_MAX_M || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
+  if (k < 0 || k > QLIN_KNOB_PAIR_SPLIT || !value) return fail(QLIN_ERR_ARG, "unknown knob %d or NULL value", k);
   *value = g_knob[k].load();
   return QLIN_OK;
 }

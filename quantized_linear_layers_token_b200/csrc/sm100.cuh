@@ -109,8 +109,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // The same wait made by every lane of a converged warp; the warp agrees on
 // the outcome (a lane that saw the limit pass makes the whole warp give up).
+__device__ __forceinline__ bool warp_agree(bool ok) { return __all_sync(0xffffffffu, ok) != 0; }
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort)) != 0;
+  return warp_agree(mbar_wait(bar, parity, abort));
 }
 
 // One lane of a converged warp (elect.sync over the full mask: the lowest

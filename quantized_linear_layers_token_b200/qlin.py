@@ -47,6 +47,7 @@ QLIN_KNOB_FUSED_MOMENTUM_MAX_M = 6
 QLIN_KNOB_WAIT_NS = 7
 QLIN_KNOB_PAIR_MMA = 8
 QLIN_KNOB_CONVERT_MAX_M = 9
+QLIN_KNOB_PAIR_SPLIT = 10
 
 
 class QlinError(RuntimeError):
