@@ -31,8 +31,9 @@
 //   warp 0        X producer: activation tiles (TMA, after the grid
 //                 dependency on the previous kernel) and the compensation
 //                 operands U hi/lo.
-//   warp 1        allocates TMEM (two accumulator buffers when they fit); one
-//                 lane issues tcgen05.mma and commits.
+//   warp 1        allocates TMEM (two accumulator buffers when they fit); the
+//                 whole warp runs the MMA loop and an elected lane issues
+//                 tcgen05.mma and commits.
 //   warp 2        weight producer: packed INT4 blocks into the staging ring,
 //                 INT8 blocks and W_O^T blocks into the A ring; starts at once
 //                 (weights do not depend on the previous kernel).

@@ -25,7 +25,8 @@
 //                 counted on the even CTA's full barrier; waits for its own
 //                 empty barrier (released by the pair's MMA commit).
 //   warp 1        tensor memory allocation (both CTAs, cta_group::2); in the
-//                 even CTA one lane issues the pair MMAs and commits.
+//                 even CTA the whole warp runs the MMA loop and an elected
+//                 lane issues the pair MMAs and commits.
 //   warps 2..9    epilogue, two groups of four warps taking alternate
 //                 16-token chunks of the CTA's 128 x 256 accumulator into an
 //                 fp16 output tile in shared memory; each warp then arrives
