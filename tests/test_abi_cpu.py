@@ -187,3 +187,50 @@ def test_synthetic_inputs_are_reproducible():
     assert not np.array_equal(a["W"], c["W"])
     assert np.array_equal(synth.grad_output(1, 0, 8, 64), synth.grad_output(1, 0, 8, 64))
     assert np.array_equal(synth.outlier_scales(1, 0, 5), synth.outlier_scales(1, 0, 5))
+
+
+def header_knobs():
+    with open(os.path.join(ROOT, "include", "qlin.h")) as f:
+        text = f.read()
+    return {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(QLIN_KNOB_\w+)\s*=\s*(\d+)", text)}
+
+
+def test_knob_ids_match_the_header(q):
+    knobs = header_knobs()
+    assert knobs, "no knob enum in the header"
+    for name, value in knobs.items():
+        assert getattr(q, name) == value, name
+
+
+# documented defaults (include/qlin.h, test and measurement hooks)
+KNOB_DEFAULTS = {"PDL": 1, "CLUSTER": 1, "CLUSTER_SIZE": 0, "MAX_CTAS": 0, "MAX_TOKEN_TILE": 256,
+                 "WIDEN_MIN_M": 512, "FUSED_MOMENTUM_MAX_M": 64, "WAIT_NS": 2000000000, "PAIR_MMA": 2,
+                 "CONVERT_MAX_M": 0, "PAIR_SPLIT": 0}
+
+
+def test_knob_defaults_and_validation(q):
+    for name, value in KNOB_DEFAULTS.items():
+        assert q.qlin_debug_get(getattr(q, "QLIN_KNOB_" + name)) == value, name
+    bad = [("PDL", 2), ("CLUSTER", -1), ("CLUSTER_SIZE", 3), ("MAX_TOKEN_TILE", 32), ("PAIR_MMA", 3),
+           ("PAIR_SPLIT", 2), ("MAX_CTAS", -1), ("WIDEN_MIN_M", -5)]
+    for name, value in bad:
+        k = getattr(q, "QLIN_KNOB_" + name)
+        with pytest.raises(q.QlinError):
+            q.qlin_debug_set(k, value)
+        assert q.qlin_debug_get(k) == KNOB_DEFAULTS[name], name  # a refused value leaves the knob as it was
+    for k in (-1, max(header_knobs().values()) + 1):
+        with pytest.raises(q.QlinError):
+            q.qlin_debug_set(k, 0)
+        with pytest.raises(q.QlinError):
+            q.qlin_debug_get(k)
+
+
+def test_knobs_context_restores(q):
+    with q.knobs(pair_split=1, widen_min_m=129, pair_mma=1):
+        assert q.qlin_debug_get(q.QLIN_KNOB_PAIR_SPLIT) == 1
+        assert q.qlin_debug_get(q.QLIN_KNOB_WIDEN_MIN_M) == 129
+        with q.knobs(pair_split=0):
+            assert q.qlin_debug_get(q.QLIN_KNOB_PAIR_SPLIT) == 0
+        assert q.qlin_debug_get(q.QLIN_KNOB_PAIR_SPLIT) == 1
+    for name in ("PAIR_SPLIT", "WIDEN_MIN_M", "PAIR_MMA"):
+        assert q.qlin_debug_get(getattr(q, "QLIN_KNOB_" + name)) == KNOB_DEFAULTS[name]
