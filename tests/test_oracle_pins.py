@@ -14,7 +14,8 @@ from quantized_linear_layers_token_b200 import synth
 
 
 def f16_bits(x):
-    return np.ascontiguousarray(np.asarray(x, np.float16)).view(np.uint16)
+    with np.errstate(over="ignore"):  # values past the fp16 range round to infinity, as intended
+        return np.ascontiguousarray(np.asarray(x, np.float16)).view(np.uint16)
 
 
 # ---------------------------------------------------------------------------
